@@ -1,0 +1,332 @@
+/*
+ * kivi_oracle.c -- plain, slow, single-threaded CPU oracle for the KIVI
+ * asymmetric 2/4-bit KV cache and its decode attention.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark load this file.  It shares nothing with the
+ * CUDA library and the CUDA library never calls it.
+ *
+ * Build: gcc -std=c99 -O2 -ffp-contract=off -fno-fast-math -fPIC -shared
+ * (every float operation below is one IEEE binary32 operation rounded to
+ * nearest-even; no contraction into fused multiply-adds).
+ *
+ * The four steps, in the order the method applies them:
+ *   Q  quantize a group with an asymmetric min/max scale and zero
+ *      (KIVI, study.space summary: the method is asymmetric; mlsanity.com
+ *      index page, "Abstract (arXiv)": 2-bit codes, keys per channel,
+ *      values per token);
+ *   P  pack the codes 32/bits to a 32-bit word;
+ *   S  split the cache into a quantized part and a full-precision residual
+ *      window of R recent tokens, flushing the window into the quantized
+ *      part every R tokens (study.space summary: grouped and residual
+ *      parts, value codes appended along tokens, key quantization grouped
+ *      across tokens; scholarfeed.org "KIVI" page, third quote:
+ *      fixed-length residual buffer);
+ *   A  decode attention over the dequantized quantized part and the
+ *      residual part together (study.space summary: the residual part is
+ *      combined with the grouped part when attention is computed).
+ *
+ * Parity pins for every function are in tests/test_oracle_*.py.
+ */
+#include "kivi_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+static int valid_bits(int bits) {
+  return bits == 1 || bits == 2 || bits == 4 || bits == 8 || bits == 16;
+}
+
+/*
+ * Q.  The pages name the quantizer only as asymmetric (a scale and an
+ * offset per group).  Reading: the plain min/max form, in binary32:
+ *   mn = min x_i, mx = max x_i   (strict compares, first occurrence kept)
+ *   L  = 2^bits - 1
+ *   s  = (mx - mn) / L           (one rounded subtraction, one rounded
+ *                                 division)
+ *   z  = mn                      (a float offset, not an integer zero-point)
+ *   c_i = clamp(round_half_even((x_i - mn) / s), 0, L), or 0 when s == 0.
+ * The quotient is a true division, not a multiply by 1/s.
+ */
+int kivi_oracle_quantize_group(const float *x, long long n, long long stride,
+                               int bits, float *scale, float *zero,
+                               uint16_t *codes) {
+  long long i;
+  float mn, mx, L, range, s;
+  if (!x || !scale || !zero || !codes || n <= 0 || !valid_bits(bits))
+    return KIVI_ORACLE_ERR_ARG;
+  mn = x[0];
+  mx = x[0];
+  for (i = 1; i < n; ++i) {
+    float v = x[i * stride];
+    if (v < mn) mn = v;
+    if (v > mx) mx = v;
+  }
+  L = (float)((1u << bits) - 1u);
+  range = mx - mn;
+  s = range / L;
+  *scale = s;
+  *zero = mn;
+  for (i = 0; i < n; ++i) {
+    if (s == 0.0f) {
+      codes[i] = 0;
+    } else {
+      float t = (x[i * stride] - mn) / s;
+      float c = nearbyintf(t); /* default rounding mode: half to even */
+      if (c < 0.0f) c = 0.0f;
+      if (c > L) c = L;
+      codes[i] = (uint16_t)c;
+    }
+  }
+  return KIVI_ORACLE_OK;
+}
+
+/*
+ * P.  Reading (the pages give no bit layout): E = 32/bits codes per word,
+ * the first code in the least significant bits.
+ */
+uint32_t kivi_oracle_pack_word(const uint16_t *codes, int bits) {
+  int i, E = 32 / bits;
+  uint32_t mask = (uint32_t)((1u << bits) - 1u);
+  uint32_t w = 0;
+  for (i = 0; i < E; ++i) w |= ((uint32_t)codes[i] & mask) << (bits * i);
+  return w;
+}
+
+static uint32_t unpack_code(uint32_t word, int pos, int bits) {
+  uint32_t mask = (uint32_t)((1u << bits) - 1u);
+  return (word >> (bits * pos)) & mask;
+}
+
+/* D.  x_hat = c * s + z, evaluated in real arithmetic (binary64 holds
+ * c * s exactly; the one remaining rounding is far below binary32). */
+double kivi_oracle_dequant(uint32_t c, float scale, float zero) {
+  return (double)c * (double)scale + (double)zero;
+}
+
+int kivi_oracle_check_unit(const kivi_oracle_unit *u) {
+  int E;
+  if (!u || !valid_bits(u->bits)) return KIVI_ORACLE_ERR_ARG;
+  E = 32 / u->bits;
+  if (u->D <= 0 || u->G <= 0 || u->Gv <= 0 || u->R <= 0 || u->Tq < 0)
+    return KIVI_ORACLE_ERR_ARG;
+  if (u->D % E || u->D % u->Gv || u->R % u->G || u->R % E || u->Tq % u->R)
+    return KIVI_ORACLE_ERR_ARG;
+  if (u->Tq > 0 && (!u->k_codes || !u->k_scale || !u->k_zero ||
+                    !u->v_codes || !u->v_scale || !u->v_zero))
+    return KIVI_ORACLE_ERR_ARG;
+  if (!u->k_res || !u->v_res) return KIVI_ORACLE_ERR_ARG;
+  return KIVI_ORACLE_OK;
+}
+
+/*
+ * Q + P over a block of n tokens (n a multiple of G and of E), written to
+ * token positions t0 .. t0+n-1 of the quantized store.  K and V are [n][D].
+ *   keys:   per channel d, groups of G consecutive tokens (per-channel key
+ *           quantization, grouped across tokens);
+ *   values: per token t, groups of Gv consecutive channels (per-token value
+ *           quantization).
+ * Codes are first produced for every (token, channel), then packed: keys
+ * along channels within a token, values along tokens within a channel.
+ */
+static int quantize_block(kivi_oracle_unit *u, const float *K, const float *V,
+                          long long t0, long long n) {
+  const int D = u->D, bits = u->bits, G = u->G, Gv = u->Gv;
+  const int E = 32 / bits, WK = D / E, NJ = D / Gv;
+  uint16_t *ck = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(n * D));
+  uint16_t *cv = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(n * D));
+  uint16_t *tmp = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(G > E ? G : E));
+  long long t, g, i;
+  int d, j, w;
+  if (!ck || !cv || !tmp) {
+    free(ck);
+    free(cv);
+    free(tmp);
+    return KIVI_ORACLE_ERR_NOMEM;
+  }
+
+  /* keys: one group per (key group g, channel d) over G tokens */
+  for (g = 0; g < n / G; ++g) {
+    for (d = 0; d < D; ++d) {
+      long long gq = (t0 / G) + g;
+      kivi_oracle_quantize_group(&K[(g * G) * D + d], G, D, bits,
+                                 &u->k_scale[gq * D + d],
+                                 &u->k_zero[gq * D + d], tmp);
+      for (i = 0; i < G; ++i) ck[(g * G + i) * D + d] = tmp[i];
+    }
+  }
+  /* values: one group per (token t, value group j) over Gv channels */
+  for (t = 0; t < n; ++t) {
+    for (j = 0; j < NJ; ++j) {
+      kivi_oracle_quantize_group(&V[t * D + j * Gv], Gv, 1, bits,
+                                 &u->v_scale[(t0 + t) * NJ + j],
+                                 &u->v_zero[(t0 + t) * NJ + j], tmp);
+      for (i = 0; i < Gv; ++i) cv[t * D + j * Gv + i] = tmp[i];
+    }
+  }
+  /* pack keys along channels: word w of token t holds channels wE..wE+E-1 */
+  for (t = 0; t < n; ++t)
+    for (w = 0; w < WK; ++w)
+      u->k_codes[(t0 + t) * WK + w] = kivi_oracle_pack_word(&ck[t * D + w * E], bits);
+  /* pack values along tokens: word (tb, d) holds tokens tb*E..tb*E+E-1 */
+  for (t = 0; t < n / E; ++t) {
+    for (d = 0; d < D; ++d) {
+      for (i = 0; i < E; ++i) tmp[i] = cv[(t * E + i) * D + d];
+      u->v_codes[((t0 / E) + t) * D + d] = kivi_oracle_pack_word(tmp, bits);
+    }
+  }
+  free(ck);
+  free(cv);
+  free(tmp);
+  return KIVI_ORACLE_OK;
+}
+
+/*
+ * S, prefill.  Reading of "residual window of R recent tokens, flushed every
+ * R": the window is flushed just before a token would not fit, so a
+ * non-empty cache always holds 1..R residual tokens.  A prompt of T tokens
+ * therefore leaves r = ((T-1) mod R) + 1 tokens in the window and quantizes
+ * the first n_q = T - r, exactly the state T single appends would reach.
+ */
+int kivi_oracle_prefill(kivi_oracle_unit *u, const float *K, const float *V,
+                        long long T) {
+  int rc = kivi_oracle_check_unit(u);
+  long long r, nq;
+  if (rc) return rc;
+  if (T < 0 || (T > 0 && (!K || !V))) return KIVI_ORACLE_ERR_ARG;
+  if (u->n_q != 0 || u->r != 0) return KIVI_ORACLE_ERR_STATE;
+  r = (T == 0) ? 0 : ((T - 1) % u->R) + 1;
+  nq = T - r;
+  if (nq > u->Tq) return KIVI_ORACLE_ERR_CAPACITY;
+  if (nq > 0) {
+    rc = quantize_block(u, K, V, 0, nq);
+    if (rc) return rc;
+  }
+  memcpy(u->k_res, &K[nq * u->D], sizeof(float) * (size_t)(r * u->D));
+  memcpy(u->v_res, &V[nq * u->D], sizeof(float) * (size_t)(r * u->D));
+  u->n_q = nq;
+  u->r = (int)r;
+  return KIVI_ORACLE_OK;
+}
+
+/*
+ * S, append one token.  If the window is full, its R tokens are quantized
+ * (Q + P, R/G key groups and R value tokens) into token positions
+ * n_q .. n_q+R-1 and the window is emptied; then the token is written to the
+ * next window slot.
+ */
+int kivi_oracle_append(kivi_oracle_unit *u, const float *k, const float *v) {
+  int rc = kivi_oracle_check_unit(u);
+  if (rc) return rc;
+  if (!k || !v) return KIVI_ORACLE_ERR_ARG;
+  if (u->r == u->R) {
+    if (u->n_q + u->R > u->Tq) return KIVI_ORACLE_ERR_CAPACITY;
+    rc = quantize_block(u, u->k_res, u->v_res, u->n_q, u->R);
+    if (rc) return rc;
+    u->n_q += u->R;
+    u->r = 0;
+  }
+  memcpy(&u->k_res[(long long)u->r * u->D], k, sizeof(float) * (size_t)u->D);
+  memcpy(&u->v_res[(long long)u->r * u->D], v, sizeof(float) * (size_t)u->D);
+  u->r += 1;
+  return KIVI_ORACLE_OK;
+}
+
+/* D over the whole unit: token t < n_q from codes, t >= n_q from the window. */
+int kivi_oracle_dequant_keys(const kivi_oracle_unit *u, double *out) {
+  int rc = kivi_oracle_check_unit(u);
+  const int D = u ? u->D : 0;
+  long long t;
+  int d;
+  if (rc) return rc;
+  if (!out) return KIVI_ORACLE_ERR_ARG;
+  for (t = 0; t < u->n_q; ++t) {
+    const int E = 32 / u->bits;
+    for (d = 0; d < D; ++d) {
+      uint32_t word = u->k_codes[t * (D / E) + d / E];
+      uint32_t c = unpack_code(word, d % E, u->bits);
+      long long g = t / u->G;
+      out[t * D + d] = kivi_oracle_dequant(c, u->k_scale[g * D + d], u->k_zero[g * D + d]);
+    }
+  }
+  for (t = 0; t < u->r; ++t)
+    for (d = 0; d < D; ++d) out[(u->n_q + t) * D + d] = (double)u->k_res[t * D + d];
+  return KIVI_ORACLE_OK;
+}
+
+int kivi_oracle_dequant_values(const kivi_oracle_unit *u, double *out) {
+  int rc = kivi_oracle_check_unit(u);
+  const int D = u ? u->D : 0;
+  long long t;
+  int d;
+  if (rc) return rc;
+  if (!out) return KIVI_ORACLE_ERR_ARG;
+  for (t = 0; t < u->n_q; ++t) {
+    const int E = 32 / u->bits, NJ = D / u->Gv;
+    for (d = 0; d < D; ++d) {
+      uint32_t word = u->v_codes[(t / E) * D + d];
+      uint32_t c = unpack_code(word, (int)(t % E), u->bits);
+      int j = d / u->Gv;
+      out[t * D + d] = kivi_oracle_dequant(c, u->v_scale[t * NJ + j], u->v_zero[t * NJ + j]);
+    }
+  }
+  for (t = 0; t < u->r; ++t)
+    for (d = 0; d < D; ++d) out[(u->n_q + t) * D + d] = (double)u->v_res[t * D + d];
+  return KIVI_ORACLE_OK;
+}
+
+/*
+ * A.  Plain two-pass softmax attention over all n_q + r tokens, with the
+ * quantized and the residual tokens in one softmax (not two normalised
+ * parts):
+ *   l_t   = sigma * sum_d q_d * Khat_{t,d}
+ *   p_t   = exp(l_t - max_t l_t)
+ *   out_d = sum_t p_t * Vhat_{t,d} / sum_t p_t
+ * in binary64, sums in index order.
+ */
+int kivi_oracle_decode(const kivi_oracle_unit *u, const float *q, int n_heads,
+                       double sigma, double *out) {
+  int rc = kivi_oracle_check_unit(u);
+  long long T, t;
+  int h, d;
+  double *Kh, *Vh, *p;
+  if (rc) return rc;
+  if (!q || !out || n_heads <= 0) return KIVI_ORACLE_ERR_ARG;
+  T = u->n_q + u->r;
+  if (T == 0) return KIVI_ORACLE_ERR_STATE;
+  Kh = (double *)malloc(sizeof(double) * (size_t)(T * u->D));
+  Vh = (double *)malloc(sizeof(double) * (size_t)(T * u->D));
+  p = (double *)malloc(sizeof(double) * (size_t)T);
+  if (!Kh || !Vh || !p) {
+    free(Kh);
+    free(Vh);
+    free(p);
+    return KIVI_ORACLE_ERR_NOMEM;
+  }
+  kivi_oracle_dequant_keys(u, Kh);
+  kivi_oracle_dequant_values(u, Vh);
+  for (h = 0; h < n_heads; ++h) {
+    const float *qh = &q[(long long)h * u->D];
+    double m = -INFINITY, l = 0.0;
+    for (t = 0; t < T; ++t) {
+      double acc = 0.0;
+      for (d = 0; d < u->D; ++d) acc += (double)qh[d] * Kh[t * u->D + d];
+      p[t] = sigma * acc;
+      if (p[t] > m) m = p[t];
+    }
+    for (t = 0; t < T; ++t) {
+      p[t] = exp(p[t] - m);
+      l += p[t];
+    }
+    for (d = 0; d < u->D; ++d) {
+      double o = 0.0;
+      for (t = 0; t < T; ++t) o += p[t] * Vh[t * u->D + d];
+      out[(long long)h * u->D + d] = o / l;
+    }
+  }
+  free(Kh);
+  free(Vh);
+  free(p);
+  return KIVI_ORACLE_OK;
+}

@@ -1,0 +1,107 @@
+/*
+ * kivi_oracle.h -- declarations of the plain CPU oracle for the KIVI
+ * asymmetric 2/4-bit KV cache.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark load this code.  It shares no source, header
+ * or table with the CUDA library (include/kivi.h, the package's csrc/), and
+ * the CUDA library never calls it.
+ *
+ * Method sources (pages about "KIVI: A Tuning-Free Asymmetric 2bit
+ * Quantization for KV Cache"):
+ *   - mlsanity.com index page, section "Abstract (arXiv)": keys quantized
+ *     per channel, values per token, 2-bit codes.
+ *   - study.space summary page (single summary paragraph): asymmetric
+ *     quantization, key quantization grouped over tokens, value codes
+ *     appended along the token axis, caches split into a quantized
+ *     ("grouped") part and a full-precision residual part that is merged
+ *     with the quantized part in decode attention.
+ *   - scholarfeed.org "KIVI" page, third quote: the residual is a
+ *     fixed-length buffer of recent tokens kept unquantized.
+ * Where the pages say nothing (the scale/zero formula, rounding, packing
+ * order, flush timing) the oracle takes the plainest reading, stated in
+ * kivi_oracle.c beside the function that applies it.
+ */
+#ifndef KIVI_ORACLE_H
+#define KIVI_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  KIVI_ORACLE_OK = 0,
+  KIVI_ORACLE_ERR_ARG = 1,
+  KIVI_ORACLE_ERR_STATE = 2,
+  KIVI_ORACLE_ERR_CAPACITY = 3,
+  KIVI_ORACLE_ERR_NOMEM = 4
+};
+
+/*
+ * One (batch element, KV head) unit of the cache, in host memory.
+ * Let E = 32 / bits codes per 32-bit word and Tq = the quantized-store
+ * capacity in tokens.  The arrays are this unit's slices of the cache
+ * buffers, laid out as:
+ *   k_codes [Tq][D/E]   word w of token t holds channels wE..wE+E-1,
+ *                       channel wE+i in bits [bits*i, bits*i+bits)
+ *   k_scale [Tq/G][D]   one (scale, zero) per key group (G tokens) and channel
+ *   k_zero  [Tq/G][D]
+ *   v_codes [Tq/E][D]   word (tb, d) holds tokens tb*E..tb*E+E-1 of channel
+ *                       d, token tb*E+i in bits [bits*i, bits*i+bits)
+ *   v_scale [Tq][D/Gv]  one (scale, zero) per token and value group (Gv
+ *   v_zero  [Tq][D/Gv]  channels)
+ *   k_res   [R][D]      residual keys, full precision (fp32 values)
+ *   v_res   [R][D]      residual values
+ */
+typedef struct {
+  int D;
+  int bits;
+  int G;
+  int Gv;
+  int R;
+  long long Tq;
+  uint32_t *k_codes;
+  float *k_scale;
+  float *k_zero;
+  uint32_t *v_codes;
+  float *v_scale;
+  float *v_zero;
+  float *k_res;
+  float *v_res;
+  long long n_q; /* tokens held in the quantized store */
+  int r;         /* tokens held in the residual window */
+} kivi_oracle_unit;
+
+/* Q: quantize one group of n values x[0], x[stride], ..., x[(n-1)*stride]. */
+int kivi_oracle_quantize_group(const float *x, long long n, long long stride,
+                               int bits, float *scale, float *zero,
+                               uint16_t *codes);
+
+/* P: pack 32/bits codes into one word, codes[0] in the least significant bits. */
+uint32_t kivi_oracle_pack_word(const uint16_t *codes, int bits);
+
+/* D: the dequantized value of code c with (scale, zero), in real arithmetic. */
+double kivi_oracle_dequant(uint32_t c, float scale, float zero);
+
+/* S: state machine of one unit. */
+int kivi_oracle_check_unit(const kivi_oracle_unit *u);
+int kivi_oracle_prefill(kivi_oracle_unit *u, const float *K, const float *V,
+                        long long T);
+int kivi_oracle_append(kivi_oracle_unit *u, const float *k, const float *v);
+
+/* Full-precision view of the unit's keys / values: out[(n_q + r) * D]. */
+int kivi_oracle_dequant_keys(const kivi_oracle_unit *u, double *out);
+int kivi_oracle_dequant_values(const kivi_oracle_unit *u, double *out);
+
+/* A: decode attention of n_heads query heads q[n_heads][D] against the
+ * unit, out[n_heads][D]. */
+int kivi_oracle_decode(const kivi_oracle_unit *u, const float *q, int n_heads,
+                       double sigma, double *out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif

@@ -1,0 +1,141 @@
+"""Pins for the oracle's quantizer (Q), packer (P) and dequantizer (D).
+
+Method: "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache",
+study.space summary (asymmetric quantization) and mlsanity.com index page,
+"Abstract (arXiv)" (2-bit codes).  The pages give no formula or worked
+example; the pins are hand-derived values (tests/golden/quantize_examples.txt)
+and invariants that any correct asymmetric min/max quantizer satisfies.
+"""
+import os
+import struct
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "quantize_examples.txt")
+
+
+def _f32_bits(x) -> int:
+    return struct.unpack("<I", struct.pack("<f", float(x)))[0]
+
+
+def _golden():
+    rows = []
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            rows.append([p.strip() for p in line.split("|")])
+    return rows
+
+
+QROWS = [r for r in _golden() if r[0] == "Q"]
+PROWS = [r for r in _golden() if r[0] == "P"]
+
+
+@pytest.mark.parametrize("row", QROWS, ids=[f"{r[1]}b:{r[2]}" for r in QROWS])
+def test_quantize_golden(row):
+    _, bits, xs, scale_hex, zero, codes = row
+    x = np.array([float(v) for v in xs.split()], np.float32)
+    s, z, c = oracle.quantize_group(x, int(bits))
+    assert _f32_bits(s) == int(scale_hex, 16)
+    assert _f32_bits(z) == _f32_bits(np.float32(float(zero)))  # sign of zero included
+    assert c.tolist() == [int(v) for v in codes.split()]
+
+
+@pytest.mark.parametrize("row", PROWS, ids=[f"{r[1]}b:{r[3]}" for r in PROWS])
+def test_pack_golden(row):
+    _, bits, codes, word = row
+    assert oracle.pack_word([int(v) for v in codes.split()], int(bits)) == int(word, 16)
+
+
+def test_golden_file_covers_every_width():
+    assert {int(r[1]) for r in QROWS} >= {1, 2, 4}
+    assert {int(r[1]) for r in PROWS} == {1, 2, 4, 8, 16}
+
+
+def test_dequant_closed_form():
+    # c * s + z in real arithmetic; these products and sums are exact.
+    assert oracle.dequant(0, 0.75, -1.25) == -1.25
+    assert oracle.dequant(3, 0.5, -1.0) == 0.5
+    assert oracle.dequant(15, 0.125, 2.0) == 3.875
+    # binary64 keeps c * s exact where binary32 would round
+    s = np.float32(0.1)
+    assert oracle.dequant(3, s, 0.0) == 3 * float(s)
+
+
+def _groups(rng, n_groups, size):
+    """Random groups: normal, outlier-heavy (x20 like the key outlier channels),
+    tiny-range, constant, and fp16-rounded."""
+    out = []
+    for i in range(n_groups):
+        kind = i % 5
+        if kind == 0:
+            x = rng.standard_normal(size)
+        elif kind == 1:
+            x = rng.standard_normal(size) * 20.0
+        elif kind == 2:
+            x = 1.0 + rng.standard_normal(size) * 1e-6
+        elif kind == 3:
+            x = np.full(size, rng.standard_normal())
+        else:
+            x = rng.standard_normal(size).astype(np.float16)
+        out.append(np.asarray(x, np.float32))
+    return out
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+def test_invariants(bits):
+    """Code range; min -> code 0 reconstructing exactly; max -> top code;
+    reconstruction error within half a step plus the rounding slack of s,
+    the quotient and the float inputs."""
+    rng = np.random.default_rng(bits)
+    L = 2 ** bits - 1
+    for x in _groups(rng, 200, 32):
+        s, z, c = oracle.quantize_group(x, bits)
+        assert c.min() >= 0 and c.max() <= L
+        assert z == x.min()
+        if x.max() == x.min():
+            assert s == 0 and (c == 0).all()
+            assert all(oracle.dequant(ci, s, z) == xi for ci, xi in zip(c, x))
+            continue
+        imin, imax = int(np.argmin(x)), int(np.argmax(x))
+        assert c[imin] == 0 and oracle.dequant(c[imin], s, z) == x.min()
+        assert c[imax] == L
+        ulp_s = np.spacing(np.float32(s))
+        ulp_x = np.spacing(np.float32(max(abs(x.min()), abs(x.max()))))
+        bound = float(s) / 2 + (L + 1) * float(ulp_s) + float(ulp_x)
+        for ci, xi in zip(c, x):
+            assert abs(oracle.dequant(ci, s, z) - float(xi)) <= bound
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_scale_zero_do_not_depend_on_order(bits):
+    rng = np.random.default_rng(7)
+    for x in _groups(rng, 50, 32):
+        s, z, c = oracle.quantize_group(x, bits)
+        perm = rng.permutation(x.size)
+        s2, z2, c2 = oracle.quantize_group(x[perm], bits)
+        assert _f32_bits(s) == _f32_bits(s2) and _f32_bits(z) == _f32_bits(z2)
+        assert (c2 == c[perm]).all()
+
+
+def test_codes_are_monotone_in_x():
+    rng = np.random.default_rng(3)
+    for bits in (2, 4):
+        for x in _groups(rng, 40, 32):
+            s, z, c = oracle.quantize_group(x, bits)
+            order = np.argsort(x, kind="stable")
+            assert (np.diff(c[order].astype(int)) >= 0).all()
+
+
+def test_sixteen_bit_codes_track_the_input():
+    # At b = 16 the step is range / 65535: the reconstruction is nearly exact.
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal(32).astype(np.float32) * 20
+    s, z, c = oracle.quantize_group(x, 16)
+    xh = np.array([oracle.dequant(ci, s, z) for ci in c])
+    assert np.max(np.abs(xh - x)) <= (x.max() - x.min()) / 65535
