@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark: KIVI 2-bit decode attention on B200.
+
+One step = one decode step of one attention layer through the C ABI:
+kivi_append_token (the new token's K/V into the residual window, flushing
+the window into the 2-bit store every R tokens) then kivi_decode_attention
+(fused dequant + q.K + online softmax + P.V over the packed codes and the
+window, then the cross-split merge).  Workload: the Llama-2-7B-shaped layer
+(B=8, 32 heads, D=128, context 4096, 2-bit, G=32, R=128) by default.
+
+L2 hygiene: `--layers` copies of the layer cache (default 32, the model's
+depth; 4.7 GB) are visited round-robin, so each step reads a cache that is
+not L2-resident (inputs larger than the 126 MB L2).
+
+Output: one JSON line (rank 0).  `value` = decode tokens/s over all ranks
+(B tokens per step per rank); `roofline` = the split kernel's algorithmic
+bytes / its CUDA-event time vs measured HBM peak; `e2e` = the same loop with
+the step's inputs copied from pinned host memory and the output copied back
+inside the timed region; `cpu_baseline` = the CPU oracle on a bounded sample
+of the same workload.  `--impl reference` times the CPU oracle alone.
+Multi-GPU (torchrun): independent replicas, one per rank (no collective on
+the data path); the barrier and max-over-ranks timing use torch.distributed.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_asymmetric_kv_quantize_b200 import workloads as W  # noqa: E402
+
+METRIC = "decode-attention tokens/s over 2-bit KV; achieved HBM GB/s vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=4096)
+    p.add_argument("--warmup", type=int, default=64)
+    p.add_argument("--impl", choices=["kivi", "reference"], default="kivi")
+    p.add_argument("--workload", default=W.LLAMA2_7B.name, choices=sorted(W.ALL))
+    p.add_argument("--layers", type=int, default=32)
+    p.add_argument("--kernel", choices=["default", "simt"], default="default")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-budget-s", type=float, default=15.0)
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(w: W.Workload, n_q: int, r: int) -> int:
+    """Bytes one decode call must move: every code, scale and zero of the
+    quantized store, the window tokens, q in and out (per unit: K codes
+    n_q*D*b/8, K meta (n_q/G)*D*8, V codes n_q*D*b/8, V meta n_q*(D/Gv)*8,
+    window r*D*2*es; plus B*Hq*D*es each for q and out)."""
+    es = 2 if w.dtype == "f16" else 4
+    per_unit = (2 * n_q * w.D * w.bits // 8 + (n_q // w.G) * w.D * 8 + n_q * (w.D // w.Gv) * 8
+                + r * w.D * 2 * es)
+    return w.B * w.Hkv * per_unit + 2 * w.B * w.Hq * w.D * es
+
+
+# --------------------------------------------------------------- clocks (NVML)
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons every ~5 ms while running."""
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report it, keep going
+            self.err = repr(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        sms = [s for s, _ in self.samples]
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        reasons = sorted(n for b, n in _REASONS.items() if mask & b and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sms)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_kivi(args, rank, world, local):
+    import bit_asymmetric_kv_quantize_b200 as kivi
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=device)
+
+    w = W.ALL[args.workload]
+    if w.steps:  # the streaming workload's decode loop is the step loop itself
+        w = w.with_(steps=0)
+    n_layers = max(1, args.layers)
+    e2e_steps = 0 if args.no_e2e else min(args.steps, 1024)
+    per_layer = -(-(args.warmup + args.steps + e2e_steps) // n_layers) + 1
+    capacity = -(-(w.T + per_layer) // w.R) * w.R
+    Kp, Vp = W.prompt_kv(w, device=device)
+    caches = []
+    for _ in range(n_layers):
+        c = kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, capacity, R=w.R, G=w.G, Gv=w.Gv,
+                           dtype=w.torch_dtype, device=device)
+        c.prefill(Kp, Vp)
+        caches.append(c)
+    del Kp, Vp
+    P = 16
+    ks, vs, qs = [], [], []
+    for i in range(P):
+        k, v = W.step_kv(w, i, device=device)
+        ks.append(k)
+        vs.append(v)
+        qs.append(W.query(w, i, device=device))
+    out = torch.empty(w.B, w.Hq, w.D, dtype=w.torch_dtype, device=device)
+    ws = caches[0].workspace(w.Hq)
+    for c in caches[1:]:
+        c._ws = ws
+    L = kivi.lib()
+    dec = L.kivi_decode_attention if args.kernel == "default" else L.kivi_decode_attention_simt
+    stream = torch.cuda.current_stream(device)
+    sh = stream.cuda_stream
+    cstructs = [ctypes.byref(c._c) for c in caches]
+    kp = [t.data_ptr() for t in ks]
+    vp = [t.data_ptr() for t in vs]
+    qp = [t.data_ptr() for t in qs]
+    op, wp, wn = out.data_ptr(), ws.data_ptr(), ws.numel()
+
+    def step(i, ev=None):
+        li = i % n_layers
+        rc = L.kivi_append_token(cstructs[li], kp[i % P], vp[i % P], sh)
+        if rc:
+            raise RuntimeError(f"append: {L.kivi_status_string(rc)}")
+        if ev is not None:
+            L.kivi_set_timing_events(ev[0], ev[1])
+        rc = dec(cstructs[li], qp[i % P], w.Hq, 1.0, op, wp, wn, sh)
+        if rc:
+            raise RuntimeError(f"decode: {L.kivi_status_string(rc)}")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+
+    # warm-up
+    for i in range(args.warmup):
+        step(i)
+    barrier()
+
+    # per-step events around the split kernel (created by one record each)
+    evs = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize(device)
+    ev_handles = [(e0.cuda_event, e1.cuda_event) for e0, e1 in evs]
+    fills = []
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        t0.record(stream)
+        for j in range(args.steps):
+            i = args.warmup + j
+            step(i, ev_handles[j])
+            c = caches[i % n_layers]
+            fills.append((c.n_q, c.r))
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+    L.kivi_set_timing_events(None, None)
+    barrier()
+    ms = t0.elapsed_time(t1)
+    split_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    ms_max = ms
+    if world > 1:
+        tt = torch.tensor([ms], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_max = float(tt.item())
+
+    # roofline of the split kernel: algorithmic bytes / event time
+    bytes_total = sum(algorithmic_bytes(w, nq, r) for nq, r in fills)
+    split_total_ms = sum(split_ms)
+    achieved = bytes_total / (split_total_ms * 1e-3) / 1e9
+    peak, peak_src = peak_hbm()
+    n_split = caches[0].num_splits(w.Hq)
+
+    # e2e: the same loop, inputs from pinned host memory, output read back
+    e2e = None
+    if not args.no_e2e:
+        hk = [t.cpu().pin_memory() for t in ks]
+        hv = [t.cpu().pin_memory() for t in vs]
+        hq = [t.cpu().pin_memory() for t in qs]
+        ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dk, dv, dq = torch.empty_like(ks[0]), torch.empty_like(vs[0]), torch.empty_like(qs[0])
+        h2d = 3 * ks[0].numel() * ks[0].element_size()
+        d2h = out.numel() * out.element_size()
+        n_e2e = e2e_steps
+        base = args.warmup + args.steps
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for j in range(n_e2e):
+            i = base + j
+            li = i % n_layers
+            dk.copy_(hk[i % P], non_blocking=True)
+            dv.copy_(hv[i % P], non_blocking=True)
+            dq.copy_(hq[i % P], non_blocking=True)
+            rc = L.kivi_append_token(cstructs[li], dk.data_ptr(), dv.data_ptr(), sh)
+            rc |= dec(cstructs[li], dq.data_ptr(), w.Hq, 1.0, op, wp, wn, sh)
+            if rc:
+                raise RuntimeError("e2e step failed")
+            ho.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e_ms], device=device)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": world * w.B * n_e2e / (e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "ms_per_step": e_ms / n_e2e}
+
+    result = None
+    if rank == 0:
+        tokens_per_s = world * w.B * args.steps / (ms_max * 1e-3)
+        result = {
+            "metric": METRIC,
+            "value": tokens_per_s,
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32" if args.kernel == "simt" else "f16xf16+f32",
+            "data": "synthetic",
+            "config": {
+                "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                "context": w.T, "bits": w.bits, "G": w.G, "Gv": w.Gv, "R": w.R,
+                "dtype_io": w.dtype, "kernel": args.kernel, "parallelism": f"replicas{world}",
+                "layers_rotated": n_layers,
+                "l2": f"inputs larger than L2: {n_layers} layer caches visited round-robin",
+                "decode_splits": n_split,
+            },
+            "roofline": {
+                "kernel": "decode_split", "bound": "hbm", "achieved": achieved, "peak": peak,
+                "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": None,
+                "algorithmic_bytes_per_launch": bytes_total / args.steps,
+                "avg_launch_us": split_total_ms * 1e3 / args.steps,
+            },
+            "e2e": e2e,
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk.summary(),
+        }
+    for c in caches:
+        del c
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result, w
+
+
+# --------------------------------------------------------------- CPU oracle arm
+
+def oracle_sample(w: W.Workload, n_units: int, steps: int, threads: int):
+    """Time `steps` decode steps (append + decode) of the CPU oracle on
+    `n_units` units of the workload; returns (seconds per step, units)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+
+    units = [(u // w.Hkv, u % w.Hkv) for u in range(min(n_units, w.B * w.Hkv))]
+    cap = -(-(w.T + steps + 1) // w.R) * w.R
+    oc = oracle.OracleCache(w.B, w.Hkv, w.D, w.bits, w.G, w.Gv, w.R, cap, units=units)
+    g = w.with_(B=1, Hkv=1, Hq=w.gq)
+    K, V = W.prompt_kv(g)
+    Kf, Vf = K[0, 0].float().numpy(), V[0, 0].float().numpy()
+    qs = W.query(w).float().numpy()
+    step_in = [tuple(t.float().numpy() for t in W.step_kv(w, i)) for i in range(min(steps, 4))]
+    gq = w.gq
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(lambda u: oc.prefill_unit(u[0], u[1], Kf, Vf), units))
+
+        def one(u, i):
+            b, h = u
+            k, v = step_in[i % len(step_in)]
+            oc.append_unit(b, h, k[b, h], v[b, h])
+            oc.decode_unit(b, h, qs[b, h * gq:(h + 1) * gq], 1.0)
+
+        t = time.perf_counter()
+        for i in range(steps):
+            list(ex.map(lambda u: one(u, i), units))
+        dt = time.perf_counter() - t
+    return dt / steps, len(units)
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w: W.Workload, budget_s: float):
+    threads = cpu_threads()
+    # calibrate on one step of a few units, then size the sample to the budget
+    per_step, n = oracle_sample(w, threads, 1, threads)
+    per_unit_cpu = per_step * threads / n
+    n_units = min(w.B * w.Hkv, max(threads, int(threads * 4)))
+    steps = max(1, int(budget_s * threads / (per_unit_cpu * n_units)))
+    per_step, n = oracle_sample(w, n_units, steps, threads)
+    full_step = per_step * (w.B * w.Hkv) / n
+    return {"value": w.B / full_step, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{steps} steps x {n} of {w.B * w.Hkv} (batch, KV head) units, "
+                      f"append + decode, scaled to the full batch; single oracle threads "
+                      f"fanned out over units"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = W.ALL[args.workload]
+    if w.steps:
+        w = w.with_(steps=0)
+    threads = cpu_threads()
+    budget = 120.0  # seconds of wall time for warm-up + timed steps
+    per_step, n = oracle_sample(w, threads, 1, threads)
+    n_units = max(1, min(w.B * w.Hkv,
+                         int(budget / max(1, args.steps + args.warmup) / per_step * n)))
+    oracle_sample(w, n_units, max(1, args.warmup), threads)
+    per_step, n = oracle_sample(w, n_units, args.steps, threads)
+    full_step = per_step * (w.B * w.Hkv) / n
+    value = w.B / full_step
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": full_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "context": w.T, "bits": w.bits, "G": w.G, "Gv": w.Gv, "R": w.R},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: append + decode on {n} of {w.B * w.Hkv} units, "
+                                   f"scaled to the full batch"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    res, w = run_kivi(args, rank, world, local)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(w, args.cpu_budget_s)
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

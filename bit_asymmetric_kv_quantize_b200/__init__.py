@@ -1,0 +1,229 @@
+"""KIVI asymmetric 2/4-bit KV cache with fused decode attention, for NVIDIA B200.
+
+Python binding of ``libkivi.so`` (C ABI in ``include/kivi.h``).  This module
+only marshals arguments: torch supplies device memory and the current CUDA
+stream; every step of the method (quantize, pack, residual window, decode
+attention, split merge) runs in the library's CUDA kernels.  There is no CPU
+path: if the library is missing or no CUDA device is present the calls raise.
+
+Method: "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache"
+(mlsanity.com index page, "Abstract (arXiv)"; study.space summary).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkivi.so")
+
+KIVI_F16, KIVI_F32 = 0, 1
+NUM_BUFFERS = 8
+BUFFER_NAMES = ("k_codes", "k_scale", "k_zero", "v_codes", "v_scale", "v_zero", "k_res", "v_res")
+STATUS = {0: "KIVI_OK", 1: "KIVI_ERR_ARG", 2: "KIVI_ERR_UNSUPPORTED", 3: "KIVI_ERR_STATE",
+          4: "KIVI_ERR_CAPACITY", 5: "KIVI_ERR_WORKSPACE", 6: "KIVI_ERR_CUDA"}
+
+EXPORTED = (
+    "kivi_buffer_sizes", "kivi_cache_init", "kivi_quantize_prefill", "kivi_append_token",
+    "kivi_decode_workspace_bytes", "kivi_decode_attention", "kivi_decode_attention_simt",
+    "kivi_set_timing_events", "kivi_decode_num_splits", "kivi_status_string",
+)
+
+
+class KiviError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib().kivi_status_string(status).decode()}")
+
+
+class KiviDims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("D", ctypes.c_int),
+                ("bits", ctypes.c_int), ("G", ctypes.c_int), ("Gv", ctypes.c_int),
+                ("R", ctypes.c_int), ("capacity", ctypes.c_longlong), ("dtype", ctypes.c_int)]
+
+
+class KiviCacheC(ctypes.Structure):
+    _fields_ = [("dims", KiviDims),
+                ("k_codes", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
+                ("k_zero", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
+                ("v_scale", ctypes.c_void_p), ("v_zero", ctypes.c_void_p),
+                ("k_res", ctypes.c_void_p), ("v_res", ctypes.c_void_p),
+                ("n_q", ctypes.c_longlong), ("r", ctypes.c_int)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libkivi.so (built in-tree by ``python -m bit_asymmetric_kv_quantize_b200._build``)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m bit_asymmetric_kv_quantize_b200._build`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, ci, ll, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+            cp = ctypes.POINTER(KiviCacheC)
+            dp = ctypes.POINTER(KiviDims)
+            L.kivi_buffer_sizes.argtypes = [dp, ctypes.POINTER(sz * NUM_BUFFERS)]
+            L.kivi_cache_init.argtypes = [cp, dp, ctypes.POINTER(vp * NUM_BUFFERS)]
+            L.kivi_quantize_prefill.argtypes = [cp, vp, vp, ll, vp]
+            L.kivi_append_token.argtypes = [cp, vp, vp, vp]
+            L.kivi_decode_workspace_bytes.argtypes = [cp, ci]
+            L.kivi_decode_workspace_bytes.restype = sz
+            dec = [cp, vp, ci, ctypes.c_float, vp, vp, sz, vp]
+            L.kivi_decode_attention.argtypes = dec
+            L.kivi_decode_attention_simt.argtypes = dec
+            L.kivi_set_timing_events.argtypes = [vp, vp]
+            L.kivi_set_timing_events.restype = None
+            L.kivi_decode_num_splits.argtypes = [cp, ci]
+            L.kivi_status_string.argtypes = [ci]
+            L.kivi_status_string.restype = ctypes.c_char_p
+            _lib = L
+        return _lib
+
+
+def _dtype_code(dtype: torch.dtype) -> int:
+    if dtype == torch.float16:
+        return KIVI_F16
+    if dtype == torch.float32:
+        return KIVI_F32
+    raise ValueError(f"unsupported dtype {dtype}")
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise KiviError(rc, what)
+
+
+def buffer_sizes(B, Hkv, D, bits, capacity, R=128, G=32, Gv=32, dtype=torch.float16):
+    dims = KiviDims(B, Hkv, D, bits, G, Gv, R, capacity, _dtype_code(dtype))
+    out = (ctypes.c_size_t * NUM_BUFFERS)()
+    _check(lib().kivi_buffer_sizes(ctypes.byref(dims), ctypes.byref(out)), "kivi_buffer_sizes")
+    return dict(zip(BUFFER_NAMES, list(out)))
+
+
+class KiviCache:
+    """One layer's KIVI cache on a CUDA device.
+
+    Buffers are torch tensors in the library's ABI layout (see include/kivi.h);
+    ``n_q`` / ``r`` are the library-owned counters.  Calls are asynchronous on
+    torch's current stream of the cache's device.
+    """
+
+    def __init__(self, B: int, Hkv: int, D: int, bits: int, capacity: int, R: int = 128,
+                 G: int = 32, Gv: int = 32, dtype: torch.dtype = torch.float16,
+                 device="cuda"):
+        self.device = torch.device(device)
+        if self.device.type != "cuda":
+            raise ValueError("KiviCache lives in CUDA device memory")
+        if self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
+        self.dtype = dtype
+        self._dims = KiviDims(B, Hkv, D, bits, G, Gv, R, capacity, _dtype_code(dtype))
+        sizes = buffer_sizes(B, Hkv, D, bits, capacity, R, G, Gv, dtype)
+        self.buffers = {n: torch.empty(max(sizes[n], 16), dtype=torch.uint8, device=self.device)
+                        for n in BUFFER_NAMES}
+        ptrs = (ctypes.c_void_p * NUM_BUFFERS)(*[self.buffers[n].data_ptr() for n in BUFFER_NAMES])
+        self._c = KiviCacheC()
+        _check(lib().kivi_cache_init(ctypes.byref(self._c), ctypes.byref(self._dims),
+                                     ctypes.byref(ptrs)), "kivi_cache_init")
+        self._ws: Optional[torch.Tensor] = None
+        E = 32 // bits
+        Tq = capacity - R
+        self.B, self.Hkv, self.D, self.bits, self.R, self.capacity = B, Hkv, D, bits, R, capacity
+        self.shapes = {
+            "k_codes": ((B, Hkv, Tq, D // E), torch.int32),
+            "k_scale": ((B, Hkv, Tq // G, D), torch.float32),
+            "k_zero": ((B, Hkv, Tq // G, D), torch.float32),
+            "v_codes": ((B, Hkv, Tq // E, D), torch.int32),
+            "v_scale": ((B, Hkv, Tq, D // Gv), torch.float32),
+            "v_zero": ((B, Hkv, Tq, D // Gv), torch.float32),
+            "k_res": ((B, Hkv, R, D), dtype),
+            "v_res": ((B, Hkv, R, D), dtype),
+        }
+
+    # -- state
+    @property
+    def n_q(self) -> int:
+        return int(self._c.n_q)
+
+    @property
+    def r(self) -> int:
+        return int(self._c.r)
+
+    def view(self, name: str) -> torch.Tensor:
+        """A buffer viewed with its ABI shape (int32 for code words)."""
+        shape, dt = self.shapes[name]
+        n = 1
+        for s in shape:
+            n *= s
+        return self.buffers[name][: n * torch.tensor([], dtype=dt).element_size()].view(dt).view(shape)
+
+    def _stream(self) -> int:
+        return torch.cuda.current_stream(self.device).cuda_stream
+
+    def _arg(self, t: torch.Tensor, shape, name: str) -> int:
+        if t.device != self.device or t.dtype != self.dtype or not t.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous {self.dtype} tensor on {self.device}")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+        return t.data_ptr()
+
+    # -- the three calls
+    def prefill(self, K: torch.Tensor, V: torch.Tensor) -> None:
+        T = K.shape[2]
+        shape = (self.B, self.Hkv, T, self.D)
+        pk, pv = self._arg(K, shape, "K"), self._arg(V, shape, "V")
+        with torch.cuda.device(self.device):
+            _check(lib().kivi_quantize_prefill(ctypes.byref(self._c), pk, pv, T, self._stream()),
+                   "kivi_quantize_prefill")
+
+    def append(self, k: torch.Tensor, v: torch.Tensor) -> None:
+        shape = (self.B, self.Hkv, self.D)
+        pk, pv = self._arg(k, shape, "k"), self._arg(v, shape, "v")
+        with torch.cuda.device(self.device):
+            _check(lib().kivi_append_token(ctypes.byref(self._c), pk, pv, self._stream()),
+                   "kivi_append_token")
+
+    def workspace_bytes(self, Hq: int) -> int:
+        with torch.cuda.device(self.device):
+            return int(lib().kivi_decode_workspace_bytes(ctypes.byref(self._c), Hq))
+
+    def workspace(self, Hq: int) -> torch.Tensor:
+        need = self.workspace_bytes(Hq)
+        if need == 0:
+            raise KiviError(1, "kivi_decode_workspace_bytes")
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def num_splits(self, Hq: int) -> int:
+        with torch.cuda.device(self.device):
+            return int(lib().kivi_decode_num_splits(ctypes.byref(self._c), Hq))
+
+    def decode(self, q: torch.Tensor, softmax_scale: float, out: Optional[torch.Tensor] = None,
+               kernel: str = "default") -> torch.Tensor:
+        Hq = q.shape[1]
+        pq = self._arg(q, (self.B, Hq, self.D), "q")
+        if out is None:
+            out = torch.empty_like(q)
+        po = self._arg(out, (self.B, Hq, self.D), "out")
+        ws = self.workspace(Hq)
+        fn = lib().kivi_decode_attention if kernel == "default" else lib().kivi_decode_attention_simt
+        with torch.cuda.device(self.device):
+            _check(fn(ctypes.byref(self._c), pq, Hq, float(softmax_scale), po, ws.data_ptr(),
+                      ws.numel(), self._stream()), "kivi_decode_attention")
+        return out
+
+
+def set_timing_events(start: Optional[torch.cuda.Event], stop: Optional[torch.cuda.Event]) -> None:
+    """Have later decode calls on this thread record these events around the split kernel."""
+    lib().kivi_set_timing_events(start.cuda_event if start is not None else None,
+                                 stop.cuda_event if stop is not None else None)

@@ -1,0 +1,269 @@
+// kivi_api.cu -- the extern "C" boundary of libkivi.so (declared in
+// include/kivi.h): argument and state validation, the residual-window state
+// machine, the decode split heuristic, and kernel launches.  No device
+// memory is allocated and no call synchronizes.
+#include <limits.h>
+#include <stdint.h>
+
+#include "kivi.h"
+#include "kivi_internal.cuh"
+
+namespace {
+
+using kivi::CacheView;
+using kivi::DecodeArgs;
+
+thread_local cudaEvent_t g_ev0 = nullptr;
+thread_local cudaEvent_t g_ev1 = nullptr;
+
+constexpr int kMaxSplits = 64;
+
+int check_dims(const kivi_dims* d) {
+  if (!d) return KIVI_ERR_ARG;
+  if (d->B <= 0 || d->Hkv <= 0 || d->D <= 0 || d->R <= 0 || d->capacity <= 0)
+    return KIVI_ERR_ARG;
+  if (d->bits != 2 && d->bits != 4) return KIVI_ERR_UNSUPPORTED;
+  if (d->G != kivi::kG || d->Gv != kivi::kGv) return KIVI_ERR_UNSUPPORTED;
+  if (d->D != 32 && d->D != 64 && d->D != 128) return KIVI_ERR_UNSUPPORTED;
+  if (d->R % kivi::kTile != 0) return KIVI_ERR_UNSUPPORTED;
+  if (d->capacity % d->R != 0) return KIVI_ERR_UNSUPPORTED;
+  if (d->dtype != KIVI_F16 && d->dtype != KIVI_F32) return KIVI_ERR_UNSUPPORTED;
+  if ((long long)d->B * d->Hkv > 65535) return KIVI_ERR_UNSUPPORTED;  // grid y limit
+  return KIVI_OK;
+}
+
+int check_cache(const kivi_cache* c) {
+  if (!c) return KIVI_ERR_ARG;
+  int rc = check_dims(&c->dims);
+  if (rc) return rc;
+  const long long Tq = c->dims.capacity - c->dims.R;
+  if (Tq > 0 && (!c->k_codes || !c->k_scale || !c->k_zero || !c->v_codes || !c->v_scale ||
+                 !c->v_zero))
+    return KIVI_ERR_ARG;
+  if (!c->k_res || !c->v_res) return KIVI_ERR_ARG;
+  return KIVI_OK;
+}
+
+size_t elem_bytes(int dtype) { return dtype == KIVI_F32 ? 4 : 2; }
+
+CacheView view(const kivi_cache* c) {
+  CacheView v;
+  v.k_codes = c->k_codes;
+  v.k_scale = c->k_scale;
+  v.k_zero = c->k_zero;
+  v.v_codes = c->v_codes;
+  v.v_scale = c->v_scale;
+  v.v_zero = c->v_zero;
+  v.k_res = c->k_res;
+  v.v_res = c->v_res;
+  v.Tq = c->dims.capacity - c->dims.R;
+  v.R = c->dims.R;
+  return v;
+}
+
+// SM count of the current device, queried once per device.
+int device_sms() {
+  static int cached[128] = {0};
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < 128 && cached[dev] > 0) return cached[dev];
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < 128) cached[dev] = sms;
+  return sms;
+}
+
+// Upper bound on splits for this cache shape: enough CTAs for ~4 per SM,
+// never more than kMaxSplits or than the tiles a full cache holds.
+int max_splits(const kivi_dims& d, int sms) {
+  const long long units = (long long)d.B * d.Hkv;
+  long long want = (4LL * sms + units - 1) / units;
+  long long tiles = d.capacity / kivi::kTile;
+  long long s = want < tiles ? want : tiles;
+  if (s > kMaxSplits) s = kMaxSplits;
+  return s < 1 ? 1 : (int)s;
+}
+
+// Splits for the current fill: at most max_splits, each split a contiguous
+// range of whole 32-token tiles (quantized tiles first, then the window).
+void plan_splits(const kivi_cache* c, int sms, int* n_split, int* tiles_per_split) {
+  const long long tiles = c->n_q / kivi::kTile + (c->r + kivi::kTile - 1) / kivi::kTile;
+  int s = max_splits(c->dims, sms);
+  if (s > tiles) s = (int)tiles;
+  if (s < 1) s = 1;
+  long long tps = (tiles + s - 1) / s;
+  *tiles_per_split = (int)tps;
+  *n_split = (int)((tiles + tps - 1) / tps);
+}
+
+size_t workspace_bytes(const kivi_dims& d, int Hq, int sms) {
+  return (size_t)d.B * Hq * max_splits(d, sms) * (d.D + 2) * sizeof(float);
+}
+
+int decode_common(const kivi_cache* c, const void* q, int Hq, float softmax_scale, void* out,
+                  void* workspace, size_t ws_bytes, void* stream, bool simt) {
+  int rc = check_cache(c);
+  if (rc) return rc;
+  if (!q || !out || Hq <= 0 || Hq % c->dims.Hkv != 0) return KIVI_ERR_ARG;
+  const int gq = Hq / c->dims.Hkv;
+  if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KIVI_ERR_UNSUPPORTED;
+  if (c->n_q + c->r == 0) return KIVI_ERR_STATE;
+  const int sms = device_sms();
+  if (sms <= 0) return KIVI_ERR_CUDA;
+  if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(c->dims, Hq, sms))
+    return KIVI_ERR_WORKSPACE;
+  DecodeArgs a;
+  a.c = view(c);
+  a.q = q;
+  a.out = out;
+  a.ws = (float*)workspace;
+  a.units = c->dims.B * c->dims.Hkv;
+  a.Hkv = c->dims.Hkv;
+  a.gq = gq;
+  a.D = c->dims.D;
+  a.bits = c->dims.bits;
+  a.dtype = c->dims.dtype;
+  a.n_q = c->n_q;
+  a.r = c->r;
+  a.qscale = softmax_scale * kivi::kLog2e;
+  plan_splits(c, sms, &a.n_split, &a.tiles_per_split);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t err = kivi::launch_decode_simt(a, s, g_ev0, g_ev1);
+  (void)simt;
+  if (err == cudaSuccess) err = kivi::launch_decode_combine(a, s);
+  return err == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kivi_buffer_sizes(const kivi_dims* dims, size_t out_bytes[KIVI_NUM_BUFFERS]) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!out_bytes) return KIVI_ERR_ARG;
+  const long long units = (long long)dims->B * dims->Hkv;
+  const long long Tq = dims->capacity - dims->R;
+  const int E = 32 / dims->bits;
+  const size_t f = sizeof(float);
+  out_bytes[KIVI_BUF_K_CODES] = (size_t)(units * Tq * (dims->D / E)) * sizeof(uint32_t);
+  out_bytes[KIVI_BUF_K_SCALE] = (size_t)(units * (Tq / dims->G) * dims->D) * f;
+  out_bytes[KIVI_BUF_K_ZERO] = out_bytes[KIVI_BUF_K_SCALE];
+  out_bytes[KIVI_BUF_V_CODES] = (size_t)(units * (Tq / E) * dims->D) * sizeof(uint32_t);
+  out_bytes[KIVI_BUF_V_SCALE] = (size_t)(units * Tq * (dims->D / dims->Gv)) * f;
+  out_bytes[KIVI_BUF_V_ZERO] = out_bytes[KIVI_BUF_V_SCALE];
+  out_bytes[KIVI_BUF_K_RES] = (size_t)(units * dims->R * dims->D) * elem_bytes(dims->dtype);
+  out_bytes[KIVI_BUF_V_RES] = out_bytes[KIVI_BUF_K_RES];
+  return KIVI_OK;
+}
+
+int kivi_cache_init(kivi_cache* cache, const kivi_dims* dims,
+                    void* const buffers[KIVI_NUM_BUFFERS]) {
+  if (!cache || !buffers) return KIVI_ERR_ARG;
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  const bool has_store = dims->capacity > dims->R;
+  for (int i = 0; i < KIVI_NUM_BUFFERS; ++i) {
+    const bool needed = has_store || i == KIVI_BUF_K_RES || i == KIVI_BUF_V_RES;
+    if (needed && !buffers[i]) return KIVI_ERR_ARG;
+    if (((uintptr_t)buffers[i] & 15) != 0) return KIVI_ERR_ARG;
+  }
+  cache->dims = *dims;
+  cache->k_codes = (uint32_t*)buffers[KIVI_BUF_K_CODES];
+  cache->k_scale = (float*)buffers[KIVI_BUF_K_SCALE];
+  cache->k_zero = (float*)buffers[KIVI_BUF_K_ZERO];
+  cache->v_codes = (uint32_t*)buffers[KIVI_BUF_V_CODES];
+  cache->v_scale = (float*)buffers[KIVI_BUF_V_SCALE];
+  cache->v_zero = (float*)buffers[KIVI_BUF_V_ZERO];
+  cache->k_res = buffers[KIVI_BUF_K_RES];
+  cache->v_res = buffers[KIVI_BUF_V_RES];
+  cache->n_q = 0;
+  cache->r = 0;
+  return KIVI_OK;
+}
+
+int kivi_quantize_prefill(kivi_cache* cache, const void* K, const void* V, long long T,
+                          void* stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (T < 0 || (T > 0 && (!K || !V))) return KIVI_ERR_ARG;
+  if (cache->n_q != 0 || cache->r != 0) return KIVI_ERR_STATE;
+  if (T > cache->dims.capacity) return KIVI_ERR_CAPACITY;
+  if (T == 0) return KIVI_OK;
+  const int R = cache->dims.R;
+  const int r = (int)((T - 1) % R) + 1;
+  const long long n_q = T - r;
+  if (n_q / kivi::kTile + 1 > (long long)INT_MAX) return KIVI_ERR_UNSUPPORTED;
+  cudaError_t err = kivi::launch_prefill(view(cache), cache->dims.B * cache->dims.Hkv,
+                                         cache->dims.D, cache->dims.bits, cache->dims.dtype, K,
+                                         V, T, n_q, r, (cudaStream_t)stream);
+  if (err != cudaSuccess) return KIVI_ERR_CUDA;
+  cache->n_q = n_q;
+  cache->r = r;
+  return KIVI_OK;
+}
+
+int kivi_append_token(kivi_cache* cache, const void* k, const void* v, void* stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!k || !v) return KIVI_ERR_ARG;
+  if (cache->n_q + cache->r + 1 > cache->dims.capacity) return KIVI_ERR_CAPACITY;
+  const bool flush = cache->r == cache->dims.R;
+  const int slot = flush ? 0 : cache->r;
+  cudaError_t err = kivi::launch_append(view(cache), cache->dims.B * cache->dims.Hkv,
+                                        cache->dims.D, cache->dims.bits, cache->dims.dtype, k, v,
+                                        cache->n_q, slot, flush, (cudaStream_t)stream);
+  if (err != cudaSuccess) return KIVI_ERR_CUDA;
+  if (flush) cache->n_q += cache->dims.R;
+  cache->r = slot + 1;
+  return KIVI_OK;
+}
+
+size_t kivi_decode_workspace_bytes(const kivi_cache* cache, int Hq) {
+  if (check_cache(cache) != KIVI_OK || Hq <= 0 || Hq % cache->dims.Hkv != 0) return 0;
+  const int sms = device_sms();
+  if (sms <= 0) return 0;
+  return workspace_bytes(cache->dims, Hq, sms);
+}
+
+int kivi_decode_attention(const kivi_cache* cache, const void* q, int Hq, float softmax_scale,
+                          void* out, void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_common(cache, q, Hq, softmax_scale, out, workspace, workspace_bytes, stream,
+                       false);
+}
+
+int kivi_decode_attention_simt(const kivi_cache* cache, const void* q, int Hq,
+                               float softmax_scale, void* out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return decode_common(cache, q, Hq, softmax_scale, out, workspace, workspace_bytes, stream,
+                       true);
+}
+
+void kivi_set_timing_events(void* start_event, void* stop_event) {
+  g_ev0 = (cudaEvent_t)start_event;
+  g_ev1 = (cudaEvent_t)stop_event;
+}
+
+int kivi_decode_num_splits(const kivi_cache* cache, int Hq) {
+  if (check_cache(cache) != KIVI_OK || Hq <= 0 || Hq % cache->dims.Hkv != 0) return 0;
+  if (cache->n_q + cache->r == 0) return 0;
+  const int sms = device_sms();
+  if (sms <= 0) return 0;
+  int n, tps;
+  plan_splits(cache, sms, &n, &tps);
+  return n;
+}
+
+const char* kivi_status_string(int status) {
+  switch (status) {
+    case KIVI_OK: return "KIVI_OK";
+    case KIVI_ERR_ARG: return "KIVI_ERR_ARG: invalid argument";
+    case KIVI_ERR_UNSUPPORTED: return "KIVI_ERR_UNSUPPORTED: shape or format not built";
+    case KIVI_ERR_STATE: return "KIVI_ERR_STATE: cache state does not allow this call";
+    case KIVI_ERR_CAPACITY: return "KIVI_ERR_CAPACITY: tokens exceed the cache capacity";
+    case KIVI_ERR_WORKSPACE: return "KIVI_ERR_WORKSPACE: workspace missing, small or misaligned";
+    case KIVI_ERR_CUDA: return "KIVI_ERR_CUDA: CUDA launch or query failed";
+  }
+  return "unknown kivi status";
+}
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+// kivi_internal.cuh -- device-side view of a KIVI cache and small helpers
+// shared by the kernels of libkivi.so (not part of the public ABI).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kivi {
+
+constexpr int kG = 32;        // key group: tokens per (group, channel) scale
+constexpr int kGv = 32;       // value group: channels per (token, group) scale
+constexpr int kTile = 32;     // tokens per quantize tile (= kG, a multiple of E)
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Device view of one cache; per-unit strides follow the ABI layout.
+struct CacheView {
+  uint32_t* k_codes;
+  float* k_scale;
+  float* k_zero;
+  uint32_t* v_codes;
+  float* v_scale;
+  float* v_zero;
+  void* k_res;
+  void* v_res;
+  long long Tq;  // quantized-store capacity per unit, tokens
+  int R;         // residual window
+};
+
+template <int D, int BITS>
+struct Layout {
+  static constexpr int E = 32 / BITS;       // codes per word
+  static constexpr int WK = D / E;          // key words per token
+  static constexpr int NJ = D / kGv;        // value groups per token
+  static constexpr uint32_t MASK = (1u << BITS) - 1u;
+  static constexpr int L = (1 << BITS) - 1;  // top code
+  __host__ __device__ static long long k_codes_unit(long long Tq) { return Tq * WK; }
+  __host__ __device__ static long long k_meta_unit(long long Tq) { return (Tq / kG) * D; }
+  __host__ __device__ static long long v_codes_unit(long long Tq) { return (Tq / E) * D; }
+  __host__ __device__ static long long v_meta_unit(long long Tq) { return Tq * NJ; }
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Launchers (host), implemented in the .cu files.  Each returns a
+// cudaError_t from the launch.
+cudaError_t launch_prefill(const CacheView& c, int units, int D, int bits, int dtype,
+                           const void* K, const void* V, long long T, long long n_q, int r,
+                           cudaStream_t s);
+cudaError_t launch_append(const CacheView& c, int units, int D, int bits, int dtype,
+                          const void* k, const void* v, long long n_q, int slot, bool flush,
+                          cudaStream_t s);
+
+struct DecodeArgs {
+  CacheView c;
+  const void* q;   // [B][Hq][D]
+  void* out;       // [B][Hq][D]
+  float* ws;       // partials [B*Hq][n_split][D + 2]
+  int units;       // B * Hkv
+  int Hkv;
+  int gq;          // Hq / Hkv
+  int D;
+  int bits;
+  int dtype;
+  long long n_q;
+  int r;
+  float qscale;    // softmax_scale * log2(e)
+  int n_split;
+  int tiles_per_split;
+};
+
+cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s, cudaEvent_t ev0,
+                               cudaEvent_t ev1);
+cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t s);
+
+}  // namespace kivi

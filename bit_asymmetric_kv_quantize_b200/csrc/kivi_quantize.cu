@@ -1,0 +1,219 @@
+// kivi_quantize.cu -- prefill, append and flush kernels of the KIVI cache.
+//
+// Method: "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache".
+// Keys are quantized per channel over groups of kG consecutive tokens and
+// values per token over groups of kGv consecutive channels (mlsanity.com
+// index page, "Abstract (arXiv)"; study.space summary: key groups span
+// tokens).  Each group gets an asymmetric binary32 scale and zero
+// (study.space summary: asymmetric quantizer).  Recent tokens stay in a
+// full-precision window of R tokens that is quantized as a block when full
+// (study.space summary: grouped and residual parts; scholarfeed.org "KIVI"
+// page, third quote: fixed-length residual buffer).
+//
+// Bit-exactness: every group is reduced by one thread in element order with
+// strict compares (first occurrence kept among equal values, which fixes the
+// sign of a zero minimum), and the scale and quotients use the IEEE
+// round-to-nearest intrinsics __fsub_rn / __fdiv_rn and __float2int_rn
+// (half to even).  No reciprocal, no contraction.
+#include "kivi_internal.cuh"
+
+namespace kivi {
+namespace {
+
+// Quantize one tile of kTile tokens (= one key group) of one unit.
+//   Ksrc, Vsrc: the tile's first token row; rows are D elements apart.
+//   t0: token position of the tile in the quantized store (multiple of kTile).
+// blockDim.x == D.  Thread d reduces key channel d over the tile's tokens;
+// thread i reduces value group (token i / NJ, group i % NJ) over kGv channels.
+// Codes go through shared memory and are packed by all threads.
+template <int D, int BITS, typename T>
+__device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit,
+                                              const T* __restrict__ Ksrc,
+                                              const T* __restrict__ Vsrc, long long t0,
+                                              uint8_t* ck, uint8_t* cv) {
+  using Lt = Layout<D, BITS>;
+  constexpr int E = Lt::E, WK = Lt::WK, NJ = Lt::NJ;
+  const float Lf = (float)Lt::L;
+  const int tid = threadIdx.x;
+
+  // ---- keys: channel tid over kTile tokens
+  {
+    float x[kTile];
+#pragma unroll
+    for (int t = 0; t < kTile; ++t) x[t] = to_f32(Ksrc[(long long)t * D + tid]);
+    float mn = x[0], mx = x[0];
+#pragma unroll
+    for (int t = 1; t < kTile; ++t) {
+      if (x[t] < mn) mn = x[t];
+      if (x[t] > mx) mx = x[t];
+    }
+    const float s = __fdiv_rn(__fsub_rn(mx, mn), Lf);
+    const long long g = t0 / kG;
+    c.k_scale[unit * Lt::k_meta_unit(c.Tq) + g * D + tid] = s;
+    c.k_zero[unit * Lt::k_meta_unit(c.Tq) + g * D + tid] = mn;
+#pragma unroll
+    for (int t = 0; t < kTile; ++t) {
+      int code = 0;
+      if (s != 0.0f) {
+        code = __float2int_rn(__fdiv_rn(__fsub_rn(x[t], mn), s));
+        code = min(max(code, 0), Lt::L);
+      }
+      ck[t * D + tid] = (uint8_t)code;
+    }
+  }
+  // ---- values: token tid / NJ, channel group tid % NJ
+  {
+    const int t = tid / NJ, j = tid % NJ;
+    const T* src = Vsrc + (long long)t * D + j * kGv;
+    float x[kGv];
+#pragma unroll
+    for (int i = 0; i < kGv; ++i) x[i] = to_f32(src[i]);
+    float mn = x[0], mx = x[0];
+#pragma unroll
+    for (int i = 1; i < kGv; ++i) {
+      if (x[i] < mn) mn = x[i];
+      if (x[i] > mx) mx = x[i];
+    }
+    const float s = __fdiv_rn(__fsub_rn(mx, mn), Lf);
+    const long long mo = unit * Lt::v_meta_unit(c.Tq) + (t0 + t) * NJ + j;
+    c.v_scale[mo] = s;
+    c.v_zero[mo] = mn;
+#pragma unroll
+    for (int i = 0; i < kGv; ++i) {
+      int code = 0;
+      if (s != 0.0f) {
+        code = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], mn), s));
+        code = min(max(code, 0), Lt::L);
+      }
+      cv[t * D + j * kGv + i] = (uint8_t)code;
+    }
+  }
+  __syncthreads();
+  // ---- pack: keys along channels, values along tokens; D*BITS words each
+  constexpr int NW = kTile * WK;  // == (kTile / E) * D == D * BITS
+  uint32_t* kdst = c.k_codes + unit * Lt::k_codes_unit(c.Tq) + t0 * WK;
+  uint32_t* vdst = c.v_codes + unit * Lt::v_codes_unit(c.Tq) + (t0 / E) * D;
+#pragma unroll
+  for (int k = tid; k < NW; k += D) {
+    const int t = k / WK, w = k % WK;
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) word |= (uint32_t)ck[t * D + w * E + i] << (BITS * i);
+    kdst[k] = word;
+  }
+#pragma unroll
+  for (int k = tid; k < NW; k += D) {
+    const int tb = k / D, d = k % D;
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) word |= (uint32_t)cv[(tb * E + i) * D + d] << (BITS * i);
+    vdst[k] = word;
+  }
+  __syncthreads();
+}
+
+// grid (n_q / kTile + 1, units); the last x-block copies the r window tokens.
+template <int D, int BITS, typename T>
+__global__ void __launch_bounds__(D) prefill_kernel(CacheView c, const T* __restrict__ K,
+                                                    const T* __restrict__ V, long long T_len,
+                                                    long long n_q, int r) {
+  __shared__ uint8_t ck[kTile * D];
+  __shared__ uint8_t cv[kTile * D];
+  const long long unit = blockIdx.y;
+  const long long tile = blockIdx.x;
+  const T* Ku = K + unit * T_len * D;
+  const T* Vu = V + unit * T_len * D;
+  if (tile < n_q / kTile) {
+    quantize_tile<D, BITS, T>(c, unit, Ku + tile * kTile * D, Vu + tile * kTile * D,
+                              tile * kTile, ck, cv);
+  } else {
+    T* kr = reinterpret_cast<T*>(c.k_res) + unit * c.R * D;
+    T* vr = reinterpret_cast<T*>(c.v_res) + unit * c.R * D;
+    for (int i = threadIdx.x; i < r * D; i += D) {
+      kr[i] = Ku[n_q * D + i];
+      vr[i] = Vu[n_q * D + i];
+    }
+  }
+}
+
+// grid (units).  If `flush`, quantize the R window tokens into store
+// positions n_q..n_q+R-1 first; then write the new token into window `slot`.
+template <int D, int BITS, typename T>
+__global__ void __launch_bounds__(D) append_kernel(CacheView c, const T* __restrict__ k,
+                                                   const T* __restrict__ v, long long n_q,
+                                                   int slot, int flush) {
+  __shared__ uint8_t ck[kTile * D];
+  __shared__ uint8_t cv[kTile * D];
+  const long long unit = blockIdx.x;
+  T* kr = reinterpret_cast<T*>(c.k_res) + unit * c.R * D;
+  T* vr = reinterpret_cast<T*>(c.v_res) + unit * c.R * D;
+  if (flush) {
+    for (int tile = 0; tile < c.R / kTile; ++tile)
+      quantize_tile<D, BITS, T>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
+                                n_q + tile * kTile, ck, cv);
+  }
+  kr[(long long)slot * D + threadIdx.x] = k[unit * D + threadIdx.x];
+  vr[(long long)slot * D + threadIdx.x] = v[unit * D + threadIdx.x];
+}
+
+template <int D, int BITS, typename T>
+cudaError_t prefill_t(const CacheView& c, int units, const void* K, const void* V,
+                      long long T_len, long long n_q, int r, cudaStream_t s) {
+  dim3 grid((unsigned)(n_q / kTile + 1), (unsigned)units);
+  prefill_kernel<D, BITS, T><<<grid, D, 0, s>>>(c, (const T*)K, (const T*)V, T_len, n_q, r);
+  return cudaGetLastError();
+}
+
+template <int D, int BITS, typename T>
+cudaError_t append_t(const CacheView& c, int units, const void* k, const void* v, long long n_q,
+                     int slot, bool flush, cudaStream_t s) {
+  append_kernel<D, BITS, T><<<units, D, 0, s>>>(c, (const T*)k, (const T*)v, n_q, slot,
+                                                flush ? 1 : 0);
+  return cudaGetLastError();
+}
+
+template <int BITS, typename T>
+cudaError_t prefill_d(int D, const CacheView& c, int units, const void* K, const void* V,
+                      long long T_len, long long n_q, int r, cudaStream_t s) {
+  switch (D) {
+    case 32: return prefill_t<32, BITS, T>(c, units, K, V, T_len, n_q, r, s);
+    case 64: return prefill_t<64, BITS, T>(c, units, K, V, T_len, n_q, r, s);
+    case 128: return prefill_t<128, BITS, T>(c, units, K, V, T_len, n_q, r, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int BITS, typename T>
+cudaError_t append_d(int D, const CacheView& c, int units, const void* k, const void* v,
+                     long long n_q, int slot, bool flush, cudaStream_t s) {
+  switch (D) {
+    case 32: return append_t<32, BITS, T>(c, units, k, v, n_q, slot, flush, s);
+    case 64: return append_t<64, BITS, T>(c, units, k, v, n_q, slot, flush, s);
+    case 128: return append_t<128, BITS, T>(c, units, k, v, n_q, slot, flush, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const CacheView& c, int units, int D, int bits, int dtype,
+                           const void* K, const void* V, long long T, long long n_q, int r,
+                           cudaStream_t s) {
+  if (bits == 2 && dtype == 0) return prefill_d<2, __half>(D, c, units, K, V, T, n_q, r, s);
+  if (bits == 2 && dtype == 1) return prefill_d<2, float>(D, c, units, K, V, T, n_q, r, s);
+  if (bits == 4 && dtype == 0) return prefill_d<4, __half>(D, c, units, K, V, T, n_q, r, s);
+  if (bits == 4 && dtype == 1) return prefill_d<4, float>(D, c, units, K, V, T, n_q, r, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_append(const CacheView& c, int units, int D, int bits, int dtype,
+                          const void* k, const void* v, long long n_q, int slot, bool flush,
+                          cudaStream_t s) {
+  if (bits == 2 && dtype == 0) return append_d<2, __half>(D, c, units, k, v, n_q, slot, flush, s);
+  if (bits == 2 && dtype == 1) return append_d<2, float>(D, c, units, k, v, n_q, slot, flush, s);
+  if (bits == 4 && dtype == 0) return append_d<4, __half>(D, c, units, k, v, n_q, slot, flush, s);
+  if (bits == 4 && dtype == 1) return append_d<4, float>(D, c, units, k, v, n_q, slot, flush, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kivi

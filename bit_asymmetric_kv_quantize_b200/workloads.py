@@ -11,10 +11,8 @@ shaped attention layers; no datasets or weights are used):
     magnitudes), the same channels for every batch element and token;
   V ~ N(0, 1) (no outlier pattern in values);
   q ~ N(0, 1) / sqrt(D).
-Every (batch element, KV head) unit is drawn from its own torch CPU
-generator, so any unit of a full-size workload can be regenerated alone, bit
-for bit, for sampled oracle checks.  Values are drawn in float32 and cast to
-the workload dtype with round-to-nearest-even.
+Values are drawn in float32 from a seeded torch generator on the target
+device and cast to the workload dtype with round-to-nearest-even.
 """
 from __future__ import annotations
 
@@ -93,47 +91,58 @@ ALL = {w.name: w for w in (TINY, LLAMA2_7B, MISTRAL_7B, STREAMING, LLAMA2_13B_2B
 
 
 def outlier_channels(w: Workload, h: int) -> torch.Tensor:
+    """The fixed outlier key channels of KV head h (same for every sequence and token)."""
     if w.outlier_channels is not None:
         return torch.tensor(w.outlier_channels, dtype=torch.long)
     return torch.randperm(w.D, generator=_gen(_seed(w.seed, "outlier", h)))[: w.n_outliers]
 
 
-def unit_kv(w: Workload, b: int, h: int, T: Optional[int] = None):
-    """Prompt keys and values of one unit: (K [T][D], V [T][D]) in the workload dtype."""
-    T = w.T if T is None else T
-    g = _gen(_seed(w.seed, "kv", b, h))
-    K = torch.randn(T, w.D, generator=g, dtype=torch.float32)
-    V = torch.randn(T, w.D, generator=g, dtype=torch.float32)
-    K[:, outlier_channels(w, h)] *= w.outlier_scale
-    return K.to(w.torch_dtype), V.to(w.torch_dtype)
+def key_channel_scale(w: Workload) -> torch.Tensor:
+    """[Hkv][D] multiplier: outlier_scale on each head's outlier channels, else 1."""
+    m = torch.ones(w.Hkv, w.D, dtype=torch.float32)
+    for h in range(w.Hkv):
+        m[h, outlier_channels(w, h)] = w.outlier_scale
+    return m
+
+
+def _device_gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
 
 
 def prompt_kv(w: Workload, T: Optional[int] = None, device="cpu"):
-    """Whole prompt: (K, V) [B][Hkv][T][D] in the workload dtype, unit by unit."""
+    """Prompt keys and values [B][Hkv][T][D] in the workload dtype.
+
+    Drawn in float32 one sequence at a time from one generator on `device`
+    (CPU: torch's CPU generator; CUDA: torch's Philox generator), so the
+    values depend on the device; the oracle is always given the very tensor
+    the library was given, copied to the host."""
     T = w.T if T is None else T
+    device = torch.device(device)
+    g = _device_gen(device, _seed(w.seed, "kv"))
+    mult = key_channel_scale(w).to(device)[:, None, :]
     K = torch.empty(w.B, w.Hkv, T, w.D, dtype=w.torch_dtype, device=device)
     V = torch.empty_like(K)
     for b in range(w.B):
-        for h in range(w.Hkv):
-            k, v = unit_kv(w, b, h, T)
-            K[b, h].copy_(k)
-            V[b, h].copy_(v)
+        k = torch.randn(w.Hkv, T, w.D, generator=g, dtype=torch.float32, device=device)
+        K[b].copy_(k * mult)
+        V[b].copy_(torch.randn(w.Hkv, T, w.D, generator=g, dtype=torch.float32, device=device))
     return K, V
 
 
-def query(w: Workload, step: int = -1) -> torch.Tensor:
-    """q [B][Hq][D] for the decode after the prompt (step -1) or after decode step `step`."""
+def query(w: Workload, step: int = -1, device="cpu") -> torch.Tensor:
+    """q [B][Hq][D] for the decode after the prompt (step -1) or at decode step `step`."""
     tag, idx = ("q", ()) if step < 0 else ("step_q", (step,))
-    g = _gen(_seed(w.seed, tag, *idx))
-    q = torch.randn(w.B, w.Hq, w.D, generator=g, dtype=torch.float32) / math.sqrt(w.D)
-    return q.to(w.torch_dtype)
+    g = _device_gen(device, _seed(w.seed, tag, *idx))
+    q = torch.randn(w.B, w.Hq, w.D, generator=g, dtype=torch.float32, device=device)
+    return (q / math.sqrt(w.D)).to(w.torch_dtype)
 
 
-def step_kv(w: Workload, step: int):
+def step_kv(w: Workload, step: int, device="cpu"):
     """The token appended at decode step `step`: (k, v) [B][Hkv][D]."""
-    g = _gen(_seed(w.seed, "step_kv", step))
-    k = torch.randn(w.B, w.Hkv, w.D, generator=g, dtype=torch.float32)
-    v = torch.randn(w.B, w.Hkv, w.D, generator=g, dtype=torch.float32)
-    for h in range(w.Hkv):
-        k[:, h, outlier_channels(w, h)] *= w.outlier_scale
+    g = _device_gen(device, _seed(w.seed, "step_kv", step))
+    k = torch.randn(w.B, w.Hkv, w.D, generator=g, dtype=torch.float32, device=device)
+    v = torch.randn(w.B, w.Hkv, w.D, generator=g, dtype=torch.float32, device=device)
+    k = k * key_channel_scale(w).to(device)[None]
     return k.to(w.torch_dtype), v.to(w.torch_dtype)

@@ -1,0 +1,223 @@
+/*
+ * kivi.h -- C ABI of libkivi.so: a KIVI-style asymmetric 2/4-bit KV cache
+ * with a full-precision residual window and fused decode attention, for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache".
+ *   - mlsanity.com index page, section "Abstract (arXiv)": keys are
+ *     quantized per channel, values per token, to 2 bits; loading the KV
+ *     cache, not arithmetic, limits decode speed.
+ *   - study.space summary page (one summary paragraph): the quantizer is
+ *     asymmetric; key groups span tokens; value codes are appended along the
+ *     token axis; each cache is split into a quantized ("grouped") part and
+ *     a full-precision residual part, and decode attention over the
+ *     quantized part is combined with the residual part.
+ *   - scholarfeed.org "KIVI" page, third quote: the residual is a
+ *     fixed-length buffer of the most recent tokens, kept unquantized
+ *     (a mixed-precision cache).
+ *   - same page, first quote: a 4-bit variant of KIVI exists.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer named "device" is CUDA device memory on the current
+ *     device; the library never allocates, frees or copies host memory on
+ *     the caller's behalf, never allocates device memory and never
+ *     synchronizes.  All work is enqueued on `stream` (a cudaStream_t passed
+ *     as void*; NULL is the legacy default stream) and is asynchronous.
+ *   - Every call returns a kivi_status.  Argument, shape, state and capacity
+ *     errors are detected on the host before anything is enqueued and leave
+ *     the cache state unchanged.  KIVI_ERR_CUDA reports a launch error
+ *     (cudaGetLastError after the launch); the host counters are then not
+ *     advanced.  Nothing throws across this boundary.
+ *   - A kivi_cache is not thread safe: calls on one cache must be
+ *     serialized by the caller (they update its host-side counters).
+ *
+ * Cache layout (part of the ABI; all arrays dense, row-major).  With
+ * E = 32/bits codes per 32-bit word, Tq = capacity - R quantized tokens per
+ * sequence, NG = Tq/G key groups and NJ = D/Gv value groups per token:
+ *   k_codes  uint32 [B][Hkv][Tq][D/E]   word w of token t packs channels
+ *                                        wE..wE+E-1; channel wE+i in bits
+ *                                        [bits*i, bits*i+bits)
+ *   k_scale  float  [B][Hkv][NG][D]     one scale and zero per key group
+ *   k_zero   float  [B][Hkv][NG][D]     (G consecutive tokens) and channel
+ *   v_codes  uint32 [B][Hkv][Tq/E][D]   word (tb, d) packs tokens
+ *                                        tb*E..tb*E+E-1 of channel d;
+ *                                        token tb*E+i in bits
+ *                                        [bits*i, bits*i+bits)
+ *   v_scale  float  [B][Hkv][Tq][NJ]    one scale and zero per token and
+ *   v_zero   float  [B][Hkv][Tq][NJ]    value group (Gv consecutive channels)
+ *   k_res    dtype  [B][Hkv][R][D]      residual window, input precision;
+ *   v_res    dtype  [B][Hkv][R][D]      slots 0..r-1 hold the newest tokens
+ * Each code packs along the axis its attention product contracts over
+ * (channels for keys, tokens for values).
+ *
+ * Quantizer (fixed binary32 formula; codes, scales and zeros are bit-exact
+ * functions of the inputs): for a group x_0..x_{n-1},
+ *   mn = min x_i, mx = max x_i (first occurrence kept among equal values),
+ *   s = (mx - mn) / (2^bits - 1), z = mn  (each op rounded to nearest),
+ *   c_i = clamp(round_half_even((x_i - mn) / s), 0, 2^bits - 1), or 0 if s == 0.
+ * Dequantized value: c * s + z.
+ *
+ * Residual window ("flush before write"): a non-empty cache holds
+ * r in [1, R] residual tokens.  Prefill of T tokens leaves
+ * r = ((T-1) mod R) + 1 and quantizes the first n_q = T - r; appending to a
+ * full window first quantizes its R tokens into positions n_q..n_q+R-1.
+ * prefill(T) and T single appends therefore produce identical bytes.
+ */
+#ifndef KIVI_H
+#define KIVI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KIVI_API __attribute__((visibility("default")))
+#else
+#define KIVI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KIVI_OK = 0,
+  KIVI_ERR_ARG = 1,         /* null pointer, negative size, Hq not a multiple of Hkv */
+  KIVI_ERR_UNSUPPORTED = 2, /* bits, G, Gv, D, R or dtype outside the built kernels */
+  KIVI_ERR_STATE = 3,       /* prefill on a non-empty cache; decode on an empty one */
+  KIVI_ERR_CAPACITY = 4,    /* the tokens would not fit in `capacity` */
+  KIVI_ERR_WORKSPACE = 5,   /* workspace missing, too small or misaligned */
+  KIVI_ERR_CUDA = 6         /* a CUDA launch or device query failed */
+} kivi_status;
+
+typedef enum { KIVI_F16 = 0, KIVI_F32 = 1 } kivi_dtype;
+
+/* Shape of one cache (one attention layer).  Supported: bits in {2, 4},
+ * G = 32, Gv = 32, D in {32, 64, 128}, R a positive multiple of 32,
+ * capacity a positive multiple of R, dtype KIVI_F16 or KIVI_F32. */
+typedef struct {
+  int B;              /* sequences (batch) */
+  int Hkv;            /* key/value heads */
+  int D;              /* head dimension (channels) */
+  int bits;           /* code width */
+  int G;              /* key group: tokens sharing one scale/zero per channel */
+  int Gv;             /* value group: channels sharing one scale/zero per token */
+  int R;              /* residual window length in tokens */
+  long long capacity; /* max tokens per sequence, quantized + residual */
+  int dtype;          /* kivi_dtype of K, V, q, out and the residual window */
+} kivi_dims;
+
+enum {
+  KIVI_BUF_K_CODES = 0,
+  KIVI_BUF_K_SCALE = 1,
+  KIVI_BUF_K_ZERO = 2,
+  KIVI_BUF_V_CODES = 3,
+  KIVI_BUF_V_SCALE = 4,
+  KIVI_BUF_V_ZERO = 5,
+  KIVI_BUF_K_RES = 6,
+  KIVI_BUF_V_RES = 7,
+  KIVI_NUM_BUFFERS = 8
+};
+
+/* A cache: the caller's device buffers (layout above) plus host counters
+ * that the library owns and advances.  n_q and r are the same for every
+ * sequence of the batch. */
+typedef struct {
+  kivi_dims dims;
+  uint32_t *k_codes;
+  float *k_scale;
+  float *k_zero;
+  uint32_t *v_codes;
+  float *v_scale;
+  float *v_zero;
+  void *k_res;
+  void *v_res;
+  long long n_q; /* tokens per sequence in the quantized store */
+  int r;         /* tokens per sequence in the residual window */
+} kivi_cache;
+
+/* Byte size of each of the KIVI_NUM_BUFFERS buffers for `dims`, written to
+ * out_bytes[KIVI_BUF_*].  Pure host arithmetic.
+ * Errors: KIVI_ERR_ARG (null), KIVI_ERR_UNSUPPORTED (dims not supported). */
+KIVI_API int kivi_buffer_sizes(const kivi_dims *dims, size_t out_bytes[KIVI_NUM_BUFFERS]);
+
+/* Bind `buffers[KIVI_BUF_*]` (device pointers, each 16-byte aligned and at
+ * least kivi_buffer_sizes() bytes; the caller keeps ownership) to `cache`
+ * and set n_q = r = 0.  No device work; buffer contents are not read until
+ * written by prefill/append.
+ * Errors: KIVI_ERR_ARG (null or misaligned pointer), KIVI_ERR_UNSUPPORTED. */
+KIVI_API int kivi_cache_init(kivi_cache *cache, const kivi_dims *dims,
+                    void *const buffers[KIVI_NUM_BUFFERS]);
+
+/* Prefill: quantize a prompt of T tokens into an empty cache.
+ * K, V: device, dims.dtype, [B][Hkv][T][D] contiguous.  Tokens 0..n_q-1
+ * (n_q = T - r, r = ((T-1) mod R) + 1) are quantized: keys per (key group,
+ * channel) over G tokens, values per (token, value group) over Gv channels;
+ * tokens n_q..T-1 are copied unmodified into the residual window.
+ * (KIVI, study.space summary: grouped parts quantized, residual parts kept
+ * in full precision; mlsanity.com abstract: per-channel keys, per-token
+ * values.)
+ * Errors: KIVI_ERR_ARG, KIVI_ERR_STATE (cache not empty),
+ * KIVI_ERR_CAPACITY (T > capacity), KIVI_ERR_CUDA. */
+KIVI_API int kivi_quantize_prefill(kivi_cache *cache, const void *K, const void *V,
+                          long long T, void *stream);
+
+/* Append one token per sequence.  k, v: device, dims.dtype, [B][Hkv][D].
+ * If the window is full (r == R) its R tokens are first quantized into the
+ * store (R/G key groups, R value tokens) and the window emptied (one kernel
+ * launch either way).  (KIVI, study.space summary: new codes appended along
+ * the token axis, key groups formed across tokens; scholarfeed.org "KIVI"
+ * page: fixed-length residual buffer.)
+ * Errors: KIVI_ERR_ARG, KIVI_ERR_CAPACITY (n_q + r + 1 > capacity),
+ * KIVI_ERR_CUDA. */
+KIVI_API int kivi_append_token(kivi_cache *cache, const void *k, const void *v,
+                      void *stream);
+
+/* Bytes of device workspace kivi_decode_attention needs for Hq query heads
+ * at any fill level of this cache (0 on error).  Host arithmetic only. */
+KIVI_API size_t kivi_decode_workspace_bytes(const kivi_cache *cache, int Hq);
+
+/* Decode attention for one new query per sequence and head, computed
+ * directly over the packed codes plus the residual window, with one softmax
+ * over all n_q + r tokens:
+ *   out[b][h] = sum_t p_t * Vhat_t / sum_t p_t,
+ *   p_t = exp(softmax_scale * <q[b][h], Khat_t> - max),
+ * where Khat/Vhat are the dequantized codes for t < n_q and the stored
+ * window tokens after that.  Query head h reads KV head h / (Hq/Hkv).
+ * q, out: device, dims.dtype, [B][Hq][D] contiguous.  workspace: device,
+ * 16-byte aligned, at least kivi_decode_workspace_bytes(cache, Hq) bytes,
+ * scratch that is fully written before it is read.
+ * (KIVI, study.space summary: attention over the quantized part, then
+ * combined with the residual part; mlsanity.com abstract: cache loading
+ * bounds decode.)
+ * Errors: KIVI_ERR_ARG (null, Hq % Hkv != 0, Hq/Hkv > 8), KIVI_ERR_STATE
+ * (empty cache), KIVI_ERR_WORKSPACE, KIVI_ERR_CUDA. */
+KIVI_API int kivi_decode_attention(const kivi_cache *cache, const void *q, int Hq,
+                          float softmax_scale, void *out, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/* Same result as kivi_decode_attention (same arguments, same workspace
+ * rule) computed by the plain CUDA-core (SIMT) kernel instead of the
+ * tensor-core kernel; kept as the measured alternative. */
+KIVI_API int kivi_decode_attention_simt(const kivi_cache *cache, const void *q,
+                               int Hq, float softmax_scale, void *out,
+                               void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/* Optional timing hook: if start/stop are non-NULL cudaEvent_t handles,
+ * later decode calls on this thread record `start` just before and `stop`
+ * just after the launch of the dominant (split) decode kernel, on the
+ * call's stream.  Pass NULL, NULL to turn it off. */
+KIVI_API void kivi_set_timing_events(void *start_event, void *stop_event);
+
+/* Number of context splits the decode kernel would use for this cache's
+ * current fill level and Hq (>= 1), or 0 on error. */
+KIVI_API int kivi_decode_num_splits(const kivi_cache *cache, int Hq);
+
+/* Human-readable name of a kivi_status. */
+KIVI_API const char *kivi_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KIVI_H */

@@ -1,0 +1,150 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol that
+include/kivi.h declares, and rejects bad arguments on the host before any
+CUDA call.  (No compute call runs here.)"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import bit_asymmetric_kv_quantize_b200 as kivi
+from bit_asymmetric_kv_quantize_b200 import KiviCacheC, KiviDims
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kivi.h")
+
+ERR_ARG, ERR_UNSUPPORTED, ERR_STATE, ERR_CAPACITY = 1, 2, 3, 4
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"KIVI_API\s+[\w\s\*]*?\b(kivi_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    L = kivi.lib()
+    for s in syms:
+        assert hasattr(L, s), s
+    assert set(syms) == set(kivi.EXPORTED)
+
+
+def _dims(**kw):
+    d = dict(B=2, Hkv=4, D=128, bits=2, G=32, Gv=32, R=128, capacity=4096, dtype=kivi.KIVI_F16)
+    d.update(kw)
+    return KiviDims(d["B"], d["Hkv"], d["D"], d["bits"], d["G"], d["Gv"], d["R"], d["capacity"],
+                    d["dtype"])
+
+
+def _sizes(dims):
+    out = (ctypes.c_size_t * 8)()
+    rc = kivi.lib().kivi_buffer_sizes(ctypes.byref(dims), ctypes.byref(out))
+    return rc, list(out)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("D", [32, 64, 128])
+def test_buffer_sizes_follow_the_layout(bits, D):
+    B, H, R, cap = 3, 5, 64, 640
+    rc, s = _sizes(_dims(B=B, Hkv=H, D=D, bits=bits, R=R, capacity=cap))
+    assert rc == 0
+    E, Tq, u = 32 // bits, cap - R, B * H
+    assert s[0] == u * Tq * (D // E) * 4           # k_codes
+    assert s[1] == s[2] == u * (Tq // 32) * D * 4  # k_scale, k_zero
+    assert s[3] == u * (Tq // E) * D * 4           # v_codes
+    assert s[4] == s[5] == u * Tq * (D // 32) * 4  # v_scale, v_zero
+    assert s[6] == s[7] == u * R * D * 2           # k_res, v_res (fp16)
+    # 2-bit codes + fp32 scale/zero per 32: 0.5 byte per key and per value element
+    if bits == 2:
+        assert sum(s[:6]) == u * Tq * D * 2 * 0.5
+
+
+@pytest.mark.parametrize("kw,rc", [
+    (dict(bits=3), ERR_UNSUPPORTED), (dict(bits=8), ERR_UNSUPPORTED),
+    (dict(G=16), ERR_UNSUPPORTED), (dict(Gv=64), ERR_UNSUPPORTED),
+    (dict(D=96), ERR_UNSUPPORTED), (dict(R=48), ERR_UNSUPPORTED),
+    (dict(capacity=4100), ERR_UNSUPPORTED), (dict(dtype=7), ERR_UNSUPPORTED),
+    (dict(B=0), ERR_ARG), (dict(Hkv=-1), ERR_ARG), (dict(capacity=0), ERR_ARG),
+])
+def test_unsupported_dims(kw, rc):
+    assert _sizes(_dims(**kw))[0] == rc
+
+
+def _fake_cache(**kw):
+    """A cache bound to fake (never dereferenced) aligned addresses."""
+    dims = _dims(**kw)
+    c = KiviCacheC()
+    ptrs = (ctypes.c_void_p * 8)(*[0x10000 * (i + 1) for i in range(8)])
+    assert kivi.lib().kivi_cache_init(ctypes.byref(c), ctypes.byref(dims), ctypes.byref(ptrs)) == 0
+    assert (c.n_q, c.r) == (0, 0)
+    return c
+
+
+def test_cache_init_rejects_null_and_misaligned():
+    L = kivi.lib()
+    dims = _dims()
+    c = KiviCacheC()
+    ptrs = (ctypes.c_void_p * 8)(*[0x10000 * (i + 1) for i in range(8)])
+    ptrs[3] = None
+    assert L.kivi_cache_init(ctypes.byref(c), ctypes.byref(dims), ctypes.byref(ptrs)) == ERR_ARG
+    ptrs[3] = 0x30008  # 8-byte aligned only
+    assert L.kivi_cache_init(ctypes.byref(c), ctypes.byref(dims), ctypes.byref(ptrs)) == ERR_ARG
+    assert L.kivi_cache_init(None, ctypes.byref(dims), ctypes.byref(ptrs)) == ERR_ARG
+
+
+def test_window_only_cache_needs_no_store_buffers():
+    dims = _dims(R=128, capacity=128)
+    c = KiviCacheC()
+    ptrs = (ctypes.c_void_p * 8)(None, None, None, None, None, None, 0x1000, 0x2000)
+    assert kivi.lib().kivi_cache_init(ctypes.byref(c), ctypes.byref(dims), ctypes.byref(ptrs)) == 0
+
+
+def test_host_side_state_and_capacity_errors():
+    L = kivi.lib()
+    fake = ctypes.c_void_p(0x5000)
+    c = _fake_cache(R=128, capacity=256)
+    assert L.kivi_quantize_prefill(ctypes.byref(c), fake, fake, -1, None) == ERR_ARG
+    assert L.kivi_quantize_prefill(ctypes.byref(c), None, fake, 5, None) == ERR_ARG
+    assert L.kivi_quantize_prefill(ctypes.byref(c), fake, fake, 257, None) == ERR_CAPACITY
+    assert L.kivi_quantize_prefill(ctypes.byref(c), fake, fake, 0, None) == 0  # no-op
+    assert (c.n_q, c.r) == (0, 0)
+    # decode on an empty cache, and with a query head count that is not a multiple of Hkv
+    assert L.kivi_decode_attention(ctypes.byref(c), fake, 4, 1.0, fake, fake, 1 << 20, None) == ERR_STATE
+    assert L.kivi_decode_attention(ctypes.byref(c), fake, 6, 1.0, fake, fake, 1 << 20, None) == ERR_ARG
+    assert L.kivi_decode_attention(ctypes.byref(c), fake, 12, 1.0, fake, fake, 1 << 20, None) == ERR_UNSUPPORTED
+    # pretend a full cache: prefill refused (not empty), append refused (no room)
+    c.n_q, c.r = 128, 128
+    assert L.kivi_quantize_prefill(ctypes.byref(c), fake, fake, 1, None) == ERR_STATE
+    assert L.kivi_append_token(ctypes.byref(c), fake, fake, None) == ERR_CAPACITY
+    assert L.kivi_append_token(ctypes.byref(c), None, fake, None) == ERR_ARG
+    assert (c.n_q, c.r) == (128, 128)  # unchanged by refused calls
+
+
+def test_status_strings():
+    L = kivi.lib()
+    for code, name in kivi.STATUS.items():
+        assert L.kivi_status_string(code).decode().startswith(name)
+    assert b"unknown" in L.kivi_status_string(99)
+
+
+def test_product_path_refuses_cpu_tensors():
+    with pytest.raises((ValueError, RuntimeError)):
+        kivi.KiviCache(1, 1, 32, 2, 64, R=32, dtype=torch.float32, device="cpu")
+
+
+def test_oracle_and_library_share_no_source():
+    """The oracle and the CUDA path are independent: no file includes or imports the other."""
+    csrc = os.path.join(ROOT, "bit_asymmetric_kv_quantize_b200", "csrc")
+    for f in os.listdir(csrc):
+        text = open(os.path.join(csrc, f)).read()
+        assert not re.search(r'#\s*include\s*[<"][^>"]*oracle', text), f
+    for f in ("kivi_oracle.c", "kivi_oracle.h", "__init__.py"):
+        text = open(os.path.join(ROOT, "oracle", f)).read()
+        assert not re.search(r'#\s*include\s*[<"]kivi\.h', text), f
+        assert not re.search(r"(import|from)\s+bit_asymmetric_kv_quantize_b200", text), f
+    pkg = os.path.join(ROOT, "bit_asymmetric_kv_quantize_b200")
+    for f in os.listdir(pkg):
+        if f.endswith(".py"):
+            assert "import oracle" not in open(os.path.join(pkg, f)).read(), f

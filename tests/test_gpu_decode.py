@@ -1,0 +1,167 @@
+"""GPU parity of decode attention against the oracle, through the C ABI.
+
+Bar: max |gpu - oracle| <= 2e-3 and mean <= 1e-3 (kivi_testlib), the oracle
+in binary64 over the dequantized cache.  Both the tensor-core kernel
+(kivi_decode_attention) and the CUDA-core kernel (kivi_decode_attention_simt)
+are checked.
+
+Method: "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache",
+study.space summary: decode attention over the quantized part, combined with
+the full-precision residual part (one softmax over both here).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import bit_asymmetric_kv_quantize_b200 as kivi
+from bit_asymmetric_kv_quantize_b200 import workloads as W
+from kivi_testlib import (assert_decode_close, assert_state_equal, decode_error, gpu_cache,
+                          oracle_append, oracle_cache, oracle_prefill, sample_units)
+
+pytestmark = pytest.mark.gpu
+KERNELS = ["default", "simt"]
+
+
+def small(D=64, bits=2, dtype="f16", R=32, T=200, B=2, Hkv=2, gq=1, seed=3):
+    return W.Workload(f"dec-d{D}-b{bits}-{dtype}-g{gq}-t{T}", B=B, Hq=Hkv * gq, Hkv=Hkv, D=D,
+                      T=T, bits=bits, R=R, dtype=dtype, seed=seed)
+
+
+def run(w, kernel, sigma=None, capacity=None):
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w, capacity=capacity)
+    gc.prefill(K, V)
+    oc = oracle_cache(w, capacity=capacity)
+    oracle_prefill(oc, K, V)
+    q = W.query(w, device="cuda")
+    sigma = 1.0 / math.sqrt(w.D) if sigma is None else sigma
+    out = gc.decode(q, sigma, kernel=kernel)
+    return gc, oc, q, out, sigma
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("gq", [1, 2, 4, 8])
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("D", [32, 64, 128])
+def test_decode_shapes(D, bits, dtype, gq, kernel):
+    for T in (1, 33, 161, 1000):
+        w = small(D=D, bits=bits, dtype=dtype, gq=gq, T=T)
+        gc, oc, q, out, sigma = run(w, kernel, capacity=1024)
+        assert_decode_close(out, oc, q, sigma)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("sigma", [1.0, 0.3, 2.0])
+def test_decode_softmax_scale(sigma, kernel):
+    w = small(D=128, gq=4, T=700)
+    gc, oc, q, out, sigma = run(w, kernel, sigma=sigma, capacity=1024)
+    assert_decode_close(out, oc, q, sigma)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("T", [64 * 32 + 1, 5000, 9000])
+def test_decode_many_splits(T, kernel):
+    """One unit, long context: the context is split over many CTAs and merged."""
+    w = small(D=128, B=1, Hkv=1, gq=4, T=T, R=128)
+    gc, oc, q, out, sigma = run(w, kernel, capacity=9216)
+    assert gc.num_splits(w.Hq) > 8
+    assert_decode_close(out, oc, q, sigma)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_decode_constant_values_and_zero_query(kernel):
+    w = small(D=64, gq=2, T=300)
+    K, V = W.prompt_kv(w, device="cuda")
+    V.fill_(0.625)
+    gc = gpu_cache(w, capacity=512)
+    gc.prefill(K, V)
+    q = W.query(w, device="cuda")
+    out = gc.decode(q, 0.125, kernel=kernel)
+    assert torch.allclose(out.float(), torch.full_like(out.float(), 0.625), atol=1e-3)
+    # q = 0: uniform weights -> the mean of the dequantized values (oracle)
+    K2, V2 = W.prompt_kv(w, device="cuda")
+    gc2 = gpu_cache(w, capacity=512)
+    gc2.prefill(K2, V2)
+    oc2 = oracle_cache(w, capacity=512)
+    oracle_prefill(oc2, K2, V2)
+    qz = torch.zeros_like(q)
+    assert_decode_close(gc2.decode(qz, 1.0, kernel=kernel), oc2, qz, 1.0)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_decode_tiny_workload(kernel):
+    w = W.TINY
+    gc, oc, q, out, _ = run(w, kernel, sigma=1.0)
+    assert (gc.n_q, gc.r) == (224, 32)
+    assert_decode_close(out, oc, q, 1.0)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("w", [W.LLAMA2_7B, W.MISTRAL_7B], ids=lambda w: w.name)
+def test_decode_layer_workloads_full(w, kernel):
+    """Every head of the full-size layer against the oracle (q carries 1/sqrt(D): sigma = 1)."""
+    gc, oc, q, out, _ = run(w, kernel, sigma=1.0)
+    assert_decode_close(out, oc, q, 1.0)
+
+
+@pytest.mark.parametrize("w", [W.LLAMA2_13B_2BIT, W.LLAMA2_13B_4BIT], ids=lambda w: w.name)
+def test_decode_large_batch_sampled(w):
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w)
+    gc.prefill(K, V)
+    units = sample_units(w, 16)
+    oc = oracle_cache(w, units=units)
+    oracle_prefill(oc, K, V)
+    q = W.query(w, device="cuda")
+    for kernel in KERNELS:
+        assert_decode_close(gc.decode(q, 1.0, kernel=kernel), oc, q, 1.0, units=units)
+
+
+def test_streaming_workload_every_step():
+    """Prompt of 32768 tokens, then 512 steps of append + decode (window flush
+    every 128 steps).  Two sampled units are checked at every step; the
+    quantized store of the sampled units is compared bit for bit after every
+    flush."""
+    w = W.STREAMING
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w)
+    gc.prefill(K, V)
+    units = sample_units(w, 2, seed=5)
+    oc = oracle_cache(w, units=units)
+    oracle_prefill(oc, K, V)
+    del K, V
+    assert_state_equal(gc, oc)
+    worst = 0.0
+    for step in range(w.steps):
+        k, v = W.step_kv(w, step, device="cuda")
+        gc.append(k, v)
+        oracle_append(oc, k, v)
+        q = W.query(w, step, device="cuda")
+        out = gc.decode(q, 1.0)
+        mx, _ = assert_decode_close(out, oc, q, 1.0, units=units)
+        worst = max(worst, mx)
+        if gc.r == 1:
+            assert_state_equal(gc, oc)
+    assert gc.n_q + gc.r == w.T + w.steps
+    print(f"streaming worst max-abs {worst:.3e}")
+
+
+def test_decode_errors_on_device():
+    w = small(D=64, T=100)
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w, capacity=512)
+    gc.prefill(K, V)
+    q = W.query(w, device="cuda")
+    out = torch.empty_like(q)
+    L = kivi.lib()
+    import ctypes
+    ws = gc.workspace(w.Hq)
+    rc = L.kivi_decode_attention(ctypes.byref(gc._c), q.data_ptr(), w.Hq, 1.0, out.data_ptr(),
+                                 ws.data_ptr(), 16, None)
+    assert rc == 5  # workspace too small
+    rc = L.kivi_decode_attention(ctypes.byref(gc._c), q.data_ptr(), w.Hq, 1.0, out.data_ptr(),
+                                 ws.data_ptr() + 4, ws.numel() - 4, None)
+    assert rc == 5  # misaligned

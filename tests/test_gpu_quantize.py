@@ -1,0 +1,141 @@
+"""GPU parity of the prefill / append / flush path against the oracle: the
+quantized store (codes, scales, zeros) and the residual window are compared
+bit for bit, through the C ABI (libkivi.so via the ctypes binding).
+
+Method: "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache"
+(mlsanity.com index page, "Abstract (arXiv)": per-channel keys, per-token
+values; study.space summary: asymmetric groups, quantized and residual
+parts, codes appended along tokens).
+"""
+import numpy as np
+import pytest
+import torch
+
+import bit_asymmetric_kv_quantize_b200 as kivi
+from bit_asymmetric_kv_quantize_b200 import workloads as W
+from kivi_testlib import (assert_state_equal, gpu_cache, oracle_append, oracle_cache,
+                          oracle_prefill, sample_units)
+
+pytestmark = pytest.mark.gpu
+
+
+def small(D=64, bits=2, dtype="f16", R=64, T=200, B=2, Hkv=3, gq=1, capacity=512, seed=1):
+    return W.Workload(f"small-d{D}-b{bits}-{dtype}-r{R}-t{T}", B=B, Hq=Hkv * gq, Hkv=Hkv, D=D,
+                      T=T, bits=bits, R=R, dtype=dtype, seed=seed).with_()
+
+
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("T", [1, 31, 64, 65, 127, 128, 129, 333])
+def test_prefill_bit_exact(D, bits, dtype, T):
+    w = small(D=D, bits=bits, dtype=dtype, T=T)
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w, capacity=512)
+    gc.prefill(K, V)
+    oc = oracle_cache(w, capacity=512)
+    oracle_prefill(oc, K, V)
+    assert (gc.n_q, gc.r) == (T - ((T - 1) % 64 + 1), (T - 1) % 64 + 1)
+    assert_state_equal(gc, oc)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("R", [32, 128])
+def test_append_and_flush_bit_exact(bits, R):
+    """Prefill, then appends across several window flushes; the state matches
+    the oracle after every append."""
+    w = small(D=128, bits=bits, R=R, T=R + 5, B=2, Hkv=2)
+    K, V = W.prompt_kv(w, device="cuda")
+    cap = R * 8
+    gc = gpu_cache(w, capacity=cap)
+    oc = oracle_cache(w, capacity=cap)
+    gc.prefill(K, V)
+    oracle_prefill(oc, K, V)
+    assert_state_equal(gc, oc)
+    for step in range(3 * R):
+        k, v = W.step_kv(w, step, device="cuda")
+        gc.append(k, v)
+        oracle_append(oc, k, v)
+        if gc.r in (1, R) or step % 17 == 0:
+            assert_state_equal(gc, oc)
+    assert_state_equal(gc, oc)
+    assert gc.n_q + gc.r == R + 5 + 3 * R
+
+
+@pytest.mark.parametrize("T", [0, 1, 32, 63, 64, 65, 129, 300])
+def test_prefill_equals_appends(T):
+    """prefill(T) and T single appends write identical bytes."""
+    w = small(D=64, bits=2, R=64, T=T, dtype="f16")
+    K, V = W.prompt_kv(w, device="cuda")
+    a, b = gpu_cache(w, capacity=512), gpu_cache(w, capacity=512)
+    a.prefill(K, V)
+    for t in range(T):
+        b.append(K[:, :, t].contiguous(), V[:, :, t].contiguous())
+    assert (a.n_q, a.r) == (b.n_q, b.r)
+    n_q, r = a.n_q, a.r
+    lim = {"k_codes": n_q, "k_scale": n_q // 32, "k_zero": n_q // 32, "v_codes": n_q // 16,
+           "v_scale": n_q, "v_zero": n_q, "k_res": r, "v_res": r}
+    for name in kivi.BUFFER_NAMES:
+        assert torch.equal(a.view(name)[:, :, :lim[name]], b.view(name)[:, :, :lim[name]]), name
+
+
+def test_special_values_bit_exact():
+    """Signed zeros (first occurrence decides the zero's sign), constant groups
+    (scale 0), fp16 extremes and subnormals, huge outlier channels."""
+    w = small(D=64, bits=2, R=32, T=32 * 6 + 3, B=1, Hkv=2, dtype="f16")
+    K, V = W.prompt_kv(w, device="cuda")
+    K[0, 0, 0:32, 0] = 0.0                       # constant channel group
+    K[0, 0, 0:32, 1] = -0.0
+    K[0, 0, 0:16, 2] = -0.0                      # -0 first, then +0
+    K[0, 0, 16:32, 2] = 0.0
+    K[0, 0, 32:48, 3] = 0.0                      # +0 first, then -0
+    K[0, 0, 48:64, 3] = -0.0
+    K[0, 1, 64:96, 5] = 65504.0                  # fp16 max, constant
+    K[0, 1, 64:80, 6] = -65504.0                 # full fp16 range in one group
+    K[0, 1, 80:96, 6] = 65504.0
+    K[0, 1, 96:128, 7] = torch.arange(32, device="cuda", dtype=torch.float16) * 6e-8  # subnormals
+    V[0, 0, 3, :32] = -0.0                       # constant value group (-0)
+    V[0, 0, 4, :32] = 1.5
+    V[0, 1, 5, 0:16] = 0.0
+    V[0, 1, 5, 16:32] = -0.0
+    V[0, 1, 6, 32:64] = torch.arange(32, device="cuda", dtype=torch.float16) * 1e3
+    gc = gpu_cache(w, capacity=512)
+    gc.prefill(K, V)
+    oc = oracle_cache(w, capacity=512)
+    oracle_prefill(oc, K, V)
+    assert_state_equal(gc, oc)
+
+
+def test_tiny_workload_full():
+    w = W.TINY
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w)
+    gc.prefill(K, V)
+    oc = oracle_cache(w)
+    oracle_prefill(oc, K, V)
+    assert (gc.n_q, gc.r) == (224, 32)
+    assert_state_equal(gc, oc)
+
+
+@pytest.mark.parametrize("w", [W.LLAMA2_7B, W.MISTRAL_7B], ids=lambda w: w.name)
+def test_layer_workloads_full(w):
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w)
+    gc.prefill(K, V)
+    oc = oracle_cache(w)
+    oracle_prefill(oc, K, V)
+    assert (gc.n_q, gc.r) == (w.T - w.R, w.R)
+    assert_state_equal(gc, oc)
+
+
+@pytest.mark.parametrize("w", [W.LLAMA2_13B_2BIT, W.LLAMA2_13B_4BIT], ids=lambda w: w.name)
+def test_large_batch_workload_sampled(w):
+    """Full-size 13B-shaped layer (64 x 40 units, 8192 tokens): every unit is
+    quantized on the GPU, 24 sampled units are checked against the oracle."""
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w)
+    gc.prefill(K, V)
+    units = sample_units(w, 24)
+    oc = oracle_cache(w, units=units)
+    oracle_prefill(oc, K, V)
+    assert_state_equal(gc, oc)
