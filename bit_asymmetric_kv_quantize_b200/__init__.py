@@ -25,12 +25,14 @@ KIVI_F16, KIVI_F32 = 0, 1
 NUM_BUFFERS = 8
 BUFFER_NAMES = ("k_codes", "k_scale", "k_zero", "v_codes", "v_scale", "v_zero", "k_res", "v_res")
 STATUS = {0: "KIVI_OK", 1: "KIVI_ERR_ARG", 2: "KIVI_ERR_UNSUPPORTED", 3: "KIVI_ERR_STATE",
-          4: "KIVI_ERR_CAPACITY", 5: "KIVI_ERR_WORKSPACE", 6: "KIVI_ERR_CUDA"}
+          4: "KIVI_ERR_CAPACITY", 5: "KIVI_ERR_WORKSPACE", 6: "KIVI_ERR_CUDA",
+          7: "KIVI_ERR_SCRATCH_LIMIT"}
 
 EXPORTED = (
     "kivi_buffer_sizes", "kivi_cache_init", "kivi_quantize_prefill", "kivi_append_token",
     "kivi_decode_workspace_bytes", "kivi_decode_attention", "kivi_decode_attention_simt",
     "kivi_set_timing_events", "kivi_decode_num_splits", "kivi_status_string",
+    "kivi_decode_attention_noalloc",
 )
 
 
@@ -80,6 +82,7 @@ def lib() -> ctypes.CDLL:
             dec = [cp, vp, ci, ctypes.c_float, vp, vp, sz, vp]
             L.kivi_decode_attention.argtypes = dec
             L.kivi_decode_attention_simt.argtypes = dec
+            L.kivi_decode_attention_noalloc.argtypes = [cp, vp, ci, ctypes.c_float, vp, vp]
             L.kivi_set_timing_events.argtypes = [vp, vp]
             L.kivi_set_timing_events.restype = None
             L.kivi_decode_num_splits.argtypes = [cp, ci]

@@ -5,6 +5,8 @@
 #include <limits.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "kivi.h"
 #include "kivi_internal.cuh"
 
@@ -133,6 +135,30 @@ int decode_common(const kivi_cache* c, const void* q, int Hq, float softmax_scal
   return err == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA;
 }
 
+// ---- static scratch for kivi_decode_attention_noalloc ----------------------
+// One fixed array per device, reserved when the library's module is loaded.
+// Host code must not use the symbol itself as a device address: its device
+// address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KIVI_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 128;
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KIVI_ERR_CUDA;
+  void* p = g_noalloc_ptr[dev].load();
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return KIVI_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev].store(p);
+  }
+  *out = p;
+  return KIVI_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -238,6 +264,52 @@ int kivi_decode_attention_simt(const kivi_cache* cache, const void* q, int Hq,
                        true);
 }
 
+int kivi_decode_attention_noalloc(const kivi_cache* cache, const void* q, int Hq,
+                                  float softmax_scale, void* out, void* stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!q || !out || Hq <= 0 || Hq % cache->dims.Hkv != 0) return KIVI_ERR_ARG;
+  const int gq = Hq / cache->dims.Hkv;
+  if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KIVI_ERR_UNSUPPORTED;
+  if (cache->n_q + cache->r == 0) return KIVI_ERR_STATE;
+  const size_t per_split = (size_t)cache->dims.B * Hq * (cache->dims.D + 2) * sizeof(float);
+  if (per_split > KIVI_NOALLOC_SCRATCH_BYTES) return KIVI_ERR_SCRATCH_LIMIT;
+  const int sms = device_sms();
+  if (sms <= 0) return KIVI_ERR_CUDA;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  DecodeArgs a;
+  a.c = view(cache);
+  a.q = q;
+  a.out = out;
+  a.ws = (float*)scratch;
+  a.units = cache->dims.B * cache->dims.Hkv;
+  a.Hkv = cache->dims.Hkv;
+  a.gq = gq;
+  a.D = cache->dims.D;
+  a.bits = cache->dims.bits;
+  a.dtype = cache->dims.dtype;
+  a.n_q = cache->n_q;
+  a.r = cache->r;
+  a.qscale = softmax_scale * kivi::kLog2e;
+  // the usual split plan, with the split count capped by the scratch size
+  const long long tiles =
+      cache->n_q / kivi::kTile + (cache->r + kivi::kTile - 1) / kivi::kTile;
+  long long s = max_splits(cache->dims, sms);
+  const long long fit = (long long)(KIVI_NOALLOC_SCRATCH_BYTES / per_split);
+  if (s > fit) s = fit;
+  if (s > tiles) s = tiles;
+  if (s < 1) s = 1;
+  const long long tps = (tiles + s - 1) / s;
+  a.tiles_per_split = (int)tps;
+  a.n_split = (int)((tiles + tps - 1) / tps);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t err = kivi::launch_decode_simt(a, st, g_ev0, g_ev1);
+  if (err == cudaSuccess) err = kivi::launch_decode_combine(a, st);
+  return err == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA;
+}
+
 void kivi_set_timing_events(void* start_event, void* stop_event) {
   g_ev0 = (cudaEvent_t)start_event;
   g_ev1 = (cudaEvent_t)stop_event;
@@ -262,6 +334,8 @@ const char* kivi_status_string(int status) {
     case KIVI_ERR_CAPACITY: return "KIVI_ERR_CAPACITY: tokens exceed the cache capacity";
     case KIVI_ERR_WORKSPACE: return "KIVI_ERR_WORKSPACE: workspace missing, small or misaligned";
     case KIVI_ERR_CUDA: return "KIVI_ERR_CUDA: CUDA launch or query failed";
+    case KIVI_ERR_SCRATCH_LIMIT:
+      return "KIVI_ERR_SCRATCH_LIMIT: request exceeds the fixed scratch of the no-allocation call";
   }
   return "unknown kivi status";
 }

@@ -86,7 +86,8 @@ typedef enum {
   KIVI_ERR_STATE = 3,       /* prefill on a non-empty cache; decode on an empty one */
   KIVI_ERR_CAPACITY = 4,    /* the tokens would not fit in `capacity` */
   KIVI_ERR_WORKSPACE = 5,   /* workspace missing, too small or misaligned */
-  KIVI_ERR_CUDA = 6         /* a CUDA launch or device query failed */
+  KIVI_ERR_CUDA = 6,        /* a CUDA launch or device query failed */
+  KIVI_ERR_SCRATCH_LIMIT = 7 /* request exceeds the fixed scratch of the _noalloc call */
 } kivi_status;
 
 typedef enum { KIVI_F16 = 0, KIVI_F32 = 1 } kivi_dtype;
@@ -212,6 +213,35 @@ KIVI_API void kivi_set_timing_events(void *start_event, void *stop_event);
 /* Number of context splits the decode kernel would use for this cache's
  * current fill level and Hq (>= 1), or 0 on error. */
 KIVI_API int kivi_decode_num_splits(const kivi_cache *cache, int Hq);
+
+/* Size of the fixed device scratch used by kivi_decode_attention_noalloc. */
+#define KIVI_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+/* Decode attention for callers that cannot allocate device memory.
+ * No counterpart on the pages: this is a library convenience, not part of
+ * the method.  Same arguments and result as kivi_decode_attention, minus the
+ * workspace: the cross-split partials go to a static device array of
+ * KIVI_NOALLOC_SCRATCH_BYTES (4 MiB) that the library reserves on every GPU
+ * it is loaded on, for the life of the process.  It is meant for callers
+ * that run where device allocation is unavailable or not allowed once they
+ * are running -- for example a plugin inside an inference engine that has
+ * already reserved all device memory for its own pool, or a latency-bound
+ * loop that must not call cudaMalloc because it can synchronize the device.
+ *   - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
+ *     library call.  The first call on a device looks up the scratch
+ *     array's device address (cudaGetSymbolAddress) with that device
+ *     current and keeps it; make that first call before any stream capture.
+ *   - The split count is capped so that B * Hq * splits * (D + 2) * 4 bytes
+ *     fit; if even one split does not fit, the call returns
+ *     KIVI_ERR_SCRATCH_LIMIT and launches nothing.
+ *   - All calls on a device share the one array, and it keeps whatever the
+ *     last call wrote (every byte a call reads it first writes itself).
+ *     Calls whose kernels overlap on the GPU (for example on two streams
+ *     without ordering between them) race on it: serialize them.
+ * Errors: as kivi_decode_attention (without KIVI_ERR_WORKSPACE), plus
+ * KIVI_ERR_SCRATCH_LIMIT. */
+KIVI_API int kivi_decode_attention_noalloc(const kivi_cache *cache, const void *q, int Hq,
+                                           float softmax_scale, void *out, void *stream);
 
 /* Human-readable name of a kivi_status. */
 KIVI_API const char *kivi_status_string(int status);
