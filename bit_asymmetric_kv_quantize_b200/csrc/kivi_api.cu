@@ -97,8 +97,41 @@ void plan_splits(const kivi_cache* c, int sms, int* n_split, int* tiles_per_spli
   *n_split = (int)((tiles + tps - 1) / tps);
 }
 
+// Tensor-core kernel: the quantized tiles in splits of a multiple of 4 tiles
+// (one pipeline stage), about kTcCtasPerSm CTAs per SM, plus one split that
+// holds only the residual window.
+constexpr int kTcCtasPerSm = 6;
+
+int tc_max_qsplits(const kivi_dims& d, int sms) {
+  const long long units = (long long)d.B * d.Hkv;
+  long long want = (kTcCtasPerSm * (long long)sms + units - 1) / units;
+  const long long stages = (d.capacity - d.R) / (4 * kivi::kTile);
+  if (want > stages) want = stages;
+  if (want > kMaxSplits - 1) want = kMaxSplits - 1;
+  return want < 1 ? 1 : (int)want;
+}
+
+void plan_tc(const kivi_cache* c, int sms, int* n_split, int* tiles_per_split) {
+  const long long n_qt = c->n_q / kivi::kTile;
+  int nq = 0;
+  long long tps = 4;
+  if (n_qt > 0) {
+    long long s = tc_max_qsplits(c->dims, sms);
+    if (s > (n_qt + 3) / 4) s = (n_qt + 3) / 4;
+    if (s < 1) s = 1;
+    tps = (n_qt + s - 1) / s;
+    tps = (tps + 3) / 4 * 4;
+    nq = (int)((n_qt + tps - 1) / tps);
+  }
+  *tiles_per_split = (int)tps;
+  *n_split = nq + (c->r > 0 ? 1 : 0);
+}
+
 size_t workspace_bytes(const kivi_dims& d, int Hq, int sms) {
-  return (size_t)d.B * Hq * max_splits(d, sms) * (d.D + 2) * sizeof(float);
+  int s = max_splits(d, sms);
+  const int t = tc_max_qsplits(d, sms) + 1;
+  if (t > s) s = t;
+  return (size_t)d.B * Hq * s * (d.D + 2) * sizeof(float);
 }
 
 int decode_common(const kivi_cache* c, const void* q, int Hq, float softmax_scale, void* out,
@@ -127,10 +160,15 @@ int decode_common(const kivi_cache* c, const void* q, int Hq, float softmax_scal
   a.n_q = c->n_q;
   a.r = c->r;
   a.qscale = softmax_scale * kivi::kLog2e;
-  plan_splits(c, sms, &a.n_split, &a.tiles_per_split);
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t err = kivi::launch_decode_simt(a, s, g_ev0, g_ev1);
-  (void)simt;
+  cudaError_t err;
+  if (simt) {
+    plan_splits(c, sms, &a.n_split, &a.tiles_per_split);
+    err = kivi::launch_decode_simt(a, s, g_ev0, g_ev1);
+  } else {
+    plan_tc(c, sms, &a.n_split, &a.tiles_per_split);
+    err = kivi::launch_decode_tc(a, s, g_ev0, g_ev1);
+  }
   if (err == cudaSuccess) err = kivi::launch_decode_combine(a, s);
   return err == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA;
 }
@@ -321,7 +359,7 @@ int kivi_decode_num_splits(const kivi_cache* cache, int Hq) {
   const int sms = device_sms();
   if (sms <= 0) return 0;
   int n, tps;
-  plan_splits(cache, sms, &n, &tps);
+  plan_tc(cache, sms, &n, &tps);
   return n;
 }
 

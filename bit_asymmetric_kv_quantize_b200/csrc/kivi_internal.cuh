@@ -84,12 +84,15 @@ struct DecodeArgs {
   long long n_q;
   int r;
   float qscale;    // softmax_scale * log2(e)
-  int n_split;
-  int tiles_per_split;
+  int n_split;          // splits per unit (the tensor-core kernel's last one
+                        // holds only the residual window when r > 0)
+  int tiles_per_split;  // 32-token quantized tiles per split
 };
 
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s, cudaEvent_t ev0,
                                cudaEvent_t ev1);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t s, cudaEvent_t ev0,
+                             cudaEvent_t ev1);
 cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t s);
 
 }  // namespace kivi
