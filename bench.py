@@ -67,6 +67,22 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest `value` over all ranks (every rank gets it); identity for one rank."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, batch: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s of `world` independent replicas, each decoding `batch`
+    sequences for `steps` steps, timed by the slowest rank."""
+    return world * batch * steps / (ms_max * 1e-3)
+
+
 def peak_hbm():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -242,11 +258,7 @@ def run_kivi(args, rank, world, local):
     barrier()
     ms = t0.elapsed_time(t1)
     split_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
-    ms_max = ms
-    if world > 1:
-        tt = torch.tensor([ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_max = float(tt.item())
+    ms_max = max_over_ranks(ms, world, device)
 
     # roofline of the split kernel: algorithmic bytes / event time
     bytes_total = sum(algorithmic_bytes(w, nq, r) for nq, r in fills)
@@ -283,18 +295,14 @@ def run_kivi(args, rank, world, local):
             ho.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(device)
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e_ms], device=device)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
-        e2e = {"value": world * w.B * n_e2e / (e_ms * 1e-3), "unit": "tokens/s",
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+        e2e = {"value": replica_throughput(world, w.B, n_e2e, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": e_ms / n_e2e}
 
     result = None
     if rank == 0:
-        tokens_per_s = world * w.B * args.steps / (ms_max * 1e-3)
+        tokens_per_s = replica_throughput(world, w.B, args.steps, ms_max)
         result = {
             "metric": METRIC,
             "value": tokens_per_s,
@@ -324,7 +332,7 @@ def run_kivi(args, rank, world, local):
                 "avg_launch_us": split_total_ms * 1e3 / args.steps,
             },
             "e2e": e2e,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": 2 * args.steps,
             "clocks": clk.summary(),
         }
     for c in caches:

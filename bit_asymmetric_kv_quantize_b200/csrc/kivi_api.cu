@@ -97,60 +97,92 @@ void plan_splits(const kivi_cache* c, int sms, int* n_split, int* tiles_per_spli
   *n_split = (int)((tiles + tps - 1) / tps);
 }
 
-// Tensor-core kernel: the quantized tiles in splits of a multiple of 4 tiles
-// (one pipeline stage), about kTcCtasPerSm CTAs per SM, plus one split that
-// holds only the residual window.
-constexpr int kTcCtasPerSm = 6;
+// Tensor-core kernel: persistent stream-K plan.  Every unit is laid out as
+// n_q/32 work indices (its quantized 32-token tiles) followed by
+// kWinWeight * ceil(r/32) indices standing for its residual window; the
+// units' indices end to end are cut into n_cta equal ranges of W >= 4.  A
+// unit is covered by the CTAs whose ranges meet its tiles or its window start
+// index -- at most ceil((n_q/32 + 1) / W) + 1 CTA segments, each writing one
+// partial -- and the last of them also takes the window.
+constexpr int kTcCtasPerSm = 3;  // upper bound; the kernel instance decides
+constexpr int kWinWeight = 3;  // cost of a window tile, in quantized tiles
 
-int tc_max_qsplits(const kivi_dims& d, int sms) {
+struct StreamPlan {
+  int n_cta;
+  long long W;
+  int max_seg;
+  int win_weight;
+};
+
+long long ceil_div(long long x, long long y) { return (x + y - 1) / y; }
+
+// Partial slots per unit that any fill level of this cache can need.
+int tc_seg_cap(const kivi_dims& d, int sms) {
   const long long units = (long long)d.B * d.Hkv;
-  long long want = (kTcCtasPerSm * (long long)sms + units - 1) / units;
-  const long long stages = (d.capacity - d.R) / (4 * kivi::kTile);
-  if (want > stages) want = stages;
-  if (want > kMaxSplits - 1) want = kMaxSplits - 1;
-  return want < 1 ? 1 : (int)want;
+  long long s = ceil_div((long long)kTcCtasPerSm * sms, units);
+  const long long t = ceil_div((d.capacity - d.R) / kivi::kTile + 1, 4);
+  if (t < s) s = t;
+  return (int)s + 1;
 }
 
-void plan_tc(const kivi_cache* c, int sms, int* n_split, int* tiles_per_split) {
+// ctas_per_sm: resident CTAs per SM of the kernel instance (<= kTcCtasPerSm);
+// seg_cap: largest number of partial slots per unit the workspace holds.
+void plan_stream(const kivi_cache* c, int sms, int ctas_per_sm, int seg_cap, StreamPlan* p) {
+  const long long units = (long long)c->dims.B * c->dims.Hkv;
   const long long n_qt = c->n_q / kivi::kTile;
-  int nq = 0;
-  long long tps = 4;
-  if (n_qt > 0) {
-    long long s = tc_max_qsplits(c->dims, sms);
-    if (s > (n_qt + 3) / 4) s = (n_qt + 3) / 4;
-    if (s < 1) s = 1;
-    tps = (n_qt + s - 1) / s;
-    tps = (tps + 3) / 4 * 4;
-    nq = (int)((n_qt + tps - 1) / tps);
+  const int ww = c->r > 0 ? kWinWeight * (int)ceil_div(c->r, kivi::kTile) : 1;
+  const long long UP = n_qt + ww;
+  const long long total = units * UP;
+  const long long P =
+      (long long)(ctas_per_sm < kTcCtasPerSm ? ctas_per_sm : kTcCtasPerSm) * sms;
+  long long W = ceil_div(total, P);
+  if (W < 12) W = 12;  // at least one full stage per CTA
+  if (seg_cap <= 1) {
+    W = UP;  // one CTA per unit: ranges align with the units
+  } else if (ceil_div(n_qt + 1, W) + 1 > seg_cap) {
+    W = ceil_div(n_qt + 1, seg_cap - 1);
   }
-  *tiles_per_split = (int)tps;
-  *n_split = nq + (c->r > 0 ? 1 : 0);
+  p->W = W;
+  p->win_weight = ww;
+  p->n_cta = (int)ceil_div(total, W);
+  p->max_seg = (W % UP == 0) ? 1 : (int)(ceil_div(n_qt + 1, W) + 1);
+}
+
+// Workspace: per-unit arrival counters (8 bytes each, 16-byte aligned block)
+// followed by the split partials [B*Hq][n_split][D + 2] floats.
+size_t counter_bytes(const kivi_dims& d) {
+  return ((size_t)d.B * d.Hkv * 8 + 15) / 16 * 16;
+}
+
+int ws_splits(const kivi_dims& d, int sms) {
+  int s = max_splits(d, sms);
+  const int t = tc_seg_cap(d, sms);
+  return t > s ? t : s;
 }
 
 size_t workspace_bytes(const kivi_dims& d, int Hq, int sms) {
-  int s = max_splits(d, sms);
-  const int t = tc_max_qsplits(d, sms) + 1;
-  if (t > s) s = t;
-  return (size_t)d.B * Hq * s * (d.D + 2) * sizeof(float);
+  return counter_bytes(d) + (size_t)d.B * Hq * ws_splits(d, sms) * (d.D + 2) * sizeof(float);
 }
 
-int decode_common(const kivi_cache* c, const void* q, int Hq, float softmax_scale, void* out,
-                  void* workspace, size_t ws_bytes, void* stream, bool simt) {
-  int rc = check_cache(c);
-  if (rc) return rc;
-  if (!q || !out || Hq <= 0 || Hq % c->dims.Hkv != 0) return KIVI_ERR_ARG;
+std::atomic<unsigned int> g_epoch{0};
+
+unsigned int next_epoch() {
+  unsigned int e = ++g_epoch;
+  if (e == 0) e = ++g_epoch;  // 0 never tags a call
+  return e;
+}
+
+// Validate, plan and launch one decode.  `ws` holds the arrival counters and
+// the partials; the split count is capped at `split_cap`.
+int decode_launch(const kivi_cache* c, const void* q, int Hq, float softmax_scale, void* out,
+                  void* ws, int split_cap, int sms, void* stream, bool simt) {
   const int gq = Hq / c->dims.Hkv;
-  if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KIVI_ERR_UNSUPPORTED;
-  if (c->n_q + c->r == 0) return KIVI_ERR_STATE;
-  const int sms = device_sms();
-  if (sms <= 0) return KIVI_ERR_CUDA;
-  if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(c->dims, Hq, sms))
-    return KIVI_ERR_WORKSPACE;
   DecodeArgs a;
   a.c = view(c);
   a.q = q;
   a.out = out;
-  a.ws = (float*)workspace;
+  a.ctr = (unsigned long long*)ws;
+  a.ws = (float*)((char*)ws + counter_bytes(c->dims));
   a.units = c->dims.B * c->dims.Hkv;
   a.Hkv = c->dims.Hkv;
   a.gq = gq;
@@ -160,17 +192,54 @@ int decode_common(const kivi_cache* c, const void* q, int Hq, float softmax_scal
   a.n_q = c->n_q;
   a.r = c->r;
   a.qscale = softmax_scale * kivi::kLog2e;
+  a.epoch = next_epoch();
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t err;
   if (simt) {
     plan_splits(c, sms, &a.n_split, &a.tiles_per_split);
+    if (a.n_split > split_cap) {  // re-plan with fewer, longer splits
+      const long long tiles = c->n_q / kivi::kTile + (c->r + kivi::kTile - 1) / kivi::kTile;
+      const long long tps = (tiles + split_cap - 1) / split_cap;
+      a.tiles_per_split = (int)tps;
+      a.n_split = (int)((tiles + tps - 1) / tps);
+    }
     err = kivi::launch_decode_simt(a, s, g_ev0, g_ev1);
   } else {
-    plan_tc(c, sms, &a.n_split, &a.tiles_per_split);
+    int occ = 0;
+    if (kivi::decode_tc_ctas_per_sm(a, &occ) != cudaSuccess) return KIVI_ERR_CUDA;
+    StreamPlan sp;
+    plan_stream(c, sms, occ, split_cap, &sp);
+    a.n_cta = sp.n_cta;
+    a.tiles_per_cta = sp.W;
+    a.max_seg = sp.max_seg;
+    a.win_weight = sp.win_weight;
+    a.n_split = sp.max_seg;
+    a.tiles_per_split = 0;
     err = kivi::launch_decode_tc(a, s, g_ev0, g_ev1);
   }
-  if (err == cudaSuccess) err = kivi::launch_decode_combine(a, s);
   return err == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA;
+}
+
+int decode_checks(const kivi_cache* c, const void* q, int Hq, const void* out) {
+  int rc = check_cache(c);
+  if (rc) return rc;
+  if (!q || !out || Hq <= 0 || Hq % c->dims.Hkv != 0) return KIVI_ERR_ARG;
+  const int gq = Hq / c->dims.Hkv;
+  if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KIVI_ERR_UNSUPPORTED;
+  if (c->n_q + c->r == 0) return KIVI_ERR_STATE;
+  return KIVI_OK;
+}
+
+int decode_common(const kivi_cache* c, const void* q, int Hq, float softmax_scale, void* out,
+                  void* workspace, size_t ws_bytes, void* stream, bool simt) {
+  int rc = decode_checks(c, q, Hq, out);
+  if (rc) return rc;
+  const int sms = device_sms();
+  if (sms <= 0) return KIVI_ERR_CUDA;
+  if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(c->dims, Hq, sms))
+    return KIVI_ERR_WORKSPACE;
+  return decode_launch(c, q, Hq, softmax_scale, out, workspace, ws_splits(c->dims, sms), sms,
+                       stream, simt);
 }
 
 // ---- static scratch for kivi_decode_attention_noalloc ----------------------
@@ -304,48 +373,21 @@ int kivi_decode_attention_simt(const kivi_cache* cache, const void* q, int Hq,
 
 int kivi_decode_attention_noalloc(const kivi_cache* cache, const void* q, int Hq,
                                   float softmax_scale, void* out, void* stream) {
-  int rc = check_cache(cache);
+  int rc = decode_checks(cache, q, Hq, out);
   if (rc) return rc;
-  if (!q || !out || Hq <= 0 || Hq % cache->dims.Hkv != 0) return KIVI_ERR_ARG;
-  const int gq = Hq / cache->dims.Hkv;
-  if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KIVI_ERR_UNSUPPORTED;
-  if (cache->n_q + cache->r == 0) return KIVI_ERR_STATE;
+  // the scratch holds the per-unit counters, then the partials of at most
+  // `fit` splits
   const size_t per_split = (size_t)cache->dims.B * Hq * (cache->dims.D + 2) * sizeof(float);
-  if (per_split > KIVI_NOALLOC_SCRATCH_BYTES) return KIVI_ERR_SCRATCH_LIMIT;
+  const size_t cbytes = counter_bytes(cache->dims);
+  if (cbytes + per_split > KIVI_NOALLOC_SCRATCH_BYTES) return KIVI_ERR_SCRATCH_LIMIT;
   const int sms = device_sms();
   if (sms <= 0) return KIVI_ERR_CUDA;
   void* scratch = nullptr;
   rc = noalloc_scratch(&scratch);
   if (rc) return rc;
-  DecodeArgs a;
-  a.c = view(cache);
-  a.q = q;
-  a.out = out;
-  a.ws = (float*)scratch;
-  a.units = cache->dims.B * cache->dims.Hkv;
-  a.Hkv = cache->dims.Hkv;
-  a.gq = gq;
-  a.D = cache->dims.D;
-  a.bits = cache->dims.bits;
-  a.dtype = cache->dims.dtype;
-  a.n_q = cache->n_q;
-  a.r = cache->r;
-  a.qscale = softmax_scale * kivi::kLog2e;
-  // the usual split plan, with the split count capped by the scratch size
-  const long long tiles =
-      cache->n_q / kivi::kTile + (cache->r + kivi::kTile - 1) / kivi::kTile;
-  long long s = max_splits(cache->dims, sms);
-  const long long fit = (long long)(KIVI_NOALLOC_SCRATCH_BYTES / per_split);
-  if (s > fit) s = fit;
-  if (s > tiles) s = tiles;
-  if (s < 1) s = 1;
-  const long long tps = (tiles + s - 1) / s;
-  a.tiles_per_split = (int)tps;
-  a.n_split = (int)((tiles + tps - 1) / tps);
-  cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t err = kivi::launch_decode_simt(a, st, g_ev0, g_ev1);
-  if (err == cudaSuccess) err = kivi::launch_decode_combine(a, st);
-  return err == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA;
+  const long long fit = (long long)((KIVI_NOALLOC_SCRATCH_BYTES - cbytes) / per_split);
+  const int cap = (int)(fit < ws_splits(cache->dims, sms) ? fit : ws_splits(cache->dims, sms));
+  return decode_launch(cache, q, Hq, softmax_scale, out, scratch, cap, sms, stream, false);
 }
 
 void kivi_set_timing_events(void* start_event, void* stop_event) {
@@ -358,9 +400,16 @@ int kivi_decode_num_splits(const kivi_cache* cache, int Hq) {
   if (cache->n_q + cache->r == 0) return 0;
   const int sms = device_sms();
   if (sms <= 0) return 0;
-  int n, tps;
-  plan_tc(cache, sms, &n, &tps);
-  return n;
+  DecodeArgs a;
+  a.D = cache->dims.D;
+  a.bits = cache->dims.bits;
+  a.gq = Hq / cache->dims.Hkv;
+  a.dtype = cache->dims.dtype;
+  int occ = 0;
+  if (kivi::decode_tc_ctas_per_sm(a, &occ) != cudaSuccess) return 0;
+  StreamPlan sp;
+  plan_stream(cache, sms, occ, ws_splits(cache->dims, sms), &sp);
+  return sp.max_seg;
 }
 
 const char* kivi_status_string(int status) {

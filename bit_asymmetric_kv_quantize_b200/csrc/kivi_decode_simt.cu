@@ -1,6 +1,5 @@
 // kivi_decode_simt.cu -- split-context decode attention over the packed
-// KIVI cache on CUDA cores (SIMT), and the cross-split merge shared by every
-// decode kernel.
+// KIVI cache on CUDA cores (SIMT); the split merge is fused in (finish_unit).
 //
 // Method: "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache",
 // study.space summary: decode attention is computed over the quantized
@@ -9,7 +8,7 @@
 // owns a contiguous range of 32-token tiles of one (batch, KV head) unit for
 // all query heads of the GQA group, keeps a running max m, sum l and
 // unnormalised accumulator per head, and writes (m, l, acc[D]) to the
-// workspace; the merge kernel rescales the splits to a common max.
+// workspace; the last CTA of the unit rescales the splits to a common max.
 //
 // Keys use the factored form  q.khat = sum_d (q_d s_gd) c_td + sum_d q_d z_gd
 // (scale and zero are per key group and channel); values are dequantized as
@@ -239,25 +238,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_simt(DecodeArgs a) {
     }
     P[2 + d] = num;
   }
-}
-
-// grid (B * Hq), block D: out = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s
-template <int D, typename T>
-__global__ void __launch_bounds__(D) decode_combine(const float* __restrict__ ws,
-                                                    T* __restrict__ out, int n_split) {
-  const long long row = blockIdx.x;
-  const float* P = ws + row * n_split * (D + 2);
-  float M = kNegInf;
-  for (int s = 0; s < n_split; ++s) M = fmaxf(M, P[s * (D + 2)]);
-  float num = 0.f, den = 0.f;
-  for (int s = 0; s < n_split; ++s) {
-    const float ms = P[s * (D + 2)];
-    if (ms == kNegInf) continue;
-    const float sc = exp2f(ms - M);
-    num = fmaf(sc, P[s * (D + 2) + 2 + threadIdx.x], num);
-    den = fmaf(sc, P[s * (D + 2) + 1], den);
-  }
-  out[row * D + threadIdx.x] = from_f32<T>(num / den);
+  __shared__ int last_flag;
+  finish_unit<D, GQ, T>(a, b, kv, &last_flag);
 }
 
 template <int D, int BITS, int GQ, typename T>
@@ -300,26 +282,6 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s, cudaEvent_t 
   if (a.bits == 4 && a.dtype == 0) return simt_d<4, __half>(a, s, e0, e1);
   if (a.bits == 4 && a.dtype == 1) return simt_d<4, float>(a, s, e0, e1);
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t s) {
-  const unsigned rows = (unsigned)((long long)a.units * a.gq);
-  if (a.dtype == 0) {
-    switch (a.D) {
-      case 32: decode_combine<32, __half><<<rows, 32, 0, s>>>(a.ws, (__half*)a.out, a.n_split); break;
-      case 64: decode_combine<64, __half><<<rows, 64, 0, s>>>(a.ws, (__half*)a.out, a.n_split); break;
-      case 128: decode_combine<128, __half><<<rows, 128, 0, s>>>(a.ws, (__half*)a.out, a.n_split); break;
-      default: return cudaErrorInvalidValue;
-    }
-  } else {
-    switch (a.D) {
-      case 32: decode_combine<32, float><<<rows, 32, 0, s>>>(a.ws, (float*)a.out, a.n_split); break;
-      case 64: decode_combine<64, float><<<rows, 64, 0, s>>>(a.ws, (float*)a.out, a.n_split); break;
-      case 128: decode_combine<128, float><<<rows, 128, 0, s>>>(a.ws, (float*)a.out, a.n_split); break;
-      default: return cudaErrorInvalidValue;
-    }
-  }
-  return cudaGetLastError();
 }
 
 }  // namespace kivi

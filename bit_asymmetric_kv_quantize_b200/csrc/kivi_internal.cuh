@@ -87,12 +87,82 @@ struct DecodeArgs {
   int n_split;          // splits per unit (the tensor-core kernel's last one
                         // holds only the residual window when r > 0)
   int tiles_per_split;  // 32-token quantized tiles per split
+  unsigned long long* ctr;  // per-unit arrival counters (in the workspace)
+  unsigned int epoch;       // tag of this call in the counters (never 0)
+  // tensor-core kernel (persistent, stream-K): each unit occupies
+  // n_q/32 + win_weight consecutive work indices (its quantized tiles, then
+  // its residual window weighted as win_weight tiles); CTA c owns indices
+  // [c * tiles_per_cta, (c + 1) * tiles_per_cta); partials are
+  // [units][max_seg][GQ][D + 2]
+  int n_cta;
+  long long tiles_per_cta;
+  int max_seg;
+  int win_weight;
 };
+
+constexpr float kNaN = __builtin_nanf("");
+
+// End of a split CTA, after it wrote its (m, l, acc[D]) partials: the last CTA
+// of the unit to arrive merges all splits of the unit into out.  Arrival is
+// counted in a per-unit 64-bit word tagged with this call's epoch in the high
+// half, so counters left by earlier calls are simply restarted; no zeroing
+// and no waiting (a lock-free compare-and-swap, bounded retries).
+// out[b][kv*GQ + h][d] = sum_s 2^(m_s - M) acc_s[d] / sum_s 2^(m_s - M) l_s.
+template <int D, int GQ, typename T>
+__device__ __forceinline__ void finish_unit(const DecodeArgs& a, long long b, int kv,
+                                            int* flag) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long* ctr = a.ctr + (b * a.Hkv + kv);
+    const unsigned long long ep = (unsigned long long)a.epoch << 32;
+    unsigned long long v = atomicAdd(ctr, 0ull);
+    int last = -1;  // -1: gave up (publish NaN)
+    for (int it = 0; it < 4096; ++it) {
+      const unsigned long long nv = ((v >> 32) == a.epoch) ? v + 1ull : (ep | 1ull);
+      const unsigned long long old = atomicCAS(ctr, v, nv);
+      if (old == v) {
+        last = ((long long)(nv & 0xffffffffull) == (long long)a.n_split) ? 1 : 0;
+        break;
+      }
+      v = old;
+    }
+    *flag = last;
+  }
+  __syncthreads();
+  const int last = *flag;
+  if (last == 0) return;
+  __threadfence();
+  const int Hq = a.Hkv * GQ;
+  T* out = reinterpret_cast<T*>(a.out);
+  for (int idx = threadIdx.x; idx < GQ * D; idx += blockDim.x) {
+    const int h = idx / D, d = idx % D;
+    const long long row = b * Hq + (long long)kv * GQ + h;
+    float res = kNaN;
+    if (last > 0) {
+      const float* P = a.ws + row * a.n_split * (D + 2);
+      float M = -__builtin_huge_valf();
+      for (int s = 0; s < a.n_split; ++s) M = fmaxf(M, __ldcg(P + s * (D + 2)));
+      float num = 0.f, den = 0.f;
+      for (int s = 0; s < a.n_split; ++s) {
+        const float ms = __ldcg(P + s * (D + 2));
+        if (ms == -__builtin_huge_valf()) continue;
+        const float sc = exp2f(ms - M);
+        num = fmaf(sc, __ldcg(P + s * (D + 2) + 2 + d), num);
+        den = fmaf(sc, __ldcg(P + s * (D + 2) + 1), den);
+      }
+      res = num / den;
+    }
+    out[row * D + d] = from_f32<T>(res);
+  }
+}
 
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s, cudaEvent_t ev0,
                                cudaEvent_t ev1);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t s, cudaEvent_t ev0,
                              cudaEvent_t ev1);
-cudaError_t launch_decode_combine(const DecodeArgs& a, cudaStream_t s);
+// Resident CTAs per SM of the tensor-core kernel instance that `a` selects
+// (uses a.D, a.bits, a.gq, a.dtype).
+cudaError_t decode_tc_ctas_per_sm(const DecodeArgs& a, int* ctas_per_sm);
 
 }  // namespace kivi

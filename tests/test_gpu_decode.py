@@ -67,7 +67,7 @@ def test_decode_many_splits(T, kernel):
     """One unit, long context: the context is split over many CTAs and merged."""
     w = small(D=128, B=1, Hkv=1, gq=4, T=T, R=128)
     gc, oc, q, out, sigma = run(w, kernel, capacity=9216)
-    assert gc.num_splits(w.Hq) > 8
+    assert gc.num_splits(w.Hq) > 4
     assert_decode_close(out, oc, q, sigma)
 
 
