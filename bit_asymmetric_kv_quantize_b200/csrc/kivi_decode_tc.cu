@@ -9,47 +9,71 @@
 // enter one online softmax; each CTA writes (m, l, acc[D]) per query head to
 // the workspace and the last CTA of the unit merges the splits.
 //
-// Per CTA: one (batch, KV head) unit and a contiguous range of 32-token tiles
-// (one key group each), all query heads of the GQA group.  The last split of
-// a unit owns the residual window and runs on CUDA cores; every other split
-// streams its tiles:
+// Per CTA: a contiguous range of work indices over (unit, 32-token tile)
+// pairs (persistent, stream-K), all query heads of the GQA group.  The CTA
+// that ends a unit also folds in the unit's residual window (CUDA cores).
 //   * memory: a producer warp issues 1-D bulk copies (cp.async.bulk,
 //     completion on a "full" mbarrier) of each stage -- NW tiles of key
 //     codes, key scales, key zeros, value codes, value scales, value zeros,
 //     six contiguous ranges -- into a ring of shared-memory stages; NW
 //     consumer warps take one tile each and release the stage on an "empty"
-//     mbarrier.  No CTA-wide barrier in the streaming loop.  The grid is
-//     exactly the CTAs that fit at once (persistent).
-//   * scores: S = K q'^T on tensor cores: key codes as the A operand
-//     (16 tokens x 16 channels per mma), taken from one 32-bit word per token
-//     by a shift and a mask -- a code c in the low mantissa bits of an fp16
-//     is the exact subnormal c * 2^-24, so no conversion is needed and 2^24
-//     is restored on the fp32 result; q'_{h,d} = q_{h,d} s_{g,d} split into
-//     fp16 hi and lo columns of B.  score = 2^24 S + sum_d q_d z_{g,d}.
+//     mbarrier.  No CTA-wide barrier in the streaming loop.
+//   * codes as fp16 operands: a 2-bit word holds code i at bits 2i, a 4-bit
+//     word code i at bits 4i.  A "pair" (two codes, one per 16-bit half) is
+//     taken out with a mask after at most one shift, which leaves each code
+//     at some bit e < 10 of its half: read as fp16 that is the exact
+//     subnormal c * 2^(e - 24).  The other operand's row for that k carries
+//     the factor 2^(S - e), so every product is c * x * 2^(S - 24) and the
+//     fp32 result is rescaled once by 2^(24 - S).
+//   * scores: S = K q'^T, key codes as the A operand (16 tokens x 16
+//     channels per mma; lane tq of a row owns the code pairs
+//     [tq*D/8, (tq+1)*D/8) of the token), q'_{h,d} = q_{h,d} s_{g,d} split
+//     into fp16 hi and lo; head h uses columns 2(h%4) (hi) and 2(h%4)+1 (lo)
+//     of n-tile h/4, so each lane's accumulator pair is one head.
+//     score = sum_d q'_d c_d + sum_d q_d z_{g,d}.
 //   * softmax: running max and sum in log2 units (q pre-scaled by
-//     softmax_scale * log2 e, exp2f).
+//     softmax_scale * log2 e, exp2f); the cross-lane max is formed only when
+//     some score exceeds the running max (a warp vote), so p <= 1 always.
 //   * values: O += V^T p' on tensor cores, value codes as the A operand
-//     (16 channels x 16 tokens, same shift-and-mask), p'_{t,h} =
-//     p_{t,h} s_{t,j} split into hi and lo columns of B; the zero enters as
-//     sum_t p_t z_{t,j} per value group.
+//     (16 channels x 16 tokens), p'_{t,h} = p_{t,h} s_{t,j} split into hi and
+//     lo columns as above; the zero enters as sum_t p_t z_{t,j}.
 // The q' and p' fragments are built cooperatively (each lane converts a few
-// values and stores them in fragment order in per-warp shared memory).  The
-// channel (key) and token (value) order inside an mma k-slice follows the
-// bit order of the words.
+// values and stores them in fragment order, XOR-swizzled, in per-warp shared
+// memory).
 #include "kivi_internal.cuh"
 
 namespace kivi {
 namespace {
 
 constexpr float kNegInf = -__builtin_huge_valf();
-constexpr float kTwo24 = 16777216.0f;
 constexpr long long kWaitCycles = 1LL << 32;  // ~2 s: bounded wait on our own copies
+
+// Code pairs of one 32-bit word.  2-bit: pair i (i < 8) = codes i and i + 8;
+// 4-bit: pair i (i < 4) = codes i and i + 4.  (w >> shift(i)) & mask(i) puts
+// the pair's codes at bit e(i) of the low and the high half.
+template <int BITS>
+struct Pairs;
+template <>
+struct Pairs<2> {
+  static constexpr int PPW = 8;   // pairs per word
+  static constexpr int EMAX = 8;  // largest e
+  __host__ __device__ static constexpr int e(int i) { return i < 5 ? 2 * i : 2 * (i - 5); }
+  __host__ __device__ static constexpr int shift(int i) { return i < 5 ? 0 : 10; }
+  __host__ __device__ static constexpr uint32_t mask(int i) { return 0x00030003u << e(i); }
+};
+template <>
+struct Pairs<4> {
+  static constexpr int PPW = 4;
+  static constexpr int EMAX = 4;
+  __host__ __device__ static constexpr int e(int i) { return 4 * (i & 1); }
+  __host__ __device__ static constexpr int shift(int i) { return i < 2 ? 0 : 8; }
+  __host__ __device__ static constexpr uint32_t mask(int i) { return 0x000F000Fu << e(i); }
+};
 
 // NW consumer warps (one 32-token tile each per stage) and one producer warp
 // per CTA.  Measured on B200: one query head per KV head runs best as three
-// 4-warp CTAs per SM (124 registers); grouped heads need ~160 registers per
-// thread and run best as one CTA per SM with 11 (GQ 2, 4) or 7 (GQ 8)
-// consumer warps sharing one ring.
+// 4-warp CTAs per SM; grouped heads run best as one CTA per SM with 11
+// (GQ 2, 4) or 7 (GQ 8) consumer warps sharing one ring.
 template <int D, int BITS, int GQ>
 struct Geo {
   static constexpr int NW = GQ == 1 ? 4 : (GQ == 8 ? 7 : 11);
@@ -59,6 +83,7 @@ struct Geo {
   static constexpr int WK = D / E;       // key words per token
   static constexpr int NJ = D / kGv;     // value groups per token
   static constexpr int KSL = D / 16;     // k-slices of the score product
+  static constexpr int NSL = kTile / 16;  // k-slices of the value product
   static constexpr int KC_B = kTile * WK * 4;
   static constexpr int KM_B = D * 4;
   static constexpr int VC_B = (kTile / E) * D * 4;
@@ -72,11 +97,12 @@ struct Geo {
   static constexpr int O_VZ = O_VS + kStage * VM_B;
   static constexpr int STAGE_B = O_VZ + kStage * VM_B;
   static constexpr int NSTAGE = NW == 4 ? (BITS == 2 ? 3 : 2) : 2;
-  static constexpr int NPB = GQ == 8 ? 2 : 1;          // hi/lo in separate B operands
-  // per-warp scratch (bytes)
-  static constexpr int QB_B = NPB * KSL * 32 * 8;      // q' B fragments (score product)
-  static constexpr int PB_B = NPB * NJ * 2 * 32 * 8;   // p' B fragments (value product)
-  static constexpr int PBUF_B = GQ * kTile * 4;        // p per head and token
+  static constexpr int NPB = GQ == 8 ? 2 : 1;  // n-tiles of 8 columns (4 heads x hi, lo)
+  static constexpr int PST = kTile + 8;        // p buffer stride per head (floats)
+  // per-warp scratch (bytes): fragment blocks of 32 lanes x 2 words
+  static constexpr int QB_B = NPB * KSL * 256;        // q' B fragments (score product)
+  static constexpr int PB_B = NPB * NJ * NSL * 256;   // p' B fragments (value product)
+  static constexpr int PBUF_B = GQ * PST * 4;         // p per head and token
   static constexpr int WARP_B = QB_B + PB_B + PBUF_B;
   // whole CTA
   static constexpr int O_WARP = NSTAGE * STAGE_B;
@@ -86,7 +112,16 @@ struct Geo {
   static constexpr int O_FLAG = O_BAR + 2 * NSTAGE * 8;
   static constexpr int SMEM_B = O_FLAG + 16;
   static_assert(SMEM_B <= 227 * 1024, "shared memory per CTA");
+  static_assert(O_BAR % 8 == 0 && WARP_B % 16 == 0, "alignment");
   static constexpr int MIN_CTAS = NW == 4 ? 3 : 1;
+  // key operand: code pairs per lane and row, words a lane loads per row
+  static constexpr int PPL = D / 8;
+  static constexpr int PPW = Pairs<BITS>::PPW;
+  static constexpr bool WHOLE = PPL >= PPW;  // a lane's pairs fill whole words
+  static constexpr int NWL = WHOLE ? PPL / PPW : 1;
+  // operand scale offsets: the factor 2^(S - e) lies in [2^-S, 2^S]
+  static constexpr int SK = Pairs<BITS>::EMAX / 2;
+  static constexpr int SV = BITS == 2 ? 3 : 2;  // value e: 2-bit 0,2,4,6; 4-bit 0,4
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -130,56 +165,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// D (16x8, fp32) += A (16x16, fp16, row) * B (16x8, fp16, col).  Not volatile:
+// no side effects, so the compiler may schedule independent chains together.
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Position of element i (0..15) of a k-slice inside an mma fragment:
-// lane group `tq` (threadID_in_group), k-pair `kp` (0: k = 2tq,2tq+1;
-// 1: k = 2tq+8, 2tq+9) and half `hf` of the 32-bit register.  It mirrors the
-// shift-and-mask extraction: 2-bit words give pairs (i, i+8) and
-// (i+4, i+12), 4-bit word pairs give (i, i+4) and (i+8, i+12).
-template <int BITS>
-__device__ __forceinline__ void slot_of(int i, int& tq, int& kp, int& hf) {
-  tq = i & 3;
-  if (BITS == 2) {
-    kp = (i >> 2) & 1;
-    hf = i >> 3;
-  } else {
-    kp = i >> 3;
-    hf = (i >> 2) & 1;
-  }
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) {
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Two fp16 codes (exact subnormals c * 2^-24) per register: k-pairs tq, tq+4.
-template <int BITS>
-__device__ __forceinline__ void codes_pair(uint32_t w_lo, uint32_t w_hi, int tq, uint32_t& kp0,
-                                           uint32_t& kp1) {
-  if (BITS == 2) {
-    const uint32_t w1 = w_lo >> (2 * tq);
-    kp0 = w1 & 0x00030003u;
-    kp1 = (w1 >> 8) & 0x00030003u;
-  } else {
-    kp0 = (w_lo >> (4 * tq)) & 0x000F000Fu;
-    kp1 = (w_hi >> (4 * tq)) & 0x000F000Fu;
-  }
+// x = hi + lo in fp16 for two values at once (low half: a, high half: b).
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 f = __half22float2(h);
+  hi = h2_bits(h);
+  lo = h2_bits(__floats2half2_rn(a - f.x, b - f.y));
 }
 
-__device__ __forceinline__ void split_f16(float x, __half& hi, __half& lo) {
-  hi = __float2half_rn(x);
-  lo = __float2half_rn(x - __half2float(hi));
-}
-
-// Column of the fragment B operands (q' and p') that holds the hi or lo part
-// of head h: GQ <= 4 packs hi in columns 0..3 and lo in 4..7 of one
-// operand; GQ == 8 uses two operands (hi, lo) with column h each.
-template <int GQ>
-__device__ __forceinline__ int col_of(int h, int lo) { return GQ == 8 ? h : h + 4 * lo; }
+// Word offset of fragment slot `lane2` (= 4 n + tq) in a 64-word B block for
+// k-slice `sl`: an XOR swizzle that keeps the cooperative fragment stores
+// free of bank conflicts while each lane still reads a contiguous 8 bytes.
+__device__ __forceinline__ int frag_word(int lane2, int sl) { return 2 * (lane2 ^ (4 * (sl & 3))); }
 
 // Consumer-only barrier (the producer warp keeps streaming meanwhile).
 template <int NW>
@@ -191,15 +202,17 @@ template <int D, int BITS, int GQ, typename T>
 __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::MIN_CTAS)
     decode_stream_tc(DecodeArgs a) {
   using G = Geo<D, BITS, GQ>;
+  using PR = Pairs<BITS>;
   constexpr int kW = G::NW;
-  constexpr int kThreads = G::THREADS;
   constexpr int kStage = G::kStage;
-  (void)kThreads;
   using Lt = Layout<D, BITS>;
-  constexpr int E = G::E, WK = G::WK, NJ = G::NJ, KSL = G::KSL;
+  constexpr int E = G::E, WK = G::WK, NJ = G::NJ, KSL = G::KSL, NSL = G::NSL;
   constexpr int NM = D / 16;  // value m-tiles (16 channels each)
   constexpr int NPB = G::NPB;
+  constexpr int PST = G::PST;
   constexpr int CPL = D / 32;  // window path: channels per lane
+  constexpr float kKeyOut = (float)(1 << (24 - G::SK));
+  constexpr float kValOut = (float)(1 << (24 - G::SV));
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -232,6 +245,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp < kW) {
+    // fragment columns of absent heads stay zero
     unsigned char* wb = smem + G::O_WARP + warp * G::WARP_B;
     for (int i = lane; i < (G::QB_B + G::PB_B) / 4; i += 32) reinterpret_cast<uint32_t*>(wb)[i] = 0u;
   }
@@ -286,20 +300,68 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
   } else {
     // ---------------- consumer warps
     unsigned char* wb = smem + G::O_WARP + warp * G::WARP_B;
-    uint32_t* qB = reinterpret_cast<uint32_t*>(wb);
-    __half* qBh = reinterpret_cast<__half*>(wb);
-    uint32_t* pB = reinterpret_cast<uint32_t*>(wb + G::QB_B);
-    __half* pBh = reinterpret_cast<__half*>(wb + G::QB_B);
-    float* pbuf = reinterpret_cast<float*>(wb + G::QB_B + G::PB_B);
+    uint32_t* qB = reinterpret_cast<uint32_t*>(wb);                 // [NPB][KSL][64]
+    uint32_t* pB = reinterpret_cast<uint32_t*>(wb + G::QB_B);       // [NPB][NJ][NSL][64]
+    __half* pBh = reinterpret_cast<__half*>(pB);
+    float* pbuf = reinterpret_cast<float*>(wb + G::QB_B + G::PB_B);  // [GQ][PST]
 
-    // score-side head pair of this lane: hA = 2*(tq & 1) (GQ <= 4) or 2*tq
-    // (GQ == 8), and hA + 1; the P.V accumulator columns 2tq, 2tq+1 hold the
-    // same two heads (hi or lo part)
-    const int hA = GQ == 8 ? 2 * tq : 2 * (tq & 1);
-    const int hB = hA + 1;
-    const bool vA = hA < GQ, vB = hB < GQ;
-    const bool owner = (GQ == 8 || tq < 2);  // lanes whose columns are the hi parts
-    constexpr float kCodeScale = kTwo24;  // codes enter the mma as c * 2^-24
+    // -- q' build: lane classes.  Head class hc = lane % GL builds heads
+    // hc + GL x; within a class, lane index jl = lane / GL takes the
+    // "couples" (two adjacent pairs of one owner lane: B registers b0, b1 of
+    // k-slice sl for owner tq_o) with tq_o = jl & 3, sl = (jl >> 2) + (8/GL) m.
+    constexpr int GL = GQ < 4 ? GQ : 4;
+    constexpr int HX = GQ / GL;
+    constexpr int MC = (KSL * GL + 7) / 8;
+    const int hc = lane % GL, jl = lane / GL;
+    int cp_ch[MC];       // first channel c0 of the couple (pairs: c0, c0+1 | c0+PPW, c0+PPW+1)
+    int cp_w[MC];        // word offset of the owner's slot for column 0 in block sl
+    int cp_s3[MC];       // sl & 3 (swizzle)
+    float cp_f0[MC], cp_f1[MC];  // 2^(SK - e) of the two pairs
+    bool cp_ok[MC];
+#pragma unroll
+    for (int m = 0; m < MC; ++m) {
+      const int tq_o = jl & 3, sl = (jl >> 2) + (8 / GL) * m;
+      cp_ok[m] = sl < KSL;
+      const int slc = cp_ok[m] ? sl : 0;
+      const int pidx0 = tq_o * G::PPL + 2 * slc;
+      const int wd = pidx0 / G::PPW, i0 = pidx0 % G::PPW;
+      cp_ch[m] = wd * E + i0;
+      cp_s3[m] = slc & 3;
+      cp_w[m] = slc * 64 + 2 * tq_o;
+      cp_f0[m] = __int_as_float((127 + G::SK - PR::e(i0)) << 23);
+      cp_f1[m] = __int_as_float((127 + G::SK - PR::e(i0 + 1)) << 23);
+    }
+    // -- key operand (D = 32, 2-bit): a lane's four pairs sit in word tq/2,
+    // pairs 4 (tq & 1) + jj -- shifts and masks differ per lane
+    uint32_t kS[4], kM[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int i = 4 * (tq & 1) + jj;
+      kS[jj] = (uint32_t)Pairs<2>::shift(i);
+      kM[jj] = Pairs<2>::mask(i);
+    }
+    // -- value operand: lane tq takes the pairs at e = 2 tq (2-bit) or
+    // 4 (tq & 1) (4-bit) of its word; a0 / a1 unshifted, a2 / a3 after >> 8
+    const uint32_t vM = BITS == 2 ? (0x00030003u << (2 * tq))
+                                  : ((tq & 1) ? 0x00F000F0u : 0x000F000Fu);
+    const int vtw = BITS == 2 ? 0 : (tq >> 1);  // token-word offset of this lane
+    // -- p' build, lane = token t: its k-slice, owner slot and e
+    int pt_sl, pt_tq, pt_kp, pt_hf, pt_e;
+    if (BITS == 2) {
+      const int i = lane & 15;
+      pt_sl = lane >> 4; pt_tq = i & 3; pt_kp = (i >> 2) & 1; pt_hf = (i >> 3) & 1; pt_e = 2 * pt_tq;
+    } else {
+      const int tw = lane >> 3, i = lane & 7;
+      pt_sl = tw >> 1; pt_tq = 2 * (tw & 1) + (i & 1); pt_kp = (i >> 1) & 1; pt_hf = (i >> 2) & 1;
+      pt_e = 4 * (i & 1);
+    }
+    const float pt_f = __int_as_float((127 + G::SV - pt_e) << 23);
+    const int pt_base = pt_sl * 128 + 2 * pt_kp + pt_hf;  // halves, block (0, 0, pt_sl)
+    const int pt_s3 = pt_sl & 3;
+
+    bool vh[NPB];  // this lane's score / accumulator head tq + 4p exists
+#pragma unroll
+    for (int p = 0; p < NPB; ++p) vh[p] = tq + 4 * p < GQ;
 
     long long st = 0;  // ring position, in step with the producer
     for (long long u = G0 / UP; G0 < G1 && u <= (G1 - 1) / UP; ++u) {
@@ -318,27 +380,38 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
       const int n_seg = (int)(l_cta - f_cta + 1);
       const bool window_owner = a.r > 0 && cta == l_cta;
 
-      float qv[GQ][NJ];  // q for the cooperative q' build: channels lane + 32 i
+      // q (scaled by softmax_scale log2 e) at this lane's couple channels,
+      // order c0, c0+PPW, c0+1, c0+PPW+1 (b0 low, b0 high, b1 low, b1 high)
+      float qf[HX][MC][4];
 #pragma unroll
-      for (int h = 0; h < GQ; ++h)
+      for (int x = 0; x < HX; ++x)
 #pragma unroll
-        for (int i = 0; i < NJ; ++i) qv[h][i] = to_f32(qg[h * D + lane + 32 * i]) * a.qscale;
+        for (int m = 0; m < MC; ++m) {
+          const T* qh = qg + (hc + GL * x) * D + cp_ch[m];
+          qf[x][m][0] = to_f32(qh[0]) * a.qscale;
+          qf[x][m][1] = to_f32(qh[G::PPW]) * a.qscale;
+          qf[x][m][2] = to_f32(qh[1]) * a.qscale;
+          qf[x][m][3] = to_f32(qh[G::PPW + 1]) * a.qscale;
+        }
       if (window_owner)
         for (int i = tid; i < GQ * D; i += kW * 32) qs[i] = to_f32(qg[i]) * a.qscale;
 
-      float m_run[2] = {kNegInf, kNegInf}, l_part[2] = {0.f, 0.f};
-      float bv[GQ][NJ];  // sum_t p z per (head, value group), lane partial (token = lane)
+      float m_run[NPB], l_part[NPB];
       float acc[NPB][NM][4];
+      float bv[GQ][NJ];  // sum_t p z per (head, value group), lane partial (lane = token)
 #pragma unroll
-      for (int h = 0; h < GQ; ++h)
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) bv[h][j] = 0.f;
-#pragma unroll
-      for (int p = 0; p < NPB; ++p)
+      for (int p = 0; p < NPB; ++p) {
+        m_run[p] = kNegInf;
+        l_part[p] = 0.f;
 #pragma unroll
         for (int m = 0; m < NM; ++m)
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[p][m][e] = 0.f;
+      }
+#pragma unroll
+      for (int h = 0; h < GQ; ++h)
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) bv[h][j] = 0.f;
 
       for (long long t0 = t_beg; t0 < t_end; t0 += kStage, ++st) {
         const int s = (int)(st % G::NSTAGE);
@@ -357,38 +430,69 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
           const float* vs = reinterpret_cast<const float*>(buf + G::O_VS) + warp * kTile * NJ;
           const float* vz = reinterpret_cast<const float*>(buf + G::O_VZ) + warp * kTile * NJ;
 
-          // -- q' = q * s (this key group): hi/lo fp16 in B-fragment order; bias = q . z
-          float bk[GQ];
+          // -- q' = q s 2^(SK - e) (hi, lo) into the B fragments; bias = q . z
+          float bk[HX];
 #pragma unroll
-          for (int h = 0; h < GQ; ++h) bk[h] = 0.f;
+          for (int x = 0; x < HX; ++x) bk[x] = 0.f;
 #pragma unroll
-          for (int i = 0; i < NJ; ++i) {
-            const int ch = lane + 32 * i;
-            const float sv = ks[ch], zv = kz[ch];
-            int t4, kp, hf;
-            slot_of<BITS>(ch & 15, t4, kp, hf);
-            const int sl = ch >> 4;
+          for (int m = 0; m < MC; ++m) {
+            if (!cp_ok[m]) continue;
+            const float2 sA = *reinterpret_cast<const float2*>(ks + cp_ch[m]);
+            const float2 sB = *reinterpret_cast<const float2*>(ks + cp_ch[m] + G::PPW);
+            const float2 zA = *reinterpret_cast<const float2*>(kz + cp_ch[m]);
+            const float2 zB = *reinterpret_cast<const float2*>(kz + cp_ch[m] + G::PPW);
+            const float s0 = sA.x * cp_f0[m], s1 = sB.x * cp_f0[m];
+            const float s2 = sA.y * cp_f1[m], s3 = sB.y * cp_f1[m];
 #pragma unroll
-            for (int h = 0; h < GQ; ++h) {
-              bk[h] = fmaf(qv[h][i], zv, bk[h]);
-              __half hi, lo;
-              split_f16(qv[h][i] * sv, hi, lo);
-              const int ih = ((sl * 32 + col_of<GQ>(h, 0) * 4 + t4) * 2 + kp) * 2 + hf;
-              const int il = ((sl * 32 + col_of<GQ>(h, 1) * 4 + t4) * 2 + kp) * 2 + hf;
-              qBh[ih] = hi;
-              qBh[il + (NPB == 2 ? KSL * 32 * 4 : 0)] = lo;
+            for (int x = 0; x < HX; ++x) {
+              const int h = hc + GL * x;
+              uint2 hi, lo;
+              split2(qf[x][m][0] * s0, qf[x][m][1] * s1, hi.x, lo.x);
+              split2(qf[x][m][2] * s2, qf[x][m][3] * s3, hi.y, lo.y);
+              uint32_t* blk = qB + (h >> 2) * KSL * 64 + cp_w[m];
+              const int nh = 2 * (h & 3);
+              *reinterpret_cast<uint2*>(blk + 8 * (nh ^ cp_s3[m])) = hi;
+              *reinterpret_cast<uint2*>(blk + 8 * ((nh + 1) ^ cp_s3[m])) = lo;
+              float t = bk[x];
+              t = fmaf(qf[x][m][0], zA.x, t);
+              t = fmaf(qf[x][m][1], zB.x, t);
+              t = fmaf(qf[x][m][2], zA.y, t);
+              t = fmaf(qf[x][m][3], zB.y, t);
+              bk[x] = t;
             }
           }
-          float bkA = 0.f, bkB = 0.f;
+          // sum over the lanes of a head class; lane tq then holds head tq + 4p
 #pragma unroll
-          for (int h = 0; h < GQ; ++h) {
-            bk[h] = warp_sum(bk[h]);
-            if (h == hA) bkA = bk[h];
-            if (h == hB) bkB = bk[h];
-          }
+          for (int x = 0; x < HX; ++x)
+#pragma unroll
+            for (int o = GL; o < 32; o <<= 1) bk[x] += __shfl_xor_sync(0xffffffffu, bk[x], o);
           __syncwarp();
 
           // -- scores: 2 m-tiles of 16 tokens (rows g, g+8), KSL k-slices
+          uint32_t kw[2][2][G::NWL];
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const uint32_t* row = kc + (16 * mt + 8 * r + g) * WK + (G::WHOLE ? tq * G::NWL : (tq >> 1));
+              if constexpr (G::NWL == 4) {
+                const uint4 v = *reinterpret_cast<const uint4*>(row);
+                kw[mt][r][0] = v.x; kw[mt][r][1] = v.y; kw[mt][r][2] = v.z; kw[mt][r][3] = v.w;
+              } else if constexpr (G::NWL == 2) {
+                const uint2 v = *reinterpret_cast<const uint2*>(row);
+                kw[mt][r][0] = v.x; kw[mt][r][1] = v.y;
+              } else {
+                kw[mt][r][0] = row[0];
+              }
+            }
+          auto key_reg = [&](const uint32_t (&w)[G::NWL], int jj) -> uint32_t {
+            if constexpr (G::WHOLE) {
+              const int i = jj % G::PPW;
+              return (w[jj / G::PPW] >> PR::shift(i)) & PR::mask(i);
+            } else {
+              return (w[0] >> kS[jj & 3]) & kM[jj & 3];
+            }
+          };
           float dq[NPB][2][4];
 #pragma unroll
           for (int p = 0; p < NPB; ++p)
@@ -397,148 +501,130 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
 #pragma unroll
               for (int e = 0; e < 4; ++e) dq[p][mt][e] = 0.f;
 #pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            const uint32_t* r0 = kc + (16 * mt + g) * WK;
-            const uint32_t* r1 = kc + (16 * mt + g + 8) * WK;
-            uint32_t w0[WK], w1[WK];
+          for (int sl = 0; sl < KSL; ++sl) {
+            uint2 bq[NPB];
 #pragma unroll
-            for (int w = 0; w < WK; w += 2) {
-              const uint2 x0 = *reinterpret_cast<const uint2*>(r0 + w);
-              const uint2 x1 = *reinterpret_cast<const uint2*>(r1 + w);
-              w0[w] = x0.x;
-              w0[w + 1] = x0.y;
-              w1[w] = x1.x;
-              w1[w + 1] = x1.y;
-            }
+            for (int p = 0; p < NPB; ++p)
+              bq[p] = *reinterpret_cast<const uint2*>(qB + (p * KSL + sl) * 64 + frag_word(lane, sl));
 #pragma unroll
-            for (int sl = 0; sl < KSL; ++sl) {
-              uint32_t a0, a1, a2, a3;
-              if (BITS == 2) {
-                codes_pair<2>(w0[sl], 0u, tq, a0, a2);
-                codes_pair<2>(w1[sl], 0u, tq, a1, a3);
-              } else {
-                codes_pair<4>(w0[2 * sl], w0[2 * sl + 1], tq, a0, a2);
-                codes_pair<4>(w1[2 * sl], w1[2 * sl + 1], tq, a1, a3);
-              }
+            for (int mt = 0; mt < 2; ++mt) {
+              const uint32_t a0 = key_reg(kw[mt][0], 2 * sl), a2 = key_reg(kw[mt][0], 2 * sl + 1);
+              const uint32_t a1 = key_reg(kw[mt][1], 2 * sl), a3 = key_reg(kw[mt][1], 2 * sl + 1);
 #pragma unroll
-              for (int p = 0; p < NPB; ++p) {
-                const uint2 bb =
-                    *reinterpret_cast<const uint2*>(qB + p * KSL * 32 * 2 + (sl * 32 + lane) * 2);
-                mma16816(dq[p][mt], a0, a1, a2, a3, bb.x, bb.y);
-              }
+              for (int p = 0; p < NPB; ++p) mma16816(dq[p][mt], a0, a1, a2, a3, bq[p].x, bq[p].y);
             }
           }
 
-          // -- hi + lo, bias: lane holds heads hA (col 2tq) and hB (col 2tq+1)
-          // for tokens 16mt + g (e = 0,1) and 16mt + g + 8 (e = 2,3)
-          float sc[2][4];
+          // -- scores of head tq + 4p for tokens g, g+8, 16+g, 24+g
+          float sc[NPB][4];
 #pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
+          for (int p = 0; p < NPB; ++p) {
+            const float bias = bk[HX > 1 ? p : 0];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float v = dq[0][mt][e];
-              if (NPB == 2) v += dq[NPB - 1][mt][e];
-              else v += __shfl_xor_sync(0xffffffffu, v, 2);
-              const int hh = e & 1, ti = mt * 2 + (e >> 1);
-              sc[hh][ti] = fmaf(v, kCodeScale, hh ? bkB : bkA);
+            for (int mt = 0; mt < 2; ++mt) {
+              sc[p][2 * mt] = fmaf(dq[p][mt][0] + dq[p][mt][1], kKeyOut, bias);
+              sc[p][2 * mt + 1] = fmaf(dq[p][mt][2] + dq[p][mt][3], kKeyOut, bias);
             }
-          // -- online softmax per head over the tile's 32 tokens (8 lanes x 4)
-          float alpha[2], p[2][4];
+          }
+          // -- online softmax: the running max moves only when a score exceeds it
+          float lm[NPB];
+          bool need = false;
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            float tm = fmaxf(fmaxf(sc[hh][0], sc[hh][1]), fmaxf(sc[hh][2], sc[hh][3]));
-            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
-            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
-            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
-            const float mn = fmaxf(m_run[hh], tm);
-            alpha[hh] = exp2f(m_run[hh] - mn);
+          for (int p = 0; p < NPB; ++p) {
+            lm[p] = fmaxf(fmaxf(sc[p][0], sc[p][1]), fmaxf(sc[p][2], sc[p][3]));
+            need |= vh[p] && lm[p] > m_run[p];
+          }
+          if (__any_sync(0xffffffffu, need)) {
+            float al[NPB];
+#pragma unroll
+            for (int p = 0; p < NPB; ++p) {
+              float tm = lm[p];
+              tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
+              tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
+              tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
+              const float mn = fmaxf(m_run[p], tm);
+              al[p] = exp2f(m_run[p] - mn);
+              m_run[p] = mn;
+              l_part[p] *= al[p];
+#pragma unroll
+              for (int m = 0; m < NM; ++m)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[p][m][e] *= al[p];
+            }
+#pragma unroll
+            for (int h = 0; h < GQ; ++h) {
+              const float ah = __shfl_sync(0xffffffffu, al[h >> 2], h & 3);
+#pragma unroll
+              for (int j = 0; j < NJ; ++j) bv[h][j] *= ah;
+            }
+          }
+#pragma unroll
+          for (int p = 0; p < NPB; ++p) {
             float ps = 0.f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              p[hh][i] = exp2f(sc[hh][i] - mn);
-              ps += p[hh][i];
+              const float pv = exp2f(sc[p][i] - m_run[p]);
+              ps += pv;
+              if (vh[p]) pbuf[(tq + 4 * p) * PST + 16 * (i >> 1) + 8 * (i & 1) + g] = pv;
             }
-            l_part[hh] = fmaf(l_part[hh], alpha[hh], ps);
-            m_run[hh] = mn;
+            l_part[p] += ps;
           }
-          if (owner) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int tok = 16 * (i >> 1) + g + 8 * (i & 1);
-              if (vA) pbuf[hA * kTile + tok] = p[0][i];
-              if (vB) pbuf[hB * kTile + tok] = p[1][i];
-            }
-          }
-          // rescale the P.V accumulators only if a running max moved
-          if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-#pragma unroll
-            for (int q2 = 0; q2 < NPB; ++q2)
-#pragma unroll
-              for (int m = 0; m < NM; ++m) {
-                acc[q2][m][0] *= alpha[0];
-                acc[q2][m][1] *= alpha[1];
-                acc[q2][m][2] *= alpha[0];
-                acc[q2][m][3] *= alpha[1];
-              }
-          }
-          // per-head alpha for the lane-partial value bias (heads live in lanes 0..3)
-          float al[GQ];
-#pragma unroll
-          for (int h = 0; h < GQ; ++h)
-            al[h] = __shfl_sync(0xffffffffu, (h & 1) ? alpha[1] : alpha[0], h >> 1);
           __syncwarp();
 
-          // -- p' = p * s_v (hi/lo, B-fragment order); bias_v += p * z_v
+          // -- p' = p s_v 2^(SV - e) (hi, lo) into the B fragments; bias_v += p z_v
           {
-            const int t = lane;
-            int t4, kp, hf;
-            slot_of<BITS>(t & 15, t4, kp, hf);
-            const int Hs = t >> 4;
+            float sv[NJ], zv[NJ];
+            if constexpr (NJ == 4) {
+              const float4 s4 = *reinterpret_cast<const float4*>(vs + lane * NJ);
+              const float4 z4 = *reinterpret_cast<const float4*>(vz + lane * NJ);
+              sv[0] = s4.x; sv[1] = s4.y; sv[2] = s4.z; sv[3] = s4.w;
+              zv[0] = z4.x; zv[1] = z4.y; zv[2] = z4.z; zv[3] = z4.w;
+            } else {
 #pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-              const float sv = vs[t * NJ + j], zv = vz[t * NJ + j];
+              for (int j = 0; j < NJ; ++j) {
+                sv[j] = vs[lane * NJ + j];
+                zv[j] = vz[lane * NJ + j];
+              }
+            }
 #pragma unroll
-              for (int h = 0; h < GQ; ++h) {
-                const float ph = pbuf[h * kTile + t];
-                bv[h][j] = fmaf(ph, zv, bv[h][j] * al[h]);
-                __half hi, lo;
-                split_f16(ph * sv, hi, lo);
-                const int ih = (((j * 2 + Hs) * 32 + col_of<GQ>(h, 0) * 4 + t4) * 2 + kp) * 2 + hf;
-                const int il = (((j * 2 + Hs) * 32 + col_of<GQ>(h, 1) * 4 + t4) * 2 + kp) * 2 + hf;
-                pBh[ih] = hi;
-                pBh[il + (NPB == 2 ? NJ * 2 * 32 * 4 : 0)] = lo;
+            for (int h = 0; h < GQ; ++h) {
+              const float ph = pbuf[h * PST + lane];
+              const float phf = ph * pt_f;
+              const int nh = 2 * (h & 3);
+              const int o_hi = pt_base + 4 * (4 * (nh ^ pt_s3) + pt_tq);
+              const int o_lo = pt_base + 4 * (4 * ((nh + 1) ^ pt_s3) + pt_tq);
+#pragma unroll
+              for (int j = 0; j < NJ; ++j) {
+                bv[h][j] = fmaf(ph, zv[j], bv[h][j]);
+                const float x = phf * sv[j];
+                const __half hi = __float2half_rn(x);
+                const __half lo = __float2half_rn(x - __half2float(hi));
+                __half* blk = pBh + ((h >> 2) * NJ + j) * NSL * 128;
+                blk[o_hi] = hi;
+                blk[o_lo] = lo;
               }
             }
           }
           __syncwarp();
 
-          // -- P.V: per value group j, m-tiles 2j (channels 32j+4g, +1) and 2j+1 (+2, +3)
+          // -- P.V: per value group j and k-slice sl, m-tiles 2j (channels
+          // 32j+4g, +1) and 2j+1 (+2, +3)
 #pragma unroll
           for (int j = 0; j < NJ; ++j) {
 #pragma unroll
-            for (int Hs = 0; Hs < 2; ++Hs) {
-              uint32_t A0[4], A1[4];
-              if (BITS == 2) {
-                const uint4 w = *reinterpret_cast<const uint4*>(vc + Hs * D + 32 * j + 4 * g);
-                codes_pair<2>(w.x, 0u, tq, A0[0], A0[2]);
-                codes_pair<2>(w.y, 0u, tq, A0[1], A0[3]);
-                codes_pair<2>(w.z, 0u, tq, A1[0], A1[2]);
-                codes_pair<2>(w.w, 0u, tq, A1[1], A1[3]);
-              } else {
-                const uint4 x0 = *reinterpret_cast<const uint4*>(vc + (2 * Hs) * D + 32 * j + 4 * g);
-                const uint4 x1 =
-                    *reinterpret_cast<const uint4*>(vc + (2 * Hs + 1) * D + 32 * j + 4 * g);
-                codes_pair<4>(x0.x, x1.x, tq, A0[0], A0[2]);
-                codes_pair<4>(x0.y, x1.y, tq, A0[1], A0[3]);
-                codes_pair<4>(x0.z, x1.z, tq, A1[0], A1[2]);
-                codes_pair<4>(x0.w, x1.w, tq, A1[1], A1[3]);
-              }
+            for (int sl = 0; sl < NSL; ++sl) {
+              const int tw = BITS == 2 ? sl : 2 * sl + vtw;
+              const uint4 w = *reinterpret_cast<const uint4*>(vc + tw * D + 32 * j + 4 * g);
+              const uint32_t x0 = w.x & vM, x2 = (w.x >> 8) & vM;
+              const uint32_t x1 = w.y & vM, x3 = (w.y >> 8) & vM;
+              const uint32_t y0 = w.z & vM, y2 = (w.z >> 8) & vM;
+              const uint32_t y1 = w.w & vM, y3 = (w.w >> 8) & vM;
 #pragma unroll
-              for (int q2 = 0; q2 < NPB; ++q2) {
+              for (int p = 0; p < NPB; ++p) {
                 const uint2 bb = *reinterpret_cast<const uint2*>(
-                    pB + q2 * (NJ * 2 * 32 * 2) + ((j * 2 + Hs) * 32 + lane) * 2);
-                mma16816(acc[q2][2 * j], A0[0], A0[1], A0[2], A0[3], bb.x, bb.y);
-                mma16816(acc[q2][2 * j + 1], A1[0], A1[1], A1[2], A1[3], bb.x, bb.y);
+                    pB + ((p * NJ + j) * NSL + sl) * 64 + frag_word(lane, sl));
+                mma16816(acc[p][2 * j], x0, x1, x2, x3, bb.x, bb.y);
+                mma16816(acc[p][2 * j + 1], y0, y1, y2, y3, bb.x, bb.y);
               }
             }
           }
@@ -550,58 +636,42 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
 
       // ---- this warp's streamed state -> mg slot `warp`
       {
-        float lt[2];
+        float lt[NPB];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float v = l_part[hh];
+        for (int p = 0; p < NPB; ++p) {
+          float v = l_part[p];
           v += __shfl_xor_sync(0xffffffffu, v, 4);
           v += __shfl_xor_sync(0xffffffffu, v, 8);
           v += __shfl_xor_sync(0xffffffffu, v, 16);
-          lt[hh] = v;
+          lt[p] = v;
         }
 #pragma unroll
         for (int h = 0; h < GQ; ++h)
 #pragma unroll
           for (int j = 0; j < NJ; ++j) bv[h][j] = warp_sum(bv[h][j]);
-        if (g == 0 && owner) {
-          if (vA) {
-            mg_m[warp * GQ + hA] = m_run[0];
-            mg_l[warp * GQ + hA] = lt[0];
+#pragma unroll
+        for (int p = 0; p < NPB; ++p) {
+          if (!vh[p]) continue;
+          const int h = tq + 4 * p;
+          if (g == 0) {
+            mg_m[warp * GQ + h] = m_run[p];
+            mg_l[warp * GQ + h] = lt[p];
           }
-          if (vB) {
-            mg_m[warp * GQ + hB] = m_run[1];
-            mg_l[warp * GQ + hB] = lt[1];
-          }
-        }
 #pragma unroll
-        for (int m = 0; m < NM; ++m) {
-          const int j = m >> 1, mm = m & 1;
-          const int ch0 = 32 * j + 4 * g + 2 * mm;
-          float v[4];
+          for (int m = 0; m < NM; ++m) {
+            const int j = m >> 1;
+            const int ch = 32 * j + 4 * g + 2 * (m & 1);
+            float bias = 0.f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            v[e] = acc[0][m][e];
-            if (NPB == 2) v[e] += acc[NPB - 1][m][e];
-            else v[e] += __shfl_xor_sync(0xffffffffu, v[e], 2);
-          }
-          if (owner) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int h = (e & 1) ? hB : hA;
-              const int ch = ch0 + (e >> 1);
-              if (h < GQ) {
-                float bias = 0.f;
-#pragma unroll
-                for (int hh = 0; hh < GQ; ++hh)
-                  if (hh == h) bias = bv[hh][j];
-                mg_acc[(warp * GQ + h) * D + ch] = fmaf(v[e], kCodeScale, bias);
-              }
-            }
+            for (int hh = 0; hh < GQ; ++hh)
+              if (hh == h) bias = bv[hh][j];
+            float* dst = mg_acc + (warp * GQ + h) * D + ch;
+            dst[0] = fmaf(acc[p][m][0] + acc[p][m][1], kValOut, bias);
+            dst[1] = fmaf(acc[p][m][2] + acc[p][m][3], kValOut, bias);
           }
         }
       }
       __syncwarp();
-
       // ---- residual window (CTA that ends the unit): warp w takes window
       // tiles w, w+4, ... on CUDA cores, folded into its mg slot
       if (window_owner && !failed) {
