@@ -99,13 +99,18 @@ void plan_splits(const kivi_cache* c, int sms, int* n_split, int* tiles_per_spli
 
 // Tensor-core kernel: persistent stream-K plan.  Every unit is laid out as
 // n_q/32 work indices (its quantized 32-token tiles) followed by
-// kWinWeight * ceil(r/32) indices standing for its residual window; the
-// units' indices end to end are cut into n_cta equal ranges of W >= 4.  A
-// unit is covered by the CTAs whose ranges meet its tiles or its window start
-// index -- at most ceil((n_q/32 + 1) / W) + 1 CTA segments, each writing one
-// partial -- and the last of them also takes the window.
+// kWinWeight * ceil(r/32) + kMergeWeight indices standing for its residual
+// window and for the end-of-unit merge; the units' indices end to end are
+// cut into n_cta equal ranges of W >= 12.  A unit is covered by the CTAs
+// whose ranges meet its tiles or its window start index -- at most
+// ceil((n_q/32 + 1) / W) + 1 CTA segments, each writing one partial -- and
+// the last of them also takes the window.  Measured on B200 (per-CTA
+// timelines): a 32-token window tile costs about three quantized tiles and
+// the end of a unit segment (partial write, arrival, merge) about eight, so
+// a CTA whose range crosses a unit boundary gets correspondingly fewer tiles.
 constexpr int kTcCtasPerSm = 3;  // upper bound; the kernel instance decides
-constexpr int kWinWeight = 3;  // cost of a window tile, in quantized tiles
+constexpr int kWinWeight = 3;    // cost of a window tile, in quantized tiles
+constexpr int kMergeWeight = 8;  // cost of a unit end, in quantized tiles
 
 struct StreamPlan {
   int n_cta;
@@ -130,7 +135,7 @@ int tc_seg_cap(const kivi_dims& d, int sms) {
 void plan_stream(const kivi_cache* c, int sms, int ctas_per_sm, int seg_cap, StreamPlan* p) {
   const long long units = (long long)c->dims.B * c->dims.Hkv;
   const long long n_qt = c->n_q / kivi::kTile;
-  const int ww = c->r > 0 ? kWinWeight * (int)ceil_div(c->r, kivi::kTile) : 1;
+  const int ww = (c->r > 0 ? kWinWeight * (int)ceil_div(c->r, kivi::kTile) : 1) + kMergeWeight;
   const long long UP = n_qt + ww;
   const long long total = units * UP;
   const long long P =

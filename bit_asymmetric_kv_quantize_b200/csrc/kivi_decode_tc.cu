@@ -47,6 +47,7 @@ namespace {
 
 constexpr float kNegInf = -__builtin_huge_valf();
 constexpr long long kWaitCycles = 1LL << 32;  // ~2 s: bounded wait on our own copies
+constexpr int kSuspendNs = 1000;  // a waiting thread sleeps up to this long per try
 
 // Code pairs of one 32-bit word.  2-bit: pair i (i < 8) = codes i and i + 8;
 // 4-bit: pair i (i < 4) = codes i and i + 4.  (w >> shift(i)) & mask(i) puts
@@ -70,15 +71,17 @@ struct Pairs<4> {
   __host__ __device__ static constexpr uint32_t mask(int i) { return 0x000F000Fu << e(i); }
 };
 
-// NW consumer warps (one 32-token tile each per stage) and one producer warp
-// per CTA.  Measured on B200: one query head per KV head runs best as three
-// 4-warp CTAs per SM; grouped heads run best as one CTA per SM with 11
-// (GQ 2, 4) or 7 (GQ 8) consumer warps sharing one ring.
+// NW consumer warps (TPW 32-token tiles each per stage) and one producer
+// warp per CTA.  Measured on B200: one query head per KV head runs best as
+// 4-warp CTAs, two tiles per warp at 2-bit (two CTAs per SM) and one at 4-bit
+// (three per SM); grouped heads run best as one CTA per SM with 11 (GQ 2, 4)
+// or 7 (GQ 8) consumer warps sharing one ring.
 template <int D, int BITS, int GQ>
 struct Geo {
   static constexpr int NW = GQ == 1 ? 4 : (GQ == 8 ? 7 : 11);
+  static constexpr int TPW = (GQ == 1 && BITS == 2) ? 2 : 1;  // tiles per warp and stage
   static constexpr int THREADS = (NW + 1) * 32;
-  static constexpr int kStage = NW;             // tiles per pipeline stage
+  static constexpr int kStage = NW * TPW;       // tiles per pipeline stage
   static constexpr int E = 32 / BITS;
   static constexpr int WK = D / E;       // key words per token
   static constexpr int NJ = D / kGv;     // value groups per token
@@ -96,14 +99,14 @@ struct Geo {
   static constexpr int O_VS = O_VC + kStage * VC_B;
   static constexpr int O_VZ = O_VS + kStage * VM_B;
   static constexpr int STAGE_B = O_VZ + kStage * VM_B;
-  static constexpr int NSTAGE = NW == 4 ? (BITS == 2 ? 3 : 2) : 2;
+  static constexpr int NSTAGE = (NW == 4 && TPW == 1 && BITS == 2) ? 3 : 2;
   static constexpr int NPB = GQ == 8 ? 2 : 1;  // n-tiles of 8 columns (4 heads x hi, lo)
-  static constexpr int PST = kTile + 8;        // p buffer stride per head (floats)
+  static constexpr int PST = TPW * kTile + 8;  // p buffer stride per head (floats)
   // per-warp scratch (bytes): fragment blocks of 32 lanes x 2 words
   static constexpr int QB_B = NPB * KSL * 256;        // q' B fragments (score product)
   static constexpr int PB_B = NPB * NJ * NSL * 256;   // p' B fragments (value product)
   static constexpr int PBUF_B = GQ * PST * 4;         // p per head and token
-  static constexpr int WARP_B = QB_B + PB_B + PBUF_B;
+  static constexpr int WARP_B = TPW * (QB_B + PB_B) + PBUF_B;
   // whole CTA
   static constexpr int O_WARP = NSTAGE * STAGE_B;
   static constexpr int O_QS = O_WARP + NW * WARP_B;    // q (fp32, scaled) for the window path
@@ -113,7 +116,7 @@ struct Geo {
   static constexpr int SMEM_B = O_FLAG + 16;
   static_assert(SMEM_B <= 227 * 1024, "shared memory per CTA");
   static_assert(O_BAR % 8 == 0 && WARP_B % 16 == 0, "alignment");
-  static constexpr int MIN_CTAS = NW == 4 ? 3 : 1;
+  static constexpr int MIN_CTAS = NW == 4 ? (TPW == 2 ? 2 : 3) : 1;
   // key operand: code pairs per lane and row, words a lane loads per row
   static constexpr int PPL = D / 8;
   static constexpr int PPW = Pairs<BITS>::PPW;
@@ -150,9 +153,9 @@ __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t b
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -210,6 +213,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
   constexpr int NM = D / 16;  // value m-tiles (16 channels each)
   constexpr int NPB = G::NPB;
   constexpr int PST = G::PST;
+  constexpr int TPW = G::TPW;
   constexpr int CPL = D / 32;  // window path: channels per lane
   constexpr float kKeyOut = (float)(1 << (24 - G::SK));
   constexpr float kValOut = (float)(1 << (24 - G::SV));
@@ -247,7 +251,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
   if (warp < kW) {
     // fragment columns of absent heads stay zero
     unsigned char* wb = smem + G::O_WARP + warp * G::WARP_B;
-    for (int i = lane; i < (G::QB_B + G::PB_B) / 4; i += 32) reinterpret_cast<uint32_t*>(wb)[i] = 0u;
+    for (int i = lane; i < TPW * (G::QB_B + G::PB_B) / 4; i += 32) reinterpret_cast<uint32_t*>(wb)[i] = 0u;
   }
   __syncthreads();
 
@@ -300,10 +304,10 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
   } else {
     // ---------------- consumer warps
     unsigned char* wb = smem + G::O_WARP + warp * G::WARP_B;
-    uint32_t* qB = reinterpret_cast<uint32_t*>(wb);                 // [NPB][KSL][64]
-    uint32_t* pB = reinterpret_cast<uint32_t*>(wb + G::QB_B);       // [NPB][NJ][NSL][64]
+    uint32_t* qB = reinterpret_cast<uint32_t*>(wb);                     // [TPW][NPB][KSL][64]
+    uint32_t* pB = reinterpret_cast<uint32_t*>(wb + TPW * G::QB_B);     // [TPW][NPB][NJ][NSL][64]
     __half* pBh = reinterpret_cast<__half*>(pB);
-    float* pbuf = reinterpret_cast<float*>(wb + G::QB_B + G::PB_B);  // [GQ][PST]
+    float* pbuf = reinterpret_cast<float*>(wb + TPW * (G::QB_B + G::PB_B));  // [GQ][PST]
 
     // -- q' build: lane classes.  Head class hc = lane % GL builds heads
     // hc + GL x; within a class, lane index jl = lane / GL takes the
@@ -359,6 +363,9 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
     const int pt_base = pt_sl * 128 + 2 * pt_kp + pt_hf;  // halves, block (0, 0, pt_sl)
     const int pt_s3 = pt_sl & 3;
 
+    // B-fragment column n = g of this lane carries a head (hi or lo part);
+    // lanes of absent heads' columns use zeros without loading them
+    const bool bcol = GQ >= 4 || g < 2 * GQ;
     bool vh[NPB];  // this lane's score / accumulator head tq + 4p exists
 #pragma unroll
     for (int p = 0; p < NPB; ++p) vh[p] = tq + 4 * p < GQ;
@@ -421,70 +428,96 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
           break;
         }
         const unsigned char* buf = smem + s * G::STAGE_B;
-        if (t0 + warp < t_end) {
-          const uint32_t* kc = reinterpret_cast<const uint32_t*>(buf + G::O_KC) + warp * kTile * WK;
-          const float* ks = reinterpret_cast<const float*>(buf + G::O_KS) + warp * D;
-          const float* kz = reinterpret_cast<const float*>(buf + G::O_KZ) + warp * D;
-          const uint32_t* vc =
-              reinterpret_cast<const uint32_t*>(buf + G::O_VC) + warp * (kTile / E) * D;
-          const float* vs = reinterpret_cast<const float*>(buf + G::O_VS) + warp * kTile * NJ;
-          const float* vz = reinterpret_cast<const float*>(buf + G::O_VZ) + warp * kTile * NJ;
+        const long long tw0 = t0 + (long long)warp * TPW;  // this warp's first tile
+        if (tw0 < t_end) {
+          // this warp's TPW tiles; a tile past the end of the segment reuses
+          // tile 0's data and is masked out (its scores are -inf, so p = 0)
+          bool tv[TPW];
+          const uint32_t* kc[TPW];
+          const float* ks[TPW];
+          const float* kz[TPW];
+          const uint32_t* vc[TPW];
+          const float* vs[TPW];
+          const float* vz[TPW];
+#pragma unroll
+          for (int tt = 0; tt < TPW; ++tt) {
+            tv[tt] = tw0 + tt < t_end;
+            const int ti = warp * TPW + (tv[tt] ? tt : 0);
+            kc[tt] = reinterpret_cast<const uint32_t*>(buf + G::O_KC) + ti * kTile * WK;
+            ks[tt] = reinterpret_cast<const float*>(buf + G::O_KS) + ti * D;
+            kz[tt] = reinterpret_cast<const float*>(buf + G::O_KZ) + ti * D;
+            vc[tt] = reinterpret_cast<const uint32_t*>(buf + G::O_VC) + ti * (kTile / E) * D;
+            vs[tt] = reinterpret_cast<const float*>(buf + G::O_VS) + ti * kTile * NJ;
+            vz[tt] = reinterpret_cast<const float*>(buf + G::O_VZ) + ti * kTile * NJ;
+          }
 
           // -- q' = q s 2^(SK - e) (hi, lo) into the B fragments; bias = q . z
-          float bk[HX];
+          float bk[TPW][HX];
 #pragma unroll
-          for (int x = 0; x < HX; ++x) bk[x] = 0.f;
+          for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+            for (int x = 0; x < HX; ++x) bk[tt][x] = 0.f;
 #pragma unroll
           for (int m = 0; m < MC; ++m) {
             if (!cp_ok[m]) continue;
-            const float2 sA = *reinterpret_cast<const float2*>(ks + cp_ch[m]);
-            const float2 sB = *reinterpret_cast<const float2*>(ks + cp_ch[m] + G::PPW);
-            const float2 zA = *reinterpret_cast<const float2*>(kz + cp_ch[m]);
-            const float2 zB = *reinterpret_cast<const float2*>(kz + cp_ch[m] + G::PPW);
-            const float s0 = sA.x * cp_f0[m], s1 = sB.x * cp_f0[m];
-            const float s2 = sA.y * cp_f1[m], s3 = sB.y * cp_f1[m];
 #pragma unroll
-            for (int x = 0; x < HX; ++x) {
-              const int h = hc + GL * x;
-              uint2 hi, lo;
-              split2(qf[x][m][0] * s0, qf[x][m][1] * s1, hi.x, lo.x);
-              split2(qf[x][m][2] * s2, qf[x][m][3] * s3, hi.y, lo.y);
-              uint32_t* blk = qB + (h >> 2) * KSL * 64 + cp_w[m];
-              const int nh = 2 * (h & 3);
-              *reinterpret_cast<uint2*>(blk + 8 * (nh ^ cp_s3[m])) = hi;
-              *reinterpret_cast<uint2*>(blk + 8 * ((nh + 1) ^ cp_s3[m])) = lo;
-              float t = bk[x];
-              t = fmaf(qf[x][m][0], zA.x, t);
-              t = fmaf(qf[x][m][1], zB.x, t);
-              t = fmaf(qf[x][m][2], zA.y, t);
-              t = fmaf(qf[x][m][3], zB.y, t);
-              bk[x] = t;
+            for (int tt = 0; tt < TPW; ++tt) {
+              const float2 sA = *reinterpret_cast<const float2*>(ks[tt] + cp_ch[m]);
+              const float2 sB = *reinterpret_cast<const float2*>(ks[tt] + cp_ch[m] + G::PPW);
+              const float2 zA = *reinterpret_cast<const float2*>(kz[tt] + cp_ch[m]);
+              const float2 zB = *reinterpret_cast<const float2*>(kz[tt] + cp_ch[m] + G::PPW);
+              const float s0 = sA.x * cp_f0[m], s1 = sB.x * cp_f0[m];
+              const float s2 = sA.y * cp_f1[m], s3 = sB.y * cp_f1[m];
+#pragma unroll
+              for (int x = 0; x < HX; ++x) {
+                const int h = hc + GL * x;
+                uint2 hi, lo;
+                split2(qf[x][m][0] * s0, qf[x][m][1] * s1, hi.x, lo.x);
+                split2(qf[x][m][2] * s2, qf[x][m][3] * s3, hi.y, lo.y);
+                uint32_t* blk = qB + tt * (G::QB_B / 4) + (h >> 2) * KSL * 64 + cp_w[m];
+                const int nh = 2 * (h & 3);
+                *reinterpret_cast<uint2*>(blk + 8 * (nh ^ cp_s3[m])) = hi;
+                *reinterpret_cast<uint2*>(blk + 8 * ((nh + 1) ^ cp_s3[m])) = lo;
+                float t = bk[tt][x];
+                t = fmaf(qf[x][m][0], zA.x, t);
+                t = fmaf(qf[x][m][1], zB.x, t);
+                t = fmaf(qf[x][m][2], zA.y, t);
+                t = fmaf(qf[x][m][3], zB.y, t);
+                bk[tt][x] = t;
+              }
             }
           }
           // sum over the lanes of a head class; lane tq then holds head tq + 4p
 #pragma unroll
-          for (int x = 0; x < HX; ++x)
+          for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
-            for (int o = GL; o < 32; o <<= 1) bk[x] += __shfl_xor_sync(0xffffffffu, bk[x], o);
+            for (int x = 0; x < HX; ++x)
+#pragma unroll
+              for (int o = GL; o < 32; o <<= 1)
+                bk[tt][x] += __shfl_xor_sync(0xffffffffu, bk[tt][x], o);
           __syncwarp();
 
-          // -- scores: 2 m-tiles of 16 tokens (rows g, g+8), KSL k-slices
-          uint32_t kw[2][2][G::NWL];
+          // -- scores: per tile 2 m-tiles of 16 tokens (rows g, g+8), KSL k-slices
+          uint32_t kw[TPW][2][2][G::NWL];
 #pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
+          for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const uint32_t* row = kc + (16 * mt + 8 * r + g) * WK + (G::WHOLE ? tq * G::NWL : (tq >> 1));
-              if constexpr (G::NWL == 4) {
-                const uint4 v = *reinterpret_cast<const uint4*>(row);
-                kw[mt][r][0] = v.x; kw[mt][r][1] = v.y; kw[mt][r][2] = v.z; kw[mt][r][3] = v.w;
-              } else if constexpr (G::NWL == 2) {
-                const uint2 v = *reinterpret_cast<const uint2*>(row);
-                kw[mt][r][0] = v.x; kw[mt][r][1] = v.y;
-              } else {
-                kw[mt][r][0] = row[0];
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+              for (int r = 0; r < 2; ++r) {
+                const uint32_t* row = kc[tt] + (16 * mt + 8 * r + g) * WK +
+                                      (G::WHOLE ? tq * G::NWL : (tq >> 1));
+                if constexpr (G::NWL == 4) {
+                  const uint4 v = *reinterpret_cast<const uint4*>(row);
+                  kw[tt][mt][r][0] = v.x; kw[tt][mt][r][1] = v.y;
+                  kw[tt][mt][r][2] = v.z; kw[tt][mt][r][3] = v.w;
+                } else if constexpr (G::NWL == 2) {
+                  const uint2 v = *reinterpret_cast<const uint2*>(row);
+                  kw[tt][mt][r][0] = v.x; kw[tt][mt][r][1] = v.y;
+                } else {
+                  kw[tt][mt][r][0] = row[0];
+                }
               }
-            }
           auto key_reg = [&](const uint32_t (&w)[G::NWL], int jj) -> uint32_t {
             if constexpr (G::WHOLE) {
               const int i = jj % G::PPW;
@@ -493,46 +526,63 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
               return (w[0] >> kS[jj & 3]) & kM[jj & 3];
             }
           };
-          float dq[NPB][2][4];
+          float dq[TPW][NPB][2][4];
 #pragma unroll
-          for (int p = 0; p < NPB; ++p)
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) dq[p][mt][e] = 0.f;
-#pragma unroll
-          for (int sl = 0; sl < KSL; ++sl) {
-            uint2 bq[NPB];
+          for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
             for (int p = 0; p < NPB; ++p)
-              bq[p] = *reinterpret_cast<const uint2*>(qB + (p * KSL + sl) * 64 + frag_word(lane, sl));
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-              const uint32_t a0 = key_reg(kw[mt][0], 2 * sl), a2 = key_reg(kw[mt][0], 2 * sl + 1);
-              const uint32_t a1 = key_reg(kw[mt][1], 2 * sl), a3 = key_reg(kw[mt][1], 2 * sl + 1);
+              for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-              for (int p = 0; p < NPB; ++p) mma16816(dq[p][mt], a0, a1, a2, a3, bq[p].x, bq[p].y);
+                for (int e = 0; e < 4; ++e) dq[tt][p][mt][e] = 0.f;
+#pragma unroll
+          for (int sl = 0; sl < KSL; ++sl) {
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt) {
+              uint2 bq[NPB];
+#pragma unroll
+              for (int p = 0; p < NPB; ++p)
+                bq[p] = bcol ? *reinterpret_cast<const uint2*>(qB + tt * (G::QB_B / 4) +
+                                                               (p * KSL + sl) * 64 + frag_word(lane, sl))
+                             : make_uint2(0u, 0u);
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt) {
+                const uint32_t a0 = key_reg(kw[tt][mt][0], 2 * sl);
+                const uint32_t a2 = key_reg(kw[tt][mt][0], 2 * sl + 1);
+                const uint32_t a1 = key_reg(kw[tt][mt][1], 2 * sl);
+                const uint32_t a3 = key_reg(kw[tt][mt][1], 2 * sl + 1);
+#pragma unroll
+                for (int p = 0; p < NPB; ++p)
+                  mma16816(dq[tt][p][mt], a0, a1, a2, a3, bq[p].x, bq[p].y);
+              }
             }
           }
 
-          // -- scores of head tq + 4p for tokens g, g+8, 16+g, 24+g
-          float sc[NPB][4];
+          // -- scores of head tq + 4p for tokens 32 tt + {g, g+8, 16+g, 24+g}
+          float sc[NPB][4 * TPW];
 #pragma unroll
-          for (int p = 0; p < NPB; ++p) {
-            const float bias = bk[HX > 1 ? p : 0];
+          for (int p = 0; p < NPB; ++p)
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-              sc[p][2 * mt] = fmaf(dq[p][mt][0] + dq[p][mt][1], kKeyOut, bias);
-              sc[p][2 * mt + 1] = fmaf(dq[p][mt][2] + dq[p][mt][3], kKeyOut, bias);
+            for (int tt = 0; tt < TPW; ++tt) {
+              const float bias = bk[tt][HX > 1 ? p : 0];
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt) {
+                const float v0 = fmaf(dq[tt][p][mt][0] + dq[tt][p][mt][1], kKeyOut, bias);
+                const float v1 = fmaf(dq[tt][p][mt][2] + dq[tt][p][mt][3], kKeyOut, bias);
+                sc[p][4 * tt + 2 * mt] = tv[tt] ? v0 : kNegInf;
+                sc[p][4 * tt + 2 * mt + 1] = tv[tt] ? v1 : kNegInf;
+              }
             }
-          }
           // -- online softmax: the running max moves only when a score exceeds it
           float lm[NPB];
           bool need = false;
 #pragma unroll
           for (int p = 0; p < NPB; ++p) {
-            lm[p] = fmaxf(fmaxf(sc[p][0], sc[p][1]), fmaxf(sc[p][2], sc[p][3]));
-            need |= vh[p] && lm[p] > m_run[p];
+            float v = sc[p][0];
+#pragma unroll
+            for (int i = 1; i < 4 * TPW; ++i) v = fmaxf(v, sc[p][i]);
+            lm[p] = v;
+            need |= vh[p] && v > m_run[p];
           }
           if (__any_sync(0xffffffffu, need)) {
             float al[NPB];
@@ -562,33 +612,35 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
           for (int p = 0; p < NPB; ++p) {
             float ps = 0.f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 4 * TPW; ++i) {
               const float pv = exp2f(sc[p][i] - m_run[p]);
               ps += pv;
-              if (vh[p]) pbuf[(tq + 4 * p) * PST + 16 * (i >> 1) + 8 * (i & 1) + g] = pv;
+              const int tok = 32 * (i >> 2) + 16 * ((i >> 1) & 1) + 8 * (i & 1) + g;
+              if (vh[p]) pbuf[(tq + 4 * p) * PST + tok] = pv;
             }
             l_part[p] += ps;
           }
           __syncwarp();
 
           // -- p' = p s_v 2^(SV - e) (hi, lo) into the B fragments; bias_v += p z_v
-          {
+#pragma unroll
+          for (int tt = 0; tt < TPW; ++tt) {
             float sv[NJ], zv[NJ];
             if constexpr (NJ == 4) {
-              const float4 s4 = *reinterpret_cast<const float4*>(vs + lane * NJ);
-              const float4 z4 = *reinterpret_cast<const float4*>(vz + lane * NJ);
+              const float4 s4 = *reinterpret_cast<const float4*>(vs[tt] + lane * NJ);
+              const float4 z4 = *reinterpret_cast<const float4*>(vz[tt] + lane * NJ);
               sv[0] = s4.x; sv[1] = s4.y; sv[2] = s4.z; sv[3] = s4.w;
               zv[0] = z4.x; zv[1] = z4.y; zv[2] = z4.z; zv[3] = z4.w;
             } else {
 #pragma unroll
               for (int j = 0; j < NJ; ++j) {
-                sv[j] = vs[lane * NJ + j];
-                zv[j] = vz[lane * NJ + j];
+                sv[j] = vs[tt][lane * NJ + j];
+                zv[j] = vz[tt][lane * NJ + j];
               }
             }
 #pragma unroll
             for (int h = 0; h < GQ; ++h) {
-              const float ph = pbuf[h * PST + lane];
+              const float ph = pbuf[h * PST + 32 * tt + lane];
               const float phf = ph * pt_f;
               const int nh = 2 * (h & 3);
               const int o_hi = pt_base + 4 * (4 * (nh ^ pt_s3) + pt_tq);
@@ -599,7 +651,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
                 const float x = phf * sv[j];
                 const __half hi = __float2half_rn(x);
                 const __half lo = __float2half_rn(x - __half2float(hi));
-                __half* blk = pBh + ((h >> 2) * NJ + j) * NSL * 128;
+                __half* blk = pBh + tt * (G::PB_B / 2) + ((h >> 2) * NJ + j) * NSL * 128;
                 blk[o_hi] = hi;
                 blk[o_lo] = lo;
               }
@@ -607,24 +659,29 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
           }
           __syncwarp();
 
-          // -- P.V: per value group j and k-slice sl, m-tiles 2j (channels
-          // 32j+4g, +1) and 2j+1 (+2, +3)
+          // -- P.V: per tile, k-slice sl and value group j, m-tiles 2j
+          // (channels 32j+4g, +1) and 2j+1 (+2, +3)
 #pragma unroll
-          for (int j = 0; j < NJ; ++j) {
+          for (int tt = 0; tt < TPW; ++tt) {
 #pragma unroll
             for (int sl = 0; sl < NSL; ++sl) {
               const int tw = BITS == 2 ? sl : 2 * sl + vtw;
-              const uint4 w = *reinterpret_cast<const uint4*>(vc + tw * D + 32 * j + 4 * g);
-              const uint32_t x0 = w.x & vM, x2 = (w.x >> 8) & vM;
-              const uint32_t x1 = w.y & vM, x3 = (w.y >> 8) & vM;
-              const uint32_t y0 = w.z & vM, y2 = (w.z >> 8) & vM;
-              const uint32_t y1 = w.w & vM, y3 = (w.w >> 8) & vM;
 #pragma unroll
-              for (int p = 0; p < NPB; ++p) {
-                const uint2 bb = *reinterpret_cast<const uint2*>(
-                    pB + ((p * NJ + j) * NSL + sl) * 64 + frag_word(lane, sl));
-                mma16816(acc[p][2 * j], x0, x1, x2, x3, bb.x, bb.y);
-                mma16816(acc[p][2 * j + 1], y0, y1, y2, y3, bb.x, bb.y);
+              for (int j = 0; j < NJ; ++j) {
+                const uint4 w = *reinterpret_cast<const uint4*>(vc[tt] + tw * D + 32 * j + 4 * g);
+                const uint32_t x0 = w.x & vM, x2 = (w.x >> 8) & vM;
+                const uint32_t x1 = w.y & vM, x3 = (w.y >> 8) & vM;
+                const uint32_t y0 = w.z & vM, y2 = (w.z >> 8) & vM;
+                const uint32_t y1 = w.w & vM, y3 = (w.w >> 8) & vM;
+#pragma unroll
+                for (int p = 0; p < NPB; ++p) {
+                  const uint2 bb = bcol ? *reinterpret_cast<const uint2*>(
+                                              pB + tt * (G::PB_B / 4) + ((p * NJ + j) * NSL + sl) * 64 +
+                                              frag_word(lane, sl))
+                                        : make_uint2(0u, 0u);
+                  mma16816(acc[p][2 * j], x0, x1, x2, x3, bb.x, bb.y);
+                  mma16816(acc[p][2 * j + 1], y0, y1, y2, y3, bb.x, bb.y);
+                }
               }
             }
           }
@@ -826,28 +883,11 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
         P[2 + d] = num;
       }
       // ---- arrival; the last segment of the unit merges all its partials
-      __threadfence();
       consumers_sync<kW>();
-      if (tid == 0) {
-        unsigned long long* ctr = a.ctr + u;
-        const unsigned long long ep = (unsigned long long)a.epoch << 32;
-        unsigned long long v = atomicAdd(ctr, 0ull);
-        int last = -1;
-        for (int it = 0; it < 4096; ++it) {
-          const unsigned long long nv = ((v >> 32) == a.epoch) ? v + 1ull : (ep | 1ull);
-          const unsigned long long old = atomicCAS(ctr, v, nv);
-          if (old == v) {
-            last = ((long long)(nv & 0xffffffffull) == (long long)n_seg) ? 1 : 0;
-            break;
-          }
-          v = old;
-        }
-        flag[1] = last;
-      }
+      if (tid == 0) flag[1] = arrive_unit(a.ctr + u, a.epoch, n_seg);
       consumers_sync<kW>();
       const int last = flag[1];
       if (last != 0) {
-        __threadfence();
         T* out = reinterpret_cast<T*>(a.out);
         for (int idx = tid; idx < GQ * D; idx += kW * 32) {
           const int h = idx / D, d = idx % D;

@@ -102,37 +102,43 @@ struct DecodeArgs {
 
 constexpr float kNaN = __builtin_nanf("");
 
+// Arrival of one CTA at a unit's counter: a 64-bit word holding the call's
+// epoch in the high half and the arrivals in the low half; a counter left by
+// an earlier call is restarted, so no zeroing is needed.  One thread calls
+// this after a CTA barrier that follows the CTA's partial writes: the
+// compare-and-swap is acquire-release at GPU scope, so those writes are
+// visible to the CTA that arrives last, and after its next CTA barrier that
+// CTA sees every earlier arrival's partials.  Lock-free, bounded retries.
+// Returns 1 for the n-th arrival, 0 for an earlier one, -1 if retries ran out.
+__device__ __forceinline__ int arrive_unit(unsigned long long* ctr, unsigned int epoch,
+                                           long long n) {
+  const unsigned long long ep = (unsigned long long)epoch << 32;
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ctr) : "memory");
+  for (int it = 0; it < 4096; ++it) {
+    const unsigned long long nv = ((v >> 32) == epoch) ? v + 1ull : (ep | 1ull);
+    unsigned long long old;
+    asm volatile("atom.acq_rel.gpu.global.cas.b64 %0, [%1], %2, %3;"
+                 : "=l"(old)
+                 : "l"(ctr), "l"(v), "l"(nv)
+                 : "memory");
+    if (old == v) return ((long long)(nv & 0xffffffffull) == n) ? 1 : 0;
+    v = old;
+  }
+  return -1;
+}
+
 // End of a split CTA, after it wrote its (m, l, acc[D]) partials: the last CTA
-// of the unit to arrive merges all splits of the unit into out.  Arrival is
-// counted in a per-unit 64-bit word tagged with this call's epoch in the high
-// half, so counters left by earlier calls are simply restarted; no zeroing
-// and no waiting (a lock-free compare-and-swap, bounded retries).
+// of the unit to arrive merges all splits of the unit into out.
 // out[b][kv*GQ + h][d] = sum_s 2^(m_s - M) acc_s[d] / sum_s 2^(m_s - M) l_s.
 template <int D, int GQ, typename T>
 __device__ __forceinline__ void finish_unit(const DecodeArgs& a, long long b, int kv,
                                             int* flag) {
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned long long* ctr = a.ctr + (b * a.Hkv + kv);
-    const unsigned long long ep = (unsigned long long)a.epoch << 32;
-    unsigned long long v = atomicAdd(ctr, 0ull);
-    int last = -1;  // -1: gave up (publish NaN)
-    for (int it = 0; it < 4096; ++it) {
-      const unsigned long long nv = ((v >> 32) == a.epoch) ? v + 1ull : (ep | 1ull);
-      const unsigned long long old = atomicCAS(ctr, v, nv);
-      if (old == v) {
-        last = ((long long)(nv & 0xffffffffull) == (long long)a.n_split) ? 1 : 0;
-        break;
-      }
-      v = old;
-    }
-    *flag = last;
-  }
+  if (threadIdx.x == 0) *flag = arrive_unit(a.ctr + (b * a.Hkv + kv), a.epoch, a.n_split);
   __syncthreads();
   const int last = *flag;
   if (last == 0) return;
-  __threadfence();
   const int Hq = a.Hkv * GQ;
   T* out = reinterpret_cast<T*>(a.out);
   for (int idx = threadIdx.x; idx < GQ * D; idx += blockDim.x) {
