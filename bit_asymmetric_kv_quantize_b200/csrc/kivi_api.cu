@@ -105,11 +105,13 @@ void plan_splits(const kivi_cache* c, int sms, int* n_split, int* tiles_per_spli
 // whose ranges meet its tiles or its window start index -- at most
 // ceil((n_q/32 + 1) / W) + 1 CTA segments, each writing one partial -- and
 // the last of them also takes the window.  Measured on B200 (per-CTA
-// timelines): a 32-token window tile costs about three quantized tiles and
-// the end of a unit segment (partial write, arrival, merge) about eight, so
-// a CTA whose range crosses a unit boundary gets correspondingly fewer tiles.
+// timelines): a 32-token window tile costs about two quantized tiles (fp16,
+// tensor cores) or three (fp32, CUDA cores) and the end of a unit segment
+// (partial write, arrival, merge) about eight, so a CTA whose range crosses
+// a unit boundary gets correspondingly fewer tiles.
 constexpr int kTcCtasPerSm = 3;  // upper bound; the kernel instance decides
-constexpr int kWinWeight = 3;    // cost of a window tile, in quantized tiles
+constexpr int kWinWeight = 3;    // cost of a window tile, in quantized tiles (fp32, CUDA cores)
+constexpr int kWinWeightF16 = 2;  // same, fp16 window on tensor cores
 constexpr int kMergeWeight = 8;  // cost of a unit end, in quantized tiles
 
 struct StreamPlan {
@@ -135,7 +137,8 @@ int tc_seg_cap(const kivi_dims& d, int sms) {
 void plan_stream(const kivi_cache* c, int sms, int ctas_per_sm, int seg_cap, StreamPlan* p) {
   const long long units = (long long)c->dims.B * c->dims.Hkv;
   const long long n_qt = c->n_q / kivi::kTile;
-  const int ww = (c->r > 0 ? kWinWeight * (int)ceil_div(c->r, kivi::kTile) : 1) + kMergeWeight;
+  const int wtw = c->dims.dtype == KIVI_F16 ? kWinWeightF16 : kWinWeight;
+  const int ww = (c->r > 0 ? wtw * (int)ceil_div(c->r, kivi::kTile) : 1) + kMergeWeight;
   const long long UP = n_qt + ww;
   const long long total = units * UP;
   const long long P =

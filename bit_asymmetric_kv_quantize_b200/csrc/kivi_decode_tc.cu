@@ -40,6 +40,9 @@
 // The q' and p' fragments are built cooperatively (each lane converts a few
 // values and stores them in fragment order, XOR-swizzled, in per-warp shared
 // memory).
+#include <cuda.h>
+#include <string.h>
+
 #include "kivi_internal.cuh"
 
 namespace kivi {
@@ -98,7 +101,7 @@ struct Geo {
   static constexpr int O_VC = O_KZ + kStage * KM_B;
   static constexpr int O_VS = O_VC + kStage * VC_B;
   static constexpr int O_VZ = O_VS + kStage * VM_B;
-  static constexpr int STAGE_B = O_VZ + kStage * VM_B;
+  static constexpr int STAGE_B = (O_VZ + kStage * VM_B + 1023) / 1024 * 1024;
   static constexpr int NSTAGE = (NW == 4 && TPW == 1 && BITS == 2) ? 3 : 2;
   static constexpr int NPB = GQ == 8 ? 2 : 1;  // n-tiles of 8 columns (4 heads x hi, lo)
   static constexpr int PST = TPW * kTile + 8;  // p buffer stride per head (floats)
@@ -125,6 +128,17 @@ struct Geo {
   // operand scale offsets: the factor 2^(S - e) lies in [2^-S, 2^S]
   static constexpr int SK = Pairs<BITS>::EMAX / 2;
   static constexpr int SV = BITS == 2 ? 3 : 2;  // value e: 2-bit 0,2,4,6; 4-bit 0,4
+  // fp16 residual window through the ring: a window stage holds WT tokens of
+  // K, then of V, as 2-D tensor-copy boxes of BW columns (rows of RB bytes)
+  // in the hardware's 128-byte (64-byte when D = 32) swizzle
+  static constexpr int WT = kTile;
+  static constexpr int BW = D < 64 ? D : 64;
+  static constexpr int NBX = D / BW;
+  static constexpr int RB = BW * 2;
+  static constexpr int BOX_B = WT * RB;
+  static constexpr int WIN_B = 2 * NBX * BOX_B;
+  static_assert(WIN_B <= STAGE_B, "a window stage fits one ring slot");
+  static_assert(STAGE_B % 1024 == 0, "swizzled boxes start on 1024-byte boundaries");
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -148,6 +162,16 @@ __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t b
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// 2-D tensor copy (no multicast) of one box at element coordinates (x, y)
+// into shared memory, completion on an mbarrier.
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                       uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
@@ -178,6 +202,21 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Four 8x8 fp16 matrices from shared memory; lanes 8i..8i+7 give the row
+// addresses of matrix i.  .trans delivers each matrix transposed.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p))
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p))
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
@@ -203,7 +242,8 @@ __device__ __forceinline__ void consumers_sync() {
 
 template <int D, int BITS, int GQ, typename T>
 __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::MIN_CTAS)
-    decode_stream_tc(DecodeArgs a) {
+    decode_stream_tc(DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV) {
   using G = Geo<D, BITS, GQ>;
   using PR = Pairs<BITS>;
   constexpr int kW = G::NW;
@@ -217,7 +257,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
   constexpr int CPL = D / 32;  // window path: channels per lane
   constexpr float kKeyOut = (float)(1 << (24 - G::SK));
   constexpr float kValOut = (float)(1 << (24 - G::SV));
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
@@ -245,7 +285,9 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kW);
     }
-    flag[0] = 0;
+    // swizzled window boxes need 1024-byte aligned stages: refuse (abort
+    // flag, NaN outputs) rather than read a mis-swizzled layout
+    flag[0] = (sizeof(T) == 2 && (smem_u32(smem) & 1023u) != 0) ? 1 : 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp < kW) {
@@ -290,13 +332,36 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
         }
         if (*(volatile int*)&flag[0]) break;
         if (a.r > 0 && cta == (base + n_qt) / W) {
-          // this CTA owns the unit's residual window: pull it into L2 while
-          // the consumers work through the unit's last stages
-          const uint32_t wbytes = (uint32_t)((size_t)a.r * D * sizeof(T));
           const T* kr = reinterpret_cast<const T*>(c.k_res) + u * c.R * D;
           const T* vr = reinterpret_cast<const T*>(c.v_res) + u * c.R * D;
-          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kr), "r"(wbytes) : "memory");
-          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vr), "r"(wbytes) : "memory");
+          if constexpr (sizeof(T) == 2) {
+            // this CTA owns the unit's residual window: stream it through
+            // the ring, WT tokens of K and of V per stage, one row per copy
+            for (int w0 = 0; w0 < a.r; w0 += G::WT, ++st) {
+              const int s = (int)(st % G::NSTAGE);
+              if (st >= G::NSTAGE &&
+                  !mbar_wait(&empty[s], (uint32_t)(((st / G::NSTAGE) - 1) & 1))) {
+                atomicExch(&flag[0], 1);
+                break;
+              }
+              if (*(volatile int*)&flag[0]) break;
+              unsigned char* buf = smem + s * G::STAGE_B;
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              mbar_expect_tx(&full[s], (uint32_t)G::WIN_B);
+              const int y = (int)(u * c.R + w0);  // row of the [units * R][D] window
+#pragma unroll
+              for (int bx = 0; bx < G::NBX; ++bx) {
+                tma_2d(buf + bx * G::BOX_B, &tmK, bx * G::BW, y, &full[s]);
+                tma_2d(buf + (G::NBX + bx) * G::BOX_B, &tmV, bx * G::BW, y, &full[s]);
+              }
+            }
+          } else {
+            // fp32 window (CUDA-core path): pull it into L2 while the
+            // consumers work through the unit's last stages
+            const uint32_t wbytes = (uint32_t)((size_t)a.r * D * sizeof(T));
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kr), "r"(wbytes) : "memory");
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vr), "r"(wbytes) : "memory");
+          }
         }
       }
     }
@@ -400,8 +465,10 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
           qf[x][m][2] = to_f32(qh[1]) * a.qscale;
           qf[x][m][3] = to_f32(qh[G::PPW + 1]) * a.qscale;
         }
-      if (window_owner)
+      if (window_owner) {
         for (int i = tid; i < GQ * D; i += kW * 32) qs[i] = to_f32(qg[i]) * a.qscale;
+        consumers_sync<kW>();  // qs is read by whichever warps take the window
+      }
 
       float m_run[NPB], l_part[NPB];
       float acc[NPB][NM][4];
@@ -421,6 +488,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
         for (int j = 0; j < NJ; ++j) bv[h][j] = 0.f;
 
       for (long long t0 = t_beg; t0 < t_end; t0 += kStage, ++st) {
+        if (*(volatile int*)&flag[0]) break;
         const int s = (int)(st % G::NSTAGE);
         const bool ok = mbar_wait(&full[s], (uint32_t)((st / G::NSTAGE) & 1));
         if (!__all_sync(0xffffffffu, ok) || *(volatile int*)&flag[0]) {
@@ -689,10 +757,127 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }
-      const bool failed = *(volatile int*)&flag[0] != 0;
+      // ---- one fp16 window stage of nt tokens on tensor cores: S = K q
+      // (K rows by ldmatrix), the same online softmax, O += V^T p (V^T by
+      // ldmatrix.trans); rows past nt read row 0 and are masked out
+      auto window_tile = [&](const unsigned char* wbuf, int nt) {
+        const unsigned char* Kw = wbuf;
+        const unsigned char* Vw = wbuf + G::NBX * G::BOX_B;
+        // address of 16-byte chunk cc (channels 8 cc .. 8 cc + 7) of row tok:
+        // the swizzle XORs the chunk index with address bits 7.. of the row
+        auto chunk = [&](const unsigned char* base, int tok, int cc) -> const unsigned char* {
+          constexpr int CPR = G::RB / 16;  // chunks per box row
+          const unsigned char* row = base + (cc / CPR) * G::BOX_B + tok * G::RB;
+          const uint32_t ra = smem_u32(row);
+          const int x = G::RB == 128 ? (int)((ra >> 7) & 7u) : (int)((ra >> 7) & 3u);
+          return row + (((cc % CPR) ^ x) << 4);
+        };
+        float dq[NPB][2][4];
+#pragma unroll
+        for (int p = 0; p < NPB; ++p)
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dq[p][mt][e] = 0.f;
+#pragma unroll
+        for (int sl = 0; sl < KSL; ++sl) {
+          uint2 bq[NPB];
+#pragma unroll
+          for (int p = 0; p < NPB; ++p)
+            bq[p] = bcol ? *reinterpret_cast<const uint2*>(qB + (p * KSL + sl) * 64 + frag_word(lane, sl))
+                         : make_uint2(0u, 0u);
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            const int tok = 16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1);
+            uint32_t af[4];
+            ldsm_x4(af, chunk(Kw, tok < nt ? tok : 0, 2 * sl + (lane >> 4)));
+#pragma unroll
+            for (int p = 0; p < NPB; ++p) mma16816(dq[p][mt], af[0], af[1], af[2], af[3], bq[p].x, bq[p].y);
+          }
+        }
+        float sc[NPB][4];
+#pragma unroll
+        for (int p = 0; p < NPB; ++p)
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const float v = dq[p][mt][2 * r] + dq[p][mt][2 * r + 1];
+              sc[p][2 * mt + r] = (16 * mt + 8 * r + g < nt) ? v : kNegInf;
+            }
+        float lm[NPB];
+        bool need = false;
+#pragma unroll
+        for (int p = 0; p < NPB; ++p) {
+          lm[p] = fmaxf(fmaxf(sc[p][0], sc[p][1]), fmaxf(sc[p][2], sc[p][3]));
+          need |= vh[p] && lm[p] > m_run[p];
+        }
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int p = 0; p < NPB; ++p) {
+            float tm = lm[p];
+            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
+            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
+            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
+            const float mn = fmaxf(m_run[p], tm);
+            const float al = exp2f(m_run[p] - mn);
+            m_run[p] = mn;
+            l_part[p] *= al;
+#pragma unroll
+            for (int m = 0; m < NM; ++m)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[p][m][e] *= al;
+          }
+        }
+#pragma unroll
+        for (int p = 0; p < NPB; ++p) {
+          float ps = 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float pv = exp2f(sc[p][i] - m_run[p]);
+            ps += pv;
+            if (vh[p]) pbuf[(tq + 4 * p) * PST + 16 * (i >> 1) + 8 * (i & 1) + g] = pv;
+          }
+          l_part[p] += ps;
+        }
+        __syncwarp();
+        // p (hi, lo) into the value B fragments, tokens in natural order
+        {
+          const int slp = lane >> 4, kk = lane & 15;
+          const int tqk = (kk & 7) >> 1, kp = kk >> 3, hf = kk & 1;
+#pragma unroll
+          for (int h = 0; h < GQ; ++h) {
+            const float x = pbuf[h * PST + lane];
+            const __half hi = __float2half_rn(x);
+            const __half lo = __float2half_rn(x - __half2float(hi));
+            __half* blk = pBh + ((h >> 2) * NJ * NSL + slp) * 128 + 2 * kp + hf;
+            const int nh = 2 * (h & 3);
+            blk[2 * frag_word(4 * nh + tqk, slp)] = hi;
+            blk[2 * frag_word(4 * (nh + 1) + tqk, slp)] = lo;
+          }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int sl = 0; sl < NSL; ++sl) {
+          uint2 bb[NPB];
+#pragma unroll
+          for (int p = 0; p < NPB; ++p)
+            bb[p] = bcol ? *reinterpret_cast<const uint2*>(pB + (p * NJ * NSL + sl) * 64 + frag_word(lane, sl))
+                         : make_uint2(0u, 0u);
+          const int tok = 16 * sl + (lane & 7) + 8 * (lane >> 4);
+          const int tr = tok < nt ? tok : 0;
+#pragma unroll
+          for (int m = 0; m < NM; ++m) {
+            uint32_t af[4];
+            ldsm_x4_t(af, chunk(Vw, tr, 2 * m + ((lane >> 3) & 1)));
+#pragma unroll
+            for (int p = 0; p < NPB; ++p) mma16816(acc[p][m], af[0], af[1], af[2], af[3], bb[p].x, bb[p].y);
+          }
+        }
+      };
 
-      // ---- this warp's streamed state -> mg slot `warp`
-      {
+      // ---- this warp's quantized-tile state (m, l, acc + value zeros) -> mg slot
+      auto flush_code = [&]() {
         float lt[NPB];
 #pragma unroll
         for (int p = 0; p < NPB; ++p) {
@@ -727,11 +912,108 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
             dst[1] = fmaf(acc[p][m][2] + acc[p][m][3], kValOut, bias);
           }
         }
+      };
+
+      // ---- fp16 residual window on tensor cores: window stage k goes to warp
+      // k % kW, which first flushes its quantized-tile state and then keeps a
+      // separate softmax state for the window (plain q and p, scale 1)
+      bool wmode = false;
+      if constexpr (sizeof(T) == 2) {
+        if (window_owner) {
+          int k = 0;
+          for (int w0 = 0; w0 < a.r; w0 += G::WT, ++st, ++k) {
+            if (*(volatile int*)&flag[0]) break;
+            const int s = (int)(st % G::NSTAGE);
+            const bool ok = mbar_wait(&full[s], (uint32_t)((st / G::NSTAGE) & 1));
+            if (!__all_sync(0xffffffffu, ok) || *(volatile int*)&flag[0]) {
+              if (lane == 0) atomicExch(&flag[0], 1);
+              break;
+            }
+            if (k % kW == warp) {
+              if (!wmode) {
+                flush_code();
+                __syncwarp();
+                wmode = true;
+#pragma unroll
+                for (int p = 0; p < NPB; ++p) {
+                  m_run[p] = kNegInf;
+                  l_part[p] = 0.f;
+#pragma unroll
+                  for (int m = 0; m < NM; ++m)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[p][m][e] = 0.f;
+                }
+                // B fragments of plain q (hi, lo), channels in natural order:
+                // k-slice sl, k = channel - 16 sl; lane takes channel pairs
+#pragma unroll
+                for (int cp0 = 0; cp0 < D / 2; cp0 += 32) {
+                  const int cpr = cp0 + lane;  // channels 2 cpr, 2 cpr + 1
+                  if (cpr < D / 2) {
+                    const int sl = cpr >> 3, kk = 2 * (cpr & 7);
+                    const int tqk = (kk & 7) >> 1, kp = kk >> 3;
+#pragma unroll
+                    for (int h = 0; h < GQ; ++h) {
+                      const float2 x = *reinterpret_cast<const float2*>(qs + h * D + 2 * cpr);
+                      uint32_t hi, lo;
+                      split2(x.x, x.y, hi, lo);
+                      uint32_t* blk = qB + ((h >> 2) * KSL + sl) * 64 + kp;
+                      const int nh = 2 * (h & 3);
+                      blk[frag_word(4 * nh + tqk, sl)] = hi;
+                      blk[frag_word(4 * (nh + 1) + tqk, sl)] = lo;
+                    }
+                  }
+                }
+                __syncwarp();
+              }
+              window_tile(smem + s * G::STAGE_B, min(G::WT, a.r - w0));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+          }
+        }
+      }
+      const bool failed = *(volatile int*)&flag[0] != 0;
+      if (!wmode) {
+        flush_code();
+      } else {
+        // fold the window state into this warp's slot (quantized-tile state)
+        float lt[NPB], m1[NPB], l1[NPB];
+#pragma unroll
+        for (int p = 0; p < NPB; ++p) {
+          float v = l_part[p];
+          v += __shfl_xor_sync(0xffffffffu, v, 4);
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          v += __shfl_xor_sync(0xffffffffu, v, 16);
+          lt[p] = v;
+          const int h = tq + 4 * p;
+          m1[p] = vh[p] ? mg_m[warp * GQ + h] : kNegInf;
+          l1[p] = vh[p] ? mg_l[warp * GQ + h] : 0.f;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int p = 0; p < NPB; ++p) {
+          if (!vh[p]) continue;
+          const int h = tq + 4 * p;
+          const float mn = fmaxf(m1[p], m_run[p]);
+          const float s1 = m1[p] == kNegInf ? 0.f : exp2f(m1[p] - mn);
+          const float s2 = m_run[p] == kNegInf ? 0.f : exp2f(m_run[p] - mn);
+          float* dst = mg_acc + (warp * GQ + h) * D;
+#pragma unroll
+          for (int m = 0; m < NM; ++m) {
+            const int ch = 16 * m + g;
+            dst[ch] = fmaf(dst[ch], s1, (acc[p][m][0] + acc[p][m][1]) * s2);
+            dst[ch + 8] = fmaf(dst[ch + 8], s1, (acc[p][m][2] + acc[p][m][3]) * s2);
+          }
+          if (g == 0) {
+            mg_m[warp * GQ + h] = mn;
+            mg_l[warp * GQ + h] = fmaf(l1[p], s1, lt[p] * s2);
+          }
+        }
       }
       __syncwarp();
       // ---- residual window (CTA that ends the unit): warp w takes window
       // tiles w, w+4, ... on CUDA cores, folded into its mg slot
-      if (window_owner && !failed) {
+      if (sizeof(T) == 4 && window_owner && !failed) {
         consumers_sync<kW>();  // qs written by all consumer threads
         const T* kr = reinterpret_cast<const T*>(c.k_res) + u * c.R * D;
         const T* vr = reinterpret_cast<const T*>(c.v_res) + u * c.R * D;
@@ -893,21 +1175,9 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
           const int h = idx / D, d = idx % D;
           const long long row = b * Hq + (long long)kv * GQ + h;
           float res = kNaN;
-          if (last > 0) {
-            float M = kNegInf;
-            for (int sg = 0; sg < n_seg; ++sg)
-              M = fmaxf(M, __ldcg(a.ws + ((u * a.max_seg + sg) * GQ + h) * (D + 2)));
-            float num = 0.f, den = 0.f;
-            for (int sg = 0; sg < n_seg; ++sg) {
-              const float* P = a.ws + ((u * a.max_seg + sg) * GQ + h) * (D + 2);
-              const float ms = __ldcg(P);
-              if (ms == kNegInf) continue;
-              const float s2 = exp2f(ms - M);
-              num = fmaf(s2, __ldcg(P + 2 + d), num);
-              den = fmaf(s2, __ldcg(P + 1), den);
-            }
-            res = num / den;
-          }
+          if (last > 0)
+            res = merge_partials(a.ws + (u * a.max_seg * GQ + h) * (D + 2), (long long)GQ * (D + 2),
+                                 n_seg, d);
           out[row * D + d] = from_f32<T>(res);
         }
       }
@@ -944,6 +1214,40 @@ cudaError_t tc_setup(int* ctas_per_sm) {
   return cudaSuccess;
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library), looked up once.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// Tensor map of one fp16 residual buffer viewed as [units * R][D]: boxes of
+// 32 rows x min(D, 64) columns, swizzled (128-byte rows: 128B, 64-byte: 64B).
+cudaError_t window_map(CUtensorMap* m, const void* base, long long rows, int D) {
+  const EncodeTiledFn fn = encode_tiled();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)(D < 64 ? D : 64), (cuuint32_t)kTile};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
+                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        D < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int D, int BITS, int GQ, typename T>
 cudaError_t tc_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
                  int* ctas_per_sm) {
@@ -952,8 +1256,18 @@ cudaError_t tc_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_
   int occ = 0;
   cudaError_t e = tc_setup<D, BITS, GQ, T>(&occ);
   if (e != cudaSuccess) return e;
+  CUtensorMap tmK, tmV;
+  memset(&tmK, 0, sizeof(tmK));
+  memset(&tmV, 0, sizeof(tmV));
+  if (sizeof(T) == 2 && a.r > 0) {
+    const long long rows = (long long)a.units * a.c.R;
+    if (rows >= (1LL << 31)) return cudaErrorInvalidValue;  // 32-bit box coordinates
+    e = window_map(&tmK, a.c.k_res, rows, D);
+    if (e == cudaSuccess) e = window_map(&tmV, a.c.v_res, rows, D);
+    if (e != cudaSuccess) return e;
+  }
   if (e0) cudaEventRecord(e0, s);
-  decode_stream_tc<D, BITS, GQ, T><<<a.n_cta, G::THREADS, G::SMEM_B, s>>>(a);
+  decode_stream_tc<D, BITS, GQ, T><<<a.n_cta, G::THREADS, G::SMEM_B, s>>>(a, tmK, tmV);
   cudaError_t err = cudaGetLastError();
   if (e1) cudaEventRecord(e1, s);
   return err;

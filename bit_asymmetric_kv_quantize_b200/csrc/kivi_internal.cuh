@@ -128,6 +128,47 @@ __device__ __forceinline__ int arrive_unit(unsigned long long* ctr, unsigned int
   return -1;
 }
 
+// Merge of one output element over a unit's n partials P_s = (m_s, l_s,
+// acc_s[D]) (P_s at P0 + s * stride): sum_s 2^(m_s - M) acc_s[d] /
+// sum_s 2^(m_s - M) l_s with M = max_s m_s.  The partials are read in
+// batches of 8 whose loads are all issued before any is used (one L2 round
+// trip per batch); empty partials (m_s = -inf) are skipped.
+__device__ __forceinline__ float merge_partials(const float* P0, long long stride, int n, int d) {
+  constexpr int kB = 8;
+  float M = -__builtin_huge_valf(), num = 0.f, den = 0.f;
+  for (int s0 = 0; s0 < n; s0 += kB) {
+    float m[kB], l[kB], v[kB];
+#pragma unroll
+    for (int k = 0; k < kB; ++k) {
+      m[k] = -__builtin_huge_valf();
+      l[k] = 0.f;
+      v[k] = 0.f;
+      if (s0 + k < n) {
+        const float* P = P0 + (long long)(s0 + k) * stride;
+        m[k] = __ldcg(P);
+        l[k] = __ldcg(P + 1);
+        v[k] = __ldcg(P + 2 + d);
+      }
+    }
+    float Mb = M;
+#pragma unroll
+    for (int k = 0; k < kB; ++k) Mb = fmaxf(Mb, m[k]);
+    if (Mb == -__builtin_huge_valf()) continue;
+    const float sc = exp2f(M - Mb);  // 0 while M = -inf
+    num *= sc;
+    den *= sc;
+#pragma unroll
+    for (int k = 0; k < kB; ++k) {
+      if (m[k] == -__builtin_huge_valf()) continue;
+      const float e = exp2f(m[k] - Mb);
+      num = fmaf(e, v[k], num);
+      den = fmaf(e, l[k], den);
+    }
+    M = Mb;
+  }
+  return num / den;
+}
+
 // End of a split CTA, after it wrote its (m, l, acc[D]) partials: the last CTA
 // of the unit to arrive merges all splits of the unit into out.
 // out[b][kv*GQ + h][d] = sum_s 2^(m_s - M) acc_s[d] / sum_s 2^(m_s - M) l_s.
@@ -145,20 +186,7 @@ __device__ __forceinline__ void finish_unit(const DecodeArgs& a, long long b, in
     const int h = idx / D, d = idx % D;
     const long long row = b * Hq + (long long)kv * GQ + h;
     float res = kNaN;
-    if (last > 0) {
-      const float* P = a.ws + row * a.n_split * (D + 2);
-      float M = -__builtin_huge_valf();
-      for (int s = 0; s < a.n_split; ++s) M = fmaxf(M, __ldcg(P + s * (D + 2)));
-      float num = 0.f, den = 0.f;
-      for (int s = 0; s < a.n_split; ++s) {
-        const float ms = __ldcg(P + s * (D + 2));
-        if (ms == -__builtin_huge_valf()) continue;
-        const float sc = exp2f(ms - M);
-        num = fmaf(sc, __ldcg(P + s * (D + 2) + 2 + d), num);
-        den = fmaf(sc, __ldcg(P + s * (D + 2) + 1), den);
-      }
-      res = num / den;
-    }
+    if (last > 0) res = merge_partials(a.ws + row * a.n_split * (D + 2), D + 2, a.n_split, d);
     out[row * D + d] = from_f32<T>(res);
   }
 }
