@@ -2,10 +2,12 @@
 """Benchmark: KIVI 2-bit decode attention on B200.
 
 One step = one decode step of one attention layer through the C ABI:
-kivi_append_token (the new token's K/V into the residual window, flushing
-the window into the 2-bit store every R tokens) then kivi_decode_attention
-(fused dequant + q.K + online softmax + P.V over the packed codes and the
-window, then the cross-split merge).  Workload: the Llama-2-7B-shaped layer
+kivi_append_decode -- the new token's K/V into the residual window (the
+window is flushed into the 2-bit store every R tokens, as its own launch)
+and decode attention (fused dequant + q.K + online softmax + P.V over the
+packed codes and the window, then the cross-split merge), one kernel launch
+when no flush is due.  `--unfused` times kivi_append_token followed by
+kivi_decode_attention instead (two launches per step).  Workload: the Llama-2-7B-shaped layer
 (B=8, 32 heads, D=128, context 4096, 2-bit, G=32, R=128) by default.
 
 L2 hygiene: `--layers` copies of the layer cache (default 32, the model's
@@ -56,6 +58,8 @@ def parse():
     p.add_argument("--kernel", choices=["default", "simt"], default="default")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--unfused", action="store_true",
+                   help="append and decode as two calls (kivi_append_token + decode)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
     return p.parse_args()
 
@@ -212,16 +216,25 @@ def run_kivi(args, rank, world, local):
     qp = [t.data_ptr() for t in qs]
     op, wp, wn = out.data_ptr(), ws.data_ptr(), ws.numel()
 
+    fused = args.kernel == "default" and not args.unfused
+    n_launch = [0]
+
+    def step_call(li, k_ptr, v_ptr, q_ptr):
+        """One append + decode; returns the status and counts kernel launches."""
+        c = caches[li]
+        n_launch[0] += 1 + (1 if (not fused or c.r == c.R) else 0)
+        if fused:
+            return L.kivi_append_decode(cstructs[li], k_ptr, v_ptr, q_ptr, w.Hq, 1.0, op, wp, wn, sh)
+        rc = L.kivi_append_token(cstructs[li], k_ptr, v_ptr, sh)
+        return rc or dec(cstructs[li], q_ptr, w.Hq, 1.0, op, wp, wn, sh)
+
     def step(i, ev=None):
         li = i % n_layers
-        rc = L.kivi_append_token(cstructs[li], kp[i % P], vp[i % P], sh)
-        if rc:
-            raise RuntimeError(f"append: {L.kivi_status_string(rc)}")
         if ev is not None:
             L.kivi_set_timing_events(ev[0], ev[1])
-        rc = dec(cstructs[li], qp[i % P], w.Hq, 1.0, op, wp, wn, sh)
+        rc = step_call(li, kp[i % P], vp[i % P], qp[i % P])
         if rc:
-            raise RuntimeError(f"decode: {L.kivi_status_string(rc)}")
+            raise RuntimeError(f"step: {L.kivi_status_string(rc)}")
 
     def barrier():
         if world > 1:
@@ -245,6 +258,7 @@ def run_kivi(args, rank, world, local):
     fills = []
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
+    n_launch[0] = 0
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         t0.record(stream)
         for j in range(args.steps):
@@ -253,6 +267,7 @@ def run_kivi(args, rank, world, local):
             c = caches[i % n_layers]
             fills.append((c.n_q, c.r))
         t1.record(stream)
+        timed_launches = n_launch[0]
         torch.cuda.synchronize(device)
     L.kivi_set_timing_events(None, None)
     barrier()
@@ -288,8 +303,7 @@ def run_kivi(args, rank, world, local):
             dk.copy_(hk[i % P], non_blocking=True)
             dv.copy_(hv[i % P], non_blocking=True)
             dq.copy_(hq[i % P], non_blocking=True)
-            rc = L.kivi_append_token(cstructs[li], dk.data_ptr(), dv.data_ptr(), sh)
-            rc |= dec(cstructs[li], dq.data_ptr(), w.Hq, 1.0, op, wp, wn, sh)
+            rc = step_call(li, dk.data_ptr(), dv.data_ptr(), dq.data_ptr())
             if rc:
                 raise RuntimeError("e2e step failed")
             ho.copy_(out, non_blocking=True)
@@ -319,7 +333,7 @@ def run_kivi(args, rank, world, local):
             "config": {
                 "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                 "context": w.T, "bits": w.bits, "G": w.G, "Gv": w.Gv, "R": w.R,
-                "dtype_io": w.dtype, "kernel": args.kernel, "parallelism": f"replicas{world}",
+                "dtype_io": w.dtype, "kernel": args.kernel, "step": ("kivi_append_decode" if fused else "kivi_append_token+kivi_decode_attention"), "parallelism": f"replicas{world}",
                 "layers_rotated": n_layers,
                 "l2": f"inputs larger than L2: {n_layers} layer caches visited round-robin",
                 "decode_splits": n_split,
@@ -332,7 +346,7 @@ def run_kivi(args, rank, world, local):
                 "avg_launch_us": split_total_ms * 1e3 / args.steps,
             },
             "e2e": e2e,
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": timed_launches,
             "clocks": clk.summary(),
         }
     for c in caches:

@@ -32,7 +32,7 @@ EXPORTED = (
     "kivi_buffer_sizes", "kivi_cache_init", "kivi_quantize_prefill", "kivi_append_token",
     "kivi_decode_workspace_bytes", "kivi_decode_attention", "kivi_decode_attention_simt",
     "kivi_set_timing_events", "kivi_decode_num_splits", "kivi_status_string",
-    "kivi_decode_attention_noalloc",
+    "kivi_decode_attention_noalloc", "kivi_append_decode",
 )
 
 
@@ -83,6 +83,7 @@ def lib() -> ctypes.CDLL:
             L.kivi_decode_attention.argtypes = dec
             L.kivi_decode_attention_simt.argtypes = dec
             L.kivi_decode_attention_noalloc.argtypes = [cp, vp, ci, ctypes.c_float, vp, vp]
+            L.kivi_append_decode.argtypes = [cp, vp, vp, vp, ci, ctypes.c_float, vp, vp, sz, vp]
             L.kivi_set_timing_events.argtypes = [vp, vp]
             L.kivi_set_timing_events.restype = None
             L.kivi_decode_num_splits.argtypes = [cp, ci]
@@ -223,6 +224,23 @@ class KiviCache:
         with torch.cuda.device(self.device):
             _check(fn(ctypes.byref(self._c), pq, Hq, float(softmax_scale), po, ws.data_ptr(),
                       ws.numel(), self._stream()), "kivi_decode_attention")
+        return out
+
+    def append_decode(self, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor,
+                      softmax_scale: float, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """append(k, v) then decode(q) in one call (one launch unless a flush is due)."""
+        shape = (self.B, self.Hkv, self.D)
+        pk, pv = self._arg(k, shape, "k"), self._arg(v, shape, "v")
+        Hq = q.shape[1]
+        pq = self._arg(q, (self.B, Hq, self.D), "q")
+        if out is None:
+            out = torch.empty_like(q)
+        po = self._arg(out, (self.B, Hq, self.D), "out")
+        ws = self.workspace(Hq)
+        with torch.cuda.device(self.device):
+            _check(lib().kivi_append_decode(ctypes.byref(self._c), pk, pv, pq, Hq,
+                                            float(softmax_scale), po, ws.data_ptr(), ws.numel(),
+                                            self._stream()), "kivi_append_decode")
         return out
 
 

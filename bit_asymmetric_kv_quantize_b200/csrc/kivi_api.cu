@@ -183,9 +183,13 @@ unsigned int next_epoch() {
 // Validate, plan and launch one decode.  `ws` holds the arrival counters and
 // the partials; the split count is capped at `split_cap`.
 int decode_launch(const kivi_cache* c, const void* q, int Hq, float softmax_scale, void* out,
-                  void* ws, int split_cap, int sms, void* stream, bool simt) {
+                  void* ws, int split_cap, int sms, void* stream, bool simt,
+                  const void* new_k = nullptr, const void* new_v = nullptr, int new_slot = 0) {
   const int gq = Hq / c->dims.Hkv;
   DecodeArgs a;
+  a.new_k = new_k;
+  a.new_v = new_v;
+  a.new_slot = new_slot;
   a.c = view(c);
   a.q = q;
   a.out = out;
@@ -370,6 +374,39 @@ int kivi_decode_attention(const kivi_cache* cache, const void* q, int Hq, float 
                           void* out, void* workspace, size_t workspace_bytes, void* stream) {
   return decode_common(cache, q, Hq, softmax_scale, out, workspace, workspace_bytes, stream,
                        false);
+}
+
+int kivi_append_decode(kivi_cache* cache, const void* k, const void* v, const void* q, int Hq,
+                       float softmax_scale, void* out, void* workspace, size_t ws_bytes,
+                       void* stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!k || !v) return KIVI_ERR_ARG;
+  if (cache->n_q + cache->r + 1 > cache->dims.capacity) return KIVI_ERR_CAPACITY;
+  // the decode half sees the cache with the new token in it
+  kivi_cache after = *cache;
+  if (after.r == after.dims.R) {
+    after.n_q += after.dims.R;
+    after.r = 1;
+  } else {
+    after.r += 1;
+  }
+  rc = decode_checks(&after, q, Hq, out);
+  if (rc) return rc;
+  const int sms = device_sms();
+  if (sms <= 0) return KIVI_ERR_CUDA;
+  if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(cache->dims, Hq, sms))
+    return KIVI_ERR_WORKSPACE;
+  if (cache->r == cache->dims.R) {  // flush due: its own launch, then decode
+    rc = kivi_append_token(cache, k, v, stream);
+    if (rc) return rc;
+    return decode_launch(cache, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms),
+                         sms, stream, false);
+  }
+  rc = decode_launch(&after, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms), sms,
+                     stream, false, k, v, cache->r);
+  if (rc == KIVI_OK) cache->r = after.r;
+  return rc;
 }
 
 int kivi_decode_attention_simt(const kivi_cache* cache, const void* q, int Hq,

@@ -290,6 +290,23 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
     flag[0] = (sizeof(T) == 2 && (smem_u32(smem) & 1023u) != 0) ? 1 : 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (a.new_k != nullptr) {
+    // fused append: the CTA that owns a unit's window writes the unit's new
+    // token into window slot new_slot; the proxy fence and the barrier below
+    // order these writes before this CTA's tensor copies and loads of the window
+    for (long long u = G0 / UP; G0 < G1 && u <= (G1 - 1) / UP; ++u) {
+      if (cta != (u * UP + n_qt) / W) continue;
+      T* kr = reinterpret_cast<T*>(c.k_res) + (u * c.R + a.new_slot) * D;
+      T* vr = reinterpret_cast<T*>(c.v_res) + (u * c.R + a.new_slot) * D;
+      const T* kn = reinterpret_cast<const T*>(a.new_k) + u * D;
+      const T* vn = reinterpret_cast<const T*>(a.new_v) + u * D;
+      for (int i = tid; i < D; i += G::THREADS) {
+        kr[i] = kn[i];
+        vr[i] = vn[i];
+      }
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
   if (warp < kW) {
     // fragment columns of absent heads stay zero
     unsigned char* wb = smem + G::O_WARP + warp * G::WARP_B;

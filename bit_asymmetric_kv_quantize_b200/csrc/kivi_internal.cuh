@@ -98,6 +98,12 @@ struct DecodeArgs {
   long long tiles_per_cta;
   int max_seg;
   int win_weight;
+  // fused append (tensor-core kernel only): when new_k is non-null the call
+  // first writes token new_k/new_v ([B][Hkv][D]) into window slot new_slot
+  // (r above already counts it)
+  const void* new_k;
+  const void* new_v;
+  int new_slot;
 };
 
 constexpr float kNaN = __builtin_nanf("");

@@ -204,6 +204,23 @@ KIVI_API int kivi_decode_attention_simt(const kivi_cache *cache, const void *q,
                                void *workspace, size_t workspace_bytes,
                                void *stream);
 
+/* One decode step of a streaming loop: kivi_append_token(cache, k, v)
+ * followed by kivi_decode_attention over the cache that now holds the new
+ * token -- same arguments as the two calls, same result, same counter
+ * update.  When no flush is due (r < R) it is one kernel launch: the decode
+ * kernel's CTA that owns a sequence's window writes the new token into
+ * window slot r before it reads the window.  When the window is full the
+ * flush runs first as its own launch (as in kivi_append_token).  All
+ * argument checks of both calls happen before any launch, so an error
+ * leaves the cache unchanged.  The counters stay on the host, so a loop of
+ * these calls is not graph-capturable.  (KIVI, study.space summary: new
+ * tokens enter the full-precision residual part; decode attends over both
+ * parts.)
+ * Errors: those of kivi_append_token and kivi_decode_attention. */
+KIVI_API int kivi_append_decode(kivi_cache *cache, const void *k, const void *v,
+                       const void *q, int Hq, float softmax_scale, void *out,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
 /* Optional timing hook: if start/stop are non-NULL cudaEvent_t handles,
  * later decode calls on this thread record `start` just before and `stop`
  * just after the launch of the dominant (split) decode kernel, on the

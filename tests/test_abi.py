@@ -120,6 +120,17 @@ def test_host_side_state_and_capacity_errors():
     assert L.kivi_append_token(ctypes.byref(c), fake, fake, None) == ERR_CAPACITY
     assert L.kivi_append_token(ctypes.byref(c), None, fake, None) == ERR_ARG
     assert (c.n_q, c.r) == (128, 128)  # unchanged by refused calls
+    # the fused step refuses what either half would refuse, before any launch
+    assert L.kivi_append_decode(ctypes.byref(c), fake, fake, fake, 4, 1.0, fake, fake, 1 << 20,
+                                None) == ERR_CAPACITY
+    c.n_q, c.r = 0, 5
+    assert L.kivi_append_decode(ctypes.byref(c), None, fake, fake, 4, 1.0, fake, fake, 1 << 20,
+                                None) == ERR_ARG
+    assert L.kivi_append_decode(ctypes.byref(c), fake, fake, fake, 6, 1.0, fake, fake, 1 << 20,
+                                None) == ERR_ARG
+    assert L.kivi_append_decode(ctypes.byref(c), fake, fake, None, 4, 1.0, fake, fake, 1 << 20,
+                                None) == ERR_ARG
+    assert (c.n_q, c.r) == (0, 5)
 
 
 def test_status_strings():

@@ -149,6 +149,35 @@ def test_streaming_workload_every_step():
     print(f"streaming worst max-abs {worst:.3e}")
 
 
+@pytest.mark.parametrize("dtype,D", [("f16", 128), ("f16", 64), ("f32", 64)])
+@pytest.mark.parametrize("gq", [1, 4])
+def test_append_decode_matches_separate_calls(dtype, D, gq):
+    """kivi_append_decode (one launch unless a flush is due) gives bit for bit
+    the outputs and cache state of kivi_append_token + kivi_decode_attention,
+    over 150 steps that cross two flushes (R = 64), and stays within the
+    tolerance of the oracle."""
+    w = small(D=D, dtype=dtype, gq=gq, T=100, R=64, B=2, Hkv=2, seed=11)
+    K, V = W.prompt_kv(w, device="cuda")
+    fused, ref = gpu_cache(w, capacity=512), gpu_cache(w, capacity=512)
+    fused.prefill(K, V)
+    ref.prefill(K, V)
+    oc = oracle_cache(w, capacity=512)
+    oracle_prefill(oc, K, V)
+    for step in range(150):
+        k, v = W.step_kv(w, step, device="cuda")
+        q = W.query(w, step, device="cuda")
+        out_f = fused.append_decode(k, v, q, 1.0)
+        ref.append(k, v)
+        out_r = ref.decode(q, 1.0)
+        oracle_append(oc, k, v)
+        assert (fused.n_q, fused.r) == (ref.n_q, ref.r)
+        assert torch.equal(out_f, out_r), f"step {step}"
+        if step % 25 == 0 or fused.r == 1:
+            assert_decode_close(out_f, oc, q, 1.0)
+    assert fused.n_q + fused.r == 100 + 150
+    assert_state_equal(fused, oc)
+
+
 def test_decode_errors_on_device():
     w = small(D=64, T=100)
     K, V = W.prompt_kv(w, device="cuda")
