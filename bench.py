@@ -96,6 +96,28 @@ def peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def profiled_traffic(w: W.Workload):
+    """DRAM bytes per decode launch (dram__bytes_read.sum + write) from the
+    committed ncu summary of this workload, or None when there is none or the
+    decode kernel's source changed since it was captured."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", f"decode_stream_tc_{w.name.replace('-decode', '')}.md")
+    csrc = os.path.join(ROOT, "bit_asymmetric_kv_quantize_b200", "csrc")
+    try:
+        text = open(prof).read()
+        h = hashlib.sha256()
+        for f in ("kivi_decode_tc.cu", "kivi_internal.cuh"):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    except OSError:
+        return None
+    for line in text.splitlines():
+        if line.startswith("traffic_bytes_per_launch:"):
+            parts = line.replace("(", " ").replace(")", " ").split()
+            if parts and parts[-1] == h.hexdigest()[:16]:
+                return int(parts[1])
+    return None
+
+
 def algorithmic_bytes(w: W.Workload, n_q: int, r: int) -> int:
     """Bytes one decode call must move: every code, scale and zero of the
     quantized store, the window tokens, q in and out (per unit: K codes
@@ -341,7 +363,7 @@ def run_kivi(args, rank, world, local):
             "roofline": {
                 "kernel": "decode_split", "bound": "hbm", "achieved": achieved, "peak": peak,
                 "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": None,
+                "traffic": (profiled_traffic(w) if args.kernel == "default" else None),
                 "algorithmic_bytes_per_launch": bytes_total / args.steps,
                 "avg_launch_us": split_total_ms * 1e3 / args.steps,
             },
