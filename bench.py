@@ -15,8 +15,11 @@ depth; 4.7 GB) are visited round-robin, so each step reads a cache that is
 not L2-resident (inputs larger than the 126 MB L2).
 
 Output: one JSON line (rank 0).  `value` = decode tokens/s over all ranks
-(B tokens per step per rank); `roofline` = the split kernel's algorithmic
-bytes / its CUDA-event time vs measured HBM peak; `e2e` = the same loop with
+(B tokens per step per rank) over K steps with nothing recorded between
+launches; `roofline` = the decode kernel's algorithmic bytes / its CUDA-event
+time vs measured HBM peak, from K further steps with events recorded around
+each decode launch (events serialize consecutive launches, so this pass runs
+apart from the headline one); `e2e` = the same loop with
 the step's inputs copied from pinned host memory and the output copied back
 inside the timed region; `cpu_baseline` = the CPU oracle on a bounded sample
 of the same workload.  `--impl reference` times the CPU oracle alone.
@@ -207,7 +210,7 @@ def run_kivi(args, rank, world, local):
         w = w.with_(steps=0)
     n_layers = max(1, args.layers)
     e2e_steps = 0 if args.no_e2e else min(args.steps, 1024)
-    per_layer = -(-(args.warmup + args.steps + e2e_steps) // n_layers) + 1
+    per_layer = -(-(args.warmup + 2 * args.steps + e2e_steps) // n_layers) + 1
     capacity = -(-(w.T + per_layer) // w.R) * w.R
     Kp, Vp = W.prompt_kv(w, device=device)
     caches = []
@@ -277,23 +280,31 @@ def run_kivi(args, rank, world, local):
         evs.append((e0, e1))
     torch.cuda.synchronize(device)
     ev_handles = [(e0.cuda_event, e1.cuda_event) for e0, e1 in evs]
-    fills = []
+    # (1) the timed steps: nothing between consecutive launches, so a decode
+    # launch may overlap the previous one's drain (programmatic serialization)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     n_launch[0] = 0
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         t0.record(stream)
         for j in range(args.steps):
-            i = args.warmup + j
-            step(i, ev_handles[j])
-            c = caches[i % n_layers]
-            fills.append((c.n_q, c.r))
+            step(args.warmup + j)
         t1.record(stream)
         timed_launches = n_launch[0]
         torch.cuda.synchronize(device)
-    L.kivi_set_timing_events(None, None)
     barrier()
     ms = t0.elapsed_time(t1)
+    # (2) the roofline: as many further steps, CUDA events recorded by the
+    # library around each decode launch (these serialize the launches)
+    fills = []
+    for j in range(args.steps):
+        i = args.warmup + args.steps + j
+        step(i, ev_handles[j])
+        c = caches[i % n_layers]
+        fills.append((c.n_q, c.r))
+    torch.cuda.synchronize(device)
+    L.kivi_set_timing_events(None, None)
+    barrier()
     split_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
     ms_max = max_over_ranks(ms, world, device)
 
@@ -315,7 +326,7 @@ def run_kivi(args, rank, world, local):
         h2d = 3 * ks[0].numel() * ks[0].element_size()
         d2h = out.numel() * out.element_size()
         n_e2e = e2e_steps
-        base = args.warmup + args.steps
+        base = args.warmup + 2 * args.steps
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)

@@ -280,6 +280,12 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
   const long long G0 = (long long)cta * W;
   const long long G1 = min(total, G0 + W);
 
+  // launched with programmatic stream serialization: the CTAs may start
+  // while the preceding grid drains; every thread waits for it to complete
+  // (and its writes to be visible) before touching global memory, and the
+  // next grid may be scheduled as soon as SM room frees up
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     for (int s = 0; s < G::NSTAGE; ++s) {
       mbar_init(&full[s], 1);
@@ -1284,8 +1290,19 @@ cudaError_t tc_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_
     if (e != cudaSuccess) return e;
   }
   if (e0) cudaEventRecord(e0, s);
-  decode_stream_tc<D, BITS, GQ, T><<<a.n_cta, G::THREADS, G::SMEM_B, s>>>(a, tmK, tmV);
-  cudaError_t err = cudaGetLastError();
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)a.n_cta);
+  cfg.blockDim = dim3(G::THREADS);
+  cfg.dynamicSmemBytes = G::SMEM_B;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, decode_stream_tc<D, BITS, GQ, T>, a, tmK, tmV);
+  if (err == cudaSuccess) err = cudaGetLastError();
   if (e1) cudaEventRecord(e1, s);
   return err;
 }
