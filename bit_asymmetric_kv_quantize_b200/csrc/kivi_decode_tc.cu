@@ -136,8 +136,10 @@ struct Geo {
   static constexpr int NBX = D / BW;
   static constexpr int RB = BW * 2;
   static constexpr int BOX_B = WT * RB;
-  static constexpr int WIN_B = 2 * NBX * BOX_B;
-  static_assert(WIN_B <= STAGE_B, "a window stage fits one ring slot");
+  static constexpr int WTILE_B = 2 * NBX * BOX_B;     // one 32-token window tile (K, V)
+  static constexpr int WPS = STAGE_B / WTILE_B;       // window tiles per stage
+  static_assert(WPS >= 1, "a window tile fits one ring slot");
+  static_assert(WTILE_B % 1024 == 0, "window tiles keep the 1024-byte alignment");
   static_assert(STAGE_B % 1024 == 0, "swizzled boxes start on 1024-byte boundaries");
 };
 
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
           if constexpr (sizeof(T) == 2) {
             // this CTA owns the unit's residual window: stream it through
             // the ring, WT tokens of K and of V per stage, one row per copy
-            for (int w0 = 0; w0 < a.r; w0 += G::WT, ++st) {
+            for (int w0 = 0; w0 < a.r; w0 += G::WT * G::WPS, ++st) {
               const int s = (int)(st % G::NSTAGE);
               if (st >= G::NSTAGE &&
                   !mbar_wait(&empty[s], (uint32_t)(((st / G::NSTAGE) - 1) & 1))) {
@@ -369,13 +371,17 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
               }
               if (*(volatile int*)&flag[0]) break;
               unsigned char* buf = smem + s * G::STAGE_B;
+              const int ntile = min(G::WPS, (a.r - w0 + G::WT - 1) / G::WT);
               asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-              mbar_expect_tx(&full[s], (uint32_t)G::WIN_B);
-              const int y = (int)(u * c.R + w0);  // row of the [units * R][D] window
+              mbar_expect_tx(&full[s], (uint32_t)(ntile * G::WTILE_B));
+              for (int j = 0; j < ntile; ++j) {
+                unsigned char* tb = buf + j * G::WTILE_B;
+                const int y = (int)(u * c.R + w0 + j * G::WT);  // row of the [units * R][D] window
 #pragma unroll
-              for (int bx = 0; bx < G::NBX; ++bx) {
-                tma_2d(buf + bx * G::BOX_B, &tmK, bx * G::BW, y, &full[s]);
-                tma_2d(buf + (G::NBX + bx) * G::BOX_B, &tmV, bx * G::BW, y, &full[s]);
+                for (int bx = 0; bx < G::NBX; ++bx) {
+                  tma_2d(tb + bx * G::BOX_B, &tmK, bx * G::BW, y, &full[s]);
+                  tma_2d(tb + (G::NBX + bx) * G::BOX_B, &tmV, bx * G::BW, y, &full[s]);
+                }
               }
             }
           } else {
@@ -937,14 +943,15 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
         }
       };
 
-      // ---- fp16 residual window on tensor cores: window stage k goes to warp
-      // k % kW, which first flushes its quantized-tile state and then keeps a
-      // separate softmax state for the window (plain q and p, scale 1)
+      // ---- fp16 residual window on tensor cores: window tile k (WPS per
+      // stage) goes to warp k % kW, which first flushes its quantized-tile
+      // state and then keeps a separate softmax state for the window (plain q
+      // and p, scale 1)
       bool wmode = false;
       if constexpr (sizeof(T) == 2) {
         if (window_owner) {
           int k = 0;
-          for (int w0 = 0; w0 < a.r; w0 += G::WT, ++st, ++k) {
+          for (int w0 = 0; w0 < a.r; w0 += G::WT * G::WPS, ++st) {
             if (*(volatile int*)&flag[0]) break;
             const int s = (int)(st % G::NSTAGE);
             const bool ok = mbar_wait(&full[s], (uint32_t)((st / G::NSTAGE) & 1));
@@ -952,6 +959,9 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
               if (lane == 0) atomicExch(&flag[0], 1);
               break;
             }
+            for (int j = 0; j < G::WPS; ++j, ++k) {
+            const int tw0 = w0 + j * G::WT;
+            if (tw0 >= a.r) break;
             if (k % kW == warp) {
               if (!wmode) {
                 flush_code();
@@ -988,7 +998,8 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
                 }
                 __syncwarp();
               }
-              window_tile(smem + s * G::STAGE_B, min(G::WT, a.r - w0));
+              window_tile(smem + s * G::STAGE_B + j * G::WTILE_B, min(G::WT, a.r - tw0));
+            }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
