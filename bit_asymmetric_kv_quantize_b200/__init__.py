@@ -32,7 +32,8 @@ EXPORTED = (
     "kivi_buffer_sizes", "kivi_cache_init", "kivi_quantize_prefill", "kivi_append_token",
     "kivi_decode_workspace_bytes", "kivi_decode_attention", "kivi_decode_attention_simt",
     "kivi_set_timing_events", "kivi_decode_num_splits", "kivi_status_string",
-    "kivi_decode_attention_noalloc", "kivi_append_decode",
+    "kivi_decode_attention_noalloc", "kivi_append_decode", "kivi_dev_state_init",
+    "kivi_append_decode_dev",
 )
 
 
@@ -84,6 +85,9 @@ def lib() -> ctypes.CDLL:
             L.kivi_decode_attention_simt.argtypes = dec
             L.kivi_decode_attention_noalloc.argtypes = [cp, vp, ci, ctypes.c_float, vp, vp]
             L.kivi_append_decode.argtypes = [cp, vp, vp, vp, ci, ctypes.c_float, vp, vp, sz, vp]
+            L.kivi_dev_state_init.argtypes = [cp, vp, vp]
+            L.kivi_append_decode_dev.argtypes = [cp, vp, vp, vp, vp, ci, ctypes.c_float, vp, vp, sz,
+                                                 vp]
             L.kivi_set_timing_events.argtypes = [vp, vp]
             L.kivi_set_timing_events.restype = None
             L.kivi_decode_num_splits.argtypes = [cp, ci]
@@ -139,6 +143,7 @@ class KiviCache:
         _check(lib().kivi_cache_init(ctypes.byref(self._c), ctypes.byref(self._dims),
                                      ctypes.byref(ptrs)), "kivi_cache_init")
         self._ws: Optional[torch.Tensor] = None
+        self._ws_dev: Optional[torch.Tensor] = None
         E = 32 // bits
         Tq = capacity - R
         self.B, self.Hkv, self.D, self.bits, self.R, self.capacity = B, Hkv, D, bits, R, capacity
@@ -224,6 +229,46 @@ class KiviCache:
         with torch.cuda.device(self.device):
             _check(fn(ctypes.byref(self._c), pq, Hq, float(softmax_scale), po, ws.data_ptr(),
                       ws.numel(), self._stream()), "kivi_decode_attention")
+        return out
+
+    # -- device-resident counters (graph-capturable decode loop)
+    def dev_state(self) -> torch.Tensor:
+        """A 16-byte device tensor holding this cache's counters (n_q, r, status)."""
+        st = torch.zeros(16, dtype=torch.uint8, device=self.device)
+        with torch.cuda.device(self.device):
+            _check(lib().kivi_dev_state_init(ctypes.byref(self._c), st.data_ptr(), self._stream()),
+                   "kivi_dev_state_init")
+        return st
+
+    def load_dev_state(self, st: torch.Tensor) -> None:
+        """Copy the counters from a device state back into the host struct (synchronizes)."""
+        v = st.cpu()
+        n_q = int(v[:8].view(torch.int64)[0])
+        r, status = (int(x) for x in v[8:16].view(torch.int32))
+        if status != 0:
+            raise KiviError(4, "device state: cache full")
+        self._c.n_q, self._c.r = n_q, r
+
+    def append_decode_dev(self, st: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                          q: torch.Tensor, softmax_scale: float,
+                          out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """append + decode with the counters in `st` (see kivi_append_decode_dev)."""
+        shape = (self.B, self.Hkv, self.D)
+        pk, pv = self._arg(k, shape, "k"), self._arg(v, shape, "v")
+        Hq = q.shape[1]
+        pq = self._arg(q, (self.B, Hq, self.D), "q")
+        if out is None:
+            out = torch.empty_like(q)
+        po = self._arg(out, (self.B, Hq, self.D), "out")
+        need = self.workspace_bytes(Hq)
+        if self._ws_dev is None or self._ws_dev.numel() < need:
+            self._ws_dev = torch.zeros(need, dtype=torch.uint8, device=self.device)
+        ws = self._ws_dev
+        with torch.cuda.device(self.device):
+            _check(lib().kivi_append_decode_dev(ctypes.byref(self._c), st.data_ptr(), pk, pv, pq,
+                                                Hq, float(softmax_scale), po, ws.data_ptr(),
+                                                ws.numel(), self._stream()),
+                   "kivi_append_decode_dev")
         return out
 
     def append_decode(self, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor,

@@ -97,29 +97,13 @@ void plan_splits(const kivi_cache* c, int sms, int* n_split, int* tiles_per_spli
   *n_split = (int)((tiles + tps - 1) / tps);
 }
 
-// Tensor-core kernel: persistent stream-K plan.  Every unit is laid out as
-// n_q/32 work indices (its quantized 32-token tiles) followed by
-// kWinWeight * ceil(r/32) + kMergeWeight indices standing for its residual
-// window and for the end-of-unit merge; the units' indices end to end are
-// cut into n_cta equal ranges of W >= 12.  A unit is covered by the CTAs
-// whose ranges meet its tiles or its window start index -- at most
-// ceil((n_q/32 + 1) / W) + 1 CTA segments, each writing one partial -- and
-// the last of them also takes the window.  Measured on B200 (per-CTA
-// timelines): a 32-token window tile costs about two quantized tiles (fp16,
-// tensor cores) or three (fp32, CUDA cores) and the end of a unit segment
-// (partial write, arrival, merge) about eight, so a CTA whose range crosses
-// a unit boundary gets correspondingly fewer tiles.
+// Tensor-core kernel: persistent stream-K plan (kivi::plan_stream_core, the
+// same function the kernel runs in device-counter mode).  A unit is covered
+// by the CTAs whose ranges meet its tiles or its window start index -- at
+// most ceil((n_q/32 + 1) / W) + 1 CTA segments, each writing one partial --
+// and the last of them also takes the window.
 constexpr int kTcCtasPerSm = 3;  // upper bound; the kernel instance decides
-constexpr int kWinWeight = 3;    // cost of a window tile, in quantized tiles (fp32, CUDA cores)
-constexpr int kWinWeightF16 = 2;  // same, fp16 window on tensor cores
-constexpr int kMergeWeight = 8;  // cost of a unit end, in quantized tiles
-
-struct StreamPlan {
-  int n_cta;
-  long long W;
-  int max_seg;
-  int win_weight;
-};
+using kivi::StreamPlan;
 
 long long ceil_div(long long x, long long y) { return (x + y - 1) / y; }
 
@@ -132,34 +116,23 @@ int tc_seg_cap(const kivi_dims& d, int sms) {
   return (int)s + 1;
 }
 
+// CTAs of the tensor-core kernel instance that run at once.
+long long tc_ctas(int sms, int ctas_per_sm) {
+  return (long long)(ctas_per_sm < kTcCtasPerSm ? ctas_per_sm : kTcCtasPerSm) * sms;
+}
+
 // ctas_per_sm: resident CTAs per SM of the kernel instance (<= kTcCtasPerSm);
 // seg_cap: largest number of partial slots per unit the workspace holds.
 void plan_stream(const kivi_cache* c, int sms, int ctas_per_sm, int seg_cap, StreamPlan* p) {
-  const long long units = (long long)c->dims.B * c->dims.Hkv;
-  const long long n_qt = c->n_q / kivi::kTile;
-  const int wtw = c->dims.dtype == KIVI_F16 ? kWinWeightF16 : kWinWeight;
-  const int ww = (c->r > 0 ? wtw * (int)ceil_div(c->r, kivi::kTile) : 1) + kMergeWeight;
-  const long long UP = n_qt + ww;
-  const long long total = units * UP;
-  const long long P =
-      (long long)(ctas_per_sm < kTcCtasPerSm ? ctas_per_sm : kTcCtasPerSm) * sms;
-  long long W = ceil_div(total, P);
-  if (W < 12) W = 12;  // at least one full stage per CTA
-  if (seg_cap <= 1) {
-    W = UP;  // one CTA per unit: ranges align with the units
-  } else if (ceil_div(n_qt + 1, W) + 1 > seg_cap) {
-    W = ceil_div(n_qt + 1, seg_cap - 1);
-  }
-  p->W = W;
-  p->win_weight = ww;
-  p->n_cta = (int)ceil_div(total, W);
-  p->max_seg = (W % UP == 0) ? 1 : (int)(ceil_div(n_qt + 1, W) + 1);
+  *p = kivi::plan_stream_core((long long)c->dims.B * c->dims.Hkv, c->n_q, c->r,
+                              c->dims.dtype == KIVI_F16, tc_ctas(sms, ctas_per_sm), seg_cap);
 }
 
-// Workspace: per-unit arrival counters (8 bytes each, 16-byte aligned block)
-// followed by the split partials [B*Hq][n_split][D + 2] floats.
+// Workspace: per-unit arrival counters and one grid counter (8 bytes each,
+// 16-byte aligned block) followed by the split partials [B*Hq][n_split][D + 2]
+// floats.
 size_t counter_bytes(const kivi_dims& d) {
-  return ((size_t)d.B * d.Hkv * 8 + 15) / 16 * 16;
+  return ((size_t)(d.B * d.Hkv + 1) * 8 + 15) / 16 * 16;
 }
 
 int ws_splits(const kivi_dims& d, int sms) {
@@ -184,12 +157,15 @@ unsigned int next_epoch() {
 // the partials; the split count is capped at `split_cap`.
 int decode_launch(const kivi_cache* c, const void* q, int Hq, float softmax_scale, void* out,
                   void* ws, int split_cap, int sms, void* stream, bool simt,
-                  const void* new_k = nullptr, const void* new_v = nullptr, int new_slot = 0) {
+                  const void* new_k = nullptr, const void* new_v = nullptr, int new_slot = 0,
+                  void* dev_state = nullptr) {
   const int gq = Hq / c->dims.Hkv;
   DecodeArgs a;
   a.new_k = new_k;
   a.new_v = new_v;
   a.new_slot = new_slot;
+  a.dev_state = (kivi::DevState*)dev_state;
+  a.seg_cap = split_cap;
   a.c = view(c);
   a.q = q;
   a.out = out;
@@ -221,7 +197,9 @@ int decode_launch(const kivi_cache* c, const void* q, int Hq, float softmax_scal
     if (kivi::decode_tc_ctas_per_sm(a, &occ) != cudaSuccess) return KIVI_ERR_CUDA;
     StreamPlan sp;
     plan_stream(c, sms, occ, split_cap, &sp);
-    a.n_cta = sp.n_cta;
+    // device counters: the kernel plans on the device over a full grid
+    a.n_cta = dev_state ? (int)tc_ctas(sms, occ) : sp.n_cta;
+    if (dev_state) a.r = 1;  // any post-append cache has a window (tensor maps)
     a.tiles_per_cta = sp.W;
     a.max_seg = sp.max_seg;
     a.win_weight = sp.win_weight;
@@ -397,7 +375,9 @@ int kivi_append_decode(kivi_cache* cache, const void* k, const void* v, const vo
   if (sms <= 0) return KIVI_ERR_CUDA;
   if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(cache->dims, Hq, sms))
     return KIVI_ERR_WORKSPACE;
-  if (cache->r == cache->dims.R) {  // flush due: its own launch, then decode
+  // flush due, or a token not 16-byte aligned (the kernel copies it in
+  // 16-byte pieces): the append as its own launch, then decode
+  if (cache->r == cache->dims.R || ((uintptr_t)k & 15) || ((uintptr_t)v & 15)) {
     rc = kivi_append_token(cache, k, v, stream);
     if (rc) return rc;
     return decode_launch(cache, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms),
@@ -407,6 +387,38 @@ int kivi_append_decode(kivi_cache* cache, const void* k, const void* v, const vo
                      stream, false, k, v, cache->r);
   if (rc == KIVI_OK) cache->r = after.r;
   return rc;
+}
+
+int kivi_dev_state_init(const kivi_cache* cache, void* state, void* stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!state || ((uintptr_t)state & 15)) return KIVI_ERR_ARG;
+  return kivi::launch_set_state((kivi::DevState*)state, cache->n_q, cache->r,
+                                (cudaStream_t)stream) == cudaSuccess
+             ? KIVI_OK
+             : KIVI_ERR_CUDA;
+}
+
+int kivi_append_decode_dev(const kivi_cache* cache, void* state, const void* k, const void* v,
+                           const void* q, int Hq, float softmax_scale, void* out,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!state || ((uintptr_t)state & 15) || !k || !v) return KIVI_ERR_ARG;
+  kivi_cache after = *cache;  // any post-append state passes the decode checks
+  after.r = 1;
+  rc = decode_checks(&after, q, Hq, out);
+  if (rc) return rc;
+  const int sms = device_sms();
+  if (sms <= 0) return KIVI_ERR_CUDA;
+  if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(cache->dims, Hq, sms))
+    return KIVI_ERR_WORKSPACE;
+  if (kivi::launch_append_dev(view(cache), cache->dims.B * cache->dims.Hkv, cache->dims.D,
+                              cache->dims.bits, cache->dims.dtype, k, v,
+                              (const kivi::DevState*)state, (cudaStream_t)stream) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  return decode_launch(&after, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms),
+                       sms, stream, false, nullptr, nullptr, 0, state);
 }
 
 int kivi_decode_attention_simt(const kivi_cache* cache, const void* q, int Hq,

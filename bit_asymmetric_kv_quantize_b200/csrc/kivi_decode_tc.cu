@@ -244,7 +244,7 @@ __device__ __forceinline__ void consumers_sync() {
 
 template <int D, int BITS, int GQ, typename T>
 __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::MIN_CTAS)
-    decode_stream_tc(DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
+    decode_stream_tc(const DecodeArgs args, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV) {
   using G = Geo<D, BITS, GQ>;
   using PR = Pairs<BITS>;
@@ -264,6 +264,32 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
   const int cta = blockIdx.x;
+
+  // launched with programmatic stream serialization: the CTAs may start
+  // while the preceding grid drains; every thread waits for it to complete
+  // (and its writes to be visible) before touching global memory, and the
+  // next grid may be scheduled as soon as SM room frees up
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  DecodeArgs a = args;
+  const bool dev = args.dev_state != nullptr;
+  if (dev) {
+    // device counters as the preceding append launch found them; decode the
+    // cache after that append (it flushed when r was R)
+    const DevState st0 = *args.dev_state;
+    if (st0.status != 0 || st0.n_q + st0.r + 1 > args.c.Tq + args.c.R) return;  // cache full
+    const bool fl = st0.r == args.c.R;
+    a.n_q = fl ? st0.n_q + args.c.R : st0.n_q;
+    a.r = fl ? 1 : st0.r + 1;
+    const StreamPlan pl =
+        plan_stream_core(args.units, a.n_q, a.r, sizeof(T) == 2, gridDim.x, args.seg_cap);
+    a.tiles_per_cta = pl.W;
+    a.win_weight = pl.win_weight;
+    a.max_seg = pl.max_seg;
+    a.n_split = pl.max_seg;
+    a.new_k = nullptr;  // the append launch wrote the token
+  }
   const int Hq = a.Hkv * GQ;
   const CacheView& c = a.c;
 
@@ -282,12 +308,6 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
   const long long G0 = (long long)cta * W;
   const long long G1 = min(total, G0 + W);
 
-  // launched with programmatic stream serialization: the CTAs may start
-  // while the preceding grid drains; every thread waits for it to complete
-  // (and its writes to be visible) before touching global memory, and the
-  // next grid may be scheduled as soon as SM room frees up
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     for (int s = 0; s < G::NSTAGE; ++s) {
       mbar_init(&full[s], 1);
@@ -298,10 +318,11 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
     flag[0] = (sizeof(T) == 2 && (smem_u32(smem) & 1023u) != 0) ? 1 : 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (a.new_k != nullptr) {
-    // fused append: the CTA that owns a unit's window writes the unit's new
-    // token into window slot new_slot; the proxy fence and the barrier below
-    // order these writes before this CTA's tensor copies and loads of the window
+  if (sizeof(T) == 4 && a.new_k != nullptr) {
+    // fused append, fp32 window (read by generic loads after the barrier
+    // below): the CTA that owns a unit's window writes the unit's new token
+    // into window slot new_slot.  (fp16: the producer writes it just before
+    // the window's tensor copies.)
     for (long long u = G0 / UP; G0 < G1 && u <= (G1 - 1) / UP; ++u) {
       if (cta != (u * UP + n_qt) / W) continue;
       T* kr = reinterpret_cast<T*>(c.k_res) + (u * c.R + a.new_slot) * D;
@@ -313,7 +334,6 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
         vr[i] = vn[i];
       }
     }
-    asm volatile("fence.proxy.async.global;" ::: "memory");
   }
   if (warp < kW) {
     // fragment columns of absent heads stay zero
@@ -361,7 +381,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
           const T* vr = reinterpret_cast<const T*>(c.v_res) + u * c.R * D;
           if constexpr (sizeof(T) == 2) {
             // this CTA owns the unit's residual window: stream it through
-            // the ring, WT tokens of K and of V per stage, one row per copy
+            // the ring, WT tokens of K and of V per stage
             for (int w0 = 0; w0 < a.r; w0 += G::WT * G::WPS, ++st) {
               const int s = (int)(st % G::NSTAGE);
               if (st >= G::NSTAGE &&
@@ -789,18 +809,35 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
       // ---- one fp16 window stage of nt tokens on tensor cores: S = K q
       // (K rows by ldmatrix), the same online softmax, O += V^T p (V^T by
       // ldmatrix.trans); rows past nt read row 0 and are masked out
-      auto window_tile = [&](const unsigned char* wbuf, int nt) {
-        const unsigned char* Kw = wbuf;
-        const unsigned char* Vw = wbuf + G::NBX * G::BOX_B;
+      auto window_tile = [&](unsigned char* wbuf, int nt, int tw0) {
+        unsigned char* Kw = wbuf;
+        unsigned char* Vw = wbuf + G::NBX * G::BOX_B;
         // address of 16-byte chunk cc (channels 8 cc .. 8 cc + 7) of row tok:
         // the swizzle XORs the chunk index with address bits 7.. of the row
-        auto chunk = [&](const unsigned char* base, int tok, int cc) -> const unsigned char* {
+        auto chunk = [&](unsigned char* base, int tok, int cc) -> unsigned char* {
           constexpr int CPR = G::RB / 16;  // chunks per box row
-          const unsigned char* row = base + (cc / CPR) * G::BOX_B + tok * G::RB;
+          unsigned char* row = base + (cc / CPR) * G::BOX_B + tok * G::RB;
           const uint32_t ra = smem_u32(row);
           const int x = G::RB == 128 ? (int)((ra >> 7) & 7u) : (int)((ra >> 7) & 3u);
           return row + (((cc % CPR) ^ x) << 4);
         };
+        if (a.new_k != nullptr && a.new_slot >= tw0 && a.new_slot < tw0 + G::WT) {
+          // fused append: the copies brought the window before this call's
+          // token; put the token into its row here and into the cache for
+          // later calls (16 bytes per lane, K then V)
+          constexpr int NC = D * 2 / 16;  // 16-byte chunks per row
+          const int row = a.new_slot - tw0;
+          if (lane < 2 * NC) {
+            const int cc = lane % NC;
+            const bool isv = lane >= NC;
+            const uint4 x = reinterpret_cast<const uint4*>(
+                reinterpret_cast<const T*>(isv ? a.new_v : a.new_k) + u * D)[cc];
+            *reinterpret_cast<uint4*>(chunk(isv ? Vw : Kw, row, cc)) = x;
+            T* dst = reinterpret_cast<T*>(isv ? c.v_res : c.k_res) + (u * c.R + a.new_slot) * D;
+            reinterpret_cast<uint4*>(dst)[cc] = x;
+          }
+          __syncwarp();
+        }
         float dq[NPB][2][4];
 #pragma unroll
         for (int p = 0; p < NPB; ++p)
@@ -998,7 +1035,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
                 }
                 __syncwarp();
               }
-              window_tile(smem + s * G::STAGE_B + j * G::WTILE_B, min(G::WT, a.r - tw0));
+              window_tile(smem + s * G::STAGE_B + j * G::WTILE_B, min(G::WT, a.r - tw0), tw0);
             }
             }
             __syncwarp();
@@ -1200,7 +1237,13 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
       }
       // ---- arrival; the last segment of the unit merges all its partials
       consumers_sync<kW>();
-      if (tid == 0) flag[1] = arrive_unit(a.ctr + u, a.epoch, n_seg);
+      if (tid == 0) {
+        if (dev) {
+          flag[1] = arrive_unit_reset(a.ctr + u, n_seg);
+        } else {
+          flag[1] = arrive_unit(a.ctr + u, a.epoch, n_seg);
+        }
+      }
       consumers_sync<kW>();
       const int last = flag[1];
       if (last != 0) {
@@ -1220,6 +1263,11 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
     }
   }
   __syncthreads();
+  if (dev && tid == 0 && arrive_unit_reset(a.ctr + a.units, gridDim.x) == 1) {
+    // the last CTA to finish advances the device counters
+    args.dev_state->n_q = a.n_q;
+    args.dev_state->r = a.r;
+  }
 }
 
 // Opt in to the kernel's dynamic shared memory and return how many of its

@@ -70,6 +70,59 @@ cudaError_t launch_append(const CacheView& c, int units, int D, int bits, int dt
                           const void* k, const void* v, long long n_q, int slot, bool flush,
                           cudaStream_t s);
 
+// Device-resident counters of one cache (layout of kivi_dev_state).
+struct DevState {
+  long long n_q;
+  int r;
+  int status;  // 0, or 1 once an append found no room (nothing written)
+};
+// Append reading (n_q, r) from `st` on the device (flush when r == R);
+// the counters themselves are advanced by the decode that follows.
+cudaError_t launch_append_dev(const CacheView& c, int units, int D, int bits, int dtype,
+                              const void* k, const void* v, const DevState* st, cudaStream_t s);
+cudaError_t launch_set_state(DevState* st, long long n_q, int r, cudaStream_t s);
+
+// ---- stream-K plan of the tensor-core decode (host and device) -----------
+// Every unit is laid out as n_q/32 work indices (its quantized tiles)
+// followed by kWinWeight * ceil(r/32) + kMergeWeight indices standing for its
+// residual window and its end-of-unit merge; the units' indices end to end
+// are cut into equal ranges of W >= 12, one per CTA.  Measured on B200
+// (per-CTA timelines): a 32-token window tile costs about two quantized tiles
+// (fp16, tensor cores) or three (fp32, CUDA cores) and the end of a unit
+// segment (partial write, arrival, merge) about eight, so a CTA whose range
+// crosses a unit boundary gets correspondingly fewer tiles.
+constexpr int kWinWeight = 3;     // fp32 window tile, CUDA cores
+constexpr int kWinWeightF16 = 2;  // fp16 window tile, tensor cores
+constexpr int kMergeWeight = 8;   // one unit end
+struct StreamPlan {
+  int n_cta;
+  long long W;
+  int max_seg;
+  int win_weight;
+};
+// P: CTAs that run at once; seg_cap: partial slots per unit in the workspace.
+__host__ __device__ inline StreamPlan plan_stream_core(long long units, long long n_q, int r,
+                                                       bool f16, long long P, int seg_cap) {
+  StreamPlan p;
+  const long long n_qt = n_q / kTile;
+  const int wtw = f16 ? kWinWeightF16 : kWinWeight;
+  const int ww = (r > 0 ? wtw * (int)((r + kTile - 1) / kTile) : 1) + kMergeWeight;
+  const long long UP = n_qt + ww;
+  const long long total = units * UP;
+  long long W = (total + P - 1) / P;
+  if (W < 12) W = 12;  // at least one full stage per CTA
+  if (seg_cap <= 1) {
+    W = UP;  // one CTA per unit: ranges align with the units
+  } else if ((n_qt + 1 + W - 1) / W + 1 > seg_cap) {
+    W = (n_qt + 1 + seg_cap - 2) / (seg_cap - 1);
+  }
+  p.W = W;
+  p.win_weight = ww;
+  p.n_cta = (int)((total + W - 1) / W);
+  p.max_seg = (W % UP == 0) ? 1 : (int)((n_qt + 1 + W - 1) / W + 1);
+  return p;
+}
+
 struct DecodeArgs {
   CacheView c;
   const void* q;   // [B][Hq][D]
@@ -104,6 +157,14 @@ struct DecodeArgs {
   const void* new_k;
   const void* new_v;
   int new_slot;
+  // device-counter mode (tensor-core kernel): when dev_state is non-null the
+  // kernel reads (n_q, r) before the append from it, decodes over the cache
+  // after the append (which an earlier launch performed), plans the split on
+  // the device over its gridDim.x CTAs with seg_cap partial slots, writes
+  // the new counters back, and counts arrivals in self-resetting counters
+  // (the workspace's counter block must start zeroed)
+  DevState* dev_state;
+  int seg_cap;
 };
 
 constexpr float kNaN = __builtin_nanf("");
@@ -173,6 +234,18 @@ __device__ __forceinline__ float merge_partials(const float* P0, long long strid
     M = Mb;
   }
   return num / den;
+}
+
+// Arrival at a counter that starts at zero and is reset to zero by the n-th
+// arrival (device-counter mode, where launches replay with the same
+// arguments and cannot tag counters with a per-call epoch).  Same memory
+// ordering as arrive_unit.  Returns 1 for the n-th arrival, else 0.
+__device__ __forceinline__ int arrive_unit_reset(unsigned long long* ctr, long long n) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], 1;" : "=l"(old) : "l"(ctr) : "memory");
+  if ((long long)old + 1 != n) return 0;
+  asm volatile("st.relaxed.gpu.global.u64 [%0], 0;" ::"l"(ctr) : "memory");
+  return 1;
 }
 
 // End of a split CTA, after it wrote its (m, l, acc[D]) partials: the last CTA

@@ -136,24 +136,46 @@ __global__ void __launch_bounds__(D) prefill_kernel(CacheView c, const T* __rest
   }
 }
 
-// grid (units).  If `flush`, quantize the R window tokens into store
-// positions n_q..n_q+R-1 first; then write the new token into window `slot`.
+// grid (tiles, units) with tiles = R/32 when a flush may be due, else 1.
+// If `flush`, block x quantizes window tile x (tokens 32x..32x+31) into store
+// positions n_q + 32x..; block 0 then writes the new token into window
+// `slot` (its own tile has been read by then).  Device mode (st != null):
+// n_q and r come from st -- flush when r == R, slot = flush ? 0 : r -- and a
+// full cache is left alone with st->status = 1.
 template <int D, int BITS, typename T>
 __global__ void __launch_bounds__(D) append_kernel(CacheView c, const T* __restrict__ k,
                                                    const T* __restrict__ v, long long n_q,
-                                                   int slot, int flush) {
+                                                   int slot, int flush, DevState* st) {
   __shared__ uint8_t ck[kTile * D];
   __shared__ uint8_t cv[kTile * D];
-  const long long unit = blockIdx.x;
+  if (st != nullptr) {
+    const long long nq = st->n_q;
+    const int r = st->r;
+    if (st->status != 0 || nq + r + 1 > c.Tq + c.R) {
+      if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) st->status = 1;
+      return;
+    }
+    flush = r == c.R;
+    n_q = nq;
+    slot = flush ? 0 : r;
+  }
+  const long long unit = blockIdx.y;
+  const int tile = blockIdx.x;
   T* kr = reinterpret_cast<T*>(c.k_res) + unit * c.R * D;
   T* vr = reinterpret_cast<T*>(c.v_res) + unit * c.R * D;
-  if (flush) {
-    for (int tile = 0; tile < c.R / kTile; ++tile)
-      quantize_tile<D, BITS, T>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
-                                n_q + tile * kTile, ck, cv);
+  if (flush)
+    quantize_tile<D, BITS, T>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
+                              n_q + tile * kTile, ck, cv);
+  if (tile == 0) {
+    kr[(long long)slot * D + threadIdx.x] = k[unit * D + threadIdx.x];
+    vr[(long long)slot * D + threadIdx.x] = v[unit * D + threadIdx.x];
   }
-  kr[(long long)slot * D + threadIdx.x] = k[unit * D + threadIdx.x];
-  vr[(long long)slot * D + threadIdx.x] = v[unit * D + threadIdx.x];
+}
+
+__global__ void set_state_kernel(DevState* st, long long n_q, int r) {
+  st->n_q = n_q;
+  st->r = r;
+  st->status = 0;
 }
 
 template <int D, int BITS, typename T>
@@ -166,9 +188,10 @@ cudaError_t prefill_t(const CacheView& c, int units, const void* K, const void* 
 
 template <int D, int BITS, typename T>
 cudaError_t append_t(const CacheView& c, int units, const void* k, const void* v, long long n_q,
-                     int slot, bool flush, cudaStream_t s) {
-  append_kernel<D, BITS, T><<<units, D, 0, s>>>(c, (const T*)k, (const T*)v, n_q, slot,
-                                                flush ? 1 : 0);
+                     int slot, bool flush, DevState* st, cudaStream_t s) {
+  const dim3 grid((unsigned)((flush || st) ? c.R / kTile : 1), (unsigned)units);
+  append_kernel<D, BITS, T><<<grid, D, 0, s>>>(c, (const T*)k, (const T*)v, n_q, slot,
+                                               flush ? 1 : 0, st);
   return cudaGetLastError();
 }
 
@@ -185,12 +208,22 @@ cudaError_t prefill_d(int D, const CacheView& c, int units, const void* K, const
 
 template <int BITS, typename T>
 cudaError_t append_d(int D, const CacheView& c, int units, const void* k, const void* v,
-                     long long n_q, int slot, bool flush, cudaStream_t s) {
+                     long long n_q, int slot, bool flush, DevState* st, cudaStream_t s) {
   switch (D) {
-    case 32: return append_t<32, BITS, T>(c, units, k, v, n_q, slot, flush, s);
-    case 64: return append_t<64, BITS, T>(c, units, k, v, n_q, slot, flush, s);
-    case 128: return append_t<128, BITS, T>(c, units, k, v, n_q, slot, flush, s);
+    case 32: return append_t<32, BITS, T>(c, units, k, v, n_q, slot, flush, st, s);
+    case 64: return append_t<64, BITS, T>(c, units, k, v, n_q, slot, flush, st, s);
+    case 128: return append_t<128, BITS, T>(c, units, k, v, n_q, slot, flush, st, s);
   }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t append_any(const CacheView& c, int units, int D, int bits, int dtype, const void* k,
+                       const void* v, long long n_q, int slot, bool flush, DevState* st,
+                       cudaStream_t s) {
+  if (bits == 2 && dtype == 0) return append_d<2, __half>(D, c, units, k, v, n_q, slot, flush, st, s);
+  if (bits == 2 && dtype == 1) return append_d<2, float>(D, c, units, k, v, n_q, slot, flush, st, s);
+  if (bits == 4 && dtype == 0) return append_d<4, __half>(D, c, units, k, v, n_q, slot, flush, st, s);
+  if (bits == 4 && dtype == 1) return append_d<4, float>(D, c, units, k, v, n_q, slot, flush, st, s);
   return cudaErrorInvalidValue;
 }
 
@@ -209,11 +242,17 @@ cudaError_t launch_prefill(const CacheView& c, int units, int D, int bits, int d
 cudaError_t launch_append(const CacheView& c, int units, int D, int bits, int dtype,
                           const void* k, const void* v, long long n_q, int slot, bool flush,
                           cudaStream_t s) {
-  if (bits == 2 && dtype == 0) return append_d<2, __half>(D, c, units, k, v, n_q, slot, flush, s);
-  if (bits == 2 && dtype == 1) return append_d<2, float>(D, c, units, k, v, n_q, slot, flush, s);
-  if (bits == 4 && dtype == 0) return append_d<4, __half>(D, c, units, k, v, n_q, slot, flush, s);
-  if (bits == 4 && dtype == 1) return append_d<4, float>(D, c, units, k, v, n_q, slot, flush, s);
-  return cudaErrorInvalidValue;
+  return append_any(c, units, D, bits, dtype, k, v, n_q, slot, flush, nullptr, s);
+}
+
+cudaError_t launch_append_dev(const CacheView& c, int units, int D, int bits, int dtype,
+                              const void* k, const void* v, const DevState* st, cudaStream_t s) {
+  return append_any(c, units, D, bits, dtype, k, v, 0, 0, false, const_cast<DevState*>(st), s);
+}
+
+cudaError_t launch_set_state(DevState* st, long long n_q, int r, cudaStream_t s) {
+  set_state_kernel<<<1, 1, 0, s>>>(st, n_q, r);
+  return cudaGetLastError();
 }
 
 }  // namespace kivi

@@ -210,7 +210,8 @@ KIVI_API int kivi_decode_attention_simt(const kivi_cache *cache, const void *q,
  * update.  When no flush is due (r < R) it is one kernel launch: the decode
  * kernel's CTA that owns a sequence's window writes the new token into
  * window slot r before it reads the window.  When the window is full the
- * flush runs first as its own launch (as in kivi_append_token).  All
+ * flush runs first as its own launch (as in kivi_append_token), and so does
+ * the append when k or v is not 16-byte aligned.  All
  * argument checks of both calls happen before any launch, so an error
  * leaves the cache unchanged.  The counters stay on the host, so a loop of
  * these calls is not graph-capturable.  (KIVI, study.space summary: new
@@ -220,6 +221,36 @@ KIVI_API int kivi_decode_attention_simt(const kivi_cache *cache, const void *q,
 KIVI_API int kivi_append_decode(kivi_cache *cache, const void *k, const void *v,
                        const void *q, int Hq, float softmax_scale, void *out,
                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Device-resident counters of a cache: 16 bytes of device memory, 16-byte
+ * aligned, laid out as { long long n_q; int r; int status; }.  With them a
+ * decode loop runs without host round trips and can be captured in a CUDA
+ * graph: kivi_append_decode_dev reads and advances them on the device and
+ * never touches the host counters of `cache`.  status becomes 1 (and the
+ * call does nothing) once an append finds the cache full.
+ * kivi_dev_state_init: write the host counters of `cache` into `state`
+ * (asynchronously, on `stream`) and clear status.
+ * To continue with the host-counter calls afterwards, copy n_q and r back
+ * from `state` into the cache struct.  No counterpart on the pages.
+ * Errors: KIVI_ERR_ARG (null or misaligned state), KIVI_ERR_CUDA. */
+KIVI_API int kivi_dev_state_init(const kivi_cache *cache, void *state, void *stream);
+
+/* kivi_append_decode with the counters in `state` (device memory, see
+ * kivi_dev_state_init) instead of cache->n_q / cache->r: two launches every
+ * step -- an append that flushes the window on the device when r == R, and
+ * the decode, which plans its split on the device and advances the counters
+ * when it finishes.  Launch arguments do not depend on the counters, so the
+ * same two launches can be captured once and replayed.  The workspace
+ * (kivi_decode_workspace_bytes) must be zero-filled before first use and
+ * used only by these calls: they count arrivals in counters that every call
+ * leaves at zero.  (KIVI, study.space summary: append to the residual part,
+ * flush every R tokens, attend over both parts.)
+ * Errors: KIVI_ERR_ARG, KIVI_ERR_UNSUPPORTED, KIVI_ERR_WORKSPACE,
+ * KIVI_ERR_CUDA (the capacity check happens on the device: status). */
+KIVI_API int kivi_append_decode_dev(const kivi_cache *cache, void *state, const void *k,
+                           const void *v, const void *q, int Hq, float softmax_scale,
+                           void *out, void *workspace, size_t workspace_bytes,
+                           void *stream);
 
 /* Optional timing hook: if start/stop are non-NULL cudaEvent_t handles,
  * later decode calls on this thread record `start` just before and `stop`

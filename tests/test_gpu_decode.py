@@ -178,6 +178,28 @@ def test_append_decode_matches_separate_calls(dtype, D, gq):
     assert_state_equal(fused, oc)
 
 
+def test_append_decode_unaligned_token_takes_the_two_launch_path():
+    """k/v views at an 8-byte offset: same result as append + decode."""
+    w = small(D=64, dtype="f16", gq=2, T=70, R=32, B=2, Hkv=2, seed=4)
+    K, V = W.prompt_kv(w, device="cuda")
+    a, b = gpu_cache(w, capacity=256), gpu_cache(w, capacity=256)
+    a.prefill(K, V)
+    b.prefill(K, V)
+    for step in range(5):
+        k, v = W.step_kv(w, step, device="cuda")
+        kb = torch.empty(k.numel() + 4, dtype=k.dtype, device="cuda")
+        vb = torch.empty(v.numel() + 4, dtype=v.dtype, device="cuda")
+        ku = kb[4:].view(k.shape)
+        vu = vb[4:].view(v.shape)
+        ku.copy_(k)
+        vu.copy_(v)
+        assert ku.data_ptr() % 16 == 8
+        q = W.query(w, step, device="cuda")
+        out_a = a.append_decode(ku, vu, q, 1.0)
+        b.append(k, v)
+        assert torch.equal(out_a, b.decode(q, 1.0))
+
+
 def test_decode_errors_on_device():
     w = small(D=64, T=100)
     K, V = W.prompt_kv(w, device="cuda")
@@ -194,3 +216,93 @@ def test_decode_errors_on_device():
     rc = L.kivi_decode_attention(ctypes.byref(gc._c), q.data_ptr(), w.Hq, 1.0, out.data_ptr(),
                                  ws.data_ptr() + 4, ws.numel() - 4, None)
     assert rc == 5  # misaligned
+
+
+@pytest.mark.parametrize("dtype,D", [("f16", 128), ("f32", 64)])
+@pytest.mark.parametrize("gq", [1, 4])
+def test_device_counter_loop_matches_host_counters(dtype, D, gq):
+    """kivi_append_decode_dev (counters in device memory) gives bit for bit the
+    outputs and cache of kivi_append_decode over 150 steps across two flushes."""
+    w = small(D=D, dtype=dtype, gq=gq, T=100, R=64, B=2, Hkv=2, seed=12)
+    K, V = W.prompt_kv(w, device="cuda")
+    dev, host = gpu_cache(w, capacity=512), gpu_cache(w, capacity=512)
+    dev.prefill(K, V)
+    host.prefill(K, V)
+    st = dev.dev_state()
+    for step in range(150):
+        k, v = W.step_kv(w, step, device="cuda")
+        q = W.query(w, step, device="cuda")
+        out_d = dev.append_decode_dev(st, k, v, q, 1.0)
+        out_h = host.append_decode(k, v, q, 1.0)
+        assert torch.equal(out_d, out_h), f"step {step}"
+    dev.load_dev_state(st)
+    assert (dev.n_q, dev.r) == (host.n_q, host.r) == (192, 58)
+    n_q, r, E = dev.n_q, dev.r, 32 // w.bits
+    used = {"k_codes": n_q, "k_scale": n_q // w.G, "k_zero": n_q // w.G, "v_codes": n_q // E,
+            "v_scale": n_q, "v_zero": n_q, "k_res": r, "v_res": r}
+    for name, n in used.items():
+        assert torch.equal(dev.view(name)[:, :, :n], host.view(name)[:, :, :n]), name
+
+
+def test_device_counter_steps_replay_as_a_cuda_graph():
+    """Four append + decode steps captured once and replayed 40 times (fresh
+    inputs copied in before each replay, flushes every 32 tokens) equal the
+    host-counter loop step for step."""
+    w = small(D=128, dtype="f16", gq=2, T=90, R=32, B=2, Hkv=2, seed=13)
+    K, V = W.prompt_kv(w, device="cuda")
+    dev, host = gpu_cache(w, capacity=512), gpu_cache(w, capacity=512)
+    dev.prefill(K, V)
+    host.prefill(K, V)
+    st = dev.dev_state()
+    M = 4
+    ks = [torch.empty(w.B, w.Hkv, w.D, dtype=w.torch_dtype, device="cuda") for _ in range(M)]
+    vs = [torch.empty_like(x) for x in ks]
+    qs = [torch.empty(w.B, w.Hq, w.D, dtype=w.torch_dtype, device="cuda") for _ in range(M)]
+    outs = [torch.empty_like(x) for x in qs]
+    # one eager step first (library setup happens outside the capture)
+    k, v = W.step_kv(w, 0, device="cuda")
+    q = W.query(w, 0, device="cuda")
+    assert torch.equal(dev.append_decode_dev(st, k, v, q, 1.0), host.append_decode(k, v, q, 1.0))
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for j in range(M):
+                dev.append_decode_dev(st, ks[j], vs[j], qs[j], 1.0, out=outs[j])
+    torch.cuda.synchronize()
+    step = 1
+    for rep in range(40):
+        for j in range(M):
+            k, v = W.step_kv(w, step + j, device="cuda")
+            ks[j].copy_(k)
+            vs[j].copy_(v)
+            qs[j].copy_(W.query(w, step + j, device="cuda"))
+        g.replay()
+        for j in range(M):
+            k, v = W.step_kv(w, step + j, device="cuda")
+            ref = host.append_decode(k, v, W.query(w, step + j, device="cuda"), 1.0)
+            assert torch.equal(outs[j], ref), f"replay {rep} step {j}"
+        step += M
+    dev.load_dev_state(st)
+    assert (dev.n_q, dev.r) == (host.n_q, host.r)
+    del g
+
+
+def test_device_counter_full_cache_sets_status():
+    w = small(D=64, dtype="f16", gq=1, T=60, R=32, B=1, Hkv=2, seed=14)
+    K, V = W.prompt_kv(w, device="cuda")
+    c = gpu_cache(w, capacity=64)
+    c.prefill(K, V)
+    st = c.dev_state()
+    q = W.query(w, 0, device="cuda")
+    for step in range(4):  # 60 -> 64 tokens: fits
+        k, v = W.step_kv(w, step, device="cuda")
+        c.append_decode_dev(st, k, v, q, 1.0)
+    c.load_dev_state(st)
+    assert c.n_q + c.r == 64
+    k, v = W.step_kv(w, 9, device="cuda")
+    c.append_decode_dev(st, k, v, q, 1.0)  # no room: nothing happens on the device
+    with pytest.raises(kivi.KiviError):
+        c.load_dev_state(st)
