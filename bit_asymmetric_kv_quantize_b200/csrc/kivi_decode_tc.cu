@@ -321,8 +321,8 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::M
   if (sizeof(T) == 4 && a.new_k != nullptr) {
     // fused append, fp32 window (read by generic loads after the barrier
     // below): the CTA that owns a unit's window writes the unit's new token
-    // into window slot new_slot.  (fp16: the producer writes it just before
-    // the window's tensor copies.)
+    // into window slot new_slot.  (fp16: the warp that takes the window tile
+    // holding the slot patches the token into shared memory and the cache.)
     for (long long u = G0 / UP; G0 < G1 && u <= (G1 - 1) / UP; ++u) {
       if (cta != (u * UP + n_qt) / W) continue;
       T* kr = reinterpret_cast<T*>(c.k_res) + (u * c.R + a.new_slot) * D;
