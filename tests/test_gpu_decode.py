@@ -306,3 +306,26 @@ def test_device_counter_full_cache_sets_status():
     c.append_decode_dev(st, k, v, q, 1.0)  # no room: nothing happens on the device
     with pytest.raises(kivi.KiviError):
         c.load_dev_state(st)
+
+
+def test_streaming_workload_device_counters_and_fused_steps():
+    """The streaming workload at full size (B=4, 32 heads, prompt 32768, 512
+    steps, flush every 128): the device-counter step and the host-counter
+    fused step give bit for bit the outputs of append + decode at every step,
+    and the counters agree at the end."""
+    w = W.STREAMING
+    K, V = W.prompt_kv(w, device="cuda")
+    ref, fused, dev = gpu_cache(w), gpu_cache(w), gpu_cache(w)
+    for c in (ref, fused, dev):
+        c.prefill(K, V)
+    del K, V
+    st = dev.dev_state()
+    for step in range(w.steps):
+        k, v = W.step_kv(w, step, device="cuda")
+        q = W.query(w, step, device="cuda")
+        ref.append(k, v)
+        out_r = ref.decode(q, 1.0)
+        assert torch.equal(fused.append_decode(k, v, q, 1.0), out_r), f"fused step {step}"
+        assert torch.equal(dev.append_decode_dev(st, k, v, q, 1.0), out_r), f"device step {step}"
+    dev.load_dev_state(st)
+    assert (ref.n_q, ref.r) == (fused.n_q, fused.r) == (dev.n_q, dev.r)
