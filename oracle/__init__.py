@@ -49,7 +49,7 @@ class Unit(ctypes.Structure):
         ("k_codes", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("k_zero", ctypes.c_void_p),
         ("v_codes", ctypes.c_void_p), ("v_scale", ctypes.c_void_p), ("v_zero", ctypes.c_void_p),
         ("k_res", ctypes.c_void_p), ("v_res", ctypes.c_void_p),
-        ("n_q", ctypes.c_longlong), ("r", ctypes.c_int),
+        ("n_q", ctypes.c_longlong), ("r", ctypes.c_int), ("meta_f16", ctypes.c_int),
     ]
 
 
@@ -64,6 +64,9 @@ def lib():
             vp, ll, ci = ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int
             up = ctypes.POINTER(Unit)
             L.kivi_oracle_quantize_group.argtypes = [vp, ll, ll, ci, vp, vp, vp]
+            L.kivi_oracle_quantize_group_meta.argtypes = [vp, ll, ll, ci, ci, vp, vp, vp]
+            L.kivi_oracle_round_half.argtypes = [ctypes.c_float]
+            L.kivi_oracle_round_half.restype = ctypes.c_float
             L.kivi_oracle_pack_word.argtypes = [vp, ci]
             L.kivi_oracle_pack_word.restype = ctypes.c_uint32
             L.kivi_oracle_dequant.argtypes = [ctypes.c_uint32, ctypes.c_float, ctypes.c_float]
@@ -94,15 +97,23 @@ def _check(rc: int, what: str) -> None:
 
 # ---------------------------------------------------------------- Q, P, D
 
-def quantize_group(x, bits: int):
-    """Q on one group; returns (scale, zero, codes[uint16])."""
+def quantize_group(x, bits: int, meta_f16: bool = False):
+    """Q on one group; returns (scale, zero, codes[uint16]).  meta_f16: the
+    binary16-metadata format variant (scale and zero rounded to binary16, codes
+    chosen against the rounded values)."""
     x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
     s = np.zeros(1, np.float32)
     z = np.zeros(1, np.float32)
     c = np.zeros(x.size, np.uint16)
-    _check(lib().kivi_oracle_quantize_group(_ptr(x), x.size, 1, bits, _ptr(s), _ptr(z), _ptr(c)),
+    _check(lib().kivi_oracle_quantize_group_meta(_ptr(x), x.size, 1, bits, int(bool(meta_f16)),
+                                                 _ptr(s), _ptr(z), _ptr(c)),
            "quantize_group")
     return s[0], z[0], c
+
+
+def round_half(x: float) -> float:
+    """x rounded to the nearest binary16 value (ties to even)."""
+    return float(np.float32(lib().kivi_oracle_round_half(ctypes.c_float(float(x)))))
 
 
 def pack_word(codes, bits: int) -> int:
@@ -132,7 +143,8 @@ class OracleCache:
     empty), so that full-size shapes can be checked on sampled units.
     """
 
-    def __init__(self, B, Hkv, D, bits, G, Gv, R, capacity, units=None):
+    def __init__(self, B, Hkv, D, bits, G, Gv, R, capacity, units=None, meta_f16=False):
+        self.meta_f16 = bool(meta_f16)
         self.B, self.Hkv, self.D, self.bits = B, Hkv, D, bits
         self.G, self.Gv, self.R, self.capacity = G, Gv, R, capacity
         E = 32 // bits
@@ -159,6 +171,7 @@ class OracleCache:
         for name in ("k_codes", "k_scale", "k_zero", "v_codes", "v_scale", "v_zero", "k_res", "v_res"):
             setattr(u, name, getattr(self, name)[i].ctypes.data)
         u.n_q, u.r = 0, 0
+        u.meta_f16 = int(self.meta_f16)
         return u
 
     def unit(self, b, h) -> Unit:

@@ -49,12 +49,48 @@ static int valid_bits(int bits) {
  *   c_i = clamp(round_half_even((x_i - mn) / s), 0, L), or 0 when s == 0.
  * The quotient is a true division, not a multiply by 1/s.
  */
+/*
+ * Binary16 rounding, from the format's definition: 11 significant bits for
+ * normal values (|x| >= 2^-14), a fixed quantum of 2^-24 below that, round
+ * to nearest with ties to even, and magnitudes that round above 65504 (the
+ * largest finite binary16 value) become infinite.  The division by the
+ * quantum q (a power of two) and the product by q are exact in binary64.
+ */
+float kivi_oracle_round_half(float x) {
+  double a, q, r;
+  int e;
+  if (x == 0.0f || !isfinite(x)) return x;
+  a = fabs((double)x);
+  (void)frexp(a, &e); /* a = m 2^e, 0.5 <= m < 1 */
+  e -= 11;            /* quantum of an 11-bit significand */
+  if (e < -24) e = -24;
+  q = ldexp(1.0, e);
+  r = nearbyint(a / q) * q; /* default rounding mode: half to even */
+  if (r > 65504.0) r = INFINITY;
+  return (float)(x < 0.0f ? -r : r);
+}
+
 int kivi_oracle_quantize_group(const float *x, long long n, long long stride,
                                int bits, float *scale, float *zero,
                                uint16_t *codes) {
+  return kivi_oracle_quantize_group_meta(x, n, stride, bits, 0, scale, zero, codes);
+}
+
+/*
+ * Format variant (metadata in binary16).  Reading: the binary32 scale and
+ * zero above are rounded to binary16 (round to nearest even), and the codes
+ * are chosen against the rounded values, so that the stored (scale, zero)
+ * reconstruct the codes as closely as the grid allows:
+ *   s16 = half(s), z16 = half(mn), c_i = clamp(rhe((x_i - z16) / s16), 0, L),
+ *   or 0 when s16 == 0.
+ */
+int kivi_oracle_quantize_group_meta(const float *x, long long n, long long stride,
+                                    int bits, int meta_f16, float *scale,
+                                    float *zero, uint16_t *codes) {
   long long i;
-  float mn, mx, L, range, s;
-  if (!x || !scale || !zero || !codes || n <= 0 || !valid_bits(bits))
+  float mn, mx, L, range, s, z;
+  if (!x || !scale || !zero || !codes || n <= 0 || !valid_bits(bits) ||
+      (meta_f16 != 0 && meta_f16 != 1))
     return KIVI_ORACLE_ERR_ARG;
   mn = x[0];
   mx = x[0];
@@ -66,13 +102,18 @@ int kivi_oracle_quantize_group(const float *x, long long n, long long stride,
   L = (float)((1u << bits) - 1u);
   range = mx - mn;
   s = range / L;
+  z = mn;
+  if (meta_f16) {
+    s = kivi_oracle_round_half(s);
+    z = kivi_oracle_round_half(mn);
+  }
   *scale = s;
-  *zero = mn;
+  *zero = z;
   for (i = 0; i < n; ++i) {
     if (s == 0.0f) {
       codes[i] = 0;
     } else {
-      float t = (x[i * stride] - mn) / s;
+      float t = (x[i * stride] - z) / s;
       float c = nearbyintf(t); /* default rounding mode: half to even */
       if (c < 0.0f) c = 0.0f;
       if (c > L) c = L;
@@ -150,18 +191,18 @@ static int quantize_block(kivi_oracle_unit *u, const float *K, const float *V,
   for (g = 0; g < n / G; ++g) {
     for (d = 0; d < D; ++d) {
       long long gq = (t0 / G) + g;
-      kivi_oracle_quantize_group(&K[(g * G) * D + d], G, D, bits,
-                                 &u->k_scale[gq * D + d],
-                                 &u->k_zero[gq * D + d], tmp);
+      kivi_oracle_quantize_group_meta(&K[(g * G) * D + d], G, D, bits, u->meta_f16,
+                                      &u->k_scale[gq * D + d],
+                                      &u->k_zero[gq * D + d], tmp);
       for (i = 0; i < G; ++i) ck[(g * G + i) * D + d] = tmp[i];
     }
   }
   /* values: one group per (token t, value group j) over Gv channels */
   for (t = 0; t < n; ++t) {
     for (j = 0; j < NJ; ++j) {
-      kivi_oracle_quantize_group(&V[t * D + j * Gv], Gv, 1, bits,
-                                 &u->v_scale[(t0 + t) * NJ + j],
-                                 &u->v_zero[(t0 + t) * NJ + j], tmp);
+      kivi_oracle_quantize_group_meta(&V[t * D + j * Gv], Gv, 1, bits, u->meta_f16,
+                                      &u->v_scale[(t0 + t) * NJ + j],
+                                      &u->v_zero[(t0 + t) * NJ + j], tmp);
       for (i = 0; i < Gv; ++i) cv[t * D + j * Gv + i] = tmp[i];
     }
   }

@@ -72,12 +72,23 @@ typedef struct {
   float *v_res;
   long long n_q; /* tokens held in the quantized store */
   int r;         /* tokens held in the residual window */
+  int meta_f16;  /* 1: scales and zeros stored in binary16 (format variant) */
 } kivi_oracle_unit;
 
 /* Q: quantize one group of n values x[0], x[stride], ..., x[(n-1)*stride]. */
 int kivi_oracle_quantize_group(const float *x, long long n, long long stride,
                                int bits, float *scale, float *zero,
                                uint16_t *codes);
+
+/* Q with the metadata stored in binary16 when meta_f16 is 1: the scale and
+ * zero are rounded to binary16 and the codes are chosen against the rounded
+ * values (a format variant; meta_f16 = 0 is kivi_oracle_quantize_group). */
+int kivi_oracle_quantize_group_meta(const float *x, long long n, long long stride,
+                                    int bits, int meta_f16, float *scale,
+                                    float *zero, uint16_t *codes);
+
+/* x rounded to the nearest IEEE binary16 value (ties to even), as a float. */
+float kivi_oracle_round_half(float x);
 
 /* P: pack 32/bits codes into one word, codes[0] in the least significant bits. */
 uint32_t kivi_oracle_pack_word(const uint16_t *codes, int bits);

@@ -16,8 +16,8 @@ import pytest
 import oracle
 
 
-def _cache(D=32, bits=2, G=32, Gv=32, R=32, capacity=128, B=1, Hkv=1):
-    return oracle.OracleCache(B, Hkv, D, bits, G, Gv, R, capacity)
+def _cache(D=32, bits=2, G=32, Gv=32, R=32, capacity=128, B=1, Hkv=1, meta_f16=False):
+    return oracle.OracleCache(B, Hkv, D, bits, G, Gv, R, capacity, meta_f16=meta_f16)
 
 
 def test_pack_axes_hand_words():
@@ -104,6 +104,34 @@ def test_prefill_equals_appends(bits, T):
         assert np.array_equal(getattr(a, name).view(np.uint32), getattr(b, name).view(np.uint32)), name
     assert np.array_equal(a.k_res[0, :ua.r], b.k_res[0, :ub.r])
     assert np.array_equal(a.v_res[0, :ua.r], b.v_res[0, :ub.r])
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_binary16_metadata_cache_matches_group_quantizer(bits):
+    """With binary16 metadata the cache's block quantizer gives, group by
+    group, exactly the single-group binary16 quantizer; prefill(T) equals T
+    appends; and the metadata are binary16 values."""
+    rng = np.random.default_rng(40 + bits)
+    D, R, T = 64, 32, 130
+    K = (rng.standard_normal((T, D)) * np.where(np.arange(D) % 17 == 3, 20, 1)).astype(np.float16).astype(np.float32)
+    V = rng.standard_normal((T, D)).astype(np.float16).astype(np.float32)
+    a = _cache(D=D, bits=bits, R=R, capacity=256, meta_f16=True)
+    b = _cache(D=D, bits=bits, R=R, capacity=256, meta_f16=True)
+    a.prefill_unit(0, 0, K, V)
+    for t in range(T):
+        b.append_unit(0, 0, K[t], V[t])
+    for name in ("k_codes", "k_scale", "k_zero", "v_codes", "v_scale", "v_zero"):
+        assert np.array_equal(getattr(a, name).view(np.uint32), getattr(b, name).view(np.uint32)), name
+    n_q = a.unit(0, 0).n_q
+    for g in range(n_q // 32):
+        for d in (0, 3, 17, 63):
+            s, z, c = oracle.quantize_group(K[32 * g:32 * g + 32, d], bits, meta_f16=True)
+            assert a.k_scale[0, g, d] == s and a.k_zero[0, g, d] == z
+    for t in (0, 31, n_q - 1):
+        s, z, _ = oracle.quantize_group(V[t, 32:64], bits, meta_f16=True)
+        assert a.v_scale[0, t, 1] == s and a.v_zero[0, t, 1] == z
+    ks = a.k_scale[0, :n_q // 32]
+    assert np.array_equal(ks, ks.astype(np.float16).astype(np.float32))
 
 
 def test_flush_quantizes_the_window():

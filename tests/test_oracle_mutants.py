@@ -25,17 +25,17 @@ MUTANTS = [
     ("levels_off_by_one", "L = (float)((1u << bits) - 1u);", "L = (float)(1u << bits);"),
     ("round_half_up", "float c = nearbyintf(t);", "float c = floorf(t + 0.5f);"),
     ("round_truncate", "float c = nearbyintf(t);", "float c = truncf(t);"),
-    ("reciprocal_multiply", "float t = (x[i * stride] - mn) / s;",
-     "float t = (x[i * stride] - mn) * (1.0f / s);"),
-    ("binary64_quotient", "float t = (x[i * stride] - mn) / s;\n      float c = nearbyintf(t);",
-     "double t = ((double)x[i * stride] - (double)mn) / (double)s;\n"
+    ("reciprocal_multiply", "float t = (x[i * stride] - z) / s;",
+     "float t = (x[i * stride] - z) * (1.0f / s);"),
+    ("binary64_quotient", "float t = (x[i * stride] - z) / s;\n      float c = nearbyintf(t);",
+     "double t = ((double)x[i * stride] - (double)z) / (double)s;\n"
      "      float c = (float)nearbyint(t);"),
-    ("zero_is_max", "*zero = mn;", "*zero = mx;"),
+    ("zero_is_max", "  z = mn;\n", "  z = mx;\n"),
     ("min_keeps_last_tie", "if (v < mn) mn = v;", "if (v <= mn) mn = v;"),
     ("pack_msb_first", "w |= ((uint32_t)codes[i] & mask) << (bits * i);",
      "w |= ((uint32_t)codes[i] & mask) << (bits * (E - 1 - i));"),
-    ("keys_grouped_per_token", "kivi_oracle_quantize_group(&K[(g * G) * D + d], G, D, bits,",
-     "kivi_oracle_quantize_group(&K[(g * G) * D + d], G, 1, bits,"),
+    ("keys_grouped_per_token", "kivi_oracle_quantize_group_meta(&K[(g * G) * D + d], G, D, bits,",
+     "kivi_oracle_quantize_group_meta(&K[(g * G) * D + d], G, 1, bits,"),
     ("value_pack_transposed", "for (i = 0; i < E; ++i) tmp[i] = cv[(t * E + i) * D + d];",
      "for (i = 0; i < E; ++i) tmp[i] = cv[(t * E) * D + (d / E) * E + i];"),
     ("residual_length", "r = (T == 0) ? 0 : ((T - 1) % u->R) + 1;", "r = T % u->R;"),
@@ -51,6 +51,13 @@ MUTANTS = [
      "for (d = 0; d < u->D; ++d) acc += (double)qh[d] * Vh[t * u->D + d];"),
     ("sigma_dropped", "p[t] = sigma * acc;", "p[t] = acc;"),
     ("unnormalised", "out[(long long)h * u->D + d] = o / l;", "out[(long long)h * u->D + d] = o;"),
+    # binary16-metadata variant
+    ("codes_against_unrounded_scale",
+     "    s = kivi_oracle_round_half(s);\n    z = kivi_oracle_round_half(mn);\n  }\n  *scale = s;",
+     "    z = kivi_oracle_round_half(mn);\n  }\n  *scale = meta_f16 ? kivi_oracle_round_half(s) : s;"),
+    ("half_ties_away", "r = nearbyint(a / q) * q;", "r = round(a / q) * q;"),
+    ("half_no_subnormal_quantum", "if (e < -24) e = -24;", ""),
+    ("half_overflow_kept", "if (r > 65504.0) r = INFINITY;", ""),
 ]
 
 

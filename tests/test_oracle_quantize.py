@@ -34,6 +34,8 @@ def _golden():
 
 QROWS = [r for r in _golden() if r[0] == "Q"]
 PROWS = [r for r in _golden() if r[0] == "P"]
+MROWS = [r for r in _golden() if r[0] == "M"]
+HROWS = [r for r in _golden() if r[0] == "H"]
 
 
 @pytest.mark.parametrize("row", QROWS, ids=[f"{r[1]}b:{r[2]}" for r in QROWS])
@@ -50,6 +52,67 @@ def test_quantize_golden(row):
 def test_pack_golden(row):
     _, bits, codes, word = row
     assert oracle.pack_word([int(v) for v in codes.split()], int(bits)) == int(word, 16)
+
+
+@pytest.mark.parametrize("row", MROWS, ids=[f"{r[1]}b:{r[2]}" for r in MROWS])
+def test_quantize_binary16_metadata_golden(row):
+    _, bits, xs, scale_hex, zero, codes = row
+    x = np.array([float(v) for v in xs.split()], np.float32)
+    s, z, c = oracle.quantize_group(x, int(bits), meta_f16=True)
+    assert int(np.float16(s).view(np.uint16)) == int(scale_hex, 16)
+    assert float(np.float16(s)) == float(s)  # the stored scale is a binary16 value
+    assert _f32_bits(z) == _f32_bits(np.float32(float(zero)))
+    assert c.tolist() == [int(v) for v in codes.split()]
+
+
+@pytest.mark.parametrize("row", HROWS, ids=[r[1] for r in HROWS])
+def test_round_half_golden(row):
+    _, x_hex, h_hex = row
+    x = struct.unpack("<f", struct.pack("<I", int(x_hex, 16)))[0]
+    got = oracle.round_half(x)
+    want = np.array([int(h_hex, 16)], np.uint16).view(np.float16)[0]
+    assert (np.isinf(got) and np.isinf(want) and np.sign(got) == np.sign(want)) or \
+        _f32_bits(got) == _f32_bits(np.float32(want))
+
+
+def test_round_half_matches_numpy_binary16():
+    """Against numpy's float16 conversion (round to nearest even) on binary32
+    values across every binary16 binade, the subnormals, the ties and the
+    overflow boundary."""
+    rng = np.random.default_rng(7)
+    halves = np.arange(0, 0x7c00, dtype=np.uint16).view(np.float16).astype(np.float32)
+    nxt = np.nextafter(halves, np.float32(np.inf))
+    prv = np.nextafter(halves, np.float32(0))
+    mids = (halves[:-1].astype(np.float64) + halves[1:]) / 2
+    xs = np.concatenate([halves, nxt, prv, mids.astype(np.float32),
+                         np.nextafter(mids.astype(np.float32), np.float32(np.inf)),
+                         rng.standard_normal(20000).astype(np.float32) * 10.0 ** rng.integers(-8, 5, 20000),
+                         np.float32([65504, 65519.996, 65520, 1e6, 1e-9, 3e-8])])
+    xs = np.concatenate([xs, -xs])
+    with np.errstate(over="ignore"):
+        want = xs.astype(np.float16).astype(np.float32)
+    got = np.array([oracle.round_half(float(v)) for v in xs], np.float32)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_binary16_metadata_invariants(bits):
+    """Binary16 scale and zero (fp16 inputs, whose minimum is a binary16
+    value): codes in range, the minimum reconstructs exactly, and every value
+    reconstructs within half a step of the stored grid plus the scale's
+    rounding carried over the L steps to the maximum."""
+    rng = np.random.default_rng(bits)
+    L = (1 << bits) - 1
+    for gi in range(400):
+        x = (rng.standard_normal(32) * (20.0 if gi % 3 == 0 else 1.0)).astype(np.float16).astype(np.float32)
+        s16, z16, c = oracle.quantize_group(x, bits, meta_f16=True)
+        s32, z32, _ = oracle.quantize_group(x, bits)
+        assert float(np.float16(s16)) == float(s16) and z16 == x.min()
+        assert c.min() >= 0 and c.max() <= L
+        assert c[int(np.argmin(x))] == 0
+        xh = c.astype(np.float64) * s16 + z16
+        bound = max(s16 / 2, L * abs(float(s32) - float(s16))) + 4 * np.spacing(np.float32(np.abs(x).max()))
+        assert np.all(np.abs(xh - x) <= bound + s16 * 1e-6)
 
 
 def test_golden_file_covers_every_width():
