@@ -64,7 +64,21 @@ def parse():
     p.add_argument("--unfused", action="store_true",
                    help="append and decode as two calls (kivi_append_token + decode)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
+    p.add_argument("--meta", choices=["f32", "f16"], default="f32",
+                   help="scale/zero storage: binary32, or the binary16 format variant "
+                        "(fp16 workloads)")
     return p.parse_args()
+
+
+def bench_workload(args) -> W.Workload:
+    """The workload named by --workload with the --meta storage; the streaming
+    workload's decode loop is the step loop itself (steps = 0 here)."""
+    w = W.ALL[args.workload]
+    if w.steps:
+        w = w.with_(steps=0)
+    if args.meta == "f16":
+        w = w.with_(meta="f16", name=w.name + "-meta16")
+    return w
 
 
 def dist_env():
@@ -109,7 +123,7 @@ def profiled_traffic(w: W.Workload):
     try:
         text = open(prof).read()
         h = hashlib.sha256()
-        for f in ("kivi_decode_tc.cu", "kivi_internal.cuh"):
+        for f in ("kivi_decode_tc.cuh", "kivi_decode_tc.cu", "kivi_internal.cuh"):
             h.update(open(os.path.join(csrc, f), "rb").read())
     except OSError:
         return None
@@ -124,11 +138,13 @@ def profiled_traffic(w: W.Workload):
 def algorithmic_bytes(w: W.Workload, n_q: int, r: int) -> int:
     """Bytes one decode call must move: every code, scale and zero of the
     quantized store, the window tokens, q in and out (per unit: K codes
-    n_q*D*b/8, K meta (n_q/G)*D*8, V codes n_q*D*b/8, V meta n_q*(D/Gv)*8,
-    window r*D*2*es; plus B*Hq*D*es each for q and out)."""
+    n_q*D*b/8, K meta (n_q/G)*D*2*ms, V codes n_q*D*b/8, V meta
+    n_q*(D/Gv)*2*ms, window r*D*2*es; plus B*Hq*D*es each for q and out;
+    ms = 4, or 2 with binary16 scales and zeros)."""
     es = 2 if w.dtype == "f16" else 4
-    per_unit = (2 * n_q * w.D * w.bits // 8 + (n_q // w.G) * w.D * 8 + n_q * (w.D // w.Gv) * 8
-                + r * w.D * 2 * es)
+    ms = 2 if w.meta == "f16" else 4
+    per_unit = (2 * n_q * w.D * w.bits // 8 + (n_q // w.G) * w.D * 2 * ms
+                + n_q * (w.D // w.Gv) * 2 * ms + r * w.D * 2 * es)
     return w.B * w.Hkv * per_unit + 2 * w.B * w.Hq * w.D * es
 
 
@@ -205,9 +221,7 @@ def run_kivi(args, rank, world, local):
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=device)
 
-    w = W.ALL[args.workload]
-    if w.steps:  # the streaming workload's decode loop is the step loop itself
-        w = w.with_(steps=0)
+    w = bench_workload(args)
     n_layers = max(1, args.layers)
     e2e_steps = 0 if args.no_e2e else min(args.steps, 1024)
     per_layer = -(-(args.warmup + 2 * args.steps + e2e_steps) // n_layers) + 1
@@ -216,7 +230,7 @@ def run_kivi(args, rank, world, local):
     caches = []
     for _ in range(n_layers):
         c = kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, capacity, R=w.R, G=w.G, Gv=w.Gv,
-                           dtype=w.torch_dtype, device=device)
+                           dtype=w.torch_dtype, device=device, meta=w.torch_meta)
         c.prefill(Kp, Vp)
         caches.append(c)
     del Kp, Vp
@@ -366,7 +380,9 @@ def run_kivi(args, rank, world, local):
             "config": {
                 "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                 "context": w.T, "bits": w.bits, "G": w.G, "Gv": w.Gv, "R": w.R,
-                "dtype_io": w.dtype, "kernel": args.kernel, "step": ("kivi_append_decode" if fused else "kivi_append_token+kivi_decode_attention"), "parallelism": f"replicas{world}",
+                "dtype_io": w.dtype, "meta": w.meta, "kernel": args.kernel,
+                "step": ("kivi_append_decode" if fused else "kivi_append_token+kivi_decode_attention"),
+                "parallelism": f"replicas{world}",
                 "layers_rotated": n_layers,
                 "l2": f"inputs larger than L2: {n_layers} layer caches visited round-robin",
                 "decode_splits": n_split,
@@ -400,7 +416,8 @@ def oracle_sample(w: W.Workload, n_units: int, steps: int, threads: int):
 
     units = [(u // w.Hkv, u % w.Hkv) for u in range(min(n_units, w.B * w.Hkv))]
     cap = -(-(w.T + steps + 1) // w.R) * w.R
-    oc = oracle.OracleCache(w.B, w.Hkv, w.D, w.bits, w.G, w.Gv, w.R, cap, units=units)
+    oc = oracle.OracleCache(w.B, w.Hkv, w.D, w.bits, w.G, w.Gv, w.R, cap, units=units,
+                            meta_f16=w.meta == "f16")
     g = w.with_(B=1, Hkv=1, Hq=w.gq)
     K, V = W.prompt_kv(g)
     Kf, Vf = K[0, 0].float().numpy(), V[0, 0].float().numpy()
@@ -448,9 +465,7 @@ def cpu_baseline(w: W.Workload, budget_s: float):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    w = W.ALL[args.workload]
-    if w.steps:
-        w = w.with_(steps=0)
+    w = bench_workload(args)
     threads = cpu_threads()
     budget = 120.0  # seconds of wall time for warm-up + timed steps
     per_step, n = oracle_sample(w, threads, 1, threads)
@@ -466,7 +481,8 @@ def run_reference(args, rank, world):
         "ms_per_step": full_step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                   "context": w.T, "bits": w.bits, "G": w.G, "Gv": w.Gv, "R": w.R},
+                   "context": w.T, "bits": w.bits, "G": w.G, "Gv": w.Gv, "R": w.R,
+                   "meta": w.meta},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": f"each step: append + decode on {n} of {w.B * w.Hkv} units, "
                                    f"scaled to the full batch"},

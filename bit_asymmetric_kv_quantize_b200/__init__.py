@@ -22,6 +22,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libkivi.so")
 
 KIVI_F16, KIVI_F32 = 0, 1
+KIVI_META_F32, KIVI_META_F16 = 0, 1
 NUM_BUFFERS = 8
 BUFFER_NAMES = ("k_codes", "k_scale", "k_zero", "v_codes", "v_scale", "v_zero", "k_res", "v_res")
 STATUS = {0: "KIVI_OK", 1: "KIVI_ERR_ARG", 2: "KIVI_ERR_UNSUPPORTED", 3: "KIVI_ERR_STATE",
@@ -46,7 +47,8 @@ class KiviError(RuntimeError):
 class KiviDims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("D", ctypes.c_int),
                 ("bits", ctypes.c_int), ("G", ctypes.c_int), ("Gv", ctypes.c_int),
-                ("R", ctypes.c_int), ("capacity", ctypes.c_longlong), ("dtype", ctypes.c_int)]
+                ("R", ctypes.c_int), ("capacity", ctypes.c_longlong), ("dtype", ctypes.c_int),
+                ("meta", ctypes.c_int)]
 
 
 class KiviCacheC(ctypes.Structure):
@@ -105,13 +107,24 @@ def _dtype_code(dtype: torch.dtype) -> int:
     raise ValueError(f"unsupported dtype {dtype}")
 
 
+def _meta_code(meta: torch.dtype) -> int:
+    """Scale/zero element type: torch.float32 (binary32) or torch.float16
+    (the binary16-metadata format variant, fp16 caches only)."""
+    if meta == torch.float32:
+        return KIVI_META_F32
+    if meta == torch.float16:
+        return KIVI_META_F16
+    raise ValueError(f"unsupported metadata dtype {meta}")
+
+
 def _check(rc: int, what: str) -> None:
     if rc != 0:
         raise KiviError(rc, what)
 
 
-def buffer_sizes(B, Hkv, D, bits, capacity, R=128, G=32, Gv=32, dtype=torch.float16):
-    dims = KiviDims(B, Hkv, D, bits, G, Gv, R, capacity, _dtype_code(dtype))
+def buffer_sizes(B, Hkv, D, bits, capacity, R=128, G=32, Gv=32, dtype=torch.float16,
+                 meta=torch.float32):
+    dims = KiviDims(B, Hkv, D, bits, G, Gv, R, capacity, _dtype_code(dtype), _meta_code(meta))
     out = (ctypes.c_size_t * NUM_BUFFERS)()
     _check(lib().kivi_buffer_sizes(ctypes.byref(dims), ctypes.byref(out)), "kivi_buffer_sizes")
     return dict(zip(BUFFER_NAMES, list(out)))
@@ -122,20 +135,24 @@ class KiviCache:
 
     Buffers are torch tensors in the library's ABI layout (see include/kivi.h);
     ``n_q`` / ``r`` are the library-owned counters.  Calls are asynchronous on
-    torch's current stream of the cache's device.
+    torch's current stream of the cache's device.  ``meta`` is the element
+    type of the scales and zeros: torch.float32, or torch.float16 for the
+    binary16-metadata format variant (fp16 caches only).
     """
 
     def __init__(self, B: int, Hkv: int, D: int, bits: int, capacity: int, R: int = 128,
                  G: int = 32, Gv: int = 32, dtype: torch.dtype = torch.float16,
-                 device="cuda"):
+                 device="cuda", meta: torch.dtype = torch.float32):
         self.device = torch.device(device)
         if self.device.type != "cuda":
             raise ValueError("KiviCache lives in CUDA device memory")
         if self.device.index is None:
             self.device = torch.device("cuda", torch.cuda.current_device())
         self.dtype = dtype
-        self._dims = KiviDims(B, Hkv, D, bits, G, Gv, R, capacity, _dtype_code(dtype))
-        sizes = buffer_sizes(B, Hkv, D, bits, capacity, R, G, Gv, dtype)
+        self.meta = meta
+        self._dims = KiviDims(B, Hkv, D, bits, G, Gv, R, capacity, _dtype_code(dtype),
+                              _meta_code(meta))
+        sizes = buffer_sizes(B, Hkv, D, bits, capacity, R, G, Gv, dtype, meta)
         self.buffers = {n: torch.empty(max(sizes[n], 16), dtype=torch.uint8, device=self.device)
                         for n in BUFFER_NAMES}
         ptrs = (ctypes.c_void_p * NUM_BUFFERS)(*[self.buffers[n].data_ptr() for n in BUFFER_NAMES])
@@ -149,11 +166,11 @@ class KiviCache:
         self.B, self.Hkv, self.D, self.bits, self.R, self.capacity = B, Hkv, D, bits, R, capacity
         self.shapes = {
             "k_codes": ((B, Hkv, Tq, D // E), torch.int32),
-            "k_scale": ((B, Hkv, Tq // G, D), torch.float32),
-            "k_zero": ((B, Hkv, Tq // G, D), torch.float32),
+            "k_scale": ((B, Hkv, Tq // G, D), meta),
+            "k_zero": ((B, Hkv, Tq // G, D), meta),
             "v_codes": ((B, Hkv, Tq // E, D), torch.int32),
-            "v_scale": ((B, Hkv, Tq, D // Gv), torch.float32),
-            "v_zero": ((B, Hkv, Tq, D // Gv), torch.float32),
+            "v_scale": ((B, Hkv, Tq, D // Gv), meta),
+            "v_zero": ((B, Hkv, Tq, D // Gv), meta),
             "k_res": ((B, Hkv, R, D), dtype),
             "v_res": ((B, Hkv, R, D), dtype),
         }

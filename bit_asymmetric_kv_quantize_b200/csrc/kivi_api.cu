@@ -30,6 +30,8 @@ int check_dims(const kivi_dims* d) {
   if (d->R % kivi::kTile != 0) return KIVI_ERR_UNSUPPORTED;
   if (d->capacity % d->R != 0) return KIVI_ERR_UNSUPPORTED;
   if (d->dtype != KIVI_F16 && d->dtype != KIVI_F32) return KIVI_ERR_UNSUPPORTED;
+  if (d->meta != KIVI_META_F32 && d->meta != KIVI_META_F16) return KIVI_ERR_UNSUPPORTED;
+  if (d->meta == KIVI_META_F16 && d->dtype != KIVI_F16) return KIVI_ERR_UNSUPPORTED;
   if ((long long)d->B * d->Hkv > 65535) return KIVI_ERR_UNSUPPORTED;  // grid y limit
   return KIVI_OK;
 }
@@ -47,6 +49,7 @@ int check_cache(const kivi_cache* c) {
 }
 
 size_t elem_bytes(int dtype) { return dtype == KIVI_F32 ? 4 : 2; }
+size_t meta_bytes(int meta) { return meta == KIVI_META_F16 ? 2 : 4; }
 
 CacheView view(const kivi_cache* c) {
   CacheView v;
@@ -60,6 +63,7 @@ CacheView view(const kivi_cache* c) {
   v.v_res = c->v_res;
   v.Tq = c->dims.capacity - c->dims.R;
   v.R = c->dims.R;
+  v.meta = c->dims.meta;
   return v;
 }
 
@@ -177,6 +181,7 @@ int decode_launch(const kivi_cache* c, const void* q, int Hq, float softmax_scal
   a.D = c->dims.D;
   a.bits = c->dims.bits;
   a.dtype = c->dims.dtype;
+  a.meta = c->dims.meta;
   a.n_q = c->n_q;
   a.r = c->r;
   a.qscale = softmax_scale * kivi::kLog2e;
@@ -267,7 +272,7 @@ int kivi_buffer_sizes(const kivi_dims* dims, size_t out_bytes[KIVI_NUM_BUFFERS])
   const long long units = (long long)dims->B * dims->Hkv;
   const long long Tq = dims->capacity - dims->R;
   const int E = 32 / dims->bits;
-  const size_t f = sizeof(float);
+  const size_t f = meta_bytes(dims->meta);
   out_bytes[KIVI_BUF_K_CODES] = (size_t)(units * Tq * (dims->D / E)) * sizeof(uint32_t);
   out_bytes[KIVI_BUF_K_SCALE] = (size_t)(units * (Tq / dims->G) * dims->D) * f;
   out_bytes[KIVI_BUF_K_ZERO] = out_bytes[KIVI_BUF_K_SCALE];
@@ -292,11 +297,11 @@ int kivi_cache_init(kivi_cache* cache, const kivi_dims* dims,
   }
   cache->dims = *dims;
   cache->k_codes = (uint32_t*)buffers[KIVI_BUF_K_CODES];
-  cache->k_scale = (float*)buffers[KIVI_BUF_K_SCALE];
-  cache->k_zero = (float*)buffers[KIVI_BUF_K_ZERO];
+  cache->k_scale = buffers[KIVI_BUF_K_SCALE];
+  cache->k_zero = buffers[KIVI_BUF_K_ZERO];
   cache->v_codes = (uint32_t*)buffers[KIVI_BUF_V_CODES];
-  cache->v_scale = (float*)buffers[KIVI_BUF_V_SCALE];
-  cache->v_zero = (float*)buffers[KIVI_BUF_V_ZERO];
+  cache->v_scale = buffers[KIVI_BUF_V_SCALE];
+  cache->v_zero = buffers[KIVI_BUF_V_ZERO];
   cache->k_res = buffers[KIVI_BUF_K_RES];
   cache->v_res = buffers[KIVI_BUF_V_RES];
   cache->n_q = 0;
@@ -462,6 +467,7 @@ int kivi_decode_num_splits(const kivi_cache* cache, int Hq) {
   a.bits = cache->dims.bits;
   a.gq = Hq / cache->dims.Hkv;
   a.dtype = cache->dims.dtype;
+  a.meta = cache->dims.meta;
   int occ = 0;
   if (kivi::decode_tc_ctas_per_sm(a, &occ) != cudaSuccess) return 0;
   StreamPlan sp;

@@ -41,7 +41,7 @@ struct Words<4> {
   }
 };
 
-template <int D, int BITS, int GQ, typename T>
+template <int D, int BITS, int GQ, typename T, typename MT>
 __global__ void __launch_bounds__(kWarps * 32) decode_split_simt(DecodeArgs a) {
   using Lt = Layout<D, BITS>;
   constexpr int E = Lt::E, WK = Lt::WK, NJ = Lt::NJ;
@@ -72,11 +72,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_simt(DecodeArgs a) {
   const long long last = min(total, first + a.tiles_per_split);
 
   const uint32_t* kc = c.k_codes + unit * Lt::k_codes_unit(c.Tq);
-  const float* ksc = c.k_scale + unit * Lt::k_meta_unit(c.Tq);
-  const float* kze = c.k_zero + unit * Lt::k_meta_unit(c.Tq);
+  const MT* ksc = reinterpret_cast<const MT*>(c.k_scale) + unit * Lt::k_meta_unit(c.Tq);
+  const MT* kze = reinterpret_cast<const MT*>(c.k_zero) + unit * Lt::k_meta_unit(c.Tq);
   const uint32_t* vc = c.v_codes + unit * Lt::v_codes_unit(c.Tq);
-  const float* vsc = c.v_scale + unit * Lt::v_meta_unit(c.Tq);
-  const float* vze = c.v_zero + unit * Lt::v_meta_unit(c.Tq);
+  const MT* vsc = reinterpret_cast<const MT*>(c.v_scale) + unit * Lt::v_meta_unit(c.Tq);
+  const MT* vze = reinterpret_cast<const MT*>(c.v_zero) + unit * Lt::v_meta_unit(c.Tq);
   const T* kr = reinterpret_cast<const T*>(c.k_res) + unit * c.R * D;
   const T* vr = reinterpret_cast<const T*>(c.v_res) + unit * c.R * D;
 
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_simt(DecodeArgs a) {
 #pragma unroll
       for (int i = 0; i < CPL; ++i) {
         const int d = lane + 32 * i;
-        const float s = ksc[tile * D + d], z = kze[tile * D + d];
+        const float s = to_f32(ksc[tile * D + d]), z = to_f32(kze[tile * D + d]);
 #pragma unroll
         for (int h = 0; h < GQ; ++h) {
           qk[warp][h][d] = qs[h][d] * s;
@@ -114,8 +114,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_simt(DecodeArgs a) {
       for (int h = 0; h < GQ; ++h) lg[h] = warp_sum(bias[h]);
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
-        vs[warp][lane][j] = vsc[(tok0 + lane) * NJ + j];
-        vz[warp][lane][j] = vze[(tok0 + lane) * NJ + j];
+        vs[warp][lane][j] = to_f32(vsc[(tok0 + lane) * NJ + j]);
+        vz[warp][lane][j] = to_f32(vze[(tok0 + lane) * NJ + j]);
       }
       __syncwarp();
       // scores: lane = token tok0 + lane
@@ -242,33 +242,33 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_simt(DecodeArgs a) {
   finish_unit<D, GQ, T>(a, b, kv, &last_flag);
 }
 
-template <int D, int BITS, int GQ, typename T>
+template <int D, int BITS, int GQ, typename T, typename MT>
 cudaError_t simt_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1) {
   dim3 grid((unsigned)a.n_split, (unsigned)a.units);
   if (e0) cudaEventRecord(e0, s);
-  decode_split_simt<D, BITS, GQ, T><<<grid, kWarps * 32, 0, s>>>(a);
+  decode_split_simt<D, BITS, GQ, T, MT><<<grid, kWarps * 32, 0, s>>>(a);
   cudaError_t err = cudaGetLastError();
   if (e1) cudaEventRecord(e1, s);
   return err;
 }
 
-template <int D, int BITS, typename T>
+template <int D, int BITS, typename T, typename M>
 cudaError_t simt_g(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1) {
   switch (a.gq) {
-    case 1: return simt_t<D, BITS, 1, T>(a, s, e0, e1);
-    case 2: return simt_t<D, BITS, 2, T>(a, s, e0, e1);
-    case 4: return simt_t<D, BITS, 4, T>(a, s, e0, e1);
-    case 8: return simt_t<D, BITS, 8, T>(a, s, e0, e1);
+    case 1: return simt_t<D, BITS, 1, T, M>(a, s, e0, e1);
+    case 2: return simt_t<D, BITS, 2, T, M>(a, s, e0, e1);
+    case 4: return simt_t<D, BITS, 4, T, M>(a, s, e0, e1);
+    case 8: return simt_t<D, BITS, 8, T, M>(a, s, e0, e1);
   }
   return cudaErrorInvalidValue;
 }
 
-template <int BITS, typename T>
+template <int BITS, typename T, typename M>
 cudaError_t simt_d(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1) {
   switch (a.D) {
-    case 32: return simt_g<32, BITS, T>(a, s, e0, e1);
-    case 64: return simt_g<64, BITS, T>(a, s, e0, e1);
-    case 128: return simt_g<128, BITS, T>(a, s, e0, e1);
+    case 32: return simt_g<32, BITS, T, M>(a, s, e0, e1);
+    case 64: return simt_g<64, BITS, T, M>(a, s, e0, e1);
+    case 128: return simt_g<128, BITS, T, M>(a, s, e0, e1);
   }
   return cudaErrorInvalidValue;
 }
@@ -277,10 +277,17 @@ cudaError_t simt_d(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEven
 
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0,
                                cudaEvent_t e1) {
-  if (a.bits == 2 && a.dtype == 0) return simt_d<2, __half>(a, s, e0, e1);
-  if (a.bits == 2 && a.dtype == 1) return simt_d<2, float>(a, s, e0, e1);
-  if (a.bits == 4 && a.dtype == 0) return simt_d<4, __half>(a, s, e0, e1);
-  if (a.bits == 4 && a.dtype == 1) return simt_d<4, float>(a, s, e0, e1);
+  if (a.meta == 1) {  // binary16 scales and zeros: fp16 caches only
+    if (a.dtype != 0) return cudaErrorInvalidValue;
+    if (a.bits == 2) return simt_d<2, __half, __half>(a, s, e0, e1);
+    if (a.bits == 4) return simt_d<4, __half, __half>(a, s, e0, e1);
+    return cudaErrorInvalidValue;
+  }
+  if (a.meta != 0) return cudaErrorInvalidValue;
+  if (a.bits == 2 && a.dtype == 0) return simt_d<2, __half, float>(a, s, e0, e1);
+  if (a.bits == 2 && a.dtype == 1) return simt_d<2, float, float>(a, s, e0, e1);
+  if (a.bits == 4 && a.dtype == 0) return simt_d<4, __half, float>(a, s, e0, e1);
+  if (a.bits == 4 && a.dtype == 1) return simt_d<4, float, float>(a, s, e0, e1);
   return cudaErrorInvalidValue;
 }
 

@@ -1,1398 +1,19 @@
-// kivi_decode_tc.cu -- split-context decode attention over the packed KIVI
-// cache with both contractions on tensor cores (mma.sync, fp16 operands,
-// fp32 accumulation), the split merge fused in.
-//
-// Method: "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache",
-// study.space summary: decode attention runs over the quantized ("grouped")
-// part and is combined with the full-precision residual part; mlsanity.com
-// index page, "Abstract (arXiv)": loading the cache bounds decode.  Both parts
-// enter one online softmax; each CTA writes (m, l, acc[D]) per query head to
-// the workspace and the last CTA of the unit merges the splits.
-//
-// Per CTA: a contiguous range of work indices over (unit, 32-token tile)
-// pairs (persistent, stream-K), all query heads of the GQA group.  The CTA
-// that ends a unit also folds in the unit's residual window (CUDA cores).
-//   * memory: a producer warp issues 1-D bulk copies (cp.async.bulk,
-//     completion on a "full" mbarrier) of each stage -- NW tiles of key
-//     codes, key scales, key zeros, value codes, value scales, value zeros,
-//     six contiguous ranges -- into a ring of shared-memory stages; NW
-//     consumer warps take one tile each and release the stage on an "empty"
-//     mbarrier.  No CTA-wide barrier in the streaming loop.
-//   * codes as fp16 operands: a 2-bit word holds code i at bits 2i, a 4-bit
-//     word code i at bits 4i.  A "pair" (two codes, one per 16-bit half) is
-//     taken out with a mask after at most one shift, which leaves each code
-//     at some bit e < 10 of its half: read as fp16 that is the exact
-//     subnormal c * 2^(e - 24).  The other operand's row for that k carries
-//     the factor 2^(S - e), so every product is c * x * 2^(S - 24) and the
-//     fp32 result is rescaled once by 2^(24 - S).
-//   * scores: S = K q'^T, key codes as the A operand (16 tokens x 16
-//     channels per mma; lane tq of a row owns the code pairs
-//     [tq*D/8, (tq+1)*D/8) of the token), q'_{h,d} = q_{h,d} s_{g,d} split
-//     into fp16 hi and lo; head h uses columns 2(h%4) (hi) and 2(h%4)+1 (lo)
-//     of n-tile h/4, so each lane's accumulator pair is one head.
-//     score = sum_d q'_d c_d + sum_d q_d z_{g,d}.
-//   * softmax: running max and sum in log2 units (q pre-scaled by
-//     softmax_scale * log2 e, exp2f); the cross-lane max is formed only when
-//     some score exceeds the running max (a warp vote), so p <= 1 always.
-//   * values: O += V^T p' on tensor cores, value codes as the A operand
-//     (16 channels x 16 tokens), p'_{t,h} = p_{t,h} s_{t,j} split into hi and
-//     lo columns as above; the zero enters as sum_t p_t z_{t,j}.
-// The q' and p' fragments are built cooperatively (each lane converts a few
-// values and stores them in fragment order, XOR-swizzled, in per-warp shared
-// memory).
-#include <cuda.h>
-#include <string.h>
-
-#include "kivi_internal.cuh"
+// kivi_decode_tc.cu -- instances of the tensor-core decode kernel
+// (kivi_decode_tc.cuh) with binary32 scales and zeros, and the entry points
+// that select an instance.
+#include "kivi_decode_tc.cuh"
 
 namespace kivi {
 namespace {
 
-constexpr float kNegInf = -__builtin_huge_valf();
-constexpr long long kWaitCycles = 1LL << 32;  // ~2 s: bounded wait on our own copies
-constexpr int kSuspendNs = 1000;  // a waiting thread sleeps up to this long per try
-
-// Code pairs of one 32-bit word.  2-bit: pair i (i < 8) = codes i and i + 8;
-// 4-bit: pair i (i < 4) = codes i and i + 4.  (w >> shift(i)) & mask(i) puts
-// the pair's codes at bit e(i) of the low and the high half.
-template <int BITS>
-struct Pairs;
-template <>
-struct Pairs<2> {
-  static constexpr int PPW = 8;   // pairs per word
-  static constexpr int EMAX = 8;  // largest e
-  __host__ __device__ static constexpr int e(int i) { return i < 5 ? 2 * i : 2 * (i - 5); }
-  __host__ __device__ static constexpr int shift(int i) { return i < 5 ? 0 : 10; }
-  __host__ __device__ static constexpr uint32_t mask(int i) { return 0x00030003u << e(i); }
-};
-template <>
-struct Pairs<4> {
-  static constexpr int PPW = 4;
-  static constexpr int EMAX = 4;
-  __host__ __device__ static constexpr int e(int i) { return 4 * (i & 1); }
-  __host__ __device__ static constexpr int shift(int i) { return i < 2 ? 0 : 8; }
-  __host__ __device__ static constexpr uint32_t mask(int i) { return 0x000F000Fu << e(i); }
-};
-
-// NW consumer warps (TPW 32-token tiles each per stage) and one producer
-// warp per CTA.  Measured on B200: one query head per KV head runs best as
-// 4-warp CTAs, two tiles per warp at 2-bit (two CTAs per SM) and one at 4-bit
-// (three per SM); grouped heads run best as one CTA per SM with 11 (GQ 2, 4)
-// or 7 (GQ 8) consumer warps sharing one ring.
-template <int D, int BITS, int GQ>
-struct Geo {
-  static constexpr int NW = GQ == 1 ? 4 : (GQ == 8 ? 7 : 11);
-  static constexpr int TPW = (GQ == 1 && BITS == 2) ? 2 : 1;  // tiles per warp and stage
-  static constexpr int THREADS = (NW + 1) * 32;
-  static constexpr int kStage = NW * TPW;       // tiles per pipeline stage
-  static constexpr int E = 32 / BITS;
-  static constexpr int WK = D / E;       // key words per token
-  static constexpr int NJ = D / kGv;     // value groups per token
-  static constexpr int KSL = D / 16;     // k-slices of the score product
-  static constexpr int NSL = kTile / 16;  // k-slices of the value product
-  static constexpr int KC_B = kTile * WK * 4;
-  static constexpr int KM_B = D * 4;
-  static constexpr int VC_B = (kTile / E) * D * 4;
-  static constexpr int VM_B = kTile * NJ * 4;
-  static constexpr int TILE_B = KC_B + 2 * KM_B + VC_B + 2 * VM_B;
-  static constexpr int O_KC = 0;
-  static constexpr int O_KS = O_KC + kStage * KC_B;
-  static constexpr int O_KZ = O_KS + kStage * KM_B;
-  static constexpr int O_VC = O_KZ + kStage * KM_B;
-  static constexpr int O_VS = O_VC + kStage * VC_B;
-  static constexpr int O_VZ = O_VS + kStage * VM_B;
-  static constexpr int STAGE_B = (O_VZ + kStage * VM_B + 1023) / 1024 * 1024;
-  static constexpr int NSTAGE = (NW == 4 && TPW == 1 && BITS == 2) ? 3 : 2;
-  static constexpr int NPB = GQ == 8 ? 2 : 1;  // n-tiles of 8 columns (4 heads x hi, lo)
-  static constexpr int PST = TPW * kTile + 8;  // p buffer stride per head (floats)
-  // per-warp scratch (bytes): fragment blocks of 32 lanes x 2 words
-  static constexpr int QB_B = NPB * KSL * 256;        // q' B fragments (score product)
-  static constexpr int PB_B = NPB * NJ * NSL * 256;   // p' B fragments (value product)
-  static constexpr int PBUF_B = GQ * PST * 4;         // p per head and token
-  static constexpr int WARP_B = TPW * (QB_B + PB_B) + PBUF_B;
-  // whole CTA
-  static constexpr int O_WARP = NSTAGE * STAGE_B;
-  static constexpr int O_QS = O_WARP + NW * WARP_B;    // q (fp32, scaled) for the window path
-  static constexpr int O_MG = O_QS + GQ * D * 4;       // per-warp (m, l, acc[D]) for the merge
-  static constexpr int O_BAR = O_MG + NW * GQ * (D + 2) * 4;  // full[NSTAGE], empty[NSTAGE]
-  static constexpr int O_FLAG = O_BAR + 2 * NSTAGE * 8;
-  static constexpr int SMEM_B = O_FLAG + 16;
-  static_assert(SMEM_B <= 227 * 1024, "shared memory per CTA");
-  static_assert(O_BAR % 8 == 0 && WARP_B % 16 == 0, "alignment");
-  static constexpr int MIN_CTAS = NW == 4 ? (TPW == 2 ? 2 : 3) : 1;
-  // key operand: code pairs per lane and row, words a lane loads per row
-  static constexpr int PPL = D / 8;
-  static constexpr int PPW = Pairs<BITS>::PPW;
-  static constexpr bool WHOLE = PPL >= PPW;  // a lane's pairs fill whole words
-  static constexpr int NWL = WHOLE ? PPL / PPW : 1;
-  // operand scale offsets: the factor 2^(S - e) lies in [2^-S, 2^S]
-  static constexpr int SK = Pairs<BITS>::EMAX / 2;
-  static constexpr int SV = BITS == 2 ? 3 : 2;  // value e: 2-bit 0,2,4,6; 4-bit 0,4
-  // fp16 residual window through the ring: a window stage holds WT tokens of
-  // K, then of V, as 2-D tensor-copy boxes of BW columns (rows of RB bytes)
-  // in the hardware's 128-byte (64-byte when D = 32) swizzle
-  static constexpr int WT = kTile;
-  static constexpr int BW = D < 64 ? D : 64;
-  static constexpr int NBX = D / BW;
-  static constexpr int RB = BW * 2;
-  static constexpr int BOX_B = WT * RB;
-  static constexpr int WTILE_B = 2 * NBX * BOX_B;     // one 32-token window tile (K, V)
-  static constexpr int WPS = STAGE_B / WTILE_B;       // window tiles per stage
-  static_assert(WPS >= 1, "a window tile fits one ring slot");
-  static_assert(WTILE_B % 1024 == 0, "window tiles keep the 1024-byte alignment");
-  static_assert(STAGE_B % 1024 == 0, "swizzled boxes start on 1024-byte boundaries");
-};
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, int count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-// 2-D tensor copy (no multicast) of one box at element coordinates (x, y)
-// into shared memory, completion on an mbarrier.
-__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                       uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendNs)
-      : "memory");
-  return ok != 0;
-}
-// Wait for a phase; gives up (returns false) after kWaitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return false;
-  }
-  return true;
-}
-
-// D (16x8, fp32) += A (16x16, fp16, row) * B (16x8, fp16, col).  Not volatile:
-// no side effects, so the compiler may schedule independent chains together.
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Four 8x8 fp16 matrices from shared memory; lanes 8i..8i+7 give the row
-// addresses of matrix i.  .trans delivers each matrix transposed.
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(p))
-               : "memory");
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(p))
-               : "memory");
-}
-
-__device__ __forceinline__ uint32_t h2_bits(__half2 h) {
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// x = hi + lo in fp16 for two values at once (low half: a, high half: b).
-__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
-  const __half2 h = __floats2half2_rn(a, b);
-  const float2 f = __half22float2(h);
-  hi = h2_bits(h);
-  lo = h2_bits(__floats2half2_rn(a - f.x, b - f.y));
-}
-
-// Word offset of fragment slot `lane2` (= 4 n + tq) in a 64-word B block for
-// k-slice `sl`: an XOR swizzle that keeps the cooperative fragment stores
-// free of bank conflicts while each lane still reads a contiguous 8 bytes.
-__device__ __forceinline__ int frag_word(int lane2, int sl) { return 2 * (lane2 ^ (4 * (sl & 3))); }
-
-// Consumer-only barrier (the producer warp keeps streaming meanwhile).
-template <int NW>
-__device__ __forceinline__ void consumers_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
-}
-
-template <int D, int BITS, int GQ, typename T>
-__global__ void __launch_bounds__(Geo<D, BITS, GQ>::THREADS, Geo<D, BITS, GQ>::MIN_CTAS)
-    decode_stream_tc(const DecodeArgs args, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV) {
-  using G = Geo<D, BITS, GQ>;
-  using PR = Pairs<BITS>;
-  constexpr int kW = G::NW;
-  constexpr int kStage = G::kStage;
-  using Lt = Layout<D, BITS>;
-  constexpr int E = G::E, WK = G::WK, NJ = G::NJ, KSL = G::KSL, NSL = G::NSL;
-  constexpr int NM = D / 16;  // value m-tiles (16 channels each)
-  constexpr int NPB = G::NPB;
-  constexpr int PST = G::PST;
-  constexpr int TPW = G::TPW;
-  constexpr int CPL = D / 32;  // window path: channels per lane
-  constexpr float kKeyOut = (float)(1 << (24 - G::SK));
-  constexpr float kValOut = (float)(1 << (24 - G::SV));
-  extern __shared__ __align__(1024) unsigned char smem[];
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, tq = lane & 3;
-  const int cta = blockIdx.x;
-
-  // launched with programmatic stream serialization: the CTAs may start
-  // while the preceding grid drains; every thread waits for it to complete
-  // (and its writes to be visible) before touching global memory, and the
-  // next grid may be scheduled as soon as SM room frees up
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-  DecodeArgs a = args;
-  const bool dev = args.dev_state != nullptr;
-  if (dev) {
-    // device counters as the preceding append launch found them; decode the
-    // cache after that append (it flushed when r was R)
-    const DevState st0 = *args.dev_state;
-    if (st0.status != 0 || st0.n_q + st0.r + 1 > args.c.Tq + args.c.R) return;  // cache full
-    const bool fl = st0.r == args.c.R;
-    a.n_q = fl ? st0.n_q + args.c.R : st0.n_q;
-    a.r = fl ? 1 : st0.r + 1;
-    const StreamPlan pl =
-        plan_stream_core(args.units, a.n_q, a.r, sizeof(T) == 2, gridDim.x, args.seg_cap);
-    a.tiles_per_cta = pl.W;
-    a.win_weight = pl.win_weight;
-    a.max_seg = pl.max_seg;
-    a.n_split = pl.max_seg;
-    a.new_k = nullptr;  // the append launch wrote the token
-  }
-  const int Hq = a.Hkv * GQ;
-  const CacheView& c = a.c;
-
-  float* qs = reinterpret_cast<float*>(smem + G::O_QS);
-  float* mg_m = reinterpret_cast<float*>(smem + G::O_MG);  // [kW][GQ]
-  float* mg_l = mg_m + kW * GQ;                              // [kW][GQ]
-  float* mg_acc = mg_l + kW * GQ;                            // [kW][GQ][D]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::O_BAR);
-  uint64_t* empty = full + G::NSTAGE;
-  int* flag = reinterpret_cast<int*>(smem + G::O_FLAG);  // [0] abort, [1] merge flag
-
-  const long long n_qt = a.n_q / kTile;
-  const long long UP = n_qt + a.win_weight;  // work indices per unit
-  const long long total = (long long)a.units * UP;
-  const long long W = a.tiles_per_cta;
-  const long long G0 = (long long)cta * W;
-  const long long G1 = min(total, G0 + W);
-
-  if (tid == 0) {
-    for (int s = 0; s < G::NSTAGE; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kW);
-    }
-    // swizzled window boxes need 1024-byte aligned stages: refuse (abort
-    // flag, NaN outputs) rather than read a mis-swizzled layout
-    flag[0] = (sizeof(T) == 2 && (smem_u32(smem) & 1023u) != 0) ? 1 : 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (sizeof(T) == 4 && a.new_k != nullptr) {
-    // fused append, fp32 window (read by generic loads after the barrier
-    // below): the CTA that owns a unit's window writes the unit's new token
-    // into window slot new_slot.  (fp16: the warp that takes the window tile
-    // holding the slot patches the token into shared memory and the cache.)
-    for (long long u = G0 / UP; G0 < G1 && u <= (G1 - 1) / UP; ++u) {
-      if (cta != (u * UP + n_qt) / W) continue;
-      T* kr = reinterpret_cast<T*>(c.k_res) + (u * c.R + a.new_slot) * D;
-      T* vr = reinterpret_cast<T*>(c.v_res) + (u * c.R + a.new_slot) * D;
-      const T* kn = reinterpret_cast<const T*>(a.new_k) + u * D;
-      const T* vn = reinterpret_cast<const T*>(a.new_v) + u * D;
-      for (int i = tid; i < D; i += G::THREADS) {
-        kr[i] = kn[i];
-        vr[i] = vn[i];
-      }
-    }
-  }
-  if (warp < kW) {
-    // fragment columns of absent heads stay zero
-    unsigned char* wb = smem + G::O_WARP + warp * G::WARP_B;
-    for (int i = lane; i < TPW * (G::QB_B + G::PB_B) / 4; i += 32) reinterpret_cast<uint32_t*>(wb)[i] = 0u;
-  }
-  __syncthreads();
-
-  if (warp == kW) {
-    // ---------------- producer warp: one thread streams this CTA's stages
-    if (lane == 0 && G0 < G1) {
-      long long st = 0;
-      for (long long u = G0 / UP; u <= (G1 - 1) / UP; ++u) {
-        const long long base = u * UP;
-        if (cta < base / W || cta > (base + n_qt) / W) continue;  // no work of u here
-        const long long t_end = min(G1 - base, n_qt);
-        const uint32_t* kc_u = c.k_codes + u * Lt::k_codes_unit(c.Tq);
-        const float* ks_u = c.k_scale + u * Lt::k_meta_unit(c.Tq);
-        const float* kz_u = c.k_zero + u * Lt::k_meta_unit(c.Tq);
-        const uint32_t* vc_u = c.v_codes + u * Lt::v_codes_unit(c.Tq);
-        const float* vs_u = c.v_scale + u * Lt::v_meta_unit(c.Tq);
-        const float* vz_u = c.v_zero + u * Lt::v_meta_unit(c.Tq);
-        for (long long t0 = max(G0 - base, 0ll); t0 < t_end; t0 += kStage, ++st) {
-          const int s = (int)(st % G::NSTAGE);
-          if (st >= G::NSTAGE &&
-              !mbar_wait(&empty[s], (uint32_t)(((st / G::NSTAGE) - 1) & 1))) {
-            atomicExch(&flag[0], 1);
-            break;
-          }
-          if (*(volatile int*)&flag[0]) break;
-          unsigned char* buf = smem + s * G::STAGE_B;
-          const int n = (int)min((long long)kStage, t_end - t0);
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          mbar_expect_tx(&full[s], (uint32_t)(n * G::TILE_B));
-          bulk_copy(buf + G::O_KC, kc_u + t0 * kTile * WK, n * G::KC_B, &full[s]);
-          bulk_copy(buf + G::O_KS, ks_u + t0 * D, n * G::KM_B, &full[s]);
-          bulk_copy(buf + G::O_KZ, kz_u + t0 * D, n * G::KM_B, &full[s]);
-          bulk_copy(buf + G::O_VC, vc_u + t0 * (kTile / E) * D, n * G::VC_B, &full[s]);
-          bulk_copy(buf + G::O_VS, vs_u + t0 * kTile * NJ, n * G::VM_B, &full[s]);
-          bulk_copy(buf + G::O_VZ, vz_u + t0 * kTile * NJ, n * G::VM_B, &full[s]);
-        }
-        if (*(volatile int*)&flag[0]) break;
-        if (a.r > 0 && cta == (base + n_qt) / W) {
-          const T* kr = reinterpret_cast<const T*>(c.k_res) + u * c.R * D;
-          const T* vr = reinterpret_cast<const T*>(c.v_res) + u * c.R * D;
-          if constexpr (sizeof(T) == 2) {
-            // this CTA owns the unit's residual window: stream it through
-            // the ring, WT tokens of K and of V per stage
-            for (int w0 = 0; w0 < a.r; w0 += G::WT * G::WPS, ++st) {
-              const int s = (int)(st % G::NSTAGE);
-              if (st >= G::NSTAGE &&
-                  !mbar_wait(&empty[s], (uint32_t)(((st / G::NSTAGE) - 1) & 1))) {
-                atomicExch(&flag[0], 1);
-                break;
-              }
-              if (*(volatile int*)&flag[0]) break;
-              unsigned char* buf = smem + s * G::STAGE_B;
-              const int ntile = min(G::WPS, (a.r - w0 + G::WT - 1) / G::WT);
-              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-              mbar_expect_tx(&full[s], (uint32_t)(ntile * G::WTILE_B));
-              for (int j = 0; j < ntile; ++j) {
-                unsigned char* tb = buf + j * G::WTILE_B;
-                const int y = (int)(u * c.R + w0 + j * G::WT);  // row of the [units * R][D] window
-#pragma unroll
-                for (int bx = 0; bx < G::NBX; ++bx) {
-                  tma_2d(tb + bx * G::BOX_B, &tmK, bx * G::BW, y, &full[s]);
-                  tma_2d(tb + (G::NBX + bx) * G::BOX_B, &tmV, bx * G::BW, y, &full[s]);
-                }
-              }
-            }
-          } else {
-            // fp32 window (CUDA-core path): pull it into L2 while the
-            // consumers work through the unit's last stages
-            const uint32_t wbytes = (uint32_t)((size_t)a.r * D * sizeof(T));
-            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kr), "r"(wbytes) : "memory");
-            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vr), "r"(wbytes) : "memory");
-          }
-        }
-      }
-    }
-    __syncwarp();
-  } else {
-    // ---------------- consumer warps
-    unsigned char* wb = smem + G::O_WARP + warp * G::WARP_B;
-    uint32_t* qB = reinterpret_cast<uint32_t*>(wb);                     // [TPW][NPB][KSL][64]
-    uint32_t* pB = reinterpret_cast<uint32_t*>(wb + TPW * G::QB_B);     // [TPW][NPB][NJ][NSL][64]
-    __half* pBh = reinterpret_cast<__half*>(pB);
-    float* pbuf = reinterpret_cast<float*>(wb + TPW * (G::QB_B + G::PB_B));  // [GQ][PST]
-
-    // -- q' build: lane classes.  Head class hc = lane % GL builds heads
-    // hc + GL x; within a class, lane index jl = lane / GL takes the
-    // "couples" (two adjacent pairs of one owner lane: B registers b0, b1 of
-    // k-slice sl for owner tq_o) with tq_o = jl & 3, sl = (jl >> 2) + (8/GL) m.
-    constexpr int GL = GQ < 4 ? GQ : 4;
-    constexpr int HX = GQ / GL;
-    constexpr int MC = (KSL * GL + 7) / 8;
-    const int hc = lane % GL, jl = lane / GL;
-    int cp_ch[MC];       // first channel c0 of the couple (pairs: c0, c0+1 | c0+PPW, c0+PPW+1)
-    int cp_w[MC];        // word offset of the owner's slot for column 0 in block sl
-    int cp_s3[MC];       // sl & 3 (swizzle)
-    float cp_f0[MC], cp_f1[MC];  // 2^(SK - e) of the two pairs
-    bool cp_ok[MC];
-#pragma unroll
-    for (int m = 0; m < MC; ++m) {
-      const int tq_o = jl & 3, sl = (jl >> 2) + (8 / GL) * m;
-      cp_ok[m] = sl < KSL;
-      const int slc = cp_ok[m] ? sl : 0;
-      const int pidx0 = tq_o * G::PPL + 2 * slc;
-      const int wd = pidx0 / G::PPW, i0 = pidx0 % G::PPW;
-      cp_ch[m] = wd * E + i0;
-      cp_s3[m] = slc & 3;
-      cp_w[m] = slc * 64 + 2 * tq_o;
-      cp_f0[m] = __int_as_float((127 + G::SK - PR::e(i0)) << 23);
-      cp_f1[m] = __int_as_float((127 + G::SK - PR::e(i0 + 1)) << 23);
-    }
-    // -- key operand (D = 32, 2-bit): a lane's four pairs sit in word tq/2,
-    // pairs 4 (tq & 1) + jj -- shifts and masks differ per lane
-    uint32_t kS[4], kM[4];
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int i = 4 * (tq & 1) + jj;
-      kS[jj] = (uint32_t)Pairs<2>::shift(i);
-      kM[jj] = Pairs<2>::mask(i);
-    }
-    // -- value operand: lane tq takes the pairs at e = 2 tq (2-bit) or
-    // 4 (tq & 1) (4-bit) of its word; a0 / a1 unshifted, a2 / a3 after >> 8
-    const uint32_t vM = BITS == 2 ? (0x00030003u << (2 * tq))
-                                  : ((tq & 1) ? 0x00F000F0u : 0x000F000Fu);
-    const int vtw = BITS == 2 ? 0 : (tq >> 1);  // token-word offset of this lane
-    // -- p' build, lane = token t: its k-slice, owner slot and e
-    int pt_sl, pt_tq, pt_kp, pt_hf, pt_e;
-    if (BITS == 2) {
-      const int i = lane & 15;
-      pt_sl = lane >> 4; pt_tq = i & 3; pt_kp = (i >> 2) & 1; pt_hf = (i >> 3) & 1; pt_e = 2 * pt_tq;
-    } else {
-      const int tw = lane >> 3, i = lane & 7;
-      pt_sl = tw >> 1; pt_tq = 2 * (tw & 1) + (i & 1); pt_kp = (i >> 1) & 1; pt_hf = (i >> 2) & 1;
-      pt_e = 4 * (i & 1);
-    }
-    const float pt_f = __int_as_float((127 + G::SV - pt_e) << 23);
-    const int pt_base = pt_sl * 128 + 2 * pt_kp + pt_hf;  // halves, block (0, 0, pt_sl)
-    const int pt_s3 = pt_sl & 3;
-
-    // B-fragment column n = g of this lane carries a head (hi or lo part);
-    // lanes of absent heads' columns use zeros without loading them
-    const bool bcol = GQ >= 4 || g < 2 * GQ;
-    bool vh[NPB];  // this lane's score / accumulator head tq + 4p exists
-#pragma unroll
-    for (int p = 0; p < NPB; ++p) vh[p] = tq + 4 * p < GQ;
-
-    long long st = 0;  // ring position, in step with the producer
-    for (long long u = G0 / UP; G0 < G1 && u <= (G1 - 1) / UP; ++u) {
-      const long long base = u * UP;
-      // CTAs f_cta..l_cta cover the unit's tiles and its window start index;
-      // l_cta owns the window
-      const long long f_cta = base / W;
-      const long long l_cta = (base + n_qt) / W;
-      if (cta < f_cta || cta > l_cta) continue;
-      const long long b = u / a.Hkv;
-      const int kv = (int)(u % a.Hkv);
-      const T* qg = reinterpret_cast<const T*>(a.q) + (b * Hq + (long long)kv * GQ) * D;
-      const long long t_beg = max(G0 - base, 0ll);
-      const long long t_end = min(G1 - base, n_qt);
-      const int slot = (int)(cta - f_cta);
-      const int n_seg = (int)(l_cta - f_cta + 1);
-      const bool window_owner = a.r > 0 && cta == l_cta;
-
-      // q (scaled by softmax_scale log2 e) at this lane's couple channels,
-      // order c0, c0+PPW, c0+1, c0+PPW+1 (b0 low, b0 high, b1 low, b1 high)
-      float qf[HX][MC][4];
-#pragma unroll
-      for (int x = 0; x < HX; ++x)
-#pragma unroll
-        for (int m = 0; m < MC; ++m) {
-          const T* qh = qg + (hc + GL * x) * D + cp_ch[m];
-          qf[x][m][0] = to_f32(qh[0]) * a.qscale;
-          qf[x][m][1] = to_f32(qh[G::PPW]) * a.qscale;
-          qf[x][m][2] = to_f32(qh[1]) * a.qscale;
-          qf[x][m][3] = to_f32(qh[G::PPW + 1]) * a.qscale;
-        }
-      if (window_owner) {
-        for (int i = tid; i < GQ * D; i += kW * 32) qs[i] = to_f32(qg[i]) * a.qscale;
-        consumers_sync<kW>();  // qs is read by whichever warps take the window
-      }
-
-      float m_run[NPB], l_part[NPB];
-      float acc[NPB][NM][4];
-      float bv[GQ][NJ];  // sum_t p z per (head, value group), lane partial (lane = token)
-#pragma unroll
-      for (int p = 0; p < NPB; ++p) {
-        m_run[p] = kNegInf;
-        l_part[p] = 0.f;
-#pragma unroll
-        for (int m = 0; m < NM; ++m)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[p][m][e] = 0.f;
-      }
-#pragma unroll
-      for (int h = 0; h < GQ; ++h)
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) bv[h][j] = 0.f;
-
-      for (long long t0 = t_beg; t0 < t_end; t0 += kStage, ++st) {
-        if (*(volatile int*)&flag[0]) break;
-        const int s = (int)(st % G::NSTAGE);
-        const bool ok = mbar_wait(&full[s], (uint32_t)((st / G::NSTAGE) & 1));
-        if (!__all_sync(0xffffffffu, ok) || *(volatile int*)&flag[0]) {
-          if (lane == 0) atomicExch(&flag[0], 1);
-          break;
-        }
-        const unsigned char* buf = smem + s * G::STAGE_B;
-        const long long tw0 = t0 + (long long)warp * TPW;  // this warp's first tile
-        if (tw0 < t_end) {
-          // this warp's TPW tiles; a tile past the end of the segment reuses
-          // tile 0's data and is masked out (its scores are -inf, so p = 0)
-          bool tv[TPW];
-          const uint32_t* kc[TPW];
-          const float* ks[TPW];
-          const float* kz[TPW];
-          const uint32_t* vc[TPW];
-          const float* vs[TPW];
-          const float* vz[TPW];
-#pragma unroll
-          for (int tt = 0; tt < TPW; ++tt) {
-            tv[tt] = tw0 + tt < t_end;
-            const int ti = warp * TPW + (tv[tt] ? tt : 0);
-            kc[tt] = reinterpret_cast<const uint32_t*>(buf + G::O_KC) + ti * kTile * WK;
-            ks[tt] = reinterpret_cast<const float*>(buf + G::O_KS) + ti * D;
-            kz[tt] = reinterpret_cast<const float*>(buf + G::O_KZ) + ti * D;
-            vc[tt] = reinterpret_cast<const uint32_t*>(buf + G::O_VC) + ti * (kTile / E) * D;
-            vs[tt] = reinterpret_cast<const float*>(buf + G::O_VS) + ti * kTile * NJ;
-            vz[tt] = reinterpret_cast<const float*>(buf + G::O_VZ) + ti * kTile * NJ;
-          }
-
-          // -- q' = q s 2^(SK - e) (hi, lo) into the B fragments; bias = q . z
-          float bk[TPW][HX];
-#pragma unroll
-          for (int tt = 0; tt < TPW; ++tt)
-#pragma unroll
-            for (int x = 0; x < HX; ++x) bk[tt][x] = 0.f;
-#pragma unroll
-          for (int m = 0; m < MC; ++m) {
-            if (!cp_ok[m]) continue;
-#pragma unroll
-            for (int tt = 0; tt < TPW; ++tt) {
-              const float2 sA = *reinterpret_cast<const float2*>(ks[tt] + cp_ch[m]);
-              const float2 sB = *reinterpret_cast<const float2*>(ks[tt] + cp_ch[m] + G::PPW);
-              const float2 zA = *reinterpret_cast<const float2*>(kz[tt] + cp_ch[m]);
-              const float2 zB = *reinterpret_cast<const float2*>(kz[tt] + cp_ch[m] + G::PPW);
-              const float s0 = sA.x * cp_f0[m], s1 = sB.x * cp_f0[m];
-              const float s2 = sA.y * cp_f1[m], s3 = sB.y * cp_f1[m];
-#pragma unroll
-              for (int x = 0; x < HX; ++x) {
-                const int h = hc + GL * x;
-                uint2 hi, lo;
-                split2(qf[x][m][0] * s0, qf[x][m][1] * s1, hi.x, lo.x);
-                split2(qf[x][m][2] * s2, qf[x][m][3] * s3, hi.y, lo.y);
-                uint32_t* blk = qB + tt * (G::QB_B / 4) + (h >> 2) * KSL * 64 + cp_w[m];
-                const int nh = 2 * (h & 3);
-                *reinterpret_cast<uint2*>(blk + 8 * (nh ^ cp_s3[m])) = hi;
-                *reinterpret_cast<uint2*>(blk + 8 * ((nh + 1) ^ cp_s3[m])) = lo;
-                float t = bk[tt][x];
-                t = fmaf(qf[x][m][0], zA.x, t);
-                t = fmaf(qf[x][m][1], zB.x, t);
-                t = fmaf(qf[x][m][2], zA.y, t);
-                t = fmaf(qf[x][m][3], zB.y, t);
-                bk[tt][x] = t;
-              }
-            }
-          }
-          // sum over the lanes of a head class; lane tq then holds head tq + 4p
-#pragma unroll
-          for (int tt = 0; tt < TPW; ++tt)
-#pragma unroll
-            for (int x = 0; x < HX; ++x)
-#pragma unroll
-              for (int o = GL; o < 32; o <<= 1)
-                bk[tt][x] += __shfl_xor_sync(0xffffffffu, bk[tt][x], o);
-          __syncwarp();
-
-          // -- scores: per tile 2 m-tiles of 16 tokens (rows g, g+8), KSL k-slices
-          uint32_t kw[TPW][2][2][G::NWL];
-#pragma unroll
-          for (int tt = 0; tt < TPW; ++tt)
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-              for (int r = 0; r < 2; ++r) {
-                const uint32_t* row = kc[tt] + (16 * mt + 8 * r + g) * WK +
-                                      (G::WHOLE ? tq * G::NWL : (tq >> 1));
-                if constexpr (G::NWL == 4) {
-                  const uint4 v = *reinterpret_cast<const uint4*>(row);
-                  kw[tt][mt][r][0] = v.x; kw[tt][mt][r][1] = v.y;
-                  kw[tt][mt][r][2] = v.z; kw[tt][mt][r][3] = v.w;
-                } else if constexpr (G::NWL == 2) {
-                  const uint2 v = *reinterpret_cast<const uint2*>(row);
-                  kw[tt][mt][r][0] = v.x; kw[tt][mt][r][1] = v.y;
-                } else {
-                  kw[tt][mt][r][0] = row[0];
-                }
-              }
-          auto key_reg = [&](const uint32_t (&w)[G::NWL], int jj) -> uint32_t {
-            if constexpr (G::WHOLE) {
-              const int i = jj % G::PPW;
-              return (w[jj / G::PPW] >> PR::shift(i)) & PR::mask(i);
-            } else {
-              return (w[0] >> kS[jj & 3]) & kM[jj & 3];
-            }
-          };
-          float dq[TPW][NPB][2][4];
-#pragma unroll
-          for (int tt = 0; tt < TPW; ++tt)
-#pragma unroll
-            for (int p = 0; p < NPB; ++p)
-#pragma unroll
-              for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dq[tt][p][mt][e] = 0.f;
-#pragma unroll
-          for (int sl = 0; sl < KSL; ++sl) {
-#pragma unroll
-            for (int tt = 0; tt < TPW; ++tt) {
-              uint2 bq[NPB];
-#pragma unroll
-              for (int p = 0; p < NPB; ++p)
-                bq[p] = bcol ? *reinterpret_cast<const uint2*>(qB + tt * (G::QB_B / 4) +
-                                                               (p * KSL + sl) * 64 + frag_word(lane, sl))
-                             : make_uint2(0u, 0u);
-#pragma unroll
-              for (int mt = 0; mt < 2; ++mt) {
-                const uint32_t a0 = key_reg(kw[tt][mt][0], 2 * sl);
-                const uint32_t a2 = key_reg(kw[tt][mt][0], 2 * sl + 1);
-                const uint32_t a1 = key_reg(kw[tt][mt][1], 2 * sl);
-                const uint32_t a3 = key_reg(kw[tt][mt][1], 2 * sl + 1);
-#pragma unroll
-                for (int p = 0; p < NPB; ++p)
-                  mma16816(dq[tt][p][mt], a0, a1, a2, a3, bq[p].x, bq[p].y);
-              }
-            }
-          }
-
-          // -- scores of head tq + 4p for tokens 32 tt + {g, g+8, 16+g, 24+g}
-          float sc[NPB][4 * TPW];
-#pragma unroll
-          for (int p = 0; p < NPB; ++p)
-#pragma unroll
-            for (int tt = 0; tt < TPW; ++tt) {
-              const float bias = bk[tt][HX > 1 ? p : 0];
-#pragma unroll
-              for (int mt = 0; mt < 2; ++mt) {
-                const float v0 = fmaf(dq[tt][p][mt][0] + dq[tt][p][mt][1], kKeyOut, bias);
-                const float v1 = fmaf(dq[tt][p][mt][2] + dq[tt][p][mt][3], kKeyOut, bias);
-                sc[p][4 * tt + 2 * mt] = tv[tt] ? v0 : kNegInf;
-                sc[p][4 * tt + 2 * mt + 1] = tv[tt] ? v1 : kNegInf;
-              }
-            }
-          // -- online softmax: the running max moves only when a score exceeds it
-          float lm[NPB];
-          bool need = false;
-#pragma unroll
-          for (int p = 0; p < NPB; ++p) {
-            float v = sc[p][0];
-#pragma unroll
-            for (int i = 1; i < 4 * TPW; ++i) v = fmaxf(v, sc[p][i]);
-            lm[p] = v;
-            need |= vh[p] && v > m_run[p];
-          }
-          if (__any_sync(0xffffffffu, need)) {
-            float al[NPB];
-#pragma unroll
-            for (int p = 0; p < NPB; ++p) {
-              float tm = lm[p];
-              tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
-              tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
-              tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
-              const float mn = fmaxf(m_run[p], tm);
-              al[p] = exp2f(m_run[p] - mn);
-              m_run[p] = mn;
-              l_part[p] *= al[p];
-#pragma unroll
-              for (int m = 0; m < NM; ++m)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[p][m][e] *= al[p];
-            }
-#pragma unroll
-            for (int h = 0; h < GQ; ++h) {
-              const float ah = __shfl_sync(0xffffffffu, al[h >> 2], h & 3);
-#pragma unroll
-              for (int j = 0; j < NJ; ++j) bv[h][j] *= ah;
-            }
-          }
-#pragma unroll
-          for (int p = 0; p < NPB; ++p) {
-            float ps = 0.f;
-#pragma unroll
-            for (int i = 0; i < 4 * TPW; ++i) {
-              const float pv = exp2f(sc[p][i] - m_run[p]);
-              ps += pv;
-              const int tok = 32 * (i >> 2) + 16 * ((i >> 1) & 1) + 8 * (i & 1) + g;
-              if (vh[p]) pbuf[(tq + 4 * p) * PST + tok] = pv;
-            }
-            l_part[p] += ps;
-          }
-          __syncwarp();
-
-          // -- p' = p s_v 2^(SV - e) (hi, lo) into the B fragments; bias_v += p z_v
-#pragma unroll
-          for (int tt = 0; tt < TPW; ++tt) {
-            float sv[NJ], zv[NJ];
-            if constexpr (NJ == 4) {
-              const float4 s4 = *reinterpret_cast<const float4*>(vs[tt] + lane * NJ);
-              const float4 z4 = *reinterpret_cast<const float4*>(vz[tt] + lane * NJ);
-              sv[0] = s4.x; sv[1] = s4.y; sv[2] = s4.z; sv[3] = s4.w;
-              zv[0] = z4.x; zv[1] = z4.y; zv[2] = z4.z; zv[3] = z4.w;
-            } else {
-#pragma unroll
-              for (int j = 0; j < NJ; ++j) {
-                sv[j] = vs[tt][lane * NJ + j];
-                zv[j] = vz[tt][lane * NJ + j];
-              }
-            }
-#pragma unroll
-            for (int h = 0; h < GQ; ++h) {
-              const float ph = pbuf[h * PST + 32 * tt + lane];
-              const float phf = ph * pt_f;
-              const int nh = 2 * (h & 3);
-              const int o_hi = pt_base + 4 * (4 * (nh ^ pt_s3) + pt_tq);
-              const int o_lo = pt_base + 4 * (4 * ((nh + 1) ^ pt_s3) + pt_tq);
-#pragma unroll
-              for (int j = 0; j < NJ; ++j) {
-                bv[h][j] = fmaf(ph, zv[j], bv[h][j]);
-                const float x = phf * sv[j];
-                const __half hi = __float2half_rn(x);
-                const __half lo = __float2half_rn(x - __half2float(hi));
-                __half* blk = pBh + tt * (G::PB_B / 2) + ((h >> 2) * NJ + j) * NSL * 128;
-                blk[o_hi] = hi;
-                blk[o_lo] = lo;
-              }
-            }
-          }
-          __syncwarp();
-
-          // -- P.V: per tile, k-slice sl and value group j, m-tiles 2j
-          // (channels 32j+4g, +1) and 2j+1 (+2, +3)
-#pragma unroll
-          for (int tt = 0; tt < TPW; ++tt) {
-#pragma unroll
-            for (int sl = 0; sl < NSL; ++sl) {
-              const int tw = BITS == 2 ? sl : 2 * sl + vtw;
-#pragma unroll
-              for (int j = 0; j < NJ; ++j) {
-                const uint4 w = *reinterpret_cast<const uint4*>(vc[tt] + tw * D + 32 * j + 4 * g);
-                const uint32_t x0 = w.x & vM, x2 = (w.x >> 8) & vM;
-                const uint32_t x1 = w.y & vM, x3 = (w.y >> 8) & vM;
-                const uint32_t y0 = w.z & vM, y2 = (w.z >> 8) & vM;
-                const uint32_t y1 = w.w & vM, y3 = (w.w >> 8) & vM;
-#pragma unroll
-                for (int p = 0; p < NPB; ++p) {
-                  const uint2 bb = bcol ? *reinterpret_cast<const uint2*>(
-                                              pB + tt * (G::PB_B / 4) + ((p * NJ + j) * NSL + sl) * 64 +
-                                              frag_word(lane, sl))
-                                        : make_uint2(0u, 0u);
-                  mma16816(acc[p][2 * j], x0, x1, x2, x3, bb.x, bb.y);
-                  mma16816(acc[p][2 * j + 1], y0, y1, y2, y3, bb.x, bb.y);
-                }
-              }
-            }
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-      }
-      // ---- one fp16 window stage of nt tokens on tensor cores: S = K q
-      // (K rows by ldmatrix), the same online softmax, O += V^T p (V^T by
-      // ldmatrix.trans); rows past nt read row 0 and are masked out
-      auto window_tile = [&](unsigned char* wbuf, int nt, int tw0) {
-        unsigned char* Kw = wbuf;
-        unsigned char* Vw = wbuf + G::NBX * G::BOX_B;
-        // address of 16-byte chunk cc (channels 8 cc .. 8 cc + 7) of row tok:
-        // the swizzle XORs the chunk index with address bits 7.. of the row
-        auto chunk = [&](unsigned char* base, int tok, int cc) -> unsigned char* {
-          constexpr int CPR = G::RB / 16;  // chunks per box row
-          unsigned char* row = base + (cc / CPR) * G::BOX_B + tok * G::RB;
-          const uint32_t ra = smem_u32(row);
-          const int x = G::RB == 128 ? (int)((ra >> 7) & 7u) : (int)((ra >> 7) & 3u);
-          return row + (((cc % CPR) ^ x) << 4);
-        };
-        if (a.new_k != nullptr && a.new_slot >= tw0 && a.new_slot < tw0 + G::WT) {
-          // fused append: the copies brought the window before this call's
-          // token; put the token into its row here and into the cache for
-          // later calls (16 bytes per lane, K then V)
-          constexpr int NC = D * 2 / 16;  // 16-byte chunks per row
-          const int row = a.new_slot - tw0;
-          if (lane < 2 * NC) {
-            const int cc = lane % NC;
-            const bool isv = lane >= NC;
-            const uint4 x = reinterpret_cast<const uint4*>(
-                reinterpret_cast<const T*>(isv ? a.new_v : a.new_k) + u * D)[cc];
-            *reinterpret_cast<uint4*>(chunk(isv ? Vw : Kw, row, cc)) = x;
-            T* dst = reinterpret_cast<T*>(isv ? c.v_res : c.k_res) + (u * c.R + a.new_slot) * D;
-            reinterpret_cast<uint4*>(dst)[cc] = x;
-          }
-          __syncwarp();
-        }
-        float dq[NPB][2][4];
-#pragma unroll
-        for (int p = 0; p < NPB; ++p)
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dq[p][mt][e] = 0.f;
-#pragma unroll
-        for (int sl = 0; sl < KSL; ++sl) {
-          uint2 bq[NPB];
-#pragma unroll
-          for (int p = 0; p < NPB; ++p)
-            bq[p] = bcol ? *reinterpret_cast<const uint2*>(qB + (p * KSL + sl) * 64 + frag_word(lane, sl))
-                         : make_uint2(0u, 0u);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            const int tok = 16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1);
-            uint32_t af[4];
-            ldsm_x4(af, chunk(Kw, tok < nt ? tok : 0, 2 * sl + (lane >> 4)));
-#pragma unroll
-            for (int p = 0; p < NPB; ++p) mma16816(dq[p][mt], af[0], af[1], af[2], af[3], bq[p].x, bq[p].y);
-          }
-        }
-        float sc[NPB][4];
-#pragma unroll
-        for (int p = 0; p < NPB; ++p)
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const float v = dq[p][mt][2 * r] + dq[p][mt][2 * r + 1];
-              sc[p][2 * mt + r] = (16 * mt + 8 * r + g < nt) ? v : kNegInf;
-            }
-        float lm[NPB];
-        bool need = false;
-#pragma unroll
-        for (int p = 0; p < NPB; ++p) {
-          lm[p] = fmaxf(fmaxf(sc[p][0], sc[p][1]), fmaxf(sc[p][2], sc[p][3]));
-          need |= vh[p] && lm[p] > m_run[p];
-        }
-        if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-          for (int p = 0; p < NPB; ++p) {
-            float tm = lm[p];
-            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
-            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
-            tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
-            const float mn = fmaxf(m_run[p], tm);
-            const float al = exp2f(m_run[p] - mn);
-            m_run[p] = mn;
-            l_part[p] *= al;
-#pragma unroll
-            for (int m = 0; m < NM; ++m)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) acc[p][m][e] *= al;
-          }
-        }
-#pragma unroll
-        for (int p = 0; p < NPB; ++p) {
-          float ps = 0.f;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float pv = exp2f(sc[p][i] - m_run[p]);
-            ps += pv;
-            if (vh[p]) pbuf[(tq + 4 * p) * PST + 16 * (i >> 1) + 8 * (i & 1) + g] = pv;
-          }
-          l_part[p] += ps;
-        }
-        __syncwarp();
-        // p (hi, lo) into the value B fragments, tokens in natural order
-        {
-          const int slp = lane >> 4, kk = lane & 15;
-          const int tqk = (kk & 7) >> 1, kp = kk >> 3, hf = kk & 1;
-#pragma unroll
-          for (int h = 0; h < GQ; ++h) {
-            const float x = pbuf[h * PST + lane];
-            const __half hi = __float2half_rn(x);
-            const __half lo = __float2half_rn(x - __half2float(hi));
-            __half* blk = pBh + ((h >> 2) * NJ * NSL + slp) * 128 + 2 * kp + hf;
-            const int nh = 2 * (h & 3);
-            blk[2 * frag_word(4 * nh + tqk, slp)] = hi;
-            blk[2 * frag_word(4 * (nh + 1) + tqk, slp)] = lo;
-          }
-        }
-        __syncwarp();
-#pragma unroll
-        for (int sl = 0; sl < NSL; ++sl) {
-          uint2 bb[NPB];
-#pragma unroll
-          for (int p = 0; p < NPB; ++p)
-            bb[p] = bcol ? *reinterpret_cast<const uint2*>(pB + (p * NJ * NSL + sl) * 64 + frag_word(lane, sl))
-                         : make_uint2(0u, 0u);
-          const int tok = 16 * sl + (lane & 7) + 8 * (lane >> 4);
-          const int tr = tok < nt ? tok : 0;
-#pragma unroll
-          for (int m = 0; m < NM; ++m) {
-            uint32_t af[4];
-            ldsm_x4_t(af, chunk(Vw, tr, 2 * m + ((lane >> 3) & 1)));
-#pragma unroll
-            for (int p = 0; p < NPB; ++p) mma16816(acc[p][m], af[0], af[1], af[2], af[3], bb[p].x, bb[p].y);
-          }
-        }
-      };
-
-      // ---- this warp's quantized-tile state (m, l, acc + value zeros) -> mg slot
-      auto flush_code = [&]() {
-        float lt[NPB];
-#pragma unroll
-        for (int p = 0; p < NPB; ++p) {
-          float v = l_part[p];
-          v += __shfl_xor_sync(0xffffffffu, v, 4);
-          v += __shfl_xor_sync(0xffffffffu, v, 8);
-          v += __shfl_xor_sync(0xffffffffu, v, 16);
-          lt[p] = v;
-        }
-#pragma unroll
-        for (int h = 0; h < GQ; ++h)
-#pragma unroll
-          for (int j = 0; j < NJ; ++j) bv[h][j] = warp_sum(bv[h][j]);
-#pragma unroll
-        for (int p = 0; p < NPB; ++p) {
-          if (!vh[p]) continue;
-          const int h = tq + 4 * p;
-          if (g == 0) {
-            mg_m[warp * GQ + h] = m_run[p];
-            mg_l[warp * GQ + h] = lt[p];
-          }
-#pragma unroll
-          for (int m = 0; m < NM; ++m) {
-            const int j = m >> 1;
-            const int ch = 32 * j + 4 * g + 2 * (m & 1);
-            float bias = 0.f;
-#pragma unroll
-            for (int hh = 0; hh < GQ; ++hh)
-              if (hh == h) bias = bv[hh][j];
-            float* dst = mg_acc + (warp * GQ + h) * D + ch;
-            dst[0] = fmaf(acc[p][m][0] + acc[p][m][1], kValOut, bias);
-            dst[1] = fmaf(acc[p][m][2] + acc[p][m][3], kValOut, bias);
-          }
-        }
-      };
-
-      // ---- fp16 residual window on tensor cores: window tile k (WPS per
-      // stage) goes to warp k % kW, which first flushes its quantized-tile
-      // state and then keeps a separate softmax state for the window (plain q
-      // and p, scale 1)
-      bool wmode = false;
-      if constexpr (sizeof(T) == 2) {
-        if (window_owner) {
-          int k = 0;
-          for (int w0 = 0; w0 < a.r; w0 += G::WT * G::WPS, ++st) {
-            if (*(volatile int*)&flag[0]) break;
-            const int s = (int)(st % G::NSTAGE);
-            const bool ok = mbar_wait(&full[s], (uint32_t)((st / G::NSTAGE) & 1));
-            if (!__all_sync(0xffffffffu, ok) || *(volatile int*)&flag[0]) {
-              if (lane == 0) atomicExch(&flag[0], 1);
-              break;
-            }
-            for (int j = 0; j < G::WPS; ++j, ++k) {
-            const int tw0 = w0 + j * G::WT;
-            if (tw0 >= a.r) break;
-            if (k % kW == warp) {
-              if (!wmode) {
-                flush_code();
-                __syncwarp();
-                wmode = true;
-#pragma unroll
-                for (int p = 0; p < NPB; ++p) {
-                  m_run[p] = kNegInf;
-                  l_part[p] = 0.f;
-#pragma unroll
-                  for (int m = 0; m < NM; ++m)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[p][m][e] = 0.f;
-                }
-                // B fragments of plain q (hi, lo), channels in natural order:
-                // k-slice sl, k = channel - 16 sl; lane takes channel pairs
-#pragma unroll
-                for (int cp0 = 0; cp0 < D / 2; cp0 += 32) {
-                  const int cpr = cp0 + lane;  // channels 2 cpr, 2 cpr + 1
-                  if (cpr < D / 2) {
-                    const int sl = cpr >> 3, kk = 2 * (cpr & 7);
-                    const int tqk = (kk & 7) >> 1, kp = kk >> 3;
-#pragma unroll
-                    for (int h = 0; h < GQ; ++h) {
-                      const float2 x = *reinterpret_cast<const float2*>(qs + h * D + 2 * cpr);
-                      uint32_t hi, lo;
-                      split2(x.x, x.y, hi, lo);
-                      uint32_t* blk = qB + ((h >> 2) * KSL + sl) * 64 + kp;
-                      const int nh = 2 * (h & 3);
-                      blk[frag_word(4 * nh + tqk, sl)] = hi;
-                      blk[frag_word(4 * (nh + 1) + tqk, sl)] = lo;
-                    }
-                  }
-                }
-                __syncwarp();
-              }
-              window_tile(smem + s * G::STAGE_B + j * G::WTILE_B, min(G::WT, a.r - tw0), tw0);
-            }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-          }
-        }
-      }
-      const bool failed = *(volatile int*)&flag[0] != 0;
-      if (!wmode) {
-        flush_code();
-      } else {
-        // fold the window state into this warp's slot (quantized-tile state)
-        float lt[NPB], m1[NPB], l1[NPB];
-#pragma unroll
-        for (int p = 0; p < NPB; ++p) {
-          float v = l_part[p];
-          v += __shfl_xor_sync(0xffffffffu, v, 4);
-          v += __shfl_xor_sync(0xffffffffu, v, 8);
-          v += __shfl_xor_sync(0xffffffffu, v, 16);
-          lt[p] = v;
-          const int h = tq + 4 * p;
-          m1[p] = vh[p] ? mg_m[warp * GQ + h] : kNegInf;
-          l1[p] = vh[p] ? mg_l[warp * GQ + h] : 0.f;
-        }
-        __syncwarp();
-#pragma unroll
-        for (int p = 0; p < NPB; ++p) {
-          if (!vh[p]) continue;
-          const int h = tq + 4 * p;
-          const float mn = fmaxf(m1[p], m_run[p]);
-          const float s1 = m1[p] == kNegInf ? 0.f : exp2f(m1[p] - mn);
-          const float s2 = m_run[p] == kNegInf ? 0.f : exp2f(m_run[p] - mn);
-          float* dst = mg_acc + (warp * GQ + h) * D;
-#pragma unroll
-          for (int m = 0; m < NM; ++m) {
-            const int ch = 16 * m + g;
-            dst[ch] = fmaf(dst[ch], s1, (acc[p][m][0] + acc[p][m][1]) * s2);
-            dst[ch + 8] = fmaf(dst[ch + 8], s1, (acc[p][m][2] + acc[p][m][3]) * s2);
-          }
-          if (g == 0) {
-            mg_m[warp * GQ + h] = mn;
-            mg_l[warp * GQ + h] = fmaf(l1[p], s1, lt[p] * s2);
-          }
-        }
-      }
-      __syncwarp();
-      // ---- residual window (CTA that ends the unit): warp w takes window
-      // tiles w, w+4, ... on CUDA cores, folded into its mg slot
-      if (sizeof(T) == 4 && window_owner && !failed) {
-        consumers_sync<kW>();  // qs written by all consumer threads
-        const T* kr = reinterpret_cast<const T*>(c.k_res) + u * c.R * D;
-        const T* vr = reinterpret_cast<const T*>(c.v_res) + u * c.R * D;
-        const int d0 = lane * CPL;
-        float wm[GQ], wl[GQ], wacc[GQ][CPL];
-#pragma unroll
-        for (int h = 0; h < GQ; ++h) {
-          wm[h] = kNegInf;
-          wl[h] = 0.f;
-#pragma unroll
-          for (int k = 0; k < CPL; ++k) wacc[h][k] = 0.f;
-        }
-        const int nwt = (a.r + kTile - 1) / kTile;
-        constexpr int VEC = 16 / (int)sizeof(T);  // elements per 16-byte load
-        for (int wt = warp; wt < nwt; wt += kW) {
-          const int t_in = wt * kTile + lane;
-          const int nt = min(kTile, a.r - wt * kTile);
-          float lg[GQ];
-#pragma unroll
-          for (int h = 0; h < GQ; ++h) lg[h] = 0.f;
-          if (t_in < a.r) {
-            // lane = token: its key row, 16 bytes per load, 8 loads in flight
-            const uint4* row = reinterpret_cast<const uint4*>(kr + (long long)t_in * D);
-            constexpr int NV = D / VEC;
-            constexpr int CH = NV < 8 ? NV : 8;
-#pragma unroll
-            for (int v0 = 0; v0 < NV; v0 += CH) {
-              uint4 raw[CH];
-#pragma unroll
-              for (int v = 0; v < CH; ++v) raw[v] = row[v0 + v];
-#pragma unroll
-              for (int v = 0; v < CH; ++v) {
-                const T* e = reinterpret_cast<const T*>(&raw[v]);
-#pragma unroll
-                for (int x4 = 0; x4 < VEC; x4 += 4) {
-#pragma unroll
-                  for (int h = 0; h < GQ; ++h) {
-                    const float4 q4 = *reinterpret_cast<const float4*>(&qs[h * D + (v0 + v) * VEC + x4]);
-                    lg[h] = fmaf(q4.x, to_f32(e[x4]), lg[h]);
-                    lg[h] = fmaf(q4.y, to_f32(e[x4 + 1]), lg[h]);
-                    lg[h] = fmaf(q4.z, to_f32(e[x4 + 2]), lg[h]);
-                    lg[h] = fmaf(q4.w, to_f32(e[x4 + 3]), lg[h]);
-                  }
-                }
-              }
-            }
-          } else {
-#pragma unroll
-            for (int h = 0; h < GQ; ++h) lg[h] = kNegInf;
-          }
-          float pw[GQ];
-#pragma unroll
-          for (int h = 0; h < GQ; ++h) {
-            const float mt = warp_max(lg[h]);
-            const float mn = fmaxf(wm[h], mt);
-            const float al = exp2f(wm[h] - mn);
-            pw[h] = exp2f(lg[h] - mn);
-            wl[h] = fmaf(wl[h], al, pw[h]);
-#pragma unroll
-            for (int k = 0; k < CPL; ++k) wacc[h][k] *= al;
-            wm[h] = mn;
-          }
-          // lane = channels d0..d0+CPL-1; NX token rows in flight
-          constexpr int NX = GQ >= 4 ? 4 : 8;
-          for (int t8 = 0; t8 < nt; t8 += NX) {
-            float vf[NX][CPL];
-#pragma unroll
-            for (int x = 0; x < NX; ++x) {
-              const int t = t8 + x;
-              const T* row = vr + (long long)(wt * kTile + min(t, nt - 1)) * D + d0;
-              if (CPL * sizeof(T) == 16) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(row);
-                const T* e = reinterpret_cast<const T*>(&raw);
-#pragma unroll
-                for (int k = 0; k < CPL; ++k) vf[x][k] = to_f32(e[k]);
-              } else if (CPL * sizeof(T) == 8) {
-                const uint2 raw = *reinterpret_cast<const uint2*>(row);
-                const T* e = reinterpret_cast<const T*>(&raw);
-#pragma unroll
-                for (int k = 0; k < CPL; ++k) vf[x][k] = to_f32(e[k]);
-              } else {
-#pragma unroll
-                for (int k = 0; k < CPL; ++k) vf[x][k] = to_f32(row[k]);
-              }
-            }
-#pragma unroll
-            for (int x = 0; x < NX; ++x) {
-#pragma unroll
-              for (int h = 0; h < GQ; ++h) {
-                const float pt = __shfl_sync(0xffffffffu, pw[h], (t8 + x) & 31);
-                if (t8 + x < nt) {
-#pragma unroll
-                  for (int k = 0; k < CPL; ++k) wacc[h][k] = fmaf(pt, vf[x][k], wacc[h][k]);
-                }
-              }
-            }
-          }
-        }
-        // fold the window state into this warp's slot (same warp wrote it)
-#pragma unroll
-        for (int h = 0; h < GQ; ++h) {
-          const float lw = warp_sum(wl[h]);
-          const float m1 = mg_m[warp * GQ + h];
-          const float mn = fmaxf(m1, wm[h]);
-          const float s1 = m1 == kNegInf ? 0.f : exp2f(m1 - mn);
-          const float s2 = wm[h] == kNegInf ? 0.f : exp2f(wm[h] - mn);
-#pragma unroll
-          for (int k = 0; k < CPL; ++k) {
-            float* x = &mg_acc[(warp * GQ + h) * D + d0 + k];
-            *x = *x * s1 + wacc[h][k] * s2;
-          }
-          __syncwarp();
-          if (lane == 0) {
-            mg_l[warp * GQ + h] = mg_l[warp * GQ + h] * s1 + lw * s2;
-            mg_m[warp * GQ + h] = mn;
-          }
-          __syncwarp();
-        }
-      }
-      consumers_sync<kW>();
-
-      // ---- merge the warps, write this CTA's partial for unit u
-      for (int idx = tid; idx < GQ * D; idx += kW * 32) {
-        const int h = idx / D, d = idx % D;
-        float M = kNegInf;
-#pragma unroll
-        for (int w = 0; w < kW; ++w) M = fmaxf(M, mg_m[w * GQ + h]);
-        float num = 0.f, den = 0.f;
-        if (M != kNegInf) {
-#pragma unroll
-          for (int w = 0; w < kW; ++w) {
-            const float mw = mg_m[w * GQ + h];
-            if (mw == kNegInf) continue;
-            const float s2 = exp2f(mw - M);
-            num = fmaf(s2, mg_acc[(w * GQ + h) * D + d], num);
-            den = fmaf(s2, mg_l[w * GQ + h], den);
-          }
-        }
-        float* P = a.ws + ((u * a.max_seg + slot) * GQ + h) * (D + 2);
-        if (failed) {
-          M = 0.f;
-          den = kNaN;
-          num = kNaN;
-        }
-        if (d == 0) {
-          P[0] = M;
-          P[1] = den;
-        }
-        P[2 + d] = num;
-      }
-      // ---- arrival; the last segment of the unit merges all its partials
-      consumers_sync<kW>();
-      if (tid == 0) {
-        if (dev) {
-          flag[1] = arrive_unit_reset(a.ctr + u, n_seg);
-        } else {
-          flag[1] = arrive_unit(a.ctr + u, a.epoch, n_seg);
-        }
-      }
-      consumers_sync<kW>();
-      const int last = flag[1];
-      if (last != 0) {
-        T* out = reinterpret_cast<T*>(a.out);
-        for (int idx = tid; idx < GQ * D; idx += kW * 32) {
-          const int h = idx / D, d = idx % D;
-          const long long row = b * Hq + (long long)kv * GQ + h;
-          float res = kNaN;
-          if (last > 0)
-            res = merge_partials(a.ws + (u * a.max_seg * GQ + h) * (D + 2), (long long)GQ * (D + 2),
-                                 n_seg, d);
-          out[row * D + d] = from_f32<T>(res);
-        }
-      }
-      consumers_sync<kW>();  // mg buffers and flag[1] are reused by the next unit
-      if (failed) break;
-    }
-  }
-  __syncthreads();
-  if (dev && tid == 0 && arrive_unit_reset(a.ctr + a.units, gridDim.x) == 1) {
-    // the last CTA to finish advances the device counters
-    args.dev_state->n_q = a.n_q;
-    args.dev_state->r = a.r;
-  }
-}
-
-// Opt in to the kernel's dynamic shared memory and return how many of its
-// CTAs fit on one SM (both once per device).
-template <int D, int BITS, int GQ, typename T>
-cudaError_t tc_setup(int* ctas_per_sm) {
-  using G = Geo<D, BITS, GQ>;
-  static int occ[128] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 128 && occ[dev] > 0) {
-    *ctas_per_sm = occ[dev];
-    return cudaSuccess;
-  }
-  e = cudaFuncSetAttribute(decode_stream_tc<D, BITS, GQ, T>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_B);
-  if (e != cudaSuccess) return e;
-  int n = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_tc<D, BITS, GQ, T>,
-                                                    G::THREADS, G::SMEM_B);
-  if (e != cudaSuccess) return e;
-  if (n < 1) return cudaErrorInvalidConfiguration;
-  if (dev >= 0 && dev < 128) occ[dev] = n;
-  *ctas_per_sm = n;
-  return cudaSuccess;
-}
-
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
-// against the driver library), looked up once.
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-EncodeTiledFn encode_tiled() {
-  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<EncodeTiledFn>(f);
-  }();
-  return fn;
-}
-
-// Tensor map of one fp16 residual buffer viewed as [units * R][D]: boxes of
-// 32 rows x min(D, 64) columns, swizzled (128-byte rows: 128B, 64-byte: 64B).
-cudaError_t window_map(CUtensorMap* m, const void* base, long long rows, int D) {
-  const EncodeTiledFn fn = encode_tiled();
-  if (!fn) return cudaErrorNotSupported;
-  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)(D < 64 ? D : 64), (cuuint32_t)kTile};
-  const cuuint32_t es[2] = {1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
-                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        D < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-template <int D, int BITS, int GQ, typename T>
-cudaError_t tc_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
-                 int* ctas_per_sm) {
-  using G = Geo<D, BITS, GQ>;
-  if (ctas_per_sm) return tc_setup<D, BITS, GQ, T>(ctas_per_sm);
-  int occ = 0;
-  cudaError_t e = tc_setup<D, BITS, GQ, T>(&occ);
-  if (e != cudaSuccess) return e;
-  CUtensorMap tmK, tmV;
-  memset(&tmK, 0, sizeof(tmK));
-  memset(&tmV, 0, sizeof(tmV));
-  if (sizeof(T) == 2 && a.r > 0) {
-    const long long rows = (long long)a.units * a.c.R;
-    if (rows >= (1LL << 31)) return cudaErrorInvalidValue;  // 32-bit box coordinates
-    e = window_map(&tmK, a.c.k_res, rows, D);
-    if (e == cudaSuccess) e = window_map(&tmV, a.c.v_res, rows, D);
-    if (e != cudaSuccess) return e;
-  }
-  if (e0) cudaEventRecord(e0, s);
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((unsigned)a.n_cta);
-  cfg.blockDim = dim3(G::THREADS);
-  cfg.dynamicSmemBytes = G::SMEM_B;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, decode_stream_tc<D, BITS, GQ, T>, a, tmK, tmV);
-  if (err == cudaSuccess) err = cudaGetLastError();
-  if (e1) cudaEventRecord(e1, s);
-  return err;
-}
-
-template <int D, int BITS, typename T>
-cudaError_t tc_g(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1, int* occ) {
-  switch (a.gq) {
-    case 1: return tc_t<D, BITS, 1, T>(a, s, e0, e1, occ);
-    case 2: return tc_t<D, BITS, 2, T>(a, s, e0, e1, occ);
-    case 4: return tc_t<D, BITS, 4, T>(a, s, e0, e1, occ);
-    case 8: return tc_t<D, BITS, 8, T>(a, s, e0, e1, occ);
-  }
-  return cudaErrorInvalidValue;
-}
-
-template <int BITS, typename T>
-cudaError_t tc_d(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1, int* occ) {
-  switch (a.D) {
-    case 32: return tc_g<32, BITS, T>(a, s, e0, e1, occ);
-    case 64: return tc_g<64, BITS, T>(a, s, e0, e1, occ);
-    case 128: return tc_g<128, BITS, T>(a, s, e0, e1, occ);
-  }
-  return cudaErrorInvalidValue;
-}
-
 cudaError_t tc_dispatch(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
                         int* occ) {
-  if (a.bits == 2 && a.dtype == 0) return tc_d<2, __half>(a, s, e0, e1, occ);
-  if (a.bits == 2 && a.dtype == 1) return tc_d<2, float>(a, s, e0, e1, occ);
-  if (a.bits == 4 && a.dtype == 0) return tc_d<4, __half>(a, s, e0, e1, occ);
-  if (a.bits == 4 && a.dtype == 1) return tc_d<4, float>(a, s, e0, e1, occ);
+  if (a.meta == 1) return tc_dispatch_meta16(a, s, e0, e1, occ);
+  if (a.meta != 0) return cudaErrorInvalidValue;
+  if (a.bits == 2 && a.dtype == 0) return tc_d<2, __half, float>(a, s, e0, e1, occ);
+  if (a.bits == 2 && a.dtype == 1) return tc_d<2, float, float>(a, s, e0, e1, occ);
+  if (a.bits == 4 && a.dtype == 0) return tc_d<4, __half, float>(a, s, e0, e1, occ);
+  if (a.bits == 4 && a.dtype == 1) return tc_d<4, float, float>(a, s, e0, e1, occ);
   return cudaErrorInvalidValue;
 }
 

@@ -13,18 +13,20 @@ constexpr int kGv = 32;       // value group: channels per (token, group) scale
 constexpr int kTile = 32;     // tokens per quantize tile (= kG, a multiple of E)
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Device view of one cache; per-unit strides follow the ABI layout.
+// Device view of one cache; per-unit strides follow the ABI layout.  The
+// scales and zeros are binary32 (meta 0) or binary16 (meta 1) elements.
 struct CacheView {
   uint32_t* k_codes;
-  float* k_scale;
-  float* k_zero;
+  void* k_scale;
+  void* k_zero;
   uint32_t* v_codes;
-  float* v_scale;
-  float* v_zero;
+  void* v_scale;
+  void* v_zero;
   void* k_res;
   void* v_res;
   long long Tq;  // quantized-store capacity per unit, tokens
   int R;         // residual window
+  int meta;      // 0: binary32 scales and zeros, 1: binary16
 };
 
 template <int D, int BITS>
@@ -49,6 +51,46 @@ template <>
 __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
+
+// A scale or zero as stored: binary32 unchanged, or rounded to binary16 (to
+// nearest, ties to even; the format variant with binary16 metadata).
+template <typename M>
+__device__ __forceinline__ float round_meta(float x);
+template <>
+__device__ __forceinline__ float round_meta<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float round_meta<__half>(float x) {
+  return __half2float(__float2half_rn(x));
+}
+
+// N consecutive scales or zeros (N in {1, 2, 4}) from an address aligned to
+// N elements, widened to float.
+template <int N>
+__device__ __forceinline__ void load_meta(const float* p, float (&o)[N]) {
+  if constexpr (N == 4) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+  } else if constexpr (N == 2) {
+    const float2 v = *reinterpret_cast<const float2*>(p);
+    o[0] = v.x; o[1] = v.y;
+  } else {
+    o[0] = p[0];
+  }
+}
+template <int N>
+__device__ __forceinline__ void load_meta(const __half* p, float (&o)[N]) {
+  if constexpr (N == 4) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+    o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+  } else if constexpr (N == 2) {
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(p));
+    o[0] = a.x; o[1] = a.y;
+  } else {
+    o[0] = __half2float(p[0]);
+  }
+}
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -134,6 +176,7 @@ struct DecodeArgs {
   int D;
   int bits;
   int dtype;
+  int meta;        // element type of the scales and zeros (as CacheView::meta)
   long long n_q;
   int r;
   float qscale;    // softmax_scale * log2(e)
@@ -275,7 +318,11 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s, cudaEvent_t 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t s, cudaEvent_t ev0,
                              cudaEvent_t ev1);
 // Resident CTAs per SM of the tensor-core kernel instance that `a` selects
-// (uses a.D, a.bits, a.gq, a.dtype).
+// (uses a.D, a.bits, a.gq, a.dtype, a.meta).
 cudaError_t decode_tc_ctas_per_sm(const DecodeArgs& a, int* ctas_per_sm);
+// The tensor-core instances with binary16 scales and zeros (fp16 caches);
+// occ non-null: return the resident CTAs per SM instead of launching.
+cudaError_t tc_dispatch_meta16(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0,
+                               cudaEvent_t e1, int* occ);
 
 }  // namespace kivi

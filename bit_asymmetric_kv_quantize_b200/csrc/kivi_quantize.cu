@@ -15,6 +15,11 @@
 // sign of a zero minimum), and the scale and quotients use the IEEE
 // round-to-nearest intrinsics __fsub_rn / __fdiv_rn and __float2int_rn
 // (half to even).  No reciprocal, no contraction.
+//
+// Format variant with binary16 scales and zeros (M = __half, fp16 caches):
+// the binary32 scale and minimum are rounded to binary16 (nearest, ties to
+// even) and the codes are chosen against the rounded pair, so that the
+// stored scale and zero reproduce them as closely as the code grid allows.
 #include "kivi_internal.cuh"
 
 namespace kivi {
@@ -26,7 +31,7 @@ namespace {
 // blockDim.x == D.  Thread d reduces key channel d over the tile's tokens;
 // thread i reduces value group (token i / NJ, group i % NJ) over kGv channels.
 // Codes go through shared memory and are packed by all threads.
-template <int D, int BITS, typename T>
+template <int D, int BITS, typename T, typename M>
 __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit,
                                               const T* __restrict__ Ksrc,
                                               const T* __restrict__ Vsrc, long long t0,
@@ -47,15 +52,16 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
       if (x[t] < mn) mn = x[t];
       if (x[t] > mx) mx = x[t];
     }
-    const float s = __fdiv_rn(__fsub_rn(mx, mn), Lf);
+    const float s = round_meta<M>(__fdiv_rn(__fsub_rn(mx, mn), Lf));
+    const float z = round_meta<M>(mn);
     const long long g = t0 / kG;
-    c.k_scale[unit * Lt::k_meta_unit(c.Tq) + g * D + tid] = s;
-    c.k_zero[unit * Lt::k_meta_unit(c.Tq) + g * D + tid] = mn;
+    reinterpret_cast<M*>(c.k_scale)[unit * Lt::k_meta_unit(c.Tq) + g * D + tid] = from_f32<M>(s);
+    reinterpret_cast<M*>(c.k_zero)[unit * Lt::k_meta_unit(c.Tq) + g * D + tid] = from_f32<M>(z);
 #pragma unroll
     for (int t = 0; t < kTile; ++t) {
       int code = 0;
       if (s != 0.0f) {
-        code = __float2int_rn(__fdiv_rn(__fsub_rn(x[t], mn), s));
+        code = __float2int_rn(__fdiv_rn(__fsub_rn(x[t], z), s));
         code = min(max(code, 0), Lt::L);
       }
       ck[t * D + tid] = (uint8_t)code;
@@ -74,15 +80,16 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
       if (x[i] < mn) mn = x[i];
       if (x[i] > mx) mx = x[i];
     }
-    const float s = __fdiv_rn(__fsub_rn(mx, mn), Lf);
+    const float s = round_meta<M>(__fdiv_rn(__fsub_rn(mx, mn), Lf));
+    const float z = round_meta<M>(mn);
     const long long mo = unit * Lt::v_meta_unit(c.Tq) + (t0 + t) * NJ + j;
-    c.v_scale[mo] = s;
-    c.v_zero[mo] = mn;
+    reinterpret_cast<M*>(c.v_scale)[mo] = from_f32<M>(s);
+    reinterpret_cast<M*>(c.v_zero)[mo] = from_f32<M>(z);
 #pragma unroll
     for (int i = 0; i < kGv; ++i) {
       int code = 0;
       if (s != 0.0f) {
-        code = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], mn), s));
+        code = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], z), s));
         code = min(max(code, 0), Lt::L);
       }
       cv[t * D + j * kGv + i] = (uint8_t)code;
@@ -113,7 +120,7 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
 }
 
 // grid (n_q / kTile + 1, units); the last x-block copies the r window tokens.
-template <int D, int BITS, typename T>
+template <int D, int BITS, typename T, typename M>
 __global__ void __launch_bounds__(D) prefill_kernel(CacheView c, const T* __restrict__ K,
                                                     const T* __restrict__ V, long long T_len,
                                                     long long n_q, int r) {
@@ -124,8 +131,8 @@ __global__ void __launch_bounds__(D) prefill_kernel(CacheView c, const T* __rest
   const T* Ku = K + unit * T_len * D;
   const T* Vu = V + unit * T_len * D;
   if (tile < n_q / kTile) {
-    quantize_tile<D, BITS, T>(c, unit, Ku + tile * kTile * D, Vu + tile * kTile * D,
-                              tile * kTile, ck, cv);
+    quantize_tile<D, BITS, T, M>(c, unit, Ku + tile * kTile * D, Vu + tile * kTile * D,
+                                 tile * kTile, ck, cv);
   } else {
     T* kr = reinterpret_cast<T*>(c.k_res) + unit * c.R * D;
     T* vr = reinterpret_cast<T*>(c.v_res) + unit * c.R * D;
@@ -142,7 +149,7 @@ __global__ void __launch_bounds__(D) prefill_kernel(CacheView c, const T* __rest
 // `slot` (its own tile has been read by then).  Device mode (st != null):
 // n_q and r come from st -- flush when r == R, slot = flush ? 0 : r -- and a
 // full cache is left alone with st->status = 1.
-template <int D, int BITS, typename T>
+template <int D, int BITS, typename T, typename M>
 __global__ void __launch_bounds__(D) append_kernel(CacheView c, const T* __restrict__ k,
                                                    const T* __restrict__ v, long long n_q,
                                                    int slot, int flush, DevState* st) {
@@ -164,8 +171,8 @@ __global__ void __launch_bounds__(D) append_kernel(CacheView c, const T* __restr
   T* kr = reinterpret_cast<T*>(c.k_res) + unit * c.R * D;
   T* vr = reinterpret_cast<T*>(c.v_res) + unit * c.R * D;
   if (flush)
-    quantize_tile<D, BITS, T>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
-                              n_q + tile * kTile, ck, cv);
+    quantize_tile<D, BITS, T, M>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
+                                 n_q + tile * kTile, ck, cv);
   if (tile == 0) {
     kr[(long long)slot * D + threadIdx.x] = k[unit * D + threadIdx.x];
     vr[(long long)slot * D + threadIdx.x] = v[unit * D + threadIdx.x];
@@ -178,41 +185,41 @@ __global__ void set_state_kernel(DevState* st, long long n_q, int r) {
   st->status = 0;
 }
 
-template <int D, int BITS, typename T>
+template <int D, int BITS, typename T, typename M>
 cudaError_t prefill_t(const CacheView& c, int units, const void* K, const void* V,
                       long long T_len, long long n_q, int r, cudaStream_t s) {
   dim3 grid((unsigned)(n_q / kTile + 1), (unsigned)units);
-  prefill_kernel<D, BITS, T><<<grid, D, 0, s>>>(c, (const T*)K, (const T*)V, T_len, n_q, r);
+  prefill_kernel<D, BITS, T, M><<<grid, D, 0, s>>>(c, (const T*)K, (const T*)V, T_len, n_q, r);
   return cudaGetLastError();
 }
 
-template <int D, int BITS, typename T>
+template <int D, int BITS, typename T, typename M>
 cudaError_t append_t(const CacheView& c, int units, const void* k, const void* v, long long n_q,
                      int slot, bool flush, DevState* st, cudaStream_t s) {
   const dim3 grid((unsigned)((flush || st) ? c.R / kTile : 1), (unsigned)units);
-  append_kernel<D, BITS, T><<<grid, D, 0, s>>>(c, (const T*)k, (const T*)v, n_q, slot,
-                                               flush ? 1 : 0, st);
+  append_kernel<D, BITS, T, M><<<grid, D, 0, s>>>(c, (const T*)k, (const T*)v, n_q, slot,
+                                                  flush ? 1 : 0, st);
   return cudaGetLastError();
 }
 
-template <int BITS, typename T>
+template <int BITS, typename T, typename M>
 cudaError_t prefill_d(int D, const CacheView& c, int units, const void* K, const void* V,
                       long long T_len, long long n_q, int r, cudaStream_t s) {
   switch (D) {
-    case 32: return prefill_t<32, BITS, T>(c, units, K, V, T_len, n_q, r, s);
-    case 64: return prefill_t<64, BITS, T>(c, units, K, V, T_len, n_q, r, s);
-    case 128: return prefill_t<128, BITS, T>(c, units, K, V, T_len, n_q, r, s);
+    case 32: return prefill_t<32, BITS, T, M>(c, units, K, V, T_len, n_q, r, s);
+    case 64: return prefill_t<64, BITS, T, M>(c, units, K, V, T_len, n_q, r, s);
+    case 128: return prefill_t<128, BITS, T, M>(c, units, K, V, T_len, n_q, r, s);
   }
   return cudaErrorInvalidValue;
 }
 
-template <int BITS, typename T>
+template <int BITS, typename T, typename M>
 cudaError_t append_d(int D, const CacheView& c, int units, const void* k, const void* v,
                      long long n_q, int slot, bool flush, DevState* st, cudaStream_t s) {
   switch (D) {
-    case 32: return append_t<32, BITS, T>(c, units, k, v, n_q, slot, flush, st, s);
-    case 64: return append_t<64, BITS, T>(c, units, k, v, n_q, slot, flush, st, s);
-    case 128: return append_t<128, BITS, T>(c, units, k, v, n_q, slot, flush, st, s);
+    case 32: return append_t<32, BITS, T, M>(c, units, k, v, n_q, slot, flush, st, s);
+    case 64: return append_t<64, BITS, T, M>(c, units, k, v, n_q, slot, flush, st, s);
+    case 128: return append_t<128, BITS, T, M>(c, units, k, v, n_q, slot, flush, st, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -220,10 +227,17 @@ cudaError_t append_d(int D, const CacheView& c, int units, const void* k, const 
 cudaError_t append_any(const CacheView& c, int units, int D, int bits, int dtype, const void* k,
                        const void* v, long long n_q, int slot, bool flush, DevState* st,
                        cudaStream_t s) {
-  if (bits == 2 && dtype == 0) return append_d<2, __half>(D, c, units, k, v, n_q, slot, flush, st, s);
-  if (bits == 2 && dtype == 1) return append_d<2, float>(D, c, units, k, v, n_q, slot, flush, st, s);
-  if (bits == 4 && dtype == 0) return append_d<4, __half>(D, c, units, k, v, n_q, slot, flush, st, s);
-  if (bits == 4 && dtype == 1) return append_d<4, float>(D, c, units, k, v, n_q, slot, flush, st, s);
+  if (c.meta == 1) {  // binary16 scales and zeros: fp16 caches only
+    if (dtype != 0) return cudaErrorInvalidValue;
+    if (bits == 2) return append_d<2, __half, __half>(D, c, units, k, v, n_q, slot, flush, st, s);
+    if (bits == 4) return append_d<4, __half, __half>(D, c, units, k, v, n_q, slot, flush, st, s);
+    return cudaErrorInvalidValue;
+  }
+  if (c.meta != 0) return cudaErrorInvalidValue;
+  if (bits == 2 && dtype == 0) return append_d<2, __half, float>(D, c, units, k, v, n_q, slot, flush, st, s);
+  if (bits == 2 && dtype == 1) return append_d<2, float, float>(D, c, units, k, v, n_q, slot, flush, st, s);
+  if (bits == 4 && dtype == 0) return append_d<4, __half, float>(D, c, units, k, v, n_q, slot, flush, st, s);
+  if (bits == 4 && dtype == 1) return append_d<4, float, float>(D, c, units, k, v, n_q, slot, flush, st, s);
   return cudaErrorInvalidValue;
 }
 
@@ -232,10 +246,17 @@ cudaError_t append_any(const CacheView& c, int units, int D, int bits, int dtype
 cudaError_t launch_prefill(const CacheView& c, int units, int D, int bits, int dtype,
                            const void* K, const void* V, long long T, long long n_q, int r,
                            cudaStream_t s) {
-  if (bits == 2 && dtype == 0) return prefill_d<2, __half>(D, c, units, K, V, T, n_q, r, s);
-  if (bits == 2 && dtype == 1) return prefill_d<2, float>(D, c, units, K, V, T, n_q, r, s);
-  if (bits == 4 && dtype == 0) return prefill_d<4, __half>(D, c, units, K, V, T, n_q, r, s);
-  if (bits == 4 && dtype == 1) return prefill_d<4, float>(D, c, units, K, V, T, n_q, r, s);
+  if (c.meta == 1) {  // binary16 scales and zeros: fp16 caches only
+    if (dtype != 0) return cudaErrorInvalidValue;
+    if (bits == 2) return prefill_d<2, __half, __half>(D, c, units, K, V, T, n_q, r, s);
+    if (bits == 4) return prefill_d<4, __half, __half>(D, c, units, K, V, T, n_q, r, s);
+    return cudaErrorInvalidValue;
+  }
+  if (c.meta != 0) return cudaErrorInvalidValue;
+  if (bits == 2 && dtype == 0) return prefill_d<2, __half, float>(D, c, units, K, V, T, n_q, r, s);
+  if (bits == 2 && dtype == 1) return prefill_d<2, float, float>(D, c, units, K, V, T, n_q, r, s);
+  if (bits == 4 && dtype == 0) return prefill_d<4, __half, float>(D, c, units, K, V, T, n_q, r, s);
+  if (bits == 4 && dtype == 1) return prefill_d<4, float, float>(D, c, units, K, V, T, n_q, r, s);
   return cudaErrorInvalidValue;
 }
 

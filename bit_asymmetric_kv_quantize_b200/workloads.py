@@ -51,6 +51,7 @@ class Workload:
     Gv: int = 32
     R: int = 128
     dtype: str = "f16"  # "f16" or "f32"
+    meta: str = "f32"   # scale/zero storage: "f32", or "f16" (binary16 variant, f16 caches)
     steps: int = 0      # decode steps, each appending one token, after prefill
     outlier_channels: Optional[Tuple[int, ...]] = None  # fixed set, else 4 random per head
     n_outliers: int = 4
@@ -60,6 +61,10 @@ class Workload:
     @property
     def torch_dtype(self):
         return torch.float16 if self.dtype == "f16" else torch.float32
+
+    @property
+    def torch_meta(self):
+        return torch.float16 if self.meta == "f16" else torch.float32
 
     @property
     def gq(self) -> int:

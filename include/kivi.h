@@ -37,25 +37,27 @@
  *   k_codes  uint32 [B][Hkv][Tq][D/E]   word w of token t packs channels
  *                                        wE..wE+E-1; channel wE+i in bits
  *                                        [bits*i, bits*i+bits)
- *   k_scale  float  [B][Hkv][NG][D]     one scale and zero per key group
- *   k_zero   float  [B][Hkv][NG][D]     (G consecutive tokens) and channel
+ *   k_scale  meta   [B][Hkv][NG][D]     one scale and zero per key group
+ *   k_zero   meta   [B][Hkv][NG][D]     (G consecutive tokens) and channel
  *   v_codes  uint32 [B][Hkv][Tq/E][D]   word (tb, d) packs tokens
  *                                        tb*E..tb*E+E-1 of channel d;
  *                                        token tb*E+i in bits
  *                                        [bits*i, bits*i+bits)
- *   v_scale  float  [B][Hkv][Tq][NJ]    one scale and zero per token and
- *   v_zero   float  [B][Hkv][Tq][NJ]    value group (Gv consecutive channels)
+ *   v_scale  meta   [B][Hkv][Tq][NJ]    one scale and zero per token and
+ *   v_zero   meta   [B][Hkv][Tq][NJ]    value group (Gv consecutive channels)
  *   k_res    dtype  [B][Hkv][R][D]      residual window, input precision;
  *   v_res    dtype  [B][Hkv][R][D]      slots 0..r-1 hold the newest tokens
  * Each code packs along the axis its attention product contracts over
- * (channels for keys, tokens for values).
+ * (channels for keys, tokens for values).  "meta" is binary32 (float), or
+ * binary16 when dims.meta = KIVI_META_F16 (see kivi_meta).
  *
  * Quantizer (fixed binary32 formula; codes, scales and zeros are bit-exact
  * functions of the inputs): for a group x_0..x_{n-1},
  *   mn = min x_i, mx = max x_i (first occurrence kept among equal values),
  *   s = (mx - mn) / (2^bits - 1), z = mn  (each op rounded to nearest),
  *   c_i = clamp(round_half_even((x_i - mn) / s), 0, 2^bits - 1), or 0 if s == 0.
- * Dequantized value: c * s + z.
+ * Dequantized value: c * s + z.  (With binary16 metadata s and z are first
+ * rounded to binary16; see kivi_meta.)
  *
  * Residual window ("flush before write"): a non-empty cache holds
  * r in [1, R] residual tokens.  Prefill of T tokens leaves
@@ -92,9 +94,24 @@ typedef enum {
 
 typedef enum { KIVI_F16 = 0, KIVI_F32 = 1 } kivi_dtype;
 
+/* Element type of the scales and zeros.  KIVI_META_F16 is the format
+ * variant with binary16 metadata (fp16 caches only): the binary32 scale s
+ * and minimum mn of a group are rounded to nearest-even binary16, s16 and
+ * z16, and the codes are chosen against them:
+ *   c_i = clamp(round_half_even((x_i - z16) / s16), 0, 2^bits - 1), or 0 if
+ *   s16 == 0; dequantized value c * s16 + z16.
+ * It halves the metadata bytes; at 2 bits the binary32 scales and zeros are
+ * half of what the decode streams per quantized token, so binary16 cuts
+ * those bytes by a quarter.  (KIVI, study.space summary:
+ * each group keeps an asymmetric scale and offset; the pages fix no
+ * storage precision for them.) */
+typedef enum { KIVI_META_F32 = 0, KIVI_META_F16 = 1 } kivi_meta;
+
 /* Shape of one cache (one attention layer).  Supported: bits in {2, 4},
  * G = 32, Gv = 32, D in {32, 64, 128}, R a positive multiple of 32,
- * capacity a positive multiple of R, dtype KIVI_F16 or KIVI_F32. */
+ * capacity a positive multiple of R, dtype KIVI_F16 or KIVI_F32, meta
+ * KIVI_META_F32 or (with dtype KIVI_F16) KIVI_META_F16.  A zero-filled
+ * meta field selects binary32 metadata. */
 typedef struct {
   int B;              /* sequences (batch) */
   int Hkv;            /* key/value heads */
@@ -105,6 +122,7 @@ typedef struct {
   int R;              /* residual window length in tokens */
   long long capacity; /* max tokens per sequence, quantized + residual */
   int dtype;          /* kivi_dtype of K, V, q, out and the residual window */
+  int meta;           /* kivi_meta of k_scale, k_zero, v_scale, v_zero */
 } kivi_dims;
 
 enum {
@@ -125,11 +143,11 @@ enum {
 typedef struct {
   kivi_dims dims;
   uint32_t *k_codes;
-  float *k_scale;
-  float *k_zero;
+  void *k_scale; /* float, or uint16_t binary16 bits when dims.meta = KIVI_META_F16 */
+  void *k_zero;
   uint32_t *v_codes;
-  float *v_scale;
-  float *v_zero;
+  void *v_scale;
+  void *v_zero;
   void *k_res;
   void *v_res;
   long long n_q; /* tokens per sequence in the quantized store */

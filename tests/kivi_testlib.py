@@ -2,7 +2,8 @@
 
 Bars (stated once, used by every parity test):
   - codes, scales, zeros and the residual window: bit-exact (compared as
-    32-bit words / binary32 bit patterns, the window after exact upcast);
+    32-bit words / binary32 bit patterns; fp16 windows and binary16 scales
+    and zeros after exact upcast to binary32);
   - decode attention output: max |gpu - oracle| <= 2e-3 and
     mean |gpu - oracle| <= 1e-3, the oracle computed in binary64 from the
     dequantized cache.
@@ -22,12 +23,12 @@ MEAN_ABS = 1e-3
 
 def gpu_cache(w: W.Workload, capacity=None) -> kivi.KiviCache:
     return kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, capacity or w.capacity, R=w.R, G=w.G,
-                          Gv=w.Gv, dtype=w.torch_dtype, device="cuda")
+                          Gv=w.Gv, dtype=w.torch_dtype, device="cuda", meta=w.torch_meta)
 
 
 def oracle_cache(w: W.Workload, units=None, capacity=None) -> oracle.OracleCache:
     return oracle.OracleCache(w.B, w.Hkv, w.D, w.bits, w.G, w.Gv, w.R, capacity or w.capacity,
-                              units=units)
+                              units=units, meta_f16=w.meta == "f16")
 
 
 def oracle_prefill(oc: oracle.OracleCache, K: torch.Tensor, V: torch.Tensor):
@@ -56,7 +57,7 @@ def assert_state_equal(gc: kivi.KiviCache, oc: oracle.OracleCache, units=None):
     g = {}
     for name in kivi.BUFFER_NAMES:
         t = gc.view(name)[bs]
-        g[name] = t.float().cpu().numpy() if name.endswith("_res") else t.cpu().numpy()
+        g[name] = t.float().cpu().numpy() if t.is_floating_point() else t.cpu().numpy()
     bi = {b: i for i, b in enumerate(bs)}
     lim = {"k_codes": n_q, "k_scale": n_q // 32, "k_zero": n_q // 32, "v_codes": n_q // E, "v_scale": n_q, "v_zero": n_q,
            "k_res": r, "v_res": r}

@@ -32,10 +32,11 @@ def test_library_exports_every_declared_symbol():
 
 
 def _dims(**kw):
-    d = dict(B=2, Hkv=4, D=128, bits=2, G=32, Gv=32, R=128, capacity=4096, dtype=kivi.KIVI_F16)
+    d = dict(B=2, Hkv=4, D=128, bits=2, G=32, Gv=32, R=128, capacity=4096, dtype=kivi.KIVI_F16,
+             meta=kivi.KIVI_META_F32)
     d.update(kw)
     return KiviDims(d["B"], d["Hkv"], d["D"], d["bits"], d["G"], d["Gv"], d["R"], d["capacity"],
-                    d["dtype"])
+                    d["dtype"], d["meta"])
 
 
 def _sizes(dims):
@@ -61,7 +62,35 @@ def test_buffer_sizes_follow_the_layout(bits, D):
         assert sum(s[:6]) == u * Tq * D * 2 * 0.5
 
 
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("D", [32, 64, 128])
+def test_binary16_metadata_halves_the_scale_and_zero_buffers(bits, D):
+    B, H, R, cap = 3, 5, 64, 640
+    rc32, s32 = _sizes(_dims(B=B, Hkv=H, D=D, bits=bits, R=R, capacity=cap))
+    rc16, s16 = _sizes(_dims(B=B, Hkv=H, D=D, bits=bits, R=R, capacity=cap, meta=kivi.KIVI_META_F16))
+    assert rc32 == rc16 == 0
+    for i in (1, 2, 4, 5):  # k_scale, k_zero, v_scale, v_zero
+        assert 2 * s16[i] == s32[i]
+    for i in (0, 3, 6, 7):  # codes and window unchanged
+        assert s16[i] == s32[i]
+    # 2-bit codes + binary16 scale/zero per 32: 3/8 byte per key and per value element
+    if bits == 2:
+        u, Tq = B * H, cap - R
+        assert sum(s16[:6]) == u * Tq * D * 2 * 0.375
+
+
+def test_dims_struct_matches_the_header():
+    # the Python mirror of kivi_dims: nine ints/longs, then the metadata type
+    names = [f[0] for f in KiviDims._fields_]
+    assert names == ["B", "Hkv", "D", "bits", "G", "Gv", "R", "capacity", "dtype", "meta"]
+    text = open(HEADER).read()
+    body = text[text.index("typedef struct {\n  int B;"):text.index("} kivi_dims;")]
+    assert re.findall(r"\b(?:int|long long)\s+(\w+);", body) == names
+
+
 @pytest.mark.parametrize("kw,rc", [
+    (dict(meta=2), ERR_UNSUPPORTED), (dict(meta=-1), ERR_UNSUPPORTED),
+    (dict(meta=kivi.KIVI_META_F16, dtype=kivi.KIVI_F32), ERR_UNSUPPORTED),
     (dict(bits=3), ERR_UNSUPPORTED), (dict(bits=8), ERR_UNSUPPORTED),
     (dict(G=16), ERR_UNSUPPORTED), (dict(Gv=64), ERR_UNSUPPORTED),
     (dict(D=96), ERR_UNSUPPORTED), (dict(R=48), ERR_UNSUPPORTED),
