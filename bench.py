@@ -7,7 +7,9 @@ window is flushed into the 2-bit store every R tokens, as its own launch)
 and decode attention (fused dequant + q.K + online softmax + P.V over the
 packed codes and the window, then the cross-split merge), one kernel launch
 when no flush is due.  `--unfused` times kivi_append_token followed by
-kivi_decode_attention instead (two launches per step).  Workload: the Llama-2-7B-shaped layer
+kivi_decode_attention instead (two launches per step).  The ragged workload
+(per-sequence prompt lengths) times kivi_ragged_append_decode: the append
+(each sequence flushing on its own) and the decode, two launches per step.  Workload: the Llama-2-7B-shaped layer
 (B=8, 32 heads, D=128, context 4096, 2-bit, G=32, R=128) by default.
 
 L2 hygiene: `--layers` copies of the layer cache (default 32, the model's
@@ -143,9 +145,15 @@ def algorithmic_bytes(w: W.Workload, n_q: int, r: int) -> int:
     ms = 4, or 2 with binary16 scales and zeros)."""
     es = 2 if w.dtype == "f16" else 4
     ms = 2 if w.meta == "f16" else 4
-    per_unit = (2 * n_q * w.D * w.bits // 8 + (n_q // w.G) * w.D * 2 * ms
-                + n_q * (w.D // w.Gv) * 2 * ms + r * w.D * 2 * es)
-    return w.B * w.Hkv * per_unit + 2 * w.B * w.Hq * w.D * es
+
+    def per_unit(nq, rr):
+        return (2 * nq * w.D * w.bits // 8 + (nq // w.G) * w.D * 2 * ms
+                + nq * (w.D // w.Gv) * 2 * ms + rr * w.D * 2 * es)
+
+    io = 2 * w.B * w.Hq * w.D * es
+    if isinstance(n_q, (list, tuple)):  # ragged: one (n_q, r) per sequence
+        return w.Hkv * sum(per_unit(nq, rr) for nq, rr in zip(n_q, r)) + io
+    return w.B * w.Hkv * per_unit(n_q, r) + io
 
 
 # --------------------------------------------------------------- clocks (NVML)
@@ -222,16 +230,29 @@ def run_kivi(args, rank, world, local):
         dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=device)
 
     w = bench_workload(args)
+    ragged = w.len_min > 0
+    if ragged and (args.kernel != "default" or args.unfused):
+        raise SystemExit("ragged workloads run the fused tensor-core step only")
     n_layers = max(1, args.layers)
     e2e_steps = 0 if args.no_e2e else min(args.steps, 1024)
     per_layer = -(-(args.warmup + 2 * args.steps + e2e_steps) // n_layers) + 1
     capacity = -(-(w.T + per_layer) // w.R) * w.R
     Kp, Vp = W.prompt_kv(w, device=device)
-    caches = []
+    lens = W.seq_lengths(w)
+    lens_dev = lens.to(device)
+    caches, states = [], []
+    # ragged: every layer's per-sequence counters, followed on the host for
+    # the algorithmic bytes (the library keeps them on the device)
+    host_len = []
     for _ in range(n_layers):
         c = kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, capacity, R=w.R, G=w.G, Gv=w.Gv,
                            dtype=w.torch_dtype, device=device, meta=w.torch_meta)
-        c.prefill(Kp, Vp)
+        if ragged:
+            states.append(c.ragged_prefill(Kp, Vp, lens_dev))
+            rr = [int((x - 1) % w.R) + 1 for x in lens.tolist()]
+            host_len.append(([int(x) - y for x, y in zip(lens.tolist(), rr)], rr))
+        else:
+            c.prefill(Kp, Vp)
         caches.append(c)
     del Kp, Vp
     P = 16
@@ -242,7 +263,9 @@ def run_kivi(args, rank, world, local):
         vs.append(v)
         qs.append(W.query(w, i, device=device))
     out = torch.empty(w.B, w.Hq, w.D, dtype=w.torch_dtype, device=device)
-    ws = caches[0].workspace(w.Hq)
+    # (ragged: zero-filled, shared by every layer's calls; the arrival
+    # counters reset themselves)
+    ws = caches[0]._ragged_ws(w.Hq) if ragged else caches[0].workspace(w.Hq)
     for c in caches[1:]:
         c._ws = ws
     L = kivi.lib()
@@ -258,9 +281,22 @@ def run_kivi(args, rank, world, local):
     fused = args.kernel == "default" and not args.unfused
     n_launch = [0]
 
+    stp = [t.data_ptr() for t in states]
+
     def step_call(li, k_ptr, v_ptr, q_ptr):
         """One append + decode; returns the status and counts kernel launches."""
         c = caches[li]
+        if ragged:
+            n_launch[0] += 2  # the append (per-sequence flushes), then the decode
+            nq, rr = host_len[li]
+            for b in range(w.B):
+                if rr[b] == w.R:
+                    nq[b] += w.R
+                    rr[b] = 1
+                else:
+                    rr[b] += 1
+            return L.kivi_ragged_append_decode(cstructs[li], stp[li], k_ptr, v_ptr, q_ptr, w.Hq,
+                                               1.0, op, wp, wn, sh)
         n_launch[0] += 1 + (1 if (not fused or c.r == c.R) else 0)
         if fused:
             return L.kivi_append_decode(cstructs[li], k_ptr, v_ptr, q_ptr, w.Hq, 1.0, op, wp, wn, sh)
@@ -315,7 +351,11 @@ def run_kivi(args, rank, world, local):
         i = args.warmup + args.steps + j
         step(i, ev_handles[j])
         c = caches[i % n_layers]
-        fills.append((c.n_q, c.r))
+        if ragged:
+            nq, rr = host_len[i % n_layers]
+            fills.append((list(nq), list(rr)))
+        else:
+            fills.append((c.n_q, c.r))
     torch.cuda.synchronize(device)
     L.kivi_set_timing_events(None, None)
     barrier()
@@ -381,11 +421,14 @@ def run_kivi(args, rank, world, local):
                 "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                 "context": w.T, "bits": w.bits, "G": w.G, "Gv": w.Gv, "R": w.R,
                 "dtype_io": w.dtype, "meta": w.meta, "kernel": args.kernel,
-                "step": ("kivi_append_decode" if fused else "kivi_append_token+kivi_decode_attention"),
+                "step": ("kivi_ragged_append_decode" if ragged else
+                         "kivi_append_decode" if fused else "kivi_append_token+kivi_decode_attention"),
                 "parallelism": f"replicas{world}",
                 "layers_rotated": n_layers,
                 "l2": f"inputs larger than L2: {n_layers} layer caches visited round-robin",
                 "decode_splits": n_split,
+                **({"lengths": {"min": int(lens.min()), "max": int(lens.max()),
+                                "mean": float(lens.float().mean())}} if ragged else {}),
             },
             "roofline": {
                 "kernel": "decode_split", "bound": "hbm", "achieved": achieved, "peak": peak,
@@ -410,11 +453,18 @@ def run_kivi(args, rank, world, local):
 
 def oracle_sample(w: W.Workload, n_units: int, steps: int, threads: int):
     """Time `steps` decode steps (append + decode) of the CPU oracle on
-    `n_units` units of the workload; returns (seconds per step, units)."""
+    `n_units` units of the workload spread evenly over the batch (each at its
+    sequence's prompt length); returns (seconds per step, units, factor that
+    scales the sample's time to the whole batch by tokens held)."""
     import oracle
     from concurrent.futures import ThreadPoolExecutor
 
-    units = [(u // w.Hkv, u % w.Hkv) for u in range(min(n_units, w.B * w.Hkv))]
+    total = w.B * w.Hkv
+    n = max(1, min(n_units, total))
+    picks = sorted({(i * total) // n for i in range(n)})
+    units = [(u // w.Hkv, u % w.Hkv) for u in picks]
+    lens = [int(x) for x in W.seq_lengths(w)]
+    scale = (w.Hkv * sum(lens)) / sum(lens[b] for b, _ in units)
     cap = -(-(w.T + steps + 1) // w.R) * w.R
     oc = oracle.OracleCache(w.B, w.Hkv, w.D, w.bits, w.G, w.Gv, w.R, cap, units=units,
                             meta_f16=w.meta == "f16")
@@ -425,7 +475,8 @@ def oracle_sample(w: W.Workload, n_units: int, steps: int, threads: int):
     step_in = [tuple(t.float().numpy() for t in W.step_kv(w, i)) for i in range(min(steps, 4))]
     gq = w.gq
     with ThreadPoolExecutor(threads) as ex:
-        list(ex.map(lambda u: oc.prefill_unit(u[0], u[1], Kf, Vf), units))
+        list(ex.map(lambda u: oc.prefill_unit(u[0], u[1], Kf[:lens[u[0]]], Vf[:lens[u[0]]]),
+                    units))
 
         def one(u, i):
             b, h = u
@@ -437,7 +488,7 @@ def oracle_sample(w: W.Workload, n_units: int, steps: int, threads: int):
         for i in range(steps):
             list(ex.map(lambda u: one(u, i), units))
         dt = time.perf_counter() - t
-    return dt / steps, len(units)
+    return dt / steps, len(units), scale
 
 
 def cpu_threads():
@@ -450,16 +501,16 @@ def cpu_threads():
 def cpu_baseline(w: W.Workload, budget_s: float):
     threads = cpu_threads()
     # calibrate on one step of a few units, then size the sample to the budget
-    per_step, n = oracle_sample(w, threads, 1, threads)
+    per_step, n, _ = oracle_sample(w, threads, 1, threads)
     per_unit_cpu = per_step * threads / n
     n_units = min(w.B * w.Hkv, max(threads, int(threads * 4)))
     steps = max(1, int(budget_s * threads / (per_unit_cpu * n_units)))
-    per_step, n = oracle_sample(w, n_units, steps, threads)
-    full_step = per_step * (w.B * w.Hkv) / n
+    per_step, n, scale = oracle_sample(w, n_units, steps, threads)
+    full_step = per_step * scale
     return {"value": w.B / full_step, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{steps} steps x {n} of {w.B * w.Hkv} (batch, KV head) units, "
-                      f"append + decode, scaled to the full batch; single oracle threads "
-                      f"fanned out over units"}
+            "sample": f"{steps} steps x {n} of {w.B * w.Hkv} (batch, KV head) units spread "
+                      f"over the batch, append + decode, scaled to the full batch by tokens "
+                      f"held; single oracle threads fanned out over units"}
 
 
 def run_reference(args, rank, world):
@@ -468,12 +519,12 @@ def run_reference(args, rank, world):
     w = bench_workload(args)
     threads = cpu_threads()
     budget = 120.0  # seconds of wall time for warm-up + timed steps
-    per_step, n = oracle_sample(w, threads, 1, threads)
+    per_step, n, _ = oracle_sample(w, threads, 1, threads)
     n_units = max(1, min(w.B * w.Hkv,
                          int(budget / max(1, args.steps + args.warmup) / per_step * n)))
     oracle_sample(w, n_units, max(1, args.warmup), threads)
-    per_step, n = oracle_sample(w, n_units, args.steps, threads)
-    full_step = per_step * (w.B * w.Hkv) / n
+    per_step, n, scale = oracle_sample(w, n_units, args.steps, threads)
+    full_step = per_step * scale
     value = w.B / full_step
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",

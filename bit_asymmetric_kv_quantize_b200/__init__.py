@@ -34,7 +34,8 @@ EXPORTED = (
     "kivi_decode_workspace_bytes", "kivi_decode_attention", "kivi_decode_attention_simt",
     "kivi_set_timing_events", "kivi_decode_num_splits", "kivi_status_string",
     "kivi_decode_attention_noalloc", "kivi_append_decode", "kivi_dev_state_init",
-    "kivi_append_decode_dev",
+    "kivi_append_decode_dev", "kivi_ragged_prefill", "kivi_ragged_append", "kivi_ragged_decode",
+    "kivi_ragged_append_decode",
 )
 
 
@@ -90,6 +91,11 @@ def lib() -> ctypes.CDLL:
             L.kivi_dev_state_init.argtypes = [cp, vp, vp]
             L.kivi_append_decode_dev.argtypes = [cp, vp, vp, vp, vp, ci, ctypes.c_float, vp, vp, sz,
                                                  vp]
+            L.kivi_ragged_prefill.argtypes = [cp, vp, vp, vp, ll, vp, vp]
+            L.kivi_ragged_append.argtypes = [cp, vp, vp, vp, vp]
+            L.kivi_ragged_decode.argtypes = [cp, vp, vp, ci, ctypes.c_float, vp, vp, sz, vp]
+            L.kivi_ragged_append_decode.argtypes = [cp, vp, vp, vp, vp, ci, ctypes.c_float, vp, vp,
+                                                    sz, vp]
             L.kivi_set_timing_events.argtypes = [vp, vp]
             L.kivi_set_timing_events.restype = None
             L.kivi_decode_num_splits.argtypes = [cp, ci]
@@ -304,6 +310,79 @@ class KiviCache:
                                             float(softmax_scale), po, ws.data_ptr(), ws.numel(),
                                             self._stream()), "kivi_append_decode")
         return out
+
+
+    # -- ragged batches (per-sequence lengths on the device)
+    def ragged_prefill(self, K: torch.Tensor, V: torch.Tensor, lens: torch.Tensor) -> torch.Tensor:
+        """Prefill sequence b with its first lens[b] tokens of K[b], V[b]
+        ([B][Hkv][T_max][D], padded); returns the device state (B x 16 bytes)
+        that the other ragged calls take."""
+        T_max = K.shape[2]
+        shape = (self.B, self.Hkv, T_max, self.D)
+        pk, pv = self._arg(K, shape, "K"), self._arg(V, shape, "V")
+        if (lens.device != self.device or lens.dtype != torch.int64 or tuple(lens.shape) != (self.B,)
+                or not lens.is_contiguous()):
+            raise ValueError(f"lens: expected a contiguous int64 tensor of shape ({self.B},) on "
+                             f"{self.device}")
+        st = torch.zeros(16 * self.B, dtype=torch.uint8, device=self.device)
+        with torch.cuda.device(self.device):
+            _check(lib().kivi_ragged_prefill(ctypes.byref(self._c), st.data_ptr(), pk, pv, T_max,
+                                             lens.data_ptr(), self._stream()),
+                   "kivi_ragged_prefill")
+        return st
+
+    def _ragged_ws(self, Hq: int) -> torch.Tensor:
+        need = self.workspace_bytes(Hq)
+        if self._ws_dev is None or self._ws_dev.numel() < need:
+            self._ws_dev = torch.zeros(need, dtype=torch.uint8, device=self.device)
+        return self._ws_dev
+
+    def ragged_append(self, st: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
+        shape = (self.B, self.Hkv, self.D)
+        pk, pv = self._arg(k, shape, "k"), self._arg(v, shape, "v")
+        with torch.cuda.device(self.device):
+            _check(lib().kivi_ragged_append(ctypes.byref(self._c), st.data_ptr(), pk, pv,
+                                            self._stream()), "kivi_ragged_append")
+
+    def ragged_decode(self, st: torch.Tensor, q: torch.Tensor, softmax_scale: float,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        Hq = q.shape[1]
+        pq = self._arg(q, (self.B, Hq, self.D), "q")
+        if out is None:
+            out = torch.empty_like(q)
+        po = self._arg(out, (self.B, Hq, self.D), "out")
+        ws = self._ragged_ws(Hq)
+        with torch.cuda.device(self.device):
+            _check(lib().kivi_ragged_decode(ctypes.byref(self._c), st.data_ptr(), pq, Hq,
+                                            float(softmax_scale), po, ws.data_ptr(), ws.numel(),
+                                            self._stream()), "kivi_ragged_decode")
+        return out
+
+    def ragged_append_decode(self, st: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                             q: torch.Tensor, softmax_scale: float,
+                             out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        shape = (self.B, self.Hkv, self.D)
+        pk, pv = self._arg(k, shape, "k"), self._arg(v, shape, "v")
+        Hq = q.shape[1]
+        pq = self._arg(q, (self.B, Hq, self.D), "q")
+        if out is None:
+            out = torch.empty_like(q)
+        po = self._arg(out, (self.B, Hq, self.D), "out")
+        ws = self._ragged_ws(Hq)
+        with torch.cuda.device(self.device):
+            _check(lib().kivi_ragged_append_decode(ctypes.byref(self._c), st.data_ptr(), pk, pv, pq,
+                                                   Hq, float(softmax_scale), po, ws.data_ptr(),
+                                                   ws.numel(), self._stream()),
+                   "kivi_ragged_append_decode")
+        return out
+
+
+def ragged_lengths(st: torch.Tensor):
+    """(n_q, r, status) lists of a ragged device state (copies it to the host)."""
+    v = st.cpu().view(torch.int64).view(-1, 2)
+    n_q = v[:, 0].tolist()
+    rs = v[:, 1].contiguous().view(torch.int32).view(-1, 2)
+    return n_q, rs[:, 0].tolist(), rs[:, 1].tolist()
 
 
 def set_timing_events(start: Optional[torch.cuda.Event], stop: Optional[torch.cuda.Event]) -> None:

@@ -36,6 +36,11 @@ int check_dims(const kivi_dims* d) {
   return KIVI_OK;
 }
 
+// n_q of a cache filled by kivi_ragged_prefill: its counters live in the
+// caller's device state, and the host-counter calls refuse it.
+constexpr long long kRaggedMark = -1;
+bool is_ragged(const kivi_cache* c) { return c->n_q == kRaggedMark; }
+
 int check_cache(const kivi_cache* c) {
   if (!c) return KIVI_ERR_ARG;
   int rc = check_dims(&c->dims);
@@ -162,9 +167,11 @@ unsigned int next_epoch() {
 int decode_launch(const kivi_cache* c, const void* q, int Hq, float softmax_scale, void* out,
                   void* ws, int split_cap, int sms, void* stream, bool simt,
                   const void* new_k = nullptr, const void* new_v = nullptr, int new_slot = 0,
-                  void* dev_state = nullptr) {
+                  void* dev_state = nullptr, bool ragged = false, bool pending = false) {
   const int gq = Hq / c->dims.Hkv;
   DecodeArgs a;
+  a.ragged = ragged ? 1 : 0;
+  a.pending = pending ? 1 : 0;
   a.new_k = new_k;
   a.new_v = new_v;
   a.new_slot = new_slot;
@@ -221,7 +228,26 @@ int decode_checks(const kivi_cache* c, const void* q, int Hq, const void* out) {
   if (!q || !out || Hq <= 0 || Hq % c->dims.Hkv != 0) return KIVI_ERR_ARG;
   const int gq = Hq / c->dims.Hkv;
   if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KIVI_ERR_UNSUPPORTED;
-  if (c->n_q + c->r == 0) return KIVI_ERR_STATE;
+  if (is_ragged(c) || c->n_q + c->r == 0) return KIVI_ERR_STATE;
+  return KIVI_OK;
+}
+
+// Checks of the ragged calls: a cache filled by kivi_ragged_prefill, a
+// 16-byte aligned state, and (decode) a query shape and workspace.
+int ragged_checks(const kivi_cache* c, const void* state, const void* q, int Hq, const void* out,
+                  const void* workspace, size_t ws_bytes, int* sms) {
+  int rc = check_cache(c);
+  if (rc) return rc;
+  if (!state || ((uintptr_t)state & 15)) return KIVI_ERR_ARG;
+  if (!is_ragged(c)) return KIVI_ERR_STATE;
+  if (!q) return KIVI_OK;  // append only
+  if (!out || Hq <= 0 || Hq % c->dims.Hkv != 0) return KIVI_ERR_ARG;
+  const int gq = Hq / c->dims.Hkv;
+  if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KIVI_ERR_UNSUPPORTED;
+  *sms = device_sms();
+  if (*sms <= 0) return KIVI_ERR_CUDA;
+  if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(c->dims, Hq, *sms))
+    return KIVI_ERR_WORKSPACE;
   return KIVI_OK;
 }
 
@@ -334,6 +360,7 @@ int kivi_append_token(kivi_cache* cache, const void* k, const void* v, void* str
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!k || !v) return KIVI_ERR_ARG;
+  if (is_ragged(cache)) return KIVI_ERR_STATE;
   if (cache->n_q + cache->r + 1 > cache->dims.capacity) return KIVI_ERR_CAPACITY;
   const bool flush = cache->r == cache->dims.R;
   const int slot = flush ? 0 : cache->r;
@@ -365,6 +392,7 @@ int kivi_append_decode(kivi_cache* cache, const void* k, const void* v, const vo
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!k || !v) return KIVI_ERR_ARG;
+  if (is_ragged(cache)) return KIVI_ERR_STATE;
   if (cache->n_q + cache->r + 1 > cache->dims.capacity) return KIVI_ERR_CAPACITY;
   // the decode half sees the cache with the new token in it
   kivi_cache after = *cache;
@@ -398,6 +426,7 @@ int kivi_dev_state_init(const kivi_cache* cache, void* state, void* stream) {
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!state || ((uintptr_t)state & 15)) return KIVI_ERR_ARG;
+  if (is_ragged(cache)) return KIVI_ERR_STATE;
   return kivi::launch_set_state((kivi::DevState*)state, cache->n_q, cache->r,
                                 (cudaStream_t)stream) == cudaSuccess
              ? KIVI_OK
@@ -410,6 +439,7 @@ int kivi_append_decode_dev(const kivi_cache* cache, void* state, const void* k, 
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!state || ((uintptr_t)state & 15) || !k || !v) return KIVI_ERR_ARG;
+  if (is_ragged(cache)) return KIVI_ERR_STATE;
   kivi_cache after = *cache;  // any post-append state passes the decode checks
   after.r = 1;
   rc = decode_checks(&after, q, Hq, out);
@@ -424,6 +454,74 @@ int kivi_append_decode_dev(const kivi_cache* cache, void* state, const void* k, 
     return KIVI_ERR_CUDA;
   return decode_launch(&after, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms),
                        sms, stream, false, nullptr, nullptr, 0, state);
+}
+
+int kivi_ragged_prefill(kivi_cache* cache, void* state, const void* K, const void* V,
+                        long long T_max, const long long* lens, void* stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (!state || ((uintptr_t)state & 15) || !K || !V || !lens || T_max < 1) return KIVI_ERR_ARG;
+  if (cache->n_q != 0 || cache->r != 0) return KIVI_ERR_STATE;
+  if (T_max / kivi::kTile + 1 > (long long)INT_MAX) return KIVI_ERR_UNSUPPORTED;
+  cudaError_t err = kivi::launch_prefill_ragged(
+      view(cache), cache->dims.B * cache->dims.Hkv, cache->dims.Hkv, cache->dims.D,
+      cache->dims.bits, cache->dims.dtype, K, V, T_max, lens, (kivi::DevState*)state,
+      (cudaStream_t)stream);
+  if (err != cudaSuccess) return KIVI_ERR_CUDA;
+  cache->n_q = kRaggedMark;
+  cache->r = 0;
+  return KIVI_OK;
+}
+
+int kivi_ragged_append(const kivi_cache* cache, void* state, const void* k, const void* v,
+                       void* stream) {
+  int sms = 0;
+  int rc = ragged_checks(cache, state, nullptr, 0, nullptr, nullptr, 0, &sms);
+  if (rc) return rc;
+  if (!k || !v) return KIVI_ERR_ARG;
+  const int units = cache->dims.B * cache->dims.Hkv;
+  if (kivi::launch_append_ragged(view(cache), units, cache->dims.Hkv, cache->dims.D,
+                                 cache->dims.bits, cache->dims.dtype, k, v,
+                                 (const kivi::DevState*)state, (cudaStream_t)stream) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  return kivi::launch_advance_ragged((kivi::DevState*)state, cache->dims.B,
+                                     cache->dims.capacity - cache->dims.R, cache->dims.R,
+                                     (cudaStream_t)stream) == cudaSuccess
+             ? KIVI_OK
+             : KIVI_ERR_CUDA;
+}
+
+int kivi_ragged_decode(const kivi_cache* cache, const void* state, const void* q, int Hq,
+                       float softmax_scale, void* out, void* workspace, size_t ws_bytes,
+                       void* stream) {
+  int sms = 0;
+  int rc = ragged_checks(cache, state, q, Hq, out, workspace, ws_bytes, &sms);
+  if (rc) return rc;
+  kivi_cache any = *cache;  // host counters unused: every length is read on the device
+  any.n_q = 0;
+  any.r = 1;
+  return decode_launch(&any, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms),
+                       sms, stream, false, nullptr, nullptr, 0, const_cast<void*>(state), true,
+                       false);
+}
+
+int kivi_ragged_append_decode(const kivi_cache* cache, void* state, const void* k,
+                              const void* v, const void* q, int Hq, float softmax_scale,
+                              void* out, void* workspace, size_t ws_bytes, void* stream) {
+  if (!k || !v) return KIVI_ERR_ARG;
+  int sms = 0;
+  int rc = ragged_checks(cache, state, q, Hq, out, workspace, ws_bytes, &sms);
+  if (rc) return rc;
+  const int units = cache->dims.B * cache->dims.Hkv;
+  if (kivi::launch_append_ragged(view(cache), units, cache->dims.Hkv, cache->dims.D,
+                                 cache->dims.bits, cache->dims.dtype, k, v,
+                                 (const kivi::DevState*)state, (cudaStream_t)stream) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  kivi_cache any = *cache;
+  any.n_q = 0;
+  any.r = 1;
+  return decode_launch(&any, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms),
+                       sms, stream, false, nullptr, nullptr, 0, state, true, true);
 }
 
 int kivi_decode_attention_simt(const kivi_cache* cache, const void* q, int Hq,
@@ -459,6 +557,7 @@ void kivi_set_timing_events(void* start_event, void* stop_event) {
 
 int kivi_decode_num_splits(const kivi_cache* cache, int Hq) {
   if (check_cache(cache) != KIVI_OK || Hq <= 0 || Hq % cache->dims.Hkv != 0) return 0;
+  if (is_ragged(cache)) return 0;
   if (cache->n_q + cache->r == 0) return 0;
   const int sms = device_sms();
   if (sms <= 0) return 0;

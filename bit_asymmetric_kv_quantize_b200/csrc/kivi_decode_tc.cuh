@@ -241,13 +241,133 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 // free of bank conflicts while each lane still reads a contiguous 8 bytes.
 __device__ __forceinline__ int frag_word(int lane2, int sl) { return 2 * (lane2 ^ (4 * (sl & 3))); }
 
+// ---- the units of a CTA's work range ---------------------------------------
+// A cursor over consecutive units: unit u occupies work indices
+// [base, base + up), its quantized tiles first (n_qt of them), then its
+// window of r tokens and its end-of-unit weight.  Uniform batches: every unit
+// has the same n_qt and r and base = u * up.  Ragged batches: the lengths of
+// sequence b (units b * Hkv .. b * Hkv + Hkv - 1) come from its DevState.
+struct UnitCur {
+  long long u, base, n_qt, up;
+  int r;
+};
+
+__device__ __forceinline__ SeqLen ragged_len(const DecodeArgs& a, long long b) {
+  return seq_len(a.dev_state[b], a.pending != 0, a.c.Tq, a.c.R);
+}
+
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ long long warp_max_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Ragged plan (every lane of the calling warp, same result in every warp):
+// total work indices over all units and the stream-K range length W for P
+// CTAs (plan_ragged_w).
+__device__ __forceinline__ long long ragged_plan(const DecodeArgs& a, bool f16, long long P,
+                                                 long long* total, int* max_seg) {
+  const int lane = threadIdx.x & 31;
+  const long long B = a.units / a.Hkv;
+  long long tot = 0, mx = 0;
+  for (long long b0 = 0; b0 < B; b0 += 32) {
+    if (b0 + lane < B) {
+      const SeqLen L = ragged_len(a, b0 + lane);
+      tot += unit_work(L.n_q, L.r, f16) * a.Hkv;
+      mx = max(mx, L.n_q / kTile);
+    }
+  }
+  tot = warp_sum_ll(tot);
+  mx = warp_max_ll(mx);
+  *total = tot;
+  return plan_ragged_w(tot, mx, P, a.seg_cap, max_seg);
+}
+
+// The unit holding work index G0 (every lane of the calling warp).  Returns
+// u = units when G0 is past the last unit.
+template <bool RAG>
+__device__ __forceinline__ UnitCur cur_first(const DecodeArgs& a, bool f16, long long G0,
+                                             long long UP, long long n_qt) {
+  UnitCur c;
+  if constexpr (!RAG) {
+    c.u = G0 / UP;
+    c.base = c.u * UP;
+    c.n_qt = n_qt;
+    c.up = UP;
+    c.r = a.r;
+    return c;
+  } else {
+  const int lane = threadIdx.x & 31;
+  const long long B = a.units / a.Hkv;
+  long long pre = 0;  // work indices of the sequences before this chunk
+  for (long long b0 = 0; b0 < B; b0 += 32) {
+    const long long b = b0 + lane;
+    SeqLen L;
+    L.n_q = 0;
+    L.r = 0;
+    long long w = 0;
+    if (b < B) {
+      L = ragged_len(a, b);
+      w = unit_work(L.n_q, L.r, f16) * a.Hkv;
+    }
+    long long inc = w;  // inclusive scan over the chunk
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long t = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += t;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, b < B && G0 < pre + inc);
+    if (hit != 0u) {  // the first such lane's sequence holds G0
+      const int l = __ffs(hit) - 1;
+      const long long e = __shfl_sync(0xffffffffu, pre + inc - w, l);
+      const long long nq = __shfl_sync(0xffffffffu, L.n_q, l);
+      const int r = __shfl_sync(0xffffffffu, L.r, l);
+      c.up = unit_work(nq, r, f16);
+      const long long h = (G0 - e) / c.up;
+      c.u = (b0 + l) * a.Hkv + h;
+      c.base = e + h * c.up;
+      c.n_qt = nq / kTile;
+      c.r = r;
+      return c;
+    }
+    pre = __shfl_sync(0xffffffffu, pre + inc, 31);
+  }
+  c.u = a.units;
+  c.base = pre;
+  c.n_qt = 0;
+  c.up = 1;
+  c.r = 0;
+  return c;
+  }
+}
+
+// Step to the next unit (any thread; ragged: reads the next sequence's
+// lengths at a sequence boundary).
+template <bool RAG>
+__device__ __forceinline__ void cur_next(const DecodeArgs& a, bool f16, UnitCur& c) {
+  c.base += c.up;
+  ++c.u;
+  if (RAG && c.u < a.units && c.u % a.Hkv == 0) {
+    const SeqLen L = ragged_len(a, c.u / a.Hkv);
+    c.n_qt = L.n_q / kTile;
+    c.r = L.r;
+    c.up = unit_work(L.n_q, L.r, f16);
+  }
+}
+
 // Consumer-only barrier (the producer warp keeps streaming meanwhile).
 template <int NW>
 __device__ __forceinline__ void consumers_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
 }
 
-template <int D, int BITS, int GQ, typename T, typename MT>
+// RAG: ragged batch (per-sequence lengths in dev_state; device-counter mode)
+template <int D, int BITS, int GQ, typename T, typename MT, bool RAG>
 __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
                                   Geo<D, BITS, GQ, sizeof(MT)>::MIN_CTAS)
     decode_stream_tc(const DecodeArgs args, const __grid_constant__ CUtensorMap tmK,
@@ -280,7 +400,19 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
 
   DecodeArgs a = args;
   const bool dev = args.dev_state != nullptr;
-  if (dev) {
+  constexpr bool kF16 = sizeof(T) == 2;
+  long long total_ragged = 0;
+  if constexpr (RAG) {
+    // ragged batch: every warp plans from the sequences' own lengths
+    int ms = 0;
+    a.tiles_per_cta = ragged_plan(a, kF16, gridDim.x, &total_ragged, &ms);
+    a.max_seg = ms;
+    a.n_split = ms;
+    a.win_weight = 1;
+    a.n_q = 0;
+    a.r = 0;
+    a.new_k = nullptr;
+  } else if (dev) {
     // device counters as the preceding append launch found them; decode the
     // cache after that append (it flushed when r was R)
     const DevState st0 = *args.dev_state;
@@ -308,8 +440,8 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
   int* flag = reinterpret_cast<int*>(smem + G::O_FLAG);  // [0] abort, [1] merge flag
 
   const long long n_qt = a.n_q / kTile;
-  const long long UP = n_qt + a.win_weight;  // work indices per unit
-  const long long total = (long long)a.units * UP;
+  const long long UP = n_qt + a.win_weight;  // work indices per unit (uniform batches)
+  const long long total = RAG ? total_ragged : (long long)a.units * UP;
   const long long W = a.tiles_per_cta;
   const long long G0 = (long long)cta * W;
   const long long G1 = min(total, G0 + W);
@@ -350,12 +482,18 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
 
   if (warp == kW) {
     // ---------------- producer warp: one thread streams this CTA's stages
+    const UnitCur cu0 = cur_first<RAG>(a, kF16, G0, UP, n_qt);
     if (lane == 0 && G0 < G1) {
       long long st = 0;
-      for (long long u = G0 / UP; u <= (G1 - 1) / UP; ++u) {
-        const long long base = u * UP;
-        if (cta < base / W || cta > (base + n_qt) / W) continue;  // no work of u here
-        const long long t_end = min(G1 - base, n_qt);
+      for (UnitCur cu = cu0; cu.u < a.units && cu.base < G1; cur_next<RAG>(a, kF16, cu)) {
+        const long long u = cu.u, base = cu.base, n_qt_u = cu.n_qt;
+        const int r_u = cu.r;
+        if (cta < base / W || cta > (base + n_qt_u) / W) continue;  // no work of u here
+        if ((base + n_qt_u) / W - base / W + 1 > a.max_seg) {  // (cannot happen: plan bound)
+          atomicExch(&flag[0], 1);
+          break;
+        }
+        const long long t_end = min(G1 - base, n_qt_u);
         const uint32_t* kc_u = c.k_codes + u * Lt::k_codes_unit(c.Tq);
         const MT* ks_u = reinterpret_cast<const MT*>(c.k_scale) + u * Lt::k_meta_unit(c.Tq);
         const MT* kz_u = reinterpret_cast<const MT*>(c.k_zero) + u * Lt::k_meta_unit(c.Tq);
@@ -382,13 +520,13 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           bulk_copy(buf + G::O_VZ, vz_u + t0 * kTile * NJ, n * G::VM_B, &full[s]);
         }
         if (*(volatile int*)&flag[0]) break;
-        if (a.r > 0 && cta == (base + n_qt) / W) {
+        if (r_u > 0 && cta == (base + n_qt_u) / W) {
           const T* kr = reinterpret_cast<const T*>(c.k_res) + u * c.R * D;
           const T* vr = reinterpret_cast<const T*>(c.v_res) + u * c.R * D;
           if constexpr (sizeof(T) == 2) {
             // this CTA owns the unit's residual window: stream it through
             // the ring, WT tokens of K and of V per stage
-            for (int w0 = 0; w0 < a.r; w0 += G::WT * G::WPS, ++st) {
+            for (int w0 = 0; w0 < r_u; w0 += G::WT * G::WPS, ++st) {
               const int s = (int)(st % G::NSTAGE);
               if (st >= G::NSTAGE &&
                   !mbar_wait(&empty[s], (uint32_t)(((st / G::NSTAGE) - 1) & 1))) {
@@ -397,7 +535,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
               }
               if (*(volatile int*)&flag[0]) break;
               unsigned char* buf = smem + s * G::STAGE_B;
-              const int ntile = min(G::WPS, (a.r - w0 + G::WT - 1) / G::WT);
+              const int ntile = min(G::WPS, (r_u - w0 + G::WT - 1) / G::WT);
               asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
               mbar_expect_tx(&full[s], (uint32_t)(ntile * G::WTILE_B));
               for (int j = 0; j < ntile; ++j) {
@@ -413,7 +551,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           } else {
             // fp32 window (CUDA-core path): pull it into L2 while the
             // consumers work through the unit's last stages
-            const uint32_t wbytes = (uint32_t)((size_t)a.r * D * sizeof(T));
+            const uint32_t wbytes = (uint32_t)((size_t)r_u * D * sizeof(T));
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kr), "r"(wbytes) : "memory");
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vr), "r"(wbytes) : "memory");
           }
@@ -491,21 +629,24 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
     for (int p = 0; p < NPB; ++p) vh[p] = tq + 4 * p < GQ;
 
     long long st = 0;  // ring position, in step with the producer
-    for (long long u = G0 / UP; G0 < G1 && u <= (G1 - 1) / UP; ++u) {
-      const long long base = u * UP;
+    const UnitCur cu0 = cur_first<RAG>(a, kF16, G0, UP, n_qt);
+    for (UnitCur cu = cu0; G0 < G1 && cu.u < a.units && cu.base < G1; cur_next<RAG>(a, kF16, cu)) {
+      const long long u = cu.u, base = cu.base, n_qt_u = cu.n_qt;
+      const int r_u = cu.r;
       // CTAs f_cta..l_cta cover the unit's tiles and its window start index;
       // l_cta owns the window
       const long long f_cta = base / W;
-      const long long l_cta = (base + n_qt) / W;
+      const long long l_cta = (base + n_qt_u) / W;
       if (cta < f_cta || cta > l_cta) continue;
+      if (l_cta - f_cta + 1 > a.max_seg) break;  // (cannot happen: plan bound; producer aborts)
       const long long b = u / a.Hkv;
       const int kv = (int)(u % a.Hkv);
       const T* qg = reinterpret_cast<const T*>(a.q) + (b * Hq + (long long)kv * GQ) * D;
       const long long t_beg = max(G0 - base, 0ll);
-      const long long t_end = min(G1 - base, n_qt);
+      const long long t_end = min(G1 - base, n_qt_u);
       const int slot = (int)(cta - f_cta);
       const int n_seg = (int)(l_cta - f_cta + 1);
-      const bool window_owner = a.r > 0 && cta == l_cta;
+      const bool window_owner = r_u > 0 && cta == l_cta;
 
       // q (scaled by softmax_scale log2 e) at this lane's couple channels,
       // order c0, c0+PPW, c0+1, c0+PPW+1 (b0 low, b0 high, b1 low, b1 high)
@@ -985,7 +1126,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
       if constexpr (sizeof(T) == 2) {
         if (window_owner) {
           int k = 0;
-          for (int w0 = 0; w0 < a.r; w0 += G::WT * G::WPS, ++st) {
+          for (int w0 = 0; w0 < r_u; w0 += G::WT * G::WPS, ++st) {
             if (*(volatile int*)&flag[0]) break;
             const int s = (int)(st % G::NSTAGE);
             const bool ok = mbar_wait(&full[s], (uint32_t)((st / G::NSTAGE) & 1));
@@ -995,7 +1136,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
             }
             for (int j = 0; j < G::WPS; ++j, ++k) {
             const int tw0 = w0 + j * G::WT;
-            if (tw0 >= a.r) break;
+            if (tw0 >= r_u) break;
             if (k % kW == warp) {
               if (!wmode) {
                 flush_code();
@@ -1032,7 +1173,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
                 }
                 __syncwarp();
               }
-              window_tile(smem + s * G::STAGE_B + j * G::WTILE_B, min(G::WT, a.r - tw0), tw0);
+              window_tile(smem + s * G::STAGE_B + j * G::WTILE_B, min(G::WT, r_u - tw0), tw0);
             }
             }
             __syncwarp();
@@ -1094,15 +1235,15 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
 #pragma unroll
           for (int k = 0; k < CPL; ++k) wacc[h][k] = 0.f;
         }
-        const int nwt = (a.r + kTile - 1) / kTile;
+        const int nwt = (r_u + kTile - 1) / kTile;
         constexpr int VEC = 16 / (int)sizeof(T);  // elements per 16-byte load
         for (int wt = warp; wt < nwt; wt += kW) {
           const int t_in = wt * kTile + lane;
-          const int nt = min(kTile, a.r - wt * kTile);
+          const int nt = min(kTile, r_u - wt * kTile);
           float lg[GQ];
 #pragma unroll
           for (int h = 0; h < GQ; ++h) lg[h] = 0.f;
-          if (t_in < a.r) {
+          if (t_in < r_u) {
             // lane = token: its key row, 16 bytes per load, 8 loads in flight
             const uint4* row = reinterpret_cast<const uint4*>(kr + (long long)t_in * D);
             constexpr int NV = D / VEC;
@@ -1260,16 +1401,30 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
     }
   }
   __syncthreads();
-  if (dev && tid == 0 && arrive_unit_reset(a.ctr + a.units, gridDim.x) == 1) {
+  if (!RAG && dev && tid == 0 && arrive_unit_reset(a.ctr + a.units, gridDim.x) == 1) {
     // the last CTA to finish advances the device counters
     args.dev_state->n_q = a.n_q;
     args.dev_state->r = a.r;
+  }
+  if (RAG && a.pending) {
+    // the last CTA to finish advances every sequence that took its token
+    if (tid == 0) flag[1] = arrive_unit_reset(a.ctr + a.units, gridDim.x);
+    __syncthreads();
+    if (flag[1] == 1) {
+      for (long long b = tid; b < a.units / a.Hkv; b += G::THREADS) {
+        const SeqLen L = ragged_len(a, b);
+        if (L.ok) {
+          args.dev_state[b].n_q = L.n_q;
+          args.dev_state[b].r = L.r;
+        }
+      }
+    }
   }
 }
 
 // Opt in to the kernel's dynamic shared memory and return how many of its
 // CTAs fit on one SM (both once per device).
-template <int D, int BITS, int GQ, typename T, typename MT>
+template <int D, int BITS, int GQ, typename T, typename MT, bool RAG>
 cudaError_t tc_setup(int* ctas_per_sm) {
   using G = Geo<D, BITS, GQ, sizeof(MT)>;
   static int occ[128] = {};
@@ -1280,11 +1435,11 @@ cudaError_t tc_setup(int* ctas_per_sm) {
     *ctas_per_sm = occ[dev];
     return cudaSuccess;
   }
-  e = cudaFuncSetAttribute(decode_stream_tc<D, BITS, GQ, T, MT>,
+  e = cudaFuncSetAttribute(decode_stream_tc<D, BITS, GQ, T, MT, RAG>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_B);
   if (e != cudaSuccess) return e;
   int n = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_tc<D, BITS, GQ, T, MT>,
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_tc<D, BITS, GQ, T, MT, RAG>,
                                                     G::THREADS, G::SMEM_B);
   if (e != cudaSuccess) return e;
   if (n < 1) return cudaErrorInvalidConfiguration;
@@ -1327,13 +1482,13 @@ cudaError_t window_map(CUtensorMap* m, const void* base, long long rows, int D) 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D, int BITS, int GQ, typename T, typename MT>
+template <int D, int BITS, int GQ, typename T, typename MT, bool RAG>
 cudaError_t tc_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
                  int* ctas_per_sm) {
   using G = Geo<D, BITS, GQ, sizeof(MT)>;
-  if (ctas_per_sm) return tc_setup<D, BITS, GQ, T, MT>(ctas_per_sm);
+  if (ctas_per_sm) return tc_setup<D, BITS, GQ, T, MT, RAG>(ctas_per_sm);
   int occ = 0;
-  cudaError_t e = tc_setup<D, BITS, GQ, T, MT>(&occ);
+  cudaError_t e = tc_setup<D, BITS, GQ, T, MT, RAG>(&occ);
   if (e != cudaSuccess) return e;
   CUtensorMap tmK, tmV;
   memset(&tmK, 0, sizeof(tmK));
@@ -1357,29 +1512,30 @@ cudaError_t tc_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, decode_stream_tc<D, BITS, GQ, T, MT>, a, tmK, tmV);
+  cudaError_t err =
+      cudaLaunchKernelEx(&cfg, decode_stream_tc<D, BITS, GQ, T, MT, RAG>, a, tmK, tmV);
   if (err == cudaSuccess) err = cudaGetLastError();
   if (e1) cudaEventRecord(e1, s);
   return err;
 }
 
-template <int D, int BITS, typename T, typename MT>
+template <int D, int BITS, typename T, typename MT, bool RAG>
 cudaError_t tc_g(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1, int* occ) {
   switch (a.gq) {
-    case 1: return tc_t<D, BITS, 1, T, MT>(a, s, e0, e1, occ);
-    case 2: return tc_t<D, BITS, 2, T, MT>(a, s, e0, e1, occ);
-    case 4: return tc_t<D, BITS, 4, T, MT>(a, s, e0, e1, occ);
-    case 8: return tc_t<D, BITS, 8, T, MT>(a, s, e0, e1, occ);
+    case 1: return tc_t<D, BITS, 1, T, MT, RAG>(a, s, e0, e1, occ);
+    case 2: return tc_t<D, BITS, 2, T, MT, RAG>(a, s, e0, e1, occ);
+    case 4: return tc_t<D, BITS, 4, T, MT, RAG>(a, s, e0, e1, occ);
+    case 8: return tc_t<D, BITS, 8, T, MT, RAG>(a, s, e0, e1, occ);
   }
   return cudaErrorInvalidValue;
 }
 
-template <int BITS, typename T, typename MT>
+template <int BITS, typename T, typename MT, bool RAG>
 cudaError_t tc_d(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1, int* occ) {
   switch (a.D) {
-    case 32: return tc_g<32, BITS, T, MT>(a, s, e0, e1, occ);
-    case 64: return tc_g<64, BITS, T, MT>(a, s, e0, e1, occ);
-    case 128: return tc_g<128, BITS, T, MT>(a, s, e0, e1, occ);
+    case 32: return tc_g<32, BITS, T, MT, RAG>(a, s, e0, e1, occ);
+    case 64: return tc_g<64, BITS, T, MT, RAG>(a, s, e0, e1, occ);
+    case 128: return tc_g<128, BITS, T, MT, RAG>(a, s, e0, e1, occ);
   }
   return cudaErrorInvalidValue;
 }

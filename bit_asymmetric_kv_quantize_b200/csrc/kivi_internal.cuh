@@ -122,6 +122,19 @@ struct DevState {
 // the counters themselves are advanced by the decode that follows.
 cudaError_t launch_append_dev(const CacheView& c, int units, int D, int bits, int dtype,
                               const void* k, const void* v, const DevState* st, cudaStream_t s);
+// Ragged batch: st holds one DevState per sequence (Hkv units each); every
+// sequence appends one token and flushes on its own when its r == R.
+cudaError_t launch_append_ragged(const CacheView& c, int units, int Hkv, int D, int bits,
+                                 int dtype, const void* k, const void* v, const DevState* st,
+                                 cudaStream_t s);
+// After launch_append_ragged: advance the B sequences that took their token.
+cudaError_t launch_advance_ragged(DevState* st, long long B, long long Tq, int R, cudaStream_t s);
+// Ragged prefill: K, V [units][T_max][D]; sequence b has lens[b] tokens
+// (device); writes st[b] = {n_q, r, 0}, or {0, 0, 1} for a length outside
+// [1, capacity] (nothing else written for it).
+cudaError_t launch_prefill_ragged(const CacheView& c, int units, int Hkv, int D, int bits,
+                                  int dtype, const void* K, const void* V, long long T_max,
+                                  const long long* lens, DevState* st, cudaStream_t s);
 cudaError_t launch_set_state(DevState* st, long long n_q, int r, cudaStream_t s);
 
 // ---- stream-K plan of the tensor-core decode (host and device) -----------
@@ -163,6 +176,52 @@ __host__ __device__ inline StreamPlan plan_stream_core(long long units, long lon
   p.n_cta = (int)((total + W - 1) / W);
   p.max_seg = (W % UP == 0) ? 1 : (int)((n_qt + 1 + W - 1) / W + 1);
   return p;
+}
+
+// ---- ragged batches: per-sequence lengths in device memory ---------------
+// Lengths (n_q, r) of one sequence as a decode sees them: after the append
+// that the same step made when `pending`, else as stored.  ok = false for a
+// sequence the append refused (status set) or whose counters are not a valid
+// fill of the cache; such a sequence is decoded as empty (NaN output).
+struct SeqLen {
+  long long n_q;
+  int r;
+  bool ok;
+};
+__host__ __device__ inline SeqLen seq_len(const DevState& s, bool pending, long long Tq, int R) {
+  SeqLen o;
+  o.n_q = 0;
+  o.r = 0;
+  o.ok = false;
+  if (s.status != 0 || s.n_q < 0 || s.n_q > Tq || s.n_q % R != 0 || s.r < 0 || s.r > R) return o;
+  if (pending) {
+    if (s.n_q + s.r + 1 > Tq + R) return o;
+    const bool fl = s.r == R;
+    o.n_q = fl ? s.n_q + R : s.n_q;
+    o.r = fl ? 1 : s.r + 1;
+  } else {
+    o.n_q = s.n_q;
+    o.r = s.r;
+  }
+  o.ok = true;
+  return o;
+}
+// Work indices of one unit in the stream-K plan (as plan_stream_core).
+__host__ __device__ inline long long unit_work(long long n_q, int r, bool f16) {
+  const int wtw = f16 ? kWinWeightF16 : kWinWeight;
+  return n_q / kTile + (r > 0 ? wtw * (int)((r + kTile - 1) / kTile) : 1) + kMergeWeight;
+}
+// Stream-K range length W for a ragged batch: total work indices over P
+// CTAs, at least 12, and long enough that no unit of n_qt_max tiles spans
+// more than seg_cap CTA segments (seg_cap >= 2).  Returns W; *max_seg gets
+// the segment bound floor(n_qt_max / W) + 2.
+__host__ __device__ inline long long plan_ragged_w(long long total, long long n_qt_max, long long P,
+                                                   int seg_cap, int* max_seg) {
+  long long W = (total + P - 1) / P;
+  if (W < 12) W = 12;
+  if ((n_qt_max + 1 + W - 1) / W + 1 > seg_cap) W = (n_qt_max + 1 + seg_cap - 2) / (seg_cap - 1);
+  *max_seg = (int)((n_qt_max + 1 + W - 1) / W + 1);
+  return W;
 }
 
 struct DecodeArgs {
@@ -208,6 +267,12 @@ struct DecodeArgs {
   // (the workspace's counter block must start zeroed)
   DevState* dev_state;
   int seg_cap;
+  // ragged batch (tensor-core kernel, device-counter mode): dev_state holds
+  // one DevState per sequence (units / Hkv of them); the plan follows each
+  // sequence's own lengths, and when `pending` the state is the one before
+  // this step's append and the last CTA advances every valid sequence
+  int ragged;
+  int pending;
 };
 
 constexpr float kNaN = __builtin_nanf("");
@@ -320,9 +385,14 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t s, cudaEvent_t ev
 // Resident CTAs per SM of the tensor-core kernel instance that `a` selects
 // (uses a.D, a.bits, a.gq, a.dtype, a.meta).
 cudaError_t decode_tc_ctas_per_sm(const DecodeArgs& a, int* ctas_per_sm);
-// The tensor-core instances with binary16 scales and zeros (fp16 caches);
-// occ non-null: return the resident CTAs per SM instead of launching.
+// The tensor-core instances with binary16 scales and zeros (fp16 caches),
+// and the ragged-batch instances (binary32, binary16 metadata); occ
+// non-null: return the resident CTAs per SM instead of launching.
 cudaError_t tc_dispatch_meta16(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0,
                                cudaEvent_t e1, int* occ);
+cudaError_t tc_dispatch_ragged(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0,
+                               cudaEvent_t e1, int* occ);
+cudaError_t tc_dispatch_ragged_meta16(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0,
+                                      cudaEvent_t e1, int* occ);
 
 }  // namespace kivi

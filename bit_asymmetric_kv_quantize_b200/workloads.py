@@ -13,6 +13,9 @@ shaped attention layers; no datasets or weights are used):
   q ~ N(0, 1) / sqrt(D).
 Values are drawn in float32 from a seeded torch generator on the target
 device and cast to the workload dtype with round-to-nearest-even.
+Ragged batches (len_min > 0): sequence lengths uniform in [len_min, T]
+(seeded), with the first sequence at T and the second at len_min, standing
+in for a serving batch's mix of prompt lengths.
 """
 from __future__ import annotations
 
@@ -22,7 +25,7 @@ from typing import Optional, Tuple
 
 import torch
 
-_TAG = {"outlier": 1, "kv": 2, "q": 3, "step_kv": 4, "step_q": 5}
+_TAG = {"outlier": 1, "kv": 2, "q": 3, "step_kv": 4, "step_q": 5, "lens": 6}
 
 
 def _seed(base: int, tag: str, *idx: int) -> int:
@@ -53,6 +56,7 @@ class Workload:
     dtype: str = "f16"  # "f16" or "f32"
     meta: str = "f32"   # scale/zero storage: "f32", or "f16" (binary16 variant, f16 caches)
     steps: int = 0      # decode steps, each appending one token, after prefill
+    len_min: int = 0    # > 0: ragged batch, prompt lengths in [len_min, T] (T is the longest)
     outlier_channels: Optional[Tuple[int, ...]] = None  # fixed set, else 4 random per head
     n_outliers: int = 4
     outlier_scale: float = 20.0
@@ -80,7 +84,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five workloads: a tiny parity case and four attention-layer shapes.
+# The workloads: a tiny parity case, attention-layer shapes, and a ragged batch.
 TINY = Workload("tiny-b1h1d32-t256-f32", B=1, Hq=1, Hkv=1, D=32, T=256, bits=2, G=32, Gv=32,
                 R=32, dtype="f32", outlier_channels=(3, 17))
 LLAMA2_7B = Workload("llama2-7b-decode-b8h32d128-t4096", B=8, Hq=32, Hkv=32, D=128, T=4096, bits=2)
@@ -91,8 +95,25 @@ STREAMING = Workload("streaming-b4h32d128-prompt32768-512steps", B=4, Hq=32, Hkv
 LLAMA2_13B_2BIT = Workload("llama2-13b-b64h40d128-t8192-2bit", B=64, Hq=40, Hkv=40, D=128,
                            T=8192, bits=2)
 LLAMA2_13B_4BIT = LLAMA2_13B_2BIT.with_(name="llama2-13b-b64h40d128-t8192-4bit", bits=4)
+RAGGED = Workload("ragged-b32h32d128-len256-8192", B=32, Hq=32, Hkv=32, D=128, T=8192, bits=2,
+                  len_min=256)
 
-ALL = {w.name: w for w in (TINY, LLAMA2_7B, MISTRAL_7B, STREAMING, LLAMA2_13B_2BIT, LLAMA2_13B_4BIT)}
+ALL = {w.name: w for w in (TINY, LLAMA2_7B, MISTRAL_7B, STREAMING, LLAMA2_13B_2BIT, LLAMA2_13B_4BIT,
+                           RAGGED)}
+
+
+def seq_lengths(w: Workload) -> torch.Tensor:
+    """Prompt length of every sequence (int64 [B], CPU): T for a uniform
+    batch; for a ragged one uniform in [len_min, T], sequence 0 at T and
+    sequence 1 at len_min."""
+    if w.len_min <= 0:
+        return torch.full((w.B,), w.T, dtype=torch.int64)
+    lens = torch.randint(w.len_min, w.T + 1, (w.B,), generator=_gen(_seed(w.seed, "lens")),
+                         dtype=torch.int64)
+    lens[0] = w.T
+    if w.B > 1:
+        lens[1] = w.len_min
+    return lens
 
 
 def outlier_channels(w: Workload, h: int) -> torch.Tensor:

@@ -270,6 +270,57 @@ KIVI_API int kivi_append_decode_dev(const kivi_cache *cache, void *state, const 
                            void *out, void *workspace, size_t workspace_bytes,
                            void *stream);
 
+/* Ragged batches: every sequence b has its own length, held on the device
+ * in state[b] (B entries of the kivi_dev_state_init layout:
+ * { long long n_q; int r; int status; }, 16 bytes each, 16-byte aligned).
+ * A cache filled by kivi_ragged_prefill is used only with the kivi_ragged_*
+ * calls (the host-counter calls refuse it with KIVI_ERR_STATE); the buffer
+ * layout is unchanged, each sequence filling its own units from position 0.
+ * A sequence whose counters are not a valid fill, or that ran out of room
+ * (status 1), is left untouched by later appends and decodes to NaN.
+ * All decode work is planned on the device from the sequences' lengths
+ * (tensor-core kernel; the same stream-K split over every unit's own tiles
+ * and window), so launch arguments never depend on the lengths.
+ * The workspace (kivi_decode_workspace_bytes) must be zero-filled before
+ * first use and shared only with other kivi_ragged_* / *_dev calls.
+ * (KIVI, study.space summary: a grouped part plus a residual part per
+ * sequence; scholarfeed.org "KIVI" page: mixed-precision caches do not fit
+ * uniform paged blocks, hence per-sequence counters here.) */
+
+/* Prefill of a ragged batch into an empty cache.  K, V: device, dims.dtype,
+ * [B][Hkv][T_max][D] (padded; sequence b uses its first lens[b] tokens).
+ * lens: device, int64 [B].  Writes state[b] = { n_q_b, r_b, 0 } with
+ * r_b = ((lens[b]-1) mod R) + 1 and n_q_b = lens[b] - r_b, or { 0, 0, 1 }
+ * when lens[b] is outside [1, min(T_max, capacity)] (nothing else written).
+ * Errors: KIVI_ERR_ARG, KIVI_ERR_STATE (cache not empty), KIVI_ERR_CUDA. */
+KIVI_API int kivi_ragged_prefill(kivi_cache *cache, void *state, const void *K, const void *V,
+                        long long T_max, const long long *lens, void *stream);
+
+/* One token per sequence (k, v: device, dims.dtype, [B][Hkv][D]); a sequence
+ * whose window is full flushes it first, on its own.  Two launches (the
+ * append, then a B-thread counter update).  A sequence without room gets
+ * status 1 and takes nothing.
+ * Errors: KIVI_ERR_ARG, KIVI_ERR_STATE, KIVI_ERR_CUDA. */
+KIVI_API int kivi_ragged_append(const kivi_cache *cache, void *state, const void *k,
+                       const void *v, void *stream);
+
+/* Decode attention of a ragged batch over each sequence's own n_q + r
+ * tokens (arguments as kivi_decode_attention; state is only read).
+ * Errors: KIVI_ERR_ARG, KIVI_ERR_UNSUPPORTED, KIVI_ERR_STATE,
+ * KIVI_ERR_WORKSPACE, KIVI_ERR_CUDA. */
+KIVI_API int kivi_ragged_decode(const kivi_cache *cache, const void *state, const void *q,
+                       int Hq, float softmax_scale, void *out, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+/* kivi_ragged_append then kivi_ragged_decode as two launches: the decode
+ * reads the counters as the append found them, decodes the cache with the
+ * new tokens in it, and its last CTA advances every sequence's counters.
+ * Capturable in a CUDA graph.  Same errors as kivi_ragged_decode. */
+KIVI_API int kivi_ragged_append_decode(const kivi_cache *cache, void *state, const void *k,
+                              const void *v, const void *q, int Hq, float softmax_scale,
+                              void *out, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
 /* Optional timing hook: if start/stop are non-NULL cudaEvent_t handles,
  * later decode calls on this thread record `start` just before and `stop`
  * just after the launch of the dominant (split) decode kernel, on the

@@ -188,3 +188,51 @@ def test_oracle_and_library_share_no_source():
     for f in os.listdir(pkg):
         if f.endswith(".py"):
             assert "import oracle" not in open(os.path.join(pkg, f)).read(), f
+
+
+def test_ragged_calls_validate_on_the_host():
+    """Ragged calls check their arguments before any launch, and ragged and
+    host-counter calls refuse each other's caches."""
+    L = kivi.lib()
+    fake = ctypes.c_void_p(0x5000)
+    c = _fake_cache(R=128, capacity=512)
+    # a cache not filled by kivi_ragged_prefill
+    assert L.kivi_ragged_append(ctypes.byref(c), fake, fake, fake, None) == ERR_STATE
+    assert L.kivi_ragged_decode(ctypes.byref(c), fake, fake, 4, 1.0, fake, fake, 1 << 20,
+                                None) == ERR_STATE
+    # state null or not 16-byte aligned
+    assert L.kivi_ragged_append(ctypes.byref(c), None, fake, fake, None) == ERR_ARG
+    assert L.kivi_ragged_append(ctypes.byref(c), ctypes.c_void_p(0x5008), fake, fake,
+                                None) == ERR_ARG
+    assert L.kivi_ragged_prefill(ctypes.byref(c), None, fake, fake, 100, fake, None) == ERR_ARG
+    assert L.kivi_ragged_prefill(ctypes.byref(c), fake, fake, fake, 0, fake, None) == ERR_ARG
+    assert L.kivi_ragged_prefill(ctypes.byref(c), fake, fake, fake, 100, None, None) == ERR_ARG
+    # a ragged cache (its host counters carry the ragged mark)
+    c.n_q, c.r = -1, 0
+    assert L.kivi_append_token(ctypes.byref(c), fake, fake, None) == ERR_STATE
+    assert L.kivi_decode_attention(ctypes.byref(c), fake, 4, 1.0, fake, fake, 1 << 20,
+                                   None) == ERR_STATE
+    assert L.kivi_append_decode(ctypes.byref(c), fake, fake, fake, 4, 1.0, fake, fake, 1 << 20,
+                                None) == ERR_STATE
+    assert L.kivi_dev_state_init(ctypes.byref(c), fake, None) == ERR_STATE
+    assert L.kivi_quantize_prefill(ctypes.byref(c), fake, fake, 10, None) == ERR_STATE
+    assert L.kivi_ragged_prefill(ctypes.byref(c), fake, fake, fake, 100, fake, None) == ERR_STATE
+    assert L.kivi_decode_num_splits(ctypes.byref(c), 4) == 0
+    # shape errors of the ragged decode come before any device query
+    assert L.kivi_ragged_decode(ctypes.byref(c), fake, fake, 6, 1.0, fake, fake, 1 << 20,
+                                None) == ERR_ARG
+    assert L.kivi_ragged_decode(ctypes.byref(c), fake, fake, 12, 1.0, fake, fake, 1 << 20,
+                                None) == ERR_UNSUPPORTED
+    assert L.kivi_ragged_append_decode(ctypes.byref(c), fake, None, fake, fake, 4, 1.0, fake,
+                                       fake, 1 << 20, None) == ERR_ARG
+
+
+def test_ragged_lengths_of_a_state():
+    """The Python reader of a ragged state follows the 16-byte layout."""
+    st = torch.zeros(3 * 16, dtype=torch.uint8)
+    v = st.view(torch.int64).view(3, 2)
+    v[:, 0] = torch.tensor([0, 4096, 1 << 40])
+    w = st.view(torch.int32).view(3, 4)
+    w[:, 2] = torch.tensor([1, 128, 7], dtype=torch.int32)
+    w[:, 3] = torch.tensor([0, 0, 1], dtype=torch.int32)
+    assert kivi.ragged_lengths(st) == ([0, 4096, 1 << 40], [1, 128, 7], [0, 0, 1])
