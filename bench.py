@@ -66,6 +66,10 @@ def parse():
     p.add_argument("--unfused", action="store_true",
                    help="append and decode as two calls (kivi_append_token + decode)")
     p.add_argument("--cpu-budget-s", type=float, default=15.0)
+    p.add_argument("--paged", choices=["shuffled", "sequential"], default=None,
+                   help="ragged workloads: quantized store in pages of R tokens from a pool, "
+                        "through a block table whose pages are shuffled over the pool or "
+                        "consecutive per sequence")
     p.add_argument("--meta", choices=["f32", "f16"], default="f32",
                    help="scale/zero storage: binary32, or the binary16 format variant "
                         "(fp16 workloads)")
@@ -233,6 +237,8 @@ def run_kivi(args, rank, world, local):
     ragged = w.len_min > 0
     if ragged and (args.kernel != "default" or args.unfused):
         raise SystemExit("ragged workloads run the fused tensor-core step only")
+    if args.paged and not ragged:
+        raise SystemExit("--paged needs a ragged workload")
     n_layers = max(1, args.layers)
     e2e_steps = 0 if args.no_e2e else min(args.steps, 1024)
     per_layer = -(-(args.warmup + 2 * args.steps + e2e_steps) // n_layers) + 1
@@ -244,9 +250,21 @@ def run_kivi(args, rank, world, local):
     # ragged: every layer's per-sequence counters, followed on the host for
     # the algorithmic bytes (the library keeps them on the device)
     host_len = []
-    for _ in range(n_layers):
-        c = kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, capacity, R=w.R, G=w.G, Gv=w.Gv,
-                           dtype=w.torch_dtype, device=device, meta=w.torch_meta)
+    pps = capacity // w.R - 1
+    for li in range(n_layers):
+        if args.paged:
+            # every layer its own pool with a shuffled table (distinct pages)
+            g = torch.Generator().manual_seed(li)
+            n_pages = w.B * pps
+            order = (torch.randperm(n_pages, generator=g) if args.paged == "shuffled"
+                     else torch.arange(n_pages))
+            bt = order.to(torch.int32).view(w.B, pps)
+            c = kivi.PagedKiviCache(w.B, w.Hkv, w.D, w.bits, pps, n_pages, bt.to(device).contiguous(),
+                                    R=w.R, G=w.G, Gv=w.Gv, dtype=w.torch_dtype, device=device,
+                                    meta=w.torch_meta)
+        else:
+            c = kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, capacity, R=w.R, G=w.G, Gv=w.Gv,
+                               dtype=w.torch_dtype, device=device, meta=w.torch_meta)
         if ragged:
             states.append(c.ragged_prefill(Kp, Vp, lens_dev))
             rr = [int((x - 1) % w.R) + 1 for x in lens.tolist()]
@@ -421,6 +439,8 @@ def run_kivi(args, rank, world, local):
                 "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                 "context": w.T, "bits": w.bits, "G": w.G, "Gv": w.Gv, "R": w.R,
                 "dtype_io": w.dtype, "meta": w.meta, "kernel": args.kernel,
+                **({"paged": f"pages of {w.R} tokens, {args.paged} block table"}
+                   if args.paged else {}),
                 "step": ("kivi_ragged_append_decode" if ragged else
                          "kivi_append_decode" if fused else "kivi_append_token+kivi_decode_attention"),
                 "parallelism": f"replicas{world}",

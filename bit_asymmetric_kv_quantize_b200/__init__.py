@@ -35,7 +35,7 @@ EXPORTED = (
     "kivi_set_timing_events", "kivi_decode_num_splits", "kivi_status_string",
     "kivi_decode_attention_noalloc", "kivi_append_decode", "kivi_dev_state_init",
     "kivi_append_decode_dev", "kivi_ragged_prefill", "kivi_ragged_append", "kivi_ragged_decode",
-    "kivi_ragged_append_decode",
+    "kivi_ragged_append_decode", "kivi_paged_buffer_sizes", "kivi_paged_cache_init",
 )
 
 
@@ -58,7 +58,9 @@ class KiviCacheC(ctypes.Structure):
                 ("k_zero", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
                 ("v_scale", ctypes.c_void_p), ("v_zero", ctypes.c_void_p),
                 ("k_res", ctypes.c_void_p), ("v_res", ctypes.c_void_p),
-                ("n_q", ctypes.c_longlong), ("r", ctypes.c_int)]
+                ("n_q", ctypes.c_longlong), ("r", ctypes.c_int),
+                ("block_table", ctypes.c_void_p), ("pages_per_seq", ctypes.c_int),
+                ("num_pages", ctypes.c_longlong)]
 
 
 _lock = threading.Lock()
@@ -96,6 +98,8 @@ def lib() -> ctypes.CDLL:
             L.kivi_ragged_decode.argtypes = [cp, vp, vp, ci, ctypes.c_float, vp, vp, sz, vp]
             L.kivi_ragged_append_decode.argtypes = [cp, vp, vp, vp, vp, ci, ctypes.c_float, vp, vp,
                                                     sz, vp]
+            L.kivi_paged_buffer_sizes.argtypes = [dp, ll, ctypes.POINTER(sz * NUM_BUFFERS)]
+            L.kivi_paged_cache_init.argtypes = [cp, dp, ctypes.POINTER(vp * NUM_BUFFERS), vp, ci, ll]
             L.kivi_set_timing_events.argtypes = [vp, vp]
             L.kivi_set_timing_events.restype = None
             L.kivi_decode_num_splits.argtypes = [cp, ci]
@@ -375,6 +379,61 @@ class KiviCache:
                                                    ws.numel(), self._stream()),
                    "kivi_ragged_append_decode")
         return out
+
+
+class PagedKiviCache(KiviCache):
+    """A ragged-batch cache whose quantized store is pages of R tokens from a
+    pool of ``num_pages`` pages, addressed through ``block_table`` (int32
+    [B][pages_per_seq] on the device, owned by the caller; page l of sequence
+    b is pool page block_table[b, l]).  Filled with ``ragged_prefill`` and used
+    with the ragged calls only.  Pool views: ``view(name)`` gives the pool
+    arrays ([num_pages][Hkv]...) and the per-sequence windows."""
+
+    def __init__(self, B: int, Hkv: int, D: int, bits: int, pages_per_seq: int, num_pages: int,
+                 block_table: torch.Tensor, R: int = 128, G: int = 32, Gv: int = 32,
+                 dtype: torch.dtype = torch.float16, device="cuda",
+                 meta: torch.dtype = torch.float32):
+        self.device = torch.device(device)
+        if self.device.type != "cuda":
+            raise ValueError("PagedKiviCache lives in CUDA device memory")
+        if self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
+        if (block_table.device != self.device or block_table.dtype != torch.int32
+                or tuple(block_table.shape) != (B, pages_per_seq) or not block_table.is_contiguous()):
+            raise ValueError(f"block_table: expected a contiguous int32 tensor of shape "
+                             f"({B}, {pages_per_seq}) on {self.device}")
+        capacity = (pages_per_seq + 1) * R
+        self.dtype, self.meta = dtype, meta
+        self.block_table = block_table
+        self.pages_per_seq, self.num_pages = pages_per_seq, num_pages
+        self._dims = KiviDims(B, Hkv, D, bits, G, Gv, R, capacity, _dtype_code(dtype),
+                              _meta_code(meta))
+        out = (ctypes.c_size_t * NUM_BUFFERS)()
+        _check(lib().kivi_paged_buffer_sizes(ctypes.byref(self._dims), num_pages, ctypes.byref(out)),
+               "kivi_paged_buffer_sizes")
+        sizes = dict(zip(BUFFER_NAMES, list(out)))
+        self.buffers = {n: torch.empty(max(sizes[n], 16), dtype=torch.uint8, device=self.device)
+                        for n in BUFFER_NAMES}
+        ptrs = (ctypes.c_void_p * NUM_BUFFERS)(*[self.buffers[n].data_ptr() for n in BUFFER_NAMES])
+        self._c = KiviCacheC()
+        _check(lib().kivi_paged_cache_init(ctypes.byref(self._c), ctypes.byref(self._dims),
+                                           ctypes.byref(ptrs), block_table.data_ptr(),
+                                           pages_per_seq, num_pages), "kivi_paged_cache_init")
+        self._ws: Optional[torch.Tensor] = None
+        self._ws_dev: Optional[torch.Tensor] = None
+        E = 32 // bits
+        self.B, self.Hkv, self.D, self.bits, self.R, self.capacity = B, Hkv, D, bits, R, capacity
+        P = num_pages
+        self.shapes = {
+            "k_codes": ((P, Hkv, R, D // E), torch.int32),
+            "k_scale": ((P, Hkv, R // G, D), meta),
+            "k_zero": ((P, Hkv, R // G, D), meta),
+            "v_codes": ((P, Hkv, R // E, D), torch.int32),
+            "v_scale": ((P, Hkv, R, D // Gv), meta),
+            "v_zero": ((P, Hkv, R, D // Gv), meta),
+            "k_res": ((B, Hkv, R, D), dtype),
+            "v_res": ((B, Hkv, R, D), dtype),
+        }
 
 
 def ragged_lengths(st: torch.Tensor):

@@ -40,6 +40,8 @@ int check_dims(const kivi_dims* d) {
 // caller's device state, and the host-counter calls refuse it.
 constexpr long long kRaggedMark = -1;
 bool is_ragged(const kivi_cache* c) { return c->n_q == kRaggedMark; }
+// Caches whose counters live on the device: ragged-filled or paged ones.
+bool device_counted(const kivi_cache* c) { return is_ragged(c) || c->block_table != nullptr; }
 
 int check_cache(const kivi_cache* c) {
   if (!c) return KIVI_ERR_ARG;
@@ -69,6 +71,10 @@ CacheView view(const kivi_cache* c) {
   v.Tq = c->dims.capacity - c->dims.R;
   v.R = c->dims.R;
   v.meta = c->dims.meta;
+  v.bt = c->block_table;
+  v.pps = c->pages_per_seq;
+  v.n_pages = c->num_pages;
+  v.Hkv = c->dims.Hkv;
   return v;
 }
 
@@ -228,7 +234,7 @@ int decode_checks(const kivi_cache* c, const void* q, int Hq, const void* out) {
   if (!q || !out || Hq <= 0 || Hq % c->dims.Hkv != 0) return KIVI_ERR_ARG;
   const int gq = Hq / c->dims.Hkv;
   if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return KIVI_ERR_UNSUPPORTED;
-  if (is_ragged(c) || c->n_q + c->r == 0) return KIVI_ERR_STATE;
+  if (device_counted(c) || c->n_q + c->r == 0) return KIVI_ERR_STATE;
   return KIVI_OK;
 }
 
@@ -332,6 +338,48 @@ int kivi_cache_init(kivi_cache* cache, const kivi_dims* dims,
   cache->v_res = buffers[KIVI_BUF_V_RES];
   cache->n_q = 0;
   cache->r = 0;
+  cache->block_table = nullptr;
+  cache->pages_per_seq = 0;
+  cache->num_pages = 0;
+  return KIVI_OK;
+}
+
+int kivi_paged_buffer_sizes(const kivi_dims* dims, long long num_pages,
+                            size_t out_bytes[KIVI_NUM_BUFFERS]) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!out_bytes || num_pages < 1) return KIVI_ERR_ARG;
+  // a pool of num_pages pages of R tokens is the contiguous layout of
+  // num_pages * Hkv units of R tokens each; the windows are per sequence
+  kivi_dims pool = *dims;
+  pool.B = 1;
+  pool.capacity = 2 * (long long)dims->R;  // Tq = R
+  size_t one[KIVI_NUM_BUFFERS];
+  rc = kivi_buffer_sizes(&pool, one);
+  if (rc) return rc;
+  for (int i = 0; i < KIVI_BUF_K_RES; ++i) out_bytes[i] = one[i] * (size_t)num_pages;
+  const long long units = (long long)dims->B * dims->Hkv;
+  out_bytes[KIVI_BUF_K_RES] = (size_t)(units * dims->R * dims->D) * elem_bytes(dims->dtype);
+  out_bytes[KIVI_BUF_V_RES] = out_bytes[KIVI_BUF_K_RES];
+  return KIVI_OK;
+}
+
+int kivi_paged_cache_init(kivi_cache* cache, const kivi_dims* dims,
+                          void* const buffers[KIVI_NUM_BUFFERS], const int32_t* block_table,
+                          int pages_per_seq, long long num_pages) {
+  if (!cache || !buffers || !block_table || ((uintptr_t)block_table & 3)) return KIVI_ERR_ARG;
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (pages_per_seq < 1 || num_pages < 1 || num_pages > (long long)INT_MAX ||
+      dims->capacity != ((long long)pages_per_seq + 1) * dims->R)
+    return KIVI_ERR_ARG;
+  for (int i = 0; i < KIVI_NUM_BUFFERS; ++i)
+    if (!buffers[i] || ((uintptr_t)buffers[i] & 15) != 0) return KIVI_ERR_ARG;
+  rc = kivi_cache_init(cache, dims, buffers);
+  if (rc) return rc;
+  cache->block_table = block_table;
+  cache->pages_per_seq = pages_per_seq;
+  cache->num_pages = num_pages;
   return KIVI_OK;
 }
 
@@ -340,7 +388,7 @@ int kivi_quantize_prefill(kivi_cache* cache, const void* K, const void* V, long 
   int rc = check_cache(cache);
   if (rc) return rc;
   if (T < 0 || (T > 0 && (!K || !V))) return KIVI_ERR_ARG;
-  if (cache->n_q != 0 || cache->r != 0) return KIVI_ERR_STATE;
+  if (cache->n_q != 0 || cache->r != 0 || cache->block_table) return KIVI_ERR_STATE;
   if (T > cache->dims.capacity) return KIVI_ERR_CAPACITY;
   if (T == 0) return KIVI_OK;
   const int R = cache->dims.R;
@@ -360,7 +408,7 @@ int kivi_append_token(kivi_cache* cache, const void* k, const void* v, void* str
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!k || !v) return KIVI_ERR_ARG;
-  if (is_ragged(cache)) return KIVI_ERR_STATE;
+  if (device_counted(cache)) return KIVI_ERR_STATE;
   if (cache->n_q + cache->r + 1 > cache->dims.capacity) return KIVI_ERR_CAPACITY;
   const bool flush = cache->r == cache->dims.R;
   const int slot = flush ? 0 : cache->r;
@@ -392,7 +440,7 @@ int kivi_append_decode(kivi_cache* cache, const void* k, const void* v, const vo
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!k || !v) return KIVI_ERR_ARG;
-  if (is_ragged(cache)) return KIVI_ERR_STATE;
+  if (device_counted(cache)) return KIVI_ERR_STATE;
   if (cache->n_q + cache->r + 1 > cache->dims.capacity) return KIVI_ERR_CAPACITY;
   // the decode half sees the cache with the new token in it
   kivi_cache after = *cache;
@@ -426,7 +474,7 @@ int kivi_dev_state_init(const kivi_cache* cache, void* state, void* stream) {
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!state || ((uintptr_t)state & 15)) return KIVI_ERR_ARG;
-  if (is_ragged(cache)) return KIVI_ERR_STATE;
+  if (device_counted(cache)) return KIVI_ERR_STATE;
   return kivi::launch_set_state((kivi::DevState*)state, cache->n_q, cache->r,
                                 (cudaStream_t)stream) == cudaSuccess
              ? KIVI_OK
@@ -439,7 +487,7 @@ int kivi_append_decode_dev(const kivi_cache* cache, void* state, const void* k, 
   int rc = check_cache(cache);
   if (rc) return rc;
   if (!state || ((uintptr_t)state & 15) || !k || !v) return KIVI_ERR_ARG;
-  if (is_ragged(cache)) return KIVI_ERR_STATE;
+  if (device_counted(cache)) return KIVI_ERR_STATE;
   kivi_cache after = *cache;  // any post-append state passes the decode checks
   after.r = 1;
   rc = decode_checks(&after, q, Hq, out);
@@ -557,7 +605,7 @@ void kivi_set_timing_events(void* start_event, void* stop_event) {
 
 int kivi_decode_num_splits(const kivi_cache* cache, int Hq) {
   if (check_cache(cache) != KIVI_OK || Hq <= 0 || Hq % cache->dims.Hkv != 0) return 0;
-  if (is_ragged(cache)) return 0;
+  if (device_counted(cache)) return 0;
   if (cache->n_q + cache->r == 0) return 0;
   const int sms = device_sms();
   if (sms <= 0) return 0;

@@ -494,14 +494,25 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           break;
         }
         const long long t_end = min(G1 - base, n_qt_u);
-        const uint32_t* kc_u = c.k_codes + u * Lt::k_codes_unit(c.Tq);
-        const MT* ks_u = reinterpret_cast<const MT*>(c.k_scale) + u * Lt::k_meta_unit(c.Tq);
-        const MT* kz_u = reinterpret_cast<const MT*>(c.k_zero) + u * Lt::k_meta_unit(c.Tq);
-        const uint32_t* vc_u = c.v_codes + u * Lt::v_codes_unit(c.Tq);
-        const MT* vs_u = reinterpret_cast<const MT*>(c.v_scale) + u * Lt::v_meta_unit(c.Tq);
-        const MT* vz_u = reinterpret_cast<const MT*>(c.v_zero) + u * Lt::v_meta_unit(c.Tq);
+        const long long Ts = store_tokens(c);  // tokens per unit slot of the arrays
+        const uint32_t* kc_u = c.k_codes + u * Lt::k_codes_unit(Ts);
+        const MT* ks_u = reinterpret_cast<const MT*>(c.k_scale) + u * Lt::k_meta_unit(Ts);
+        const MT* kz_u = reinterpret_cast<const MT*>(c.k_zero) + u * Lt::k_meta_unit(Ts);
+        const uint32_t* vc_u = c.v_codes + u * Lt::v_codes_unit(Ts);
+        const MT* vs_u = reinterpret_cast<const MT*>(c.v_scale) + u * Lt::v_meta_unit(Ts);
+        const MT* vz_u = reinterpret_cast<const MT*>(c.v_zero) + u * Lt::v_meta_unit(Ts);
+        // paged store: this unit's row of the block table and its head
+        const int* pg_row = nullptr;
+        int pg_head = 0;
+        if constexpr (RAG) {
+          if (c.bt != nullptr) {
+            pg_row = c.bt + (u / c.Hkv) * c.pps;
+            pg_head = (int)(u % c.Hkv);
+          }
+        }
         for (long long t0 = max(G0 - base, 0ll); t0 < t_end; t0 += kStage, ++st) {
           const int s = (int)(st % G::NSTAGE);
+          const int n = (int)min((long long)kStage, t_end - t0);
           if (st >= G::NSTAGE &&
               !mbar_wait(&empty[s], (uint32_t)(((st / G::NSTAGE) - 1) & 1))) {
             atomicExch(&flag[0], 1);
@@ -509,15 +520,49 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           }
           if (*(volatile int*)&flag[0]) break;
           unsigned char* buf = smem + s * G::STAGE_B;
-          const int n = (int)min((long long)kStage, t_end - t0);
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           mbar_expect_tx(&full[s], (uint32_t)(n * G::TILE_B));
-          bulk_copy(buf + G::O_KC, kc_u + t0 * kTile * WK, n * G::KC_B, &full[s]);
-          bulk_copy(buf + G::O_KS, ks_u + t0 * D, n * G::KM_B, &full[s]);
-          bulk_copy(buf + G::O_KZ, kz_u + t0 * D, n * G::KM_B, &full[s]);
-          bulk_copy(buf + G::O_VC, vc_u + t0 * (kTile / E) * D, n * G::VC_B, &full[s]);
-          bulk_copy(buf + G::O_VS, vs_u + t0 * kTile * NJ, n * G::VM_B, &full[s]);
-          bulk_copy(buf + G::O_VZ, vz_u + t0 * kTile * NJ, n * G::VM_B, &full[s]);
+          if (!RAG || c.bt == nullptr) {
+            bulk_copy(buf + G::O_KC, kc_u + t0 * kTile * WK, n * G::KC_B, &full[s]);
+            bulk_copy(buf + G::O_KS, ks_u + t0 * D, n * G::KM_B, &full[s]);
+            bulk_copy(buf + G::O_KZ, kz_u + t0 * D, n * G::KM_B, &full[s]);
+            bulk_copy(buf + G::O_VC, vc_u + t0 * (kTile / E) * D, n * G::VC_B, &full[s]);
+            bulk_copy(buf + G::O_VS, vs_u + t0 * kTile * NJ, n * G::VM_B, &full[s]);
+            bulk_copy(buf + G::O_VZ, vz_u + t0 * kTile * NJ, n * G::VM_B, &full[s]);
+          } else {
+            // paged store: one run of copies per page the stage touches (the
+            // single producer thread is on the critical path: one 32-bit
+            // division per stage, pages stepped from there)
+            const int tpp = c.R / kTile;  // tiles per page
+            int lp = (int)t0 / tpp;
+            int stl = (int)t0 - lp * tpp;
+            for (int o = 0; o < n;) {
+              const int pg = lp < c.pps ? pg_row[lp] : -1;
+              if (pg < 0 || pg >= c.n_pages) {  // page outside the table or pool
+                atomicExch(&flag[0], 1);
+                break;
+              }
+              const long long su = (long long)pg * c.Hkv + pg_head;
+              const int run = min(n - o, tpp - stl);
+              const uint32_t* kc = c.k_codes + su * Lt::k_codes_unit(Ts);
+              const MT* ks = reinterpret_cast<const MT*>(c.k_scale) + su * Lt::k_meta_unit(Ts);
+              const MT* kz = reinterpret_cast<const MT*>(c.k_zero) + su * Lt::k_meta_unit(Ts);
+              const uint32_t* vc = c.v_codes + su * Lt::v_codes_unit(Ts);
+              const MT* vs = reinterpret_cast<const MT*>(c.v_scale) + su * Lt::v_meta_unit(Ts);
+              const MT* vz = reinterpret_cast<const MT*>(c.v_zero) + su * Lt::v_meta_unit(Ts);
+              bulk_copy(buf + G::O_KC + o * G::KC_B, kc + stl * kTile * WK, run * G::KC_B, &full[s]);
+              bulk_copy(buf + G::O_KS + o * G::KM_B, ks + stl * D, run * G::KM_B, &full[s]);
+              bulk_copy(buf + G::O_KZ + o * G::KM_B, kz + stl * D, run * G::KM_B, &full[s]);
+              bulk_copy(buf + G::O_VC + o * G::VC_B, vc + stl * (kTile / E) * D, run * G::VC_B,
+                        &full[s]);
+              bulk_copy(buf + G::O_VS + o * G::VM_B, vs + stl * kTile * NJ, run * G::VM_B, &full[s]);
+              bulk_copy(buf + G::O_VZ + o * G::VM_B, vz + stl * kTile * NJ, run * G::VM_B, &full[s]);
+              o += run;
+              ++lp;
+              stl = 0;
+            }
+            if (*(volatile int*)&flag[0]) break;
+          }
         }
         if (*(volatile int*)&flag[0]) break;
         if (r_u > 0 && cta == (base + n_qt_u) / W) {

@@ -27,7 +27,41 @@ struct CacheView {
   long long Tq;  // quantized-store capacity per unit, tokens
   int R;         // residual window
   int meta;      // 0: binary32 scales and zeros, 1: binary16
+  // paged store (bt != null): the quantized store of sequence b is pages of
+  // R tokens, page l at pool slot bt[b * pps + l]; the arrays hold n_pages
+  // slots of Hkv units of R tokens (contiguous stores: bt null, a unit's
+  // arrays span Tq tokens)
+  const int* bt;
+  int pps;
+  long long n_pages;
+  int Hkv;
 };
+
+// Tokens per unit slot of the store arrays (the per-unit stride).
+__host__ __device__ inline long long store_tokens(const CacheView& c) {
+  return c.bt ? (long long)c.R : c.Tq;
+}
+// Slot of 32-token tile t of unit u in the store arrays: the array unit su
+// and the tile st within it.  Paged: the sequence's page t / (R/32) through
+// the block table; false when that page is past the table or its id outside
+// the pool (nothing may be read or written then).
+__host__ __device__ inline bool store_tile(const CacheView& c, long long u, long long t,
+                                           long long* su, long long* st) {
+  if (c.bt == nullptr) {
+    *su = u;
+    *st = t;
+    return true;
+  }
+  const long long tpp = c.R / kTile;
+  const long long lp = t / tpp;
+  if (t < 0 || lp >= c.pps) return false;
+  const long long b = u / c.Hkv;
+  const long long pg = c.bt[b * c.pps + lp];
+  if (pg < 0 || pg >= c.n_pages) return false;
+  *su = pg * c.Hkv + u % c.Hkv;
+  *st = t % tpp;
+  return true;
+}
 
 template <int D, int BITS>
 struct Layout {

@@ -31,6 +31,9 @@ namespace {
 // blockDim.x == D.  Thread d reduces key channel d over the tile's tokens;
 // thread i reduces value group (token i / NJ, group i % NJ) over kGv channels.
 // Codes go through shared memory and are packed by all threads.
+// Paged stores: the tile goes to its page's slot (a page outside the block
+// table or the pool writes nothing; the callers have refused such a
+// sequence already).
 template <int D, int BITS, typename T, typename M>
 __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit,
                                               const T* __restrict__ Ksrc,
@@ -40,6 +43,13 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
   constexpr int E = Lt::E, WK = Lt::WK, NJ = Lt::NJ;
   const float Lf = (float)Lt::L;
   const int tid = threadIdx.x;
+  const long long Ts = store_tokens(c);
+  {
+    long long su, stl;
+    if (!store_tile(c, unit, t0 / kTile, &su, &stl)) return;  // same for the whole block
+    unit = su;
+    t0 = stl * kTile;
+  }
 
   // ---- keys: channel tid over kTile tokens
   {
@@ -55,8 +65,8 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
     const float s = round_meta<M>(__fdiv_rn(__fsub_rn(mx, mn), Lf));
     const float z = round_meta<M>(mn);
     const long long g = t0 / kG;
-    reinterpret_cast<M*>(c.k_scale)[unit * Lt::k_meta_unit(c.Tq) + g * D + tid] = from_f32<M>(s);
-    reinterpret_cast<M*>(c.k_zero)[unit * Lt::k_meta_unit(c.Tq) + g * D + tid] = from_f32<M>(z);
+    reinterpret_cast<M*>(c.k_scale)[unit * Lt::k_meta_unit(Ts) + g * D + tid] = from_f32<M>(s);
+    reinterpret_cast<M*>(c.k_zero)[unit * Lt::k_meta_unit(Ts) + g * D + tid] = from_f32<M>(z);
 #pragma unroll
     for (int t = 0; t < kTile; ++t) {
       int code = 0;
@@ -82,7 +92,7 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
     }
     const float s = round_meta<M>(__fdiv_rn(__fsub_rn(mx, mn), Lf));
     const float z = round_meta<M>(mn);
-    const long long mo = unit * Lt::v_meta_unit(c.Tq) + (t0 + t) * NJ + j;
+    const long long mo = unit * Lt::v_meta_unit(Ts) + (t0 + t) * NJ + j;
     reinterpret_cast<M*>(c.v_scale)[mo] = from_f32<M>(s);
     reinterpret_cast<M*>(c.v_zero)[mo] = from_f32<M>(z);
 #pragma unroll
@@ -98,8 +108,8 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
   __syncthreads();
   // ---- pack: keys along channels, values along tokens; D*BITS words each
   constexpr int NW = kTile * WK;  // == (kTile / E) * D == D * BITS
-  uint32_t* kdst = c.k_codes + unit * Lt::k_codes_unit(c.Tq) + t0 * WK;
-  uint32_t* vdst = c.v_codes + unit * Lt::v_codes_unit(c.Tq) + (t0 / E) * D;
+  uint32_t* kdst = c.k_codes + unit * Lt::k_codes_unit(Ts) + t0 * WK;
+  uint32_t* vdst = c.v_codes + unit * Lt::v_codes_unit(Ts) + (t0 / E) * D;
 #pragma unroll
   for (int k = tid; k < NW; k += D) {
     const int t = k / WK, w = k % WK;
@@ -139,9 +149,19 @@ __global__ void __launch_bounds__(D) prefill_kernel(CacheView c, const T* __rest
   if (lens != nullptr) {
     const long long b = unit / Hkv;
     const long long n = lens[b];
-    const bool ok = n >= 1 && n <= T_len && n <= c.Tq + c.R;
+    bool ok = n >= 1 && n <= T_len && n <= c.Tq + c.R;
     r = ok ? (int)((n - 1) % c.R) + 1 : 0;
     n_q = ok ? n - r : 0;
+    if (ok && c.bt != nullptr) {  // every page the prompt fills must be in the pool
+      for (long long l = 0; l < n_q / c.R; ++l) {
+        const int pg = c.bt[b * c.pps + l];
+        ok = ok && pg >= 0 && pg < c.n_pages;
+      }
+      if (!ok) {
+        r = 0;
+        n_q = 0;
+      }
+    }
     if (tile == gridDim.x - 1 && unit == b * Hkv && threadIdx.x == 0) {
       DevState v;
       v.n_q = n_q;
@@ -184,8 +204,13 @@ __global__ void __launch_bounds__(D) append_kernel(CacheView c, const T* __restr
     const long long nq = s0.n_q;
     const int r = s0.r;
     // counters that are not a valid fill of the cache are refused too
-    if (s0.status != 0 || nq < 0 || nq > c.Tq || nq % c.R != 0 || r < 0 || r > c.R ||
-        nq + r + 1 > c.Tq + c.R) {
+    bool bad = s0.status != 0 || nq < 0 || nq > c.Tq || nq % c.R != 0 || r < 0 || r > c.R ||
+               nq + r + 1 > c.Tq + c.R;
+    if (!bad && c.bt != nullptr && r == c.R) {  // the flush fills page nq / R
+      const long long pg = c.bt[sb * c.pps + nq / c.R];
+      bad = pg < 0 || pg >= c.n_pages;
+    }
+    if (bad) {
       if (blockIdx.x == 0 && blockIdx.y == sb * (Hkv > 0 ? Hkv : 1) && threadIdx.x == 0)
         ss->status = 1;
       return;

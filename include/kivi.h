@@ -152,6 +152,10 @@ typedef struct {
   void *v_res;
   long long n_q; /* tokens per sequence in the quantized store */
   int r;         /* tokens per sequence in the residual window */
+  /* paged store (kivi_paged_cache_init); NULL / 0 for a contiguous cache */
+  const int32_t *block_table; /* device, [B][pages_per_seq] pool page ids */
+  int pages_per_seq;
+  long long num_pages;        /* pages in the pool */
 } kivi_cache;
 
 /* Byte size of each of the KIVI_NUM_BUFFERS buffers for `dims`, written to
@@ -286,6 +290,34 @@ KIVI_API int kivi_append_decode_dev(const kivi_cache *cache, void *state, const 
  * (KIVI, study.space summary: a grouped part plus a residual part per
  * sequence; scholarfeed.org "KIVI" page: mixed-precision caches do not fit
  * uniform paged blocks, hence per-sequence counters here.) */
+
+/* Paged store (ragged batches only).  The quantized store of every
+ * sequence is a list of pages of R tokens (one flushed window each) taken
+ * from a shared pool: page l of sequence b is pool page
+ * block_table[b * pages_per_seq + l] (device int32, owned and filled by the
+ * caller; distinct sequences must not share a page).  Pool layout, per
+ * page and KV head, the contiguous layout above with Tq = R:
+ *   k_codes uint32 [num_pages][Hkv][R][D/E]   k_scale, k_zero [num_pages][Hkv][R/G][D]
+ *   v_codes uint32 [num_pages][Hkv][R/E][D]   v_scale, v_zero [num_pages][Hkv][R][NJ]
+ * The residual windows stay per sequence, [B][Hkv][R][D] (a mixed-precision
+ * cache keeps its full-precision part apart from the uniform pages:
+ * scholarfeed.org "KIVI" page, second quote).  dims.capacity must be
+ * (pages_per_seq + 1) * R.  A page id outside [0, num_pages) where a
+ * sequence needs a page refuses that sequence (status 1) at prefill or
+ * flush time.
+ * kivi_paged_buffer_sizes: byte sizes of the 8 buffers for a pool of
+ * num_pages pages.  Errors: KIVI_ERR_ARG, KIVI_ERR_UNSUPPORTED. */
+KIVI_API int kivi_paged_buffer_sizes(const kivi_dims *dims, long long num_pages,
+                            size_t out_bytes[KIVI_NUM_BUFFERS]);
+
+/* Bind a pool (buffers as sized by kivi_paged_buffer_sizes, 16-byte
+ * aligned) and a block table to `cache`; the cache is then filled with
+ * kivi_ragged_prefill and used with the kivi_ragged_* calls only.
+ * Errors: KIVI_ERR_ARG (null or misaligned pointer, capacity not
+ * (pages_per_seq + 1) * R, num_pages < 1), KIVI_ERR_UNSUPPORTED. */
+KIVI_API int kivi_paged_cache_init(kivi_cache *cache, const kivi_dims *dims,
+                          void *const buffers[KIVI_NUM_BUFFERS], const int32_t *block_table,
+                          int pages_per_seq, long long num_pages);
 
 /* Prefill of a ragged batch into an empty cache.  K, V: device, dims.dtype,
  * [B][Hkv][T_max][D] (padded; sequence b uses its first lens[b] tokens).

@@ -236,3 +236,56 @@ def test_ragged_lengths_of_a_state():
     w[:, 2] = torch.tensor([1, 128, 7], dtype=torch.int32)
     w[:, 3] = torch.tensor([0, 0, 1], dtype=torch.int32)
     assert kivi.ragged_lengths(st) == ([0, 4096, 1 << 40], [1, 128, 7], [0, 0, 1])
+
+
+def test_cache_struct_matches_the_header():
+    names = [f[0] for f in KiviCacheC._fields_]
+    text = open(HEADER).read()
+    body = text[text.index("typedef struct {\n  kivi_dims dims;"):text.index("} kivi_cache;")]
+    declared = re.findall(r"\b(\w+);", re.sub(r"/\*.*?\*/", "", body, flags=re.S))
+    assert declared == names
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_paged_buffer_sizes(bits):
+    B, H, D, R, P = 3, 5, 128, 64, 11
+    dims = _dims(B=B, Hkv=H, D=D, bits=bits, R=R, capacity=4 * R)
+    out = (ctypes.c_size_t * 8)()
+    assert kivi.lib().kivi_paged_buffer_sizes(ctypes.byref(dims), P, ctypes.byref(out)) == 0
+    E = 32 // bits
+    s = list(out)
+    assert s[0] == P * H * R * (D // E) * 4
+    assert s[1] == s[2] == P * H * (R // 32) * D * 4
+    assert s[3] == P * H * (R // E) * D * 4
+    assert s[4] == s[5] == P * H * R * (D // 32) * 4
+    assert s[6] == s[7] == B * H * R * D * 2
+    assert kivi.lib().kivi_paged_buffer_sizes(ctypes.byref(dims), 0, ctypes.byref(out)) == ERR_ARG
+
+
+def test_paged_cache_init_and_refusals():
+    L = kivi.lib()
+    R = 64
+    dims = _dims(R=R, capacity=5 * R)  # 4 pages per sequence + the window
+    ptrs = (ctypes.c_void_p * 8)(*[0x10000 * (i + 1) for i in range(8)])
+    bt = ctypes.c_void_p(0x90000)
+    c = KiviCacheC()
+    assert L.kivi_paged_cache_init(ctypes.byref(c), ctypes.byref(dims), ctypes.byref(ptrs), None, 4,
+                                   16) == ERR_ARG
+    assert L.kivi_paged_cache_init(ctypes.byref(c), ctypes.byref(dims), ctypes.byref(ptrs), bt, 3,
+                                   16) == ERR_ARG  # capacity is not (3 + 1) * R
+    assert L.kivi_paged_cache_init(ctypes.byref(c), ctypes.byref(dims), ctypes.byref(ptrs), bt, 4,
+                                   0) == ERR_ARG
+    assert L.kivi_paged_cache_init(ctypes.byref(c), ctypes.byref(dims), ctypes.byref(ptrs), bt, 4,
+                                   16) == 0
+    assert (c.block_table, c.pages_per_seq, c.num_pages, c.n_q, c.r) == (0x90000, 4, 16, 0, 0)
+    fake = ctypes.c_void_p(0x5000)
+    # a paged cache takes the ragged calls only
+    assert L.kivi_quantize_prefill(ctypes.byref(c), fake, fake, 10, None) == ERR_STATE
+    assert L.kivi_append_token(ctypes.byref(c), fake, fake, None) == ERR_STATE
+    assert L.kivi_dev_state_init(ctypes.byref(c), fake, None) == ERR_STATE
+    c.n_q, c.r = 64, 5
+    assert L.kivi_decode_attention(ctypes.byref(c), fake, 4, 1.0, fake, fake, 1 << 20,
+                                   None) == ERR_STATE
+    # a contiguous cache carries no block table
+    c2 = _fake_cache()
+    assert (c2.block_table, c2.pages_per_seq, c2.num_pages) == (None, 0, 0)
