@@ -273,6 +273,7 @@ def run_kivi(args, rank, world, local):
             c.prefill(Kp, Vp)
         caches.append(c)
     del Kp, Vp
+    torch.cuda.empty_cache()
     P = 16
     ks, vs, qs = [], [], []
     for i in range(P):
