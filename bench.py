@@ -235,6 +235,8 @@ def run_kivi(args, rank, world, local):
 
     w = bench_workload(args)
     ragged = w.len_min > 0
+    if args.paged:
+        w = w.with_(name=f"{w.name}-paged-{args.paged}")
     if ragged and (args.kernel != "default" or args.unfused):
         raise SystemExit("ragged workloads run the fused tensor-core step only")
     if args.paged and not ragged:
@@ -251,6 +253,7 @@ def run_kivi(args, rank, world, local):
     # the algorithmic bytes (the library keeps them on the device)
     host_len = []
     pps = capacity // w.R - 1
+    pre_ev = []  # CUDA events around each layer's prefill
     for li in range(n_layers):
         if args.paged:
             # every layer its own pool with a shuffled table (distinct pages)
@@ -265,13 +268,50 @@ def run_kivi(args, rank, world, local):
         else:
             c = kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, capacity, R=w.R, G=w.G, Gv=w.Gv,
                                dtype=w.torch_dtype, device=device, meta=w.torch_meta)
+        pe = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        pe[0].record()
         if ragged:
             states.append(c.ragged_prefill(Kp, Vp, lens_dev))
             rr = [int((x - 1) % w.R) + 1 for x in lens.tolist()]
             host_len.append(([int(x) - y for x, y in zip(lens.tolist(), rr)], rr))
         else:
             c.prefill(Kp, Vp)
+        pe[1].record()
+        pre_ev.append(pe)
         caches.append(c)
+    # append alone (host counters): 2R + 8 calls on a scratch cache of the
+    # same shape, each between CUDA events, split into flush and plain steps
+    append_times = None
+    if not ragged:
+        sc = kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, -(-(w.T + 2 * w.R + 8) // w.R) * w.R, R=w.R,
+                            G=w.G, Gv=w.Gv, dtype=w.torch_dtype, device=device, meta=w.torch_meta)
+        sc.prefill(Kp, Vp)
+        k0, v0 = W.step_kv(w, 0, device=device)
+        evs_a = []
+        for i in range(2 * w.R + 8):
+            ea = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            flush = sc.r == sc.R
+            # keep the GPU busy while the host enqueues the call, so that the
+            # events bracket device time only (not the host's launch latency)
+            torch.cuda._sleep(200_000)
+            ea[0].record()
+            sc.append(k0, v0)
+            ea[1].record()
+            evs_a.append((flush, ea))
+        torch.cuda.synchronize(device)
+        t_fl = [e[0].elapsed_time(e[1]) * 1e3 for f, e in evs_a[4:] if f]
+        t_pl = [e[0].elapsed_time(e[1]) * 1e3 for f, e in evs_a[4:] if not f]
+        append_times = {"call": "kivi_append_token", "plain_us": statistics.median(t_pl),
+                        "flush_us": statistics.median(t_fl) if t_fl else None,
+                        "flushes_timed": len(t_fl)}
+        del sc
+    torch.cuda.synchronize(device)
+    pre_us = statistics.median(e0.elapsed_time(e1) * 1e3 for e0, e1 in pre_ev[1:] or pre_ev)
+    es_in = 2 if w.dtype == "f16" else 4
+    pre_tokens = int(lens.sum()) if ragged else w.B * w.T
+    prefill_times = {"call": "kivi_ragged_prefill" if ragged else "kivi_quantize_prefill",
+                     "us": pre_us, "tokens_per_s": pre_tokens / (pre_us * 1e-6),
+                     "input_GBps": 2 * pre_tokens * w.Hkv * w.D * es_in / (pre_us * 1e-6) / 1e9}
     del Kp, Vp
     torch.cuda.empty_cache()
     P = 16
@@ -383,6 +423,9 @@ def run_kivi(args, rank, world, local):
 
     # roofline of the split kernel: algorithmic bytes / event time
     bytes_total = sum(algorithmic_bytes(w, nq, r) for nq, r in fills)
+    # tokens attended per step (summed over sequences, per KV head), mean over the fills
+    ctx_tokens = statistics.mean((sum(nq) + sum(r)) if isinstance(nq, list) else w.B * (nq + r)
+                                 for nq, r in fills)
     split_total_ms = sum(split_ms)
     achieved = bytes_total / (split_total_ms * 1e-3) / 1e9
     peak, peak_src = peak_hbm()
@@ -391,12 +434,17 @@ def run_kivi(args, rank, world, local):
     # e2e: the same loop, inputs from pinned host memory, output read back
     e2e = None
     if not args.no_e2e:
-        hk = [t.cpu().pin_memory() for t in ks]
-        hv = [t.cpu().pin_memory() for t in vs]
-        hq = [t.cpu().pin_memory() for t in qs]
+        # each step's k, v and q staged in one pinned host buffer and brought
+        # over in one copy; k, v, q are views of one device buffer
+        nk, nq_ = ks[0].numel(), qs[0].numel()
+        hs = [torch.cat([ks[j].flatten(), vs[j].flatten(), qs[j].flatten()]).cpu().pin_memory()
+              for j in range(P)]
         ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        dk, dv, dq = torch.empty_like(ks[0]), torch.empty_like(vs[0]), torch.empty_like(qs[0])
-        h2d = 3 * ks[0].numel() * ks[0].element_size()
+        dst = torch.empty_like(hs[0], device=device)
+        dk = dst[:nk].view(ks[0].shape)
+        dv = dst[nk:2 * nk].view(vs[0].shape)
+        dq = dst[2 * nk:].view(qs[0].shape)
+        h2d = hs[0].numel() * hs[0].element_size()
         d2h = out.numel() * out.element_size()
         n_e2e = e2e_steps
         base = args.warmup + 2 * args.steps
@@ -406,9 +454,7 @@ def run_kivi(args, rank, world, local):
         for j in range(n_e2e):
             i = base + j
             li = i % n_layers
-            dk.copy_(hk[i % P], non_blocking=True)
-            dv.copy_(hv[i % P], non_blocking=True)
-            dq.copy_(hq[i % P], non_blocking=True)
+            dst.copy_(hs[i % P], non_blocking=True)
             rc = step_call(li, dk.data_ptr(), dv.data_ptr(), dq.data_ptr())
             if rc:
                 raise RuntimeError("e2e step failed")
@@ -458,6 +504,9 @@ def run_kivi(args, rank, world, local):
                 "algorithmic_bytes_per_launch": bytes_total / args.steps,
                 "avg_launch_us": split_total_ms * 1e3 / args.steps,
             },
+            "context_tokens_per_s": ctx_tokens * w.Hkv / (ms_max / args.steps * 1e-3) * world,
+            "prefill": prefill_times,
+            "append": append_times,
             "e2e": e2e,
             "gpu_launches": timed_launches,
             "clocks": clk.summary(),
@@ -512,6 +561,16 @@ def oracle_sample(w: W.Workload, n_units: int, steps: int, threads: int):
     return dt / steps, len(units), scale
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_threads():
     try:
         return len(os.sched_getaffinity(0))
@@ -528,7 +587,7 @@ def cpu_baseline(w: W.Workload, budget_s: float):
     steps = max(1, int(budget_s * threads / (per_unit_cpu * n_units)))
     per_step, n, scale = oracle_sample(w, n_units, steps, threads)
     full_step = per_step * scale
-    return {"value": w.B / full_step, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+    return {"value": w.B / full_step, "unit": "tokens/s", "cores": threads, "cpu_model": cpu_model(), "kind": "oracle",
             "sample": f"{steps} steps x {n} of {w.B * w.Hkv} (batch, KV head) units spread "
                       f"over the batch, append + decode, scaled to the full batch by tokens "
                       f"held; single oracle threads fanned out over units"}
@@ -555,7 +614,7 @@ def run_reference(args, rank, world):
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                    "context": w.T, "bits": w.bits, "G": w.G, "Gv": w.Gv, "R": w.R,
                    "meta": w.meta},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "cpu_model": cpu_model(), "kind": "oracle",
                          "sample": f"each step: append + decode on {n} of {w.B * w.Hkv} units, "
                                    f"scaled to the full batch"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
