@@ -24,7 +24,7 @@ int check_dims(const kivi_dims* d) {
   if (!d) return KIVI_ERR_ARG;
   if (d->B <= 0 || d->Hkv <= 0 || d->D <= 0 || d->R <= 0 || d->capacity <= 0)
     return KIVI_ERR_ARG;
-  if (d->bits != 2 && d->bits != 4) return KIVI_ERR_UNSUPPORTED;
+  if (d->bits != 1 && d->bits != 2 && d->bits != 4) return KIVI_ERR_UNSUPPORTED;
   if (d->G != kivi::kG || d->Gv != kivi::kGv) return KIVI_ERR_UNSUPPORTED;
   if (d->D != 32 && d->D != 64 && d->D != 128) return KIVI_ERR_UNSUPPORTED;
   if (d->R % kivi::kTile != 0) return KIVI_ERR_UNSUPPORTED;

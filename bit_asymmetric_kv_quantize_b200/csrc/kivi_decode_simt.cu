@@ -279,11 +279,14 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t s, cudaEvent_t 
                                cudaEvent_t e1) {
   if (a.meta == 1) {  // binary16 scales and zeros: fp16 caches only
     if (a.dtype != 0) return cudaErrorInvalidValue;
+    if (a.bits == 1) return simt_d<1, __half, __half>(a, s, e0, e1);
     if (a.bits == 2) return simt_d<2, __half, __half>(a, s, e0, e1);
     if (a.bits == 4) return simt_d<4, __half, __half>(a, s, e0, e1);
     return cudaErrorInvalidValue;
   }
   if (a.meta != 0) return cudaErrorInvalidValue;
+  if (a.bits == 1 && a.dtype == 0) return simt_d<1, __half, float>(a, s, e0, e1);
+  if (a.bits == 1 && a.dtype == 1) return simt_d<1, float, float>(a, s, e0, e1);
   if (a.bits == 2 && a.dtype == 0) return simt_d<2, __half, float>(a, s, e0, e1);
   if (a.bits == 2 && a.dtype == 1) return simt_d<2, float, float>(a, s, e0, e1);
   if (a.bits == 4 && a.dtype == 0) return simt_d<4, __half, float>(a, s, e0, e1);

@@ -15,6 +15,8 @@ cudaError_t tc_dispatch(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cud
   }
   if (a.meta == 1) return tc_dispatch_meta16(a, s, e0, e1, occ);
   if (a.meta != 0) return cudaErrorInvalidValue;
+  if (a.bits == 1 && a.dtype == 0) return tc_d<1, __half, float, false>(a, s, e0, e1, occ);
+  if (a.bits == 1 && a.dtype == 1) return tc_d<1, float, float, false>(a, s, e0, e1, occ);
   if (a.bits == 2 && a.dtype == 0) return tc_d<2, __half, float, false>(a, s, e0, e1, occ);
   if (a.bits == 2 && a.dtype == 1) return tc_d<2, float, float, false>(a, s, e0, e1, occ);
   if (a.bits == 4 && a.dtype == 0) return tc_d<4, __half, float, false>(a, s, e0, e1, occ);

@@ -57,11 +57,20 @@ constexpr float kNegInf = -__builtin_huge_valf();
 constexpr long long kWaitCycles = 1LL << 32;  // ~2 s: bounded wait on our own copies
 constexpr int kSuspendNs = 1000;  // a waiting thread sleeps up to this long per try
 
-// Code pairs of one 32-bit word.  2-bit: pair i (i < 8) = codes i and i + 8;
-// 4-bit: pair i (i < 4) = codes i and i + 4.  (w >> shift(i)) & mask(i) puts
-// the pair's codes at bit e(i) of the low and the high half.
+// Code pairs of one 32-bit word.  1-bit: pair i (i < 16) = codes i and
+// i + 16; 2-bit: pair i (i < 8) = codes i and i + 8; 4-bit: pair i (i < 4) =
+// codes i and i + 4.  (w >> shift(i)) & mask(i) puts the pair's codes at bit
+// e(i) of the low and the high half.
 template <int BITS>
 struct Pairs;
+template <>
+struct Pairs<1> {
+  static constexpr int PPW = 16;  // pairs per word
+  static constexpr int EMAX = 9;  // largest e
+  __host__ __device__ static constexpr int e(int i) { return i < 10 ? i : i - 10; }
+  __host__ __device__ static constexpr int shift(int i) { return i < 10 ? 0 : 10; }
+  __host__ __device__ static constexpr uint32_t mask(int i) { return 0x00010001u << e(i); }
+};
 template <>
 struct Pairs<2> {
   static constexpr int PPW = 8;   // pairs per word
@@ -87,7 +96,8 @@ struct Pairs<4> {
 template <int D, int BITS, int GQ, int MB>
 struct Geo {
   static constexpr int NW = GQ == 1 ? 4 : (GQ == 8 ? 7 : 11);
-  static constexpr int TPW = (GQ == 1 && BITS == 2) ? 2 : 1;  // tiles per warp and stage
+  // tiles per warp and stage (1-bit MHA also needs two to fit a window tile in a stage)
+  static constexpr int TPW = (GQ == 1 && BITS <= 2) ? 2 : 1;
   static constexpr int THREADS = (NW + 1) * 32;
   static constexpr int kStage = NW * TPW;       // tiles per pipeline stage
   static constexpr int E = 32 / BITS;
@@ -106,7 +116,18 @@ struct Geo {
   static constexpr int O_VC = O_KZ + kStage * KM_B;
   static constexpr int O_VS = O_VC + kStage * VC_B;
   static constexpr int O_VZ = O_VS + kStage * VM_B;
-  static constexpr int STAGE_B = (O_VZ + kStage * VM_B + 1023) / 1024 * 1024;
+  // fp16 residual window through the ring: a window stage holds WT tokens of
+  // K, then of V, as 2-D tensor-copy boxes of BW columns (rows of RB bytes)
+  // in the hardware's 128-byte (64-byte when D = 32) swizzle
+  static constexpr int WT = kTile;
+  static constexpr int BW = D < 64 ? D : 64;
+  static constexpr int NBX = D / BW;
+  static constexpr int RB = BW * 2;
+  static constexpr int BOX_B = WT * RB;
+  static constexpr int WTILE_B = 2 * NBX * BOX_B;     // one 32-token window tile (K, V)
+  // a stage holds kStage code tiles, and at least one window tile
+  static constexpr int CODE_STAGE_B = (O_VZ + kStage * VM_B + 1023) / 1024 * 1024;
+  static constexpr int STAGE_B = CODE_STAGE_B < WTILE_B ? WTILE_B : CODE_STAGE_B;
   static constexpr int NSTAGE = (NW == 4 && TPW == 1 && BITS == 2) ? 3 : 2;
   static constexpr int NPB = GQ == 8 ? 2 : 1;  // n-tiles of 8 columns (4 heads x hi, lo)
   static constexpr int PST = TPW * kTile + 8;  // p buffer stride per head (floats)
@@ -132,16 +153,7 @@ struct Geo {
   static constexpr int NWL = WHOLE ? PPL / PPW : 1;
   // operand scale offsets: the factor 2^(S - e) lies in [2^-S, 2^S]
   static constexpr int SK = Pairs<BITS>::EMAX / 2;
-  static constexpr int SV = BITS == 2 ? 3 : 2;  // value e: 2-bit 0,2,4,6; 4-bit 0,4
-  // fp16 residual window through the ring: a window stage holds WT tokens of
-  // K, then of V, as 2-D tensor-copy boxes of BW columns (rows of RB bytes)
-  // in the hardware's 128-byte (64-byte when D = 32) swizzle
-  static constexpr int WT = kTile;
-  static constexpr int BW = D < 64 ? D : 64;
-  static constexpr int NBX = D / BW;
-  static constexpr int RB = BW * 2;
-  static constexpr int BOX_B = WT * RB;
-  static constexpr int WTILE_B = 2 * NBX * BOX_B;     // one 32-token window tile (K, V)
+  static constexpr int SV = BITS == 2 ? 3 : 2;  // value e: 1-bit 0..3; 2-bit 0,2,4,6; 4-bit 0,4
   static constexpr int WPS = STAGE_B / WTILE_B;       // window tiles per stage
   static_assert(WPS >= 1, "a window tile fits one ring slot");
   static_assert(WTILE_B % 1024 == 0, "window tiles keep the 1024-byte alignment");
@@ -638,23 +650,33 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
       cp_f0[m] = __int_as_float((127 + G::SK - PR::e(i0)) << 23);
       cp_f1[m] = __int_as_float((127 + G::SK - PR::e(i0 + 1)) << 23);
     }
-    // -- key operand (D = 32, 2-bit): a lane's four pairs sit in word tq/2,
-    // pairs 4 (tq & 1) + jj -- shifts and masks differ per lane
-    uint32_t kS[4], kM[4];
+    // -- key operand when a lane's PPL pairs are part of one word (2-bit
+    // D = 32, 1-bit D = 32, 64): they sit in word tq PPL / PPW, pairs
+    // (tq PPL) % PPW + jj -- shifts and masks differ per lane
+    constexpr int NKS = G::WHOLE ? 1 : G::PPL;
+    uint32_t kS[NKS], kM[NKS];
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int i = 4 * (tq & 1) + jj;
-      kS[jj] = (uint32_t)Pairs<2>::shift(i);
-      kM[jj] = Pairs<2>::mask(i);
+    for (int jj = 0; jj < NKS; ++jj) {
+      const int i = (tq * G::PPL) % G::PPW + jj;
+      kS[jj] = (uint32_t)PR::shift(i);
+      kM[jj] = PR::mask(i);
     }
     // -- value operand: lane tq takes the pairs at e = 2 tq (2-bit) or
-    // 4 (tq & 1) (4-bit) of its word; a0 / a1 unshifted, a2 / a3 after >> 8
-    const uint32_t vM = BITS == 2 ? (0x00030003u << (2 * tq))
-                                  : ((tq & 1) ? 0x00F000F0u : 0x000F000Fu);
-    const int vtw = BITS == 2 ? 0 : (tq >> 1);  // token-word offset of this lane
+    // 4 (tq & 1) (4-bit) of its word; a0 / a1 unshifted, a2 / a3 after >> 8.
+    // 1-bit: one word holds the tile's 32 tokens (low half 0..15, high half
+    // 16..31); k-slice sl takes tokens 8 sl .. 8 sl + 7 and their +16
+    // partners, lane tq the pair at bit tq after a shift by 8 sl (a0 / a1)
+    // or 8 sl + 4 (a2 / a3)
+    const uint32_t vM = BITS == 1 ? (0x00010001u << tq)
+                        : BITS == 2 ? (0x00030003u << (2 * tq))
+                                    : ((tq & 1) ? 0x00F000F0u : 0x000F000Fu);
+    const int vtw = BITS == 4 ? (tq >> 1) : 0;  // token-word offset of this lane
     // -- p' build, lane = token t: its k-slice, owner slot and e
     int pt_sl, pt_tq, pt_kp, pt_hf, pt_e;
-    if (BITS == 2) {
+    if (BITS == 1) {
+      const int i = lane & 15;
+      pt_hf = lane >> 4; pt_sl = i >> 3; pt_kp = (i >> 2) & 1; pt_tq = i & 3; pt_e = pt_tq;
+    } else if (BITS == 2) {
       const int i = lane & 15;
       pt_sl = lane >> 4; pt_tq = i & 3; pt_kp = (i >> 2) & 1; pt_hf = (i >> 3) & 1; pt_e = 2 * pt_tq;
     } else {
@@ -816,7 +838,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
 #pragma unroll
               for (int r = 0; r < 2; ++r) {
                 const uint32_t* row = kc[tt] + (16 * mt + 8 * r + g) * WK +
-                                      (G::WHOLE ? tq * G::NWL : (tq >> 1));
+                                      (G::WHOLE ? tq * G::NWL : (tq * G::PPL) / G::PPW);
                 if constexpr (G::NWL == 4) {
                   const uint4 v = *reinterpret_cast<const uint4*>(row);
                   kw[tt][mt][r][0] = v.x; kw[tt][mt][r][1] = v.y;
@@ -833,7 +855,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
               const int i = jj % G::PPW;
               return (w[jj / G::PPW] >> PR::shift(i)) & PR::mask(i);
             } else {
-              return (w[0] >> kS[jj & 3]) & kM[jj & 3];
+              return (w[0] >> kS[jj]) & kM[jj];
             }
           };
           float dq[TPW][NPB][2][4];
@@ -965,14 +987,19 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           for (int tt = 0; tt < TPW; ++tt) {
 #pragma unroll
             for (int sl = 0; sl < NSL; ++sl) {
-              const int tw = BITS == 2 ? sl : 2 * sl + vtw;
+              const int tw = BITS == 1 ? 0 : BITS == 2 ? sl : 2 * sl + vtw;
+              constexpr int SH = BITS == 1 ? 4 : 8;  // shift to the a2 / a3 pairs
+              const int s0 = BITS == 1 ? 8 * sl : 0;  // 1-bit: this slice's byte
 #pragma unroll
               for (int j = 0; j < NJ; ++j) {
-                const uint4 w = *reinterpret_cast<const uint4*>(vc[tt] + tw * D + 32 * j + 4 * g);
-                const uint32_t x0 = w.x & vM, x2 = (w.x >> 8) & vM;
-                const uint32_t x1 = w.y & vM, x3 = (w.y >> 8) & vM;
-                const uint32_t y0 = w.z & vM, y2 = (w.z >> 8) & vM;
-                const uint32_t y1 = w.w & vM, y3 = (w.w >> 8) & vM;
+                uint4 w = *reinterpret_cast<const uint4*>(vc[tt] + tw * D + 32 * j + 4 * g);
+                if (BITS == 1) {
+                  w.x >>= s0; w.y >>= s0; w.z >>= s0; w.w >>= s0;
+                }
+                const uint32_t x0 = w.x & vM, x2 = (w.x >> SH) & vM;
+                const uint32_t x1 = w.y & vM, x3 = (w.y >> SH) & vM;
+                const uint32_t y0 = w.z & vM, y2 = (w.z >> SH) & vM;
+                const uint32_t y1 = w.w & vM, y3 = (w.w >> SH) & vM;
 #pragma unroll
                 for (int p = 0; p < NPB; ++p) {
                   const uint2 bb = bcol ? *reinterpret_cast<const uint2*>(

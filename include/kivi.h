@@ -107,7 +107,7 @@ typedef enum { KIVI_F16 = 0, KIVI_F32 = 1 } kivi_dtype;
  * storage precision for them.) */
 typedef enum { KIVI_META_F32 = 0, KIVI_META_F16 = 1 } kivi_meta;
 
-/* Shape of one cache (one attention layer).  Supported: bits in {2, 4},
+/* Shape of one cache (one attention layer).  Supported: bits in {1, 2, 4},
  * G = 32, Gv = 32, D in {32, 64, 128}, R a positive multiple of 32,
  * capacity a positive multiple of R, dtype KIVI_F16 or KIVI_F32, meta
  * KIVI_META_F32 or (with dtype KIVI_F16) KIVI_META_F16.  A zero-filled

@@ -45,7 +45,7 @@ def _sizes(dims):
     return rc, list(out)
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_buffer_sizes_follow_the_layout(bits, D):
     B, H, R, cap = 3, 5, 64, 640
@@ -62,7 +62,7 @@ def test_buffer_sizes_follow_the_layout(bits, D):
         assert sum(s[:6]) == u * Tq * D * 2 * 0.5
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_binary16_metadata_halves_the_scale_and_zero_buffers(bits, D):
     B, H, R, cap = 3, 5, 64, 640
@@ -246,7 +246,7 @@ def test_cache_struct_matches_the_header():
     assert declared == names
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 4])
 def test_paged_buffer_sizes(bits):
     B, H, D, R, P = 3, 5, 128, 64, 11
     dims = _dims(B=B, Hkv=H, D=D, bits=bits, R=R, capacity=4 * R)

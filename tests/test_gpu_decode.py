@@ -44,7 +44,7 @@ def run(w, kernel, sigma=None, capacity=None):
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("gq", [1, 2, 4, 8])
 @pytest.mark.parametrize("dtype", ["f16", "f32"])
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_decode_shapes(D, bits, dtype, gq, kernel):
     for T in (1, 33, 161, 1000):

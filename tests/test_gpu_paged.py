@@ -86,7 +86,7 @@ def prefill_three(w, lens, pps, num_pages, units=None, seed=0):
 
 @pytest.mark.parametrize("meta", ["f32", "f16"])
 @pytest.mark.parametrize("gq", [1, 4, 8])
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_prefill_and_decode(D, bits, gq, meta):
     w = small(D=D, bits=bits, gq=gq, T=700, B=5, meta=meta)

@@ -96,7 +96,7 @@ def test_prefill_lengths_and_refusals():
 @pytest.mark.parametrize("meta", ["f32", "f16"])
 @pytest.mark.parametrize("gq", [1, 2, 4, 8])
 @pytest.mark.parametrize("dtype", ["f16", "f32"])
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_decode_shapes(D, bits, dtype, gq, meta):
     if meta == "f16" and dtype == "f32":
