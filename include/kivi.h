@@ -1,5 +1,5 @@
 /*
- * kivi.h -- C ABI of libkivi.so: a KIVI-style asymmetric 2/4-bit KV cache
+ * kivi.h -- C ABI of libkivi.so: a KIVI-style asymmetric 1/2/4-bit KV cache
  * with a full-precision residual window and fused decode attention, for
  * NVIDIA B200 (sm_100a).
  *
