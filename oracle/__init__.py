@@ -65,6 +65,7 @@ def lib():
             up = ctypes.POINTER(Unit)
             L.kivi_oracle_quantize_group.argtypes = [vp, ll, ll, ci, vp, vp, vp]
             L.kivi_oracle_quantize_group_meta.argtypes = [vp, ll, ll, ci, ci, vp, vp, vp]
+            L.kivi_oracle_quantize_group_sparse.argtypes = [vp, ll, ll, ci, ci, vp, vp, vp, vp, vp]
             L.kivi_oracle_round_half.argtypes = [ctypes.c_float]
             L.kivi_oracle_round_half.restype = ctypes.c_float
             L.kivi_oracle_pack_word.argtypes = [vp, ci]
@@ -109,6 +110,21 @@ def quantize_group(x, bits: int, meta_f16: bool = False):
                                                  _ptr(s), _ptr(z), _ptr(c)),
            "quantize_group")
     return s[0], z[0], c
+
+
+def quantize_group_sparse(x, bits: int, k: int):
+    """Q, dense-and-sparse variant on one group: returns (scale, zero,
+    codes[uint16], outlier indices[int64], outlier values[float32]); the k
+    largest-magnitude entries are kept exactly, the rest quantized by Q."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    s, z = ctypes.c_float(), ctypes.c_float()
+    codes = np.zeros(x.size, np.uint16)
+    idx = np.zeros(max(k, 1), np.int64)
+    val = np.zeros(max(k, 1), np.float32)
+    _check(lib().kivi_oracle_quantize_group_sparse(_ptr(x), x.size, 1, bits, k, ctypes.byref(s),
+                                                   ctypes.byref(z), _ptr(codes), _ptr(idx),
+                                                   _ptr(val)), "quantize_group_sparse")
+    return s.value, z.value, codes, idx[:k], val[:k]
 
 
 def round_half(x: float) -> float:

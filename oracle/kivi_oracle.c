@@ -124,6 +124,66 @@ int kivi_oracle_quantize_group_meta(const float *x, long long n, long long strid
 }
 
 /*
+ * Q, dense-and-sparse variant (KVQuant on the codewithpapers.app page,
+ * abstract item (iv): outliers are isolated separately for each vector so
+ * that they do not skew its quantization range).  Reading: the vector is
+ * the quantization group; its k entries of largest magnitude (equal
+ * magnitudes: the lower index first) are kept exactly in a sparse list, in
+ * ascending index order, and Q runs over the other n - k entries in their
+ * order; an outlier's dense code is 0.  Requires 0 <= k < n.
+ */
+int kivi_oracle_quantize_group_sparse(const float *x, long long n, long long stride, int bits,
+                                      int k, float *scale, float *zero, uint16_t *codes,
+                                      long long *out_idx, float *out_val) {
+  long long i, j, m, picked;
+  unsigned char *is_out;
+  float *rest;
+  uint16_t *rest_codes;
+  int rc;
+  if (!x || !scale || !zero || !codes || n <= 0 || !valid_bits(bits) || k < 0 || k >= n ||
+      (k > 0 && (!out_idx || !out_val)))
+    return KIVI_ORACLE_ERR_ARG;
+  is_out = (unsigned char *)calloc((size_t)n, 1);
+  rest = (float *)malloc((size_t)n * sizeof(float));
+  rest_codes = (uint16_t *)malloc((size_t)n * sizeof(uint16_t));
+  if (!is_out || !rest || !rest_codes) {
+    free(is_out);
+    free(rest);
+    free(rest_codes);
+    return KIVI_ORACLE_ERR_ARG;
+  }
+  /* k passes, each taking the largest magnitude not yet taken */
+  for (picked = 0; picked < k; ++picked) {
+    long long best = -1;
+    for (i = 0; i < n; ++i) {
+      if (is_out[i]) continue;
+      if (best < 0 || fabsf(x[i * stride]) > fabsf(x[best * stride])) best = i;
+    }
+    is_out[best] = 1;
+  }
+  /* the remaining entries, in order, through Q */
+  for (i = 0, m = 0; i < n; ++i)
+    if (!is_out[i]) rest[m++] = x[i * stride];
+  rc = kivi_oracle_quantize_group(rest, m, 1, bits, scale, zero, rest_codes);
+  if (rc == KIVI_ORACLE_OK) {
+    for (i = 0, j = 0, m = 0; i < n; ++i) {
+      if (is_out[i]) {
+        codes[i] = 0;
+        out_idx[j] = i;
+        out_val[j] = x[i * stride];
+        ++j;
+      } else {
+        codes[i] = rest_codes[m++];
+      }
+    }
+  }
+  free(is_out);
+  free(rest);
+  free(rest_codes);
+  return rc;
+}
+
+/*
  * P.  Reading (the pages give no bit layout): E = 32/bits codes per word,
  * the first code in the least significant bits.
  */

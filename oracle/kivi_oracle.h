@@ -87,6 +87,14 @@ int kivi_oracle_quantize_group_meta(const float *x, long long n, long long strid
                                     int bits, int meta_f16, float *scale,
                                     float *zero, uint16_t *codes);
 
+/* Q, dense-and-sparse variant: the k entries of largest magnitude (ties:
+ * lower index first) go to out_idx / out_val in ascending index order with
+ * dense code 0; the other n - k entries are quantized by Q in their order.
+ * Requires 0 <= k < n. */
+int kivi_oracle_quantize_group_sparse(const float *x, long long n, long long stride, int bits,
+                                      int k, float *scale, float *zero, uint16_t *codes,
+                                      long long *out_idx, float *out_val);
+
 /* x rounded to the nearest IEEE binary16 value (ties to even), as a float. */
 float kivi_oracle_round_half(float x);
 

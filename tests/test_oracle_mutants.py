@@ -58,6 +58,14 @@ MUTANTS = [
     ("half_ties_away", "r = nearbyint(a / q) * q;", "r = round(a / q) * q;"),
     ("half_no_subnormal_quantum", "if (e < -24) e = -24;", ""),
     ("half_overflow_kept", "if (r > 65504.0) r = INFINITY;", ""),
+    ("sparse_takes_smallest",
+     "if (best < 0 || fabsf(x[i * stride]) > fabsf(x[best * stride])) best = i;",
+     "if (best < 0 || fabsf(x[i * stride]) < fabsf(x[best * stride])) best = i;"),
+    ("sparse_tie_takes_last",
+     "if (best < 0 || fabsf(x[i * stride]) > fabsf(x[best * stride])) best = i;",
+     "if (best < 0 || fabsf(x[i * stride]) >= fabsf(x[best * stride])) best = i;"),
+    ("sparse_outliers_kept_in_range", "    if (!is_out[i]) rest[m++] = x[i * stride];",
+     "    rest[m++] = x[i * stride];"),
 ]
 
 

@@ -36,6 +36,7 @@ QROWS = [r for r in _golden() if r[0] == "Q"]
 PROWS = [r for r in _golden() if r[0] == "P"]
 MROWS = [r for r in _golden() if r[0] == "M"]
 HROWS = [r for r in _golden() if r[0] == "H"]
+SROWS = [r for r in _golden() if r[0] == "S"]
 
 
 @pytest.mark.parametrize("row", QROWS, ids=[f"{r[1]}b:{r[2]}" for r in QROWS])
@@ -202,3 +203,80 @@ def test_sixteen_bit_codes_track_the_input():
     s, z, c = oracle.quantize_group(x, 16)
     xh = np.array([oracle.dequant(ci, s, z) for ci in c])
     assert np.max(np.abs(xh - x)) <= (x.max() - x.min()) / 65535
+
+
+# ---- dense-and-sparse variant (KVQuant, codewithpapers.app page, abstract
+# item (iv): outliers isolated per vector so they do not skew its range).
+# Reading: per group, the k largest magnitudes (lower index first among
+# equals) kept exactly with dense code 0, Q over the others in order.
+
+@pytest.mark.parametrize("row", SROWS, ids=[f"{r[1]}b-k{r[2]}:{r[3]}" for r in SROWS])
+def test_sparse_golden(row):
+    _, bits, k, xs, scale_hex, zero, codes, idx, vals = row
+    x = np.array([float(v) for v in xs.split()], np.float32)
+    s, z, c, oi, ov = oracle.quantize_group_sparse(x, int(bits), int(k))
+    assert _f32_bits(s) == int(scale_hex, 16)
+    assert _f32_bits(z) == _f32_bits(np.float32(float(zero)))
+    assert c.tolist() == [int(v) for v in codes.split()]
+    assert oi.tolist() == [int(v) for v in idx.split()]
+    assert ov.tolist() == [float(v) for v in vals.split()]
+
+
+def test_sparse_golden_covers_ties_and_both_signs():
+    ks = {int(r[2]) for r in SROWS}
+    assert {0, 1, 2} <= ks and len(SROWS) >= 5
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4])
+def test_sparse_selection_and_reduction(bits):
+    """Brute force on random groups with planted outliers: the outlier set is
+    the k largest magnitudes (lower index first among equals, found by a
+    stable sort); the other codes are those of Q on the remaining entries in
+    order; k = 0 is Q exactly; reconstruction is exact on the outliers and
+    within Q's bound on the rest."""
+    rng = np.random.default_rng(11 + bits)
+    for trial in range(300):
+        n = int(rng.integers(2, 40))
+        x = rng.standard_normal(n).astype(np.float32)
+        if trial % 3 == 0:
+            x[rng.integers(0, n, 2)] *= 50
+        if trial % 5 == 0:
+            x[: n // 2] = np.round(x[: n // 2])  # equal magnitudes
+        k = int(rng.integers(0, min(n, 5)))
+        s, z, c, oi, ov = oracle.quantize_group_sparse(x, bits, k)
+        order = sorted(range(n), key=lambda i: (-abs(float(x[i])), i))
+        want = sorted(order[:k])
+        assert oi.tolist() == want
+        assert np.array_equal(ov, x[want])
+        keep = [i for i in range(n) if i not in set(want)]
+        s0, z0, c0 = oracle.quantize_group(x[keep], bits)
+        assert _f32_bits(s) == _f32_bits(s0) and _f32_bits(z) == _f32_bits(z0)
+        assert c[keep].tolist() == c0.tolist() and all(c[i] == 0 for i in want)
+        if k == 0:
+            s1, z1, c1 = oracle.quantize_group(x, bits)
+            assert _f32_bits(s) == _f32_bits(s1) and c.tolist() == c1.tolist()
+        # reconstruction: outliers exact, the rest within the bound over their range
+        xr = x[keep].astype(np.float64)
+        xh = np.array([oracle.dequant(int(c[i]), s, z) for i in keep])
+        L = 2 ** bits - 1
+        bound = s / 2 + 2 ** bits * np.spacing(np.float32(s)) + np.spacing(np.float32(np.max(np.abs(xr))))
+        assert np.all(np.abs(xh - xr) <= bound + 1e-12)
+        assert np.all(c <= L)
+
+
+def test_sparse_isolation_narrows_the_error_of_a_skewed_group():
+    """One planted outlier: isolating it shrinks the step by the outlier's
+    share of the range, and the other entries' error to within half the new
+    step (with it, they all fall on code 0, off by their own spread)."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(32).astype(np.float32)
+    x[7] = 200.0
+    s0, z0, c0 = oracle.quantize_group(x, 2)
+    s1, z1, c1, oi, ov = oracle.quantize_group_sparse(x, 2, 1)
+    assert oi.tolist() == [7] and ov.tolist() == [200.0]
+    rest = [i for i in range(32) if i != 7]
+    e0 = max(abs(oracle.dequant(int(c0[i]), s0, z0) - float(x[i])) for i in rest)
+    e1 = max(abs(oracle.dequant(int(c1[i]), s1, z1) - float(x[i])) for i in rest)
+    assert s1 < s0 / 30
+    assert e1 <= s1 / 2 * (1 + 1e-6)
+    assert all(c0[i] == 0 for i in rest) and e1 < e0 / 5
