@@ -50,6 +50,9 @@ class Unit(ctypes.Structure):
         ("v_codes", ctypes.c_void_p), ("v_scale", ctypes.c_void_p), ("v_zero", ctypes.c_void_p),
         ("k_res", ctypes.c_void_p), ("v_res", ctypes.c_void_p),
         ("n_q", ctypes.c_longlong), ("r", ctypes.c_int), ("meta_f16", ctypes.c_int),
+        ("k_out", ctypes.c_int), ("v_out", ctypes.c_int),
+        ("k_out_idx", ctypes.c_void_p), ("k_out_val", ctypes.c_void_p),
+        ("v_out_idx", ctypes.c_void_p), ("v_out_val", ctypes.c_void_p),
     ]
 
 
@@ -159,8 +162,12 @@ class OracleCache:
     empty), so that full-size shapes can be checked on sampled units.
     """
 
-    def __init__(self, B, Hkv, D, bits, G, Gv, R, capacity, units=None, meta_f16=False):
+    def __init__(self, B, Hkv, D, bits, G, Gv, R, capacity, units=None, meta_f16=False,
+                 outliers=(0, 0)):
+        """outliers = (k_out, v_out): the dense-and-sparse variant keeps that
+        many largest magnitudes of every key / value group exactly."""
         self.meta_f16 = bool(meta_f16)
+        self.k_out, self.v_out = (int(outliers[0]), int(outliers[1]))
         self.B, self.Hkv, self.D, self.bits = B, Hkv, D, bits
         self.G, self.Gv, self.R, self.capacity = G, Gv, R, capacity
         E = 32 // bits
@@ -179,15 +186,22 @@ class OracleCache:
         self.v_zero = np.zeros((n, Tq, D // Gv), np.float32)
         self.k_res = np.zeros((n, R, D), np.float32)
         self.v_res = np.zeros((n, R, D), np.float32)
+        ko, vo = max(self.k_out, 1), max(self.v_out, 1)
+        self.k_out_idx = np.zeros((n, Tq // G, D, ko), np.int32)
+        self.k_out_val = np.zeros((n, Tq // G, D, ko), np.float32)
+        self.v_out_idx = np.zeros((n, Tq, D // Gv, vo), np.int32)
+        self.v_out_val = np.zeros((n, Tq, D // Gv, vo), np.float32)
         self._u = [self._make_unit(i) for i in range(n)]
 
     def _make_unit(self, i):
         u = Unit()
         u.D, u.bits, u.G, u.Gv, u.R, u.Tq = self.D, self.bits, self.G, self.Gv, self.R, self.Tq
-        for name in ("k_codes", "k_scale", "k_zero", "v_codes", "v_scale", "v_zero", "k_res", "v_res"):
+        for name in ("k_codes", "k_scale", "k_zero", "v_codes", "v_scale", "v_zero", "k_res", "v_res",
+                     "k_out_idx", "k_out_val", "v_out_idx", "v_out_val"):
             setattr(u, name, getattr(self, name)[i].ctypes.data)
         u.n_q, u.r = 0, 0
         u.meta_f16 = int(self.meta_f16)
+        u.k_out, u.v_out = self.k_out, self.v_out
         return u
 
     def unit(self, b, h) -> Unit:

@@ -218,6 +218,15 @@ int kivi_oracle_check_unit(const kivi_oracle_unit *u) {
                     !u->v_codes || !u->v_scale || !u->v_zero))
     return KIVI_ORACLE_ERR_ARG;
   if (!u->k_res || !u->v_res) return KIVI_ORACLE_ERR_ARG;
+  /* dense-and-sparse: fewer outliers than group entries (and at most 64),
+   * binary32 metadata, the lists present */
+  if (u->k_out < 0 || u->k_out >= u->G || u->k_out > 64 || u->v_out < 0 || u->v_out >= u->Gv ||
+      u->v_out > 64)
+    return KIVI_ORACLE_ERR_ARG;
+  if ((u->k_out > 0 || u->v_out > 0) && u->meta_f16) return KIVI_ORACLE_ERR_ARG;
+  if (u->Tq > 0 && ((u->k_out > 0 && (!u->k_out_idx || !u->k_out_val)) ||
+                    (u->v_out > 0 && (!u->v_out_idx || !u->v_out_val))))
+    return KIVI_ORACLE_ERR_ARG;
   return KIVI_ORACLE_OK;
 }
 
@@ -247,22 +256,44 @@ static int quantize_block(kivi_oracle_unit *u, const float *K, const float *V,
     return KIVI_ORACLE_ERR_NOMEM;
   }
 
+  long long oi[64];
+  float ov[64];
+  int m;
   /* keys: one group per (key group g, channel d) over G tokens */
   for (g = 0; g < n / G; ++g) {
     for (d = 0; d < D; ++d) {
       long long gq = (t0 / G) + g;
-      kivi_oracle_quantize_group_meta(&K[(g * G) * D + d], G, D, bits, u->meta_f16,
-                                      &u->k_scale[gq * D + d],
-                                      &u->k_zero[gq * D + d], tmp);
+      if (u->k_out > 0) {
+        kivi_oracle_quantize_group_sparse(&K[(g * G) * D + d], G, D, bits, u->k_out,
+                                          &u->k_scale[gq * D + d], &u->k_zero[gq * D + d], tmp,
+                                          oi, ov);
+        for (m = 0; m < u->k_out; ++m) {
+          u->k_out_idx[(gq * D + d) * u->k_out + m] = (int32_t)oi[m];
+          u->k_out_val[(gq * D + d) * u->k_out + m] = ov[m];
+        }
+      } else {
+        kivi_oracle_quantize_group_meta(&K[(g * G) * D + d], G, D, bits, u->meta_f16,
+                                        &u->k_scale[gq * D + d],
+                                        &u->k_zero[gq * D + d], tmp);
+      }
       for (i = 0; i < G; ++i) ck[(g * G + i) * D + d] = tmp[i];
     }
   }
   /* values: one group per (token t, value group j) over Gv channels */
   for (t = 0; t < n; ++t) {
     for (j = 0; j < NJ; ++j) {
-      kivi_oracle_quantize_group_meta(&V[t * D + j * Gv], Gv, 1, bits, u->meta_f16,
-                                      &u->v_scale[(t0 + t) * NJ + j],
-                                      &u->v_zero[(t0 + t) * NJ + j], tmp);
+      const long long mo = (t0 + t) * NJ + j;
+      if (u->v_out > 0) {
+        kivi_oracle_quantize_group_sparse(&V[t * D + j * Gv], Gv, 1, bits, u->v_out,
+                                          &u->v_scale[mo], &u->v_zero[mo], tmp, oi, ov);
+        for (m = 0; m < u->v_out; ++m) {
+          u->v_out_idx[mo * u->v_out + m] = (int32_t)oi[m];
+          u->v_out_val[mo * u->v_out + m] = ov[m];
+        }
+      } else {
+        kivi_oracle_quantize_group_meta(&V[t * D + j * Gv], Gv, 1, bits, u->meta_f16,
+                                        &u->v_scale[mo], &u->v_zero[mo], tmp);
+      }
       for (i = 0; i < Gv; ++i) cv[t * D + j * Gv + i] = tmp[i];
     }
   }
@@ -351,6 +382,15 @@ int kivi_oracle_dequant_keys(const kivi_oracle_unit *u, double *out) {
       out[t * D + d] = kivi_oracle_dequant(c, u->k_scale[g * D + d], u->k_zero[g * D + d]);
     }
   }
+  /* dense-and-sparse: the kept outliers replace their dense values */
+  for (t = 0; u->k_out > 0 && t < u->n_q / u->G; ++t) {
+    int m;
+    for (d = 0; d < D; ++d)
+      for (m = 0; m < u->k_out; ++m) {
+        const long long e = (t * D + d) * u->k_out + m;
+        out[(t * u->G + u->k_out_idx[e]) * D + d] = (double)u->k_out_val[e];
+      }
+  }
   for (t = 0; t < u->r; ++t)
     for (d = 0; d < D; ++d) out[(u->n_q + t) * D + d] = (double)u->k_res[t * D + d];
   return KIVI_ORACLE_OK;
@@ -371,6 +411,16 @@ int kivi_oracle_dequant_values(const kivi_oracle_unit *u, double *out) {
       int j = d / u->Gv;
       out[t * D + d] = kivi_oracle_dequant(c, u->v_scale[t * NJ + j], u->v_zero[t * NJ + j]);
     }
+  }
+  /* dense-and-sparse: the kept outliers replace their dense values */
+  for (t = 0; u->v_out > 0 && t < u->n_q; ++t) {
+    const int NJ = D / u->Gv;
+    int j, m;
+    for (j = 0; j < NJ; ++j)
+      for (m = 0; m < u->v_out; ++m) {
+        const long long e = (t * NJ + j) * u->v_out + m;
+        out[t * D + j * u->Gv + u->v_out_idx[e]] = (double)u->v_out_val[e];
+      }
   }
   for (t = 0; t < u->r; ++t)
     for (d = 0; d < D; ++d) out[(u->n_q + t) * D + d] = (double)u->v_res[t * D + d];

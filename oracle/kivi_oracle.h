@@ -54,6 +54,12 @@ enum {
  *   v_zero  [Tq][D/Gv]  channels)
  *   k_res   [R][D]      residual keys, full precision (fp32 values)
  *   v_res   [R][D]      residual values
+ * Dense-and-sparse variant (k_out / v_out > 0, binary32 metadata only): every
+ * key group keeps its k_out largest magnitudes exactly and every value group
+ * its v_out largest (kivi_oracle_quantize_group_sparse), listed in
+ *   k_out_idx, k_out_val [Tq/G][D][k_out]   token within the group, value
+ *   v_out_idx, v_out_val [Tq][D/Gv][v_out]  channel within the group, value
+ * in ascending index order; their dense codes are 0.
  */
 typedef struct {
   int D;
@@ -73,6 +79,12 @@ typedef struct {
   long long n_q; /* tokens held in the quantized store */
   int r;         /* tokens held in the residual window */
   int meta_f16;  /* 1: scales and zeros stored in binary16 (format variant) */
+  int k_out;     /* outliers kept per key group (dense-and-sparse variant), 0: none */
+  int v_out;     /* outliers kept per value group */
+  int32_t *k_out_idx;
+  float *k_out_val;
+  int32_t *v_out_idx;
+  float *v_out_val;
 } kivi_oracle_unit;
 
 /* Q: quantize one group of n values x[0], x[stride], ..., x[(n-1)*stride]. */

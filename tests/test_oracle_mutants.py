@@ -17,7 +17,7 @@ import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PIN_FILES = ["tests/test_oracle_quantize.py", "tests/test_oracle_cache.py",
-             "tests/test_oracle_attention.py"]
+             "tests/test_oracle_attention.py", "tests/test_oracle_sparse_cache.py"]
 
 # (name, exact text in kivi_oracle.c, replacement)
 MUTANTS = [
@@ -66,6 +66,11 @@ MUTANTS = [
      "if (best < 0 || fabsf(x[i * stride]) >= fabsf(x[best * stride])) best = i;"),
     ("sparse_outliers_kept_in_range", "    if (!is_out[i]) rest[m++] = x[i * stride];",
      "    rest[m++] = x[i * stride];"),
+    ("sparse_key_outliers_not_restored",
+     "        out[(t * u->G + u->k_out_idx[e]) * D + d] = (double)u->k_out_val[e];", ""),
+    ("sparse_value_outlier_group_offset_dropped",
+     "        out[t * D + j * u->Gv + u->v_out_idx[e]] = (double)u->v_out_val[e];",
+     "        out[t * D + u->v_out_idx[e]] = (double)u->v_out_val[e];"),
 ]
 
 
