@@ -69,6 +69,8 @@ def lib():
             L.kivi_oracle_quantize_group.argtypes = [vp, ll, ll, ci, vp, vp, vp]
             L.kivi_oracle_quantize_group_meta.argtypes = [vp, ll, ll, ci, ci, vp, vp, vp]
             L.kivi_oracle_quantize_group_sparse.argtypes = [vp, ll, ll, ci, ci, vp, vp, vp, vp, vp]
+            L.kivi_oracle_pack_planes.argtypes = [vp, vp]
+            L.kivi_oracle_pack_planes.restype = None
             L.kivi_oracle_round_half.argtypes = [ctypes.c_float]
             L.kivi_oracle_round_half.restype = ctypes.c_float
             L.kivi_oracle_pack_word.argtypes = [vp, ci]
@@ -130,6 +132,15 @@ def quantize_group_sparse(x, bits: int, k: int):
     return s.value, z.value, codes, idx[:k], val[:k]
 
 
+def pack_planes(codes):
+    """32 codes (3-bit) as three bit-plane words."""
+    c = np.ascontiguousarray(codes, dtype=np.uint16)
+    assert c.size == 32
+    w = np.zeros(3, np.uint32)
+    lib().kivi_oracle_pack_planes(_ptr(c), _ptr(w))
+    return [int(x) for x in w]
+
+
 def round_half(x: float) -> float:
     """x rounded to the nearest binary16 value (ties to even)."""
     return float(np.float32(lib().kivi_oracle_round_half(ctypes.c_float(float(x)))))
@@ -170,18 +181,20 @@ class OracleCache:
         self.k_out, self.v_out = (int(outliers[0]), int(outliers[1]))
         self.B, self.Hkv, self.D, self.bits = B, Hkv, D, bits
         self.G, self.Gv, self.R, self.capacity = G, Gv, R, capacity
-        E = 32 // bits
-        self.E = E
+        # codes per block and words per block (3 bits: 32 codes in three bit planes)
+        E = 32 if bits == 3 else 32 // bits
+        WB = 3 if bits == 3 else 1
+        self.E, self.WB = E, WB
         Tq = capacity - R
         self.Tq = Tq
         self.units = sorted(set(units)) if units is not None else [
             (b, h) for b in range(B) for h in range(Hkv)]
         self._slot = {u: i for i, u in enumerate(self.units)}
         n = len(self.units)
-        self.k_codes = np.zeros((n, Tq, D // E), np.uint32)
+        self.k_codes = np.zeros((n, Tq, D // E * WB), np.uint32)
         self.k_scale = np.zeros((n, Tq // G, D), np.float32)
         self.k_zero = np.zeros((n, Tq // G, D), np.float32)
-        self.v_codes = np.zeros((n, Tq // E, D), np.uint32)
+        self.v_codes = np.zeros((n, Tq // E * WB, D), np.uint32)
         self.v_scale = np.zeros((n, Tq, D // Gv), np.float32)
         self.v_zero = np.zeros((n, Tq, D // Gv), np.float32)
         self.k_res = np.zeros((n, R, D), np.float32)

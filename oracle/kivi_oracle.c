@@ -35,8 +35,14 @@
 #include <string.h>
 
 static int valid_bits(int bits) {
-  return bits == 1 || bits == 2 || bits == 4 || bits == 8 || bits == 16;
+  return bits == 1 || bits == 2 || bits == 3 || bits == 4 || bits == 8 || bits == 16;
 }
+
+/* Code blocks of the packed layout: CB codes in WB words.  Widths that
+ * divide 32 pack CB = 32/bits codes into one word; 3 bits packs CB = 32
+ * codes into three bit-plane words. */
+static int block_codes(int bits) { return bits == 3 ? 32 : 32 / bits; }
+static int block_words(int bits) { return bits == 3 ? 3 : 1; }
 
 /*
  * Q.  The pages name the quantizer only as asymmetric (a scale and an
@@ -195,9 +201,33 @@ uint32_t kivi_oracle_pack_word(const uint16_t *codes, int bits) {
   return w;
 }
 
-static uint32_t unpack_code(uint32_t word, int pos, int bits) {
-  uint32_t mask = (uint32_t)((1u << bits) - 1u);
-  return (word >> (bits * pos)) & mask;
+/*
+ * P for 3 bits (a format variant; the pages name 3-bit quantization only in
+ * KVQuant's abstract).  Reading: 3 does not divide 32, so a block of 32
+ * codes is stored as three bit planes, word b holding bit b of code i in
+ * its bit i.
+ */
+void kivi_oracle_pack_planes(const uint16_t *codes, uint32_t *words) {
+  int i, b;
+  for (b = 0; b < 3; ++b) {
+    uint32_t w = 0;
+    for (i = 0; i < 32; ++i) w |= (uint32_t)((codes[i] >> b) & 1u) << i;
+    words[b] = w;
+  }
+}
+
+static void pack_block(const uint16_t *codes, int bits, uint32_t *words) {
+  if (bits == 3)
+    kivi_oracle_pack_planes(codes, words);
+  else
+    words[0] = kivi_oracle_pack_word(codes, bits);
+}
+
+/* code at position pos of a block whose first word is w[0] */
+static uint32_t unpack_block(const uint32_t *w, int pos, int bits) {
+  if (bits == 3)
+    return ((w[0] >> pos) & 1u) | (((w[1] >> pos) & 1u) << 1) | (((w[2] >> pos) & 1u) << 2);
+  return (w[0] >> (bits * pos)) & (uint32_t)((1u << bits) - 1u);
 }
 
 /* D.  x_hat = c * s + z, evaluated in real arithmetic (binary64 holds
@@ -209,7 +239,7 @@ double kivi_oracle_dequant(uint32_t c, float scale, float zero) {
 int kivi_oracle_check_unit(const kivi_oracle_unit *u) {
   int E;
   if (!u || !valid_bits(u->bits)) return KIVI_ORACLE_ERR_ARG;
-  E = 32 / u->bits;
+  E = block_codes(u->bits);
   if (u->D <= 0 || u->G <= 0 || u->Gv <= 0 || u->R <= 0 || u->Tq < 0)
     return KIVI_ORACLE_ERR_ARG;
   if (u->D % E || u->D % u->Gv || u->R % u->G || u->R % E || u->Tq % u->R)
@@ -243,7 +273,8 @@ int kivi_oracle_check_unit(const kivi_oracle_unit *u) {
 static int quantize_block(kivi_oracle_unit *u, const float *K, const float *V,
                           long long t0, long long n) {
   const int D = u->D, bits = u->bits, G = u->G, Gv = u->Gv;
-  const int E = 32 / bits, WK = D / E, NJ = D / Gv;
+  /* E codes per block of WB words; a token's keys take WK words */
+  const int E = block_codes(bits), WB = block_words(bits), WK = (D / E) * WB, NJ = D / Gv;
   uint16_t *ck = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(n * D));
   uint16_t *cv = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(n * D));
   uint16_t *tmp = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(G > E ? G : E));
@@ -297,15 +328,20 @@ static int quantize_block(kivi_oracle_unit *u, const float *K, const float *V,
       for (i = 0; i < Gv; ++i) cv[t * D + j * Gv + i] = tmp[i];
     }
   }
-  /* pack keys along channels: word w of token t holds channels wE..wE+E-1 */
+  /* pack keys along channels: block w of token t holds channels wE..wE+E-1
+   * in words [w WB, w WB + WB) of the token's WK words */
   for (t = 0; t < n; ++t)
-    for (w = 0; w < WK; ++w)
-      u->k_codes[(t0 + t) * WK + w] = kivi_oracle_pack_word(&ck[t * D + w * E], bits);
-  /* pack values along tokens: word (tb, d) holds tokens tb*E..tb*E+E-1 */
+    for (w = 0; w < D / E; ++w)
+      pack_block(&ck[t * D + w * E], bits, &u->k_codes[(t0 + t) * WK + w * WB]);
+  /* pack values along tokens: block (tb, d) holds tokens tb*E..tb*E+E-1 of
+   * channel d in word rows tb WB .. tb WB + WB - 1 */
   for (t = 0; t < n / E; ++t) {
     for (d = 0; d < D; ++d) {
+      uint32_t words[3];
+      int b;
       for (i = 0; i < E; ++i) tmp[i] = cv[(t * E + i) * D + d];
-      u->v_codes[((t0 / E) + t) * D + d] = kivi_oracle_pack_word(tmp, bits);
+      pack_block(tmp, bits, words);
+      for (b = 0; b < WB; ++b) u->v_codes[(((t0 / E) + t) * WB + b) * D + d] = words[b];
     }
   }
   free(ck);
@@ -374,10 +410,10 @@ int kivi_oracle_dequant_keys(const kivi_oracle_unit *u, double *out) {
   if (rc) return rc;
   if (!out) return KIVI_ORACLE_ERR_ARG;
   for (t = 0; t < u->n_q; ++t) {
-    const int E = 32 / u->bits;
+    const int E = block_codes(u->bits), WB = block_words(u->bits);
     for (d = 0; d < D; ++d) {
-      uint32_t word = u->k_codes[t * (D / E) + d / E];
-      uint32_t c = unpack_code(word, d % E, u->bits);
+      const uint32_t *blk = &u->k_codes[t * (D / E) * WB + (d / E) * WB];
+      uint32_t c = unpack_block(blk, d % E, u->bits);
       long long g = t / u->G;
       out[t * D + d] = kivi_oracle_dequant(c, u->k_scale[g * D + d], u->k_zero[g * D + d]);
     }
@@ -404,10 +440,12 @@ int kivi_oracle_dequant_values(const kivi_oracle_unit *u, double *out) {
   if (rc) return rc;
   if (!out) return KIVI_ORACLE_ERR_ARG;
   for (t = 0; t < u->n_q; ++t) {
-    const int E = 32 / u->bits, NJ = D / u->Gv;
+    const int E = block_codes(u->bits), WB = block_words(u->bits), NJ = D / u->Gv;
     for (d = 0; d < D; ++d) {
-      uint32_t word = u->v_codes[(t / E) * D + d];
-      uint32_t c = unpack_code(word, (int)(t % E), u->bits);
+      uint32_t blk[3];
+      int b;
+      for (b = 0; b < WB; ++b) blk[b] = u->v_codes[((t / E) * WB + b) * D + d];
+      uint32_t c = unpack_block(blk, (int)(t % E), u->bits);
       int j = d / u->Gv;
       out[t * D + d] = kivi_oracle_dequant(c, u->v_scale[t * NJ + j], u->v_zero[t * NJ + j]);
     }

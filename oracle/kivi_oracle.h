@@ -54,6 +54,10 @@ enum {
  *   v_zero  [Tq][D/Gv]  channels)
  *   k_res   [R][D]      residual keys, full precision (fp32 values)
  *   v_res   [R][D]      residual values
+ * 3 bits (E = 32 codes per block of three bit-plane words,
+ * kivi_oracle_pack_planes): k_codes [Tq][D/32*3], block w of a token in
+ * words 3w..3w+2; v_codes [Tq/32*3][D], block tb of channel d in rows
+ * 3tb..3tb+2.
  * Dense-and-sparse variant (k_out / v_out > 0, binary32 metadata only): every
  * key group keeps its k_out largest magnitudes exactly and every value group
  * its v_out largest (kivi_oracle_quantize_group_sparse), listed in
@@ -112,6 +116,9 @@ float kivi_oracle_round_half(float x);
 
 /* P: pack 32/bits codes into one word, codes[0] in the least significant bits. */
 uint32_t kivi_oracle_pack_word(const uint16_t *codes, int bits);
+
+/* P for 3 bits: 32 codes as three bit planes, words[b] bit i = bit b of codes[i]. */
+void kivi_oracle_pack_planes(const uint16_t *codes, uint32_t *words);
 
 /* D: the dequantized value of code c with (scale, zero), in real arithmetic. */
 double kivi_oracle_dequant(uint32_t c, float scale, float zero);

@@ -84,7 +84,7 @@ def test_grouping_axes_exact_when_groups_are_constant():
     assert (Kh == K).all() and (Vh == V).all()
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 @pytest.mark.parametrize("T", [0, 1, 31, 32, 33, 63, 64, 65, 96, 127, 128, 129, 200])
 def test_prefill_equals_appends(bits, T):
     """prefill(T) and T single appends reach the same state bit for bit."""
@@ -180,5 +180,49 @@ def test_rejects_bad_dims():
     u = oracle.Unit()
     u.D, u.bits, u.G, u.Gv, u.R, u.Tq = 30, 2, 32, 32, 32, 32  # D not a multiple of E
     assert oracle.lib().kivi_oracle_check_unit(u) == oracle.ERR_ARG
-    u.D, u.bits = 32, 3
+    u.D, u.bits = 32, 5
     assert oracle.lib().kivi_oracle_check_unit(u) == oracle.ERR_ARG
+    u.D, u.bits = 48, 3  # 3-bit blocks are 32 channels
+    assert oracle.lib().kivi_oracle_check_unit(u) == oracle.ERR_ARG
+
+
+def test_three_bit_layout_by_blocks():
+    """3 bits: every 32-channel block of a token's keys is three bit-plane
+    words at 3w..3w+2, every 32-token block of a channel's values three rows
+    3tb..3tb+2 (kivi_oracle_pack_planes, pinned by the golden B lines); the
+    codes are those of the group quantizer."""
+    D, R = 64, 32
+    rng = np.random.default_rng(12)
+    K = rng.standard_normal((96, D)).astype(np.float32)
+    V = rng.standard_normal((96, D)).astype(np.float32)
+    oc = _cache(D=D, bits=3, R=R, capacity=128)
+    oc.prefill_unit(0, 0, K, V)
+    u = oc.unit(0, 0)
+    assert (u.n_q, u.r) == (64, 32)
+    kc = np.zeros((64, D), np.uint16)
+    for g in range(2):
+        for d in range(D):
+            kc[32 * g:32 * g + 32, d] = oracle.quantize_group(K[32 * g:32 * g + 32, d], 3)[2]
+    vc = np.zeros((64, D), np.uint16)
+    for t in range(64):
+        for j in range(2):
+            vc[t, 32 * j:32 * j + 32] = oracle.quantize_group(V[t, 32 * j:32 * j + 32], 3)[2]
+    for t in range(64):
+        for w in range(D // 32):
+            assert oc.k_codes[0, t, 3 * w:3 * w + 3].tolist() == oracle.pack_planes(kc[t, 32 * w:32 * w + 32])
+    for tb in range(2):
+        for d in range(D):
+            assert oc.v_codes[0, 3 * tb:3 * tb + 3, d].tolist() == oracle.pack_planes(vc[32 * tb:32 * tb + 32, d])
+    # reconstruction is c s + z from those codes
+    Kh, Vh = oc.dequant_unit(0, 0)
+    s = np.repeat(oc.k_scale[0, :2], 32, 0).astype(np.float64)
+    z = np.repeat(oc.k_zero[0, :2], 32, 0).astype(np.float64)
+    assert np.array_equal(Kh[:64], kc * s + z)
+    # attention at 3 bits is attention over that reconstruction
+    import torch
+    q = rng.standard_normal((2, D)).astype(np.float32)
+    out = oc.decode_unit(0, 0, q, 0.125)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q.astype(np.float64))[None, None], torch.from_numpy(Kh)[None, None],
+        torch.from_numpy(Vh)[None, None], scale=0.125)[0, 0].numpy()
+    assert np.allclose(out, ref, rtol=0, atol=1e-12)

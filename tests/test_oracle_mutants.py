@@ -43,8 +43,8 @@ MUTANTS = [
      "rc = quantize_block(u, u->k_res, u->v_res, 0, u->R);"),
     ("dequant_sign", "return (double)c * (double)scale + (double)zero;",
      "return (double)c * (double)scale - (double)zero;"),
-    ("value_unpack_index", "uint32_t c = unpack_code(word, (int)(t % E), u->bits);",
-     "uint32_t c = unpack_code(word, (int)(d % E), u->bits);"),
+    ("value_unpack_index", "uint32_t c = unpack_block(blk, (int)(t % E), u->bits);",
+     "uint32_t c = unpack_block(blk, (int)(d % E), u->bits);"),
     ("residual_key_index", "out[(u->n_q + t) * D + d] = (double)u->k_res[t * D + d];",
      "out[(u->n_q + t) * D + d] = (double)u->k_res[d];"),
     ("scores_use_values", "for (d = 0; d < u->D; ++d) acc += (double)qh[d] * Kh[t * u->D + d];",
@@ -58,6 +58,11 @@ MUTANTS = [
     ("half_ties_away", "r = nearbyint(a / q) * q;", "r = round(a / q) * q;"),
     ("half_no_subnormal_quantum", "if (e < -24) e = -24;", ""),
     ("half_overflow_kept", "if (r > 65504.0) r = INFINITY;", ""),
+    ("planes_bit_order_swapped", "    for (i = 0; i < 32; ++i) w |= (uint32_t)((codes[i] >> b) & 1u) << i;",
+     "    for (i = 0; i < 32; ++i) w |= (uint32_t)((codes[i] >> (2 - b)) & 1u) << i;"),
+    ("planes_unpack_plane_dropped",
+     "    return ((w[0] >> pos) & 1u) | (((w[1] >> pos) & 1u) << 1) | (((w[2] >> pos) & 1u) << 2);",
+     "    return ((w[0] >> pos) & 1u) | (((w[1] >> pos) & 1u) << 1);"),
     ("sparse_takes_smallest",
      "if (best < 0 || fabsf(x[i * stride]) > fabsf(x[best * stride])) best = i;",
      "if (best < 0 || fabsf(x[i * stride]) < fabsf(x[best * stride])) best = i;"),

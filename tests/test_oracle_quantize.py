@@ -37,6 +37,7 @@ PROWS = [r for r in _golden() if r[0] == "P"]
 MROWS = [r for r in _golden() if r[0] == "M"]
 HROWS = [r for r in _golden() if r[0] == "H"]
 SROWS = [r for r in _golden() if r[0] == "S"]
+BROWS = [r for r in _golden() if r[0] == "B"]
 
 
 @pytest.mark.parametrize("row", QROWS, ids=[f"{r[1]}b:{r[2]}" for r in QROWS])
@@ -117,8 +118,15 @@ def test_binary16_metadata_invariants(bits):
 
 
 def test_golden_file_covers_every_width():
-    assert {int(r[1]) for r in QROWS} >= {1, 2, 4}
+    assert {int(r[1]) for r in QROWS} >= {1, 2, 3, 4}
     assert {int(r[1]) for r in PROWS} == {1, 2, 4, 8, 16}
+    assert len(BROWS) >= 3
+
+
+@pytest.mark.parametrize("row", BROWS, ids=[r[2] for r in BROWS])
+def test_pack_planes_golden(row):
+    _, codes, words = row
+    assert oracle.pack_planes([int(v) for v in codes.split()]) == [int(w, 16) for w in words.split()]
 
 
 def test_dequant_closed_form():
@@ -151,7 +159,7 @@ def _groups(rng, n_groups, size):
     return out
 
 
-@pytest.mark.parametrize("bits", [1, 2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 8])
 def test_invariants(bits):
     """Code range; min -> code 0 reconstructing exactly; max -> top code;
     reconstruction error within half a step plus the rounding slack of s,
