@@ -289,3 +289,27 @@ def test_paged_cache_init_and_refusals():
     # a contiguous cache carries no block table
     c2 = _fake_cache()
     assert (c2.block_table, c2.pages_per_seq, c2.num_pages) == (None, 0, 0)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 4])
+def test_paged_pool_with_binary16_metadata(bits):
+    B, H, D, R, P = 2, 3, 64, 32, 9
+    out = (ctypes.c_size_t * 8)()
+    d32 = _dims(B=B, Hkv=H, D=D, bits=bits, R=R, capacity=4 * R)
+    d16 = _dims(B=B, Hkv=H, D=D, bits=bits, R=R, capacity=4 * R, meta=kivi.KIVI_META_F16)
+    L = kivi.lib()
+    assert L.kivi_paged_buffer_sizes(ctypes.byref(d32), P, ctypes.byref(out)) == 0
+    s32 = list(out)
+    assert L.kivi_paged_buffer_sizes(ctypes.byref(d16), P, ctypes.byref(out)) == 0
+    s16 = list(out)
+    E = 32 // bits
+    assert s16[0] == s32[0] == P * H * R * (D // E) * 4
+    for i in (1, 2, 4, 5):
+        assert 2 * s16[i] == s32[i]
+    assert s16[6] == s32[6] == B * H * R * D * 2
+
+
+def test_code_widths_the_library_builds():
+    # 1, 2 and 4 bits run on the GPU; 3 bits exists in the oracle only
+    for bits, rc in ((1, 0), (2, 0), (4, 0), (3, ERR_UNSUPPORTED), (8, ERR_UNSUPPORTED)):
+        assert _sizes(_dims(bits=bits))[0] == rc, bits
