@@ -20,23 +20,13 @@
 // the binary32 scale and minimum are rounded to binary16 (nearest, ties to
 // even) and the codes are chosen against the rounded pair, so that the
 // stored scale and zero reproduce them as closely as the code grid allows.
+#include "kivi_codes.cuh"
 #include "kivi_internal.cuh"
 
 namespace kivi {
 namespace {
 
-// round_half_even(fl(d / s)) clamped to [0, L], without a division for most
-// elements: q = fl(d * fl(1/s)) differs from fl(d / s) by at most
-// (d/s)(2^-23 + 2^-24 + 2^-48) (two roundings against one), below 3e-6 for
-// d/s <= 16; so when q is more than 4e-6 from the nearest half-integer both
-// round to the same integer and neither is a tie.  Otherwise (and for inf or
-// NaN q) the quotient is taken by the IEEE division.  rs = __frcp_rn(s).
-__device__ __forceinline__ int code_of(float d, float s, float rs, int L) {
-  const float q = __fmul_rn(d, rs);
-  const float f = q - floorf(q);
-  const int c = fabsf(f - 0.5f) > 4e-6f ? __float2int_rn(q) : __float2int_rn(__fdiv_rn(d, s));
-  return min(max(c, 0), L);
-}
+// (code_of and recip_rn: kivi_codes.cuh)
 
 // Quantize one tile of kTile tokens (= one key group) of one unit.
 //   Ksrc, Vsrc: the tile's first token row; rows are D elements apart.
@@ -80,7 +70,7 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
     const long long g = t0 / kG;
     reinterpret_cast<M*>(c.k_scale)[unit * Lt::k_meta_unit(Ts) + g * D + tid] = from_f32<M>(s);
     reinterpret_cast<M*>(c.k_zero)[unit * Lt::k_meta_unit(Ts) + g * D + tid] = from_f32<M>(z);
-    const float rs = __frcp_rn(s);
+    const float rs = recip_rn(s);
 #pragma unroll
     for (int t = 0; t < kTile; ++t) {
       int code = 0;
@@ -106,7 +96,7 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
     const long long mo = unit * Lt::v_meta_unit(Ts) + (t0 + t) * NJ + j;
     reinterpret_cast<M*>(c.v_scale)[mo] = from_f32<M>(s);
     reinterpret_cast<M*>(c.v_zero)[mo] = from_f32<M>(z);
-    const float rs = __frcp_rn(s);
+    const float rs = recip_rn(s);
 #pragma unroll
     for (int i = 0; i < kGv; ++i) {
       int code = 0;
