@@ -591,10 +591,17 @@ def cpu_baseline(w: W.Workload, budget_s: float):
     steps = max(1, int(budget_s * threads / (per_unit_cpu * n_units)))
     per_step, n, scale = oracle_sample(w, n_units, steps, threads)
     full_step = per_step * scale
-    return {"value": w.B / full_step, "unit": "tokens/s", "cores": threads, "cpu_model": cpu_model(), "kind": "oracle",
+    # the same loop on one thread, over a fifth of the budget
+    steps1 = max(1, int(budget_s / 5 / (per_unit_cpu * threads)))
+    per1, n1, scale1 = oracle_sample(w, threads, steps1, 1)
+    return {"value": w.B / full_step, "unit": "tokens/s", "cores": threads, "cpu_model": cpu_model(),
+            "kind": "oracle",
             "sample": f"{steps} steps x {n} of {w.B * w.Hkv} (batch, KV head) units spread "
                       f"over the batch, append + decode, scaled to the full batch by tokens "
-                      f"held; single oracle threads fanned out over units"}
+                      f"held; single oracle threads fanned out over units",
+            "single_thread": {"value": w.B / (per1 * scale1), "unit": "tokens/s",
+                              "sample": f"{steps1} steps x {n1} units on one thread, scaled "
+                                        f"the same way"}}
 
 
 def run_reference(args, rank, world):
