@@ -9,12 +9,18 @@ packed codes and the window, then the cross-split merge), one kernel launch
 when no flush is due.  `--unfused` times kivi_append_token followed by
 kivi_decode_attention instead (two launches per step).  The ragged workload
 (per-sequence prompt lengths) times kivi_ragged_append_decode: the append
-(each sequence flushing on its own) and the decode, two launches per step.  Workload: the Llama-2-7B-shaped layer
-(B=8, 32 heads, D=128, context 4096, 2-bit, G=32, R=128) by default.
+(each sequence flushing on its own) and the decode, two launches per step.
 
-L2 hygiene: `--layers` copies of the layer cache (default 32, the model's
-depth; 4.7 GB) are visited round-robin, so each step reads a cache that is
-not L2-resident (inputs larger than the 126 MB L2).
+Headline workload: the Llama-2-13B-shaped layer (B=64, 40 heads, D=128,
+context 8192, 2-bit, G=32, R=128; 2.81 GB of codes, scales and zeros per
+decode call), the largest configuration that fits one GPU.  Beside it, under
+"workloads", the Llama-2-7B layer, the Mistral-7B GQA layer, the streaming
+workload's decode step and the 13B layer at 4 bits, each with its own rate
+and roofline (headline and roofline passes only; `--no-extras` skips them).
+
+L2 hygiene: `--layers` copies of the layer cache (default: enough for about
+4 GB, at least two) are visited round-robin, so each step reads a cache that
+is not L2-resident (inputs larger than the 126 MB L2).
 
 Output: one JSON line (rank 0).  `value` = decode tokens/s over all ranks
 (B tokens per step per rank) over K steps with nothing recorded between
@@ -58,8 +64,11 @@ def parse():
     p.add_argument("--steps", type=int, default=4096)
     p.add_argument("--warmup", type=int, default=64)
     p.add_argument("--impl", choices=["kivi", "reference"], default="kivi")
-    p.add_argument("--workload", default=W.LLAMA2_7B.name, choices=sorted(W.ALL))
-    p.add_argument("--layers", type=int, default=32)
+    p.add_argument("--workload", default=W.LLAMA2_13B_2BIT.name, choices=sorted(W.ALL))
+    p.add_argument("--layers", type=int, default=0,
+                   help="layer caches visited round-robin (0: enough for ~4 GB, at least 2)")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the other workloads reported beside the headline one")
     p.add_argument("--kernel", choices=["default", "simt"], default="default")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -78,10 +87,16 @@ def parse():
     return p.parse_args()
 
 
-def bench_workload(args) -> W.Workload:
-    """The workload named by --workload with the --meta storage; the streaming
-    workload's decode loop is the step loop itself (steps = 0 here)."""
-    w = W.ALL[args.workload]
+DEFAULT_WORKLOAD = W.LLAMA2_13B_2BIT.name
+# reported beside the headline, each with its own rate and roofline
+EXTRA_WORKLOADS = (W.LLAMA2_7B.name, W.MISTRAL_7B.name, W.STREAMING.name, W.LLAMA2_13B_4BIT.name)
+
+
+def bench_workload(args, name=None) -> W.Workload:
+    """The workload named by --workload (or `name`) with the --meta storage;
+    the streaming workload's decode loop is the step loop itself (steps = 0
+    here)."""
+    w = W.ALL[name or args.workload]
     if w.steps:
         w = w.with_(steps=0)
     if args.meta == "f16":
@@ -228,7 +243,8 @@ class ClockSampler:
 # ------------------------------------------------------------------ GPU arm
 
 def run_kivi(args, rank, world, local):
-    import bit_asymmetric_kv_quantize_b200 as kivi
+    """The headline workload with every measurement, then (unless --no-extras)
+    the other decode workloads with the headline and roofline passes only."""
     import torch.distributed as dist
     from datetime import timedelta
 
@@ -236,8 +252,39 @@ def run_kivi(args, rank, world, local):
     torch.cuda.set_device(device)
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=device)
-
     w = bench_workload(args)
+    result = measure(args, w, rank, world, device, args.steps, args.warmup,
+                     args.layers or default_layers(w), full=True)
+    if not args.no_extras and args.workload == DEFAULT_WORKLOAD and not (
+            args.bits or args.meta != "f32" or args.paged or args.unfused or args.kernel != "default"):
+        extra = {}
+        for name in EXTRA_WORKLOADS:
+            we = bench_workload(args, name)
+            r = measure(args, we, rank, world, device, min(args.steps, 1024), args.warmup,
+                        default_layers(we), full=False)
+            if rank == 0:
+                extra[we.name] = r
+        if rank == 0:
+            result["workloads"] = extra
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result, w
+
+
+def default_layers(w: W.Workload) -> int:
+    """Layer caches visited round-robin: enough that the caches together are
+    far larger than the 126 MB L2 (the 13B layer alone is 2.8 GB: two)."""
+    per_layer = algorithmic_bytes(w, w.T, 0)
+    return max(2, min(32, -(-4_000_000_000 // per_layer)))
+
+
+def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, full):
+    """Time `steps` steps of workload `w` (after `warmup`); full: also the
+    prefill and append timings, e2e and clocks (the headline workload)."""
+    import bit_asymmetric_kv_quantize_b200 as kivi
+    import torch.distributed as dist
+
     ragged = w.len_min > 0
     if args.paged:
         w = w.with_(name=f"{w.name}-paged-{args.paged}")
@@ -245,9 +292,9 @@ def run_kivi(args, rank, world, local):
         raise SystemExit("ragged workloads run the fused tensor-core step only")
     if args.paged and not ragged:
         raise SystemExit("--paged needs a ragged workload")
-    n_layers = max(1, args.layers)
-    e2e_steps = 0 if args.no_e2e else min(args.steps, 1024)
-    per_layer = -(-(args.warmup + 2 * args.steps + e2e_steps) // n_layers) + 1
+    n_layers = max(1, n_layers)
+    e2e_steps = 0 if (args.no_e2e or not full) else min(steps, 1024)
+    per_layer = -(-(warmup + 2 * steps + e2e_steps) // n_layers) + 1
     capacity = -(-(w.T + per_layer) // w.R) * w.R
     Kp, Vp = W.prompt_kv(w, device=device)
     lens = W.seq_lengths(w)
@@ -286,7 +333,7 @@ def run_kivi(args, rank, world, local):
     # append alone (host counters): 2R + 8 calls on a scratch cache of the
     # same shape, each between CUDA events, split into flush and plain steps
     append_times = None
-    if not ragged:
+    if not ragged and full:
         sc = kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, -(-(w.T + 2 * w.R + 8) // w.R) * w.R, R=w.R,
                             G=w.G, Gv=w.Gv, dtype=w.torch_dtype, device=device, meta=w.torch_meta)
         sc.prefill(Kp, Vp)
@@ -380,13 +427,13 @@ def run_kivi(args, rank, world, local):
         torch.cuda.synchronize(device)
 
     # warm-up
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i)
     barrier()
 
     # per-step events around the split kernel (created by one record each)
     evs = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         e1.record(stream)
@@ -400,8 +447,10 @@ def run_kivi(args, rank, world, local):
     n_launch[0] = 0
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         t0.record(stream)
-        for j in range(args.steps):
-            step(args.warmup + j)
+        h0 = time.perf_counter()
+        for j in range(steps):
+            step(warmup + j)
+        host_us = (time.perf_counter() - h0) * 1e6 / steps
         t1.record(stream)
         timed_launches = n_launch[0]
         torch.cuda.synchronize(device)
@@ -410,8 +459,8 @@ def run_kivi(args, rank, world, local):
     # (2) the roofline: as many further steps, CUDA events recorded by the
     # library around each decode launch (these serialize the launches)
     fills = []
-    for j in range(args.steps):
-        i = args.warmup + args.steps + j
+    for j in range(steps):
+        i = warmup + steps + j
         step(i, ev_handles[j])
         c = caches[i % n_layers]
         if ragged:
@@ -451,7 +500,7 @@ def run_kivi(args, rank, world, local):
         h2d = hs[0].numel() * hs[0].element_size()
         d2h = out.numel() * out.element_size()
         n_e2e = e2e_steps
-        base = args.warmup + 2 * args.steps
+        base = warmup + 2 * steps
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -472,15 +521,15 @@ def run_kivi(args, rank, world, local):
 
     result = None
     if rank == 0:
-        tokens_per_s = replica_throughput(world, w.B, args.steps, ms_max)
+        tokens_per_s = replica_throughput(world, w.B, steps, ms_max)
         result = {
             "metric": METRIC,
             "value": tokens_per_s,
             "unit": "tokens/s",
             "n_gpus": world,
-            "steps": args.steps,
-            "warmup": args.warmup,
-            "ms_per_step": ms_max / args.steps,
+            "steps": steps,
+            "warmup": warmup,
+            "ms_per_step": ms_max / steps,
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
@@ -505,22 +554,26 @@ def run_kivi(args, rank, world, local):
                 "kernel": "decode_split", "bound": "hbm", "achieved": achieved, "peak": peak,
                 "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": (profiled_traffic(w) if args.kernel == "default" else None),
-                "algorithmic_bytes_per_launch": bytes_total / args.steps,
-                "avg_launch_us": split_total_ms * 1e3 / args.steps,
+                "algorithmic_bytes_per_launch": bytes_total / steps,
+                "avg_launch_us": split_total_ms * 1e3 / steps,
             },
-            "context_tokens_per_s": ctx_tokens * w.Hkv / (ms_max / args.steps * 1e-3) * world,
+            "context_tokens_per_s": ctx_tokens * w.Hkv / (ms_max / steps * 1e-3) * world,
             "prefill": prefill_times,
             "append": append_times,
             "e2e": e2e,
             "gpu_launches": timed_launches,
             "clocks": clk.summary(),
         }
-    for c in caches:
-        del c
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    return result, w
+        if not full:  # an extra workload: its own rate and roofline only
+            keep = ("value", "unit", "steps", "warmup", "ms_per_step", "config", "roofline",
+                    "context_tokens_per_s", "gpu_launches", "host_us_per_step")
+            result["host_us_per_step"] = host_us
+            result = {k: result[k] for k in keep}
+        else:
+            result["host_us_per_step"] = host_us
+    del caches, states, ks, vs, qs, out, ws
+    torch.cuda.empty_cache()
+    return result
 
 
 # --------------------------------------------------------------- CPU oracle arm

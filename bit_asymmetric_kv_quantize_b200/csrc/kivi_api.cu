@@ -168,12 +168,15 @@ unsigned int next_epoch() {
   return e;
 }
 
+void touch_noalloc_scratch();
+
 // Validate, plan and launch one decode.  `ws` holds the arrival counters and
 // the partials; the split count is capped at `split_cap`.
 int decode_launch(const kivi_cache* c, const void* q, int Hq, float softmax_scale, void* out,
                   void* ws, int split_cap, int sms, void* stream, bool simt,
                   const void* new_k = nullptr, const void* new_v = nullptr, int new_slot = 0,
                   void* dev_state = nullptr, bool ragged = false, bool pending = false) {
+  touch_noalloc_scratch();
   const int gq = Hq / c->dims.Hkv;
   DecodeArgs a;
   a.ragged = ragged ? 1 : 0;
@@ -270,9 +273,16 @@ int decode_common(const kivi_cache* c, const void* q, int Hq, float softmax_scal
 }
 
 // ---- static scratch for kivi_decode_attention_noalloc ----------------------
-// One fixed array per device, reserved when the library's module is loaded.
-// Host code must not use the symbol itself as a device address: its device
-// address is looked up once per device with cudaGetSymbolAddress.
+// One fixed array per device.  It exists on a device once this file's device
+// module is loaded there; under CUDA's lazy module loading (the default) that
+// happens at the first use of the symbol, i.e. the first
+// cudaGetSymbolAddress below, which also reserves the array's 4 MiB.  So that
+// this happens early, at a point the caller controls, every call that
+// launches work (prefill, append, decode of any kind) resolves the address on
+// its device first (touch_noalloc_scratch); a caller that later reserves the
+// whole device for its own pool has the array already.  Host code must not
+// use the symbol itself as a device address: its device address is looked up
+// once per device with cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[KIVI_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 128;
@@ -291,6 +301,13 @@ int noalloc_scratch(void** out) {
   }
   *out = p;
   return KIVI_OK;
+}
+
+// Resolve the scratch on the current device if not done yet (best effort:
+// a failure here is reported by the no-allocation call itself).
+void touch_noalloc_scratch() {
+  void* p = nullptr;
+  (void)noalloc_scratch(&p);
 }
 
 }  // namespace
@@ -395,6 +412,7 @@ int kivi_quantize_prefill(kivi_cache* cache, const void* K, const void* V, long 
   const int r = (int)((T - 1) % R) + 1;
   const long long n_q = T - r;
   if (n_q / kivi::kTile + 1 > (long long)INT_MAX) return KIVI_ERR_UNSUPPORTED;
+  touch_noalloc_scratch();
   cudaError_t err = kivi::launch_prefill(view(cache), cache->dims.B * cache->dims.Hkv,
                                          cache->dims.D, cache->dims.bits, cache->dims.dtype, K,
                                          V, T, n_q, r, (cudaStream_t)stream);
@@ -412,6 +430,7 @@ int kivi_append_token(kivi_cache* cache, const void* k, const void* v, void* str
   if (cache->n_q + cache->r + 1 > cache->dims.capacity) return KIVI_ERR_CAPACITY;
   const bool flush = cache->r == cache->dims.R;
   const int slot = flush ? 0 : cache->r;
+  touch_noalloc_scratch();
   cudaError_t err = kivi::launch_append(view(cache), cache->dims.B * cache->dims.Hkv,
                                         cache->dims.D, cache->dims.bits, cache->dims.dtype, k, v,
                                         cache->n_q, slot, flush, (cudaStream_t)stream);
@@ -511,6 +530,7 @@ int kivi_ragged_prefill(kivi_cache* cache, void* state, const void* K, const voi
   if (!state || ((uintptr_t)state & 15) || !K || !V || !lens || T_max < 1) return KIVI_ERR_ARG;
   if (cache->n_q != 0 || cache->r != 0) return KIVI_ERR_STATE;
   if (T_max / kivi::kTile + 1 > (long long)INT_MAX) return KIVI_ERR_UNSUPPORTED;
+  touch_noalloc_scratch();
   cudaError_t err = kivi::launch_prefill_ragged(
       view(cache), cache->dims.B * cache->dims.Hkv, cache->dims.Hkv, cache->dims.D,
       cache->dims.bits, cache->dims.dtype, K, V, T_max, lens, (kivi::DevState*)state,

@@ -15,10 +15,15 @@ namespace kivi {
 
 // round_half_even(fl(d / s)) clamped to [0, L], without a division for most
 // elements: q = fl(d * rs) with rs = fl(1/s) differs from fl(d / s) by at
-// most (d/s)(2^-23 + 2^-24 + 2^-48) (two roundings against one), below 3e-6
-// for d/s <= 16; so when q is more than 4e-6 from the nearest half-integer
+// most |d/s|(2^-23 + 2^-24 + 2^-48) (two roundings against one), below 3e-6
+// for |d/s| <= 16; so when q is more than 4e-6 from the nearest half-integer
 // both round to the same integer and neither is a tie.  Otherwise (and for
-// inf or NaN q) the quotient is taken by the IEEE division.
+// inf or NaN q) the quotient is taken by the IEEE division.  Quotients far
+// outside [-0.5, L + 0.5] (|d/s| > 16, which binary16 scales and zeros can
+// produce, or d < 0 when the rounded zero lies above an element) are safe
+// although the bound no longer holds there: with L <= 15 both q and fl(d/s)
+// then lie beyond the same end of the range, so both clamp to the same code
+// (0 or L).
 KIVI_HD inline int code_of(float d, float s, float rs, int L) {
 #ifdef __CUDA_ARCH__
   const float q = __fmul_rn(d, rs);

@@ -48,6 +48,8 @@
 #include <cuda.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "kivi_internal.cuh"
 
 namespace kivi {
@@ -1554,6 +1556,55 @@ cudaError_t window_map(CUtensorMap* m, const void* base, long long rows, int D) 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// The two window tensor maps of a cache, encoded once and kept: they depend
+// only on the window buffers, the row count and D, which a cache never
+// changes, so steady decode calls skip the encoding.  A small table per
+// process (guarded by a mutex), replaced round-robin.
+cudaError_t window_maps(const void* k_res, const void* v_res, long long rows, int D,
+                        CUtensorMap* mk, CUtensorMap* mv) {
+  struct Entry {
+    const void* k;
+    const void* v;
+    long long rows;
+    int D;
+    int dev;
+    CUtensorMap mk, mv;
+  };
+  constexpr int kN = 32;
+  static std::mutex mu;
+  static Entry table[kN];
+  static int used = 0, next = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < used; ++i) {
+      const Entry& x = table[i];
+      if (x.k == k_res && x.v == v_res && x.rows == rows && x.D == D && x.dev == dev) {
+        *mk = x.mk;
+        *mv = x.mv;
+        return cudaSuccess;
+      }
+    }
+  }
+  e = window_map(mk, k_res, rows, D);
+  if (e == cudaSuccess) e = window_map(mv, v_res, rows, D);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  Entry& x = table[next];
+  x.k = k_res;
+  x.v = v_res;
+  x.rows = rows;
+  x.D = D;
+  x.dev = dev;
+  x.mk = *mk;
+  x.mv = *mv;
+  next = (next + 1) % kN;
+  if (used < kN) ++used;
+  return cudaSuccess;
+}
+
 template <int D, int BITS, int GQ, typename T, typename MT, bool RAG>
 cudaError_t tc_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
                  int* ctas_per_sm) {
@@ -1568,8 +1619,7 @@ cudaError_t tc_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_
   if (sizeof(T) == 2 && a.r > 0) {
     const long long rows = (long long)a.units * a.c.R;
     if (rows >= (1LL << 31)) return cudaErrorInvalidValue;  // 32-bit box coordinates
-    e = window_map(&tmK, a.c.k_res, rows, D);
-    if (e == cudaSuccess) e = window_map(&tmV, a.c.v_res, rows, D);
+    e = window_maps(a.c.k_res, a.c.v_res, rows, D, &tmK, &tmV);
     if (e != cudaSuccess) return e;
   }
   if (e0) cudaEventRecord(e0, s);

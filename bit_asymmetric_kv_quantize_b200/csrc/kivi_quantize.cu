@@ -12,9 +12,14 @@
 //
 // Bit-exactness: every group is reduced by one thread in element order with
 // strict compares (first occurrence kept among equal values, which fixes the
-// sign of a zero minimum), and the scale and quotients use the IEEE
-// round-to-nearest intrinsics __fsub_rn / __fdiv_rn and __float2int_rn
-// (half to even).  No reciprocal, no contraction.
+// sign of a zero minimum); the scale uses the IEEE round-to-nearest
+// intrinsics __fsub_rn / __fdiv_rn, and each code comes from code_of
+// (kivi_codes.cuh): the product fl(d * fl(1/s)) decides the code when it lies
+// more than 4e-6 from a half-integer, else the IEEE division __fdiv_rn does,
+// rounded half to even (__float2int_rn) and clamped.  That equals
+// clamp(round_half_even(fl(d / s)), 0, L) for every input (host build of the
+// rule checked against true division in tests/test_code_rule.py).  No
+// contraction.
 //
 // Format variant with binary16 scales and zeros (M = __half, fp16 caches):
 // the binary32 scale and minimum are rounded to binary16 (nearest, ties to

@@ -377,9 +377,14 @@ KIVI_API int kivi_decode_num_splits(const kivi_cache *cache, int Hq);
  * already reserved all device memory for its own pool, or a latency-bound
  * loop that must not call cudaMalloc because it can synchronize the device.
  *   - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
- *     library call.  The first call on a device looks up the scratch
- *     array's device address (cudaGetSymbolAddress) with that device
- *     current and keeps it; make that first call before any stream capture.
+ *     library call.  The scratch array's device address is looked up
+ *     (cudaGetSymbolAddress) once per device, with that device current, by
+ *     the first call on that device that launches work: a prefill, an append
+ *     or a decode of any kind, this one included.  Under CUDA's lazy module
+ *     loading (the default) that first lookup is also when the array's 4 MiB
+ *     is reserved on the device.  So make one such call on each device
+ *     (filling a cache is enough) before reserving the rest of the device
+ *     for a pool of your own, and before any stream capture.
  *   - The split count is capped so that B * Hq * splits * (D + 2) * 4 bytes
  *     fit; if even one split does not fit, the call returns
  *     KIVI_ERR_SCRATCH_LIMIT and launches nothing.

@@ -110,3 +110,30 @@ def test_tiny_and_huge_scales(rule_lib):
                     d = (s.astype(np.float64) * (k + frac)).astype(np.float32)
                 check(rule_lib, d, s, 3)
         check(rule_lib, np.zeros_like(s), s, 3)
+
+
+@pytest.mark.parametrize("L", [1, 3, 15])
+def test_quotients_far_outside_the_code_range(rule_lib, L):
+    """Quotients well above L + 1/2 (up to 1e6) and negative numerators (the
+    binary16-metadata variant's rounded zero can lie above an element): both
+    paths clamp, to L and to 0."""
+    rng = np.random.default_rng(300 + L)
+    n = 400_000
+    s = (10.0 ** rng.uniform(-20, 20, n)).astype(np.float32)
+    big = rng.uniform(L + 0.5, 1e6, n)
+    d = (s.astype(np.float64) * big).astype(np.float32)
+    ok = np.isfinite(d)
+    check(rule_lib, d[ok], s[ok], L)
+    neg = -rng.uniform(0, 1e6, n)
+    d = (s.astype(np.float64) * neg).astype(np.float32)
+    ok = np.isfinite(d)
+    check(rule_lib, d[ok], s[ok], L)
+    # negative quotients next to -1/2 (within 40 ulps on both sides)
+    s = (10.0 ** rng.uniform(-20, 20, 5000)).astype(np.float32)
+    d = (s.astype(np.float64) * -0.5).astype(np.float32)
+    for i in range(d.size):
+        x = d[i]
+        for _ in range(int(rng.integers(0, 41))):
+            x = np.nextafter(x, np.float32(-np.inf if i % 2 else 0))
+        d[i] = x
+    check(rule_lib, d, s, L)

@@ -180,3 +180,29 @@ def test_paged_tile_map(plan_lib):
     assert tile(4, tpp) is None                # page id 11 outside a pool of 10
     assert tile(5, 3 * tpp + 1) == (3 * Hkv + 2, 1)
     assert tile(3, 4 * tpp) is None            # past the table
+
+
+@pytest.mark.parametrize("f16", [0, 1])
+@pytest.mark.parametrize("seg_cap", [1, 2])
+def test_uniform_plan_with_one_or_two_partial_slots(plan_lib, f16, seg_cap):
+    """The smallest slot counts (the no-allocation call caps the slots to what
+    its fixed scratch holds, down to one): with one slot every unit is exactly
+    one CTA's range; with two, no unit meets more than two CTAs."""
+    rng = random.Random(7 + seg_cap)
+    out = (ctypes.c_longlong * 4)()
+    for _ in range(2000):
+        R = rng.choice([32, 128])
+        n_q = R * rng.randint(0, 300)
+        r = rng.randint(0 if n_q == 0 else 1, R)
+        units = rng.randint(1, 8000)
+        P = rng.choice([148, 296, 444])
+        plan_lib.t_plan_stream(units, n_q, r, f16, P, seg_cap, out)
+        n_cta, W, max_seg, ww = list(out)
+        up = plan_lib.t_unit_work(n_q, r, f16)
+        assert n_cta * W >= units * up and (n_cta - 1) * W < units * up
+        assert max_seg <= seg_cap
+        if seg_cap == 1:
+            assert W == up and n_cta == units and max_seg == 1
+        for u in {0, 1, units // 3, units // 2, units - 1}:
+            if u < units:
+                assert segments(u * up, n_q // 32, W) <= max_seg

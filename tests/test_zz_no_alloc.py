@@ -7,7 +7,10 @@ the device).  This entry point writes its cross-split partials to a fixed
 4 MiB static device array instead of a caller workspace.  The test calls it
 through the C ABI twice in a row and checks each result against the regular
 entry point (kivi_decode_attention with a workspace), within the decode
-tolerance the parity tests use.  The file name makes pytest collect it last.
+tolerance the parity tests use, and against the CPU oracle on sampled units.
+Large batches make the scratch hold fewer split partials than a workspace
+would (down to one per unit), which the last cases exercise.  The file name
+makes pytest collect it last.
 """
 import ctypes
 import math
@@ -17,9 +20,11 @@ import torch
 
 import bit_asymmetric_kv_quantize_b200 as kivi
 from bit_asymmetric_kv_quantize_b200 import workloads as W
-from kivi_testlib import MAX_ABS, MEAN_ABS
+from kivi_testlib import (MAX_ABS, MEAN_ABS, assert_decode_close, oracle_append, oracle_cache,
+                          oracle_prefill, sample_units)
 
 pytestmark = pytest.mark.gpu
+SCRATCH_BYTES = 4 << 20  # KIVI_NOALLOC_SCRATCH_BYTES (include/kivi.h)
 
 
 def _noalloc(gc, q, sigma, out):
@@ -34,12 +39,24 @@ def _close(a, b):
     return float(d.max()) <= MAX_ABS and float(d.mean()) <= MEAN_ABS
 
 
-@pytest.mark.parametrize("gq,T", [(1, 4096), (4, 3000)])
-def test_noalloc_matches_workspace_decode_twice(gq, T):
-    w = W.Workload(f"noalloc-g{gq}-t{T}", B=4, Hq=8 * gq, Hkv=8, D=128, T=T, bits=2, R=128)
+# (B, Hkv, gq, T): small batches (the scratch holds as many split partials as
+# a workspace), the Llama-2-13B-shaped batch at a short context (room for 3
+# splits), and B * Hq = 6144 query heads, where one split per unit is all
+# that fits: every unit is then one CTA's range.
+CASES = [(4, 8, 1, 4096), (4, 8, 4, 3000), (64, 40, 1, 300), (128, 48, 1, 300)]
+
+
+@pytest.mark.parametrize("B,Hkv,gq,T", CASES)
+def test_noalloc_matches_workspace_decode_twice(B, Hkv, gq, T):
+    w = W.Workload(f"noalloc-b{B}h{Hkv}-g{gq}-t{T}", B=B, Hq=Hkv * gq, Hkv=Hkv, D=128, T=T, bits=2,
+                   R=128)
+    per_split = B * w.Hq * (w.D + 2) * 4
     K, V = W.prompt_kv(w, device="cuda")
     gc = kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, w.capacity + 128, R=w.R, dtype=w.torch_dtype)
     gc.prefill(K, V)
+    units = sample_units(w, 24, seed=B)
+    oc = oracle_cache(w, units=units, capacity=w.capacity + 128)
+    oracle_prefill(oc, K, V)
     sigma = 1.0 / math.sqrt(w.D)
     for call in range(2):  # two calls in a row; the second reuses the shared scratch
         q = W.query(w, step=call, device="cuda")
@@ -49,8 +66,12 @@ def test_noalloc_matches_workspace_decode_twice(gq, T):
         torch.cuda.synchronize()
         assert torch.isfinite(out.float()).all()
         assert _close(out, ref), f"call {call}: noalloc result differs from the workspace call"
+        assert_decode_close(out, oc, q, sigma)
         k, v = W.step_kv(w, call, device="cuda")
         gc.append(k, v)
+        oracle_append(oc, k, v)
+    if per_split * 2 > SCRATCH_BYTES:
+        assert B * Hkv * gq > 4096  # the case meant to leave room for one split only
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch():
