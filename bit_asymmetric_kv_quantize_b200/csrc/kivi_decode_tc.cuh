@@ -130,14 +130,27 @@ struct Geo {
   // a stage holds kStage code tiles, and at least one window tile
   static constexpr int CODE_STAGE_B = (O_VZ + kStage * VM_B + 1023) / 1024 * 1024;
   static constexpr int STAGE_B = CODE_STAGE_B < WTILE_B ? WTILE_B : CODE_STAGE_B;
-  static constexpr int NSTAGE = (NW == 4 && TPW == 1 && BITS == 2) ? 3 : 2;
+  static constexpr int MIN_CTAS = NW == 4 ? (TPW == 2 ? 2 : 3) : 1;
   static constexpr int NPB = GQ == 8 ? 2 : 1;  // n-tiles of 8 columns (4 heads x hi, lo)
   static constexpr int PST = TPW * kTile + 8;  // p buffer stride per head (floats)
-  // per-warp scratch (bytes): fragment blocks of 32 lanes x 2 words
-  static constexpr int QB_B = NPB * KSL * 256;        // q' B fragments (score product)
-  static constexpr int PB_B = NPB * NJ * NSL * 256;   // p' B fragments (value product)
+  // B fragment blocks: only the lanes whose column carries a head are kept
+  // (fragment column n = lane / 4; GQ heads use columns 0 .. 2 GQ - 1): NLB
+  // lanes x 2 words per block, and the swizzle XORs lane bits 2.. with
+  // (k-slice & S3M) so that it stays inside the block
+  static constexpr int NLB = GQ == 1 ? 8 : (GQ == 2 ? 16 : 32);
+  static constexpr int BLKW = 2 * NLB;           // words per block
+  static constexpr int S3M = GQ == 1 ? 1 : 3;
+  // per-warp scratch (bytes)
+  static constexpr int QB_B = NPB * KSL * BLKW * 4;       // q' B fragments (score product)
+  static constexpr int PB_B = NPB * NJ * NSL * BLKW * 4;  // p' B fragments (value product)
   static constexpr int PBUF_B = GQ * PST * 4;         // p per head and token
   static constexpr int WARP_B = TPW * (QB_B + PB_B) + PBUF_B;
+  // ring depth: three stages where they fit beside MIN_CTAS - 1 other CTAs
+  // (228 KB of shared memory per SM, 1 KB of it reserved per CTA), else two:
+  // the bytes in flight per SM bound the achieved bandwidth
+  static constexpr int REST_B = NW * WARP_B + GQ * D * 4 + NW * GQ * (D + 2) * 4 + 6 * 8 + 16;
+  static constexpr int SMEM_LIMIT = 228 * 1024 / MIN_CTAS - 1024;
+  static constexpr int NSTAGE = 3 * STAGE_B + REST_B <= SMEM_LIMIT ? 3 : 2;
   // whole CTA
   static constexpr int O_WARP = NSTAGE * STAGE_B;
   static constexpr int O_QS = O_WARP + NW * WARP_B;    // q (fp32, scaled) for the window path
@@ -147,7 +160,7 @@ struct Geo {
   static constexpr int SMEM_B = O_FLAG + 16;
   static_assert(SMEM_B <= 227 * 1024, "shared memory per CTA");
   static_assert(O_BAR % 8 == 0 && WARP_B % 16 == 0, "alignment");
-  static constexpr int MIN_CTAS = NW == 4 ? (TPW == 2 ? 2 : 3) : 1;
+  static_assert(SMEM_B <= SMEM_LIMIT, "MIN_CTAS CTAs fit one SM");
   // key operand: code pairs per lane and row, words a lane loads per row
   static constexpr int PPL = D / 8;
   static constexpr int PPW = Pairs<BITS>::PPW;
@@ -250,10 +263,20 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
   lo = h2_bits(__floats2half2_rn(a - f.x, b - f.y));
 }
 
-// Word offset of fragment slot `lane2` (= 4 n + tq) in a 64-word B block for
-// k-slice `sl`: an XOR swizzle that keeps the cooperative fragment stores
-// free of bank conflicts while each lane still reads a contiguous 8 bytes.
-__device__ __forceinline__ int frag_word(int lane2, int sl) { return 2 * (lane2 ^ (4 * (sl & 3))); }
+// Word offset of fragment slot `lane2` (= 4 n + tq) in a B block for k-slice
+// `sl`: an XOR swizzle (of lane2's column bits with sl & S3M) that spreads the
+// cooperative fragment stores over the banks while each lane still reads a
+// contiguous 8 bytes.
+template <int S3M>
+__device__ __forceinline__ int frag_word(int lane2, int sl) { return 2 * (lane2 ^ (4 * (sl & S3M))); }
+
+// x / y for non-negative x and positive y, by a 32-bit division when both fit
+// (the usual case: a few instructions instead of the 64-bit division routine).
+__device__ __forceinline__ long long div_ll(long long x, long long y) {
+  if (((unsigned long long)x | (unsigned long long)y) >> 32 == 0)
+    return (long long)((unsigned)x / (unsigned)y);
+  return x / y;
+}
 
 // ---- the units of a CTA's work range ---------------------------------------
 // A cursor over consecutive units: unit u occupies work indices
@@ -309,7 +332,7 @@ __device__ __forceinline__ UnitCur cur_first(const DecodeArgs& a, bool f16, long
                                              long long UP, long long n_qt) {
   UnitCur c;
   if constexpr (!RAG) {
-    c.u = G0 / UP;
+    c.u = div_ll(G0, UP);
     c.base = c.u * UP;
     c.n_qt = n_qt;
     c.up = UP;
@@ -397,6 +420,9 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
   constexpr int PST = G::PST;
   constexpr int TPW = G::TPW;
   constexpr int CPL = D / 32;  // window path: channels per lane
+  constexpr int BLKW = G::BLKW;  // words per B fragment block
+  constexpr int S3M = G::S3M;
+  auto fw = [](int lane2, int sl) { return frag_word<S3M>(lane2, sl); };
   constexpr float kKeyOut = (float)(1 << (24 - G::SK));
   constexpr float kValOut = (float)(1 << (24 - G::SV));
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -487,23 +513,30 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
       }
     }
   }
-  if (warp < kW) {
-    // fragment columns of absent heads stay zero
-    unsigned char* wb = smem + G::O_WARP + warp * G::WARP_B;
-    for (int i = lane; i < TPW * (G::QB_B + G::PB_B) / 4; i += 32) reinterpret_cast<uint32_t*>(wb)[i] = 0u;
-  }
   __syncthreads();
 
   if (warp == kW) {
     // ---------------- producer warp: one thread streams this CTA's stages
     const UnitCur cu0 = cur_first<RAG>(a, kF16, G0, UP, n_qt);
     if (lane == 0 && G0 < G1) {
-      long long st = 0;
+      // ring position: slot rs, its fill round's parity rph; a slot is
+      // refilled once the consumers released its previous fill
+      int rs = 0;
+      uint32_t rph = 0;
+      bool rwrap = false;
+      auto adv = [&]() {
+        if (++rs == G::NSTAGE) {
+          rs = 0;
+          rph ^= 1u;
+          rwrap = true;
+        }
+      };
       for (UnitCur cu = cu0; cu.u < a.units && cu.base < G1; cur_next<RAG>(a, kF16, cu)) {
         const long long u = cu.u, base = cu.base, n_qt_u = cu.n_qt;
         const int r_u = cu.r;
-        if (cta < base / W || cta > (base + n_qt_u) / W) continue;  // no work of u here
-        if ((base + n_qt_u) / W - base / W + 1 > a.max_seg) {  // (cannot happen: plan bound)
+        const long long f_cta = div_ll(base, W), l_cta = div_ll(base + n_qt_u, W);
+        if (cta < f_cta || cta > l_cta) continue;  // no work of u here
+        if (l_cta - f_cta + 1 > a.max_seg) {  // (cannot happen: plan bound)
           atomicExch(&flag[0], 1);
           break;
         }
@@ -524,11 +557,10 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
             pg_head = (int)(u % c.Hkv);
           }
         }
-        for (long long t0 = max(G0 - base, 0ll); t0 < t_end; t0 += kStage, ++st) {
-          const int s = (int)(st % G::NSTAGE);
-          const int n = (int)min((long long)kStage, t_end - t0);
-          if (st >= G::NSTAGE &&
-              !mbar_wait(&empty[s], (uint32_t)(((st / G::NSTAGE) - 1) & 1))) {
+        for (int t0 = (int)max(G0 - base, 0ll); t0 < (int)t_end; t0 += kStage, adv()) {
+          const int s = rs;
+          const int n = min(kStage, (int)t_end - t0);
+          if (rwrap && !mbar_wait(&empty[s], rph ^ 1u)) {
             atomicExch(&flag[0], 1);
             break;
           }
@@ -537,12 +569,12 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           mbar_expect_tx(&full[s], (uint32_t)(n * G::TILE_B));
           if (!RAG || c.bt == nullptr) {
-            bulk_copy(buf + G::O_KC, kc_u + t0 * kTile * WK, n * G::KC_B, &full[s]);
-            bulk_copy(buf + G::O_KS, ks_u + t0 * D, n * G::KM_B, &full[s]);
-            bulk_copy(buf + G::O_KZ, kz_u + t0 * D, n * G::KM_B, &full[s]);
-            bulk_copy(buf + G::O_VC, vc_u + t0 * (kTile / E) * D, n * G::VC_B, &full[s]);
-            bulk_copy(buf + G::O_VS, vs_u + t0 * kTile * NJ, n * G::VM_B, &full[s]);
-            bulk_copy(buf + G::O_VZ, vz_u + t0 * kTile * NJ, n * G::VM_B, &full[s]);
+            bulk_copy(buf + G::O_KC, kc_u + (long long)t0 * kTile * WK, n * G::KC_B, &full[s]);
+            bulk_copy(buf + G::O_KS, ks_u + (long long)t0 * D, n * G::KM_B, &full[s]);
+            bulk_copy(buf + G::O_KZ, kz_u + (long long)t0 * D, n * G::KM_B, &full[s]);
+            bulk_copy(buf + G::O_VC, vc_u + (long long)t0 * (kTile / E) * D, n * G::VC_B, &full[s]);
+            bulk_copy(buf + G::O_VS, vs_u + (long long)t0 * kTile * NJ, n * G::VM_B, &full[s]);
+            bulk_copy(buf + G::O_VZ, vz_u + (long long)t0 * kTile * NJ, n * G::VM_B, &full[s]);
           } else {
             // paged store: one run of copies per page the stage touches (the
             // single producer thread is on the critical path: one 32-bit
@@ -579,16 +611,15 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           }
         }
         if (*(volatile int*)&flag[0]) break;
-        if (r_u > 0 && cta == (base + n_qt_u) / W) {
+        if (r_u > 0 && cta == l_cta) {
           const T* kr = reinterpret_cast<const T*>(c.k_res) + u * c.R * D;
           const T* vr = reinterpret_cast<const T*>(c.v_res) + u * c.R * D;
           if constexpr (sizeof(T) == 2) {
             // this CTA owns the unit's residual window: stream it through
             // the ring, WT tokens of K and of V per stage
-            for (int w0 = 0; w0 < r_u; w0 += G::WT * G::WPS, ++st) {
-              const int s = (int)(st % G::NSTAGE);
-              if (st >= G::NSTAGE &&
-                  !mbar_wait(&empty[s], (uint32_t)(((st / G::NSTAGE) - 1) & 1))) {
+            for (int w0 = 0; w0 < r_u; w0 += G::WT * G::WPS, adv()) {
+              const int s = rs;
+              if (rwrap && !mbar_wait(&empty[s], rph ^ 1u)) {
                 atomicExch(&flag[0], 1);
                 break;
               }
@@ -621,8 +652,12 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
   } else {
     // ---------------- consumer warps
     unsigned char* wb = smem + G::O_WARP + warp * G::WARP_B;
-    uint32_t* qB = reinterpret_cast<uint32_t*>(wb);                     // [TPW][NPB][KSL][64]
-    uint32_t* pB = reinterpret_cast<uint32_t*>(wb + TPW * G::QB_B);     // [TPW][NPB][NJ][NSL][64]
+    // fragment columns of absent heads stay zero (after the CTA barrier, so
+    // that the producer starts streaming meanwhile)
+    for (int i = lane; i < TPW * (G::QB_B + G::PB_B) / 4; i += 32) reinterpret_cast<uint32_t*>(wb)[i] = 0u;
+    __syncwarp();
+    uint32_t* qB = reinterpret_cast<uint32_t*>(wb);                     // [TPW][NPB][KSL][BLKW]
+    uint32_t* pB = reinterpret_cast<uint32_t*>(wb + TPW * G::QB_B);     // [TPW][NPB][NJ][NSL][BLKW]
     __half* pBh = reinterpret_cast<__half*>(pB);
     float* pbuf = reinterpret_cast<float*>(wb + TPW * (G::QB_B + G::PB_B));  // [GQ][PST]
 
@@ -647,8 +682,8 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
       const int pidx0 = tq_o * G::PPL + 2 * slc;
       const int wd = pidx0 / G::PPW, i0 = pidx0 % G::PPW;
       cp_ch[m] = wd * E + i0;
-      cp_s3[m] = slc & 3;
-      cp_w[m] = slc * 64 + 2 * tq_o;
+      cp_s3[m] = slc & S3M;
+      cp_w[m] = slc * BLKW + 2 * tq_o;
       cp_f0[m] = __int_as_float((127 + G::SK - PR::e(i0)) << 23);
       cp_f1[m] = __int_as_float((127 + G::SK - PR::e(i0 + 1)) << 23);
     }
@@ -687,8 +722,8 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
       pt_e = 4 * (i & 1);
     }
     const float pt_f = __int_as_float((127 + G::SV - pt_e) << 23);
-    const int pt_base = pt_sl * 128 + 2 * pt_kp + pt_hf;  // halves, block (0, 0, pt_sl)
-    const int pt_s3 = pt_sl & 3;
+    const int pt_base = pt_sl * 2 * BLKW + 2 * pt_kp + pt_hf;  // halves, block (0, 0, pt_sl)
+    const int pt_s3 = pt_sl & S3M;
 
     // B-fragment column n = g of this lane carries a head (hi or lo part);
     // lanes of absent heads' columns use zeros without loading them
@@ -697,15 +732,23 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
 #pragma unroll
     for (int p = 0; p < NPB; ++p) vh[p] = tq + 4 * p < GQ;
 
-    long long st = 0;  // ring position, in step with the producer
+    // ring position, in step with the producer: slot rs, fill parity rph
+    int rs = 0;
+    uint32_t rph = 0;
+    auto adv = [&]() {
+      if (++rs == G::NSTAGE) {
+        rs = 0;
+        rph ^= 1u;
+      }
+    };
     const UnitCur cu0 = cur_first<RAG>(a, kF16, G0, UP, n_qt);
     for (UnitCur cu = cu0; G0 < G1 && cu.u < a.units && cu.base < G1; cur_next<RAG>(a, kF16, cu)) {
       const long long u = cu.u, base = cu.base, n_qt_u = cu.n_qt;
       const int r_u = cu.r;
       // CTAs f_cta..l_cta cover the unit's tiles and its window start index;
       // l_cta owns the window
-      const long long f_cta = base / W;
-      const long long l_cta = (base + n_qt_u) / W;
+      const long long f_cta = div_ll(base, W);
+      const long long l_cta = div_ll(base + n_qt_u, W);
       if (cta < f_cta || cta > l_cta) continue;
       if (l_cta - f_cta + 1 > a.max_seg) break;  // (cannot happen: plan bound; producer aborts)
       const long long b = u / a.Hkv;
@@ -752,17 +795,17 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
 #pragma unroll
         for (int j = 0; j < NJ; ++j) bv[h][j] = 0.f;
 
-      for (long long t0 = t_beg; t0 < t_end; t0 += kStage, ++st) {
+      for (int t0 = (int)t_beg; t0 < (int)t_end; t0 += kStage, adv()) {
         if (*(volatile int*)&flag[0]) break;
-        const int s = (int)(st % G::NSTAGE);
-        const bool ok = mbar_wait(&full[s], (uint32_t)((st / G::NSTAGE) & 1));
+        const int s = rs;
+        const bool ok = mbar_wait(&full[s], rph);
         if (!__all_sync(0xffffffffu, ok) || *(volatile int*)&flag[0]) {
           if (lane == 0) atomicExch(&flag[0], 1);
           break;
         }
         const unsigned char* buf = smem + s * G::STAGE_B;
-        const long long tw0 = t0 + (long long)warp * TPW;  // this warp's first tile
-        if (tw0 < t_end) {
+        const int tw0 = t0 + warp * TPW;  // this warp's first tile
+        if (tw0 < (int)t_end) {
           // this warp's TPW tiles; a tile past the end of the segment reuses
           // tile 0's data and is masked out (its scores are -inf, so p = 0)
           bool tv[TPW];
@@ -774,7 +817,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           const MT* vz[TPW];
 #pragma unroll
           for (int tt = 0; tt < TPW; ++tt) {
-            tv[tt] = tw0 + tt < t_end;
+            tv[tt] = tw0 + tt < (int)t_end;
             const int ti = warp * TPW + (tv[tt] ? tt : 0);
             kc[tt] = reinterpret_cast<const uint32_t*>(buf + G::O_KC) + ti * kTile * WK;
             ks[tt] = reinterpret_cast<const MT*>(buf + G::O_KS) + ti * D;
@@ -808,7 +851,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
                 uint2 hi, lo;
                 split2(qf[x][m][0] * s0, qf[x][m][1] * s1, hi.x, lo.x);
                 split2(qf[x][m][2] * s2, qf[x][m][3] * s3, hi.y, lo.y);
-                uint32_t* blk = qB + tt * (G::QB_B / 4) + (h >> 2) * KSL * 64 + cp_w[m];
+                uint32_t* blk = qB + tt * (G::QB_B / 4) + (h >> 2) * KSL * BLKW + cp_w[m];
                 const int nh = 2 * (h & 3);
                 *reinterpret_cast<uint2*>(blk + 8 * (nh ^ cp_s3[m])) = hi;
                 *reinterpret_cast<uint2*>(blk + 8 * ((nh + 1) ^ cp_s3[m])) = lo;
@@ -877,7 +920,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
 #pragma unroll
               for (int p = 0; p < NPB; ++p)
                 bq[p] = bcol ? *reinterpret_cast<const uint2*>(qB + tt * (G::QB_B / 4) +
-                                                               (p * KSL + sl) * 64 + frag_word(lane, sl))
+                                                               (p * KSL + sl) * BLKW + fw(lane, sl))
                              : make_uint2(0u, 0u);
 #pragma unroll
               for (int mt = 0; mt < 2; ++mt) {
@@ -975,7 +1018,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
                 const float x = phf * sv[j];
                 const __half hi = __float2half_rn(x);
                 const __half lo = __float2half_rn(x - __half2float(hi));
-                __half* blk = pBh + tt * (G::PB_B / 2) + ((h >> 2) * NJ + j) * NSL * 128;
+                __half* blk = pBh + tt * (G::PB_B / 2) + ((h >> 2) * NJ + j) * NSL * 2 * BLKW;
                 blk[o_hi] = hi;
                 blk[o_lo] = lo;
               }
@@ -1005,8 +1048,8 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
 #pragma unroll
                 for (int p = 0; p < NPB; ++p) {
                   const uint2 bb = bcol ? *reinterpret_cast<const uint2*>(
-                                              pB + tt * (G::PB_B / 4) + ((p * NJ + j) * NSL + sl) * 64 +
-                                              frag_word(lane, sl))
+                                              pB + tt * (G::PB_B / 4) + ((p * NJ + j) * NSL + sl) * BLKW +
+                                              fw(lane, sl))
                                         : make_uint2(0u, 0u);
                   mma16816(acc[p][2 * j], x0, x1, x2, x3, bb.x, bb.y);
                   mma16816(acc[p][2 * j + 1], y0, y1, y2, y3, bb.x, bb.y);
@@ -1062,7 +1105,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           uint2 bq[NPB];
 #pragma unroll
           for (int p = 0; p < NPB; ++p)
-            bq[p] = bcol ? *reinterpret_cast<const uint2*>(qB + (p * KSL + sl) * 64 + frag_word(lane, sl))
+            bq[p] = bcol ? *reinterpret_cast<const uint2*>(qB + (p * KSL + sl) * BLKW + fw(lane, sl))
                          : make_uint2(0u, 0u);
 #pragma unroll
           for (int mt = 0; mt < 2; ++mt) {
@@ -1128,10 +1171,10 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
             const float x = pbuf[h * PST + lane];
             const __half hi = __float2half_rn(x);
             const __half lo = __float2half_rn(x - __half2float(hi));
-            __half* blk = pBh + ((h >> 2) * NJ * NSL + slp) * 128 + 2 * kp + hf;
+            __half* blk = pBh + ((h >> 2) * NJ * NSL + slp) * 2 * BLKW + 2 * kp + hf;
             const int nh = 2 * (h & 3);
-            blk[2 * frag_word(4 * nh + tqk, slp)] = hi;
-            blk[2 * frag_word(4 * (nh + 1) + tqk, slp)] = lo;
+            blk[2 * fw(4 * nh + tqk, slp)] = hi;
+            blk[2 * fw(4 * (nh + 1) + tqk, slp)] = lo;
           }
         }
         __syncwarp();
@@ -1140,7 +1183,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           uint2 bb[NPB];
 #pragma unroll
           for (int p = 0; p < NPB; ++p)
-            bb[p] = bcol ? *reinterpret_cast<const uint2*>(pB + (p * NJ * NSL + sl) * 64 + frag_word(lane, sl))
+            bb[p] = bcol ? *reinterpret_cast<const uint2*>(pB + (p * NJ * NSL + sl) * BLKW + fw(lane, sl))
                          : make_uint2(0u, 0u);
           const int tok = 16 * sl + (lane & 7) + 8 * (lane >> 4);
           const int tr = tok < nt ? tok : 0;
@@ -1200,10 +1243,10 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
       if constexpr (sizeof(T) == 2) {
         if (window_owner) {
           int k = 0;
-          for (int w0 = 0; w0 < r_u; w0 += G::WT * G::WPS, ++st) {
+          for (int w0 = 0; w0 < r_u; w0 += G::WT * G::WPS, adv()) {
             if (*(volatile int*)&flag[0]) break;
-            const int s = (int)(st % G::NSTAGE);
-            const bool ok = mbar_wait(&full[s], (uint32_t)((st / G::NSTAGE) & 1));
+            const int s = rs;
+            const bool ok = mbar_wait(&full[s], rph);
             if (!__all_sync(0xffffffffu, ok) || *(volatile int*)&flag[0]) {
               if (lane == 0) atomicExch(&flag[0], 1);
               break;
@@ -1238,10 +1281,10 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
                       const float2 x = *reinterpret_cast<const float2*>(qs + h * D + 2 * cpr);
                       uint32_t hi, lo;
                       split2(x.x, x.y, hi, lo);
-                      uint32_t* blk = qB + ((h >> 2) * KSL + sl) * 64 + kp;
+                      uint32_t* blk = qB + ((h >> 2) * KSL + sl) * BLKW + kp;
                       const int nh = 2 * (h & 3);
-                      blk[frag_word(4 * nh + tqk, sl)] = hi;
-                      blk[frag_word(4 * (nh + 1) + tqk, sl)] = lo;
+                      blk[fw(4 * nh + tqk, sl)] = hi;
+                      blk[fw(4 * (nh + 1) + tqk, sl)] = lo;
                     }
                   }
                 }
