@@ -407,7 +407,7 @@ def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, f
                     rr[b] += 1
             return L.kivi_ragged_append_decode(cstructs[li], stp[li], k_ptr, v_ptr, q_ptr, w.Hq,
                                                1.0, op, wp, wn, sh)
-        n_launch[0] += 1 + (1 if (not fused or c.r == c.R) else 0)
+        n_launch[0] += 1 if fused else 2  # fused: one launch, a due flush included
         if fused:
             return L.kivi_append_decode(cstructs[li], k_ptr, v_ptr, q_ptr, w.Hq, 1.0, op, wp, wn, sh)
         rc = L.kivi_append_token(cstructs[li], k_ptr, v_ptr, sh)
@@ -486,7 +486,7 @@ def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, f
 
     # e2e: the same loop, inputs from pinned host memory, output read back
     e2e = None
-    if not args.no_e2e:
+    if e2e_steps:
         # each step's k, v and q staged in one pinned host buffer and brought
         # over in one copy; k, v, q are views of one device buffer
         nk, nq_ = ks[0].numel(), qs[0].numel()

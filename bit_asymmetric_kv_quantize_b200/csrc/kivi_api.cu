@@ -143,11 +143,11 @@ void plan_stream(const kivi_cache* c, int sms, int ctas_per_sm, int seg_cap, Str
                               c->dims.dtype == KIVI_F16, tc_ctas(sms, ctas_per_sm), seg_cap);
 }
 
-// Workspace: per-unit arrival counters and one grid counter (8 bytes each,
-// 16-byte aligned block) followed by the split partials [B*Hq][n_split][D + 2]
-// floats.
+// Workspace: per-unit arrival counters, a grid arrival counter and a grid
+// barrier counter (8 bytes each, 16-byte aligned block) followed by the split
+// partials [B*Hq][n_split][D + 2] floats.
 size_t counter_bytes(const kivi_dims& d) {
-  return ((size_t)(d.B * d.Hkv + 1) * 8 + 15) / 16 * 16;
+  return ((size_t)(d.B * d.Hkv + 2) * 8 + 15) / 16 * 16;
 }
 
 int ws_splits(const kivi_dims& d, int sms) {
@@ -175,12 +175,14 @@ void touch_noalloc_scratch();
 int decode_launch(const kivi_cache* c, const void* q, int Hq, float softmax_scale, void* out,
                   void* ws, int split_cap, int sms, void* stream, bool simt,
                   const void* new_k = nullptr, const void* new_v = nullptr, int new_slot = 0,
-                  void* dev_state = nullptr, bool ragged = false, bool pending = false) {
+                  void* dev_state = nullptr, bool ragged = false, bool pending = false,
+                  bool flush = false) {
   touch_noalloc_scratch();
   const int gq = Hq / c->dims.Hkv;
   DecodeArgs a;
   a.ragged = ragged ? 1 : 0;
   a.pending = pending ? 1 : 0;
+  a.flush = flush ? 1 : 0;
   a.new_k = new_k;
   a.new_v = new_v;
   a.new_slot = new_slot;
@@ -475,17 +477,24 @@ int kivi_append_decode(kivi_cache* cache, const void* k, const void* v, const vo
   if (sms <= 0) return KIVI_ERR_CUDA;
   if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(cache->dims, Hq, sms))
     return KIVI_ERR_WORKSPACE;
-  // flush due, or a token not 16-byte aligned (the kernel copies it in
-  // 16-byte pieces): the append as its own launch, then decode
-  if (cache->r == cache->dims.R || ((uintptr_t)k & 15) || ((uintptr_t)v & 15)) {
+  // a token not 16-byte aligned (the kernel copies it in 16-byte pieces):
+  // the append as its own launch, then decode
+  if (((uintptr_t)k & 15) || ((uintptr_t)v & 15)) {
     rc = kivi_append_token(cache, k, v, stream);
     if (rc) return rc;
     return decode_launch(cache, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms),
                          sms, stream, false);
   }
+  // one launch: a due flush (full window) is quantized into the store by the
+  // decode kernel itself before it reads the store; the token goes to window
+  // slot r (slot 0 after a flush)
+  const bool flush = cache->r == cache->dims.R;
   rc = decode_launch(&after, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms), sms,
-                     stream, false, k, v, cache->r);
-  if (rc == KIVI_OK) cache->r = after.r;
+                     stream, false, k, v, flush ? 0 : cache->r, nullptr, false, false, flush);
+  if (rc == KIVI_OK) {
+    cache->n_q = after.n_q;
+    cache->r = after.r;
+  }
   return rc;
 }
 
@@ -515,12 +524,20 @@ int kivi_append_decode_dev(const kivi_cache* cache, void* state, const void* k, 
   if (sms <= 0) return KIVI_ERR_CUDA;
   if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(cache->dims, Hq, sms))
     return KIVI_ERR_WORKSPACE;
-  if (kivi::launch_append_dev(view(cache), cache->dims.B * cache->dims.Hkv, cache->dims.D,
-                              cache->dims.bits, cache->dims.dtype, k, v,
-                              (const kivi::DevState*)state, (cudaStream_t)stream) != cudaSuccess)
-    return KIVI_ERR_CUDA;
+  if (((uintptr_t)k & 15) || ((uintptr_t)v & 15)) {
+    // a token not 16-byte aligned: the append as its own launch, then decode
+    if (kivi::launch_append_dev(view(cache), cache->dims.B * cache->dims.Hkv, cache->dims.D,
+                                cache->dims.bits, cache->dims.dtype, k, v,
+                                (const kivi::DevState*)state, (cudaStream_t)stream) != cudaSuccess)
+      return KIVI_ERR_CUDA;
+    return decode_launch(&after, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms),
+                         sms, stream, false, nullptr, nullptr, 0, state);
+  }
+  // one launch: the decode kernel reads the counters, flushes a full window
+  // into the store, writes the token into its window slot, decodes, and its
+  // last CTA advances the counters
   return decode_launch(&after, q, Hq, softmax_scale, out, workspace, ws_splits(cache->dims, sms),
-                       sms, stream, false, nullptr, nullptr, 0, state);
+                       sms, stream, false, k, v, 0, state);
 }
 
 int kivi_ragged_prefill(kivi_cache* cache, void* state, const void* K, const void* V,

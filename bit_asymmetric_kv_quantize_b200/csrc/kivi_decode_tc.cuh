@@ -51,6 +51,7 @@
 #include <mutex>
 
 #include "kivi_internal.cuh"
+#include "kivi_quantize_tile.cuh"
 
 namespace kivi {
 namespace {
@@ -453,20 +454,27 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
     a.r = 0;
     a.new_k = nullptr;
   } else if (dev) {
-    // device counters as the preceding append launch found them; decode the
-    // cache after that append (it flushed when r was R)
+    // device counters as they stand before this step's append; decode the
+    // cache after it (a flush first when r was R).  With new_k set this
+    // launch performs the append itself (the flush below, the token into
+    // window slot r, or slot 0 after a flush); else an earlier launch did.
     const DevState st0 = *args.dev_state;
-    if (st0.status != 0 || st0.n_q + st0.r + 1 > args.c.Tq + args.c.R) return;  // cache full
+    if (st0.status != 0 || st0.n_q + st0.r + 1 > args.c.Tq + args.c.R) {
+      // cache full: nothing is written and the state says so
+      if (args.new_k != nullptr && cta == 0 && threadIdx.x == 0) args.dev_state->status = 1;
+      return;
+    }
     const bool fl = st0.r == args.c.R;
     a.n_q = fl ? st0.n_q + args.c.R : st0.n_q;
     a.r = fl ? 1 : st0.r + 1;
+    a.flush = (fl && args.new_k != nullptr) ? 1 : 0;
+    a.new_slot = fl ? 0 : st0.r;
     const StreamPlan pl =
         plan_stream_core(args.units, a.n_q, a.r, sizeof(T) == 2, gridDim.x, args.seg_cap);
     a.tiles_per_cta = pl.W;
     a.win_weight = pl.win_weight;
     a.max_seg = pl.max_seg;
     a.n_split = pl.max_seg;
-    a.new_k = nullptr;  // the append launch wrote the token
   }
   const int Hq = a.Hkv * GQ;
   const CacheView& c = a.c;
@@ -495,6 +503,33 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
     // flag, NaN outputs) rather than read a mis-swizzled layout
     flag[0] = (sizeof(T) == 2 && (smem_u32(smem) & 1023u) != 0) ? 1 : 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (!RAG && a.flush) {
+    // a due window flush folded into this launch: every unit's R window
+    // tokens are quantized into the store at positions n_q - R .. n_q - 1
+    // (n_q counts them already), the tiles spread over all CTAs and taken by
+    // threads 0 .. D-1 of each in the ring's shared memory, which is not in
+    // use yet; then a grid barrier (the persistent grid's CTAs are all
+    // resident), after which the stream reads those tiles like any other
+    uint8_t* ck = smem;
+    uint8_t* cv = smem + kTile * D;
+    const int wt = c.R / kTile;
+    const long long nft = (long long)a.units * wt;
+    for (long long f = cta; f < nft; f += gridDim.x) {
+      if (tid < D) {
+        const long long u = f / wt;
+        const int x = (int)(f - u * wt);
+        const T* kr = reinterpret_cast<const T*>(c.k_res) + (u * c.R + x * kTile) * D;
+        const T* vr = reinterpret_cast<const T*>(c.v_res) + (u * c.R + x * kTile) * D;
+        quantize_tile<D, BITS, T, MT, 2>(c, u, kr, vr, a.n_q - c.R + x * kTile, ck, cv);
+      }
+    }
+    // the store's new tiles are read by bulk copies (the async proxy)
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncthreads();
+    if (tid == 0 && !grid_barrier(a.ctr + a.units + 1, dev ? 0u : a.epoch, gridDim.x))
+      atomicExch(&flag[0], 1);
+    __syncthreads();
   }
   if (sizeof(T) == 4 && a.new_k != nullptr) {
     // fused append, fp32 window (read by generic loads after the barrier
@@ -1519,9 +1554,11 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
   }
   __syncthreads();
   if (!RAG && dev && tid == 0 && arrive_unit_reset(a.ctr + a.units, gridDim.x) == 1) {
-    // the last CTA to finish advances the device counters
+    // the last CTA to finish advances the device counters (and clears the
+    // flush barrier's count: every CTA is past it)
     args.dev_state->n_q = a.n_q;
     args.dev_state->r = a.r;
+    if (a.flush) asm volatile("st.relaxed.gpu.global.u64 [%0], 0;" ::"l"(a.ctr + a.units + 1) : "memory");
   }
   if (RAG && a.pending) {
     // the last CTA to finish advances every sequence that took its token

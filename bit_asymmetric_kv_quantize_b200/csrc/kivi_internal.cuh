@@ -307,6 +307,11 @@ struct DecodeArgs {
   // this step's append and the last CTA advances every valid sequence
   int ragged;
   int pending;
+  // uniform batches, fused append (new_k set): the window is full and is
+  // quantized into the store by this launch before the decode reads it (the
+  // host sets it; in device-counter mode the kernel decides from the
+  // counters).  n_q above already counts the flushed tokens.
+  int flush;
 };
 
 constexpr float kNaN = __builtin_nanf("");
@@ -388,6 +393,54 @@ __device__ __forceinline__ int arrive_unit_reset(unsigned long long* ctr, long l
   if ((long long)old + 1 != n) return 0;
   asm volatile("st.relaxed.gpu.global.u64 [%0], 0;" ::"l"(ctr) : "memory");
   return 1;
+}
+
+// Grid-wide barrier of one launch whose CTAs are all resident at once (the
+// persistent decode grid): thread 0 of each of the n CTAs arrives at *ctr and
+// waits (acquire, bounded by ~2 s of clock cycles) until all have.  epoch != 0:
+// the word carries the call's epoch in its high half, like arrive_unit, so a
+// count left by an earlier call restarts: a CTA that finds a stale word tries
+// once to swap in (epoch, 1); every other arrival is a fetch-and-add, since
+// only this launch's CTAs write the word once it holds this epoch (hundreds
+// of CTAs retrying compare-and-swaps on one word would serialize for many
+// microseconds).  epoch == 0: a plain count that starts at zero and that the
+// caller resets once every CTA is past it.  Returns false if the wait ran out.
+__device__ __forceinline__ bool grid_barrier(unsigned long long* ctr, unsigned int epoch,
+                                             long long n) {
+  if (epoch != 0) {
+    const unsigned long long ep = (unsigned long long)epoch << 32;
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ctr) : "memory");
+    bool counted = false;
+    for (int it = 0; it < 64 && (v >> 32) != epoch; ++it) {
+      unsigned long long old;
+      asm volatile("atom.acq_rel.gpu.global.cas.b64 %0, [%1], %2, %3;"
+                   : "=l"(old)
+                   : "l"(ctr), "l"(v), "l"(ep | 1ull)
+                   : "memory");
+      if (old == v) {
+        counted = true;
+        break;
+      }
+      v = old;
+    }
+    if (!counted) {
+      if ((v >> 32) != epoch) return false;
+      asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(ctr) : "memory");
+    }
+  } else {
+    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(ctr) : "memory");
+  }
+  const long long t0 = clock64();
+  for (;;) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ctr) : "memory");
+    const bool done = epoch != 0 ? ((v >> 32) == epoch && (long long)(v & 0xffffffffull) >= n)
+                                 : (long long)v >= n;
+    if (done) return true;
+    if (clock64() - t0 > (1LL << 32)) return false;
+    asm volatile("nanosleep.u32 64;" ::: "memory");
+  }
 }
 
 // End of a split CTA, after it wrote its (m, l, acc[D]) partials: the last CTA

@@ -25,113 +25,13 @@
 // the binary32 scale and minimum are rounded to binary16 (nearest, ties to
 // even) and the codes are chosen against the rounded pair, so that the
 // stored scale and zero reproduce them as closely as the code grid allows.
-#include "kivi_codes.cuh"
 #include "kivi_internal.cuh"
+#include "kivi_quantize_tile.cuh"
 
 namespace kivi {
 namespace {
 
-// (code_of and recip_rn: kivi_codes.cuh)
-
-// Quantize one tile of kTile tokens (= one key group) of one unit.
-//   Ksrc, Vsrc: the tile's first token row; rows are D elements apart.
-//   t0: token position of the tile in the quantized store (multiple of kTile).
-// blockDim.x == D.  Thread d reduces key channel d over the tile's tokens;
-// thread i reduces value group (token i / NJ, group i % NJ) over kGv channels.
-// Codes go through shared memory and are packed by all threads.
-// Paged stores: the tile goes to its page's slot (a page outside the block
-// table or the pool writes nothing; the callers have refused such a
-// sequence already).
-template <int D, int BITS, typename T, typename M>
-__device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit,
-                                              const T* __restrict__ Ksrc,
-                                              const T* __restrict__ Vsrc, long long t0,
-                                              uint8_t* ck, uint8_t* cv) {
-  using Lt = Layout<D, BITS>;
-  constexpr int E = Lt::E, WK = Lt::WK, NJ = Lt::NJ;
-  const float Lf = (float)Lt::L;
-  const int tid = threadIdx.x;
-  const long long Ts = store_tokens(c);
-  {
-    long long su, stl;
-    if (!store_tile(c, unit, t0 / kTile, &su, &stl)) return;  // same for the whole block
-    unit = su;
-    t0 = stl * kTile;
-  }
-
-  // ---- keys: channel tid over kTile tokens
-  {
-    float x[kTile];
-#pragma unroll
-    for (int t = 0; t < kTile; ++t) x[t] = to_f32(Ksrc[(long long)t * D + tid]);
-    float mn = x[0], mx = x[0];
-#pragma unroll
-    for (int t = 1; t < kTile; ++t) {
-      if (x[t] < mn) mn = x[t];
-      if (x[t] > mx) mx = x[t];
-    }
-    const float s = round_meta<M>(__fdiv_rn(__fsub_rn(mx, mn), Lf));
-    const float z = round_meta<M>(mn);
-    const long long g = t0 / kG;
-    reinterpret_cast<M*>(c.k_scale)[unit * Lt::k_meta_unit(Ts) + g * D + tid] = from_f32<M>(s);
-    reinterpret_cast<M*>(c.k_zero)[unit * Lt::k_meta_unit(Ts) + g * D + tid] = from_f32<M>(z);
-    const float rs = recip_rn(s);
-#pragma unroll
-    for (int t = 0; t < kTile; ++t) {
-      int code = 0;
-      if (s != 0.0f) code = code_of(__fsub_rn(x[t], z), s, rs, Lt::L);
-      ck[t * D + tid] = (uint8_t)code;
-    }
-  }
-  // ---- values: token tid / NJ, channel group tid % NJ
-  {
-    const int t = tid / NJ, j = tid % NJ;
-    const T* src = Vsrc + (long long)t * D + j * kGv;
-    float x[kGv];
-#pragma unroll
-    for (int i = 0; i < kGv; ++i) x[i] = to_f32(src[i]);
-    float mn = x[0], mx = x[0];
-#pragma unroll
-    for (int i = 1; i < kGv; ++i) {
-      if (x[i] < mn) mn = x[i];
-      if (x[i] > mx) mx = x[i];
-    }
-    const float s = round_meta<M>(__fdiv_rn(__fsub_rn(mx, mn), Lf));
-    const float z = round_meta<M>(mn);
-    const long long mo = unit * Lt::v_meta_unit(Ts) + (t0 + t) * NJ + j;
-    reinterpret_cast<M*>(c.v_scale)[mo] = from_f32<M>(s);
-    reinterpret_cast<M*>(c.v_zero)[mo] = from_f32<M>(z);
-    const float rs = recip_rn(s);
-#pragma unroll
-    for (int i = 0; i < kGv; ++i) {
-      int code = 0;
-      if (s != 0.0f) code = code_of(__fsub_rn(x[i], z), s, rs, Lt::L);
-      cv[t * D + j * kGv + i] = (uint8_t)code;
-    }
-  }
-  __syncthreads();
-  // ---- pack: keys along channels, values along tokens; D*BITS words each
-  constexpr int NW = kTile * WK;  // == (kTile / E) * D == D * BITS
-  uint32_t* kdst = c.k_codes + unit * Lt::k_codes_unit(Ts) + t0 * WK;
-  uint32_t* vdst = c.v_codes + unit * Lt::v_codes_unit(Ts) + (t0 / E) * D;
-#pragma unroll
-  for (int k = tid; k < NW; k += D) {
-    const int t = k / WK, w = k % WK;
-    uint32_t word = 0;
-#pragma unroll
-    for (int i = 0; i < E; ++i) word |= (uint32_t)ck[t * D + w * E + i] << (BITS * i);
-    kdst[k] = word;
-  }
-#pragma unroll
-  for (int k = tid; k < NW; k += D) {
-    const int tb = k / D, d = k % D;
-    uint32_t word = 0;
-#pragma unroll
-    for (int i = 0; i < E; ++i) word |= (uint32_t)cv[(tb * E + i) * D + d] << (BITS * i);
-    vdst[k] = word;
-  }
-  __syncthreads();
-}
+// (quantize_tile: kivi_quantize_tile.cuh; code_of and recip_rn: kivi_codes.cuh)
 
 // grid (n_q / kTile + 1, units); the last x-block copies the r window tokens.
 // Ragged (lens != null): grid (T_len / kTile + 1, units); sequence b = unit /
@@ -176,7 +76,7 @@ __global__ void __launch_bounds__(D) prefill_kernel(CacheView c, const T* __rest
     if (!ok) return;
   }
   if (tile < n_q / kTile) {
-    quantize_tile<D, BITS, T, M>(c, unit, Ku + tile * kTile * D, Vu + tile * kTile * D,
+    quantize_tile<D, BITS, T, M, 0>(c, unit, Ku + tile * kTile * D, Vu + tile * kTile * D,
                                  tile * kTile, ck, cv);
   } else if (tile == gridDim.x - 1) {
     T* kr = reinterpret_cast<T*>(c.k_res) + unit * c.R * D;
@@ -228,7 +128,7 @@ __global__ void __launch_bounds__(D) append_kernel(CacheView c, const T* __restr
   T* kr = reinterpret_cast<T*>(c.k_res) + unit * c.R * D;
   T* vr = reinterpret_cast<T*>(c.v_res) + unit * c.R * D;
   if (flush)
-    quantize_tile<D, BITS, T, M>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
+    quantize_tile<D, BITS, T, M, 0>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
                                  n_q + tile * kTile, ck, cv);
   if (tile == 0) {
     kr[(long long)slot * D + threadIdx.x] = k[unit * D + threadIdx.x];

@@ -229,13 +229,14 @@ KIVI_API int kivi_decode_attention_simt(const kivi_cache *cache, const void *q,
 /* One decode step of a streaming loop: kivi_append_token(cache, k, v)
  * followed by kivi_decode_attention over the cache that now holds the new
  * token -- same arguments as the two calls, same result, same counter
- * update.  When no flush is due (r < R) it is one kernel launch: the decode
- * kernel's CTA that owns a sequence's window writes the new token into
- * window slot r before it reads the window.  When the window is full the
- * flush runs first as its own launch (as in kivi_append_token), and so does
- * the append when k or v is not 16-byte aligned.  All
- * argument checks of both calls happen before any launch, so an error
- * leaves the cache unchanged.  The counters stay on the host, so a loop of
+ * update -- in one kernel launch: when the window is full (r == R) the
+ * decode kernel first quantizes it into the store (every CTA takes a share
+ * of the window tiles, then a grid-wide barrier), and the warp that reads
+ * the window tile holding the new token's slot (r, or 0 after a flush)
+ * writes the token there, into shared memory and the cache.  Only a k or v
+ * that is not 16-byte aligned takes two launches (the append on its own
+ * first).  All argument checks of both calls happen before any launch, so
+ * an error leaves the cache unchanged.  The counters stay on the host, so a loop of
  * these calls is not graph-capturable.  (KIVI, study.space summary: new
  * tokens enter the full-precision residual part; decode attends over both
  * parts.)
@@ -258,11 +259,14 @@ KIVI_API int kivi_append_decode(kivi_cache *cache, const void *k, const void *v,
 KIVI_API int kivi_dev_state_init(const kivi_cache *cache, void *state, void *stream);
 
 /* kivi_append_decode with the counters in `state` (device memory, see
- * kivi_dev_state_init) instead of cache->n_q / cache->r: two launches every
- * step -- an append that flushes the window on the device when r == R, and
- * the decode, which plans its split on the device and advances the counters
- * when it finishes.  Launch arguments do not depend on the counters, so the
- * same two launches can be captured once and replayed.  The workspace
+ * kivi_dev_state_init) instead of cache->n_q / cache->r, in one kernel
+ * launch per step: the decode kernel reads the counters, quantizes a full
+ * window (r == R) into the store before it reads the store (all CTAs, then a
+ * grid-wide barrier), writes the token into its window slot, plans its split
+ * on the device, and its last CTA advances the counters.  Launch arguments
+ * do not depend on the counters, so the launch can be captured once and
+ * replayed.  (A k or v that is not 16-byte aligned takes two launches: the
+ * append on its own, then the decode.)  The workspace
  * (kivi_decode_workspace_bytes) must be zero-filled before first use and
  * used only by these calls: they count arrivals in counters that every call
  * leaves at zero.  (KIVI, study.space summary: append to the residual part,

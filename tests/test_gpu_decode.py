@@ -329,3 +329,74 @@ def test_streaming_workload_device_counters_and_fused_steps():
         assert torch.equal(dev.append_decode_dev(st, k, v, q, 1.0), out_r), f"device step {step}"
     dev.load_dev_state(st)
     assert (ref.n_q, ref.r) == (fused.n_q, fused.r) == (dev.n_q, dev.r)
+
+
+def _kernel_nodes(g) -> int:
+    """Kernel launches captured in a torch CUDA graph (cuda-python runtime API)."""
+    import cuda.bindings.runtime as rt
+    graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+    err, nodes, n = rt.cudaGraphGetNodes(graph, 0)
+    assert err == rt.cudaError_t.cudaSuccess
+    err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+    assert err == rt.cudaError_t.cudaSuccess
+    kinds = [rt.cudaGraphNodeGetType(x)[1] for x in nodes]
+    return sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_fused_steps_are_one_launch_each_flushes_included(dtype):
+    """kivi_append_decode and kivi_append_decode_dev launch one kernel per
+    step, also on the steps whose full window is flushed into the store (the
+    decode kernel quantizes it itself); captured steps equal the separate
+    append + decode calls bit for bit and stay within the bars vs the oracle."""
+    w = small(D=128, dtype=dtype, gq=4, T=96, R=32, B=2, Hkv=2, seed=21)  # r = 32: flush due
+    K, V = W.prompt_kv(w, device="cuda")
+    fused, dev, ref = (gpu_cache(w, capacity=512) for _ in range(3))
+    for c in (fused, dev, ref):
+        c.prefill(K, V)
+    oc = oracle_cache(w, capacity=512)
+    oracle_prefill(oc, K, V)
+    st = dev.dev_state()
+    assert fused.r == fused.R
+    # one eager step of each (library setup outside the captures)
+    k, v = W.step_kv(w, 0, device="cuda")
+    q = W.query(w, 0, device="cuda")
+    a = fused.append_decode(k, v, q, 1.0)
+    b = dev.append_decode_dev(st, k, v, q, 1.0)
+    ref.append(k, v)
+    c0 = ref.decode(q, 1.0)
+    oracle_append(oc, k, v)
+    assert torch.equal(a, c0) and torch.equal(b, c0)
+    assert_decode_close(a, oc, q, 1.0)
+    torch.cuda.synchronize()
+    # steps 1..40 cross the next flush (r reaches 32 again at step 31)
+    for step in range(1, 41):
+        k, v = W.step_kv(w, step, device="cuda")
+        q = W.query(w, step, device="cuda")
+        flush = fused.r == fused.R
+        outs = []
+        for c, call in ((fused, lambda: fused.append_decode(k, v, q, 1.0)),
+                        (dev, lambda: dev.append_decode_dev(st, k, v, q, 1.0))):
+            g = torch.cuda.CUDAGraph(keep_graph=True)
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    out = call()
+            torch.cuda.synchronize()
+            assert _kernel_nodes(g) == 1, (step, flush)
+            g.instantiate()
+            g.replay()
+            torch.cuda.synchronize()
+            outs.append(out)
+            del g
+        ref.append(k, v)
+        c0 = ref.decode(q, 1.0)
+        oracle_append(oc, k, v)
+        assert torch.equal(outs[0], c0), step
+        assert torch.equal(outs[1], c0), step
+        if flush or step % 10 == 0:
+            assert_decode_close(outs[0], oc, q, 1.0)
+    dev.load_dev_state(st)
+    assert (dev.n_q, dev.r) == (fused.n_q, fused.r) == (ref.n_q, ref.r)
+    assert_state_equal(fused, oc)
