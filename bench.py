@@ -79,7 +79,7 @@ def parse():
                    help="ragged workloads: quantized store in pages of R tokens from a pool, "
                         "through a block table whose pages are shuffled over the pool or "
                         "consecutive per sequence")
-    p.add_argument("--bits", type=int, choices=[1, 2, 4], default=None,
+    p.add_argument("--bits", type=int, choices=[1, 2, 3, 4], default=None,
                    help="code width other than the workload's (a format variant)")
     p.add_argument("--meta", choices=["f32", "f16"], default="f32",
                    help="scale/zero storage: binary32, or the binary16 format variant "
@@ -102,7 +102,8 @@ def bench_workload(args, name=None) -> W.Workload:
     if args.meta == "f16":
         w = w.with_(meta="f16", name=w.name + "-meta16")
     if args.bits is not None and args.bits != w.bits:
-        w = w.with_(bits=args.bits, name=f"{w.name}-{args.bits}bit")
+        base = w.name[:-len("-2bit")] if w.name.endswith("-2bit") else w.name
+        w = w.with_(bits=args.bits, name=f"{base}-{args.bits}bit")
     return w
 
 

@@ -127,6 +127,12 @@ def _meta_code(meta: torch.dtype) -> int:
     raise ValueError(f"unsupported metadata dtype {meta}")
 
 
+def _code_block(bits: int):
+    """(codes per block, 32-bit words per block): 32/bits codes in one word,
+    or at 3 bits 32 codes as three bit-plane words (include/kivi.h)."""
+    return (32, 3) if bits == 3 else (32 // bits, 1)
+
+
 def _check(rc: int, what: str) -> None:
     if rc != 0:
         raise KiviError(rc, what)
@@ -171,14 +177,14 @@ class KiviCache:
                                      ctypes.byref(ptrs)), "kivi_cache_init")
         self._ws: Optional[torch.Tensor] = None
         self._ws_dev: Optional[torch.Tensor] = None
-        E = 32 // bits
+        E, WB = _code_block(bits)
         Tq = capacity - R
         self.B, self.Hkv, self.D, self.bits, self.R, self.capacity = B, Hkv, D, bits, R, capacity
         self.shapes = {
-            "k_codes": ((B, Hkv, Tq, D // E), torch.int32),
+            "k_codes": ((B, Hkv, Tq, D // E * WB), torch.int32),
             "k_scale": ((B, Hkv, Tq // G, D), meta),
             "k_zero": ((B, Hkv, Tq // G, D), meta),
-            "v_codes": ((B, Hkv, Tq // E, D), torch.int32),
+            "v_codes": ((B, Hkv, Tq // E * WB, D), torch.int32),
             "v_scale": ((B, Hkv, Tq, D // Gv), meta),
             "v_zero": ((B, Hkv, Tq, D // Gv), meta),
             "k_res": ((B, Hkv, R, D), dtype),
@@ -421,14 +427,14 @@ class PagedKiviCache(KiviCache):
                                            pages_per_seq, num_pages), "kivi_paged_cache_init")
         self._ws: Optional[torch.Tensor] = None
         self._ws_dev: Optional[torch.Tensor] = None
-        E = 32 // bits
+        E, WB = _code_block(bits)
         self.B, self.Hkv, self.D, self.bits, self.R, self.capacity = B, Hkv, D, bits, R, capacity
         P = num_pages
         self.shapes = {
-            "k_codes": ((P, Hkv, R, D // E), torch.int32),
+            "k_codes": ((P, Hkv, R, D // E * WB), torch.int32),
             "k_scale": ((P, Hkv, R // G, D), meta),
             "k_zero": ((P, Hkv, R // G, D), meta),
-            "v_codes": ((P, Hkv, R // E, D), torch.int32),
+            "v_codes": ((P, Hkv, R // E * WB, D), torch.int32),
             "v_scale": ((P, Hkv, R, D // Gv), meta),
             "v_zero": ((P, Hkv, R, D // Gv), meta),
             "k_res": ((B, Hkv, R, D), dtype),

@@ -24,7 +24,7 @@ int check_dims(const kivi_dims* d) {
   if (!d) return KIVI_ERR_ARG;
   if (d->B <= 0 || d->Hkv <= 0 || d->D <= 0 || d->R <= 0 || d->capacity <= 0)
     return KIVI_ERR_ARG;
-  if (d->bits != 1 && d->bits != 2 && d->bits != 4) return KIVI_ERR_UNSUPPORTED;
+  if (d->bits != 1 && d->bits != 2 && d->bits != 3 && d->bits != 4) return KIVI_ERR_UNSUPPORTED;
   if (d->G != kivi::kG || d->Gv != kivi::kGv) return KIVI_ERR_UNSUPPORTED;
   if (d->D != 32 && d->D != 64 && d->D != 128) return KIVI_ERR_UNSUPPORTED;
   if (d->R % kivi::kTile != 0) return KIVI_ERR_UNSUPPORTED;
@@ -266,6 +266,7 @@ int decode_common(const kivi_cache* c, const void* q, int Hq, float softmax_scal
                   void* workspace, size_t ws_bytes, void* stream, bool simt) {
   int rc = decode_checks(c, q, Hq, out);
   if (rc) return rc;
+  if (simt && c->dims.bits == 3) return KIVI_ERR_UNSUPPORTED;  // CUDA-core kernel: 1, 2, 4 bits
   const int sms = device_sms();
   if (sms <= 0) return KIVI_ERR_CUDA;
   if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(c->dims, Hq, sms))
@@ -322,12 +323,14 @@ int kivi_buffer_sizes(const kivi_dims* dims, size_t out_bytes[KIVI_NUM_BUFFERS])
   if (!out_bytes) return KIVI_ERR_ARG;
   const long long units = (long long)dims->B * dims->Hkv;
   const long long Tq = dims->capacity - dims->R;
-  const int E = 32 / dims->bits;
+  // E codes per block of WB words: 32/b in one word, or 32 as three bit planes at 3 bits
+  const int E = dims->bits == 3 ? 32 : 32 / dims->bits;
+  const int WB = dims->bits == 3 ? 3 : 1;
   const size_t f = meta_bytes(dims->meta);
-  out_bytes[KIVI_BUF_K_CODES] = (size_t)(units * Tq * (dims->D / E)) * sizeof(uint32_t);
+  out_bytes[KIVI_BUF_K_CODES] = (size_t)(units * Tq * (dims->D / E) * WB) * sizeof(uint32_t);
   out_bytes[KIVI_BUF_K_SCALE] = (size_t)(units * (Tq / dims->G) * dims->D) * f;
   out_bytes[KIVI_BUF_K_ZERO] = out_bytes[KIVI_BUF_K_SCALE];
-  out_bytes[KIVI_BUF_V_CODES] = (size_t)(units * (Tq / E) * dims->D) * sizeof(uint32_t);
+  out_bytes[KIVI_BUF_V_CODES] = (size_t)(units * (Tq / E) * WB * dims->D) * sizeof(uint32_t);
   out_bytes[KIVI_BUF_V_SCALE] = (size_t)(units * Tq * (dims->D / dims->Gv)) * f;
   out_bytes[KIVI_BUF_V_ZERO] = out_bytes[KIVI_BUF_V_SCALE];
   out_bytes[KIVI_BUF_K_RES] = (size_t)(units * dims->R * dims->D) * elem_bytes(dims->dtype);

@@ -8,6 +8,8 @@ namespace {
 
 cudaError_t tc_dispatch(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
                         int* occ) {
+  if (a.bits == 3) return a.ragged ? tc_dispatch_3bit_ragged(a, s, e0, e1, occ)
+                                   : tc_dispatch_3bit(a, s, e0, e1, occ);
   if (a.ragged) {
     if (a.meta == 1) return tc_dispatch_ragged_meta16(a, s, e0, e1, occ);
     if (a.meta != 0) return cudaErrorInvalidValue;

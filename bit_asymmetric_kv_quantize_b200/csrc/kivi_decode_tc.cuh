@@ -82,6 +82,25 @@ struct Pairs<2> {
   __host__ __device__ static constexpr int shift(int i) { return i < 5 ? 0 : 10; }
   __host__ __device__ static constexpr uint32_t mask(int i) { return 0x00030003u << e(i); }
 };
+// 3 bits: a block of 32 codes is three bit-plane words; pair i (i < 16) =
+// codes i and i + 16, taken from each plane by the 1-bit rule but with e
+// kept below 8 (a shift by 8 for i >= 8), so that the three planes' bits of
+// a code land at bits e, e + 1, e + 2 of its half: the exact subnormal
+// c 2^(e - 24), c < 8.
+template <>
+struct Pairs<3> {
+  static constexpr int PPW = 16;  // pairs per block
+  static constexpr int EMAX = 7;
+  __host__ __device__ static constexpr int e(int i) { return i & 7; }
+  __host__ __device__ static constexpr int shift(int i) { return i < 8 ? 0 : 8; }
+  __host__ __device__ static constexpr uint32_t mask(int i) { return 0x00010001u << e(i); }
+};
+// The code pair of three bit planes p0, p1, p2 after a right shift by sh,
+// placed at bit e of each half by mask m = 0x00010001 << e.
+__device__ __forceinline__ uint32_t planes3(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t sh,
+                                            uint32_t m) {
+  return ((p0 >> sh) & m) | (((p1 >> sh) << 1) & (m << 1)) | (((p2 >> sh) << 2) & (m << 2));
+}
 template <>
 struct Pairs<4> {
   static constexpr int PPW = 4;
@@ -101,16 +120,17 @@ struct Geo {
   static constexpr int NW = GQ == 1 ? 4 : (GQ == 8 ? 7 : 11);
   // tiles per warp and stage (1-bit MHA also needs two to fit a window tile in a stage)
   static constexpr int TPW = (GQ == 1 && BITS <= 2) ? 2 : 1;
+  static constexpr int WB = Layout<D, BITS>::WB;  // words per code block (3: bit planes)
   static constexpr int THREADS = (NW + 1) * 32;
   static constexpr int kStage = NW * TPW;       // tiles per pipeline stage
-  static constexpr int E = 32 / BITS;
-  static constexpr int WK = D / E;       // key words per token
+  static constexpr int E = Layout<D, BITS>::E;   // codes per block
+  static constexpr int WK = Layout<D, BITS>::WK;  // key words per token
   static constexpr int NJ = D / kGv;     // value groups per token
   static constexpr int KSL = D / 16;     // k-slices of the score product
   static constexpr int NSL = kTile / 16;  // k-slices of the value product
   static constexpr int KC_B = kTile * WK * 4;
   static constexpr int KM_B = D * MB;  // MB: bytes per scale or zero
-  static constexpr int VC_B = (kTile / E) * D * 4;
+  static constexpr int VC_B = (kTile / E) * WB * D * 4;
   static constexpr int VM_B = kTile * NJ * MB;
   static constexpr int TILE_B = KC_B + 2 * KM_B + VC_B + 2 * VM_B;
   static constexpr int O_KC = 0;
@@ -169,7 +189,7 @@ struct Geo {
   static constexpr int NWL = WHOLE ? PPL / PPW : 1;
   // operand scale offsets: the factor 2^(S - e) lies in [2^-S, 2^S]
   static constexpr int SK = Pairs<BITS>::EMAX / 2;
-  static constexpr int SV = BITS == 2 ? 3 : 2;  // value e: 1-bit 0..3; 2-bit 0,2,4,6; 4-bit 0,4
+  static constexpr int SV = BITS == 2 ? 3 : 2;  // value e: 1, 3-bit 0..3; 2-bit 0,2,4,6; 4-bit 0,4
   static constexpr int WPS = STAGE_B / WTILE_B;       // window tiles per stage
   static_assert(WPS >= 1, "a window tile fits one ring slot");
   static_assert(WTILE_B % 1024 == 0, "window tiles keep the 1024-byte alignment");
@@ -607,7 +627,8 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
             bulk_copy(buf + G::O_KC, kc_u + (long long)t0 * kTile * WK, n * G::KC_B, &full[s]);
             bulk_copy(buf + G::O_KS, ks_u + (long long)t0 * D, n * G::KM_B, &full[s]);
             bulk_copy(buf + G::O_KZ, kz_u + (long long)t0 * D, n * G::KM_B, &full[s]);
-            bulk_copy(buf + G::O_VC, vc_u + (long long)t0 * (kTile / E) * D, n * G::VC_B, &full[s]);
+            bulk_copy(buf + G::O_VC, vc_u + (long long)t0 * (kTile / E) * G::WB * D, n * G::VC_B,
+                      &full[s]);
             bulk_copy(buf + G::O_VS, vs_u + (long long)t0 * kTile * NJ, n * G::VM_B, &full[s]);
             bulk_copy(buf + G::O_VZ, vz_u + (long long)t0 * kTile * NJ, n * G::VM_B, &full[s]);
           } else {
@@ -634,7 +655,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
               bulk_copy(buf + G::O_KC + o * G::KC_B, kc + stl * kTile * WK, run * G::KC_B, &full[s]);
               bulk_copy(buf + G::O_KS + o * G::KM_B, ks + stl * D, run * G::KM_B, &full[s]);
               bulk_copy(buf + G::O_KZ + o * G::KM_B, kz + stl * D, run * G::KM_B, &full[s]);
-              bulk_copy(buf + G::O_VC + o * G::VC_B, vc + stl * (kTile / E) * D, run * G::VC_B,
+              bulk_copy(buf + G::O_VC + o * G::VC_B, vc + stl * (kTile / E) * G::WB * D, run * G::VC_B,
                         &full[s]);
               bulk_copy(buf + G::O_VS + o * G::VM_B, vs + stl * kTile * NJ, run * G::VM_B, &full[s]);
               bulk_copy(buf + G::O_VZ + o * G::VM_B, vz + stl * kTile * NJ, run * G::VM_B, &full[s]);
@@ -739,13 +760,13 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
     // 16..31); k-slice sl takes tokens 8 sl .. 8 sl + 7 and their +16
     // partners, lane tq the pair at bit tq after a shift by 8 sl (a0 / a1)
     // or 8 sl + 4 (a2 / a3)
-    const uint32_t vM = BITS == 1 ? (0x00010001u << tq)
+    const uint32_t vM = (BITS == 1 || BITS == 3) ? (0x00010001u << tq)
                         : BITS == 2 ? (0x00030003u << (2 * tq))
                                     : ((tq & 1) ? 0x00F000F0u : 0x000F000Fu);
     const int vtw = BITS == 4 ? (tq >> 1) : 0;  // token-word offset of this lane
     // -- p' build, lane = token t: its k-slice, owner slot and e
     int pt_sl, pt_tq, pt_kp, pt_hf, pt_e;
-    if (BITS == 1) {
+    if (BITS == 1 || BITS == 3) {
       const int i = lane & 15;
       pt_hf = lane >> 4; pt_sl = i >> 3; pt_kp = (i >> 2) & 1; pt_tq = i & 3; pt_e = pt_tq;
     } else if (BITS == 2) {
@@ -857,7 +878,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
             kc[tt] = reinterpret_cast<const uint32_t*>(buf + G::O_KC) + ti * kTile * WK;
             ks[tt] = reinterpret_cast<const MT*>(buf + G::O_KS) + ti * D;
             kz[tt] = reinterpret_cast<const MT*>(buf + G::O_KZ) + ti * D;
-            vc[tt] = reinterpret_cast<const uint32_t*>(buf + G::O_VC) + ti * (kTile / E) * D;
+            vc[tt] = reinterpret_cast<const uint32_t*>(buf + G::O_VC) + ti * (kTile / E) * G::WB * D;
             vs[tt] = reinterpret_cast<const MT*>(buf + G::O_VS) + ti * kTile * NJ;
             vz[tt] = reinterpret_cast<const MT*>(buf + G::O_VZ) + ti * kTile * NJ;
           }
@@ -910,7 +931,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           __syncwarp();
 
           // -- scores: per tile 2 m-tiles of 16 tokens (rows g, g+8), KSL k-slices
-          uint32_t kw[TPW][2][2][G::NWL];
+          uint32_t kw[TPW][2][2][G::NWL * G::WB];
 #pragma unroll
           for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
@@ -918,8 +939,11 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
 #pragma unroll
               for (int r = 0; r < 2; ++r) {
                 const uint32_t* row = kc[tt] + (16 * mt + 8 * r + g) * WK +
-                                      (G::WHOLE ? tq * G::NWL : (tq * G::PPL) / G::PPW);
-                if constexpr (G::NWL == 4) {
+                                      G::WB * (G::WHOLE ? tq * G::NWL : (tq * G::PPL) / G::PPW);
+                if constexpr (BITS == 3) {
+#pragma unroll
+                  for (int x = 0; x < G::NWL * 3; ++x) kw[tt][mt][r][x] = row[x];
+                } else if constexpr (G::NWL == 4) {
                   const uint4 v = *reinterpret_cast<const uint4*>(row);
                   kw[tt][mt][r][0] = v.x; kw[tt][mt][r][1] = v.y;
                   kw[tt][mt][r][2] = v.z; kw[tt][mt][r][3] = v.w;
@@ -930,8 +954,15 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
                   kw[tt][mt][r][0] = row[0];
                 }
               }
-          auto key_reg = [&](const uint32_t (&w)[G::NWL], int jj) -> uint32_t {
-            if constexpr (G::WHOLE) {
+          auto key_reg = [&](const uint32_t (&w)[G::NWL * G::WB], int jj) -> uint32_t {
+            if constexpr (BITS == 3) {
+              if constexpr (G::WHOLE) {
+                const int i = jj % G::PPW, bk = 3 * (jj / G::PPW);
+                return planes3(w[bk], w[bk + 1], w[bk + 2], PR::shift(i), PR::mask(i));
+              } else {
+                return planes3(w[0], w[1], w[2], kS[jj], kM[jj]);
+              }
+            } else if constexpr (G::WHOLE) {
               const int i = jj % G::PPW;
               return (w[jj / G::PPW] >> PR::shift(i)) & PR::mask(i);
             } else {
@@ -1067,19 +1098,34 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           for (int tt = 0; tt < TPW; ++tt) {
 #pragma unroll
             for (int sl = 0; sl < NSL; ++sl) {
-              const int tw = BITS == 1 ? 0 : BITS == 2 ? sl : 2 * sl + vtw;
+              const int tw = (BITS == 1 || BITS == 3) ? 0 : BITS == 2 ? sl : 2 * sl + vtw;
               constexpr int SH = BITS == 1 ? 4 : 8;  // shift to the a2 / a3 pairs
               const int s0 = BITS == 1 ? 8 * sl : 0;  // 1-bit: this slice's byte
 #pragma unroll
               for (int j = 0; j < NJ; ++j) {
-                uint4 w = *reinterpret_cast<const uint4*>(vc[tt] + tw * D + 32 * j + 4 * g);
-                if (BITS == 1) {
-                  w.x >>= s0; w.y >>= s0; w.z >>= s0; w.w >>= s0;
+                uint32_t x0, x1, x2, x3, y0, y1, y2, y3;
+                if constexpr (BITS == 3) {
+                  // three bit-plane rows of the tile, each word a channel's 32
+                  // tokens (the 1-bit token order)
+                  const uint32_t* vr = vc[tt] + 32 * j + 4 * g;
+                  const uint4 p0 = *reinterpret_cast<const uint4*>(vr);
+                  const uint4 p1 = *reinterpret_cast<const uint4*>(vr + D);
+                  const uint4 p2 = *reinterpret_cast<const uint4*>(vr + 2 * D);
+                  const uint32_t sa = 8 * sl, sb = 8 * sl + 4;
+                  x0 = planes3(p0.x, p1.x, p2.x, sa, vM); x2 = planes3(p0.x, p1.x, p2.x, sb, vM);
+                  x1 = planes3(p0.y, p1.y, p2.y, sa, vM); x3 = planes3(p0.y, p1.y, p2.y, sb, vM);
+                  y0 = planes3(p0.z, p1.z, p2.z, sa, vM); y2 = planes3(p0.z, p1.z, p2.z, sb, vM);
+                  y1 = planes3(p0.w, p1.w, p2.w, sa, vM); y3 = planes3(p0.w, p1.w, p2.w, sb, vM);
+                } else {
+                  uint4 w = *reinterpret_cast<const uint4*>(vc[tt] + tw * D + 32 * j + 4 * g);
+                  if (BITS == 1) {
+                    w.x >>= s0; w.y >>= s0; w.z >>= s0; w.w >>= s0;
+                  }
+                  x0 = w.x & vM; x2 = (w.x >> SH) & vM;
+                  x1 = w.y & vM; x3 = (w.y >> SH) & vM;
+                  y0 = w.z & vM; y2 = (w.z >> SH) & vM;
+                  y1 = w.w & vM; y3 = (w.w >> SH) & vM;
                 }
-                const uint32_t x0 = w.x & vM, x2 = (w.x >> SH) & vM;
-                const uint32_t x1 = w.y & vM, x3 = (w.y >> SH) & vM;
-                const uint32_t y0 = w.z & vM, y2 = (w.z >> SH) & vM;
-                const uint32_t y1 = w.w & vM, y3 = (w.w >> SH) & vM;
 #pragma unroll
                 for (int p = 0; p < NPB; ++p) {
                   const uint2 bb = bcol ? *reinterpret_cast<const uint2*>(

@@ -63,16 +63,23 @@ __host__ __device__ inline bool store_tile(const CacheView& c, long long u, long
   return true;
 }
 
+// Codes come in blocks of E codes held in WB 32-bit words: E = 32/b codes
+// in one word (code i at bits [b i, b i + b)) for b = 1, 2, 4; at 3 bits,
+// which do not divide 32, E = 32 codes as three bit planes (word p holds bit
+// p of code i at bit i).  Keys: a token's blocks run along its channels;
+// values: a channel's blocks run along tokens (block tb of channel d in
+// rows tb*WB .. tb*WB + WB-1 of the [.][D] value-code array).
 template <int D, int BITS>
 struct Layout {
-  static constexpr int E = 32 / BITS;       // codes per word
-  static constexpr int WK = D / E;          // key words per token
+  static constexpr int E = BITS == 3 ? 32 : 32 / BITS;  // codes per block
+  static constexpr int WB = BITS == 3 ? 3 : 1;          // words per block
+  static constexpr int WK = D / E * WB;     // key words per token
   static constexpr int NJ = D / kGv;        // value groups per token
   static constexpr uint32_t MASK = (1u << BITS) - 1u;
   static constexpr int L = (1 << BITS) - 1;  // top code
   __host__ __device__ static long long k_codes_unit(long long Tq) { return Tq * WK; }
   __host__ __device__ static long long k_meta_unit(long long Tq) { return (Tq / kG) * D; }
-  __host__ __device__ static long long v_codes_unit(long long Tq) { return (Tq / E) * D; }
+  __host__ __device__ static long long v_codes_unit(long long Tq) { return (Tq / E) * WB * D; }
   __host__ __device__ static long long v_meta_unit(long long Tq) { return Tq * NJ; }
 };
 
@@ -481,5 +488,10 @@ cudaError_t tc_dispatch_ragged(const DecodeArgs& a, cudaStream_t s, cudaEvent_t 
                                cudaEvent_t e1, int* occ);
 cudaError_t tc_dispatch_ragged_meta16(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0,
                                       cudaEvent_t e1, int* occ);
+// The 3-bit (bit-plane) instances, uniform and ragged batches.
+cudaError_t tc_dispatch_3bit(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
+                             int* occ);
+cudaError_t tc_dispatch_3bit_ragged(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0,
+                                    cudaEvent_t e1, int* occ);
 
 }  // namespace kivi

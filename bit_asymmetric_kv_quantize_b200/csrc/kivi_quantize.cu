@@ -204,6 +204,7 @@ cudaError_t append_any(const CacheView& c, int units, int D, int bits, int dtype
     if (dtype != 0) return cudaErrorInvalidValue;
     if (bits == 1) return append_d<1, __half, __half>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
     if (bits == 2) return append_d<2, __half, __half>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
+    if (bits == 3) return append_d<3, __half, __half>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
     if (bits == 4) return append_d<4, __half, __half>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
     return cudaErrorInvalidValue;
   }
@@ -211,7 +212,9 @@ cudaError_t append_any(const CacheView& c, int units, int D, int bits, int dtype
   if (bits == 1 && dtype == 0) return append_d<1, __half, float>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
   if (bits == 1 && dtype == 1) return append_d<1, float, float>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
   if (bits == 2 && dtype == 0) return append_d<2, __half, float>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
+  if (bits == 3 && dtype == 0) return append_d<3, __half, float>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
   if (bits == 2 && dtype == 1) return append_d<2, float, float>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
+  if (bits == 3 && dtype == 1) return append_d<3, float, float>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
   if (bits == 4 && dtype == 0) return append_d<4, __half, float>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
   if (bits == 4 && dtype == 1) return append_d<4, float, float>(D, c, units, k, v, n_q, slot, flush, st, Hkv, s);
   return cudaErrorInvalidValue;
@@ -224,6 +227,7 @@ cudaError_t prefill_any(const CacheView& c, int units, int D, int bits, int dtyp
     if (dtype != 0) return cudaErrorInvalidValue;
     if (bits == 1) return prefill_d<1, __half, __half>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
     if (bits == 2) return prefill_d<2, __half, __half>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
+    if (bits == 3) return prefill_d<3, __half, __half>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
     if (bits == 4) return prefill_d<4, __half, __half>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
     return cudaErrorInvalidValue;
   }
@@ -231,7 +235,9 @@ cudaError_t prefill_any(const CacheView& c, int units, int D, int bits, int dtyp
   if (bits == 1 && dtype == 0) return prefill_d<1, __half, float>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
   if (bits == 1 && dtype == 1) return prefill_d<1, float, float>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
   if (bits == 2 && dtype == 0) return prefill_d<2, __half, float>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
+  if (bits == 3 && dtype == 0) return prefill_d<3, __half, float>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
   if (bits == 2 && dtype == 1) return prefill_d<2, float, float>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
+  if (bits == 3 && dtype == 1) return prefill_d<3, float, float>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
   if (bits == 4 && dtype == 0) return prefill_d<4, __half, float>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
   if (bits == 4 && dtype == 1) return prefill_d<4, float, float>(D, c, units, K, V, T, n_q, r, lens, st, Hkv, s);
   return cudaErrorInvalidValue;

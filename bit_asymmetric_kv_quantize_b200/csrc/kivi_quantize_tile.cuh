@@ -105,9 +105,32 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
   }
   tile_sync<D, BAR>();
   // ---- pack: keys along channels, values along tokens; D*BITS words each
-  constexpr int NW = kTile * WK;  // == (kTile / E) * D == D * BITS
+  constexpr int NW = kTile * WK;  // == (kTile / E) * WB * D == D * BITS
   uint32_t* kdst = c.k_codes + unit * Lt::k_codes_unit(Ts) + t0 * WK;
-  uint32_t* vdst = c.v_codes + unit * Lt::v_codes_unit(Ts) + (t0 / E) * D;
+  uint32_t* vdst = c.v_codes + unit * Lt::v_codes_unit(Ts) + (t0 / E) * Lt::WB * D;
+  if constexpr (BITS == 3) {
+    // bit planes: lane i of a warp holds code i of a block; plane p is the
+    // ballot of bit p (bit i of the word = bit p of code i)
+    const int lane = tid & 31, wp = tid >> 5;
+    constexpr int NWP = D / 32;  // warps
+    for (int pb = wp; pb < kTile * (D / 32); pb += NWP) {  // keys: (token, block)
+      const int t = pb / (D / 32), w = pb % (D / 32);
+      const uint32_t cd = ck[t * D + w * 32 + lane];
+      const uint32_t p0 = __ballot_sync(0xffffffffu, cd & 1u);
+      const uint32_t p1 = __ballot_sync(0xffffffffu, cd & 2u);
+      const uint32_t p2 = __ballot_sync(0xffffffffu, cd & 4u);
+      if (lane < 3) kdst[t * WK + 3 * w + lane] = lane == 0 ? p0 : (lane == 1 ? p1 : p2);
+    }
+    for (int d = wp; d < D; d += NWP) {  // values: channel d, the tile's 32 tokens
+      const uint32_t cd = cv[lane * D + d];
+      const uint32_t p0 = __ballot_sync(0xffffffffu, cd & 1u);
+      const uint32_t p1 = __ballot_sync(0xffffffffu, cd & 2u);
+      const uint32_t p2 = __ballot_sync(0xffffffffu, cd & 4u);
+      if (lane < 3) vdst[lane * D + d] = lane == 0 ? p0 : (lane == 1 ? p1 : p2);
+    }
+    tile_sync<D, BAR>();
+    return;
+  }
 #pragma unroll
   for (int k = tid; k < NW; k += D) {
     const int t = k / WK, w = k % WK;

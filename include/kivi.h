@@ -50,6 +50,12 @@
  * Each code packs along the axis its attention product contracts over
  * (channels for keys, tokens for values).  "meta" is binary32 (float), or
  * binary16 when dims.meta = KIVI_META_F16 (see kivi_meta).
+ * 3 bits (a format variant; 3 does not divide 32): codes come in blocks of
+ * E = 32 held as three bit-plane words, plane p holding bit p of code i in
+ * its bit i.  k_codes [B][Hkv][Tq][D/32*3]: block w of token t (channels
+ * 32w..32w+31) in words 3w..3w+2; v_codes [B][Hkv][Tq/32*3][D]: block tb of
+ * channel d (tokens 32tb..32tb+31) in rows 3tb..3tb+2.  (KVQuant page,
+ * abstract: 3-bit KV cache quantization.)
  *
  * Quantizer (fixed binary32 formula; codes, scales and zeros are bit-exact
  * functions of the inputs): for a group x_0..x_{n-1},
@@ -107,7 +113,9 @@ typedef enum { KIVI_F16 = 0, KIVI_F32 = 1 } kivi_dtype;
  * storage precision for them.) */
 typedef enum { KIVI_META_F32 = 0, KIVI_META_F16 = 1 } kivi_meta;
 
-/* Shape of one cache (one attention layer).  Supported: bits in {1, 2, 4},
+/* Shape of one cache (one attention layer).  Supported: bits in {1, 2, 3, 4}
+ * (3 bits: the tensor-core decode only; kivi_decode_attention_simt refuses
+ * it with KIVI_ERR_UNSUPPORTED),
  * G = 32, Gv = 32, D in {32, 64, 128}, R a positive multiple of 32,
  * capacity a positive multiple of R, dtype KIVI_F16 or KIVI_F32, meta
  * KIVI_META_F32 or (with dtype KIVI_F16) KIVI_META_F16.  A zero-filled

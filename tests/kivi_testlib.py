@@ -47,7 +47,7 @@ def assert_state_equal(gc: kivi.KiviCache, oc: oracle.OracleCache, units=None):
     """Bit-exact comparison of the quantized store and the window on `units`."""
     units = oc.units if units is None else units
     n_q, r = gc.n_q, gc.r
-    E = 32 // gc.bits
+    E, WB = (32, 3) if gc.bits == 3 else (32 // gc.bits, 1)
     for (b, h) in units:
         u = oc.unit(b, h)
         assert (u.n_q, u.r) == (n_q, r), ((b, h), (u.n_q, u.r), (n_q, r))
@@ -59,7 +59,7 @@ def assert_state_equal(gc: kivi.KiviCache, oc: oracle.OracleCache, units=None):
         t = gc.view(name)[bs]
         g[name] = t.float().cpu().numpy() if t.is_floating_point() else t.cpu().numpy()
     bi = {b: i for i, b in enumerate(bs)}
-    lim = {"k_codes": n_q, "k_scale": n_q // 32, "k_zero": n_q // 32, "v_codes": n_q // E, "v_scale": n_q, "v_zero": n_q,
+    lim = {"k_codes": n_q, "k_scale": n_q // 32, "k_zero": n_q // 32, "v_codes": n_q // E * WB, "v_scale": n_q, "v_zero": n_q,
            "k_res": r, "v_res": r}
     for (b, h) in units:
         i = oc.slot(b, h)

@@ -39,22 +39,27 @@ def _dims(**kw):
                     d["dtype"], d["meta"])
 
 
+def _block(bits):
+    """(codes per block, words per block): 32 codes as three bit planes at 3 bits."""
+    return (32, 3) if bits == 3 else (32 // bits, 1)
+
+
 def _sizes(dims):
     out = (ctypes.c_size_t * 8)()
     rc = kivi.lib().kivi_buffer_sizes(ctypes.byref(dims), ctypes.byref(out))
     return rc, list(out)
 
 
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_buffer_sizes_follow_the_layout(bits, D):
     B, H, R, cap = 3, 5, 64, 640
     rc, s = _sizes(_dims(B=B, Hkv=H, D=D, bits=bits, R=R, capacity=cap))
     assert rc == 0
-    E, Tq, u = 32 // bits, cap - R, B * H
-    assert s[0] == u * Tq * (D // E) * 4           # k_codes
+    (E, WB), Tq, u = _block(bits), cap - R, B * H
+    assert s[0] == u * Tq * (D // E) * WB * 4      # k_codes
     assert s[1] == s[2] == u * (Tq // 32) * D * 4  # k_scale, k_zero
-    assert s[3] == u * (Tq // E) * D * 4           # v_codes
+    assert s[3] == u * (Tq // E) * WB * D * 4      # v_codes
     assert s[4] == s[5] == u * Tq * (D // 32) * 4  # v_scale, v_zero
     assert s[6] == s[7] == u * R * D * 2           # k_res, v_res (fp16)
     # 2-bit codes + fp32 scale/zero per 32: 0.5 byte per key and per value element
@@ -62,7 +67,7 @@ def test_buffer_sizes_follow_the_layout(bits, D):
         assert sum(s[:6]) == u * Tq * D * 2 * 0.5
 
 
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_binary16_metadata_halves_the_scale_and_zero_buffers(bits, D):
     B, H, R, cap = 3, 5, 64, 640
@@ -91,7 +96,7 @@ def test_dims_struct_matches_the_header():
 @pytest.mark.parametrize("kw,rc", [
     (dict(meta=2), ERR_UNSUPPORTED), (dict(meta=-1), ERR_UNSUPPORTED),
     (dict(meta=kivi.KIVI_META_F16, dtype=kivi.KIVI_F32), ERR_UNSUPPORTED),
-    (dict(bits=3), ERR_UNSUPPORTED), (dict(bits=8), ERR_UNSUPPORTED),
+    (dict(bits=5), ERR_UNSUPPORTED), (dict(bits=8), ERR_UNSUPPORTED),
     (dict(G=16), ERR_UNSUPPORTED), (dict(Gv=64), ERR_UNSUPPORTED),
     (dict(D=96), ERR_UNSUPPORTED), (dict(R=48), ERR_UNSUPPORTED),
     (dict(capacity=4100), ERR_UNSUPPORTED), (dict(dtype=7), ERR_UNSUPPORTED),
@@ -246,17 +251,17 @@ def test_cache_struct_matches_the_header():
     assert declared == names
 
 
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 def test_paged_buffer_sizes(bits):
     B, H, D, R, P = 3, 5, 128, 64, 11
     dims = _dims(B=B, Hkv=H, D=D, bits=bits, R=R, capacity=4 * R)
     out = (ctypes.c_size_t * 8)()
     assert kivi.lib().kivi_paged_buffer_sizes(ctypes.byref(dims), P, ctypes.byref(out)) == 0
-    E = 32 // bits
+    E, WB = _block(bits)
     s = list(out)
-    assert s[0] == P * H * R * (D // E) * 4
+    assert s[0] == P * H * R * (D // E) * WB * 4
     assert s[1] == s[2] == P * H * (R // 32) * D * 4
-    assert s[3] == P * H * (R // E) * D * 4
+    assert s[3] == P * H * (R // E) * WB * D * 4
     assert s[4] == s[5] == P * H * R * (D // 32) * 4
     assert s[6] == s[7] == B * H * R * D * 2
     assert kivi.lib().kivi_paged_buffer_sizes(ctypes.byref(dims), 0, ctypes.byref(out)) == ERR_ARG
@@ -291,7 +296,7 @@ def test_paged_cache_init_and_refusals():
     assert (c2.block_table, c2.pages_per_seq, c2.num_pages) == (None, 0, 0)
 
 
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 def test_paged_pool_with_binary16_metadata(bits):
     B, H, D, R, P = 2, 3, 64, 32, 9
     out = (ctypes.c_size_t * 8)()
@@ -302,14 +307,23 @@ def test_paged_pool_with_binary16_metadata(bits):
     s32 = list(out)
     assert L.kivi_paged_buffer_sizes(ctypes.byref(d16), P, ctypes.byref(out)) == 0
     s16 = list(out)
-    E = 32 // bits
-    assert s16[0] == s32[0] == P * H * R * (D // E) * 4
+    E, WB = _block(bits)
+    assert s16[0] == s32[0] == P * H * R * (D // E) * WB * 4
     for i in (1, 2, 4, 5):
         assert 2 * s16[i] == s32[i]
     assert s16[6] == s32[6] == B * H * R * D * 2
 
 
 def test_code_widths_the_library_builds():
-    # 1, 2 and 4 bits run on the GPU; 3 bits exists in the oracle only
-    for bits, rc in ((1, 0), (2, 0), (4, 0), (3, ERR_UNSUPPORTED), (8, ERR_UNSUPPORTED)):
+    # 1, 2, 3 (bit planes) and 4 bits run on the GPU
+    for bits, rc in ((1, 0), (2, 0), (3, 0), (4, 0), (5, ERR_UNSUPPORTED), (8, ERR_UNSUPPORTED)):
         assert _sizes(_dims(bits=bits))[0] == rc, bits
+
+
+def test_three_bit_codes_are_three_planes_per_32():
+    # 3 bits: 32 codes in three words, i.e. 3/8 byte per code as at 3 bits per code
+    B, H, D, R, cap = 2, 3, 128, 64, 640
+    rc, s = _sizes(_dims(B=B, Hkv=H, D=D, bits=3, R=R, capacity=cap))
+    assert rc == 0
+    u, Tq = B * H, cap - R
+    assert s[0] == s[3] == u * Tq * D * 3 // 8

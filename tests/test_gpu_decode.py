@@ -44,9 +44,11 @@ def run(w, kernel, sigma=None, capacity=None):
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("gq", [1, 2, 4, 8])
 @pytest.mark.parametrize("dtype", ["f16", "f32"])
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_decode_shapes(D, bits, dtype, gq, kernel):
+    if bits == 3 and kernel == "simt":
+        pytest.skip("3-bit codes: tensor-core decode only")
     for T in (1, 33, 161, 1000):
         w = small(D=D, bits=bits, dtype=dtype, gq=gq, T=T)
         gc, oc, q, out, sigma = run(w, kernel, capacity=1024)
@@ -237,8 +239,9 @@ def test_device_counter_loop_matches_host_counters(dtype, D, gq):
         assert torch.equal(out_d, out_h), f"step {step}"
     dev.load_dev_state(st)
     assert (dev.n_q, dev.r) == (host.n_q, host.r) == (192, 58)
-    n_q, r, E = dev.n_q, dev.r, 32 // w.bits
-    used = {"k_codes": n_q, "k_scale": n_q // w.G, "k_zero": n_q // w.G, "v_codes": n_q // E,
+    n_q, r = dev.n_q, dev.r
+    E, WB = (32, 3) if w.bits == 3 else (32 // w.bits, 1)
+    used = {"k_codes": n_q, "k_scale": n_q // w.G, "k_zero": n_q // w.G, "v_codes": n_q // E * WB,
             "v_scale": n_q, "v_zero": n_q, "k_res": r, "v_res": r}
     for name, n in used.items():
         assert torch.equal(dev.view(name)[:, :, :n], host.view(name)[:, :, :n]), name
@@ -400,3 +403,27 @@ def test_fused_steps_are_one_launch_each_flushes_included(dtype):
     dev.load_dev_state(st)
     assert (dev.n_q, dev.r) == (fused.n_q, fused.r) == (ref.n_q, ref.r)
     assert_state_equal(fused, oc)
+
+
+
+@pytest.mark.parametrize("gq", [1, 4, 8])
+def test_three_bit_layer_sampled(gq):
+    """3-bit codes (bit planes) on a layer-sized cache: store bit-exact and
+    decode within the bars on sampled units, with fused steps across a flush."""
+    w = W.Workload(f"three-bit-g{gq}", B=4, Hq=8 * gq, Hkv=8, D=128, T=3000, bits=3, R=128, seed=31)
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w, capacity=3200)
+    gc.prefill(K, V)
+    units = sample_units(w, 8, seed=gq)
+    oc = oracle_cache(w, units=units, capacity=3200)
+    oracle_prefill(oc, K, V)
+    assert_state_equal(gc, oc, units)
+    sigma = 1.0 / math.sqrt(w.D)
+    for step in range(130):  # the window (r = 56) fills and flushes once
+        k, v = W.step_kv(w, step, device="cuda")
+        q = W.query(w, step, device="cuda")
+        out = gc.append_decode(k, v, q, sigma)
+        oracle_append(oc, k, v)
+        if step % 40 == 0 or step == 129:
+            assert_decode_close(out, oc, q, sigma, units)
+    assert_state_equal(gc, oc, units)

@@ -35,7 +35,7 @@ def test_metadata_buffers_are_binary16():
         gpu_cache(w.with_(dtype="f32"), capacity=256)  # binary16 metadata needs an fp16 cache
 
 
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 @pytest.mark.parametrize("T", [1, 64, 65, 129, 333])
 def test_prefill_bit_exact(D, bits, T):
@@ -48,7 +48,7 @@ def test_prefill_bit_exact(D, bits, T):
     assert_state_equal(gc, oc)
 
 
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 def test_append_and_flush_bit_exact(bits):
     R = 32
     w = small(D=128, bits=bits, R=R, T=R + 5)
@@ -107,9 +107,11 @@ def test_rounding_edge_cases_bit_exact():
 
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("gq", [1, 2, 4, 8])
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_decode_shapes(D, bits, gq, kernel):
+    if bits == 3 and kernel == "simt":
+        pytest.skip("3-bit codes: tensor-core decode only")
     for T in (1, 33, 161, 1000):
         w = small(D=D, bits=bits, gq=gq, T=T)
         K, V = W.prompt_kv(w, device="cuda")

@@ -60,9 +60,9 @@ def assert_paged_equal_oracle(pc, st, oc):
         u = oc.unit(b, h)
         assert status[b] == 0 and (n_q[b], r[b]) == (u.n_q, u.r), (b, h)
         got = gather_unit(pc, b, h, u.n_q, u.r)
-        E = 32 // pc.bits
+        E, WB = (32, 3) if pc.bits == 3 else (32 // pc.bits, 1)
         lim = {"k_codes": u.n_q, "k_scale": u.n_q // 32, "k_zero": u.n_q // 32,
-               "v_codes": u.n_q // E, "v_scale": u.n_q, "v_zero": u.n_q, "k_res": u.r, "v_res": u.r}
+               "v_codes": u.n_q // E * WB, "v_scale": u.n_q, "v_zero": u.n_q, "k_res": u.r, "v_res": u.r}
         i = oc.slot(b, h)
         for name, n in lim.items():
             g = np.ascontiguousarray(got[name]).view(np.uint32)
@@ -86,7 +86,7 @@ def prefill_three(w, lens, pps, num_pages, units=None, seed=0):
 
 @pytest.mark.parametrize("meta", ["f32", "f16"])
 @pytest.mark.parametrize("gq", [1, 4, 8])
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_prefill_and_decode(D, bits, gq, meta):
     w = small(D=D, bits=bits, gq=gq, T=700, B=5, meta=meta)

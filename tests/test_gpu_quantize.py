@@ -25,7 +25,7 @@ def small(D=64, bits=2, dtype="f16", R=64, T=200, B=2, Hkv=3, gq=1, capacity=512
 
 
 @pytest.mark.parametrize("dtype", ["f16", "f32"])
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 @pytest.mark.parametrize("T", [1, 31, 64, 65, 127, 128, 129, 333])
 def test_prefill_bit_exact(D, bits, dtype, T):
@@ -39,7 +39,7 @@ def test_prefill_bit_exact(D, bits, dtype, T):
     assert_state_equal(gc, oc)
 
 
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("R", [32, 128])
 def test_append_and_flush_bit_exact(bits, R):
     """Prefill, then appends across several window flushes; the state matches

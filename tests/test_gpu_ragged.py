@@ -52,7 +52,7 @@ def assert_ragged_state_equal(gc, st, oc, units=None):
     """Counters and every unit's store and window, bit for bit, at its own fill."""
     units = oc.units if units is None else units
     n_q, r, status = kivi.ragged_lengths(st)
-    E = 32 // gc.bits
+    E, WB = (32, 3) if gc.bits == 3 else (32 // gc.bits, 1)
     bufs = {}
     for name in kivi.BUFFER_NAMES:
         t = gc.view(name)
@@ -62,7 +62,7 @@ def assert_ragged_state_equal(gc, st, oc, units=None):
         assert status[b] == 0, (b, status[b])
         assert (n_q[b], r[b]) == (u.n_q, u.r), ((b, h), (n_q[b], r[b]), (u.n_q, u.r))
         lim = {"k_codes": u.n_q, "k_scale": u.n_q // 32, "k_zero": u.n_q // 32,
-               "v_codes": u.n_q // E, "v_scale": u.n_q, "v_zero": u.n_q, "k_res": u.r, "v_res": u.r}
+               "v_codes": u.n_q // E * WB, "v_scale": u.n_q, "v_zero": u.n_q, "k_res": u.r, "v_res": u.r}
         i = oc.slot(b, h)
         for name in kivi.BUFFER_NAMES:
             n = lim[name]
@@ -96,7 +96,7 @@ def test_prefill_lengths_and_refusals():
 @pytest.mark.parametrize("meta", ["f32", "f16"])
 @pytest.mark.parametrize("gq", [1, 2, 4, 8])
 @pytest.mark.parametrize("dtype", ["f16", "f32"])
-@pytest.mark.parametrize("bits", [1, 2, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("D", [32, 64, 128])
 def test_decode_shapes(D, bits, dtype, gq, meta):
     if meta == "f16" and dtype == "f32":
@@ -151,8 +151,8 @@ def test_uniform_lengths_match_the_uniform_path():
         assert (oa.float() - ob.float()).abs().max().item() <= 2e-3
     n_q, r, status = kivi.ragged_lengths(st)
     assert set(n_q) == {a.n_q} and set(r) == {a.r} and set(status) == {0}
-    E = 32 // w.bits
-    used = {"k_codes": a.n_q, "k_scale": a.n_q // 32, "k_zero": a.n_q // 32, "v_codes": a.n_q // E,
+    E, WB = (32, 3) if w.bits == 3 else (32 // w.bits, 1)
+    used = {"k_codes": a.n_q, "k_scale": a.n_q // 32, "k_zero": a.n_q // 32, "v_codes": a.n_q // E * WB,
             "v_scale": a.n_q, "v_zero": a.n_q, "k_res": a.r, "v_res": a.r}
     for name, n in used.items():
         assert torch.equal(a.view(name)[:, :, :n], b.view(name)[:, :, :n]), name
