@@ -81,6 +81,9 @@ def parse():
                         "consecutive per sequence")
     p.add_argument("--bits", type=int, choices=[1, 2, 3, 4], default=None,
                    help="code width other than the workload's (a format variant)")
+    p.add_argument("--outliers", default="0,0",
+                   help="dense-and-sparse variant: entries kept exactly per key group and per "
+                        "value group, 'k,v' (the inputs get 1%% spiked entries, x4)")
     p.add_argument("--meta", choices=["f32", "f16"], default="f32",
                    help="scale/zero storage: binary32, or the binary16 format variant "
                         "(fp16 workloads)")
@@ -101,6 +104,9 @@ def bench_workload(args, name=None) -> W.Workload:
         w = w.with_(steps=0)
     if args.meta == "f16":
         w = w.with_(meta="f16", name=w.name + "-meta16")
+    ko, vo = (int(x) for x in args.outliers.split(","))
+    if ko or vo:
+        w = w.with_(spike_frac=0.01, spike_scale=4.0, name=f"{w.name}-sparse{ko}x{vo}")
     if args.bits is not None and args.bits != w.bits:
         base = w.name[:-len("-2bit")] if w.name.endswith("-2bit") else w.name
         w = w.with_(bits=args.bits, name=f"{base}-{args.bits}bit")
@@ -161,7 +167,7 @@ def profiled_traffic(w: W.Workload):
     return None
 
 
-def algorithmic_bytes(w: W.Workload, n_q: int, r: int) -> int:
+def algorithmic_bytes(w: W.Workload, n_q: int, r: int, outliers=(0, 0)) -> int:
     """Bytes one decode call must move: every code, scale and zero of the
     quantized store, the window tokens, q in and out (per unit: K codes
     n_q*D*b/8, K meta (n_q/G)*D*2*ms, V codes n_q*D*b/8, V meta
@@ -169,10 +175,12 @@ def algorithmic_bytes(w: W.Workload, n_q: int, r: int) -> int:
     ms = 4, or 2 with binary16 scales and zeros)."""
     es = 2 if w.dtype == "f16" else 4
     ms = 2 if w.meta == "f16" else 4
+    ko, vo = outliers  # dense-and-sparse lists: an int32 index and a binary32 value per entry
 
     def per_unit(nq, rr):
         return (2 * nq * w.D * w.bits // 8 + (nq // w.G) * w.D * 2 * ms
-                + nq * (w.D // w.Gv) * 2 * ms + rr * w.D * 2 * es)
+                + nq * (w.D // w.Gv) * 2 * ms + rr * w.D * 2 * es
+                + 8 * ((nq // w.G) * w.D * ko + nq * (w.D // w.Gv) * vo))
 
     io = 2 * w.B * w.Hq * w.D * es
     if isinstance(n_q, (list, tuple)):  # ragged: one (n_q, r) per sequence
@@ -287,6 +295,7 @@ def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, f
     import torch.distributed as dist
 
     ragged = w.len_min > 0
+    outliers = tuple(int(x) for x in args.outliers.split(","))
     if args.paged:
         w = w.with_(name=f"{w.name}-paged-{args.paged}")
     if ragged and (args.kernel != "default" or args.unfused):
@@ -319,7 +328,8 @@ def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, f
                                     meta=w.torch_meta)
         else:
             c = kivi.KiviCache(w.B, w.Hkv, w.D, w.bits, capacity, R=w.R, G=w.G, Gv=w.Gv,
-                               dtype=w.torch_dtype, device=device, meta=w.torch_meta)
+                               dtype=w.torch_dtype, device=device, meta=w.torch_meta,
+                               outliers=outliers)
         pe = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
         pe[0].record()
         if ragged:
@@ -476,7 +486,7 @@ def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, f
     ms_max = max_over_ranks(ms, world, device)
 
     # roofline of the split kernel: algorithmic bytes / event time
-    bytes_total = sum(algorithmic_bytes(w, nq, r) for nq, r in fills)
+    bytes_total = sum(algorithmic_bytes(w, nq, r, outliers) for nq, r in fills)
     # tokens attended per step (summed over sequences, per KV head), mean over the fills
     ctx_tokens = statistics.mean((sum(nq) + sum(r)) if isinstance(nq, list) else w.B * (nq + r)
                                  for nq, r in fills)
@@ -540,6 +550,8 @@ def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, f
                 "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                 "context": w.T, "bits": w.bits, "G": w.G, "Gv": w.Gv, "R": w.R,
                 "dtype_io": w.dtype, "meta": w.meta, "kernel": args.kernel,
+                **({"outliers_per_group": {"keys": outliers[0], "values": outliers[1]}}
+                   if any(outliers) else {}),
                 **({"paged": f"pages of {w.R} tokens, {args.paged} block table"}
                    if args.paged else {}),
                 "step": ("kivi_ragged_append_decode" if ragged else

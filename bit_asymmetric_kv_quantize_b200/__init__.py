@@ -36,7 +36,9 @@ EXPORTED = (
     "kivi_decode_attention_noalloc", "kivi_append_decode", "kivi_dev_state_init",
     "kivi_append_decode_dev", "kivi_ragged_prefill", "kivi_ragged_append", "kivi_ragged_decode",
     "kivi_ragged_append_decode", "kivi_paged_buffer_sizes", "kivi_paged_cache_init",
+    "kivi_outlier_buffer_sizes", "kivi_cache_set_outliers",
 )
+OUTLIER_NAMES = ("k_out_idx", "k_out_val", "v_out_idx", "v_out_val")
 
 
 class KiviError(RuntimeError):
@@ -49,7 +51,7 @@ class KiviDims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("D", ctypes.c_int),
                 ("bits", ctypes.c_int), ("G", ctypes.c_int), ("Gv", ctypes.c_int),
                 ("R", ctypes.c_int), ("capacity", ctypes.c_longlong), ("dtype", ctypes.c_int),
-                ("meta", ctypes.c_int)]
+                ("meta", ctypes.c_int), ("k_out", ctypes.c_int), ("v_out", ctypes.c_int)]
 
 
 class KiviCacheC(ctypes.Structure):
@@ -60,7 +62,9 @@ class KiviCacheC(ctypes.Structure):
                 ("k_res", ctypes.c_void_p), ("v_res", ctypes.c_void_p),
                 ("n_q", ctypes.c_longlong), ("r", ctypes.c_int),
                 ("block_table", ctypes.c_void_p), ("pages_per_seq", ctypes.c_int),
-                ("num_pages", ctypes.c_longlong)]
+                ("num_pages", ctypes.c_longlong),
+                ("k_out_idx", ctypes.c_void_p), ("k_out_val", ctypes.c_void_p),
+                ("v_out_idx", ctypes.c_void_p), ("v_out_val", ctypes.c_void_p)]
 
 
 _lock = threading.Lock()
@@ -100,6 +104,8 @@ def lib() -> ctypes.CDLL:
                                                     sz, vp]
             L.kivi_paged_buffer_sizes.argtypes = [dp, ll, ctypes.POINTER(sz * NUM_BUFFERS)]
             L.kivi_paged_cache_init.argtypes = [cp, dp, ctypes.POINTER(vp * NUM_BUFFERS), vp, ci, ll]
+            L.kivi_outlier_buffer_sizes.argtypes = [dp, ctypes.POINTER(sz * 4)]
+            L.kivi_cache_set_outliers.argtypes = [cp, ctypes.POINTER(vp * 4)]
             L.kivi_set_timing_events.argtypes = [vp, vp]
             L.kivi_set_timing_events.restype = None
             L.kivi_decode_num_splits.argtypes = [cp, ci]
@@ -139,8 +145,9 @@ def _check(rc: int, what: str) -> None:
 
 
 def buffer_sizes(B, Hkv, D, bits, capacity, R=128, G=32, Gv=32, dtype=torch.float16,
-                 meta=torch.float32):
-    dims = KiviDims(B, Hkv, D, bits, G, Gv, R, capacity, _dtype_code(dtype), _meta_code(meta))
+                 meta=torch.float32, outliers=(0, 0)):
+    dims = KiviDims(B, Hkv, D, bits, G, Gv, R, capacity, _dtype_code(dtype), _meta_code(meta),
+                    int(outliers[0]), int(outliers[1]))
     out = (ctypes.c_size_t * NUM_BUFFERS)()
     _check(lib().kivi_buffer_sizes(ctypes.byref(dims), ctypes.byref(out)), "kivi_buffer_sizes")
     return dict(zip(BUFFER_NAMES, list(out)))
@@ -158,7 +165,7 @@ class KiviCache:
 
     def __init__(self, B: int, Hkv: int, D: int, bits: int, capacity: int, R: int = 128,
                  G: int = 32, Gv: int = 32, dtype: torch.dtype = torch.float16,
-                 device="cuda", meta: torch.dtype = torch.float32):
+                 device="cuda", meta: torch.dtype = torch.float32, outliers=(0, 0)):
         self.device = torch.device(device)
         if self.device.type != "cuda":
             raise ValueError("KiviCache lives in CUDA device memory")
@@ -166,19 +173,30 @@ class KiviCache:
             self.device = torch.device("cuda", torch.cuda.current_device())
         self.dtype = dtype
         self.meta = meta
+        ko, vo = (int(outliers[0]), int(outliers[1]))
         self._dims = KiviDims(B, Hkv, D, bits, G, Gv, R, capacity, _dtype_code(dtype),
-                              _meta_code(meta))
-        sizes = buffer_sizes(B, Hkv, D, bits, capacity, R, G, Gv, dtype, meta)
+                              _meta_code(meta), ko, vo)
+        sizes = buffer_sizes(B, Hkv, D, bits, capacity, R, G, Gv, dtype, meta, outliers)
         self.buffers = {n: torch.empty(max(sizes[n], 16), dtype=torch.uint8, device=self.device)
                         for n in BUFFER_NAMES}
         ptrs = (ctypes.c_void_p * NUM_BUFFERS)(*[self.buffers[n].data_ptr() for n in BUFFER_NAMES])
         self._c = KiviCacheC()
         _check(lib().kivi_cache_init(ctypes.byref(self._c), ctypes.byref(self._dims),
                                      ctypes.byref(ptrs)), "kivi_cache_init")
+        Tq = capacity - R
+        self.outliers = (ko, vo)
+        if ko or vo:  # dense-and-sparse variant: the four list buffers
+            osz = (ctypes.c_size_t * 4)()
+            _check(lib().kivi_outlier_buffer_sizes(ctypes.byref(self._dims), ctypes.byref(osz)),
+                   "kivi_outlier_buffer_sizes")
+            for n, s in zip(OUTLIER_NAMES, list(osz)):
+                self.buffers[n] = torch.empty(max(s, 16), dtype=torch.uint8, device=self.device)
+            optrs = (ctypes.c_void_p * 4)(*[self.buffers[n].data_ptr() for n in OUTLIER_NAMES])
+            _check(lib().kivi_cache_set_outliers(ctypes.byref(self._c), ctypes.byref(optrs)),
+                   "kivi_cache_set_outliers")
         self._ws: Optional[torch.Tensor] = None
         self._ws_dev: Optional[torch.Tensor] = None
         E, WB = _code_block(bits)
-        Tq = capacity - R
         self.B, self.Hkv, self.D, self.bits, self.R, self.capacity = B, Hkv, D, bits, R, capacity
         self.shapes = {
             "k_codes": ((B, Hkv, Tq, D // E * WB), torch.int32),
@@ -190,6 +208,13 @@ class KiviCache:
             "k_res": ((B, Hkv, R, D), dtype),
             "v_res": ((B, Hkv, R, D), dtype),
         }
+        if ko or vo:
+            self.shapes.update({
+                "k_out_idx": ((B, Hkv, Tq // G, D, max(ko, 1)), torch.int32),
+                "k_out_val": ((B, Hkv, Tq // G, D, max(ko, 1)), torch.float32),
+                "v_out_idx": ((B, Hkv, Tq, D // Gv, max(vo, 1)), torch.int32),
+                "v_out_val": ((B, Hkv, Tq, D // Gv, max(vo, 1)), torch.float32),
+            })
 
     # -- state
     @property

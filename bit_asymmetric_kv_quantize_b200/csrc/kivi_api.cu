@@ -33,8 +33,15 @@ int check_dims(const kivi_dims* d) {
   if (d->meta != KIVI_META_F32 && d->meta != KIVI_META_F16) return KIVI_ERR_UNSUPPORTED;
   if (d->meta == KIVI_META_F16 && d->dtype != KIVI_F16) return KIVI_ERR_UNSUPPORTED;
   if ((long long)d->B * d->Hkv > 65535) return KIVI_ERR_UNSUPPORTED;  // grid y limit
+  // dense-and-sparse variant: a few kept entries per group, binary32 metadata
+  if (d->k_out < 0 || d->v_out < 0) return KIVI_ERR_ARG;
+  if (d->k_out > kivi::kMaxOut || d->v_out > kivi::kMaxOut) return KIVI_ERR_UNSUPPORTED;
+  if ((d->k_out > 0 || d->v_out > 0) && (d->meta != KIVI_META_F32 || d->bits == 3))
+    return KIVI_ERR_UNSUPPORTED;
   return KIVI_OK;
 }
+
+bool sparse(const kivi_dims& d) { return d.k_out > 0 || d.v_out > 0; }
 
 // n_q of a cache filled by kivi_ragged_prefill: its counters live in the
 // caller's device state, and the host-counter calls refuse it.
@@ -52,6 +59,9 @@ int check_cache(const kivi_cache* c) {
                  !c->v_zero))
     return KIVI_ERR_ARG;
   if (!c->k_res || !c->v_res) return KIVI_ERR_ARG;
+  if (Tq > 0 && ((c->dims.k_out > 0 && (!c->k_out_idx || !c->k_out_val)) ||
+                 (c->dims.v_out > 0 && (!c->v_out_idx || !c->v_out_val))))
+    return KIVI_ERR_ARG;  // the outlier lists are not bound
   return KIVI_OK;
 }
 
@@ -75,6 +85,12 @@ CacheView view(const kivi_cache* c) {
   v.pps = c->pages_per_seq;
   v.n_pages = c->num_pages;
   v.Hkv = c->dims.Hkv;
+  v.k_out = c->dims.k_out;
+  v.v_out = c->dims.v_out;
+  v.k_oi = c->k_out_idx;
+  v.k_ov = c->k_out_val;
+  v.v_oi = c->v_out_idx;
+  v.v_ov = c->v_out_val;
   return v;
 }
 
@@ -266,7 +282,8 @@ int decode_common(const kivi_cache* c, const void* q, int Hq, float softmax_scal
                   void* workspace, size_t ws_bytes, void* stream, bool simt) {
   int rc = decode_checks(c, q, Hq, out);
   if (rc) return rc;
-  if (simt && c->dims.bits == 3) return KIVI_ERR_UNSUPPORTED;  // CUDA-core kernel: 1, 2, 4 bits
+  // the CUDA-core kernel: 1, 2, 4 bits, plain codes
+  if (simt && (c->dims.bits == 3 || sparse(c->dims))) return KIVI_ERR_UNSUPPORTED;
   const int sms = device_sms();
   if (sms <= 0) return KIVI_ERR_CUDA;
   if (!workspace || ((uintptr_t)workspace & 15) || ws_bytes < workspace_bytes(c->dims, Hq, sms))
@@ -363,6 +380,42 @@ int kivi_cache_init(kivi_cache* cache, const kivi_dims* dims,
   cache->block_table = nullptr;
   cache->pages_per_seq = 0;
   cache->num_pages = 0;
+  cache->k_out_idx = nullptr;
+  cache->k_out_val = nullptr;
+  cache->v_out_idx = nullptr;
+  cache->v_out_val = nullptr;
+  return KIVI_OK;
+}
+
+int kivi_outlier_buffer_sizes(const kivi_dims* dims, size_t out_bytes[4]) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!out_bytes) return KIVI_ERR_ARG;
+  const long long units = (long long)dims->B * dims->Hkv;
+  const long long Tq = dims->capacity - dims->R;
+  out_bytes[0] = (size_t)(units * (Tq / dims->G) * dims->D * dims->k_out) * 4;
+  out_bytes[1] = out_bytes[0];
+  out_bytes[2] = (size_t)(units * Tq * (dims->D / dims->Gv) * dims->v_out) * 4;
+  out_bytes[3] = out_bytes[2];
+  return KIVI_OK;
+}
+
+int kivi_cache_set_outliers(kivi_cache* cache, void* const buffers[4]) {
+  if (!cache || !buffers) return KIVI_ERR_ARG;
+  int rc = check_dims(&cache->dims);
+  if (rc) return rc;
+  if (!sparse(cache->dims) || cache->block_table) return KIVI_ERR_UNSUPPORTED;
+  if (cache->n_q != 0 || cache->r != 0) return KIVI_ERR_STATE;
+  const bool has_store = cache->dims.capacity > cache->dims.R;
+  for (int i = 0; i < 4; ++i) {
+    const bool needed = has_store && (i < 2 ? cache->dims.k_out > 0 : cache->dims.v_out > 0);
+    if (needed && !buffers[i]) return KIVI_ERR_ARG;
+    if (((uintptr_t)buffers[i] & 15) != 0) return KIVI_ERR_ARG;
+  }
+  cache->k_out_idx = (int32_t*)buffers[0];
+  cache->k_out_val = (float*)buffers[1];
+  cache->v_out_idx = (int32_t*)buffers[2];
+  cache->v_out_val = (float*)buffers[3];
   return KIVI_OK;
 }
 
@@ -392,6 +445,7 @@ int kivi_paged_cache_init(kivi_cache* cache, const kivi_dims* dims,
   if (!cache || !buffers || !block_table || ((uintptr_t)block_table & 3)) return KIVI_ERR_ARG;
   int rc = check_dims(dims);
   if (rc) return rc;
+  if (sparse(*dims)) return KIVI_ERR_UNSUPPORTED;  // outlier lists are per unit, not paged
   if (pages_per_seq < 1 || num_pages < 1 || num_pages > (long long)INT_MAX ||
       dims->capacity != ((long long)pages_per_seq + 1) * dims->R)
     return KIVI_ERR_ARG;

@@ -8,6 +8,7 @@ namespace {
 
 cudaError_t tc_dispatch(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
                         int* occ) {
+  if (a.c.k_out > 0 || a.c.v_out > 0) return tc_dispatch_sparse(a, s, e0, e1, occ);
   if (a.bits == 3) return a.ragged ? tc_dispatch_3bit_ragged(a, s, e0, e1, occ)
                                    : tc_dispatch_3bit(a, s, e0, e1, occ);
   if (a.ragged) {

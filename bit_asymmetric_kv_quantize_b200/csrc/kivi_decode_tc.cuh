@@ -115,11 +115,13 @@ struct Pairs<4> {
 // 4-warp CTAs, two tiles per warp at 2-bit (two CTAs per SM) and one at 4-bit
 // (three per SM); grouped heads run best as one CTA per SM with 11 (GQ 2, 4)
 // or 7 (GQ 8) consumer warps sharing one ring.
-template <int D, int BITS, int GQ, int MB>
+// SP: the dense-and-sparse variant (kept entries per group; their lists
+// ride in the ring beside the codes): four consumer warps, one tile each.
+template <int D, int BITS, int GQ, int MB, bool SP = false>
 struct Geo {
-  static constexpr int NW = GQ == 1 ? 4 : (GQ == 8 ? 7 : 11);
+  static constexpr int NW = SP ? 4 : (GQ == 1 ? 4 : (GQ == 8 ? 7 : 11));
   // tiles per warp and stage (1-bit MHA also needs two to fit a window tile in a stage)
-  static constexpr int TPW = (GQ == 1 && BITS <= 2) ? 2 : 1;
+  static constexpr int TPW = (!SP && GQ == 1 && BITS <= 2) ? 2 : 1;
   static constexpr int WB = Layout<D, BITS>::WB;  // words per code block (3: bit planes)
   static constexpr int THREADS = (NW + 1) * 32;
   static constexpr int kStage = NW * TPW;       // tiles per pipeline stage
@@ -139,6 +141,16 @@ struct Geo {
   static constexpr int O_VC = O_KZ + kStage * KM_B;
   static constexpr int O_VS = O_VC + kStage * VC_B;
   static constexpr int O_VZ = O_VS + kStage * VM_B;
+  // dense-and-sparse lists per tile, slots sized for kMaxOut entries per
+  // group: key (token, value) per channel, value (channel, value) per
+  // token and value group
+  static constexpr int KOI_B = SP ? D * kMaxOut * 4 : 0;
+  static constexpr int VOI_B = SP ? kTile * NJ * kMaxOut * 4 : 0;
+  static constexpr int O_KOI = O_VZ + kStage * VM_B;
+  static constexpr int O_KOV = O_KOI + kStage * KOI_B;
+  static constexpr int O_VOI = O_KOV + kStage * KOI_B;
+  static constexpr int O_VOV = O_VOI + kStage * VOI_B;
+  static constexpr int O_CODE_END = O_VOV + kStage * VOI_B;
   // fp16 residual window through the ring: a window stage holds WT tokens of
   // K, then of V, as 2-D tensor-copy boxes of BW columns (rows of RB bytes)
   // in the hardware's 128-byte (64-byte when D = 32) swizzle
@@ -149,9 +161,10 @@ struct Geo {
   static constexpr int BOX_B = WT * RB;
   static constexpr int WTILE_B = 2 * NBX * BOX_B;     // one 32-token window tile (K, V)
   // a stage holds kStage code tiles, and at least one window tile
-  static constexpr int CODE_STAGE_B = (O_VZ + kStage * VM_B + 1023) / 1024 * 1024;
+  static constexpr int CODE_STAGE_B = (O_CODE_END + 1023) / 1024 * 1024;
   static constexpr int STAGE_B = CODE_STAGE_B < WTILE_B ? WTILE_B : CODE_STAGE_B;
-  static constexpr int MIN_CTAS = NW == 4 ? (TPW == 2 ? 2 : 3) : 1;
+  static constexpr int MIN_CTAS =
+      SP ? ((GQ == 1 && BITS <= 2) ? 2 : 1) : (NW == 4 ? (TPW == 2 ? 2 : 3) : 1);
   static constexpr int NPB = GQ == 8 ? 2 : 1;  // n-tiles of 8 columns (4 heads x hi, lo)
   static constexpr int PST = TPW * kTile + 8;  // p buffer stride per head (floats)
   // B fragment blocks: only the lanes whose column carries a head are kept
@@ -165,7 +178,11 @@ struct Geo {
   static constexpr int QB_B = NPB * KSL * BLKW * 4;       // q' B fragments (score product)
   static constexpr int PB_B = NPB * NJ * NSL * BLKW * 4;  // p' B fragments (value product)
   static constexpr int PBUF_B = GQ * PST * 4;         // p per head and token
-  static constexpr int WARP_B = TPW * (QB_B + PB_B) + PBUF_B;
+  // dense-and-sparse: score corrections per head and token of the warp's
+  // tiles, and the value corrections per head and channel of its unit
+  static constexpr int CORR_B = SP ? TPW * GQ * kTile * 4 : 0;
+  static constexpr int VCORR_B = SP ? GQ * D * 4 : 0;
+  static constexpr int WARP_B = TPW * (QB_B + PB_B) + PBUF_B + CORR_B + VCORR_B;
   // ring depth: three stages where they fit beside MIN_CTAS - 1 other CTAs
   // (228 KB of shared memory per SM, 1 KB of it reserved per CTA), else two:
   // the bytes in flight per SM bound the achieved bandwidth
@@ -271,6 +288,9 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
                : "r"(smem_u32(p))
                : "memory");
 }
+
+__device__ __forceinline__ float load1(const float* p) { return *p; }
+__device__ __forceinline__ float load1(const __half* p) { return __half2float(*p); }
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) {
   return *reinterpret_cast<uint32_t*>(&h);
@@ -425,12 +445,12 @@ __device__ __forceinline__ void consumers_sync() {
 }
 
 // RAG: ragged batch (per-sequence lengths in dev_state; device-counter mode)
-template <int D, int BITS, int GQ, typename T, typename MT, bool RAG>
-__global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
-                                  Geo<D, BITS, GQ, sizeof(MT)>::MIN_CTAS)
+template <int D, int BITS, int GQ, typename T, typename MT, bool RAG, bool SP = false>
+__global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT), SP>::THREADS,
+                                  Geo<D, BITS, GQ, sizeof(MT), SP>::MIN_CTAS)
     decode_stream_tc(const DecodeArgs args, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV) {
-  using G = Geo<D, BITS, GQ, sizeof(MT)>;
+  using G = Geo<D, BITS, GQ, sizeof(MT), SP>;
   using PR = Pairs<BITS>;
   constexpr int kW = G::NW;
   constexpr int kStage = G::kStage;
@@ -622,7 +642,22 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           if (*(volatile int*)&flag[0]) break;
           unsigned char* buf = smem + s * G::STAGE_B;
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          mbar_expect_tx(&full[s], (uint32_t)(n * G::TILE_B));
+          // dense-and-sparse lists of the stage's tiles (index and value each)
+          const uint32_t kl_b = SP ? (uint32_t)(D * c.k_out * 4) : 0u;
+          const uint32_t vl_b = SP ? (uint32_t)(kTile * NJ * c.v_out * 4) : 0u;
+          mbar_expect_tx(&full[s], (uint32_t)(n * (G::TILE_B + 2 * kl_b + 2 * vl_b)));
+          if constexpr (SP) {
+            if (kl_b > 0) {
+              const long long kl = (u * (Ts / kG) + t0) * D * c.k_out;
+              bulk_copy(buf + G::O_KOI, c.k_oi + kl, n * kl_b, &full[s]);
+              bulk_copy(buf + G::O_KOV, c.k_ov + kl, n * kl_b, &full[s]);
+            }
+            if (vl_b > 0) {
+              const long long vl = (u * Ts + (long long)t0 * kTile) * NJ * c.v_out;
+              bulk_copy(buf + G::O_VOI, c.v_oi + vl, n * vl_b, &full[s]);
+              bulk_copy(buf + G::O_VOV, c.v_ov + vl, n * vl_b, &full[s]);
+            }
+          }
           if (!RAG || c.bt == nullptr) {
             bulk_copy(buf + G::O_KC, kc_u + (long long)t0 * kTile * WK, n * G::KC_B, &full[s]);
             bulk_copy(buf + G::O_KS, ks_u + (long long)t0 * D, n * G::KM_B, &full[s]);
@@ -711,6 +746,12 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
     // fragment columns of absent heads stay zero (after the CTA barrier, so
     // that the producer starts streaming meanwhile)
     for (int i = lane; i < TPW * (G::QB_B + G::PB_B) / 4; i += 32) reinterpret_cast<uint32_t*>(wb)[i] = 0u;
+    // dense-and-sparse corrections start at zero (and are left at zero)
+    float* corr = reinterpret_cast<float*>(wb + TPW * (G::QB_B + G::PB_B) + G::PBUF_B);  // [TPW][GQ][32]
+    float* vcorr = corr + TPW * GQ * kTile;                                               // [GQ][D]
+    if constexpr (SP) {
+      for (int i = lane; i < (G::CORR_B + G::VCORR_B) / 4; i += 32) corr[i] = 0.f;
+    }
     __syncwarp();
     uint32_t* qB = reinterpret_cast<uint32_t*>(wb);                     // [TPW][NPB][KSL][BLKW]
     uint32_t* pB = reinterpret_cast<uint32_t*>(wb + TPW * G::QB_B);     // [TPW][NPB][NJ][NSL][BLKW]
@@ -829,7 +870,8 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           qf[x][m][2] = to_f32(qh[1]) * a.qscale;
           qf[x][m][3] = to_f32(qh[G::PPW + 1]) * a.qscale;
         }
-      if (window_owner) {
+      if (window_owner || SP) {
+        // (dense-and-sparse: the key corrections read q at any channel)
         for (int i = tid; i < GQ * D; i += kW * 32) qs[i] = to_f32(qg[i]) * a.qscale;
         consumers_sync<kW>();  // qs is read by whichever warps take the window
       }
@@ -1016,6 +1058,41 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
                 sc[p][4 * tt + 2 * mt + 1] = tv[tt] ? v1 : kNegInf;
               }
             }
+          if constexpr (SP) {
+            // dense-and-sparse keys: a kept entry (token t, channel d, value x)
+            // was reconstructed by the codes as z_{g,d} (code 0); add
+            // q_d (x - z_{g,d}) to token t's score, for every head
+            if (c.k_out > 0) {
+              const int nk = D * c.k_out;
+#pragma unroll
+              for (int tt = 0; tt < TPW; ++tt) {
+                const int ti = warp * TPW + (tv[tt] ? tt : 0);
+                const int* oi = reinterpret_cast<const int*>(buf + G::O_KOI) + ti * nk;
+                const float* ov = reinterpret_cast<const float*>(buf + G::O_KOV) + ti * nk;
+                for (int e = lane; e < nk; e += 32) {
+                  const int d = e / c.k_out;
+                  const float dx = ov[e] - load1(kz[tt] + d);
+                  const int tok = oi[e] & (kTile - 1);
+#pragma unroll
+                  for (int h = 0; h < GQ; ++h) atomicAdd(&corr[(tt * GQ + h) * kTile + tok], qs[h * D + d] * dx);
+                }
+              }
+              __syncwarp();
+#pragma unroll
+              for (int p = 0; p < NPB; ++p) {
+                if (!vh[p]) continue;
+                const int h = tq + 4 * p;
+#pragma unroll
+                for (int i = 0; i < 4 * TPW; ++i) {
+                  const int tt = i >> 2, tok = 16 * ((i >> 1) & 1) + 8 * (i & 1) + g;
+                  float* cp = &corr[(tt * GQ + h) * kTile + tok];
+                  sc[p][i] += *cp;
+                  *cp = 0.f;
+                }
+              }
+              __syncwarp();
+            }
+          }
           // -- online softmax: the running max moves only when a score exceeds it
           float lm[NPB];
           bool need = false;
@@ -1049,6 +1126,9 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
               const float ah = __shfl_sync(0xffffffffu, al[h >> 2], h & 3);
 #pragma unroll
               for (int j = 0; j < NJ; ++j) bv[h][j] *= ah;
+              if constexpr (SP) {
+                for (int d = lane; d < D; d += 32) vcorr[h * D + d] *= ah;
+              }
             }
           }
 #pragma unroll
@@ -1065,6 +1145,31 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
           }
           __syncwarp();
 
+          if constexpr (SP) {
+            // dense-and-sparse values: a kept entry (token t, channel c, value
+            // x) was reconstructed as z_{t,j} (code 0); add p_t (x - z_{t,j})
+            // to channel c of the unit's value corrections, every head
+            if (c.v_out > 0) {
+              const int nv = kTile * NJ * c.v_out;
+#pragma unroll
+              for (int tt = 0; tt < TPW; ++tt) {
+                if (!tv[tt]) continue;
+                const int ti = warp * TPW + tt;
+                const int* oi = reinterpret_cast<const int*>(buf + G::O_VOI) + ti * nv;
+                const float* ov = reinterpret_cast<const float*>(buf + G::O_VOV) + ti * nv;
+                for (int e = lane; e < nv; e += 32) {
+                  const int tj = e / c.v_out;  // token * NJ + group
+                  const int t = tj / NJ, j = tj - t * NJ;
+                  const float dx = ov[e] - load1(vz[tt] + tj);
+                  const int ch = j * kGv + (oi[e] & (kGv - 1));
+#pragma unroll
+                  for (int h = 0; h < GQ; ++h)
+                    atomicAdd(&vcorr[h * D + ch], pbuf[h * PST + 32 * tt + t] * dx);
+                }
+              }
+              __syncwarp();
+            }
+          }
           // -- p' = p s_v 2^(SV - e) (hi, lo) into the B fragments; bias_v += p z_v
 #pragma unroll
           for (int tt = 0; tt < TPW; ++tt) {
@@ -1313,6 +1418,17 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
             dst[0] = fmaf(acc[p][m][0] + acc[p][m][1], kValOut, bias);
             dst[1] = fmaf(acc[p][m][2] + acc[p][m][3], kValOut, bias);
           }
+        }
+        if constexpr (SP) {
+          // the unit's dense-and-sparse value corrections (same softmax state)
+          __syncwarp();
+#pragma unroll
+          for (int h = 0; h < GQ; ++h)
+            for (int d = lane; d < D; d += 32) {
+              mg_acc[(warp * GQ + h) * D + d] += vcorr[h * D + d];
+              vcorr[h * D + d] = 0.f;
+            }
+          __syncwarp();
         }
       };
 
@@ -1624,9 +1740,9 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT)>::THREADS,
 
 // Opt in to the kernel's dynamic shared memory and return how many of its
 // CTAs fit on one SM (both once per device).
-template <int D, int BITS, int GQ, typename T, typename MT, bool RAG>
+template <int D, int BITS, int GQ, typename T, typename MT, bool RAG, bool SP>
 cudaError_t tc_setup(int* ctas_per_sm) {
-  using G = Geo<D, BITS, GQ, sizeof(MT)>;
+  using G = Geo<D, BITS, GQ, sizeof(MT), SP>;
   static int occ[128] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1635,11 +1751,11 @@ cudaError_t tc_setup(int* ctas_per_sm) {
     *ctas_per_sm = occ[dev];
     return cudaSuccess;
   }
-  e = cudaFuncSetAttribute(decode_stream_tc<D, BITS, GQ, T, MT, RAG>,
+  e = cudaFuncSetAttribute(decode_stream_tc<D, BITS, GQ, T, MT, RAG, SP>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_B);
   if (e != cudaSuccess) return e;
   int n = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_tc<D, BITS, GQ, T, MT, RAG>,
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_stream_tc<D, BITS, GQ, T, MT, RAG, SP>,
                                                     G::THREADS, G::SMEM_B);
   if (e != cudaSuccess) return e;
   if (n < 1) return cudaErrorInvalidConfiguration;
@@ -1731,13 +1847,13 @@ cudaError_t window_maps(const void* k_res, const void* v_res, long long rows, in
   return cudaSuccess;
 }
 
-template <int D, int BITS, int GQ, typename T, typename MT, bool RAG>
+template <int D, int BITS, int GQ, typename T, typename MT, bool RAG, bool SP>
 cudaError_t tc_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
                  int* ctas_per_sm) {
-  using G = Geo<D, BITS, GQ, sizeof(MT)>;
-  if (ctas_per_sm) return tc_setup<D, BITS, GQ, T, MT, RAG>(ctas_per_sm);
+  using G = Geo<D, BITS, GQ, sizeof(MT), SP>;
+  if (ctas_per_sm) return tc_setup<D, BITS, GQ, T, MT, RAG, SP>(ctas_per_sm);
   int occ = 0;
-  cudaError_t e = tc_setup<D, BITS, GQ, T, MT, RAG>(&occ);
+  cudaError_t e = tc_setup<D, BITS, GQ, T, MT, RAG, SP>(&occ);
   if (e != cudaSuccess) return e;
   CUtensorMap tmK, tmV;
   memset(&tmK, 0, sizeof(tmK));
@@ -1761,29 +1877,29 @@ cudaError_t tc_t(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t err =
-      cudaLaunchKernelEx(&cfg, decode_stream_tc<D, BITS, GQ, T, MT, RAG>, a, tmK, tmV);
+      cudaLaunchKernelEx(&cfg, decode_stream_tc<D, BITS, GQ, T, MT, RAG, SP>, a, tmK, tmV);
   if (err == cudaSuccess) err = cudaGetLastError();
   if (e1) cudaEventRecord(e1, s);
   return err;
 }
 
-template <int D, int BITS, typename T, typename MT, bool RAG>
+template <int D, int BITS, typename T, typename MT, bool RAG, bool SP>
 cudaError_t tc_g(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1, int* occ) {
   switch (a.gq) {
-    case 1: return tc_t<D, BITS, 1, T, MT, RAG>(a, s, e0, e1, occ);
-    case 2: return tc_t<D, BITS, 2, T, MT, RAG>(a, s, e0, e1, occ);
-    case 4: return tc_t<D, BITS, 4, T, MT, RAG>(a, s, e0, e1, occ);
-    case 8: return tc_t<D, BITS, 8, T, MT, RAG>(a, s, e0, e1, occ);
+    case 1: return tc_t<D, BITS, 1, T, MT, RAG, SP>(a, s, e0, e1, occ);
+    case 2: return tc_t<D, BITS, 2, T, MT, RAG, SP>(a, s, e0, e1, occ);
+    case 4: return tc_t<D, BITS, 4, T, MT, RAG, SP>(a, s, e0, e1, occ);
+    case 8: return tc_t<D, BITS, 8, T, MT, RAG, SP>(a, s, e0, e1, occ);
   }
   return cudaErrorInvalidValue;
 }
 
-template <int BITS, typename T, typename MT, bool RAG>
+template <int BITS, typename T, typename MT, bool RAG, bool SP = false>
 cudaError_t tc_d(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1, int* occ) {
   switch (a.D) {
-    case 32: return tc_g<32, BITS, T, MT, RAG>(a, s, e0, e1, occ);
-    case 64: return tc_g<64, BITS, T, MT, RAG>(a, s, e0, e1, occ);
-    case 128: return tc_g<128, BITS, T, MT, RAG>(a, s, e0, e1, occ);
+    case 32: return tc_g<32, BITS, T, MT, RAG, SP>(a, s, e0, e1, occ);
+    case 64: return tc_g<64, BITS, T, MT, RAG, SP>(a, s, e0, e1, occ);
+    case 128: return tc_g<128, BITS, T, MT, RAG, SP>(a, s, e0, e1, occ);
   }
   return cudaErrorInvalidValue;
 }

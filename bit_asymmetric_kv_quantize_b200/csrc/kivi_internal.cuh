@@ -12,6 +12,7 @@ constexpr int kG = 32;        // key group: tokens per (group, channel) scale
 constexpr int kGv = 32;       // value group: channels per (token, group) scale
 constexpr int kTile = 32;     // tokens per quantize tile (= kG, a multiple of E)
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxOut = 4;    // dense-and-sparse variant: kept entries per group, at most
 
 // Device view of one cache; per-unit strides follow the ABI layout.  The
 // scales and zeros are binary32 (meta 0) or binary16 (meta 1) elements.
@@ -35,6 +36,18 @@ struct CacheView {
   int pps;
   long long n_pages;
   int Hkv;
+  // dense-and-sparse variant: entries kept exactly per key / value group
+  // (0: none) and their lists, [unit][Tq/G][D][k_out] and [unit][Tq][D/Gv][v_out]
+  int k_out;
+  int v_out;
+  int* k_oi;
+  float* k_ov;
+  int* v_oi;
+  float* v_ov;
+  __host__ __device__ float* k_scale_f() const { return static_cast<float*>(k_scale); }
+  __host__ __device__ float* k_zero_f() const { return static_cast<float*>(k_zero); }
+  __host__ __device__ float* v_scale_f() const { return static_cast<float*>(v_scale); }
+  __host__ __device__ float* v_zero_f() const { return static_cast<float*>(v_zero); }
 };
 
 // Tokens per unit slot of the store arrays (the per-unit stride).
@@ -488,6 +501,9 @@ cudaError_t tc_dispatch_ragged(const DecodeArgs& a, cudaStream_t s, cudaEvent_t 
                                cudaEvent_t e1, int* occ);
 cudaError_t tc_dispatch_ragged_meta16(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0,
                                       cudaEvent_t e1, int* occ);
+// The dense-and-sparse instances (binary32 metadata; 1, 2, 4 bits).
+cudaError_t tc_dispatch_sparse(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
+                               int* occ);
 // The 3-bit (bit-plane) instances, uniform and ragged batches.
 cudaError_t tc_dispatch_3bit(const DecodeArgs& a, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1,
                              int* occ);

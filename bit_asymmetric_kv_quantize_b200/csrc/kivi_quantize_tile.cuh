@@ -9,8 +9,11 @@
 // asymmetric scale and zero (study.space summary).
 #pragma once
 
+#include <type_traits>
+
 #include "kivi_codes.cuh"
 #include "kivi_internal.cuh"
+#include "kivi_sparse.cuh"
 
 namespace kivi {
 namespace {
@@ -58,23 +61,45 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
     float x[kTile];
 #pragma unroll
     for (int t = 0; t < kTile; ++t) x[t] = to_f32(Ksrc[(long long)t * D + tid]);
-    float mn = x[0], mx = x[0];
-#pragma unroll
-    for (int t = 1; t < kTile; ++t) {
-      if (x[t] < mn) mn = x[t];
-      if (x[t] > mx) mx = x[t];
-    }
-    const float s = round_meta<M>(__fdiv_rn(__fsub_rn(mx, mn), Lf));
-    const float z = round_meta<M>(mn);
     const long long g = t0 / kG;
-    reinterpret_cast<M*>(c.k_scale)[unit * Lt::k_meta_unit(Ts) + g * D + tid] = from_f32<M>(s);
-    reinterpret_cast<M*>(c.k_zero)[unit * Lt::k_meta_unit(Ts) + g * D + tid] = from_f32<M>(z);
-    const float rs = recip_rn(s);
+    bool done = false;
+    if constexpr (std::is_same<M, float>::value) {
+      if (c.k_out > 0) {
+        // dense-and-sparse variant: the group's k_out largest magnitudes are
+        // kept exactly (listed in index order, dense code 0), the rest quantized
+        float s, z, ov[kMaxOut];
+        int codes[kTile], oi[kMaxOut];
+        quantize_group_sparse<kTile, kMaxOut>(x, c.k_out, BITS, &s, &z, codes, oi, ov);
+        c.k_scale_f()[unit * Lt::k_meta_unit(Ts) + g * D + tid] = s;
+        c.k_zero_f()[unit * Lt::k_meta_unit(Ts) + g * D + tid] = z;
 #pragma unroll
-    for (int t = 0; t < kTile; ++t) {
-      int code = 0;
-      if (s != 0.0f) code = code_of(__fsub_rn(x[t], z), s, rs, Lt::L);
-      ck[t * D + tid] = (uint8_t)code;
+        for (int t = 0; t < kTile; ++t) ck[t * D + tid] = (uint8_t)codes[t];
+        const long long lo = ((unit * (Ts / kG) + g) * D + tid) * c.k_out;
+        for (int m = 0; m < c.k_out; ++m) {
+          c.k_oi[lo + m] = oi[m];
+          c.k_ov[lo + m] = ov[m];
+        }
+        done = true;
+      }
+    }
+    if (!done) {
+      float mn = x[0], mx = x[0];
+#pragma unroll
+      for (int t = 1; t < kTile; ++t) {
+        if (x[t] < mn) mn = x[t];
+        if (x[t] > mx) mx = x[t];
+      }
+      const float s = round_meta<M>(__fdiv_rn(__fsub_rn(mx, mn), Lf));
+      const float z = round_meta<M>(mn);
+      reinterpret_cast<M*>(c.k_scale)[unit * Lt::k_meta_unit(Ts) + g * D + tid] = from_f32<M>(s);
+      reinterpret_cast<M*>(c.k_zero)[unit * Lt::k_meta_unit(Ts) + g * D + tid] = from_f32<M>(z);
+      const float rs = recip_rn(s);
+#pragma unroll
+      for (int t = 0; t < kTile; ++t) {
+        int code = 0;
+        if (s != 0.0f) code = code_of(__fsub_rn(x[t], z), s, rs, Lt::L);
+        ck[t * D + tid] = (uint8_t)code;
+      }
     }
   }
   // ---- values: token tid / NJ, channel group tid % NJ
@@ -84,23 +109,43 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
     float x[kGv];
 #pragma unroll
     for (int i = 0; i < kGv; ++i) x[i] = to_f32(src[i]);
-    float mn = x[0], mx = x[0];
-#pragma unroll
-    for (int i = 1; i < kGv; ++i) {
-      if (x[i] < mn) mn = x[i];
-      if (x[i] > mx) mx = x[i];
-    }
-    const float s = round_meta<M>(__fdiv_rn(__fsub_rn(mx, mn), Lf));
-    const float z = round_meta<M>(mn);
     const long long mo = unit * Lt::v_meta_unit(Ts) + (t0 + t) * NJ + j;
-    reinterpret_cast<M*>(c.v_scale)[mo] = from_f32<M>(s);
-    reinterpret_cast<M*>(c.v_zero)[mo] = from_f32<M>(z);
-    const float rs = recip_rn(s);
+    bool done = false;
+    if constexpr (std::is_same<M, float>::value) {
+      if (c.v_out > 0) {
+        float s, z, ov[kMaxOut];
+        int codes[kGv], oi[kMaxOut];
+        quantize_group_sparse<kGv, kMaxOut>(x, c.v_out, BITS, &s, &z, codes, oi, ov);
+        c.v_scale_f()[mo] = s;
+        c.v_zero_f()[mo] = z;
 #pragma unroll
-    for (int i = 0; i < kGv; ++i) {
-      int code = 0;
-      if (s != 0.0f) code = code_of(__fsub_rn(x[i], z), s, rs, Lt::L);
-      cv[t * D + j * kGv + i] = (uint8_t)code;
+        for (int i = 0; i < kGv; ++i) cv[t * D + j * kGv + i] = (uint8_t)codes[i];
+        const long long lo = mo * c.v_out;  // [unit][token][group][v_out]
+        for (int m = 0; m < c.v_out; ++m) {
+          c.v_oi[lo + m] = oi[m];
+          c.v_ov[lo + m] = ov[m];
+        }
+        done = true;
+      }
+    }
+    if (!done) {
+      float mn = x[0], mx = x[0];
+#pragma unroll
+      for (int i = 1; i < kGv; ++i) {
+        if (x[i] < mn) mn = x[i];
+        if (x[i] > mx) mx = x[i];
+      }
+      const float s = round_meta<M>(__fdiv_rn(__fsub_rn(mx, mn), Lf));
+      const float z = round_meta<M>(mn);
+      reinterpret_cast<M*>(c.v_scale)[mo] = from_f32<M>(s);
+      reinterpret_cast<M*>(c.v_zero)[mo] = from_f32<M>(z);
+      const float rs = recip_rn(s);
+#pragma unroll
+      for (int i = 0; i < kGv; ++i) {
+        int code = 0;
+        if (s != 0.0f) code = code_of(__fsub_rn(x[i], z), s, rs, Lt::L);
+        cv[t * D + j * kGv + i] = (uint8_t)code;
+      }
     }
   }
   tile_sync<D, BAR>();
@@ -128,24 +173,23 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
       const uint32_t p2 = __ballot_sync(0xffffffffu, cd & 4u);
       if (lane < 3) vdst[lane * D + d] = lane == 0 ? p0 : (lane == 1 ? p1 : p2);
     }
-    tile_sync<D, BAR>();
-    return;
-  }
+  } else {
 #pragma unroll
-  for (int k = tid; k < NW; k += D) {
-    const int t = k / WK, w = k % WK;
-    uint32_t word = 0;
+    for (int k = tid; k < NW; k += D) {
+      const int t = k / WK, w = k % WK;
+      uint32_t word = 0;
 #pragma unroll
-    for (int i = 0; i < E; ++i) word |= (uint32_t)ck[t * D + w * E + i] << (BITS * i);
-    kdst[k] = word;
-  }
+      for (int i = 0; i < E; ++i) word |= (uint32_t)ck[t * D + w * E + i] << (BITS * i);
+      kdst[k] = word;
+    }
 #pragma unroll
-  for (int k = tid; k < NW; k += D) {
-    const int tb = k / D, d = k % D;
-    uint32_t word = 0;
+    for (int k = tid; k < NW; k += D) {
+      const int tb = k / D, d = k % D;
+      uint32_t word = 0;
 #pragma unroll
-    for (int i = 0; i < E; ++i) word |= (uint32_t)cv[(tb * E + i) * D + d] << (BITS * i);
-    vdst[k] = word;
+      for (int i = 0; i < E; ++i) word |= (uint32_t)cv[(tb * E + i) * D + d] << (BITS * i);
+      vdst[k] = word;
+    }
   }
   tile_sync<D, BAR>();
 }

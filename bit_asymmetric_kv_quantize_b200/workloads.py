@@ -61,6 +61,8 @@ class Workload:
     n_outliers: int = 4
     outlier_scale: float = 20.0
     seed: int = 0
+    spike_frac: float = 0.0    # > 0: that fraction of single K and V entries scaled by spike_scale
+    spike_scale: float = 40.0  # (entry outliers, the case dense-and-sparse groups keep exactly)
 
     @property
     def torch_dtype(self):
@@ -152,9 +154,19 @@ def prompt_kv(w: Workload, T: Optional[int] = None, device="cpu"):
     V = torch.empty_like(K)
     for b in range(w.B):
         k = torch.randn(w.Hkv, T, w.D, generator=g, dtype=torch.float32, device=device)
+        v = torch.randn(w.Hkv, T, w.D, generator=g, dtype=torch.float32, device=device)
+        if w.spike_frac > 0:
+            k = _spikes(w, k, g)
+            v = _spikes(w, v, g)
         K[b].copy_(k * mult)
-        V[b].copy_(torch.randn(w.Hkv, T, w.D, generator=g, dtype=torch.float32, device=device))
+        V[b].copy_(v)
     return K, V
+
+
+def _spikes(w: Workload, x: torch.Tensor, g: torch.Generator) -> torch.Tensor:
+    """x with a seeded random fraction w.spike_frac of its entries scaled by w.spike_scale."""
+    m = torch.rand(x.shape, generator=g, dtype=torch.float32, device=x.device) < w.spike_frac
+    return torch.where(m, x * w.spike_scale, x)
 
 
 def query(w: Workload, step: int = -1, device="cpu") -> torch.Tensor:
@@ -170,5 +182,8 @@ def step_kv(w: Workload, step: int, device="cpu"):
     g = _device_gen(device, _seed(w.seed, "step_kv", step))
     k = torch.randn(w.B, w.Hkv, w.D, generator=g, dtype=torch.float32, device=device)
     v = torch.randn(w.B, w.Hkv, w.D, generator=g, dtype=torch.float32, device=device)
+    if w.spike_frac > 0:
+        k = _spikes(w, k, g)
+        v = _spikes(w, v, g)
     k = k * key_channel_scale(w).to(device)[None]
     return k.to(w.torch_dtype), v.to(w.torch_dtype)

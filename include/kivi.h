@@ -113,7 +113,9 @@ typedef enum { KIVI_F16 = 0, KIVI_F32 = 1 } kivi_dtype;
  * storage precision for them.) */
 typedef enum { KIVI_META_F32 = 0, KIVI_META_F16 = 1 } kivi_meta;
 
-/* Shape of one cache (one attention layer).  Supported: bits in {1, 2, 3, 4}
+/* Shape of one cache (one attention layer).  k_out = v_out = 0 (a
+ * zero-filled struct) is the plain format; see the dense-and-sparse
+ * variant below for other values.  Supported: bits in {1, 2, 3, 4}
  * (3 bits: the tensor-core decode only; kivi_decode_attention_simt refuses
  * it with KIVI_ERR_UNSUPPORTED),
  * G = 32, Gv = 32, D in {32, 64, 128}, R a positive multiple of 32,
@@ -131,6 +133,9 @@ typedef struct {
   long long capacity; /* max tokens per sequence, quantized + residual */
   int dtype;          /* kivi_dtype of K, V, q, out and the residual window */
   int meta;           /* kivi_meta of k_scale, k_zero, v_scale, v_zero */
+  int k_out;          /* dense-and-sparse variant: entries kept exactly per key
+                         group (0: plain codes; see kivi_outlier_buffer_sizes) */
+  int v_out;          /* ... per value group */
 } kivi_dims;
 
 enum {
@@ -164,6 +169,11 @@ typedef struct {
   const int32_t *block_table; /* device, [B][pages_per_seq] pool page ids */
   int pages_per_seq;
   long long num_pages;        /* pages in the pool */
+  /* dense-and-sparse variant (kivi_cache_set_outliers); NULL otherwise */
+  int32_t *k_out_idx;
+  float *k_out_val;
+  int32_t *v_out_idx;
+  float *v_out_val;
 } kivi_cache;
 
 /* Byte size of each of the KIVI_NUM_BUFFERS buffers for `dims`, written to
@@ -374,6 +384,31 @@ KIVI_API void kivi_set_timing_events(void *start_event, void *stop_event);
 /* Number of context splits the decode kernel would use for this cache's
  * current fill level and Hq (>= 1), or 0 on error. */
 KIVI_API int kivi_decode_num_splits(const kivi_cache *cache, int Hq);
+
+/* Dense-and-sparse variant (dims.k_out > 0 or dims.v_out > 0; KVQuant page,
+ * abstract item (iv): outliers isolated per vector so that they do not skew
+ * its quantization range).  Every key group (channel d over G tokens) keeps
+ * its k_out largest magnitudes exactly, and every value group (token t over
+ * Gv channels) its v_out largest; among equal magnitudes the lower index
+ * goes first.  Those entries get dense code 0 and are listed, in ascending
+ * index order, in four more device buffers:
+ *   k_out_idx int32 [B][Hkv][Tq/G][D][k_out]   token within the key group
+ *   k_out_val float [B][Hkv][Tq/G][D][k_out]   its exact value
+ *   v_out_idx int32 [B][Hkv][Tq][D/Gv][v_out]  channel within the value group
+ *   v_out_val float [B][Hkv][Tq][D/Gv][v_out]  its exact value
+ * The other entries are quantized as usual over the remaining ones (min and
+ * max taken without the kept entries).  Decode reconstructs a kept entry as
+ * its value and every other one as c * s + z.  Supported: k_out and v_out
+ * in [0, 4], binary32 metadata, bits 1, 2 or 4, contiguous caches (uniform
+ * or ragged batches; not the paged store), the tensor-core decode (the
+ * CUDA-core kernel and kivi_paged_cache_init refuse it with
+ * KIVI_ERR_UNSUPPORTED).
+ * kivi_outlier_buffer_sizes: byte sizes of the four buffers (0 for a list
+ * that is not kept).  kivi_cache_set_outliers: bind them to a cache made by
+ * kivi_cache_init (before its prefill); buffers[i] may be NULL only where
+ * its size is 0.  Errors: KIVI_ERR_ARG, KIVI_ERR_UNSUPPORTED. */
+KIVI_API int kivi_outlier_buffer_sizes(const kivi_dims *dims, size_t out_bytes[4]);
+KIVI_API int kivi_cache_set_outliers(kivi_cache *cache, void *const buffers[4]);
 
 /* Size of the fixed device scratch used by kivi_decode_attention_noalloc. */
 #define KIVI_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)

@@ -33,10 +33,10 @@ def test_library_exports_every_declared_symbol():
 
 def _dims(**kw):
     d = dict(B=2, Hkv=4, D=128, bits=2, G=32, Gv=32, R=128, capacity=4096, dtype=kivi.KIVI_F16,
-             meta=kivi.KIVI_META_F32)
+             meta=kivi.KIVI_META_F32, k_out=0, v_out=0)
     d.update(kw)
     return KiviDims(d["B"], d["Hkv"], d["D"], d["bits"], d["G"], d["Gv"], d["R"], d["capacity"],
-                    d["dtype"], d["meta"])
+                    d["dtype"], d["meta"], d["k_out"], d["v_out"])
 
 
 def _block(bits):
@@ -87,7 +87,8 @@ def test_binary16_metadata_halves_the_scale_and_zero_buffers(bits, D):
 def test_dims_struct_matches_the_header():
     # the Python mirror of kivi_dims: nine ints/longs, then the metadata type
     names = [f[0] for f in KiviDims._fields_]
-    assert names == ["B", "Hkv", "D", "bits", "G", "Gv", "R", "capacity", "dtype", "meta"]
+    assert names == ["B", "Hkv", "D", "bits", "G", "Gv", "R", "capacity", "dtype", "meta",
+                     "k_out", "v_out"]
     text = open(HEADER).read()
     body = text[text.index("typedef struct {\n  int B;"):text.index("} kivi_dims;")]
     assert re.findall(r"\b(?:int|long long)\s+(\w+);", body) == names
@@ -327,3 +328,40 @@ def test_three_bit_codes_are_three_planes_per_32():
     assert rc == 0
     u, Tq = B * H, cap - R
     assert s[0] == s[3] == u * Tq * D * 3 // 8
+
+
+
+def test_outlier_buffer_sizes_and_refusals():
+    """Dense-and-sparse variant: list sizes follow [Tq/G][D][k_out] and
+    [Tq][D/Gv][v_out] (int32 index, binary32 value); the limits and the
+    formats it does not support are refused before anything else."""
+    B, H, D, R, cap = 2, 3, 64, 64, 640
+    u, Tq = B * H, cap - R
+    out = (ctypes.c_size_t * 4)()
+    L = kivi.lib()
+    for ko, vo in ((1, 0), (0, 2), (4, 4)):
+        dims = _dims(B=B, Hkv=H, D=D, R=R, capacity=cap, k_out=ko, v_out=vo)
+        assert L.kivi_outlier_buffer_sizes(ctypes.byref(dims), ctypes.byref(out)) == 0
+        s = list(out)
+        assert s[0] == s[1] == u * (Tq // 32) * D * ko * 4
+        assert s[2] == s[3] == u * Tq * (D // 32) * vo * 4
+        assert _sizes(dims)[0] == 0  # the eight plain buffers are unchanged
+    for kw, rc in ((dict(k_out=5), ERR_UNSUPPORTED), (dict(v_out=-1), ERR_ARG),
+                   (dict(k_out=1, meta=kivi.KIVI_META_F16), ERR_UNSUPPORTED),
+                   (dict(k_out=1, bits=3), ERR_UNSUPPORTED)):
+        assert _sizes(_dims(**kw))[0] == rc, kw
+    # a sparse cache needs its lists bound before it is used, and the paged store refuses it
+    dims = _dims(R=R, capacity=5 * R, k_out=1, v_out=1)
+    ptrs = (ctypes.c_void_p * 8)(*[0x10000 * (i + 1) for i in range(8)])
+    c = KiviCacheC()
+    assert L.kivi_cache_init(ctypes.byref(c), ctypes.byref(dims), ctypes.byref(ptrs)) == 0
+    fake = ctypes.c_void_p(0x5000)
+    assert L.kivi_quantize_prefill(ctypes.byref(c), fake, fake, 10, None) == ERR_ARG
+    lists = (ctypes.c_void_p * 4)(0x100000, 0x200000, 0x300000, 0x400000)
+    assert L.kivi_cache_set_outliers(ctypes.byref(c), ctypes.byref(lists)) == 0
+    assert (c.k_out_idx, c.v_out_val) == (0x100000, 0x400000)
+    plain = _fake_cache()
+    assert L.kivi_cache_set_outliers(ctypes.byref(plain), ctypes.byref(lists)) == ERR_UNSUPPORTED
+    bt = ctypes.c_void_p(0x90000)
+    assert L.kivi_paged_cache_init(ctypes.byref(c), ctypes.byref(dims), ctypes.byref(ptrs), bt, 4,
+                                   16) == ERR_UNSUPPORTED

@@ -45,7 +45,7 @@ def test_ragged_bytes_sum_over_sequences():
 
 def test_workload_variants_from_the_command_line():
     def args(**kw):
-        d = dict(workload=W.LLAMA2_7B.name, meta="f32", bits=None)
+        d = dict(workload=W.LLAMA2_7B.name, meta="f32", bits=None, outliers="0,0")
         d.update(kw)
         return argparse.Namespace(**d)
 
@@ -54,6 +54,14 @@ def test_workload_variants_from_the_command_line():
     assert (w.meta, w.bits) == ("f16", 1) and w.name.endswith("-meta16-1bit")
     s = bench.bench_workload(args(workload=W.STREAMING.name))
     assert s.steps == 0 and s.T == W.STREAMING.T
+    sp = bench.bench_workload(args(outliers="1,1"))
+    assert sp.spike_frac > 0 and sp.name.endswith("-sparse1x1")
+    # the kept entries' lists count in the algorithmic bytes: 8 bytes per entry
+    w = W.LLAMA2_7B
+    extra = bench.algorithmic_bytes(w, 4096, 0, (1, 1)) - bench.algorithmic_bytes(w, 4096, 0)
+    assert extra == w.B * w.Hkv * 8 * ((4096 // 32) * w.D + 4096 * (w.D // 32))
+    t3 = bench.bench_workload(args(workload=W.LLAMA2_13B_2BIT.name, bits=3))
+    assert t3.name == "llama2-13b-b64h40d128-t8192-3bit"
 
 
 def test_ragged_lengths_are_seeded_and_span_the_range():
