@@ -475,8 +475,11 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT), SP>::THREADS,
   // launched with programmatic stream serialization: the CTAs may start
   // while the preceding grid drains; every thread waits for it to complete
   // (and its writes to be visible) before touching global memory, and the
-  // next grid may be scheduled as soon as SM room frees up
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // next grid may be scheduled as soon as SM room frees up.  Uniform batches
+  // with host counters read nothing from global memory to plan, so they set
+  // up shared memory first and wait just before the first global access.
+  const bool early = !RAG && args.dev_state == nullptr;
+  if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   DecodeArgs a = args;
@@ -544,6 +547,7 @@ __global__ void __launch_bounds__(Geo<D, BITS, GQ, sizeof(MT), SP>::THREADS,
     flag[0] = (sizeof(T) == 2 && (smem_u32(smem) & 1023u) != 0) ? 1 : 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (early) asm volatile("griddepcontrol.wait;" ::: "memory");
   if (!RAG && a.flush) {
     // a due window flush folded into this launch: every unit's R window
     // tokens are quantized into the store at positions n_q - R .. n_q - 1
