@@ -81,6 +81,9 @@ def parse():
                         "consecutive per sequence")
     p.add_argument("--bits", type=int, choices=[1, 2, 3, 4], default=None,
                    help="code width other than the workload's (a format variant)")
+    p.add_argument("--batch", type=int, default=None,
+                   help="batch size other than the workload's (a smaller case of the same "
+                        "kernel instance, e.g. for profiler captures)")
     p.add_argument("--outliers", default="0,0",
                    help="dense-and-sparse variant: entries kept exactly per key group and per "
                         "value group, 'k,v' (the inputs get 1%% spiked entries, x4)")
@@ -104,6 +107,8 @@ def bench_workload(args, name=None) -> W.Workload:
         w = w.with_(steps=0)
     if args.meta == "f16":
         w = w.with_(meta="f16", name=w.name + "-meta16")
+    if getattr(args, "batch", None) and args.batch != w.B:
+        w = w.with_(B=args.batch, name=f"{w.name}-batch{args.batch}")
     ko, vo = (int(x) for x in args.outliers.split(","))
     if ko or vo:
         w = w.with_(spike_frac=0.01, spike_scale=4.0, name=f"{w.name}-sparse{ko}x{vo}")
@@ -265,12 +270,17 @@ def run_kivi(args, rank, world, local):
     result = measure(args, w, rank, world, device, args.steps, args.warmup,
                      args.layers or default_layers(w), full=True)
     if not args.no_extras and args.workload == DEFAULT_WORKLOAD and not (
-            args.bits or args.meta != "f32" or args.paged or args.unfused or args.kernel != "default"):
+            args.bits or args.meta != "f32" or args.paged or args.unfused or args.kernel != "default"
+            or args.batch or args.outliers != "0,0"):
         extra = {}
         for name in EXTRA_WORKLOADS:
             we = bench_workload(args, name)
-            r = measure(args, we, rank, world, device, min(args.steps, 1024), args.warmup,
-                        default_layers(we), full=False)
+            # each layer cache takes its first append in the warm-up: the
+            # prefilled windows are full, so that append flushes (as the
+            # headline's few layers do in its warm-up)
+            nl = default_layers(we)
+            r = measure(args, we, rank, world, device, min(args.steps, 1024), max(args.warmup, nl),
+                        nl, full=False)
             if rank == 0:
                 extra[we.name] = r
         if rank == 0:
@@ -564,7 +574,8 @@ def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, f
                                 "mean": float(lens.float().mean())}} if ragged else {}),
             },
             "roofline": {
-                "kernel": "decode_split", "bound": "hbm", "achieved": achieved, "peak": peak,
+                "kernel": "decode_stream_tc" if args.kernel == "default" else "decode_split_simt",
+                "bound": "hbm", "achieved": achieved, "peak": peak,
                 "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": (profiled_traffic(w) if args.kernel == "default" else None),
                 "algorithmic_bytes_per_launch": bytes_total / steps,
