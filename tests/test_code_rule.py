@@ -1,6 +1,7 @@
-"""The quantizer's code rule (csrc/kivi_codes.cuh), built for the host: the
-reciprocal fast path with its exact-division fallback gives
-clamp(round_half_even(fl(d / s)), 0, L) -- the code the method defines --
+"""The quantizer's code rules (csrc/kivi_codes.cuh), built for the host: the
+reciprocal fast path with its exact-division fallback (code_of), and the
+rounding by 1.5 * 2^23 wherever its group check lets it stand (code_bits),
+give clamp(round_half_even(fl(d / s)), 0, L) -- the code the method defines --
 on random quotients and, above all, on quotients within a few ulps of every
 half-integer, on exact ties, and on scales whose reciprocal overflows."""
 import ctypes
@@ -32,6 +33,34 @@ extern "C" long long t_mismatches(const float* d, const float* s, long long n, i
   }
   return bad;
 }
+// code_bits (the group-checked rounding): wherever codes_need_exact lets it
+// stand, its code must equal the exact one; *flagged counts the rest
+extern "C" long long t_bits_mismatches(const float* d, const float* s, long long n, int L,
+                                       long long* first, long long* flagged) {
+  long long bad = 0;
+  *first = -1;
+  *flagged = 0;
+  for (long long i = 0; i < n; ++i) {
+    const float rs = kivi::recip_rn(s[i]);
+    float ae = 0.0f;
+    const unsigned bits = kivi::code_bits(d[i], s[i] != 0.0f ? rs : 0.0f, (float)L, &ae);
+    if (s[i] != 0.0f && kivi::codes_need_exact(ae, rs)) {
+      ++*flagged;
+      continue;
+    }
+    int want = 0;
+    if (s[i] != 0.0f) {  // a conversion that saturates: inf to L, NaN to 0
+      volatile float qv = d[i] / s[i];
+      const float q = qv;
+      want = q >= (float)L ? L : (q > 0.0f ? (int)nearbyintf(q) : 0);
+    }
+    if ((long long)bits - 0x4B400000LL != want) {
+      if (*first < 0) *first = i;
+      ++bad;
+    }
+  }
+  return bad;
+}
 '''
 
 
@@ -50,6 +79,10 @@ def rule_lib(tmp_path_factory):
     L.t_mismatches.restype = ctypes.c_longlong
     L.t_mismatches.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int,
                                ctypes.POINTER(ctypes.c_longlong)]
+    L.t_bits_mismatches.restype = ctypes.c_longlong
+    L.t_bits_mismatches.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong,
+                                    ctypes.c_int, ctypes.POINTER(ctypes.c_longlong),
+                                    ctypes.POINTER(ctypes.c_longlong)]
     return L
 
 
@@ -59,6 +92,11 @@ def check(lib, d, s, L):
     first = ctypes.c_longlong()
     bad = lib.t_mismatches(d.ctypes.data, s.ctypes.data, d.size, L, ctypes.byref(first))
     assert bad == 0, (bad, float(d[first.value]), float(s[first.value]))
+    flagged = ctypes.c_longlong()
+    bad = lib.t_bits_mismatches(d.ctypes.data, s.ctypes.data, d.size, L, ctypes.byref(first),
+                                ctypes.byref(flagged))
+    assert bad == 0, ("code_bits", bad, float(d[first.value]), float(s[first.value]))
+    return flagged.value
 
 
 @pytest.mark.parametrize("L", [1, 3, 7, 15])
@@ -68,7 +106,8 @@ def test_random_quotients(rule_lib, L):
     s = (10.0 ** rng.uniform(-30, 30, n)).astype(np.float32)
     s = s[(s > 0) & np.isfinite(s)]
     d = (s.astype(np.float64) * rng.uniform(0, L * 1.02, s.size)).astype(np.float32)
-    check(rule_lib, d, s, L)
+    flagged = check(rule_lib, d, s, L)
+    assert flagged < 1e-4 * d.size  # the group check rarely sends a group to code_of
 
 
 @pytest.mark.parametrize("L", [1, 3, 15])

@@ -79,10 +79,35 @@ def test_prefill_equals_appends(T):
         assert torch.equal(a.view(name)[:, :, :lim[name]], b.view(name)[:, :, :lim[name]]), name
 
 
-def test_special_values_bit_exact():
+@pytest.mark.parametrize("misaligned", [False, True], ids=["aligned", "misaligned"])
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_prefill_paths_bit_exact(bits, dtype, misaligned):
+    """The prefill's staged path (16-byte aligned K and V) and its general path
+    (K and V one element past an aligned address) both match the oracle."""
+    w = small(D=128, bits=bits, dtype=dtype, R=64, T=32 * 9 + 7, B=2, Hkv=2, seed=3)
+    K, V = W.prompt_kv(w, device="cuda")
+    if misaligned:
+        def shift(x):
+            buf = torch.empty(x.numel() + 1, dtype=x.dtype, device=x.device)
+            y = buf[1:].view(x.shape)
+            y.copy_(x)
+            assert y.data_ptr() % 16 != 0
+            return y
+        K, V = shift(K), shift(V)
+    gc = gpu_cache(w, capacity=512)
+    gc.prefill(K, V)
+    oc = oracle_cache(w, capacity=512)
+    oracle_prefill(oc, K, V)
+    assert_state_equal(gc, oc)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_special_values_bit_exact(D, dtype):
     """Signed zeros (first occurrence decides the zero's sign), constant groups
     (scale 0), fp16 extremes and subnormals, huge outlier channels."""
-    w = small(D=64, bits=2, R=32, T=32 * 6 + 3, B=1, Hkv=2, dtype="f16")
+    w = small(D=D, bits=2, R=32, T=32 * 6 + 3, B=1, Hkv=2, dtype=dtype)
     K, V = W.prompt_kv(w, device="cuda")
     K[0, 0, 0:32, 0] = 0.0                       # constant channel group
     K[0, 0, 0:32, 1] = -0.0
@@ -99,6 +124,20 @@ def test_special_values_bit_exact():
     V[0, 1, 5, 0:16] = 0.0
     V[0, 1, 5, 16:32] = -0.0
     V[0, 1, 6, 32:64] = torch.arange(32, device="cuda", dtype=torch.float16) * 1e3
+    V[0, 0, 7, 0:32] = torch.arange(32, device="cuda", dtype=V.dtype)  # min +0, then -0
+    V[0, 0, 7, 9] = -0.0
+    V[0, 0, 8, 0:32] = torch.arange(32, device="cuda", dtype=V.dtype)  # min -0 first
+    V[0, 0, 8, 0] = -0.0
+    V[0, 0, 8, 17] = 0.0
+    V[0, 1, 9, 0:32] = -torch.arange(32, device="cuda", dtype=V.dtype) - 1  # max -0 first
+    V[0, 1, 9, 30] = -0.0
+    V[0, 1, 9, 31] = 0.0
+    K[0, 1, 128:160, 9] = -torch.arange(32, device="cuda", dtype=K.dtype) - 1  # max +0 first
+    K[0, 1, 140, 9] = 0.0
+    K[0, 1, 150, 9] = -0.0
+    K[0, 0, 128:160, 10] = torch.arange(32, device="cuda", dtype=K.dtype)  # min -0 late
+    K[0, 0, 128, 10] = 1.0
+    K[0, 0, 159, 10] = -0.0
     gc = gpu_cache(w, capacity=512)
     gc.prefill(K, V)
     oc = oracle_cache(w, capacity=512)
