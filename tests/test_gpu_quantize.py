@@ -138,6 +138,13 @@ def test_special_values_bit_exact(D, dtype):
     K[0, 0, 128:160, 10] = torch.arange(32, device="cuda", dtype=K.dtype)  # min -0 late
     K[0, 0, 128, 10] = 1.0
     K[0, 0, 159, 10] = -0.0
+    if dtype == "f32":
+        # subnormal ranges: the scale's reciprocal overflows, the exact division decides
+        tiny = torch.arange(32, device="cuda", dtype=torch.float64) * 2.0 ** -149
+        K[0, 0, 32:64, 20] = tiny.float()
+        K[0, 1, 96:128, 21] = (tiny * 3).float()
+        V[0, 0, 10, 0:32] = tiny.float()
+        V[0, 1, 11, 32:64] = (tiny * 5).float()
     gc = gpu_cache(w, capacity=512)
     gc.prefill(K, V)
     oc = oracle_cache(w, capacity=512)
@@ -177,4 +184,55 @@ def test_large_batch_workload_sampled(w):
     units = sample_units(w, 24)
     oc = oracle_cache(w, units=units)
     oracle_prefill(oc, K, V)
+    assert_state_equal(gc, oc)
+
+
+@pytest.mark.parametrize("D", [32, 128])
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+@pytest.mark.parametrize("bits", [2, 4])
+def test_half_integer_quotients_bit_exact(bits, dtype, D):
+    """Groups whose quotients (x - min) / s land exactly on half-integers
+    (power-of-two scales: ties, rounded to even) or, for binary32 inputs,
+    one ulp either side of them: the quantizers' rounding check hands these
+    to the exact division, in the prompt quantizer and in the flush."""
+    L = (1 << bits) - 1
+    w = small(D=D, bits=bits, dtype=dtype, R=32, T=32 * 5 + 9, B=1, Hkv=2, seed=7)
+    K, V = W.prompt_kv(w, device="cuda")
+    tdt = K.dtype
+    half = torch.arange(32, device="cuda", dtype=torch.float64) % L + 0.5  # k + 1/2
+    base = torch.zeros(32, device="cuda", dtype=torch.float64)
+    base[0], base[1] = 0.0, float(L)  # min 0, max L: s = 1
+    for g, scale in enumerate((1.0, 0.25, 4.0)):  # key groups 0..2 of unit (0, 0), channels 0..7
+        col = base.clone()
+        col[2:] = half[2:]
+        for ch in range(8):
+            K[0, 0, 32 * g:32 * g + 32, ch] = (col * scale).to(tdt)
+    for t in range(20):  # value groups of tokens 0..19 of unit (0, 1), channel group 0
+        row = base.clone()
+        row[2:] = half[2:]
+        V[0, 1, t, 0:32] = (row * 2.0 ** (t % 5 - 2)).to(tdt)
+    if dtype == "f32":
+        # one ulp above and below each half-integer quotient (s = 1)
+        col = base.clone()
+        col[2:] = half[2:]
+        c32 = col.float()
+        upv, dnv = c32.clone(), c32.clone()
+        upv[2:] = torch.nextafter(c32[2:], torch.full_like(c32[2:], float("inf")))
+        dnv[2:] = torch.nextafter(c32[2:], torch.zeros_like(c32[2:]))
+        for ch in range(4):
+            K[0, 1, 0:32, ch] = upv
+            K[0, 1, 0:32, ch + 4] = dnv
+        V[0, 0, 3, 0:32] = upv
+        V[0, 0, 4, 0:32] = dnv
+    gc = gpu_cache(w, capacity=512)
+    gc.prefill(K, V)
+    oc = oracle_cache(w, capacity=512)
+    oracle_prefill(oc, K, V)
+    assert_state_equal(gc, oc)
+    # the window's tiles go through the flush with the same values
+    for step in range(40):
+        k = K[:, :, step % 32].contiguous()
+        v = V[:, :, step % 20].contiguous()
+        gc.append(k, v)
+        oracle_append(oc, k, v)
     assert_state_equal(gc, oc)
