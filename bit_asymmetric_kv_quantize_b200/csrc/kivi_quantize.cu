@@ -569,12 +569,16 @@ __global__ void __launch_bounds__(D, 8) prefill_staged_kernel(CacheView c, const
 // n_q and r come from st -- flush when r == R, slot = flush ? 0 : r -- and a
 // full cache is left alone with st->status = 1.  Ragged (Hkv > 0): st holds
 // one state per sequence b = unit / Hkv, each handled as above on its own.
-template <int D, int BITS, typename T, typename M>
-__global__ void __launch_bounds__(D) append_kernel(CacheView c, const T* __restrict__ k,
-                                                   const T* __restrict__ v, long long n_q,
-                                                   int slot, int flush, DevState* st, int Hkv) {
-  __shared__ uint8_t ck[kTile * D];
-  __shared__ uint8_t cv[kTile * D];
+// STAGED (no outlier lists, 16-byte aligned windows): the window tile is
+// staged and quantized as the prompt's tiles are (quantize_tile_staged, the
+// StagedSmem layout in dynamic shared memory).
+template <int D, int BITS, typename T, typename M, bool STAGED>
+__global__ void __launch_bounds__(D, STAGED ? 8 : 1)
+    append_kernel(CacheView c, const T* __restrict__ k, const T* __restrict__ v, long long n_q,
+                  int slot, int flush, DevState* st, int Hkv) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  __shared__ uint8_t ck[STAGED ? 1 : kTile * D];
+  __shared__ uint8_t cv[STAGED ? 1 : kTile * D];
   if (st != nullptr) {
     const long long sb = Hkv > 0 ? (long long)blockIdx.y / Hkv : 0;
     DevState* ss = st + sb;
@@ -601,9 +605,24 @@ __global__ void __launch_bounds__(D) append_kernel(CacheView c, const T* __restr
   const int tile = blockIdx.x;
   T* kr = reinterpret_cast<T*>(c.k_res) + unit * c.R * D;
   T* vr = reinterpret_cast<T*>(c.v_res) + unit * c.R * D;
-  if (flush)
-    quantize_tile<D, BITS, T, M, 0>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
-                                 n_q + tile * kTile, ck, cv);
+  if (flush) {
+    if constexpr (STAGED) {
+      using SM = StagedSmem<D, T>;
+      T* Ks = reinterpret_cast<T*>(dsm);
+      T* Vs = reinterpret_cast<T*>(dsm + SM::TILE_B);
+      int* vbad = reinterpret_cast<int*>(dsm + SM::O_BAD);
+      if (threadIdx.x < D / kGv) vbad[threadIdx.x] = 0;
+      stage_tile<D, T>(Ks, Vs, kr + tile * kTile * D, vr + tile * kTile * D);
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      __syncthreads();
+      quantize_tile_staged<D, BITS, T, M>(c, unit, n_q + tile * kTile, Ks, Vs, dsm + SM::O_CK,
+                                          reinterpret_cast<float4*>(dsm + SM::O_VZ),
+                                          reinterpret_cast<float2*>(dsm + SM::O_VS), vbad);
+    } else {
+      quantize_tile<D, BITS, T, M, 0>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
+                                   n_q + tile * kTile, ck, cv);
+    }
+  }
   if (tile == 0) {
     kr[(long long)slot * D + threadIdx.x] = k[unit * D + threadIdx.x];
     vr[(long long)slot * D + threadIdx.x] = v[unit * D + threadIdx.x];
@@ -651,8 +670,13 @@ template <int D, int BITS, typename T, typename M>
 cudaError_t append_t(const CacheView& c, int units, const void* k, const void* v, long long n_q,
                      int slot, bool flush, DevState* st, int Hkv, cudaStream_t s) {
   const dim3 grid((unsigned)((flush || st) ? c.R / kTile : 1), (unsigned)units);
-  append_kernel<D, BITS, T, M><<<grid, D, 0, s>>>(c, (const T*)k, (const T*)v, n_q, slot,
-                                                  flush ? 1 : 0, st, Hkv);
+  const bool aligned = (((uintptr_t)c.k_res | (uintptr_t)c.v_res) & 15u) == 0;
+  if (aligned && c.k_out == 0 && c.v_out == 0 && (flush || st))
+    append_kernel<D, BITS, T, M, true><<<grid, D, StagedSmem<D, T>::BYTES, s>>>(
+        c, (const T*)k, (const T*)v, n_q, slot, flush ? 1 : 0, st, Hkv);
+  else
+    append_kernel<D, BITS, T, M, false><<<grid, D, 0, s>>>(c, (const T*)k, (const T*)v, n_q, slot,
+                                                           flush ? 1 : 0, st, Hkv);
   return cudaGetLastError();
 }
 

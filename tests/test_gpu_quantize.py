@@ -187,6 +187,28 @@ def test_large_batch_workload_sampled(w):
     assert_state_equal(gc, oc)
 
 
+def test_large_batch_every_unit():
+    """Full-size 13B-shaped layer at 2 bits: the store of all 2560 units
+    against the oracle (fed per sequence from one host copy of the prompt),
+    and decode on 256 sampled units."""
+    w = W.LLAMA2_13B_2BIT
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w)
+    gc.prefill(K, V)
+    q = W.query(w, device="cuda")
+    out = gc.decode(q, 1.0)
+    torch.cuda.synchronize()
+    oc = oracle_cache(w)
+    for b in range(w.B):  # one sequence's heads at a time
+        kb, vb = K[b].float().cpu().numpy(), V[b].float().cpu().numpy()
+        for h in range(w.Hkv):
+            oc.prefill_unit(b, h, kb[h], vb[h])
+    del K, V
+    assert_state_equal(gc, oc)
+    from kivi_testlib import assert_decode_close
+    assert_decode_close(out, oc, q, 1.0, units=sample_units(w, 256, seed=11))
+
+
 @pytest.mark.parametrize("D", [32, 128])
 @pytest.mark.parametrize("dtype", ["f16", "f32"])
 @pytest.mark.parametrize("bits", [2, 4])
