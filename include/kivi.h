@@ -197,6 +197,11 @@ KIVI_API int kivi_cache_init(kivi_cache *cache, const kivi_dims *dims,
  * (KIVI, study.space summary: grouped parts quantized, residual parts kept
  * in full precision; mlsanity.com abstract: per-channel keys, per-token
  * values.)
+ * Any element alignment is accepted.  K and V 16-byte aligned (and no outlier
+ * lists) take the fast path, which stages each 32-token tile in shared memory
+ * by 16-byte asynchronous copies; the result is the same bit for bit.
+ * Inputs are expected finite: with a NaN in a group the scale, zero and codes
+ * of that group are unspecified.
  * Errors: KIVI_ERR_ARG, KIVI_ERR_STATE (cache not empty),
  * KIVI_ERR_CAPACITY (T > capacity), KIVI_ERR_CUDA. */
 KIVI_API int kivi_quantize_prefill(kivi_cache *cache, const void *K, const void *V,
