@@ -151,6 +151,34 @@ def test_streaming_workload_every_step():
     print(f"streaming worst max-abs {worst:.3e}")
 
 
+def test_streaming_workload_every_unit_at_flushes():
+    """The streaming workload's 512 fused steps (kivi_append_decode) with the
+    oracle holding all 128 units: every unit's store and window bit for bit
+    after each of the four window flushes, and every unit's output within
+    the bars at the first flush step, after the last flush and at the last
+    step."""
+    w = W.STREAMING
+    K, V = W.prompt_kv(w, device="cuda")
+    gc = gpu_cache(w)
+    gc.prefill(K, V)
+    oc = oracle_cache(w)
+    oracle_prefill(oc, K, V)
+    del K, V
+    checked = 0
+    for step in range(w.steps):
+        k, v = W.step_kv(w, step, device="cuda")
+        q = W.query(w, step, device="cuda")
+        out = gc.append_decode(k, v, q, 1.0)
+        oracle_append(oc, k, v)
+        if gc.r == 1:
+            assert_state_equal(gc, oc)
+        if step in (0, 3 * w.R + 1, w.steps - 1):
+            assert_decode_close(out, oc, q, 1.0)
+            checked += 1
+    assert checked == 3
+    assert gc.n_q + gc.r == w.T + w.steps
+
+
 @pytest.mark.parametrize("dtype,D", [("f16", 128), ("f16", 64), ("f32", 64)])
 @pytest.mark.parametrize("gq", [1, 4])
 def test_append_decode_matches_separate_calls(dtype, D, gq):
