@@ -10,16 +10,18 @@
 // (study.space summary: grouped and residual parts; scholarfeed.org "KIVI"
 // page, third quote: fixed-length residual buffer).
 //
-// Bit-exactness: every group is reduced by one thread in element order with
-// strict compares (first occurrence kept among equal values, which fixes the
-// sign of a zero minimum); the scale uses the IEEE round-to-nearest
-// intrinsics __fsub_rn / __fdiv_rn, and each code comes from code_of
-// (kivi_codes.cuh): the product fl(d * fl(1/s)) decides the code when it lies
-// more than 4e-6 from a half-integer, else the IEEE division __fdiv_rn does,
-// rounded half to even (__float2int_rn) and clamped.  That equals
-// clamp(round_half_even(fl(d / s)), 0, L) for every input (host build of the
-// rule checked against true division in tests/test_code_rule.py).  No
-// contraction.
+// Bit-exactness: a group's min and max are those of a strict-compare scan in
+// element order (first occurrence kept among equal values, which fixes the
+// sign of a zero minimum): the general path scans so, the staged path takes
+// order-free min/max and then gives a zero result the sign of the group's
+// first zero.  The scale uses the IEEE round-to-nearest intrinsics
+// __fsub_rn / __fdiv_rn.  Each code comes from code_of (kivi_codes.cuh: the
+// product fl(d * fl(1/s)) decides the code when it lies more than 4e-6 from a
+// half-integer, else the IEEE division does, rounded half to even and
+// clamped), or in the staged path from code_bits, whose group check hands
+// any such element to code_of.  Both equal clamp(round_half_even(fl(d / s)),
+// 0, L) for every finite input (host builds of both rules checked against
+// true division in tests/test_code_rule.py).  No contraction.
 //
 // Format variant with binary16 scales and zeros (M = __half, fp16 caches):
 // the binary32 scale and minimum are rounded to binary16 (nearest, ties to
