@@ -381,9 +381,22 @@ def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, f
     pre_us = statistics.median(e0.elapsed_time(e1) * 1e3 for e0, e1 in pre_ev[1:] or pre_ev)
     es_in = 2 if w.dtype == "f16" else 4
     pre_tokens = int(lens.sum()) if ragged else w.B * w.T
+    # bytes the prefill must move: the prompt's K and V in, the store and the
+    # window out (the decode's per-unit byte count without q and out)
+    io = 2 * w.B * w.Hq * w.D * es_in
+    if ragged:
+        r_pre = [(int(n) - 1) % w.R + 1 for n in lens.tolist()]
+        written = algorithmic_bytes(w, [int(n) - x for n, x in zip(lens.tolist(), r_pre)], r_pre,
+                                    outliers) - io
+    else:
+        r_pre = (w.T - 1) % w.R + 1
+        written = algorithmic_bytes(w, w.T - r_pre, r_pre, outliers) - io
+    pre_bytes = 2 * pre_tokens * w.Hkv * w.D * es_in + written
     prefill_times = {"call": "kivi_ragged_prefill" if ragged else "kivi_quantize_prefill",
                      "us": pre_us, "tokens_per_s": pre_tokens / (pre_us * 1e-6),
-                     "input_GBps": 2 * pre_tokens * w.Hkv * w.D * es_in / (pre_us * 1e-6) / 1e9}
+                     "input_GBps": 2 * pre_tokens * w.Hkv * w.D * es_in / (pre_us * 1e-6) / 1e9,
+                     "hbm_bytes": pre_bytes,
+                     "frac_of_hbm": pre_bytes / (pre_us * 1e-6) / 1e9 / peak_hbm()[0]}
     del Kp, Vp
     torch.cuda.empty_cache()
     P = 16
