@@ -29,7 +29,8 @@ time vs measured HBM peak, from K further steps with events recorded around
 each decode launch (events serialize consecutive launches, so this pass runs
 apart from the headline one); `e2e` = the same loop with
 the step's inputs copied from pinned host memory and the output copied back
-inside the timed region; `cpu_baseline` = the CPU oracle on a bounded sample
+inside the timed region (fused uniform steps: one `kivi_append_decode_host`
+call per step, which does both copies); `cpu_baseline` = the CPU oracle on a bounded sample
 of the same workload.  `--impl reference` times the CPU oracle alone.
 Multi-GPU (torchrun): independent replicas, one per rank (no collective on
 the data path); the barrier and max-over-ranks timing use torch.distributed.
@@ -538,20 +539,40 @@ def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, f
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        host_call = fused and not ragged  # the library's own host-buffer step
+        if host_call:
+            L.kivi_host_step_bytes.argtypes = [ctypes.POINTER(kivi.KiviCacheC), ctypes.c_int]
+            L.kivi_host_step_bytes.restype = ctypes.c_size_t
+            L.kivi_append_decode_host.argtypes = [ctypes.POINTER(kivi.KiviCacheC), ctypes.c_void_p,
+                                                  ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
+                                                  ctypes.c_void_p, ctypes.c_size_t,
+                                                  ctypes.c_void_p, ctypes.c_size_t,
+                                                  ctypes.c_void_p]
+            stg_n = int(L.kivi_host_step_bytes(cstructs[0], w.Hq))
+            stg = torch.empty(stg_n, dtype=torch.uint8, device=device)
         for j in range(n_e2e):
             i = base + j
             li = i % n_layers
-            dst.copy_(hs[i % P], non_blocking=True)
-            rc = step_call(li, dk.data_ptr(), dv.data_ptr(), dq.data_ptr())
+            if host_call:
+                # k | v | q from pinned host memory, the fused step, out back:
+                # one C-ABI call
+                n_launch[0] += 1
+                rc = L.kivi_append_decode_host(cstructs[li], hs[i % P].data_ptr(), w.Hq, 1.0,
+                                               ho.data_ptr(), stg.data_ptr(), stg_n, wp, wn, sh)
+            else:
+                dst.copy_(hs[i % P], non_blocking=True)
+                rc = step_call(li, dk.data_ptr(), dv.data_ptr(), dq.data_ptr())
+                if not rc:
+                    ho.copy_(out, non_blocking=True)
             if rc:
                 raise RuntimeError("e2e step failed")
-            ho.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(device)
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
         e2e = {"value": replica_throughput(world, w.B, n_e2e, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "ms_per_step": e_ms / n_e2e}
+               "ms_per_step": e_ms / n_e2e,
+               "call": "kivi_append_decode_host" if host_call else "copies + step call"}
 
     result = None
     if rank == 0:

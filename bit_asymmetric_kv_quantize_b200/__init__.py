@@ -36,7 +36,8 @@ EXPORTED = (
     "kivi_decode_attention_noalloc", "kivi_append_decode", "kivi_dev_state_init",
     "kivi_append_decode_dev", "kivi_ragged_prefill", "kivi_ragged_append", "kivi_ragged_decode",
     "kivi_ragged_append_decode", "kivi_paged_buffer_sizes", "kivi_paged_cache_init",
-    "kivi_outlier_buffer_sizes", "kivi_cache_set_outliers",
+    "kivi_outlier_buffer_sizes", "kivi_cache_set_outliers", "kivi_host_step_bytes",
+    "kivi_append_decode_host",
 )
 OUTLIER_NAMES = ("k_out_idx", "k_out_val", "v_out_idx", "v_out_val")
 
@@ -94,6 +95,10 @@ def lib() -> ctypes.CDLL:
             L.kivi_decode_attention_simt.argtypes = dec
             L.kivi_decode_attention_noalloc.argtypes = [cp, vp, ci, ctypes.c_float, vp, vp]
             L.kivi_append_decode.argtypes = [cp, vp, vp, vp, ci, ctypes.c_float, vp, vp, sz, vp]
+            L.kivi_host_step_bytes.argtypes = [cp, ci]
+            L.kivi_host_step_bytes.restype = sz
+            L.kivi_append_decode_host.argtypes = [cp, vp, ci, ctypes.c_float, vp, vp, sz, vp, sz,
+                                                  vp]
             L.kivi_dev_state_init.argtypes = [cp, vp, vp]
             L.kivi_append_decode_dev.argtypes = [cp, vp, vp, vp, vp, ci, ctypes.c_float, vp, vp, sz,
                                                  vp]
@@ -196,6 +201,7 @@ class KiviCache:
                    "kivi_cache_set_outliers")
         self._ws: Optional[torch.Tensor] = None
         self._ws_dev: Optional[torch.Tensor] = None
+        self._staging: Optional[torch.Tensor] = None
         E, WB = _code_block(bits)
         self.B, self.Hkv, self.D, self.bits, self.R, self.capacity = B, Hkv, D, bits, R, capacity
         self.shapes = {
@@ -346,6 +352,31 @@ class KiviCache:
                                             self._stream()), "kivi_append_decode")
         return out
 
+    def append_decode_host(self, kvq: torch.Tensor, Hq: int, softmax_scale: float,
+                           out: torch.Tensor) -> torch.Tensor:
+        """kivi_append_decode_host: kvq is a host tensor (pinned for the copies
+        to be asynchronous) holding k [B][Hkv][D], v [B][Hkv][D] and q
+        [B][Hq][D] back to back; out a host [B][Hq][D] tensor that holds the
+        result once the stream has reached the end of the call."""
+        n_in = (2 * self.B * self.Hkv + self.B * Hq) * self.D
+        for t, n, name in ((kvq, n_in, "kvq"), (out, self.B * Hq * self.D, "out")):
+            if t.device.type != "cpu" or t.dtype != self.dtype or not t.is_contiguous() \
+                    or t.numel() != n:
+                raise ValueError(f"{name}: expected a contiguous host {self.dtype} tensor of {n} "
+                                 "elements")
+        with torch.cuda.device(self.device):
+            need = int(lib().kivi_host_step_bytes(ctypes.byref(self._c), Hq))
+            if need == 0:
+                raise KiviError(1, "kivi_host_step_bytes")
+            if self._staging is None or self._staging.numel() < need:
+                self._staging = torch.empty(need, dtype=torch.uint8, device=self.device)
+            ws = self.workspace(Hq)
+            _check(lib().kivi_append_decode_host(ctypes.byref(self._c), kvq.data_ptr(), Hq,
+                                                 float(softmax_scale), out.data_ptr(),
+                                                 self._staging.data_ptr(), self._staging.numel(),
+                                                 ws.data_ptr(), ws.numel(), self._stream()),
+                   "kivi_append_decode_host")
+        return out
 
     # -- ragged batches (per-sequence lengths on the device)
     def ragged_prefill(self, K: torch.Tensor, V: torch.Tensor, lens: torch.Tensor) -> torch.Tensor:

@@ -512,6 +512,46 @@ int kivi_decode_attention(const kivi_cache* cache, const void* q, int Hq, float 
                        false);
 }
 
+// Staging layout of kivi_append_decode_host: k | v | q back to back (each a
+// whole number of 16-byte chunks, since D * element size is), then out at the
+// next 16-byte boundary.
+size_t kivi_host_step_bytes(const kivi_cache* cache, int Hq) {
+  if (check_cache(cache) != KIVI_OK || Hq <= 0 || Hq % cache->dims.Hkv != 0) return 0;
+  const kivi_dims& d = cache->dims;
+  const size_t es = d.dtype == KIVI_F16 ? 2 : 4;
+  const size_t kv = (size_t)d.B * d.Hkv * d.D * es, qo = (size_t)d.B * Hq * d.D * es;
+  const size_t in = (2 * kv + qo + 15) / 16 * 16;
+  return in + (qo + 15) / 16 * 16;
+}
+
+int kivi_append_decode_host(kivi_cache* cache, const void* host_kvq, int Hq, float softmax_scale,
+                            void* host_out, void* staging, size_t staging_bytes, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  const size_t need = kivi_host_step_bytes(cache, Hq);
+  if (need == 0 || !host_kvq || !host_out || !staging || ((uintptr_t)staging & 15))
+    return KIVI_ERR_ARG;
+  if (staging_bytes < need) return KIVI_ERR_WORKSPACE;
+  // the refusals that need no device, before the copy (kivi_append_decode
+  // checks everything again)
+  if (device_counted(cache)) return KIVI_ERR_STATE;
+  if (cache->n_q + cache->r + 1 > cache->dims.capacity) return KIVI_ERR_CAPACITY;
+  const kivi_dims& d = cache->dims;
+  const size_t es = d.dtype == KIVI_F16 ? 2 : 4;
+  const size_t kv = (size_t)d.B * d.Hkv * d.D * es, qo = (size_t)d.B * Hq * d.D * es;
+  unsigned char* st = static_cast<unsigned char*>(staging);
+  unsigned char* out = st + (2 * kv + qo + 15) / 16 * 16;
+  cudaStream_t s = (cudaStream_t)stream;
+  // inputs in one copy, the fused step on them, out back in one copy
+  if (cudaMemcpyAsync(st, host_kvq, 2 * kv + qo, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  const int rc = kivi_append_decode(cache, st, st + kv, st + 2 * kv, Hq, softmax_scale, out,
+                                    workspace, ws_bytes, stream);
+  if (rc != KIVI_OK) return rc;
+  if (cudaMemcpyAsync(host_out, out, qo, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  return KIVI_OK;
+}
+
 int kivi_append_decode(kivi_cache* cache, const void* k, const void* v, const void* q, int Hq,
                        float softmax_scale, void* out, void* workspace, size_t ws_bytes,
                        void* stream) {

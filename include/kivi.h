@@ -268,6 +268,31 @@ KIVI_API int kivi_append_decode(kivi_cache *cache, const void *k, const void *v,
                        const void *q, int Hq, float softmax_scale, void *out,
                        void *workspace, size_t workspace_bytes, void *stream);
 
+/* Bytes of device staging kivi_append_decode_host needs for Hq query heads
+ * (0 on error).  Host arithmetic only. */
+KIVI_API size_t kivi_host_step_bytes(const kivi_cache *cache, int Hq);
+
+/* kivi_append_decode from host memory: one step of a decode loop whose
+ * token and query arrive from, and whose output goes back to, the host.
+ * host_kvq: host, dims.dtype, k [B][Hkv][D], v [B][Hkv][D] and q [B][Hq][D]
+ * back to back.  host_out: host, dims.dtype, [B][Hq][D].  Both should be
+ * page-locked (cudaHostAlloc or registered) for the copies to be
+ * asynchronous.  staging: device, 16-byte aligned, at least
+ * kivi_host_step_bytes(cache, Hq) bytes, owned by the caller; its contents
+ * are scratch.  On `stream`: one host-to-device copy of the inputs into
+ * staging, the fused step of kivi_append_decode on them (one launch), one
+ * device-to-host copy of out into host_out.  All are asynchronous: host_out
+ * holds the result once the stream has reached the end of the call.  The
+ * host counters advance as for kivi_append_decode.
+ * Errors: KIVI_ERR_ARG (null pointer, misaligned staging, Hq not a multiple
+ * of Hkv), KIVI_ERR_WORKSPACE (staging too small), those of
+ * kivi_append_decode (nothing is copied back and the counters stay as they
+ * were), KIVI_ERR_CUDA (a copy failed to enqueue). */
+KIVI_API int kivi_append_decode_host(kivi_cache *cache, const void *host_kvq, int Hq,
+                                     float softmax_scale, void *host_out, void *staging,
+                                     size_t staging_bytes, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
 /* Device-resident counters of a cache: 16 bytes of device memory, 16-byte
  * aligned, laid out as { long long n_q; int r; int status; }.  With them a
  * decode loop runs without host round trips and can be captured in a CUDA

@@ -14,7 +14,7 @@ from bit_asymmetric_kv_quantize_b200 import KiviCacheC, KiviDims
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "kivi.h")
 
-ERR_ARG, ERR_UNSUPPORTED, ERR_STATE, ERR_CAPACITY = 1, 2, 3, 4
+ERR_ARG, ERR_UNSUPPORTED, ERR_STATE, ERR_CAPACITY, ERR_WORKSPACE = 1, 2, 3, 4, 5
 
 
 def declared_symbols():
@@ -166,6 +166,40 @@ def test_host_side_state_and_capacity_errors():
     assert L.kivi_append_decode(ctypes.byref(c), fake, fake, None, 4, 1.0, fake, fake, 1 << 20,
                                 None) == ERR_ARG
     assert (c.n_q, c.r) == (0, 5)
+
+
+def test_host_step_validates_before_any_copy():
+    """kivi_host_step_bytes is host arithmetic (k | v | q, then out at the
+    next 16-byte boundary); kivi_append_decode_host refuses bad arguments and
+    a full cache before it copies anything."""
+    L = kivi.lib()
+    L.kivi_host_step_bytes.argtypes = [ctypes.POINTER(KiviCacheC), ctypes.c_int]
+    L.kivi_host_step_bytes.restype = ctypes.c_size_t
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    L.kivi_append_decode_host.argtypes = [ctypes.POINTER(KiviCacheC), vp, ctypes.c_int,
+                                          ctypes.c_float, vp, vp, sz, vp, sz, vp]
+    c = _fake_cache(R=128, capacity=256)
+    B, Hkv, D = c.dims.B, c.dims.Hkv, c.dims.D
+    es = 2 if c.dims.dtype == 0 else 4
+    for Hq in (Hkv, 2 * Hkv):
+        kv, qo = B * Hkv * D * es, B * Hq * D * es
+        want = -(-(2 * kv + qo) // 16) * 16 + -(-qo // 16) * 16
+        assert L.kivi_host_step_bytes(ctypes.byref(c), Hq) == want
+    assert L.kivi_host_step_bytes(ctypes.byref(c), Hkv + 1) == 0
+    need = L.kivi_host_step_bytes(ctypes.byref(c), Hkv)
+    host, dev = vp(0x7000), vp(0x9000)
+
+    def call(kvq=host, out=host, staging=dev, nbytes=need, Hq=Hkv):
+        return L.kivi_append_decode_host(ctypes.byref(c), kvq, Hq, 1.0, out, staging, nbytes, dev,
+                                         1 << 20, None)
+    assert call(kvq=None) == ERR_ARG
+    assert call(out=None) == ERR_ARG
+    assert call(staging=vp(0x9008)) == ERR_ARG  # misaligned staging
+    assert call(Hq=Hkv + 1) == ERR_ARG
+    assert call(nbytes=need - 1) == ERR_WORKSPACE
+    c.n_q, c.r = 128, 128  # full
+    assert call() == ERR_CAPACITY
+    assert (c.n_q, c.r) == (128, 128)
 
 
 def test_status_strings():

@@ -455,3 +455,31 @@ def test_three_bit_layer_sampled(gq):
         if step % 40 == 0 or step == 129:
             assert_decode_close(out, oc, q, sigma, units)
     assert_state_equal(gc, oc, units)
+
+
+@pytest.mark.parametrize("dtype,D,gq", [("f16", 128, 1), ("f16", 64, 4), ("f32", 64, 1)])
+def test_append_decode_host_matches_device_call(dtype, D, gq):
+    """kivi_append_decode_host (inputs from pinned host memory, output back
+    to host memory, one call) equals kivi_append_decode on device tensors bit
+    for bit, over 70 steps that cross a flush (R = 64)."""
+    w = small(D=D, dtype=dtype, gq=gq, T=100, R=64, B=2, Hkv=2, seed=13)
+    K, V = W.prompt_kv(w, device="cuda")
+    a, b = gpu_cache(w, capacity=512), gpu_cache(w, capacity=512)
+    a.prefill(K, V)
+    b.prefill(K, V)
+    out = torch.empty(w.B, w.Hq, w.D, dtype=w.torch_dtype).pin_memory()
+    for step in range(70):
+        k, v = W.step_kv(w, step, device="cuda")
+        q = W.query(w, step, device="cuda")
+        kvq = torch.cat([k.flatten(), v.flatten(), q.flatten()]).cpu().pin_memory()
+        ref = b.append_decode(k, v, q, 1.0)
+        a.append_decode_host(kvq, w.Hq, 1.0, out)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref.cpu()), step
+        assert (a.n_q, a.r) == (b.n_q, b.r)
+    n_q, r = a.n_q, a.r
+    E = 32 // w.bits
+    lim = {"k_codes": n_q, "k_scale": n_q // 32, "k_zero": n_q // 32, "v_codes": n_q // E,
+           "v_scale": n_q, "v_zero": n_q, "k_res": r, "v_res": r}
+    for name in kivi.BUFFER_NAMES:  # the written parts of the store and window
+        assert torch.equal(a.view(name)[:, :, :lim[name]], b.view(name)[:, :, :lim[name]]), name
