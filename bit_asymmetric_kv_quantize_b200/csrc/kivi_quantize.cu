@@ -161,6 +161,31 @@ __device__ __forceinline__ F2 load2<float>(const float* p) {
   return f2(h.x, h.y);
 }
 
+// Element (t, d) of a staged tile: half-precision tiles of D >= 64 channels
+// keep tokens 16 .. 31 with the 32-element halves of each 64-element block
+// swapped.
+template <int D, typename T>
+__device__ __forceinline__ int stage_idx(int t, int d) {
+  return t * D + ((D >= 64 && sizeof(T) == 2) ? (d ^ (((t >> 4) & 1) << 5)) : d);
+}
+
+// Issue the asynchronous 16-byte copies of one tile of K and V (kTile rows of
+// D elements from Ksrc, Vsrc, 16-byte aligned) into Ks, Vs (stage_idx order),
+// as one group.
+template <int D, typename T>
+__device__ __forceinline__ void stage_tile(T* Ks, T* Vs, const T* __restrict__ Ksrc,
+                                           const T* __restrict__ Vsrc) {
+  constexpr int EPC = 16 / (int)sizeof(T);  // elements per 16-byte chunk
+  constexpr int NCH = kTile * D / EPC;      // chunks per tile
+#pragma unroll
+  for (int i = threadIdx.x; i < NCH; i += D) {
+    const int t = i / (D / EPC), d = (i % (D / EPC)) * EPC;
+    cp_async16(Ks + stage_idx<D, T>(t, d), Ksrc + i * EPC);
+    cp_async16(Vs + stage_idx<D, T>(t, d), Vsrc + i * EPC);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
 // One 32-token tile of one unit quantized from its staged copy (stage_tile,
 // complete and visible to the block): the prefill's fast path (no outlier
 // lists).  blockDim.x == D; vbad[0 .. NJ) must be 0 on entry.  Lane l of warp w
@@ -176,30 +201,6 @@ __device__ __forceinline__ F2 load2<float>(const float* p) {
 // tokens 16 .. 31 are stored with 32-element halves swapped, so that the two
 // halves of a warp read and write different banks.  Codes, scales and zeros
 // equal those of quantize_tile bit for bit.
-// Element (t, d) of a staged tile: half-precision tiles of D >= 64 channels
-// keep tokens 16 .. 31 with the 32-element halves of each 64-element block
-// swapped.
-template <int D, typename T>
-__device__ __forceinline__ int stage_idx(int t, int d) {
-  return t * D + ((D >= 64 && sizeof(T) == 2) ? (d ^ (((t >> 4) & 1) << 5)) : d);
-}
-
-// Issue the asynchronous 16-byte copies of one tile of K and V (kTile rows of
-// D elements from Ksrc, Vsrc, 16-byte aligned) into Ks, Vs, as one group.
-template <int D, typename T>
-__device__ __forceinline__ void stage_tile(T* Ks, T* Vs, const T* __restrict__ Ksrc,
-                                           const T* __restrict__ Vsrc) {
-  constexpr int EPC = 16 / (int)sizeof(T);  // elements per 16-byte chunk
-  constexpr int NCH = kTile * D / EPC;      // chunks per tile
-#pragma unroll
-  for (int i = threadIdx.x; i < NCH; i += D) {
-    const int t = i / (D / EPC), d = (i % (D / EPC)) * EPC;
-    cp_async16(Ks + stage_idx<D, T>(t, d), Ksrc + i * EPC);
-    cp_async16(Vs + stage_idx<D, T>(t, d), Vsrc + i * EPC);
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
 template <int D, int BITS, typename T, typename M>
 __device__ __forceinline__ void quantize_tile_staged(const CacheView& c, long long unit,
                                                      long long t0, const T* Ks, const T* Vs,
