@@ -486,7 +486,7 @@ __global__ void __launch_bounds__(D) prefill_kernel(CacheView c, const T* __rest
     if (!ok) return;
   }
   if (tile < n_q / kTile) {
-    quantize_tile<D, BITS, T, M, 0>(c, unit, Ku + tile * kTile * D, Vu + tile * kTile * D,
+    quantize_tile<D, BITS, T, M, 0, true>(c, unit, Ku + tile * kTile * D, Vu + tile * kTile * D,
                                  tile * kTile, ck, cv);
   } else if (tile == gridDim.x - 1) {
     T* kr = reinterpret_cast<T*>(c.k_res) + unit * c.R * D;
@@ -622,7 +622,7 @@ __global__ void __launch_bounds__(D, STAGED ? 8 : 1)
                                           reinterpret_cast<float4*>(dsm + SM::O_VZ),
                                           reinterpret_cast<float2*>(dsm + SM::O_VS), vbad);
     } else {
-      quantize_tile<D, BITS, T, M, 0>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
+      quantize_tile<D, BITS, T, M, 0, true>(c, unit, kr + tile * kTile * D, vr + tile * kTile * D,
                                    n_q + tile * kTile, ck, cv);
     }
   }

@@ -38,8 +38,9 @@ __device__ __forceinline__ void tile_sync() {
 // block call this and synchronize on named barrier BAR (the others must not).
 // Paged stores: the tile goes to its page's slot (a page outside the block
 // table or the pool writes nothing; the callers have refused such a
-// sequence already).
-template <int D, int BITS, typename T, typename M, int BAR>
+// sequence already).  REG: outlier-list groups take quantize_group_sparse_reg
+// (same output, the group kept in registers) instead of quantize_group_sparse.
+template <int D, int BITS, typename T, typename M, int BAR, bool REG = false>
 __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit,
                                               const T* __restrict__ Ksrc,
                                               const T* __restrict__ Vsrc, long long t0,
@@ -69,7 +70,10 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
         // kept exactly (listed in index order, dense code 0), the rest quantized
         float s, z, ov[kMaxOut];
         int codes[kTile], oi[kMaxOut];
-        quantize_group_sparse<kTile, kMaxOut>(x, c.k_out, BITS, &s, &z, codes, oi, ov);
+        if constexpr (REG)
+          quantize_group_sparse_reg<kTile, kMaxOut>(x, c.k_out, BITS, &s, &z, codes, oi, ov);
+        else
+          quantize_group_sparse<kTile, kMaxOut>(x, c.k_out, BITS, &s, &z, codes, oi, ov);
         c.k_scale_f()[unit * Lt::k_meta_unit(Ts) + g * D + tid] = s;
         c.k_zero_f()[unit * Lt::k_meta_unit(Ts) + g * D + tid] = z;
 #pragma unroll
@@ -115,7 +119,10 @@ __device__ __forceinline__ void quantize_tile(const CacheView& c, long long unit
       if (c.v_out > 0) {
         float s, z, ov[kMaxOut];
         int codes[kGv], oi[kMaxOut];
-        quantize_group_sparse<kGv, kMaxOut>(x, c.v_out, BITS, &s, &z, codes, oi, ov);
+        if constexpr (REG)
+          quantize_group_sparse_reg<kGv, kMaxOut>(x, c.v_out, BITS, &s, &z, codes, oi, ov);
+        else
+          quantize_group_sparse<kGv, kMaxOut>(x, c.v_out, BITS, &s, &z, codes, oi, ov);
         c.v_scale_f()[mo] = s;
         c.v_zero_f()[mo] = z;
 #pragma unroll

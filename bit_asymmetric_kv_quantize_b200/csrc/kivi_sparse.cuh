@@ -76,4 +76,86 @@ KIVI_HD inline void quantize_group_sparse(const float (&x)[N], int k, int bits, 
   }
 }
 
+#if defined(__CUDA_ARCH__)
+#define KIVI_UNROLL _Pragma("unroll")
+#else
+#define KIVI_UNROLL
+#endif
+
+// quantize_group_sparse with every array indexed at positions known when the
+// loops are unrolled: the kept set is a bit mask, each pass remembers its pick
+// by value, and the picks are sorted by index at the end (a kernel then keeps
+// the group in registers instead of local memory).  The same selection (k
+// passes, larger magnitude first, lower index on ties), bounds, codes and
+// lists bit for bit; out_idx / out_val entries past k are N / 0.  N <= 32.
+template <int N, int K>
+KIVI_HD inline void quantize_group_sparse_reg(const float (&x)[N], int k, int bits, float* scale,
+                                              float* zero, int (&codes)[N], int (&out_idx)[K],
+                                              float (&out_val)[K]) {
+  static_assert(N <= 32, "one mask bit per element");
+  uint32_t outm = 0u;
+  int pi[K];
+  float pv[K];
+  KIVI_UNROLL
+  for (int m = 0; m < K; ++m) {  // k arg-max passes over the magnitudes
+    pi[m] = N;
+    pv[m] = 0.f;
+    if (m < k) {
+      int best = -1;
+      float ba = 0.f, bx = 0.f;
+      KIVI_UNROLL
+      for (int i = 0; i < N; ++i) {
+        const float a = fabsf(x[i]);
+        const bool pick = !((outm >> i) & 1u) && (best < 0 || a > ba);
+        best = pick ? i : best;
+        ba = pick ? a : ba;
+        bx = pick ? x[i] : bx;
+      }
+      outm |= 1u << best;
+      pi[m] = best;
+      pv[m] = bx;
+    }
+  }
+  KIVI_UNROLL
+  for (int a = 0; a < K; ++a) {  // the lists in index order
+    KIVI_UNROLL
+    for (int b = 0; b + 1 < K - a; ++b) {
+      if (pi[b] > pi[b + 1]) {
+        const int ti = pi[b];
+        pi[b] = pi[b + 1];
+        pi[b + 1] = ti;
+        const float tv = pv[b];
+        pv[b] = pv[b + 1];
+        pv[b + 1] = tv;
+      }
+    }
+  }
+  float mn = 0.f, mx = 0.f;
+  bool first = true;
+  KIVI_UNROLL
+  for (int i = 0; i < N; ++i) {
+    if ((outm >> i) & 1u) continue;
+    if (first) {
+      mn = mx = x[i];
+      first = false;
+    } else {
+      if (x[i] < mn) mn = x[i];
+      if (x[i] > mx) mx = x[i];
+    }
+  }
+  const int L = (1 << bits) - 1;
+  const float s = div_rn(sub_rn(mx, mn), (float)L);
+  const float rs = recip_rn(s);
+  *scale = s;
+  *zero = mn;
+  KIVI_UNROLL
+  for (int i = 0; i < N; ++i)
+    codes[i] = ((outm >> i) & 1u) || s == 0.0f ? 0 : code_of(sub_rn(x[i], mn), s, rs, L);
+  KIVI_UNROLL
+  for (int m = 0; m < K; ++m) {
+    out_idx[m] = pi[m];
+    out_val[m] = pv[m];
+  }
+}
+
 }  // namespace kivi

@@ -31,6 +31,20 @@ extern "C" void t_group(const float* x, int k, int bits, float* s, float* z, int
     val[m] = ov[m];
   }
 }
+// the register-resident form the prompt and append kernels run
+extern "C" void t_group_reg(const float* x, int k, int bits, float* s, float* z, int* codes,
+                            int* idx, float* val) {
+  float xs[32];
+  int c[32], oi[4];
+  float ov[4];
+  for (int i = 0; i < 32; ++i) xs[i] = x[i];
+  kivi::quantize_group_sparse_reg<32, 4>(xs, k, bits, s, z, c, oi, ov);
+  for (int i = 0; i < 32; ++i) codes[i] = c[i];
+  for (int m = 0; m < k; ++m) {
+    idx[m] = oi[m];
+    val[m] = ov[m];
+  }
+}
 '''
 
 
@@ -46,24 +60,26 @@ def group_lib(tmp_path_factory):
     subprocess.run([cxx, "-std=c++17", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
                     "-shared", "-I", CSRC, "-o", str(so), str(src)], check=True)
     L = ctypes.CDLL(str(so))
-    L.t_group.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
-                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    for f in (L.t_group, L.t_group_reg):
+        f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     return L
 
 
-def run(lib, x, k, bits):
+def run(lib, x, k, bits, fn="t_group"):
     x = np.ascontiguousarray(x, np.float32)
     s, z = np.zeros(1, np.float32), np.zeros(1, np.float32)
     c = np.zeros(32, np.int32)
     oi, ov = np.zeros(4, np.int32), np.zeros(4, np.float32)
-    lib.t_group(x.ctypes.data, k, bits, s.ctypes.data, z.ctypes.data, c.ctypes.data,
-                oi.ctypes.data, ov.ctypes.data)
+    getattr(lib, fn)(x.ctypes.data, k, bits, s.ctypes.data, z.ctypes.data, c.ctypes.data,
+                     oi.ctypes.data, ov.ctypes.data)
     return s[0], z[0], c, oi[:k], ov[:k]
 
 
+@pytest.mark.parametrize("fn", ["t_group", "t_group_reg"])
 @pytest.mark.parametrize("bits", [1, 2, 3, 4])
 @pytest.mark.parametrize("k", [0, 1, 2, 4])
-def test_matches_the_oracle_bit_for_bit(group_lib, bits, k):
+def test_matches_the_oracle_bit_for_bit(group_lib, bits, k, fn):
     rng = np.random.default_rng(bits * 10 + k)
     for trial in range(3000):
         x = rng.standard_normal(32).astype(np.float32) * np.float32(10.0 ** rng.uniform(-6, 6))
@@ -74,7 +90,7 @@ def test_matches_the_oracle_bit_for_bit(group_lib, bits, k):
             x[3] = -x[5]
         if trial % 7 == 0:
             x[:] = x[0]                            # a constant group: scale 0
-        s, z, c, oi, ov = run(group_lib, x, k, bits)
+        s, z, c, oi, ov = run(group_lib, x, k, bits, fn)
         s0, z0, c0, oi0, ov0 = oracle.quantize_group_sparse(x, bits, k)
         assert np.float32(s).view(np.uint32) == np.float32(s0).view(np.uint32)
         assert np.float32(z).view(np.uint32) == np.float32(z0).view(np.uint32)
@@ -97,7 +113,9 @@ __global__ void k(const float* x, int kk, int bits, float* out, int* codes) {
   int c[32], oi[4];
   float ov[4], s, z;
   kivi::quantize_group_sparse<32, 4>(xs, kk, bits, &s, &z, c, oi, ov);
-  out[threadIdx.x] = s + z + ov[0];
+  float s2, z2;
+  kivi::quantize_group_sparse_reg<32, 4>(xs, kk, bits, &s2, &z2, c, oi, ov);
+  out[threadIdx.x] = s + z + ov[0] + s2 + z2;
   for (int i = 0; i < 32; ++i) codes[threadIdx.x * 32 + i] = c[i] + oi[i & 3];
 }
 ''')
