@@ -142,6 +142,20 @@ def test_uniform_calls_stay_inside_their_buffers(D, bits, dtype, gq):
     assert rc == 0
     assert_decode_close(out, oc, q, sigma)
     assert_guards()
+    # the host-buffer step writes only its staging (and the cache)
+    L.kivi_host_step_bytes.argtypes = [ctypes.POINTER(kivi.KiviCacheC), ctypes.c_int]
+    L.kivi_host_step_bytes.restype = ctypes.c_size_t
+    gc._staging = Guarded(int(L.kivi_host_step_bytes(ctypes.byref(gc._c), w.Hq))).inner
+    hout = torch.empty(w.B, w.Hq, D, dtype=w.torch_dtype).pin_memory()
+    for step in range(4):
+        k, v = W.step_kv(w, 2000 + step, device="cuda")
+        q = W.query(w, 2000 + step, device="cuda")
+        kvq = torch.cat([k.flatten(), v.flatten(), q.flatten()]).cpu().pin_memory()
+        gc.append_decode_host(kvq, w.Hq, sigma, hout)
+        oracle_append(oc, k, v)
+    torch.cuda.synchronize()
+    assert_decode_close(hout.cuda(), oc, q, sigma)
+    assert_guards()
 
 
 @pytest.mark.parametrize("paged", [False, True])
