@@ -151,10 +151,12 @@ def peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic(w: W.Workload):
+def profiled_traffic(w: W.Workload, alg_run: float):
     """DRAM bytes per decode launch (dram__bytes_read.sum + write) from the
-    committed ncu summary of this workload, or None when there is none or the
-    decode kernel's source changed since it was captured."""
+    committed ncu summary of this workload, scaled from the capture's fill to
+    this run's by the algorithmic bytes (the summary records both; traffic
+    follows the bytes streamed), or None when there is no summary or the decode
+    kernel's source changed since it was captured."""
     import hashlib
     prof = os.path.join(ROOT, "profiles", f"decode_stream_tc_{w.name.replace('-decode', '')}.md")
     csrc = os.path.join(ROOT, "bit_asymmetric_kv_quantize_b200", "csrc")
@@ -168,8 +170,13 @@ def profiled_traffic(w: W.Workload):
     for line in text.splitlines():
         if line.startswith("traffic_bytes_per_launch:"):
             parts = line.replace("(", " ").replace(")", " ").split()
-            if parts and parts[-1] == h.hexdigest()[:16]:
-                return int(parts[1])
+            if not parts or parts[-1] != h.hexdigest()[:16]:
+                continue
+            traffic = int(parts[1])
+            if "algorithmic_bytes_per_launch:" in parts:
+                alg_cap = int(parts[parts.index("algorithmic_bytes_per_launch:") + 1])
+                return traffic * alg_run / alg_cap
+            return float(traffic)
     return None
 
 
@@ -611,7 +618,8 @@ def measure(args, w: W.Workload, rank, world, device, steps, warmup, n_layers, f
                 "kernel": "decode_stream_tc" if args.kernel == "default" else "decode_split_simt",
                 "bound": "hbm", "achieved": achieved, "peak": peak,
                 "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": (profiled_traffic(w) if args.kernel == "default" else None),
+                "traffic": (profiled_traffic(w, bytes_total / steps)
+                            if args.kernel == "default" else None),
                 "algorithmic_bytes_per_launch": bytes_total / steps,
                 "avg_launch_us": split_total_ms * 1e3 / steps,
             },
